@@ -1,0 +1,206 @@
+"""NumPy front end of the CPU oracle (``qlora_oracle.c``).
+
+TEST INFRASTRUCTURE ONLY: the test suite, the smoke check and the bench's
+CPU-baseline leg are the only callers.  Nothing in the product package may
+import this module, and this module imports nothing from the product.
+
+Every function takes and returns host NumPy arrays.  bf16 tensors travel as
+their raw ``uint16`` bit patterns so that no library rounding sits between the
+caller and the oracle's own arithmetic.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "qlora_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+GCC_FLAGS = ["-O2", "-ffp-contract=off", "-fno-fast-math", "-fopenmp", "-shared", "-fPIC", "-std=c11"]
+
+
+def build(force: bool = False, src: str = _SRC, out: str = _LIB) -> str:
+    """Compile the oracle source into a shared library (plain gcc, fp-contract off)."""
+    if force or not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(src):
+        tmp = out + ".tmp%d" % os.getpid()
+        subprocess.check_call(["gcc", *GCC_FLAGS, "-o", tmp, src, "-lm"])
+        os.replace(tmp, out)
+    return out
+
+
+_lib = None
+
+
+def _declare(L: ctypes.CDLL) -> ctypes.CDLL:
+    p, i64, i32, f64, u32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_double, ctypes.c_uint32
+    L.oracle_normal_quantile.argtypes = [f64]
+    L.oracle_normal_quantile.restype = f64
+    L.oracle_nf4_table.argtypes = [p]
+    L.oracle_t8_table.argtypes = [p]
+    L.oracle_nf4_nearest.argtypes = [ctypes.c_float]
+    L.oracle_nf4_nearest.restype = i32
+    L.oracle_nf4_nearest_bits.argtypes = [u32, i64, p]
+    L.oracle_nf4_quantize.argtypes = [p, i32, i64, i32, p, p, p, p, p]
+    L.oracle_nf4_dequantize.argtypes = [i64, i32, p, p, p, p, ctypes.c_float, p]
+    L.oracle_linear_fwd.argtypes = [i64, i64, i64, i32, f64, p, p, p, p, p, i64, p]
+    L.oracle_linear_bwd.argtypes = [i64, i64, i64, i32, f64, p, p, p, p, p, p, i64, p, p, p]
+    L.oracle_num_threads.restype = i32
+    L.oracle_t8_nearest.argtypes = [ctypes.c_float]
+    L.oracle_t8_nearest.restype = i32
+    return L
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        _lib = _declare(ctypes.CDLL(build()))
+    return _lib
+
+
+def use_library(path: str) -> None:
+    """Point this module at another build of the oracle source (the mutation
+    tests load deliberately broken copies to show that the pins catch them)."""
+    global _lib
+    _lib = _declare(ctypes.CDLL(path))
+
+
+def t8_nearest(y: float) -> int:
+    return int(lib().oracle_t8_nearest(ctypes.c_float(y)))
+
+
+def _ptr(a: np.ndarray | None):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def num_threads() -> int:
+    return int(lib().oracle_num_threads())
+
+
+def normal_quantile(p: float) -> float:
+    return float(lib().oracle_normal_quantile(float(p)))
+
+
+def nf4_table() -> np.ndarray:
+    out = np.zeros(16, np.float32)
+    lib().oracle_nf4_table(_ptr(out))
+    return out
+
+
+def t8_table() -> np.ndarray:
+    out = np.zeros(255, np.float32)
+    lib().oracle_t8_table(_ptr(out))
+    return out
+
+
+def nf4_nearest(x: float) -> int:
+    return int(lib().oracle_nf4_nearest(ctypes.c_float(x)))
+
+
+def nf4_nearest_bits(start: int, n: int) -> np.ndarray:
+    """Nearest-code index of the n consecutive fp32 bit patterns from ``start``."""
+    out = np.zeros(n, np.uint8)
+    lib().oracle_nf4_nearest_bits(ctypes.c_uint32(start), n, _ptr(out))
+    return out
+
+
+def nf4_quantize(w: np.ndarray, double_quant: bool = True) -> dict:
+    """Blockwise NF4 quantization (+ double quantization) of a flat tensor.
+
+    ``w`` is either ``uint16`` (bf16 bit patterns) or ``float32``.
+    Returns ``codes`` (uint8, ceil(n/2)), ``absmax`` (float32, ceil(n/64)) and,
+    with double quantization, ``q8`` (uint8, nb), ``c1`` (float32, ceil(nb/256))
+    and ``offset`` (float).
+    """
+    w = np.ascontiguousarray(w).reshape(-1)
+    if w.dtype == np.uint16:
+        is_bf16 = 1
+    elif w.dtype == np.float32:
+        is_bf16 = 0
+    else:
+        raise TypeError("w must be uint16 (bf16 bits) or float32")
+    n = w.size
+    nb = (n + 63) // 64
+    nb2 = (nb + 255) // 256
+    codes = np.zeros((n + 1) // 2, np.uint8)
+    absmax = np.zeros(nb, np.float32)
+    q8 = np.zeros(nb, np.uint8)
+    c1 = np.zeros(nb2, np.float32)
+    off = np.zeros(1, np.float32)
+    lib().oracle_nf4_quantize(_ptr(w), is_bf16, n, int(bool(double_quant)), _ptr(codes),
+                              _ptr(absmax), _ptr(q8), _ptr(c1), _ptr(off))
+    out = {"codes": codes, "absmax": absmax}
+    if double_quant:
+        out.update(q8=q8, c1=c1, offset=float(off[0]))
+    return out
+
+
+def nf4_dequantize(n: int, q: dict, double_quant: bool = True) -> np.ndarray:
+    """doubleDequant: bf16 bit patterns (uint16, n) of the dequantized tensor."""
+    out = np.zeros(n, np.uint16)
+    codes = np.ascontiguousarray(q["codes"], np.uint8)
+    if double_quant:
+        q8 = np.ascontiguousarray(q["q8"], np.uint8)
+        c1 = np.ascontiguousarray(q["c1"], np.float32)
+        lib().oracle_nf4_dequantize(n, 1, _ptr(codes), None, _ptr(q8), _ptr(c1),
+                                    ctypes.c_float(q["offset"]), _ptr(out))
+    else:
+        absmax = np.ascontiguousarray(q["absmax"], np.float32)
+        lib().oracle_nf4_dequantize(n, 0, _ptr(codes), _ptr(absmax), None, None,
+                                    ctypes.c_float(0.0), _ptr(out))
+    return out
+
+
+def _bits(a: np.ndarray) -> np.ndarray:
+    a = np.ascontiguousarray(a)
+    if a.dtype != np.uint16:
+        raise TypeError("expected bf16 bit patterns (uint16)")
+    return a
+
+
+def linear_fwd(X: np.ndarray, W: np.ndarray, A: np.ndarray, B: np.ndarray, s: float,
+               rows: np.ndarray | None = None) -> np.ndarray:
+    """Y = X W^T + s (X A^T) B^T in fp64 (all inputs bf16 bits, 2-D).
+
+    ``rows`` selects rows of Y (int64 indices); None computes all of them.
+    """
+    X, W, A, B = map(_bits, (X, W, A, B))
+    M, K = X.shape
+    N = W.shape[0]
+    r = A.shape[0]
+    assert W.shape == (N, K) and A.shape == (r, K) and B.shape == (N, r)
+    if rows is not None:
+        rows = np.ascontiguousarray(rows, np.int64)
+        nrows = rows.size
+    else:
+        nrows = M
+    Y = np.zeros((nrows, N), np.float64)
+    lib().oracle_linear_fwd(M, N, K, r, float(s), _ptr(X), _ptr(W), _ptr(A), _ptr(B),
+                            _ptr(rows), nrows, _ptr(Y))
+    return Y
+
+
+def linear_bwd(dY: np.ndarray, X: np.ndarray, W: np.ndarray, A: np.ndarray, B: np.ndarray,
+               s: float, rows: np.ndarray | None = None, want_dx: bool = True):
+    """(dX, dA, dB) in fp64.  dX only for ``rows`` (all when None); dX is None
+    when ``want_dx`` is false.  There is no dW: the frozen weight has no
+    gradient."""
+    dY, X, W, A, B = map(_bits, (dY, X, W, A, B))
+    M, K = X.shape
+    N = W.shape[0]
+    r = A.shape[0]
+    assert dY.shape == (M, N) and W.shape == (N, K) and A.shape == (r, K) and B.shape == (N, r)
+    if rows is not None:
+        rows = np.ascontiguousarray(rows, np.int64)
+        nrows = rows.size
+    else:
+        nrows = M
+    dX = np.zeros((nrows, K), np.float64) if want_dx else None
+    dA = np.zeros((r, K), np.float64)
+    dB = np.zeros((N, r), np.float64)
+    lib().oracle_linear_bwd(M, N, K, r, float(s), _ptr(dY), _ptr(X), _ptr(W), _ptr(A), _ptr(B),
+                            _ptr(rows), nrows, _ptr(dX), _ptr(dA), _ptr(dB))
+    return dX, dA, dB
