@@ -1,0 +1,186 @@
+"""Torch-facing wrappers of the C ABI, same names as the C entry points.
+
+PyTorch supplies device memory and the current stream; every step of the
+path runs in the library's CUDA kernels.  Functions that produce tensors
+allocate them with ``torch.empty`` (outputs and the workspace the library asks
+for) unless the caller passes them in, which the bench does to keep
+allocation out of the timed region.
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib
+from ._lib import CNF4Weight, QLORA_BF16, QLORA_F32, check, lib
+
+BLOCKSIZE = 64
+DQ_BLOCK = 256
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream: torch.cuda.Stream | None = None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+@dataclass
+class NF4Weight:
+    """A quantized frozen weight W [rows = N, cols = K] and its constants.
+
+    codes [ceil(N*K/2)] uint8 (element 2i in the high nibble of byte i);
+    without double quantization ``absmax`` [nb] fp32; with it ``absmax_q8``
+    [nb] uint8, ``absmax_scale`` [ceil(nb/256)] fp32 and ``absmax_offset``
+    [1] fp32.
+    """
+
+    rows: int
+    cols: int
+    double_quant: bool
+    codes: torch.Tensor
+    absmax: torch.Tensor | None = None
+    absmax_q8: torch.Tensor | None = None
+    absmax_scale: torch.Tensor | None = None
+    absmax_offset: torch.Tensor | None = None
+
+    @property
+    def nblocks(self) -> int:
+        return (self.rows * self.cols + BLOCKSIZE - 1) // BLOCKSIZE
+
+    def c_struct(self) -> CNF4Weight:
+        return CNF4Weight(self.rows, self.cols, BLOCKSIZE, int(self.double_quant),
+                          _ptr(self.codes), _ptr(self.absmax), _ptr(self.absmax_q8),
+                          _ptr(self.absmax_scale), _ptr(self.absmax_offset))
+
+    def storage_bytes(self) -> int:
+        t = [self.codes, self.absmax, self.absmax_q8, self.absmax_scale, self.absmax_offset]
+        return sum(x.numel() * x.element_size() for x in t if x is not None)
+
+    @staticmethod
+    def empty(rows: int, cols: int, double_quant: bool = True, device="cuda") -> "NF4Weight":
+        n = rows * cols
+        nb = (n + BLOCKSIZE - 1) // BLOCKSIZE
+        codes = torch.empty((n + 1) // 2, dtype=torch.uint8, device=device)
+        if double_quant:
+            return NF4Weight(rows, cols, True, codes,
+                             absmax_q8=torch.empty(nb, dtype=torch.uint8, device=device),
+                             absmax_scale=torch.empty((nb + DQ_BLOCK - 1) // DQ_BLOCK, dtype=torch.float32, device=device),
+                             absmax_offset=torch.empty(1, dtype=torch.float32, device=device))
+        return NF4Weight(rows, cols, False, codes, absmax=torch.empty(nb, dtype=torch.float32, device=device))
+
+
+def _workspace(nbytes: int, device, ws: torch.Tensor | None) -> torch.Tensor:
+    if ws is not None and ws.numel() >= nbytes:
+        return ws
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def qlora_nf4_quantize_workspace(rows: int, cols: int, double_quant: bool = True) -> int:
+    return int(lib().qlora_nf4_quantize_workspace(rows, cols, BLOCKSIZE, int(double_quant)))
+
+
+def qlora_nf4_quantize(W: torch.Tensor, double_quant: bool = True, out: NF4Weight | None = None,
+                       ws: torch.Tensor | None = None) -> NF4Weight:
+    """Blockwise NF4 quantization (+ 8-bit double quantization) of a 2-D
+    bf16 or fp32 CUDA tensor."""
+    if W.dim() != 2 or not W.is_cuda or not W.is_contiguous():
+        raise ValueError("W must be a contiguous 2-D CUDA tensor")
+    if W.dtype == torch.bfloat16:
+        dt = QLORA_BF16
+    elif W.dtype == torch.float32:
+        dt = QLORA_F32
+    else:
+        raise TypeError("W must be bf16 or fp32")
+    rows, cols = W.shape
+    if out is None:
+        out = NF4Weight.empty(rows, cols, double_quant, W.device)
+    need = qlora_nf4_quantize_workspace(rows, cols, out.double_quant)
+    wsb = _workspace(need, W.device, ws) if need else None
+    cw = out.c_struct()
+    check(lib().qlora_nf4_quantize(_ptr(W), dt, ctypes.byref(cw), _ptr(wsb), need, _stream()),
+          "qlora_nf4_quantize")
+    return out
+
+
+def qlora_nf4_dequantize(w: NF4Weight, out: torch.Tensor | None = None) -> torch.Tensor:
+    """doubleDequant: the bf16 weight [rows, cols] the layer multiplies with."""
+    if out is None:
+        out = torch.empty(w.rows, w.cols, dtype=torch.bfloat16, device=w.codes.device)
+    cw = w.c_struct()
+    check(lib().qlora_nf4_dequantize(ctypes.byref(cw), _ptr(out), _stream()), "qlora_nf4_dequantize")
+    return out
+
+
+def qlora_linear_workspace(M: int, w: NF4Weight, r: int, bwd: bool) -> int:
+    cw = w.c_struct()
+    return int(lib().qlora_linear_workspace(M, ctypes.byref(cw), r, int(bwd)))
+
+
+def qlora_linear_fwd(X: torch.Tensor, w: NF4Weight, A: torch.Tensor | None, B: torch.Tensor | None,
+                     scale: float, Y: torch.Tensor | None = None,
+                     ws: torch.Tensor | None = None) -> torch.Tensor:
+    """Y = X dequant(W)^T + scale (X A^T) B^T (bf16 in/out, fp32 accumulate)."""
+    M = X.shape[0]
+    r = 0 if A is None else A.shape[0]
+    if Y is None:
+        Y = torch.empty(M, w.rows, dtype=torch.bfloat16, device=X.device)
+    need = qlora_linear_workspace(M, w, r, False)
+    wsb = _workspace(need, X.device, ws)
+    cw = w.c_struct()
+    check(lib().qlora_linear_fwd(_ptr(X), M, ctypes.byref(cw), _ptr(A), _ptr(B), r, float(scale),
+                                 _ptr(Y), _ptr(wsb), wsb.numel(), _stream()), "qlora_linear_fwd")
+    return Y
+
+
+def qlora_linear_bwd(dY: torch.Tensor, X: torch.Tensor, w: NF4Weight, A: torch.Tensor | None,
+                     B: torch.Tensor | None, scale: float, dX: torch.Tensor | None = None,
+                     dA: torch.Tensor | None = None, dB: torch.Tensor | None = None,
+                     ws: torch.Tensor | None = None, want_dx: bool = True):
+    """(dX, dA, dB) of the layer; the frozen weight gets no gradient."""
+    M = X.shape[0]
+    r = 0 if A is None else A.shape[0]
+    if want_dx and dX is None:
+        dX = torch.empty(M, w.cols, dtype=torch.bfloat16, device=X.device)
+    if r > 0:
+        if dA is None:
+            dA = torch.empty(r, w.cols, dtype=torch.float32, device=X.device)
+        if dB is None:
+            dB = torch.empty(w.rows, r, dtype=torch.float32, device=X.device)
+    need = qlora_linear_workspace(M, w, r, True)
+    wsb = _workspace(need, X.device, ws)
+    cw = w.c_struct()
+    check(lib().qlora_linear_bwd(_ptr(dY), _ptr(X), M, ctypes.byref(cw), _ptr(A), _ptr(B), r,
+                                 float(scale), _ptr(dX) if want_dx else None, _ptr(dA), _ptr(dB),
+                                 _ptr(wsb), wsb.numel(), _stream()), "qlora_linear_bwd")
+    return dX, dA, dB
+
+
+def qlora_get_last_error(stream: torch.cuda.Stream | None = None) -> int:
+    return int(lib().qlora_get_last_error(_stream(stream)))
+
+
+def qlora_nf4_table() -> list[float]:
+    buf = (ctypes.c_float * 16)()
+    lib().qlora_nf4_table(buf)
+    return list(buf)
+
+
+def qlora_nf4_encode(x: torch.Tensor, codes: torch.Tensor | None = None) -> torch.Tensor:
+    """Nearest-NF4-code index of every fp32 element of x (one code per byte)."""
+    if codes is None:
+        codes = torch.empty(x.numel(), dtype=torch.uint8, device=x.device)
+    check(lib().qlora_nf4_encode(_ptr(x), x.numel(), _ptr(codes), _stream()), "qlora_nf4_encode")
+    return codes
+
+
+def qlora_set_wait_timeout_ns(ns: int) -> None:
+    lib().qlora_set_wait_timeout_ns(int(ns))
+
+
+def qlora_debug_inject(mode: int) -> None:
+    lib().qlora_debug_inject(int(mode))

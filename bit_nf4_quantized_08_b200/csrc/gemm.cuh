@@ -1,0 +1,383 @@
+// gemm.cuh -- warp-specialized tcgen05 GEMM for sm_100a with an optional
+// NF4 dequantizing producer.
+//
+// Computes D[i][j] = sum_k Aop[i][k] * Bop[j][k] for one 128 x BN tile per
+// CTA, accumulating in TMEM (fp32), k in steps of 64 (one NF4 block column).
+//   warp 0           TMA / bulk-copy producer (one elected lane)
+//   warp 1           TMEM allocation + tcgen05.mma issue (one elected lane)
+//   warps 2..        dequant producers (expand NF4 codes into the swizzled
+//                    bf16 operand tile in shared memory), then the epilogue
+//                    (tcgen05.ld -> bf16/fp32 -> global)
+// Operand tiles use the 128-byte swizzle.  A K-major tile of R rows keeps
+// row r at byte r*128 (8-row groups 1024 B apart).  An MN-major tile keeps
+// 64-element MN chunks 8192 B apart and k-row j at byte j*128 inside a chunk.
+//
+// Dequant modes (the frozen weight W [N, K] is never written to HBM):
+//   DQ_B_K   B operand = W' rows (forward: Y = X W'^T), R = BN rows
+//   DQ_B_MN  B operand = W' viewed [k_out][n] (backward: dX = dY W'), the
+//            reduction runs over W rows, 64 per step, 256 output columns
+//   DQ_A_K   A operand = W' rows (swap-AB small-M forward: Y^T = W' X^T)
+// LoRA steps (digest sec. 4 / reproduction blog forward): extra k-steps whose
+// operands both come from TMA (e.g. [X | sU] . [W' | B]^T).
+#pragma once
+
+#include "common.cuh"
+#include "internal.h"
+#include "nf4.cuh"
+
+namespace qlora {
+
+enum { DQ_NONE = 0, DQ_B_K = 1, DQ_B_MN = 2, DQ_A_K = 3 };
+enum { EPI_BF16 = 0, EPI_BF16_T = 1, EPI_F32 = 2, EPI_F32_T = 3 };
+
+struct GemmParams {
+    CUtensorMap tmA, tmB;    // main k-steps (unused for the dequantized operand)
+    CUtensorMap tmA2, tmB2;  // LoRA k-steps
+    CUtensorMap tmCodes;     // packed NF4 codes viewed [W rows][K/2 bytes]
+    const float* scales;     // block constants a' laid out [kb][scales_ld]
+    int64_t scales_ld;
+    int dq_rows;             // valid W rows (the rest of a dequant tile is 0)
+    int dq_kbs;              // valid block columns K/64
+    int ks_main, ks_lora;    // number of k-steps of each kind
+    int ks_per_split;        // main k-steps per blockIdx.z
+    int rows, cols;          // valid extent of D
+    void* out;
+    int64_t out_ld;          // elements
+    int64_t out_split_stride;  // elements between split-K partial planes
+    uint64_t timeout_ns;
+    int inject;
+};
+
+template <int BN, int A_MN, int B_MN, int DQ>
+struct GemmShape {
+    static constexpr int BM = 128;
+    static constexpr int A_BYTES = BM * 128;
+    static constexpr int B_BYTES = BN * 128;
+    static constexpr int DQ_ROWS = DQ == DQ_B_K ? BN : (DQ == DQ_A_K ? BM : (DQ == DQ_B_MN ? 256 : 0));
+    static constexpr int NDQ_WARPS = DQ_ROWS / 32;
+    static constexpr int CODE_BYTES = DQ == DQ_B_MN ? 64 * 128 : DQ_ROWS * 32;
+    static constexpr int SCALE_BYTES = DQ == DQ_NONE ? 0 : (DQ == DQ_B_MN ? 4 * 64 * 4 : DQ_ROWS * 4);
+    static constexpr int STAGE_RAW = A_BYTES + B_BYTES + CODE_BYTES + SCALE_BYTES;
+    static constexpr int STAGE_BYTES = (STAGE_RAW + 1023) / 1024 * 1024;
+    static constexpr int NE_WARPS = NDQ_WARPS > 4 ? NDQ_WARPS : 4;
+    static constexpr int THREADS = 32 * (2 + NE_WARPS);
+    static constexpr int TMEM_COLS = BN <= 32 ? 32 : (BN <= 64 ? 64 : (BN <= 128 ? 128 : 256));
+    static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
+};
+
+template <int BN, int A_MN, int B_MN, int DQ, int STAGES>
+constexpr int gemm_smem_bytes() {
+    return GemmShape<BN, A_MN, B_MN, DQ>::STAGE_BYTES * STAGES + 1024 /*align*/ + 256 /*barriers*/;
+}
+
+template <int BN, int A_MN, int B_MN, int DQ, int EPI, int STAGES>
+__global__ void __launch_bounds__(GemmShape<BN, A_MN, B_MN, DQ>::THREADS, 1)
+    k_gemm(const __grid_constant__ GemmParams p) {
+    using S = GemmShape<BN, A_MN, B_MN, DQ>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_base = smem_u32(smem_raw);
+    const uint32_t base = (raw_base + 1023u) & ~1023u;
+    uint8_t* gbase = smem_raw + (base - raw_base);
+    const uint32_t bar_base = base + S::STAGE_BYTES * STAGES;
+    // barrier i at bar_base + 8*i: full_tma[STAGES], full_dq[STAGES], empty[STAGES], acc_full
+    auto full_tma = [&](int s) { return bar_base + 8u * s; };
+    auto full_dq = [&](int s) { return bar_base + 8u * (STAGES + s); };
+    auto empty = [&](int s) { return bar_base + 8u * (2 * STAGES + s); };
+    const uint32_t acc_full = bar_base + 8u * (3 * STAGES);
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + S::STAGE_BYTES * STAGES + 8 * (3 * STAGES + 1));
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const WaitCfg wc{p.timeout_ns};
+
+    const int tile_n = blockIdx.x, tile_m = blockIdx.y, split = blockIdx.z;
+    const int m0 = tile_m * S::BM, n0 = tile_n * BN;
+    const int k_begin = split * p.ks_per_split;
+    int k_end = k_begin + p.ks_per_split;
+    if (k_end > p.ks_main) k_end = p.ks_main;
+    const bool last_split = (split == (int)gridDim.z - 1);
+    const int n_main = k_end > k_begin ? k_end - k_begin : 0;
+    const int n_steps = n_main + (last_split ? p.ks_lora : 0);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full_tma(s), 1);
+            mbar_init(full_dq(s), S::NDQ_WARPS > 0 ? S::NDQ_WARPS : 1);
+            mbar_init(empty(s), 1);
+        }
+        mbar_init(acc_full, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&p.tmA);
+        prefetch_tensormap(&p.tmB);
+        if (p.ks_lora) {
+            prefetch_tensormap(&p.tmA2);
+            prefetch_tensormap(&p.tmB2);
+        }
+        if (DQ != DQ_NONE) prefetch_tensormap(&p.tmCodes);
+    }
+    if (warp == 1) tmem_alloc(smem_u32(tmem_holder), S::TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0 && !p.inject) {
+            int last_use[STAGES];
+            for (int s = 0; s < STAGES; ++s) last_use[s] = -1;
+            bool ok = true;
+            for (int i = 0; i < n_steps && ok; ++i) {
+                const int s = i % STAGES, u = i / STAGES;
+                if (!mbar_wait(empty(s), (u & 1) ^ 1, wc)) { ok = false; *abort_flag = 1; break; }
+                const uint32_t sA = base + s * S::STAGE_BYTES;
+                const uint32_t sB = sA + S::A_BYTES;
+                const uint32_t sC = sB + S::B_BYTES;
+                const uint32_t sS = sC + S::CODE_BYTES;
+                const bool lora = i >= n_main;
+                const int k = lora ? (i - n_main) : (k_begin + i);
+                uint32_t bytes = 0;
+                if (!lora) {
+                    if (DQ != DQ_A_K) bytes += S::A_BYTES;
+                    if (DQ != DQ_B_K && DQ != DQ_B_MN) bytes += S::B_BYTES;
+                    if (DQ != DQ_NONE) bytes += S::CODE_BYTES;
+                    if (DQ == DQ_B_K || DQ == DQ_A_K) bytes += S::DQ_ROWS * 4;
+                    if (DQ == DQ_B_MN) {
+                        for (int c = 0; c < 4; ++c)
+                            if (n0 / 64 + c < p.dq_kbs) bytes += 256;
+                    }
+                } else {
+                    bytes = S::A_BYTES + S::B_BYTES;
+                }
+                mbar_arrive_expect_tx(full_tma(s), bytes);
+                const CUtensorMap* mA = lora ? &p.tmA2 : &p.tmA;
+                const CUtensorMap* mB = lora ? &p.tmB2 : &p.tmB;
+                if (lora || DQ != DQ_A_K) {
+                    if (A_MN) {
+                        tma_load_2d(sA, mA, full_tma(s), m0, k * 64);
+                        tma_load_2d(sA + 8192, mA, full_tma(s), m0 + 64, k * 64);
+                    } else {
+                        tma_load_2d(sA, mA, full_tma(s), k * 64, m0);
+                    }
+                }
+                if (lora || (DQ != DQ_B_K && DQ != DQ_B_MN)) {
+                    if (B_MN) {
+                        for (int c = 0; c < BN / 64; ++c)
+                            tma_load_2d(sB + 8192 * c, mB, full_tma(s), n0 + 64 * c, k * 64);
+                    } else {
+                        tma_load_2d(sB, mB, full_tma(s), k * 64, n0);
+                    }
+                }
+                if (!lora && DQ != DQ_NONE) {
+                    if (DQ == DQ_B_MN) {
+                        tma_load_2d(sC, &p.tmCodes, full_tma(s), n0 / 2, k * 64);
+                        for (int c = 0; c < 4; ++c)
+                            if (n0 / 64 + c < p.dq_kbs)
+                                bulk_load(sS + 256 * c,
+                                          p.scales + (int64_t)(n0 / 64 + c) * p.scales_ld + k * 64,
+                                          256, full_tma(s));
+                    } else {
+                        const int w0 = DQ == DQ_B_K ? n0 : m0;
+                        tma_load_2d(sC, &p.tmCodes, full_tma(s), k * 32, w0);
+                        bulk_load(sS, p.scales + (int64_t)k * p.scales_ld + w0, S::DQ_ROWS * 4,
+                                  full_tma(s));
+                    }
+                }
+                last_use[s] = u;
+            }
+            // drain: every issued copy has landed before the CTA may exit
+            for (int s = 0; s < STAGES; ++s)
+                if (last_use[s] >= 0) mbar_wait(full_tma(s), last_use[s] & 1, wc);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(128, BN, A_MN, B_MN);
+            bool ok = true;
+            for (int i = 0; i < n_steps; ++i) {
+                const int s = i % STAGES, u = i / STAGES;
+                const bool lora = i >= n_main;
+                if (!mbar_wait(full_tma(s), u & 1, wc)) { ok = false; *abort_flag = 1; break; }
+                if (DQ != DQ_NONE && !lora) {
+                    if (!mbar_wait(full_dq(s), u & 1, wc)) { ok = false; *abort_flag = 1; break; }
+                }
+                tc_fence_after();
+                const uint32_t sA = base + s * S::STAGE_BYTES;
+                const uint32_t sB = sA + S::A_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint64_t ad = A_MN ? smem_desc_sw128(sA + kk * 2048, 8192, 1024)
+                                             : smem_desc_sw128(sA + kk * 32, 16, 1024);
+                    const uint64_t bd = B_MN ? smem_desc_sw128(sB + kk * 2048, 8192, 1024)
+                                             : smem_desc_sw128(sB + kk * 32, 16, 1024);
+                    umma_bf16(tmem, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(empty(s));
+            }
+            umma_commit(acc_full);
+            if (!ok) mbar_wait(acc_full, 0, wc);  // issued MMAs finish before TMEM is freed
+        }
+    } else {
+        // ------------------------------------------------------------ dequant
+        const int dw = warp - 2;
+        if (DQ != DQ_NONE && dw < S::NDQ_WARPS) {
+            const int t = dw * 32 + lane;  // block-row index inside the tile
+            uint32_t code_off, out_off;
+            int scale_idx;
+            int64_t wrow;
+            int kb_off;
+            if (DQ == DQ_B_MN) {
+                const int j = t >> 2, c = t & 3;
+                code_off = j * 128 + c * 32;
+                scale_idx = c * 64 + j;
+                out_off = c * 8192 + j * 128;
+                wrow = j;  // + 64*k
+                kb_off = c;
+            } else {
+                code_off = t * 32;
+                scale_idx = t;
+                out_off = t * 128;
+                wrow = (DQ == DQ_B_K ? n0 : m0) + t;
+                kb_off = 0;
+            }
+            const uint32_t tile_off = (DQ == DQ_A_K) ? 0u : (uint32_t)S::A_BYTES;
+            for (int i = 0; i < n_main; ++i) {
+                const int s = i % STAGES, u = i / STAGES;
+                if (!mbar_wait(full_tma(s), u & 1, wc)) { *abort_flag = 1; break; }
+                const int k = k_begin + i;
+                const uint32_t st = base + s * S::STAGE_BYTES;
+                const uint32_t sC = st + S::A_BYTES + S::B_BYTES;
+                const uint32_t sOut = st + tile_off;
+                bool valid;
+                if (DQ == DQ_B_MN)
+                    valid = (64 * k + wrow < p.dq_rows) && (n0 / 64 + kb_off < p.dq_kbs);
+                else
+                    valid = true;  // rows beyond the weight only feed masked outputs
+                if (valid) {
+                    const float a = reinterpret_cast<const float*>(gbase + s * S::STAGE_BYTES + S::A_BYTES +
+                                                                   S::B_BYTES + S::CODE_BYTES)[scale_idx];
+                    const uint4 c0 = ld_shared_v4(sC + code_off);
+                    const uint4 c1 = ld_shared_v4(sC + code_off + 16);
+                    const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                    const Nf4BlockTable tb = nf4_block_table(a);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        uint32_t o[4];
+                        nf4_expand_word(words[q], tb, o);
+                        st_shared_v4(sOut + sw128(out_off + q * 16), o[0], o[1], o[2], o[3]);
+                    }
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) st_shared_v4(sOut + sw128(out_off + q * 16), 0u, 0u, 0u, 0u);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(full_dq(s));
+            }
+        }
+        // ------------------------------------------------------------ epilogue
+        const int ew = warp - 2;
+        const int quarter = warp & 3;
+        constexpr int GROUPS = S::NE_WARPS / 4;
+        const int group = ew / 4;
+        constexpr int COLS_PER_GROUP = BN / GROUPS;
+        if (mbar_wait(acc_full, 0, wc) && !*abort_flag) {
+            tc_fence_after();
+            const int row = quarter * 32 + lane;  // D row inside the tile (TMEM lane)
+            const int grow = m0 + row;
+            const bool row_ok = grow < p.rows;
+            for (int cc = 0; cc < COLS_PER_GROUP; cc += 32) {
+                const int col0 = group * COLS_PER_GROUP + cc;
+                uint32_t v[32];
+                __syncwarp();
+                tmem_ld_32x32b_x32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)col0, v);
+                tmem_ld_wait();
+                const int gcol0 = n0 + col0;
+                if (n_steps == 0) {
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) v[q] = 0u;
+                }
+                if (row_ok) {
+                    if (EPI == EPI_BF16) {
+                        uint16_t* o = static_cast<uint16_t*>(p.out) + (int64_t)grow * p.out_ld + gcol0;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            if (gcol0 + 8 * q + 8 <= p.cols) {
+                                uint4 w;
+                                w.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]), __uint_as_float(v[8 * q + 1]));
+                                w.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
+                                w.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
+                                w.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
+                                *reinterpret_cast<uint4*>(o + 8 * q) = w;
+                            }
+                        }
+                    } else if (EPI == EPI_BF16_T) {
+                        uint16_t* o = static_cast<uint16_t*>(p.out) + grow;
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) {
+                            if (gcol0 + q < p.cols) {
+                                uint32_t h = pack_bf16x2(__uint_as_float(v[q]), 0.0f) & 0xFFFFu;
+                                o[(int64_t)(gcol0 + q) * p.out_ld] = (uint16_t)h;
+                            }
+                        }
+                    } else if (EPI == EPI_F32) {
+                        float* o = static_cast<float*>(p.out) + (int64_t)split * p.out_split_stride +
+                                   (int64_t)grow * p.out_ld + gcol0;
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            if (gcol0 + 4 * q + 4 <= p.cols)
+                                *reinterpret_cast<uint4*>(o + 4 * q) =
+                                    make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                        }
+                    } else {  // EPI_F32_T
+                        float* o = static_cast<float*>(p.out) + (int64_t)split * p.out_split_stride + grow;
+#pragma unroll
+                        for (int q = 0; q < 32; ++q)
+                            if (gcol0 + q < p.cols) o[(int64_t)(gcol0 + q) * p.out_ld] = __uint_as_float(v[q]);
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, S::TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// split-K reduction: out = cast(scale * sum_z part[z][i][j]) in fixed z order
+// ---------------------------------------------------------------------------
+enum { RED_BF16 = 0, RED_F32 = 1, RED_F32_T = 2 };
+
+__global__ void k_splitk_reduce(const float* __restrict__ part, int splits, int64_t split_stride,
+                                int rows, int cols, int64_t part_ld, float scale, int mode,
+                                void* __restrict__ out, int64_t out_ld) {
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= (int64_t)rows * cols) return;
+    const int64_t i = idx / cols, j = idx - i * cols;
+    float acc = 0.0f;
+    for (int z = 0; z < splits; ++z) acc = __fadd_rn(acc, part[z * split_stride + i * part_ld + j]);
+    acc = __fmul_rn(acc, scale);
+    if (mode == RED_BF16) {
+        uint32_t h = pack_bf16x2(acc, 0.0f) & 0xFFFFu;
+        static_cast<uint16_t*>(out)[i * out_ld + j] = (uint16_t)h;
+    } else if (mode == RED_F32) {
+        static_cast<float*>(out)[i * out_ld + j] = acc;
+    } else {
+        static_cast<float*>(out)[j * out_ld + i] = acc;
+    }
+}
+
+__global__ void k_fill_zero_f32(float* __restrict__ p, int64_t n) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+        p[i] = 0.0f;
+}
+
+}  // namespace qlora

@@ -1,0 +1,54 @@
+// internal.h -- launchers shared between the library's translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/qlora_nf4.h"
+
+namespace qlora {
+
+// Bound of every in-kernel wait of the next launches (ns).
+uint64_t wait_timeout_ns();
+int inject_mode();
+
+// ---- quantizer (quantize.cu) ----
+// Host-built search table of the fast nearest-code search (33 buckets of
+// width 1/16 over [-1, 1], see quantize.cu).
+struct Nf4SearchTable {
+    float thr[33];
+    int base[33];
+};
+const Nf4SearchTable& nf4_search_table();
+void nf4_table_host(float out[16]);
+
+cudaError_t launch_quantize_blocks(const void* W, int is_bf16, int64_t n, uint8_t* codes,
+                                   float* absmax, double* group_sums, cudaStream_t s);
+cudaError_t launch_dq_offset(const double* group_sums, int64_t ngroups, int64_t nb, float* offset,
+                             cudaStream_t s);
+cudaError_t launch_dq_quantize(const float* absmax, int64_t nb, const float* offset, uint8_t* q8,
+                               float* c1, cudaStream_t s);
+cudaError_t launch_dequantize(const qlora_nf4_weight& w, uint16_t* out, cudaStream_t s);
+cudaError_t launch_encode(const float* x, int64_t n, uint8_t* codes, cudaStream_t s);
+
+// Block constants a' of a weight, written transposed as scales[kb * ld + n]
+// (kb = block column, n = row) for the GEMM producers.
+cudaError_t launch_expand_scales(const qlora_nf4_weight& w, float* scales, int64_t ld,
+                                 cudaStream_t s);
+
+// ---- GEMMs (gemm.cu) ----
+struct LinearArgs {
+    int64_t M, N, K;
+    int r;
+    float scale;
+    const qlora_nf4_weight* w;
+};
+qlora_status linear_fwd_impl(const void* X, const LinearArgs& a, const void* A, const void* B,
+                             void* Y, void* ws, size_t ws_bytes, cudaStream_t s);
+qlora_status linear_bwd_impl(const void* dY, const void* X, const LinearArgs& a, const void* A,
+                             const void* B, void* dX, float* dA, float* dB, void* ws,
+                             size_t ws_bytes, cudaStream_t s);
+size_t linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int r, int bwd);
+
+}  // namespace qlora

@@ -1,0 +1,380 @@
+// linear.cuh -- host side of the QLoRA linear forward and backward: tensor
+// maps, workspace carving, split-K choices and the launch sequence.
+//
+// Forward (reproduction blog "LoRA formula and tensor shapes"; digest sec. 4):
+//   M > 64 :  sU = bf16(s * X A^T)   (skinny tcgen05 GEMM, split-K + reduce)
+//             Y  = [X | sU] [W' | B]^T   (dequant GEMM, LoRA as extra k-steps)
+//   M <= 64:  sU as above, then Y^T = [W' | B] [X | sU]^T with the weight as
+//             the 128-row MMA operand (tokens as the narrow N side).
+// Backward (digest sec. 4 steps 4: gradients pass through W^BF16; W frozen):
+//   sU = bf16(s X A^T), sG = bf16(s dY B)          (skinny GEMMs)
+//   dX = [dY | sG] [W' ; A]                       (dequant GEMM, MN-major W')
+//   dA = sG^T X,  dB = dY^T sU                     (skinny GEMMs over M)
+#pragma once
+
+#include <algorithm>
+#include <mutex>
+
+#include "gemm.cuh"
+#include "internal.h"
+#include "quantize.cuh"
+
+namespace qlora {
+
+// ---------------------------------------------------------------------------
+// tensor maps
+// ---------------------------------------------------------------------------
+typedef CUresult (*PFN_encodeTiled_t)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                      const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                      const cuuint32_t*, CUtensorMapInterleave,
+                                      CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                      CUtensorMapFloatOOBfill);
+
+inline PFN_encodeTiled_t encode_fn() {
+    static PFN_encodeTiled_t fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_encodeTiled_t>(p);
+    });
+    return fn;
+}
+
+// 2-D tiled map over a row-major [outer][inner] tensor.
+inline bool make_map(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int esize,
+                     uint64_t inner, uint64_t outer, uint64_t row_bytes, uint32_t box_inner,
+                     uint32_t box_outer, bool swizzle128) {
+    PFN_encodeTiled_t fn = encode_fn();
+    if (!fn) return false;
+    (void)esize;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = fn(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// bf16 row-major [outer][inner], 64 x box_outer boxes, 128-byte swizzle.
+inline bool map_bf16(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer,
+                     uint32_t box_outer) {
+    return make_map(m, ptr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, inner, outer, inner * 2, 64,
+                    box_outer, true);
+}
+
+// ---------------------------------------------------------------------------
+// launch helpers
+// ---------------------------------------------------------------------------
+template <int BN, int A_MN, int B_MN, int DQ, int EPI, int STAGES>
+inline cudaError_t launch_gemm(const GemmParams& p, dim3 grid, cudaStream_t s) {
+    using Sh = GemmShape<BN, A_MN, B_MN, DQ>;
+    constexpr int smem = gemm_smem_bytes<BN, A_MN, B_MN, DQ, STAGES>();
+    auto kern = k_gemm<BN, A_MN, B_MN, DQ, EPI, STAGES>;
+    static bool configured = false;  // attribute is per function; set once per device use
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    (void)configured;
+    kern<<<grid, Sh::THREADS, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
+inline int ceil_div(int64_t a, int64_t b) { return (int)((a + b - 1) / b); }
+inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Split-K choice: about two CTAs per SM, every split at least one k-step.
+inline void choose_splits(int tiles, int ksteps, int* splits, int* per) {
+    int S = std::max(1, (2 * 148 + tiles - 1) / std::max(1, tiles));
+    S = std::min(S, std::max(1, ksteps));
+    int p = std::max(1, (ksteps + S - 1) / S);
+    *per = p;
+    *splits = std::max(1, (ksteps + p - 1) / p);
+}
+
+inline int lora_bn(int r) { return r <= 64 ? 64 : (r <= 128 ? 128 : 256); }
+
+constexpr int kSmallM = 64;
+
+struct WsCarve {
+    char* p;
+    size_t used;
+    void* take(size_t bytes) {
+        void* r = p ? p + used : nullptr;
+        used += align256(bytes);
+        return r;
+    }
+};
+
+// Skinny GEMM out[rows][r] = scale * sum_k Aop[row][k] Bop[j][k], through
+// split-K fp32 partials and a fixed-order reduction.
+template <int A_MN, int B_MN>
+inline qlora_status skinny(const CUtensorMap& tA, const CUtensorMap& tB, int rows, int r,
+                           int ksteps, float* part, float scale, int red_mode, void* out,
+                           int64_t out_ld, cudaStream_t s) {
+    GemmParams p;
+    memset(&p, 0, sizeof(p));
+    p.tmA = tA;
+    p.tmB = tB;
+    p.tmA2 = tA;
+    p.tmB2 = tB;
+    p.tmCodes = tA;
+    const int tiles = ceil_div(rows, 128);
+    int splits, per;
+    choose_splits(tiles, ksteps, &splits, &per);
+    p.ks_main = ksteps;
+    p.ks_lora = 0;
+    p.ks_per_split = per;
+    p.rows = rows;
+    p.cols = r;
+    p.out = part;
+    p.out_ld = r;
+    p.out_split_stride = (int64_t)rows * r;
+    p.timeout_ns = wait_timeout_ns();
+    p.inject = inject_mode();
+    dim3 grid(1, tiles, splits);
+    const int bn = lora_bn(r);
+    cudaError_t e;
+    if (bn == 64)
+        e = launch_gemm<64, A_MN, B_MN, DQ_NONE, EPI_F32, 6>(p, grid, s);
+    else if (bn == 128)
+        e = launch_gemm<128, A_MN, B_MN, DQ_NONE, EPI_F32, 5>(p, grid, s);
+    else
+        e = launch_gemm<256, A_MN, B_MN, DQ_NONE, EPI_F32, 4>(p, grid, s);
+    if (e != cudaSuccess) return QLORA_ERR_CUDA;
+    const int64_t total = (int64_t)rows * r;
+    k_splitk_reduce<<<ceil_div(total, 256), 256, 0, s>>>(part, splits, (int64_t)rows * r, rows, r, r,
+                                                         scale, red_mode, out, out_ld);
+    return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+inline size_t skinny_part_bytes(int rows, int r, int ksteps) {
+    int splits, per;
+    choose_splits(ceil_div(rows, 128), ksteps, &splits, &per);
+    return (size_t)splits * rows * r * 4;
+}
+
+inline size_t small_m_part_bytes(int64_t M, int64_t N, int64_t K) {
+    int splits, per;
+    choose_splits(ceil_div(N, 128), (int)(K / 64), &splits, &per);
+    return splits > 1 ? (size_t)splits * M * N * 4 : 0;
+}
+
+// Workspace layout shared by the query and the launches.
+struct LinearWs {
+    float* scales;
+    int64_t scales_ld;
+    uint16_t* sU;
+    uint16_t* sG;
+    float* part;
+    size_t bytes;
+};
+
+inline LinearWs carve_linear_ws(void* ws, int64_t M, int64_t N, int64_t K, int r, int bwd) {
+    WsCarve c{static_cast<char*>(ws), 0};
+    LinearWs L;
+    L.scales_ld = ((N + 255) / 256) * 256;
+    L.scales = static_cast<float*>(c.take((size_t)(K / 64) * L.scales_ld * 4));
+    L.sU = r > 0 ? static_cast<uint16_t*>(c.take((size_t)M * r * 2)) : nullptr;
+    L.sG = (r > 0 && bwd) ? static_cast<uint16_t*>(c.take((size_t)M * r * 2)) : nullptr;
+    size_t part = 0;
+    if (r > 0) {
+        part = std::max(part, skinny_part_bytes((int)M, r, (int)(K / 64)));
+        if (bwd) {
+            part = std::max(part, skinny_part_bytes((int)M, r, ceil_div(N, 64)));
+            part = std::max(part, skinny_part_bytes((int)K, r, ceil_div(M, 64)));
+            part = std::max(part, skinny_part_bytes((int)N, r, ceil_div(M, 64)));
+        }
+    }
+    if (!bwd && M <= kSmallM) part = std::max(part, small_m_part_bytes(M, N, K));
+    L.part = part ? static_cast<float*>(c.take(part)) : nullptr;
+    L.bytes = c.used;
+    return L;
+}
+
+inline size_t linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int r, int bwd) {
+    return carve_linear_ws(nullptr, M, N, K, r, bwd).bytes;
+}
+
+inline bool map_codes(CUtensorMap* m, const qlora_nf4_weight& w, uint32_t box_bytes,
+                      uint32_t box_rows) {
+    return make_map(m, w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)w.cols / 2,
+                    (uint64_t)w.rows, (uint64_t)w.cols / 2, box_bytes, box_rows, false);
+}
+
+// sU = bf16(scale * X A^T) into L.sU
+inline qlora_status compute_sU(const void* X, const LinearArgs& a, const void* A,
+                               const LinearWs& L, cudaStream_t s) {
+    CUtensorMap tX, tA;
+    if (!map_bf16(&tX, X, a.K, a.M, 128)) return QLORA_ERR_CUDA;
+    if (!map_bf16(&tA, A, a.K, a.r, lora_bn(a.r))) return QLORA_ERR_CUDA;
+    return skinny<0, 0>(tX, tA, (int)a.M, a.r, (int)(a.K / 64), L.part, a.scale, RED_BF16, L.sU,
+                        a.r, s);
+}
+
+inline qlora_status linear_fwd_impl(const void* X, const LinearArgs& a, const void* A,
+                                    const void* B, void* Y, void* ws, size_t ws_bytes,
+                                    cudaStream_t s) {
+    (void)ws_bytes;
+    const qlora_nf4_weight& w = *a.w;
+    LinearWs L = carve_linear_ws(ws, a.M, a.N, a.K, a.r, 0);
+    if (launch_expand_scales(w, L.scales, L.scales_ld, s) != cudaSuccess) return QLORA_ERR_CUDA;
+    if (a.r > 0) {
+        qlora_status st = compute_sU(X, a, A, L, s);
+        if (st != QLORA_OK) return st;
+    }
+    GemmParams p;
+    memset(&p, 0, sizeof(p));
+    p.scales = L.scales;
+    p.scales_ld = L.scales_ld;
+    p.dq_rows = (int)a.N;
+    p.dq_kbs = (int)(a.K / 64);
+    p.ks_main = (int)(a.K / 64);
+    p.ks_lora = a.r > 0 ? ceil_div(a.r, 64) : 0;
+    p.timeout_ns = wait_timeout_ns();
+    p.inject = inject_mode();
+    p.out = Y;
+    if (a.M > kSmallM) {
+        // Y = [X | sU] [W' | B]^T : 128 x 256 tiles, W' dequantized into the B slot.
+        if (!map_bf16(&p.tmA, X, a.K, a.M, 128)) return QLORA_ERR_CUDA;
+        p.tmB = p.tmA;
+        if (!map_codes(&p.tmCodes, w, 32, 256)) return QLORA_ERR_CUDA;
+        if (a.r > 0) {
+            if (!map_bf16(&p.tmA2, L.sU, a.r, a.M, 128)) return QLORA_ERR_CUDA;
+            if (!map_bf16(&p.tmB2, B, a.r, a.N, 256)) return QLORA_ERR_CUDA;
+        } else {
+            p.tmA2 = p.tmA;
+            p.tmB2 = p.tmA;
+        }
+        p.ks_per_split = p.ks_main;
+        p.rows = (int)a.M;
+        p.cols = (int)a.N;
+        p.out_ld = a.N;
+        dim3 grid(ceil_div(a.N, 256), ceil_div(a.M, 128), 1);
+        if (launch_gemm<256, 0, 0, DQ_B_K, EPI_BF16, 3>(p, grid, s) != cudaSuccess)
+            return QLORA_ERR_CUDA;
+        return QLORA_OK;
+    }
+    // small M: Y^T = [W' | B] [X | sU]^T, weight rows on the 128-lane side.
+    const int bn = a.M <= 32 ? 32 : 64;
+    if (!map_bf16(&p.tmB, X, a.K, a.M, bn)) return QLORA_ERR_CUDA;
+    p.tmA = p.tmB;
+    if (!map_codes(&p.tmCodes, w, 32, 128)) return QLORA_ERR_CUDA;
+    if (a.r > 0) {
+        if (!map_bf16(&p.tmA2, B, a.r, a.N, 128)) return QLORA_ERR_CUDA;
+        if (!map_bf16(&p.tmB2, L.sU, a.r, a.M, bn)) return QLORA_ERR_CUDA;
+    } else {
+        p.tmA2 = p.tmB;
+        p.tmB2 = p.tmB;
+    }
+    const int tiles = ceil_div(a.N, 128);
+    int splits, per;
+    choose_splits(tiles, p.ks_main, &splits, &per);
+    p.ks_per_split = per;
+    p.rows = (int)a.N;
+    p.cols = (int)a.M;
+    dim3 grid(1, tiles, splits);
+    cudaError_t e;
+    if (splits == 1) {
+        p.out_ld = a.N;
+        if (bn == 32)
+            e = launch_gemm<32, 0, 0, DQ_A_K, EPI_BF16_T, 6>(p, grid, s);
+        else
+            e = launch_gemm<64, 0, 0, DQ_A_K, EPI_BF16_T, 6>(p, grid, s);
+        return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+    }
+    p.out = L.part;
+    p.out_ld = a.N;
+    p.out_split_stride = a.M * a.N;
+    if (bn == 32)
+        e = launch_gemm<32, 0, 0, DQ_A_K, EPI_F32_T, 6>(p, grid, s);
+    else
+        e = launch_gemm<64, 0, 0, DQ_A_K, EPI_F32_T, 6>(p, grid, s);
+    if (e != cudaSuccess) return QLORA_ERR_CUDA;
+    const int64_t total = a.M * a.N;
+    k_splitk_reduce<<<ceil_div(total, 256), 256, 0, s>>>(L.part, splits, a.M * a.N, (int)a.M,
+                                                         (int)a.N, a.N, 1.0f, RED_BF16, Y, a.N);
+    return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+inline qlora_status linear_bwd_impl(const void* dY, const void* X, const LinearArgs& a,
+                                    const void* A, const void* B, void* dX, float* dA, float* dB,
+                                    void* ws, size_t ws_bytes, cudaStream_t s) {
+    (void)ws_bytes;
+    const qlora_nf4_weight& w = *a.w;
+    LinearWs L = carve_linear_ws(ws, a.M, a.N, a.K, a.r, 1);
+    if (a.M == 0) {
+        if (a.r > 0) {
+            k_fill_zero_f32<<<64, 256, 0, s>>>(dA, (int64_t)a.r * a.K);
+            k_fill_zero_f32<<<64, 256, 0, s>>>(dB, a.N * a.r);
+            if (cudaGetLastError() != cudaSuccess) return QLORA_ERR_CUDA;
+        }
+        return QLORA_OK;
+    }
+    if (dX && launch_expand_scales(w, L.scales, L.scales_ld, s) != cudaSuccess) return QLORA_ERR_CUDA;
+    CUtensorMap tdY;
+    if (!map_bf16(&tdY, dY, a.N, a.M, 128)) return QLORA_ERR_CUDA;
+    if (a.r > 0) {
+        qlora_status st = compute_sU(X, a, A, L, s);
+        if (st != QLORA_OK) return st;
+        // sG = bf16(scale * dY B): Aop = dY [m][n] (K-major), Bop = B viewed [j][n] (MN-major)
+        CUtensorMap tBmn;
+        if (!map_bf16(&tBmn, B, a.r, a.N, 64)) return QLORA_ERR_CUDA;
+        st = skinny<0, 1>(tdY, tBmn, (int)a.M, a.r, ceil_div(a.N, 64), L.part, a.scale, RED_BF16,
+                          L.sG, a.r, s);
+        if (st != QLORA_OK) return st;
+    }
+    if (dX) {
+        GemmParams p;
+        memset(&p, 0, sizeof(p));
+        p.tmA = tdY;
+        p.tmB = tdY;
+        if (!map_codes(&p.tmCodes, w, 128, 64)) return QLORA_ERR_CUDA;
+        if (a.r > 0) {
+            if (!map_bf16(&p.tmA2, L.sG, a.r, a.M, 128)) return QLORA_ERR_CUDA;
+            if (!map_bf16(&p.tmB2, A, a.K, a.r, 64)) return QLORA_ERR_CUDA;
+        } else {
+            p.tmA2 = tdY;
+            p.tmB2 = tdY;
+        }
+        p.scales = L.scales;
+        p.scales_ld = L.scales_ld;
+        p.dq_rows = (int)a.N;
+        p.dq_kbs = (int)(a.K / 64);
+        p.ks_main = ceil_div(a.N, 64);
+        p.ks_lora = a.r > 0 ? ceil_div(a.r, 64) : 0;
+        p.ks_per_split = p.ks_main;
+        p.rows = (int)a.M;
+        p.cols = (int)a.K;
+        p.out = dX;
+        p.out_ld = a.K;
+        p.timeout_ns = wait_timeout_ns();
+        p.inject = inject_mode();
+        dim3 grid(ceil_div(a.K, 256), ceil_div(a.M, 128), 1);
+        if (launch_gemm<256, 0, 1, DQ_B_MN, EPI_BF16, 3>(p, grid, s) != cudaSuccess)
+            return QLORA_ERR_CUDA;
+    }
+    if (a.r > 0) {
+        // dA^T [K][r] = X^T sG : Aop = X viewed [k][m] (MN-major), Bop = sG viewed [j][m] (MN-major)
+        CUtensorMap tXmn, tGmn, tdYmn, tUmn;
+        if (!map_bf16(&tXmn, X, a.K, a.M, 64)) return QLORA_ERR_CUDA;
+        if (!map_bf16(&tGmn, L.sG, a.r, a.M, 64)) return QLORA_ERR_CUDA;
+        qlora_status st = skinny<1, 1>(tXmn, tGmn, (int)a.K, a.r, ceil_div(a.M, 64), L.part, 1.0f,
+                                       RED_F32_T, dA, a.K, s);
+        if (st != QLORA_OK) return st;
+        // dB [N][r] = dY^T sU : Aop = dY viewed [n][m] (MN-major), Bop = sU viewed [j][m]
+        if (!map_bf16(&tdYmn, dY, a.N, a.M, 64)) return QLORA_ERR_CUDA;
+        if (!map_bf16(&tUmn, L.sU, a.r, a.M, 64)) return QLORA_ERR_CUDA;
+        st = skinny<1, 1>(tdYmn, tUmn, (int)a.N, a.r, ceil_div(a.M, 64), L.part, 1.0f, RED_F32, dB,
+                          a.r, s);
+        if (st != QLORA_OK) return st;
+    }
+    return QLORA_OK;
+}
+
+}  // namespace qlora

@@ -1,0 +1,192 @@
+// qlora_nf4.cu -- the C ABI of include/qlora_nf4.h: argument validation,
+// workspace queries, the device status word, and dispatch to the kernels.
+// Single translation unit: the kernel headers below are compiled here.
+#include <stdint.h>
+#include <string.h>
+
+#include <atomic>
+
+#include "../../include/qlora_nf4.h"
+#include "common.cuh"
+#include "gemm.cuh"
+#include "internal.h"
+#include "linear.cuh"
+#include "nf4.cuh"
+#include "quantize.cuh"
+
+namespace qlora {
+
+
+static std::atomic<uint64_t> g_timeout_ns{10ull * 1000 * 1000 * 1000};
+static std::atomic<int> g_inject{0};
+
+uint64_t wait_timeout_ns() { return g_timeout_ns.load(); }
+int inject_mode() { return g_inject.load(); }
+
+static bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+static const int64_t kMaxElems = (int64_t)1 << 40;
+
+// Checks shared by every call that reads a quantized weight.
+static qlora_status check_weight(const qlora_nf4_weight* w, bool need_codes) {
+    if (!w) return QLORA_ERR_INVALID_ARG;
+    if (w->rows < 0 || w->cols < 0) return QLORA_ERR_INVALID_ARG;
+    if (w->rows > 0 && w->cols > kMaxElems / w->rows) return QLORA_ERR_INVALID_ARG;
+    if (w->double_quant != 0 && w->double_quant != 1) return QLORA_ERR_INVALID_ARG;
+    if (w->blocksize != 64) return QLORA_ERR_UNSUPPORTED;
+    const int64_t n = w->rows * w->cols;
+    if (n == 0) return QLORA_OK;
+    if (need_codes && (!w->codes || !aligned(w->codes, 16))) return QLORA_ERR_INVALID_ARG;
+    if (w->double_quant) {
+        if (!w->absmax_q8 || !aligned(w->absmax_q8, 8)) return QLORA_ERR_INVALID_ARG;
+        if (!w->absmax_scale || !aligned(w->absmax_scale, 4)) return QLORA_ERR_INVALID_ARG;
+        if (!w->absmax_offset || !aligned(w->absmax_offset, 4)) return QLORA_ERR_INVALID_ARG;
+    } else {
+        if (!w->absmax || !aligned(w->absmax, 4)) return QLORA_ERR_INVALID_ARG;
+    }
+    return QLORA_OK;
+}
+
+static size_t quantize_ws(int64_t n, int dq) {
+    if (!dq || n == 0) return 0;
+    const int64_t nb = (n + 63) / 64;
+    const int64_t ng = (n + 16383) / 16384;
+    return align256((size_t)nb * 4) + align256((size_t)ng * 8);
+}
+
+static qlora_status check_linear(int64_t M, const qlora_nf4_weight* w, int32_t r) {
+    qlora_status st = check_weight(w, true);
+    if (st != QLORA_OK) return st;
+    if (M < 0 || M > ((int64_t)1 << 31)) return QLORA_ERR_INVALID_ARG;
+    if (r < 0) return QLORA_ERR_INVALID_ARG;
+    if (w->cols < 64 || w->rows < 1) return QLORA_ERR_UNSUPPORTED;
+    if (w->cols % 64 != 0 || w->rows % 8 != 0) return QLORA_ERR_UNSUPPORTED;
+    if (w->rows >= ((int64_t)1 << 31) || w->cols >= ((int64_t)1 << 31)) return QLORA_ERR_UNSUPPORTED;
+    if (r % 8 != 0 || r > 256) return QLORA_ERR_UNSUPPORTED;
+    return QLORA_OK;
+}
+
+}  // namespace qlora
+
+using namespace qlora;
+
+extern "C" {
+
+size_t qlora_nf4_quantize_workspace(int64_t rows, int64_t cols, int32_t blocksize,
+                                    int32_t double_quant) {
+    if (rows < 0 || cols < 0 || blocksize != 64) return 0;
+    if (rows > 0 && cols > kMaxElems / rows) return 0;
+    return quantize_ws(rows * cols, double_quant);
+}
+
+qlora_status qlora_nf4_quantize(const void* W, qlora_dtype wdtype, const qlora_nf4_weight* out,
+                                void* ws, size_t ws_bytes, qlora_stream_t stream) {
+    qlora_status st = check_weight(out, true);
+    if (st != QLORA_OK) return st;
+    if (wdtype != QLORA_F32 && wdtype != QLORA_BF16) return QLORA_ERR_INVALID_ARG;
+    const int64_t n = out->rows * out->cols;
+    if (n == 0) return QLORA_OK;
+    if (!W || !aligned(W, 16)) return QLORA_ERR_INVALID_ARG;
+    if (!out->double_quant && (!out->absmax || !aligned(out->absmax, 4))) return QLORA_ERR_INVALID_ARG;
+    const size_t need = quantize_ws(n, out->double_quant);
+    if (need > 0 && (!ws || !aligned(ws, 16) || ws_bytes < need)) return QLORA_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int is_bf16 = wdtype == QLORA_BF16;
+    const int64_t nb = (n + 63) / 64;
+    if (!out->double_quant) {
+        if (launch_quantize_blocks(W, is_bf16, n, out->codes, out->absmax, nullptr, s) != cudaSuccess)
+            return QLORA_ERR_CUDA;
+        return QLORA_OK;
+    }
+    float* absmax = static_cast<float*>(ws);
+    double* sums = reinterpret_cast<double*>(static_cast<char*>(ws) + align256((size_t)nb * 4));
+    const int64_t ng = (n + 16383) / 16384;
+    if (launch_quantize_blocks(W, is_bf16, n, out->codes, absmax, sums, s) != cudaSuccess)
+        return QLORA_ERR_CUDA;
+    if (launch_dq_offset(sums, ng, nb, out->absmax_offset, s) != cudaSuccess) return QLORA_ERR_CUDA;
+    if (launch_dq_quantize(absmax, nb, out->absmax_offset, out->absmax_q8, out->absmax_scale, s) !=
+        cudaSuccess)
+        return QLORA_ERR_CUDA;
+    return QLORA_OK;
+}
+
+qlora_status qlora_nf4_dequantize(const qlora_nf4_weight* w, void* out, qlora_stream_t stream) {
+    qlora_status st = check_weight(w, true);
+    if (st != QLORA_OK) return st;
+    if (w->rows * w->cols == 0) return QLORA_OK;
+    if (!out || !aligned(out, 16)) return QLORA_ERR_INVALID_ARG;
+    if (launch_dequantize(*w, static_cast<uint16_t*>(out), reinterpret_cast<cudaStream_t>(stream)) !=
+        cudaSuccess)
+        return QLORA_ERR_CUDA;
+    return QLORA_OK;
+}
+
+size_t qlora_linear_workspace(int64_t M, const qlora_nf4_weight* w, int32_t r, int32_t bwd) {
+    if (check_linear(M, w, r) != QLORA_OK) return 0;
+    return linear_workspace_bytes(M, w->rows, w->cols, r, bwd ? 1 : 0);
+}
+
+qlora_status qlora_linear_fwd(const void* X, int64_t M, const qlora_nf4_weight* w, const void* A,
+                              const void* B, int32_t r, float scale, void* Y, void* ws,
+                              size_t ws_bytes, qlora_stream_t stream) {
+    qlora_status st = check_linear(M, w, r);
+    if (st != QLORA_OK) return st;
+    if (M == 0) return QLORA_OK;
+    if (!X || !aligned(X, 16) || !Y || !aligned(Y, 16)) return QLORA_ERR_INVALID_ARG;
+    if (r > 0 && (!A || !aligned(A, 16) || !B || !aligned(B, 16))) return QLORA_ERR_INVALID_ARG;
+    const size_t need = linear_workspace_bytes(M, w->rows, w->cols, r, 0);
+    if (!ws || !aligned(ws, 16) || ws_bytes < need) return QLORA_ERR_INVALID_ARG;
+    LinearArgs a{M, w->rows, w->cols, r, scale, w};
+    return linear_fwd_impl(X, a, A, B, Y, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+qlora_status qlora_linear_bwd(const void* dY, const void* X, int64_t M, const qlora_nf4_weight* w,
+                              const void* A, const void* B, int32_t r, float scale, void* dX,
+                              float* dA, float* dB, void* ws, size_t ws_bytes,
+                              qlora_stream_t stream) {
+    qlora_status st = check_linear(M, w, r);
+    if (st != QLORA_OK) return st;
+    if (r > 0 && (!A || !aligned(A, 16) || !B || !aligned(B, 16) || !dA || !aligned(dA, 16) ||
+                  !dB || !aligned(dB, 16)))
+        return QLORA_ERR_INVALID_ARG;
+    if (M > 0) {
+        if (!dY || !aligned(dY, 16) || !X || !aligned(X, 16)) return QLORA_ERR_INVALID_ARG;
+        if (dX && !aligned(dX, 16)) return QLORA_ERR_INVALID_ARG;
+    }
+    const size_t need = linear_workspace_bytes(M, w->rows, w->cols, r, 1);
+    if (!ws || !aligned(ws, 16) || ws_bytes < need) return QLORA_ERR_INVALID_ARG;
+    LinearArgs a{M, w->rows, w->cols, r, scale, w};
+    return linear_bwd_impl(dY, X, a, A, B, dX, dA, dB, ws, ws_bytes,
+                           reinterpret_cast<cudaStream_t>(stream));
+}
+
+qlora_status qlora_get_last_error(qlora_stream_t stream) {
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return QLORA_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return QLORA_ERR_CUDA;
+    if (v != 0) {
+        int zero = 0;
+        if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return QLORA_ERR_CUDA;
+    }
+    return static_cast<qlora_status>(v);
+}
+
+void qlora_nf4_table(float out[16]) { nf4_table_host(out); }
+
+qlora_status qlora_nf4_encode(const float* x, int64_t n, uint8_t* codes, qlora_stream_t stream) {
+    if (n < 0) return QLORA_ERR_INVALID_ARG;
+    if (n == 0) return QLORA_OK;
+    if (!x || !codes || !aligned(x, 4)) return QLORA_ERR_INVALID_ARG;
+    if (launch_encode(x, n, codes, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return QLORA_ERR_CUDA;
+    return QLORA_OK;
+}
+
+void qlora_set_wait_timeout_ns(uint64_t ns) {
+    g_timeout_ns.store(ns ? ns : 10ull * 1000 * 1000 * 1000);
+}
+
+void qlora_debug_inject(int32_t mode) { g_inject.store(mode); }
+
+}  // extern "C"

@@ -1,0 +1,430 @@
+// quantize.cuh -- NF4 blockwise quantizer, double quantization of the block
+// constants, standalone dequantization, and the block-constant expansion used
+// by the dequant-GEMM producers.  All kernels are HBM-streaming kernels:
+// 128-bit loads and stores, warp shuffles for the block reductions.
+//
+// Definitions (QLoRA blog note p19e99 sec. 2 "NF4" and sec. 3 "double
+// quantization"; QLoRA paper digest sec. 4 "NF4", "double quantization",
+// doubleDequant; tutorial "11.3 QLoRA" section "double quantization": 64
+// parameters share one fp32 constant, the constants go to 8 bits):
+//  - block b = elements [64b, 64b+64) of the flattened row-major tensor (the
+//    last block may be shorter); a_b = max |w| over the block.
+//  - x = fl32((w * p) * fl32(1 / (a_b * p))) with the exact power-of-two
+//    prescale p = 2^64 when a_b < 2^-126 (so the reciprocal stays finite),
+//    p = 1 otherwise; a zero block uses the factor 0.
+//  - code = index of the nearest NF4 value, exact ties to the lower index.
+//  - byte i of the packed codes = (code[2i] << 4) | code[2i+1].
+//  - double quantization: offset = fl32(S / nb) with S the fp64 pairwise-tree
+//    sum of all a_b (zero-padded to a power of two); d_b = fl32(a_b - offset);
+//    c1[g] = max |d_b| over blocks [256g, 256g+256); y = fl32((d_b p) *
+//    fl32(1/(c1 p))) (same prescale rule, factor 0 when c1 == 0); q8 = index
+//    of the nearest t8[k] = fl32((k-127)/127), ties to the lower index.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include <cmath>
+#include <cstring>
+
+#include "common.cuh"
+#include "internal.h"
+#include "nf4.cuh"
+
+namespace qlora {
+
+// ---------------------------------------------------------------------------
+// fast nearest-code search
+// ---------------------------------------------------------------------------
+// x in [-1.03, 1.03] falls in bucket key = RN(16 x + 16) in 0..32, i.e. the
+// closed interval [(key - 1/2)/16 - 1, (key + 1/2)/16 - 1].  Buckets are
+// narrower than the smallest gap between two decision thresholds (0.080), so
+// each holds at most one threshold T_key; base_key counts the thresholds at
+// or below the bucket's lower edge.  code(x) = base_key + (x >= T_key), where
+// threshold j is the smallest fp32 strictly above the exact midpoint of codes
+// j and j+1 (so an exact tie stays with the lower code).
+__device__ __forceinline__ int nf4_search(float x, const float2* tab) {
+    const float t = fmaf(x, 16.0f, 12582928.0f);  // 1.5 * 2^23 + 16: RN to an integer
+    const uint32_t key = min(__float_as_uint(t) - 0x4B400000u, 32u);
+    const float2 e = tab[key];
+    return __float_as_int(e.y) + (x >= e.x ? 1 : 0);
+}
+
+// ---------------------------------------------------------------------------
+// K1: quantize.  One CTA (8 warps) per group of 256 blocks (16384 elements);
+// warp w handles rows 4w..4w+3 of 512 elements; a lane holds 16 consecutive
+// elements, four lanes make one block.  Also writes the group's fp64
+// pairwise-tree sum of block maxima for the double-quantization offset.
+// ---------------------------------------------------------------------------
+template <bool BF16>
+__global__ void __launch_bounds__(256) k_quantize_blocks(const void* __restrict__ W, int64_t n,
+                                                         uint8_t* __restrict__ codes,
+                                                         float* __restrict__ absmax,
+                                                         double* __restrict__ group_sums,
+                                                         Nf4SearchTable tab) {
+    __shared__ float2 s_tab[33];
+    __shared__ double s_wsum[8];
+    if (threadIdx.x < 33)
+        s_tab[threadIdx.x] = make_float2(tab.thr[threadIdx.x], __int_as_float(tab.base[threadIdx.x]));
+    __syncthreads();
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t nb = (n + 63) >> 6;
+    constexpr int WORDS = BF16 ? 8 : 16;  // 32-bit words per lane per row
+    uint32_t raw[4][WORDS];
+    int64_t e0[4];
+
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+        e0[it] = (int64_t)blockIdx.x * 16384 + (int64_t)(warp * 4 + it) * 512 + lane * 16;
+        if (e0[it] + 16 <= n) {
+            const uint4* src = BF16 ? reinterpret_cast<const uint4*>(
+                                          static_cast<const uint16_t*>(W) + e0[it])
+                                    : reinterpret_cast<const uint4*>(
+                                          static_cast<const float*>(W) + e0[it]);
+#pragma unroll
+            for (int v = 0; v < WORDS / 4; ++v) {
+                uint4 q = __ldg(src + v);
+                raw[it][4 * v + 0] = q.x;
+                raw[it][4 * v + 1] = q.y;
+                raw[it][4 * v + 2] = q.z;
+                raw[it][4 * v + 3] = q.w;
+            }
+        } else {
+#pragma unroll
+            for (int v = 0; v < WORDS; ++v) raw[it][v] = 0u;
+            if (e0[it] < n) {
+                for (int i = 0; i < 16 && e0[it] + i < n; ++i) {
+                    if (BF16) {
+                        uint32_t h = static_cast<const uint16_t*>(W)[e0[it] + i];
+                        raw[it][i >> 1] |= h << ((i & 1) * 16);
+                    } else {
+                        raw[it][i] = __float_as_uint(static_cast<const float*>(W)[e0[it] + i]);
+                    }
+                }
+            }
+        }
+    }
+
+    double rowsum[4];
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+        float v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            if (BF16)
+                v[i] = __uint_as_float((i & 1) ? (raw[it][i >> 1] & 0xFFFF0000u)
+                                               : (raw[it][i >> 1] << 16));
+            else
+                v[i] = __uint_as_float(raw[it][i]);
+        }
+        float a = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(v[i]));
+        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+
+        const int64_t b = e0[it] >> 6;
+        const bool bvalid = b < nb;
+        if (bvalid && (lane & 3) == 0 && absmax) absmax[b] = a;
+
+        float p = 1.0f;
+        if (a < 1.17549435e-38f) p = 18446744073709551616.0f;  // 2^64, exact prescale
+        const float rcp = (a == 0.0f) ? 0.0f : __frcp_rn(__fmul_rn(a, p));
+        uint32_t c[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            float x = __fmul_rn(__fmul_rn(v[i], p), rcp);
+            c[i] = (uint32_t)nf4_search(x, s_tab);
+        }
+        uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            w0 |= ((c[2 * j] << 4) | c[2 * j + 1]) << (8 * j);
+            w1 |= ((c[8 + 2 * j] << 4) | c[8 + 2 * j + 1]) << (8 * j);
+        }
+        if (e0[it] + 16 <= n) {
+            *reinterpret_cast<uint2*>(codes + (e0[it] >> 1)) = make_uint2(w0, w1);
+        } else if (e0[it] < n) {
+            const int valid = (int)(n - e0[it]);
+            for (int j = 0; 2 * j < valid; ++j) {
+                uint32_t byte = c[2 * j] << 4;
+                if (2 * j + 1 < valid) byte |= c[2 * j + 1];
+                codes[(e0[it] >> 1) + j] = (uint8_t)byte;
+            }
+        }
+
+        // fp64 pairwise tree over the row's 8 block maxima (blocks beyond
+        // the tensor contribute zeros).
+        double d = bvalid ? (double)a : 0.0;
+        d += __shfl_xor_sync(0xffffffffu, d, 4);
+        d += __shfl_xor_sync(0xffffffffu, d, 8);
+        d += __shfl_xor_sync(0xffffffffu, d, 16);
+        rowsum[it] = d;
+    }
+    if (group_sums) {
+        if (lane == 0) s_wsum[warp] = (rowsum[0] + rowsum[1]) + (rowsum[2] + rowsum[3]);
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            double t0 = s_wsum[0] + s_wsum[1], t1 = s_wsum[2] + s_wsum[3];
+            double t2 = s_wsum[4] + s_wsum[5], t3 = s_wsum[6] + s_wsum[7];
+            group_sums[blockIdx.x] = (t0 + t1) + (t2 + t3);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// K2: offset = fl32(S / nb), S = pairwise tree over the group sums padded
+// with zeros to a power of two.  One CTA of 1024 threads; thread t sums a
+// contiguous power-of-two chunk with a binary-counter pairwise sum.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024) k_dq_offset(const double* __restrict__ sums, int64_t ng,
+                                                    int64_t nb, float* __restrict__ offset) {
+    __shared__ double s_w[32];
+    int64_t p2 = 1;
+    while (p2 < ng) p2 <<= 1;
+    const int64_t chunk = p2 > 1024 ? p2 / 1024 : 1;
+    double stack[40];
+    int64_t cnt = 0;
+    const int64_t lo = (int64_t)threadIdx.x * chunk;
+    for (int64_t i = 0; i < chunk; ++i) {
+        int64_t idx = lo + i;
+        double v = idx < ng ? sums[idx] : 0.0;
+        int lvl = 0;
+        while ((cnt >> lvl) & 1) {
+            v = stack[lvl] + v;
+            ++lvl;
+        }
+        stack[lvl] = v;
+        ++cnt;
+    }
+    int top = 0;
+    while ((1ll << top) < chunk) ++top;
+    double t = stack[top];
+    for (int o = 1; o < 32; o <<= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    if ((threadIdx.x & 31) == 0) s_w[threadIdx.x >> 5] = t;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        double u = s_w[threadIdx.x];
+        for (int o = 1; o < 32; o <<= 1) u += __shfl_xor_sync(0xffffffffu, u, o);
+        if (threadIdx.x == 0) *offset = __double2float_rn(__ddiv_rn(u, (double)nb));
+    }
+}
+
+// Nearest 8-bit code of y in [-1, 1]: candidate from rint(127 y), then the
+// exact fp64 distances of it and its two neighbours; ties to the lower index.
+__device__ __forceinline__ int nearest_t8(float y) {
+    int k0 = __float2int_rn(__fmul_rn(y, 127.0f)) + 127;
+    k0 = min(max(k0, 0), 254);
+    int best = k0;
+    double bd = fabs((double)y - (double)t8_value(k0));
+    if (k0 > 0) {
+        double d = fabs((double)y - (double)t8_value(k0 - 1));
+        if (d <= bd) {
+            bd = d;
+            best = k0 - 1;
+        }
+    }
+    if (k0 < 254) {
+        double d = fabs((double)y - (double)t8_value(k0 + 1));
+        if (d < bd) best = k0 + 1;
+    }
+    return best;
+}
+
+// ---------------------------------------------------------------------------
+// K3: second-level quantization; one warp per group of 256 block constants.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_dq_quantize(const float* __restrict__ absmax, int64_t nb,
+                                                     const float* __restrict__ offset_ptr,
+                                                     uint8_t* __restrict__ q8,
+                                                     float* __restrict__ c1) {
+    const int64_t g = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    const int64_t ng = (nb + 255) >> 8;
+    if (g >= ng) return;
+    const float off = *offset_ptr;
+    const int64_t b0 = g * 256 + lane * 8;
+    float d[8];
+    float c = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        d[i] = (b0 + i < nb) ? __fsub_rn(absmax[b0 + i], off) : 0.0f;
+        c = fmaxf(c, fabsf(d[i]));
+    }
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) c = fmaxf(c, __shfl_xor_sync(0xffffffffu, c, o));
+    float p = 1.0f;
+    if (c < 1.17549435e-38f) p = 18446744073709551616.0f;
+    const float rc = (c == 0.0f) ? 0.0f : __frcp_rn(__fmul_rn(c, p));
+    uint32_t q[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) q[i] = (uint32_t)nearest_t8(__fmul_rn(__fmul_rn(d[i], p), rc));
+    if (b0 + 8 <= nb) {
+        uint2 v;
+        v.x = q[0] | (q[1] << 8) | (q[2] << 16) | (q[3] << 24);
+        v.y = q[4] | (q[5] << 8) | (q[6] << 16) | (q[7] << 24);
+        *reinterpret_cast<uint2*>(q8 + b0) = v;
+    } else {
+        for (int i = 0; i < 8; ++i)
+            if (b0 + i < nb) q8[b0 + i] = (uint8_t)q[i];
+    }
+    if (lane == 0) c1[g] = c;
+}
+
+// ---------------------------------------------------------------------------
+// K4: standalone dequantization, one thread per 64-element block.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_dequantize(const uint8_t* __restrict__ codes, int64_t n,
+                                                    int dq, const float* __restrict__ absmax,
+                                                    const uint8_t* __restrict__ q8,
+                                                    const float* __restrict__ c1,
+                                                    const float* __restrict__ offset_ptr,
+                                                    uint16_t* __restrict__ out) {
+    const int64_t b = (int64_t)blockIdx.x * 256 + threadIdx.x;
+    const int64_t nb = (n + 63) >> 6;
+    if (b >= nb) return;
+    const float a = dq ? block_scale_dq(q8[b], c1[b >> 8], *offset_ptr) : absmax[b];
+    if ((b + 1) * 64 <= n) {
+        const uint4* src = reinterpret_cast<const uint4*>(codes + b * 32);
+        uint4 c0 = __ldg(src), c1v = __ldg(src + 1);
+        const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1v.x, c1v.y, c1v.z, c1v.w};
+        const Nf4BlockTable t = nf4_block_table(a);
+        uint4* dst = reinterpret_cast<uint4*>(out + b * 64);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            uint32_t o[4];
+            nf4_expand_word(words[i], t, o);
+            dst[i] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+    } else {
+        for (int64_t e = b * 64; e < n; ++e) {
+            uint8_t byte = codes[e >> 1];
+            int c = (e & 1) ? (byte & 15) : (byte >> 4);
+            __nv_bfloat16 h = __float2bfloat16_rn(__fmul_rn(nf4_value(c), a));
+            out[e] = *reinterpret_cast<uint16_t*>(&h);
+        }
+    }
+}
+
+// Block constants a' transposed for the GEMM producers: scales[kb*ld + n].
+__global__ void k_expand_scales(int64_t rows, int64_t kbs, int dq, const float* __restrict__ absmax,
+                                const uint8_t* __restrict__ q8, const float* __restrict__ c1,
+                                const float* __restrict__ offset_ptr, float* __restrict__ scales,
+                                int64_t ld) {
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= rows * kbs) return;
+    const int64_t kb = idx / rows, n = idx - kb * rows;
+    const int64_t b = n * kbs + kb;
+    scales[kb * ld + n] = dq ? block_scale_dq(q8[b], c1[b >> 8], *offset_ptr) : absmax[b];
+}
+
+__global__ void k_encode(const float* __restrict__ x, int64_t n, uint8_t* __restrict__ codes,
+                         Nf4SearchTable tab) {
+    __shared__ float2 s_tab[33];
+    if (threadIdx.x < 33)
+        s_tab[threadIdx.x] = make_float2(tab.thr[threadIdx.x], __int_as_float(tab.base[threadIdx.x]));
+    __syncthreads();
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        float v = fminf(fmaxf(x[i], -1.0f), 1.0f);
+        codes[i] = (uint8_t)nf4_search(v, s_tab);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+
+inline void nf4_table_host(float out[16]) {
+    for (int j = 0; j < 16; ++j) {
+        uint32_t u = kNF4Bits[j];
+        memcpy(&out[j], &u, 4);
+    }
+}
+
+inline Nf4SearchTable build_search_table() {
+    float v[16];
+    nf4_table_host(v);
+    float thr[15];
+    for (int j = 0; j < 15; ++j) {
+        double mid = 0.5 * ((double)v[j] + (double)v[j + 1]);  // exact in fp64
+        float f = (float)mid;
+        if ((double)f <= mid) f = std::nextafter(f, INFINITY);
+        thr[j] = f;
+    }
+    Nf4SearchTable t;
+    for (int k = 0; k <= 32; ++k) {
+        double lo = (k - 0.5) / 16.0 - 1.0, hi = (k + 0.5) / 16.0 - 1.0;
+        int base = 0;
+        float tk = 3.0f;  // no threshold inside the bucket
+        for (int j = 0; j < 15; ++j) {
+            if ((double)thr[j] <= lo) ++base;
+            else if ((double)thr[j] <= hi) tk = thr[j];
+        }
+        t.thr[k] = tk;
+        t.base[k] = base;
+    }
+    return t;
+}
+
+inline const Nf4SearchTable& nf4_search_table() {
+    static const Nf4SearchTable t = build_search_table();
+    return t;
+}
+
+inline cudaError_t launch_quantize_blocks(const void* W, int is_bf16, int64_t n, uint8_t* codes,
+                                          float* absmax, double* group_sums, cudaStream_t s) {
+    const int64_t ng = (n + 16383) / 16384;
+    if (ng == 0) return cudaSuccess;
+    if (is_bf16)
+        k_quantize_blocks<true><<<(unsigned)ng, 256, 0, s>>>(W, n, codes, absmax, group_sums,
+                                                              nf4_search_table());
+    else
+        k_quantize_blocks<false><<<(unsigned)ng, 256, 0, s>>>(W, n, codes, absmax, group_sums,
+                                                               nf4_search_table());
+    return cudaGetLastError();
+}
+
+inline cudaError_t launch_dq_offset(const double* group_sums, int64_t ngroups, int64_t nb,
+                                    float* offset, cudaStream_t s) {
+    k_dq_offset<<<1, 1024, 0, s>>>(group_sums, ngroups, nb, offset);
+    return cudaGetLastError();
+}
+
+inline cudaError_t launch_dq_quantize(const float* absmax, int64_t nb, const float* offset,
+                                      uint8_t* q8, float* c1, cudaStream_t s) {
+    const int64_t ng = (nb + 255) / 256;
+    if (ng == 0) return cudaSuccess;
+    k_dq_quantize<<<(unsigned)((ng + 7) / 8), 256, 0, s>>>(absmax, nb, offset, q8, c1);
+    return cudaGetLastError();
+}
+
+inline cudaError_t launch_dequantize(const qlora_nf4_weight& w, uint16_t* out, cudaStream_t s) {
+    const int64_t n = w.rows * w.cols;
+    const int64_t nb = (n + 63) / 64;
+    if (nb == 0) return cudaSuccess;
+    k_dequantize<<<(unsigned)((nb + 255) / 256), 256, 0, s>>>(
+        w.codes, n, w.double_quant, w.absmax, w.absmax_q8, w.absmax_scale, w.absmax_offset, out);
+    return cudaGetLastError();
+}
+
+inline cudaError_t launch_expand_scales(const qlora_nf4_weight& w, float* scales, int64_t ld,
+                                        cudaStream_t s) {
+    const int64_t kbs = w.cols / 64;
+    const int64_t total = w.rows * kbs;
+    if (total == 0) return cudaSuccess;
+    k_expand_scales<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(
+        w.rows, kbs, w.double_quant, w.absmax, w.absmax_q8, w.absmax_scale, w.absmax_offset,
+        scales, ld);
+    return cudaGetLastError();
+}
+
+inline cudaError_t launch_encode(const float* x, int64_t n, uint8_t* codes, cudaStream_t s) {
+    if (n == 0) return cudaSuccess;
+    int64_t blocks = (n + 255) / 256;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    k_encode<<<(unsigned)blocks, 256, 0, s>>>(x, n, codes, nf4_search_table());
+    return cudaGetLastError();
+}
+
+}  // namespace qlora

@@ -1,0 +1,194 @@
+/*
+ * qlora_nf4.h -- C ABI of the B200 (sm_100a) QLoRA NF4 frozen-linear library.
+ *
+ * The library implements one layer, the QLoRA linear of the QLoRA paper
+ * digest (aipaper.cc, "QLoRA: Efficient Finetuning of Quantized LLMs",
+ * sec. 4 "full QLoRA equation"):
+ *
+ *     Y = X * doubleDequant(c1, c2, W_nf4)^T + s * (X * A^T) * B^T
+ *
+ * in the shapes of the LoRA reproduction blog ("LoRA / QLoRA low-rank update,
+ * quantization and memory budget", section "LoRA formula and tensor shapes"):
+ * W [N = d_out, K = d_in], A [r, K], B [N, r], X [M, K], Y [M, N], s = alpha/r.
+ * Beside it sits the blockwise NF4 quantizer that produces W_nf4 (QLoRA blog
+ * note p19e99 sec. 2 "NF4"; digest sec. 4 "NF4" and "double quantization").
+ *
+ * Conventions for every entry point
+ *  - All tensor pointers are DEVICE pointers to caller-owned memory, dense and
+ *    row-major.  The library keeps no pointer after a call returns and
+ *    allocates no device memory: temporary storage comes from the caller's
+ *    workspace, whose size the matching *_workspace() query gives.
+ *  - Work is enqueued asynchronously on `stream` (NULL = legacy default).
+ *  - Arguments are validated on the host before anything is launched; a bad
+ *    argument returns QLORA_ERR_INVALID_ARG or QLORA_ERR_UNSUPPORTED and
+ *    enqueues nothing.  A failed launch returns QLORA_ERR_CUDA.
+ *  - Every wait inside a kernel is bounded in time.  A wait that runs out
+ *    records QLORA_ERR_TIMEOUT in a per-device status word and the kernel
+ *    returns; qlora_get_last_error() reports (and clears) that word.
+ *  - bf16 tensors are passed as `const void *` and hold IEEE bfloat16 bits.
+ *  - Alignment: bf16 tensors, codes and the workspace must be 16-byte
+ *    aligned; fp32 tensors 4-byte aligned (QLORA_ERR_INVALID_ARG otherwise).
+ */
+#ifndef QLORA_NF4_H
+#define QLORA_NF4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *qlora_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    QLORA_OK = 0,
+    QLORA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, negative size, small workspace */
+    QLORA_ERR_UNSUPPORTED = 2, /* valid but outside this build: blocksize != 64,
+                                  K % 64 != 0, N % 8 != 0, r % 8 != 0, r > 256 */
+    QLORA_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
+    QLORA_ERR_TIMEOUT = 4,     /* a bounded in-kernel wait ran out (reported
+                                  by qlora_get_last_error only) */
+    QLORA_ERR_WORKSPACE = 5    /* reserved */
+} qlora_status;
+
+typedef enum { QLORA_F32 = 0, QLORA_BF16 = 1 } qlora_dtype;
+
+/*
+ * A quantized frozen weight W [rows = N, cols = K].
+ * Blocks are 64 consecutive elements of the row-major flattened tensor
+ * (QLoRA tutorial "11.3 QLoRA", section "double quantization": 64 parameters
+ * share one constant); nb = ceil(rows*cols / 64), nb2 = ceil(nb / 256).
+ *   codes          [ceil(rows*cols/2)] bytes.  Element 2i sits in the high
+ *                  nibble of byte i, element 2i+1 in the low nibble; the
+ *                  nibble is the index (0..15) of the nearest NF4 code.
+ *   absmax         [nb] fp32 block absolute maxima; read/written only when
+ *                  double_quant == 0.
+ *   absmax_q8      [nb] bytes, index k of the 8-bit code (k-127)/127 of the
+ *                  centred block constant; used when double_quant == 1.
+ *   absmax_scale   [nb2] fp32 second-level constants c1 (one per 256 blocks).
+ *   absmax_offset  [1] fp32 mean of all block maxima, subtracted before the
+ *                  8-bit quantization.
+ * Dequantized weight (digest sec. 4, doubleDequant):
+ *   a'  = double_quant ? (t8[q8] * c1) + offset : absmax     (fp32, two roundings)
+ *   w'  = bf16_round_nearest_even(nf4[code] * a')
+ */
+typedef struct {
+    int64_t rows;          /* N (d_out) */
+    int64_t cols;          /* K (d_in)  */
+    int32_t blocksize;     /* must be 64 */
+    int32_t double_quant;  /* 0 or 1 */
+    uint8_t *codes;
+    float *absmax;
+    uint8_t *absmax_q8;
+    float *absmax_scale;
+    float *absmax_offset;
+} qlora_nf4_weight;
+
+/*
+ * Workspace bytes that qlora_nf4_quantize needs for a tensor of rows*cols
+ * elements (0 when double_quant == 0).  Returns 0 for invalid sizes.
+ */
+size_t qlora_nf4_quantize_workspace(int64_t rows, int64_t cols, int32_t blocksize,
+                                    int32_t double_quant);
+
+/*
+ * Blockwise NF4 quantization (QLoRA blog note p19e99 sec. 2: rescale each
+ * block by its absolute maximum into [-1, 1], store the index of the nearest
+ * of 16 normal-quantile codes in 4 bits) followed, when out->double_quant,
+ * by double quantization of the block constants to 8 bits (digest sec. 4
+ * "double quantization"; blog note sec. 3).
+ *   W      device [rows, cols] in `wdtype` (bf16 or fp32), finite values.
+ *   out    describes caller-allocated outputs; rows, cols, blocksize,
+ *          double_quant and the output pointers must be set.  Any rows*cols
+ *          >= 0 is accepted (the last block may be partial; rows*cols == 0
+ *          enqueues nothing).
+ *   ws     device workspace of at least qlora_nf4_quantize_workspace() bytes
+ *          (may be NULL when that is 0).
+ * Deterministic: the same input gives bit-identical outputs.
+ */
+qlora_status qlora_nf4_quantize(const void *W, qlora_dtype wdtype, const qlora_nf4_weight *out,
+                                void *ws, size_t ws_bytes, qlora_stream_t stream);
+
+/*
+ * doubleDequant (digest sec. 4): writes the bf16 weight w' [rows, cols] that
+ * the linear layer multiplies with.  `out` is a device bf16 buffer.
+ */
+qlora_status qlora_nf4_dequantize(const qlora_nf4_weight *w, void *out, qlora_stream_t stream);
+
+/*
+ * Workspace bytes of qlora_linear_fwd (bwd == 0) or qlora_linear_bwd
+ * (bwd == 1) for M tokens, weight w and rank r.  Returns 0 for invalid sizes.
+ */
+size_t qlora_linear_workspace(int64_t M, const qlora_nf4_weight *w, int32_t r, int32_t bwd);
+
+/*
+ * Forward of the frozen NF4 linear with a LoRA adapter (LoRA reproduction
+ * blog, "LoRA formula and tensor shapes": y = x W0^T + (alpha/r) x A^T B^T,
+ * with W0 the dequantized NF4 weight of the QLoRA paper notes, "Key design 3"):
+ *   Y[m,n] = sum_k X[m,k] w'[n,k] + scale * sum_j U[m,j] B[n,j],
+ *   U      = X A^T.
+ *   X [M, K] bf16, A [r, K] bf16, B [N, r] bf16, Y [M, N] bf16 (written).
+ *   r == 0 disables the adapter (A, B may be NULL).  M >= 0.
+ * Products accumulate in fp32; U is rounded to bf16 after scaling by `scale`.
+ * Requires K % 64 == 0, N % 8 == 0, r % 8 == 0, r <= 256.
+ */
+qlora_status qlora_linear_fwd(const void *X, int64_t M, const qlora_nf4_weight *w, const void *A,
+                              const void *B, int32_t r, float scale, void *Y, void *ws,
+                              size_t ws_bytes, qlora_stream_t stream);
+
+/*
+ * Backward of the same layer.  Gradients flow through the dequantized frozen
+ * weight into the adapters only (digest sec. 4 steps 4; the reproduction
+ * blog's invariant "the frozen weight's gradient is empty"), so there is no
+ * dW output.  With G = dY B:
+ *   dX = dY w' + scale * G A        [M, K] bf16 (written)
+ *   dA = scale * G^T X              [r, K] fp32 (written)
+ *   dB = scale * dY^T (X A^T)       [N, r] fp32 (written)
+ *   dY [M, N] bf16, X [M, K] bf16.  dX may be NULL to skip it.  With r == 0
+ *   only dX is produced.  With M == 0, dA and dB are set to zero.
+ * Same shape requirements as qlora_linear_fwd.  Deterministic (no floating
+ * point atomics on any output).
+ */
+qlora_status qlora_linear_bwd(const void *dY, const void *X, int64_t M, const qlora_nf4_weight *w,
+                              const void *A, const void *B, int32_t r, float scale, void *dX,
+                              float *dA, float *dB, void *ws, size_t ws_bytes,
+                              qlora_stream_t stream);
+
+/*
+ * Synchronizes `stream`, then returns (and clears) the device status word of
+ * the current device: QLORA_ERR_TIMEOUT if a bounded in-kernel wait ran out
+ * since the last call, QLORA_ERR_CUDA if the stream reports an error,
+ * QLORA_OK otherwise.
+ */
+qlora_status qlora_get_last_error(qlora_stream_t stream);
+
+/* Host copy of the 16 NF4 codes this library uses (sorted, index 7 == 0). */
+void qlora_nf4_table(float out[16]);
+
+/*
+ * Nearest-NF4-code search of the quantizer, exposed so that it can be checked
+ * on every fp32 input: codes[i] = index (0..15) of the NF4 code nearest to
+ * x[i], exact ties to the lower index.  x and codes are device arrays of n
+ * elements (one code per byte).  Test entry point.
+ */
+qlora_status qlora_nf4_encode(const float *x, int64_t n, uint8_t *codes, qlora_stream_t stream);
+
+/*
+ * Upper bound, in nanoseconds, of every in-kernel wait (default 10 s).
+ * Test entry point; 0 restores the default.
+ */
+void qlora_set_wait_timeout_ns(uint64_t ns);
+
+/*
+ * Fault injection for the failure-detection tests.  Mode 1 makes the next
+ * launches of the tensor-core GEMM skip their producer's loads, so that the
+ * consumers' bounded waits run out and QLORA_ERR_TIMEOUT is recorded; mode 0
+ * turns it off.  No GPU fault is raised: the kernels return normally.
+ */
+void qlora_debug_inject(int32_t mode);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QLORA_NF4_H */

@@ -1,0 +1,124 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every function include/qlora_nf4.h declares, answers workspace queries, and
+rejects bad arguments before launching anything."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qlora_nf4.h")
+
+FAKE = 0x7F0000000000  # 256-byte aligned stand-in pointer; never dereferenced
+
+
+def _declared_functions():
+    txt = open(HEADER).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    names = re.findall(r"\b(qlora_[a-z0-9_]+)\s*\(", txt)
+    return sorted(set(names))
+
+
+def test_header_and_exports(Q):
+    from bit_nf4_quantized_08_b200 import _lib
+    lib = _lib.lib()
+    declared = _declared_functions()
+    assert set(declared) == set(_lib.EXPORTS)
+    for name in declared:
+        assert hasattr(lib, name), f"{name} not exported"
+
+
+def test_nf4_table_matches_oracle(Q, O):
+    np.testing.assert_array_equal(np.array(Q.qlora_nf4_table(), np.float32).view(np.uint32),
+                                  O.nf4_table().view(np.uint32))
+
+
+def _w(rows=256, cols=256, dq=1, blocksize=64, codes=FAKE):
+    from bit_nf4_quantized_08_b200._lib import CNF4Weight
+    return CNF4Weight(rows, cols, blocksize, dq, codes, FAKE, FAKE, FAKE, FAKE)
+
+
+def test_quantize_workspace_sizes(Q):
+    from bit_nf4_quantized_08_b200._lib import lib
+    L = lib()
+    assert L.qlora_nf4_quantize_workspace(4096, 4096, 64, 0) == 0
+    n = 4096 * 4096
+    nb, ng = n // 64, n // 16384
+    assert L.qlora_nf4_quantize_workspace(4096, 4096, 64, 1) == nb * 4 + ng * 8
+    assert L.qlora_nf4_quantize_workspace(4096, 4096, 32, 1) == 0
+    assert L.qlora_nf4_quantize_workspace(-1, 4, 64, 1) == 0
+
+
+def test_quantize_rejects(Q):
+    from bit_nf4_quantized_08_b200._lib import lib, QLORA_ERR_INVALID_ARG, QLORA_ERR_UNSUPPORTED, QLORA_BF16
+    L = lib()
+    ws = FAKE
+    big = 1 << 30
+    assert L.qlora_nf4_quantize(FAKE, QLORA_BF16, None, ws, big, None) == QLORA_ERR_INVALID_ARG
+    assert L.qlora_nf4_quantize(FAKE, QLORA_BF16, ctypes.byref(_w(blocksize=128)), ws, big, None) == QLORA_ERR_UNSUPPORTED
+    assert L.qlora_nf4_quantize(None, QLORA_BF16, ctypes.byref(_w()), ws, big, None) == QLORA_ERR_INVALID_ARG
+    assert L.qlora_nf4_quantize(FAKE + 8, QLORA_BF16, ctypes.byref(_w()), ws, big, None) == QLORA_ERR_INVALID_ARG
+    assert L.qlora_nf4_quantize(FAKE, 7, ctypes.byref(_w()), ws, big, None) == QLORA_ERR_INVALID_ARG
+    assert L.qlora_nf4_quantize(FAKE, QLORA_BF16, ctypes.byref(_w()), ws, 16, None) == QLORA_ERR_INVALID_ARG
+    assert L.qlora_nf4_quantize(FAKE, QLORA_BF16, ctypes.byref(_w(dq=2)), ws, big, None) == QLORA_ERR_INVALID_ARG
+    assert L.qlora_nf4_quantize(FAKE, QLORA_BF16, ctypes.byref(_w(rows=-3)), ws, big, None) == QLORA_ERR_INVALID_ARG
+    assert L.qlora_nf4_quantize(FAKE, QLORA_BF16, ctypes.byref(_w(codes=FAKE + 4)), ws, big, None) == QLORA_ERR_INVALID_ARG
+    # an empty tensor is valid and enqueues nothing
+    assert L.qlora_nf4_quantize(None, QLORA_BF16, ctypes.byref(_w(rows=0)), None, 0, None) == 0
+
+
+def test_linear_rejects(Q):
+    from bit_nf4_quantized_08_b200._lib import lib, QLORA_ERR_INVALID_ARG, QLORA_ERR_UNSUPPORTED
+    L = lib()
+    big = 1 << 34
+    f = L.qlora_linear_fwd
+    w = _w(256, 256)
+    assert f(FAKE, 16, ctypes.byref(_w(256, 200)), FAKE, FAKE, 8, 2.0, FAKE, FAKE, big, None) == QLORA_ERR_UNSUPPORTED
+    assert f(FAKE, 16, ctypes.byref(_w(260, 256)), FAKE, FAKE, 8, 2.0, FAKE, FAKE, big, None) == QLORA_ERR_UNSUPPORTED
+    assert f(FAKE, 16, ctypes.byref(w), FAKE, FAKE, 12, 2.0, FAKE, FAKE, big, None) == QLORA_ERR_UNSUPPORTED
+    assert f(FAKE, 16, ctypes.byref(w), FAKE, FAKE, 264, 2.0, FAKE, FAKE, big, None) == QLORA_ERR_UNSUPPORTED
+    assert f(FAKE, 16, ctypes.byref(w), FAKE, FAKE, -8, 2.0, FAKE, FAKE, big, None) == QLORA_ERR_INVALID_ARG
+    assert f(FAKE, -1, ctypes.byref(w), FAKE, FAKE, 8, 2.0, FAKE, FAKE, big, None) == QLORA_ERR_INVALID_ARG
+    assert f(None, 16, ctypes.byref(w), FAKE, FAKE, 8, 2.0, FAKE, FAKE, big, None) == QLORA_ERR_INVALID_ARG
+    assert f(FAKE, 16, ctypes.byref(w), None, FAKE, 8, 2.0, FAKE, FAKE, big, None) == QLORA_ERR_INVALID_ARG
+    assert f(FAKE, 16, ctypes.byref(w), FAKE, FAKE, 8, 2.0, FAKE + 2, FAKE, big, None) == QLORA_ERR_INVALID_ARG
+    assert f(FAKE, 16, ctypes.byref(w), FAKE, FAKE, 8, 2.0, FAKE, FAKE, 64, None) == QLORA_ERR_INVALID_ARG
+    assert f(FAKE, 16, ctypes.byref(_w(256, 256, blocksize=32)), FAKE, FAKE, 8, 2.0, FAKE, FAKE, big, None) == QLORA_ERR_UNSUPPORTED
+    b = L.qlora_linear_bwd
+    assert b(FAKE, FAKE, 16, ctypes.byref(w), FAKE, FAKE, 8, 2.0, FAKE, None, FAKE, FAKE, big, None) == QLORA_ERR_INVALID_ARG
+    assert b(FAKE, FAKE, 16, ctypes.byref(w), FAKE, FAKE, 8, 2.0, FAKE + 2, FAKE, FAKE, FAKE, big, None) == QLORA_ERR_INVALID_ARG
+    assert b(FAKE, FAKE, 16, ctypes.byref(_w(256, 100)), FAKE, FAKE, 8, 2.0, FAKE, FAKE, FAKE, FAKE, big, None) == QLORA_ERR_UNSUPPORTED
+    # M == 0 forward: valid, nothing to do
+    assert f(None, 0, ctypes.byref(w), FAKE, FAKE, 8, 2.0, None, FAKE, big, None) == 0
+
+
+def test_linear_workspace_queries(Q):
+    from bit_nf4_quantized_08_b200._lib import lib
+    L = lib()
+    w = _w(4096, 4096)
+    fwd = L.qlora_linear_workspace(2048, ctypes.byref(w), 64, 0)
+    bwd = L.qlora_linear_workspace(2048, ctypes.byref(w), 64, 1)
+    # the expanded block constants alone: (K/64) x N fp32
+    assert fwd >= 64 * 4096 * 4 and bwd >= fwd
+    assert L.qlora_linear_workspace(2048, ctypes.byref(_w(4096, 100)), 64, 0) == 0
+    assert L.qlora_linear_workspace(2048, ctypes.byref(w), 12, 0) == 0
+
+
+def test_missing_library_fails_loudly(Q, tmp_path, monkeypatch):
+    from bit_nf4_quantized_08_b200 import _lib
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "nope.so"))
+    monkeypatch.setattr(_lib, "_lib", None)
+    with pytest.raises(RuntimeError, match="no CPU fallback"):
+        _lib.lib()
+
+
+def test_product_does_not_import_oracle():
+    pkg = os.path.join(ROOT, "bit_nf4_quantized_08_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h")):
+                txt = open(os.path.join(dirpath, fn)).read()
+                assert "import oracle" not in txt and "from oracle" not in txt, fn
+                assert "qlora_oracle" not in txt, fn

@@ -1,0 +1,138 @@
+"""GPU parity of the fused NF4-dequant + LoRA linear forward and backward
+against the fp64 CPU oracle, on seeded inputs that span several tiles and a
+ragged tail, plus the invariants of the pages (B = 0 is a no-op, no dW)."""
+import numpy as np
+import pytest
+import torch
+
+from bit_nf4_quantized_08_b200 import workloads as wl
+from conftest import assert_close_tol
+
+pytestmark = pytest.mark.gpu
+
+
+def _setup(Q, O, M, N, K, r, seed=0, dq=True, b_std=0.01):
+    W = wl.weight(N, K, seed=seed, dtype=torch.bfloat16)
+    inp = wl.linear_inputs(M, N, K, r, seed=seed, b_std=b_std)
+    q = Q.qlora_nf4_quantize(W.cuda(), double_quant=dq)
+    ref_q = O.nf4_quantize(wl.bits(W).reshape(-1), double_quant=dq)
+    Wd_ref = O.nf4_dequantize(N * K, ref_q, double_quant=dq).reshape(N, K)
+    return q, inp, Wd_ref
+
+
+def _fwd_both(Q, O, q, inp, Wd_ref, s, r):
+    X = inp["X"]
+    A, B = inp["A"], inp["B"]
+    Y = Q.qlora_linear_fwd(X.cuda(), q, None if r == 0 else A.cuda(), None if r == 0 else B.cuda(), s)
+    assert Q.qlora_get_last_error() == 0
+    K = X.shape[1]
+    N = Wd_ref.shape[0]
+    Ab = wl.bits(A) if r else np.zeros((0, K), np.uint16)
+    Bb = wl.bits(B) if r else np.zeros((N, 0), np.uint16)
+    ref = O.linear_fwd(wl.bits(X), Wd_ref, Ab, Bb, s)
+    return Y.float().cpu().numpy(), ref
+
+
+FWD_CASES = [
+    # (M, N, K, r): several tiles + ragged tails; small-M path for M <= 64
+    (300, 640, 512, 16),
+    (129, 264, 256, 8),
+    (65, 512, 64, 64),
+    (257, 256, 1024, 0),
+    (64, 640, 512, 16),
+    (17, 384, 256, 8),
+    (3, 1000, 512, 64),
+    (1, 256, 128, 8),
+    (33, 136, 192, 32),
+]
+
+
+@pytest.mark.parametrize("M,N,K,r", FWD_CASES)
+def test_fwd_parity(Q, O, cuda, M, N, K, r):
+    q, inp, Wd_ref = _setup(Q, O, M, N, K, r, seed=1)
+    s = 16.0 / max(r, 1)
+    got, ref = _fwd_both(Q, O, q, inp, Wd_ref, s, r)
+    assert_close_tol(got, ref, f"Y M={M} N={N} K={K} r={r}")
+
+
+@pytest.mark.parametrize("M,N,K,r", [(300, 640, 512, 16), (129, 264, 256, 8), (65, 512, 128, 64),
+                                     (200, 256, 320, 0), (7, 264, 192, 8), (130, 520, 256, 24)])
+def test_bwd_parity(Q, O, cuda, M, N, K, r):
+    q, inp, Wd_ref = _setup(Q, O, M, N, K, r, seed=2, b_std=0.05)
+    s = 2.0
+    X, dY, A, B = inp["X"], inp["dY"], inp["A"], inp["B"]
+    dX, dA, dB = Q.qlora_linear_bwd(dY.cuda(), X.cuda(), q, None if r == 0 else A.cuda(),
+                                    None if r == 0 else B.cuda(), s)
+    assert Q.qlora_get_last_error() == 0
+    Ab = wl.bits(A) if r else np.zeros((0, K), np.uint16)
+    Bb = wl.bits(B) if r else np.zeros((N, 0), np.uint16)
+    rdX, rdA, rdB = O.linear_bwd(wl.bits(dY), wl.bits(X), Wd_ref, Ab, Bb, s)
+    assert_close_tol(dX.float().cpu().numpy(), rdX, "dX")
+    if r:
+        assert_close_tol(dA.cpu().numpy(), rdA, "dA")
+        assert_close_tol(dB.cpu().numpy(), rdB, "dB")
+
+
+@pytest.mark.parametrize("M", [5, 300])
+def test_zero_B_is_noop(Q, O, cuda, M):
+    """Reproduction blog invariant: B = 0 at step 0 gives the frozen base
+    output; bitwise equal to the call with the adapter scaled by 0."""
+    N, K, r = 512, 256, 16
+    q, inp, _ = _setup(Q, O, M, N, K, r, seed=3)
+    X, A = inp["X"].cuda(), inp["A"].cuda()
+    B0 = torch.zeros(N, r, dtype=torch.bfloat16, device="cuda")
+    y0 = Q.qlora_linear_fwd(X, q, A, B0, 2.0)
+    y_s0 = Q.qlora_linear_fwd(X, q, A, inp["B"].cuda(), 0.0)
+    y_none = Q.qlora_linear_fwd(X, q, None, None, 2.0)
+    assert torch.equal(y0.view(torch.int16), y_none.view(torch.int16))
+    assert torch.equal(y_s0.view(torch.int16), y_none.view(torch.int16))
+
+
+def test_fwd_bwd_deterministic(Q, O, cuda):
+    M, N, K, r = 300, 640, 512, 16
+    q, inp, _ = _setup(Q, O, M, N, K, r, seed=4)
+    X, dY, A, B = (inp[k].cuda() for k in ("X", "dY", "A", "B"))
+    y1 = Q.qlora_linear_fwd(X, q, A, B, 1.5)
+    y2 = Q.qlora_linear_fwd(X, q, A, B, 1.5)
+    g1 = Q.qlora_linear_bwd(dY, X, q, A, B, 1.5)
+    g2 = Q.qlora_linear_bwd(dY, X, q, A, B, 1.5)
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+    for a, b in zip(g1, g2):
+        assert torch.equal(a.view(torch.int32 if a.dtype == torch.float32 else torch.int16),
+                           b.view(torch.int32 if b.dtype == torch.float32 else torch.int16))
+
+
+def test_empty_tokens(Q, O, cuda):
+    N, K, r = 256, 128, 8
+    q, inp, _ = _setup(Q, O, 1, N, K, r, seed=5)
+    X = torch.empty(0, K, dtype=torch.bfloat16, device="cuda")
+    dY = torch.empty(0, N, dtype=torch.bfloat16, device="cuda")
+    A, B = inp["A"].cuda(), inp["B"].cuda()
+    Y = Q.qlora_linear_fwd(X, q, A, B, 2.0)
+    assert Y.shape == (0, N)
+    dA = torch.full((r, K), 7.0, device="cuda")
+    dB = torch.full((N, r), 7.0, device="cuda")
+    dX, dA, dB = Q.qlora_linear_bwd(dY, X, q, A, B, 2.0, dA=dA, dB=dB)
+    torch.cuda.synchronize()
+    assert float(dA.abs().max()) == 0.0 and float(dB.abs().max()) == 0.0
+
+
+def test_timeout_is_reported_and_recovers(Q, O, cuda):
+    """Failure detection without a GPU fault: the producer skips its loads,
+    the consumers' bounded waits run out, the status word reports TIMEOUT,
+    and the next normal call on the same context is correct."""
+    M, N, K, r = 256, 256, 128, 8
+    q, inp, Wd_ref = _setup(Q, O, M, N, K, r, seed=6)
+    X, A, B = inp["X"].cuda(), inp["A"].cuda(), inp["B"].cuda()
+    Q.qlora_get_last_error()
+    Q.qlora_set_wait_timeout_ns(20_000_000)
+    Q.qlora_debug_inject(1)
+    try:
+        Q.qlora_linear_fwd(X, q, A, B, 2.0)
+        st = Q.qlora_get_last_error()
+    finally:
+        Q.qlora_debug_inject(0)
+        Q.qlora_set_wait_timeout_ns(0)
+    assert st == Q.QLORA_ERR_TIMEOUT
+    got, ref = _fwd_both(Q, O, q, inp, Wd_ref, 2.0, r)
+    assert_close_tol(got, ref, "Y after recovery")
