@@ -1,0 +1,542 @@
+#!/usr/bin/env python3
+"""Benchmark of the QLoRA NF4 frozen-linear hot path on B200.
+
+One step = one pass of the whole hot path over one batch of the
+LLaMA-7B-shaped decoder block (q/k/v/o 4096x4096, gate/up 11008x4096, down
+4096x11008; M = 4 x 512 tokens; LoRA r = 64, alpha = 16 on all seven):
+  1. blockwise NF4 quantization + double quantization of the 7 bf16 weights
+  2. forward Y = X W'^T + s (X A^T) B^T of the 7 linears
+  3. backward dX, dA, dB of the 7 linears (no dW)
+value = algorithmic fwd+bwd FLOPs of the step / device time of the step.
+
+Timing: W warm-up steps, then K steps each bracketed by CUDA events on the
+launching stream, L2 flushed (256 MiB write) between steps, barrier + device
+synchronize around the timed region, max over ranks.  Under torchrun every
+rank runs an independent replica (the layer does not shard: weak scaling).
+
+Also reported: the roofline of the dominant kernel (live CUDA-event times of
+its launches), an end-to-end figure through pinned host buffers, the CPU
+oracle on a bounded sample, sampled SM clocks, and extra measurements outside
+the step (small-M forward sweep on a 22016x8192 weight, standalone quantize
+and dequantize of 2^30 elements).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fused NF4-dequant+LoRA linear fwd/bwd TFLOP/s and weight GB/s vs B200 roofline"
+WORKLOAD = "llama7b-decoder-block: 7 NF4+DQ linears (q,k,v,o 4096x4096; gate,up 11008x4096; down 4096x11008), M=2048, r=64, alpha=16; quantize+fwd+bwd"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+WEIGHT_BYTES_PER_ELEM = 0.5 + 1 / 64 + 4 / (64 * 256)  # NF4 codes + q8 + c1 (DQ)
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-extras", action="store_true", help="skip the small-M sweep and 2^30 quantize/dequant")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--profile-case", choices=["fwd", "dx", "quantize", "dequantize", "smallm"],
+                    help="run one small case three times, untimed (for ncu captures)")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+
+def fwd_flops(M, N, K, r):
+    return 2 * M * N * K + 2 * M * r * (K + N)
+
+
+def bwd_flops(M, N, K, r):
+    return 2 * M * N * K + 4 * M * r * (K + N)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def source_hash():
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "bit_nf4_quantized_08_b200", "csrc")
+    for fn in sorted(os.listdir(d)):
+        with open(os.path.join(d, fn), "rb") as f:
+            h.update(fn.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic(kind):
+    """Per-launch DRAM bytes of a kernel from a committed ncu capture, or None
+    when absent or taken on different kernel sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kind)
+    if not e or e.get("source_hash") != source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------
+# the workload
+# ---------------------------------------------------------------------------
+
+class Block:
+    """The seven linears of one decoder block with every buffer preallocated."""
+
+    def __init__(self, torch, Q, wl, device, seed=0):
+        c = wl.CONFIGS["llama7b"]
+        self.M, self.r, self.s = c["M"], c["r"], c["alpha"] / c["r"]
+        self.layers = []
+        ws_need = 0
+        for li, (name, N, K) in enumerate(c["linears"]):
+            base = 10 * li
+            W = wl.weight(N, K, seed=seed, dtype=torch.bfloat16, device=device, index_base=base)
+            inp = wl.linear_inputs(self.M, N, K, self.r, seed=seed, device=device, index_base=base)
+            w = Q.NF4Weight.empty(N, K, True, device)
+            L = dict(name=name, N=N, K=K, W=W, w=w, X=inp["X"], dY=inp["dY"], A=inp["A"], B=inp["B"],
+                     Y=torch.empty(self.M, N, dtype=torch.bfloat16, device=device),
+                     dX=torch.empty(self.M, K, dtype=torch.bfloat16, device=device),
+                     dA=torch.empty(self.r, K, dtype=torch.float32, device=device),
+                     dB=torch.empty(N, self.r, dtype=torch.float32, device=device))
+            self.layers.append(L)
+        for L in self.layers:
+            ws_need = max(ws_need, Q.qlora_nf4_quantize_workspace(L["N"], L["K"], True),
+                          Q.qlora_linear_workspace(self.M, L["w"], self.r, False),
+                          Q.qlora_linear_workspace(self.M, L["w"], self.r, True))
+        self.ws = torch.empty(ws_need, dtype=torch.uint8, device=device)
+        self.Q = Q
+        self.flops = sum(fwd_flops(self.M, L["N"], L["K"], self.r) + bwd_flops(self.M, L["N"], L["K"], self.r)
+                         for L in self.layers)
+        self.fwd_gemm_flops = sum(2 * self.M * L["N"] * L["K"] + 2 * self.M * self.r * L["N"] for L in self.layers)
+        self.dx_gemm_flops = sum(2 * self.M * L["N"] * L["K"] + 2 * self.M * self.r * L["K"] for L in self.layers)
+        self.quant_bytes = sum(L["N"] * L["K"] * (2 + WEIGHT_BYTES_PER_ELEM) for L in self.layers)
+
+    def step(self):
+        Q, ws = self.Q, self.ws
+        for L in self.layers:
+            Q.qlora_nf4_quantize(L["W"], True, out=L["w"], ws=ws)
+        for L in self.layers:
+            Q.qlora_linear_fwd(L["X"], L["w"], L["A"], L["B"], self.s, Y=L["Y"], ws=ws)
+        for L in reversed(self.layers):
+            Q.qlora_linear_bwd(L["dY"], L["X"], L["w"], L["A"], L["B"], self.s, dX=L["dX"], dA=L["dA"],
+                               dB=L["dB"], ws=ws)
+
+
+def time_steps(torch, fn, steps, flush, dist_barrier):
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    dist_barrier()
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush()
+        starts[i].record()
+        fn()
+        ends[i].record()
+    torch.cuda.synchronize()
+    dist_barrier()
+    return [s.elapsed_time(e) for s, e in zip(starts, ends)]
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle sample (reported baseline and the reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(torch, wl, seed=0):
+    """Bounded oracle sample of one step: for each of the 7 linears of the
+    block (M=2048, r=64): full quantize + DQ + dequantize of W, forward and dX
+    on 16 of the 2048 token rows, dA and dB in full.
+    Returns (flops, seconds, description, threads)."""
+    import numpy as np
+    from oracle import oracle as O
+    O.build()
+    c = wl.CONFIGS["llama7b"]
+    M, r, s = c["M"], c["r"], c["alpha"] / c["r"]
+    rows = np.linspace(0, M - 1, 16).astype(np.int64)
+    R = rows.size
+    flops, dt = 0, 0.0
+    for li, (_, N, K) in enumerate(c["linears"]):
+        base = 10 * li
+        W = wl.weight(N, K, seed=seed, dtype=torch.bfloat16, index_base=base)
+        inp = wl.linear_inputs(M, N, K, r, seed=seed, index_base=base)
+        Xb, dYb, Ab, Bb = (wl.bits(inp[k]) for k in ("X", "dY", "A", "B"))
+        Wbits = wl.bits(W).reshape(-1)
+        t0 = time.perf_counter()
+        q = O.nf4_quantize(Wbits, double_quant=True)
+        Wd = O.nf4_dequantize(N * K, q).reshape(N, K)
+        O.linear_fwd(Xb, Wd, Ab, Bb, s, rows=rows)
+        O.linear_bwd(dYb, Xb, Wd, Ab, Bb, s, rows=rows)
+        dt += time.perf_counter() - t0
+        flops += (R * (2 * N * K + 2 * r * (K + N))      # forward rows
+                  + R * (2 * N * K + 2 * r * K)          # dX rows
+                  + 2 * M * r * (K + N)                  # U and G over all rows
+                  + 2 * M * r * K + 2 * M * N * r)       # dA, dB
+    desc = ("all 7 linears of the block (M=2048, r=64): full NF4+DQ quantize and dequantize "
+            "of W, Y and dX on 16 of 2048 token rows, dA and dB in full")
+    return flops, dt, desc, O.num_threads()
+
+
+# ---------------------------------------------------------------------------
+# extras: small-M sweep, 2^30 quantize / dequantize
+# ---------------------------------------------------------------------------
+
+def extras(torch, Q, wl, device, flush, peaks):
+    out = {}
+    c = wl.CONFIGS["sweep"]
+    (_, N, K), = c["linears"]
+    r, s = c["r"], c["alpha"] / c["r"]
+    W = wl.weight(N, K, seed=0, dtype=torch.bfloat16, device=device)
+    w = Q.qlora_nf4_quantize(W)
+    del W
+    sweep = {}
+    reps = 20
+    for M in c["Ms"]:
+        inp = wl.linear_inputs(M, N, K, r, seed=0, device=device)
+        X, A, B = inp["X"], inp["A"], inp["B"]
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=device)
+        ws = torch.empty(Q.qlora_linear_workspace(M, w, r, False), dtype=torch.uint8, device=device)
+        for _ in range(3):
+            Q.qlora_linear_fwd(X, w, A, B, s, Y=Y, ws=ws)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            Q.qlora_linear_fwd(X, w, A, B, s, Y=Y, ws=ws)
+        times = []
+        for _ in range(reps):
+            flush()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            g.replay()
+            e1.record()
+            e1.synchronize()
+            times.append(e0.elapsed_time(e1))
+        ms = statistics.median(times)
+        wbytes = N * K * WEIGHT_BYTES_PER_ELEM
+        total = wbytes + M * K * 2 + r * K * 2 + N * r * 2 + M * N * 2
+        sweep[str(M)] = {"us": round(ms * 1e3, 2), "weight_GBps": round(wbytes / ms / 1e6, 1),
+                         "total_GBps": round(total / ms / 1e6, 1),
+                         "frac_hbm": round(total / ms / 1e6 / peaks["hbm_gbs"], 3)}
+        del g
+    out["small_m_fwd_22016x8192_r64_cuda_graph"] = sweep
+
+    n = c["big_numel"]
+    Wbig = wl.weight(n // 8192, 8192, seed=0, dtype=torch.bfloat16, device=device)
+    qb = Q.NF4Weight.empty(n // 8192, 8192, True, device)
+    wsq = torch.empty(Q.qlora_nf4_quantize_workspace(n // 8192, 8192, True), dtype=torch.uint8, device=device)
+    deq = torch.empty(n // 8192, 8192, dtype=torch.bfloat16, device=device)
+    algo = n * (2 + WEIGHT_BYTES_PER_ELEM)
+    for name, fn in (("quantize_2^30_bf16", lambda: Q.qlora_nf4_quantize(Wbig, True, out=qb, ws=wsq)),
+                     ("dequantize_2^30_bf16", lambda: Q.qlora_nf4_dequantize(qb, out=deq))):
+        for _ in range(3):
+            fn()
+        times = []
+        for _ in range(5):
+            flush()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            e1.synchronize()
+            times.append(e0.elapsed_time(e1))
+        ms = statistics.median(times)
+        out[name] = {"us": round(ms * 1e3, 1), "GBps": round(algo / ms / 1e6, 1),
+                     "frac_hbm": round(algo / ms / 1e6 / peaks["hbm_gbs"], 3),
+                     "algorithmic_bytes": int(algo)}
+    del Wbig, qb, deq, wsq
+    return out
+
+
+# ---------------------------------------------------------------------------
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+    if args.profile_case:
+        return run_profile_case(args.profile_case)
+
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    from bit_nf4_quantized_08_b200 import build as qbuild
+    if rank == 0 or world == 1:
+        qbuild.build()
+    barrier()
+    import bit_nf4_quantized_08_b200 as Q
+    from bit_nf4_quantized_08_b200 import workloads as wl
+
+    peaks, peak_src = load_peaks()
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+
+    def flush():
+        flush_buf.fill_(1)
+
+    blk = Block(torch, Q, wl, device, seed=rank)
+    for _ in range(max(3, args.warmup)):
+        blk.step()
+    torch.cuda.synchronize()
+    assert Q.qlora_get_last_error() == 0
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    launches0 = Q.qlora_kernel_launches()
+    Q.qlora_profile_enable(True)
+    times = time_steps(torch, blk.step, args.steps, flush, barrier)
+    launches = Q.qlora_kernel_launches() - launches0
+    clk = clocks.stop()
+    prof = {k: Q.qlora_profile_read(k) for k in ("quantize", "fwd_gemm", "dx_gemm")}
+    Q.qlora_profile_enable(False)
+    status = Q.qlora_get_last_error()
+    assert status == 0, f"device status {status}"
+
+    total_ms = sum(times)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = blk.flops * world / (ms_per_step * 1e-3) / 1e12
+
+    # dominant kernel: the tracked kind with the largest device time
+    dom = max(("fwd_gemm", "dx_gemm"), key=lambda k: prof[k][0])
+    dom_ms, dom_n = prof[dom]
+    dom_flops = (blk.fwd_gemm_flops if dom == "fwd_gemm" else blk.dx_gemm_flops) * args.steps
+    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops"]
+    traffic = load_traffic(dom)
+    roofline = {"bound": "tensor", "kernel": f"k_gemm ({dom.replace('_', ' ')}, NF4 dequant in producer)",
+                "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4), "traffic": traffic,
+                "peak_source": f"{peak_src} bf16 dense (burst)",
+                "launches": dom_n, "avg_launch_us": round(dom_ms / max(dom_n, 1) * 1e3, 2)}
+    breakdown = {}
+    qms, qn = prof["quantize"]
+    if qn:
+        breakdown["quantize_GBps"] = round(blk.quant_bytes * args.steps / (qms * 1e-3) / 1e9, 1)
+        breakdown["quantize_frac_hbm"] = round(breakdown["quantize_GBps"] / peaks["hbm_gbs"], 3)
+    for k in ("fwd_gemm", "dx_gemm"):
+        ms_k, n_k = prof[k]
+        fl = (blk.fwd_gemm_flops if k == "fwd_gemm" else blk.dx_gemm_flops) * args.steps
+        if n_k:
+            breakdown[k + "_TFLOPs"] = round(fl / (ms_k * 1e-3) / 1e12, 1)
+            breakdown[k + "_share_of_step"] = round(ms_k / total_ms, 3)
+
+    # end to end through the public API with pinned host buffers
+    host_in = []
+    for L in blk.layers:
+        for key in ("W", "X", "dY"):
+            h = torch.empty(L[key].shape, dtype=L[key].dtype, pin_memory=True)
+            h.copy_(L[key])
+            host_in.append((h, L[key]))
+    host_out = []
+    for L in blk.layers:
+        for key in ("dA", "dB"):
+            host_out.append((torch.empty(L[key].shape, dtype=L[key].dtype, pin_memory=True), L[key]))
+    h2d = sum(h.numel() * h.element_size() for h, _ in host_in)
+    d2h = sum(h.numel() * h.element_size() for h, _ in host_out)
+
+    def e2e_step():
+        for h, d in host_in:
+            d.copy_(h, non_blocking=True)
+        blk.step()
+        for h, d in host_out:
+            h.copy_(d, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 5))
+    e2e_times = time_steps(torch, e2e_step, e2e_steps, flush, barrier)
+    e2e_ms = statistics.mean(e2e_times)
+    t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    e2e_ms = float(t.item())
+    e2e = {"value": round(blk.flops * world / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+           "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+           "ms_per_step": round(e2e_ms, 3)}
+
+    extra = None
+    if not args.no_extras:
+        del blk
+        torch.cuda.empty_cache()
+        extra = extras(torch, Q, wl, device, flush, peaks)
+
+    cpu = None
+    if rank == 0 and not args.no_cpu:
+        flops, dt, desc, threads = oracle_sample(torch, wl)
+        cpu = {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": desc, "seconds": round(dt, 2)}
+
+    if world > 1:
+        dist.barrier()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": round(ms_per_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "global_batch": 2048 * world, "seq_len": 512,
+                       "flops_per_step": blk_flops_cache(wl), "l2": "flushed between steps (256 MiB write)",
+                       "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
+            "roofline": roofline, "breakdown": breakdown, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": int(launches), "clocks": clk, "extra": extra,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def blk_flops_cache(wl):
+    c = wl.CONFIGS["llama7b"]
+    return sum(fwd_flops(c["M"], N, K, c["r"]) + bwd_flops(c["M"], N, K, c["r"]) for _, N, K in c["linears"])
+
+
+def run_profile_case(case):
+    """A small case of one kernel, launched three times: the gate-shaped
+    linear (11008x4096, M=2048, r=64) for the GEMMs, 2^26 elements for the
+    quantizer, the 22016x8192 weight at M=16 for the small-M forward."""
+    import torch
+    from bit_nf4_quantized_08_b200 import build as qbuild
+    qbuild.build()
+    import bit_nf4_quantized_08_b200 as Q
+    from bit_nf4_quantized_08_b200 import workloads as wl
+    dev = torch.device("cuda", 0)
+    if case in ("quantize", "dequantize"):
+        W = wl.weight(1 << 13, 1 << 13, seed=0, dtype=torch.bfloat16, device=dev)
+        w = Q.qlora_nf4_quantize(W)
+        for _ in range(3):
+            if case == "quantize":
+                Q.qlora_nf4_quantize(W, True, out=w)
+            else:
+                Q.qlora_nf4_dequantize(w)
+    else:
+        N, K, M = (22016, 8192, 16) if case == "smallm" else (11008, 4096, 2048)
+        r, s = 64, 0.25
+        W = wl.weight(N, K, seed=0, dtype=torch.bfloat16, device=dev)
+        w = Q.qlora_nf4_quantize(W)
+        inp = wl.linear_inputs(M, N, K, r, seed=0, device=dev)
+        for _ in range(3):
+            if case == "dx":
+                Q.qlora_linear_bwd(inp["dY"], inp["X"], w, inp["A"], inp["B"], s)
+            else:
+                Q.qlora_linear_fwd(inp["X"], w, inp["A"], inp["B"], s)
+    torch.cuda.synchronize()
+    assert Q.qlora_get_last_error() == 0
+    print("profile case", case, "ok")
+    return 0
+
+
+def run_reference(args, world, rank):
+    """Reference arm: the CPU oracle, as it stands, timed on a bounded sample
+    of the same workload per step (rank 0 only)."""
+    if rank != 0:
+        return 0
+    import torch
+    from bit_nf4_quantized_08_b200 import workloads as wl
+    for _ in range(max(0, min(args.warmup, 1))):
+        oracle_sample(torch, wl)
+    tot_flops, tot_s = 0, 0.0
+    desc, threads = "", 1
+    for _ in range(args.steps):
+        f, dt, desc, threads = oracle_sample(torch, wl)
+        tot_flops += f
+        tot_s += dt
+    value = tot_flops / tot_s / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_s / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": WORKLOAD + " (bounded CPU sample per step)"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main() or 0)

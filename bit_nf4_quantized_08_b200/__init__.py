@@ -20,4 +20,7 @@ from .api import (  # noqa: F401
     qlora_nf4_quantize_workspace,
     qlora_nf4_table,
     qlora_set_wait_timeout_ns,
+    qlora_kernel_launches,
+    qlora_profile_enable,
+    qlora_profile_read,
 )

@@ -37,7 +37,11 @@ EXPORTS = (
     "qlora_nf4_encode",
     "qlora_set_wait_timeout_ns",
     "qlora_debug_inject",
+    "qlora_kernel_launches",
+    "qlora_profile_enable",
+    "qlora_profile_read",
 )
+KERNEL_KINDS = {"quantize": 0, "dequantize": 1, "fwd_gemm": 2, "dx_gemm": 3, "smallm_gemm": 4}
 
 
 class QloraError(RuntimeError):
@@ -99,6 +103,12 @@ def lib() -> ctypes.CDLL:
     L.qlora_set_wait_timeout_ns.restype = None
     L.qlora_debug_inject.argtypes = [i32]
     L.qlora_debug_inject.restype = None
+    L.qlora_kernel_launches.argtypes = []
+    L.qlora_kernel_launches.restype = ctypes.c_uint64
+    L.qlora_profile_enable.argtypes = [i32]
+    L.qlora_profile_enable.restype = None
+    L.qlora_profile_read.argtypes = [i32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]
+    L.qlora_profile_read.restype = i32
     env = os.environ.get("QLORA_WAIT_TIMEOUT_NS")
     if env:
         L.qlora_set_wait_timeout_ns(int(env))

@@ -184,3 +184,20 @@ def qlora_set_wait_timeout_ns(ns: int) -> None:
 
 def qlora_debug_inject(mode: int) -> None:
     lib().qlora_debug_inject(int(mode))
+
+
+def qlora_kernel_launches() -> int:
+    return int(lib().qlora_kernel_launches())
+
+
+def qlora_profile_enable(on: bool) -> None:
+    lib().qlora_profile_enable(int(bool(on)))
+
+
+def qlora_profile_read(kind: str) -> tuple[float, int]:
+    """(summed device ms, launches) recorded for one tracked kernel kind."""
+    ms = ctypes.c_double()
+    n = ctypes.c_int64()
+    check(lib().qlora_profile_read(_lib.KERNEL_KINDS[kind], ctypes.byref(ms), ctypes.byref(n)),
+          "qlora_profile_read")
+    return ms.value, n.value

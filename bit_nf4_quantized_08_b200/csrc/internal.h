@@ -9,6 +9,16 @@
 
 namespace qlora {
 
+// Launch accounting and optional event timing of tracked kernels.
+void note_launch();
+struct ProfileScope {
+    int kind;
+    cudaStream_t s;
+    int slot;
+    ProfileScope(int kind, cudaStream_t s);
+    ~ProfileScope();
+};
+
 // Bound of every in-kernel wait of the next launches (ns).
 uint64_t wait_timeout_ns();
 int inject_mode();

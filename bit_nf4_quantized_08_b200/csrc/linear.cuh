@@ -73,14 +73,14 @@ inline bool map_bf16(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t o
 // launch helpers
 // ---------------------------------------------------------------------------
 template <int BN, int A_MN, int B_MN, int DQ, int EPI, int STAGES>
-inline cudaError_t launch_gemm(const GemmParams& p, dim3 grid, cudaStream_t s) {
+inline cudaError_t launch_gemm(const GemmParams& p, dim3 grid, cudaStream_t s, int prof_kind = -1) {
     using Sh = GemmShape<BN, A_MN, B_MN, DQ>;
     constexpr int smem = gemm_smem_bytes<BN, A_MN, B_MN, DQ, STAGES>();
     auto kern = k_gemm<BN, A_MN, B_MN, DQ, EPI, STAGES>;
-    static bool configured = false;  // attribute is per function; set once per device use
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    (void)configured;
+    ProfileScope ps(prof_kind, s);
+    note_launch();
     kern<<<grid, Sh::THREADS, smem, s>>>(p);
     return cudaGetLastError();
 }
@@ -148,6 +148,7 @@ inline qlora_status skinny(const CUtensorMap& tA, const CUtensorMap& tB, int row
         e = launch_gemm<256, A_MN, B_MN, DQ_NONE, EPI_F32, 4>(p, grid, s);
     if (e != cudaSuccess) return QLORA_ERR_CUDA;
     const int64_t total = (int64_t)rows * r;
+    note_launch();
     k_splitk_reduce<<<ceil_div(total, 256), 256, 0, s>>>(part, splits, (int64_t)rows * r, rows, r, r,
                                                          scale, red_mode, out, out_ld);
     return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
@@ -256,7 +257,7 @@ inline qlora_status linear_fwd_impl(const void* X, const LinearArgs& a, const vo
         p.cols = (int)a.N;
         p.out_ld = a.N;
         dim3 grid(ceil_div(a.N, 256), ceil_div(a.M, 128), 1);
-        if (launch_gemm<256, 0, 0, DQ_B_K, EPI_BF16, 3>(p, grid, s) != cudaSuccess)
+        if (launch_gemm<256, 0, 0, DQ_B_K, EPI_BF16, 3>(p, grid, s, QLORA_KERNEL_FWD_GEMM) != cudaSuccess)
             return QLORA_ERR_CUDA;
         return QLORA_OK;
     }
@@ -283,20 +284,21 @@ inline qlora_status linear_fwd_impl(const void* X, const LinearArgs& a, const vo
     if (splits == 1) {
         p.out_ld = a.N;
         if (bn == 32)
-            e = launch_gemm<32, 0, 0, DQ_A_K, EPI_BF16_T, 6>(p, grid, s);
+            e = launch_gemm<32, 0, 0, DQ_A_K, EPI_BF16_T, 6>(p, grid, s, QLORA_KERNEL_SMALLM_GEMM);
         else
-            e = launch_gemm<64, 0, 0, DQ_A_K, EPI_BF16_T, 6>(p, grid, s);
+            e = launch_gemm<64, 0, 0, DQ_A_K, EPI_BF16_T, 6>(p, grid, s, QLORA_KERNEL_SMALLM_GEMM);
         return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
     }
     p.out = L.part;
     p.out_ld = a.N;
     p.out_split_stride = a.M * a.N;
     if (bn == 32)
-        e = launch_gemm<32, 0, 0, DQ_A_K, EPI_F32_T, 6>(p, grid, s);
+        e = launch_gemm<32, 0, 0, DQ_A_K, EPI_F32_T, 6>(p, grid, s, QLORA_KERNEL_SMALLM_GEMM);
     else
-        e = launch_gemm<64, 0, 0, DQ_A_K, EPI_F32_T, 6>(p, grid, s);
+        e = launch_gemm<64, 0, 0, DQ_A_K, EPI_F32_T, 6>(p, grid, s, QLORA_KERNEL_SMALLM_GEMM);
     if (e != cudaSuccess) return QLORA_ERR_CUDA;
     const int64_t total = a.M * a.N;
+    note_launch();
     k_splitk_reduce<<<ceil_div(total, 256), 256, 0, s>>>(L.part, splits, a.M * a.N, (int)a.M,
                                                          (int)a.N, a.N, 1.0f, RED_BF16, Y, a.N);
     return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
@@ -310,7 +312,9 @@ inline qlora_status linear_bwd_impl(const void* dY, const void* X, const LinearA
     LinearWs L = carve_linear_ws(ws, a.M, a.N, a.K, a.r, 1);
     if (a.M == 0) {
         if (a.r > 0) {
+            note_launch();
             k_fill_zero_f32<<<64, 256, 0, s>>>(dA, (int64_t)a.r * a.K);
+            note_launch();
             k_fill_zero_f32<<<64, 256, 0, s>>>(dB, a.N * a.r);
             if (cudaGetLastError() != cudaSuccess) return QLORA_ERR_CUDA;
         }
@@ -356,7 +360,7 @@ inline qlora_status linear_bwd_impl(const void* dY, const void* X, const LinearA
         p.timeout_ns = wait_timeout_ns();
         p.inject = inject_mode();
         dim3 grid(ceil_div(a.K, 256), ceil_div(a.M, 128), 1);
-        if (launch_gemm<256, 0, 1, DQ_B_MN, EPI_BF16, 3>(p, grid, s) != cudaSuccess)
+        if (launch_gemm<256, 0, 1, DQ_B_MN, EPI_BF16, 3>(p, grid, s, QLORA_KERNEL_DX_GEMM) != cudaSuccess)
             return QLORA_ERR_CUDA;
     }
     if (a.r > 0) {

@@ -5,6 +5,8 @@
 #include <string.h>
 
 #include <atomic>
+#include <mutex>
+#include <vector>
 
 #include "../../include/qlora_nf4.h"
 #include "common.cuh"
@@ -19,6 +21,41 @@ namespace qlora {
 
 static std::atomic<uint64_t> g_timeout_ns{10ull * 1000 * 1000 * 1000};
 static std::atomic<int> g_inject{0};
+
+static std::atomic<uint64_t> g_launches{0};
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+// Event timing of tracked kernels (enabled by qlora_profile_enable).
+struct ProfRecord {
+    int kind;
+    cudaEvent_t start, stop;
+};
+static std::mutex g_prof_mu;
+static std::atomic<int> g_prof_on{0};
+static std::vector<ProfRecord> g_prof;  // recorded pairs, in launch order
+static std::vector<std::pair<cudaEvent_t, cudaEvent_t>> g_prof_pool;
+static size_t g_prof_used = 0;
+
+ProfileScope::ProfileScope(int k, cudaStream_t st) : kind(k), s(st), slot(-1) {
+    if (k < 0 || !g_prof_on.load()) return;
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    if (g_prof_used == g_prof_pool.size()) {
+        cudaEvent_t a, b;
+        if (cudaEventCreate(&a) != cudaSuccess) return;
+        if (cudaEventCreate(&b) != cudaSuccess) return;
+        g_prof_pool.push_back({a, b});
+    }
+    auto pr = g_prof_pool[g_prof_used++];
+    slot = (int)g_prof.size();
+    g_prof.push_back({kind, pr.first, pr.second});
+    cudaEventRecord(pr.first, s);
+}
+
+ProfileScope::~ProfileScope() {
+    if (slot < 0) return;
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    cudaEventRecord(g_prof[slot].stop, s);
+}
 
 uint64_t wait_timeout_ns() { return g_timeout_ns.load(); }
 int inject_mode() { return g_inject.load(); }
@@ -188,5 +225,32 @@ void qlora_set_wait_timeout_ns(uint64_t ns) {
 }
 
 void qlora_debug_inject(int32_t mode) { g_inject.store(mode); }
+
+uint64_t qlora_kernel_launches(void) { return g_launches.load(); }
+
+void qlora_profile_enable(int32_t on) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_prof.clear();
+    g_prof_used = 0;
+    g_prof_on.store(on ? 1 : 0);
+}
+
+qlora_status qlora_profile_read(int32_t kind, double* total_ms, int64_t* launches) {
+    if (kind < 0 || kind >= QLORA_KERNEL_KINDS || !total_ms || !launches) return QLORA_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    double t = 0.0;
+    int64_t n = 0;
+    for (const auto& r : g_prof) {
+        if (r.kind != kind) continue;
+        if (cudaEventSynchronize(r.stop) != cudaSuccess) return QLORA_ERR_CUDA;
+        float ms = 0.0f;
+        if (cudaEventElapsedTime(&ms, r.start, r.stop) != cudaSuccess) return QLORA_ERR_CUDA;
+        t += ms;
+        ++n;
+    }
+    *total_ms = t;
+    *launches = n;
+    return QLORA_OK;
+}
 
 }  // extern "C"

@@ -376,6 +376,8 @@ inline cudaError_t launch_quantize_blocks(const void* W, int is_bf16, int64_t n,
                                           float* absmax, double* group_sums, cudaStream_t s) {
     const int64_t ng = (n + 16383) / 16384;
     if (ng == 0) return cudaSuccess;
+    ProfileScope ps(QLORA_KERNEL_QUANTIZE, s);
+    note_launch();
     if (is_bf16)
         k_quantize_blocks<true><<<(unsigned)ng, 256, 0, s>>>(W, n, codes, absmax, group_sums,
                                                               nf4_search_table());
@@ -387,6 +389,7 @@ inline cudaError_t launch_quantize_blocks(const void* W, int is_bf16, int64_t n,
 
 inline cudaError_t launch_dq_offset(const double* group_sums, int64_t ngroups, int64_t nb,
                                     float* offset, cudaStream_t s) {
+    note_launch();
     k_dq_offset<<<1, 1024, 0, s>>>(group_sums, ngroups, nb, offset);
     return cudaGetLastError();
 }
@@ -395,6 +398,7 @@ inline cudaError_t launch_dq_quantize(const float* absmax, int64_t nb, const flo
                                       uint8_t* q8, float* c1, cudaStream_t s) {
     const int64_t ng = (nb + 255) / 256;
     if (ng == 0) return cudaSuccess;
+    note_launch();
     k_dq_quantize<<<(unsigned)((ng + 7) / 8), 256, 0, s>>>(absmax, nb, offset, q8, c1);
     return cudaGetLastError();
 }
@@ -403,6 +407,8 @@ inline cudaError_t launch_dequantize(const qlora_nf4_weight& w, uint16_t* out, c
     const int64_t n = w.rows * w.cols;
     const int64_t nb = (n + 63) / 64;
     if (nb == 0) return cudaSuccess;
+    ProfileScope ps(QLORA_KERNEL_DEQUANTIZE, s);
+    note_launch();
     k_dequantize<<<(unsigned)((nb + 255) / 256), 256, 0, s>>>(
         w.codes, n, w.double_quant, w.absmax, w.absmax_q8, w.absmax_scale, w.absmax_offset, out);
     return cudaGetLastError();
@@ -413,6 +419,7 @@ inline cudaError_t launch_expand_scales(const qlora_nf4_weight& w, float* scales
     const int64_t kbs = w.cols / 64;
     const int64_t total = w.rows * kbs;
     if (total == 0) return cudaSuccess;
+    note_launch();
     k_expand_scales<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(
         w.rows, kbs, w.double_quant, w.absmax, w.absmax_q8, w.absmax_scale, w.absmax_offset,
         scales, ld);
@@ -423,6 +430,7 @@ inline cudaError_t launch_encode(const float* x, int64_t n, uint8_t* codes, cuda
     if (n == 0) return cudaSuccess;
     int64_t blocks = (n + 255) / 256;
     if (blocks > 148 * 16) blocks = 148 * 16;
+    note_launch();
     k_encode<<<(unsigned)blocks, 256, 0, s>>>(x, n, codes, nf4_search_table());
     return cudaGetLastError();
 }

@@ -188,6 +188,30 @@ void qlora_set_wait_timeout_ns(uint64_t ns);
  */
 void qlora_debug_inject(int32_t mode);
 
+/*
+ * Measurement hooks (used by the benchmark).
+ * qlora_kernel_launches: number of kernels this library has launched in this
+ *   process (all devices, all streams).
+ * qlora_profile_enable(1) clears the records and starts recording a CUDA
+ *   event pair around every launch of the tracked kernels below, on the
+ *   stream the kernel is launched on; 0 stops recording.
+ * qlora_profile_read: synchronizes the recorded events and returns, for one
+ *   kind, the summed device time (ms) and the number of launches recorded.
+ *   Returns QLORA_ERR_INVALID_ARG for an unknown kind.
+ */
+typedef enum {
+    QLORA_KERNEL_QUANTIZE = 0,  /* blockwise NF4 quantizer (first kernel of qlora_nf4_quantize) */
+    QLORA_KERNEL_DEQUANTIZE = 1,
+    QLORA_KERNEL_FWD_GEMM = 2,  /* forward dequant-GEMM, M > 64 */
+    QLORA_KERNEL_DX_GEMM = 3,   /* backward dX dequant-GEMM */
+    QLORA_KERNEL_SMALLM_GEMM = 4, /* forward dequant-GEMM, M <= 64 */
+    QLORA_KERNEL_KINDS = 5
+} qlora_kernel_kind;
+
+uint64_t qlora_kernel_launches(void);
+void qlora_profile_enable(int32_t on);
+qlora_status qlora_profile_read(int32_t kind, double *total_ms, int64_t *launches);
+
 #ifdef __cplusplus
 }
 #endif
