@@ -48,12 +48,15 @@ struct GemmParams {
     int inject;
 };
 
-template <int BN, int A_MN, int B_MN, int DQ>
+// MT = number of 128-row MMA sub-tiles on the A side (1 or 2).  With MT = 2
+// one dequantized B tile feeds two accumulators (256 A rows per CTA), which
+// halves the dequant work per MMA flop.
+template <int BN, int A_MN, int B_MN, int DQ, int MT>
 struct GemmShape {
-    static constexpr int BM = 128;
+    static constexpr int BM = 128 * MT;
     static constexpr int A_BYTES = BM * 128;
     static constexpr int B_BYTES = BN * 128;
-    static constexpr int DQ_ROWS = DQ == DQ_B_K ? BN : (DQ == DQ_A_K ? BM : (DQ == DQ_B_MN ? 256 : 0));
+    static constexpr int DQ_ROWS = DQ == DQ_B_K ? BN : (DQ == DQ_A_K ? 128 : (DQ == DQ_B_MN ? 256 : 0));
     static constexpr int NDQ_WARPS = DQ_ROWS / 32;
     static constexpr int CODE_BYTES = DQ == DQ_B_MN ? 64 * 128 : DQ_ROWS * 32;
     static constexpr int SCALE_BYTES = DQ == DQ_NONE ? 0 : (DQ == DQ_B_MN ? 4 * 64 * 4 : DQ_ROWS * 4);
@@ -61,19 +64,32 @@ struct GemmShape {
     static constexpr int STAGE_BYTES = (STAGE_RAW + 1023) / 1024 * 1024;
     static constexpr int NE_WARPS = NDQ_WARPS > 4 ? NDQ_WARPS : 4;
     static constexpr int THREADS = 32 * (2 + NE_WARPS);
-    static constexpr int TMEM_COLS = BN <= 32 ? 32 : (BN <= 64 ? 64 : (BN <= 128 ? 128 : 256));
+    static constexpr int ACC_COLS = BN <= 32 ? 32 : (BN <= 64 ? 64 : (BN <= 128 ? 128 : 256));
+    static constexpr int TMEM_COLS = ACC_COLS * MT;
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
+    static_assert(MT == 1 || MT == 2, "MT");
+    static_assert(DQ != DQ_A_K || MT == 1, "a dequantized A operand is one 128-row tile");
 };
 
-template <int BN, int A_MN, int B_MN, int DQ, int STAGES>
+template <int BN, int A_MN, int B_MN, int DQ, int STAGES, int MT>
 constexpr int gemm_smem_bytes() {
-    return GemmShape<BN, A_MN, B_MN, DQ>::STAGE_BYTES * STAGES + 1024 /*align*/ + 256 /*barriers*/;
+    return GemmShape<BN, A_MN, B_MN, DQ, MT>::STAGE_BYTES * STAGES + 1024 /*align*/ + 256 /*barriers*/;
 }
 
-template <int BN, int A_MN, int B_MN, int DQ, int EPI, int STAGES>
-__global__ void __launch_bounds__(GemmShape<BN, A_MN, B_MN, DQ>::THREADS, 1)
+// Physical offset of a logical byte offset inside a TMA tile written with the
+// 32-byte swizzle (16-byte chunk index bit 0 XOR address bit 7).
+__device__ __forceinline__ uint32_t sw32(uint32_t off) { return off ^ ((off >> 3) & 0x10u); }
+
+__device__ __forceinline__ float ld_shared_f32(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+    return v;
+}
+
+template <int BN, int A_MN, int B_MN, int DQ, int EPI, int STAGES, int MT>
+__global__ void __launch_bounds__(GemmShape<BN, A_MN, B_MN, DQ, MT>::THREADS, 1)
     k_gemm(const __grid_constant__ GemmParams p) {
-    using S = GemmShape<BN, A_MN, B_MN, DQ>;
+    using S = GemmShape<BN, A_MN, B_MN, DQ, MT>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
     const uint32_t base = (raw_base + 1023u) & ~1023u;
@@ -150,17 +166,20 @@ __global__ void __launch_bounds__(GemmShape<BN, A_MN, B_MN, DQ>::THREADS, 1)
                             if (n0 / 64 + c < p.dq_kbs) bytes += 256;
                     }
                 } else {
-                    bytes = S::A_BYTES + S::B_BYTES;
+                    bytes = (DQ == DQ_A_K ? 16384 : S::A_BYTES) + S::B_BYTES;
                 }
                 mbar_arrive_expect_tx(full_tma(s), bytes);
                 const CUtensorMap* mA = lora ? &p.tmA2 : &p.tmA;
                 const CUtensorMap* mB = lora ? &p.tmB2 : &p.tmB;
                 if (lora || DQ != DQ_A_K) {
-                    if (A_MN) {
-                        tma_load_2d(sA, mA, full_tma(s), m0, k * 64);
-                        tma_load_2d(sA + 8192, mA, full_tma(s), m0 + 64, k * 64);
-                    } else {
-                        tma_load_2d(sA, mA, full_tma(s), k * 64, m0);
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) {
+                        if (A_MN) {
+                            tma_load_2d(sA + mt * 16384, mA, full_tma(s), m0 + 128 * mt, k * 64);
+                            tma_load_2d(sA + mt * 16384 + 8192, mA, full_tma(s), m0 + 128 * mt + 64, k * 64);
+                        } else {
+                            tma_load_2d(sA + mt * 16384, mA, full_tma(s), k * 64, m0 + 128 * mt);
+                        }
                     }
                 }
                 if (lora || (DQ != DQ_B_K && DQ != DQ_B_MN)) {
@@ -209,11 +228,15 @@ __global__ void __launch_bounds__(GemmShape<BN, A_MN, B_MN, DQ>::THREADS, 1)
                 const uint32_t sB = sA + S::A_BYTES;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t ad = A_MN ? smem_desc_sw128(sA + kk * 2048, 8192, 1024)
-                                             : smem_desc_sw128(sA + kk * 32, 16, 1024);
                     const uint64_t bd = B_MN ? smem_desc_sw128(sB + kk * 2048, 8192, 1024)
                                              : smem_desc_sw128(sB + kk * 32, 16, 1024);
-                    umma_bf16(tmem, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) {
+                        const uint32_t a_t = sA + mt * 16384;
+                        const uint64_t ad = A_MN ? smem_desc_sw128(a_t + kk * 2048, 8192, 1024)
+                                                 : smem_desc_sw128(a_t + kk * 32, 16, 1024);
+                        umma_bf16(tmem + mt * S::ACC_COLS, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+                    }
                 }
                 umma_commit(empty(s));
             }
@@ -229,21 +252,27 @@ __global__ void __launch_bounds__(GemmShape<BN, A_MN, B_MN, DQ>::THREADS, 1)
             int scale_idx;
             int64_t wrow;
             int kb_off;
+            uint32_t code_off2;
             if (DQ == DQ_B_MN) {
+                // codes tile [64 rows][128 B], TMA 128-byte swizzle
                 const int j = t >> 2, c = t & 3;
-                code_off = j * 128 + c * 32;
+                code_off = sw128(j * 128 + c * 32);
+                code_off2 = sw128(j * 128 + c * 32 + 16);
                 scale_idx = c * 64 + j;
                 out_off = c * 8192 + j * 128;
                 wrow = j;  // + 64*k
                 kb_off = c;
             } else {
-                code_off = t * 32;
+                // codes tile [rows][32 B], TMA 32-byte swizzle
+                code_off = sw32(t * 32);
+                code_off2 = sw32(t * 32 + 16);
                 scale_idx = t;
                 out_off = t * 128;
                 wrow = (DQ == DQ_B_K ? n0 : m0) + t;
                 kb_off = 0;
             }
             const uint32_t tile_off = (DQ == DQ_A_K) ? 0u : (uint32_t)S::A_BYTES;
+            (void)gbase;
             for (int i = 0; i < n_main; ++i) {
                 const int s = i % STAGES, u = i / STAGES;
                 if (!mbar_wait(full_tma(s), u & 1, wc)) { *abort_flag = 1; break; }
@@ -257,10 +286,9 @@ __global__ void __launch_bounds__(GemmShape<BN, A_MN, B_MN, DQ>::THREADS, 1)
                 else
                     valid = true;  // rows beyond the weight only feed masked outputs
                 if (valid) {
-                    const float a = reinterpret_cast<const float*>(gbase + s * S::STAGE_BYTES + S::A_BYTES +
-                                                                   S::B_BYTES + S::CODE_BYTES)[scale_idx];
+                    const float a = ld_shared_f32(sC + S::CODE_BYTES + 4u * scale_idx);
                     const uint4 c0 = ld_shared_v4(sC + code_off);
-                    const uint4 c1 = ld_shared_v4(sC + code_off + 16);
+                    const uint4 c1 = ld_shared_v4(sC + code_off2);
                     const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
                     const Nf4BlockTable tb = nf4_block_table(a);
 #pragma unroll
@@ -286,14 +314,16 @@ __global__ void __launch_bounds__(GemmShape<BN, A_MN, B_MN, DQ>::THREADS, 1)
         constexpr int COLS_PER_GROUP = BN / GROUPS;
         if (mbar_wait(acc_full, 0, wc) && !*abort_flag) {
             tc_fence_after();
-            const int row = quarter * 32 + lane;  // D row inside the tile (TMEM lane)
-            const int grow = m0 + row;
-            const bool row_ok = grow < p.rows;
-            for (int cc = 0; cc < COLS_PER_GROUP; cc += 32) {
+            const int row = quarter * 32 + lane;  // D row inside a 128-row sub-tile (TMEM lane)
+            for (int it = 0; it < MT * (COLS_PER_GROUP / 32); ++it) {
+                const int mt = it / (COLS_PER_GROUP / 32);
+                const int cc = (it % (COLS_PER_GROUP / 32)) * 32;
+                const int grow = m0 + 128 * mt + row;
+                const bool row_ok = grow < p.rows;
                 const int col0 = group * COLS_PER_GROUP + cc;
                 uint32_t v[32];
                 __syncwarp();
-                tmem_ld_32x32b_x32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)col0, v);
+                tmem_ld_32x32b_x32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(mt * S::ACC_COLS + col0), v);
                 tmem_ld_wait();
                 const int gcol0 = n0 + col0;
                 if (n_steps == 0) {

@@ -47,7 +47,7 @@ inline PFN_encodeTiled_t encode_fn() {
 // 2-D tiled map over a row-major [outer][inner] tensor.
 inline bool make_map(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int esize,
                      uint64_t inner, uint64_t outer, uint64_t row_bytes, uint32_t box_inner,
-                     uint32_t box_outer, bool swizzle128) {
+                     uint32_t box_outer, CUtensorMapSwizzle swz) {
     PFN_encodeTiled_t fn = encode_fn();
     if (!fn) return false;
     (void)esize;
@@ -56,8 +56,7 @@ inline bool make_map(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, in
     cuuint32_t box[2] = {box_inner, box_outer};
     cuuint32_t es[2] = {1, 1};
     CUresult r = fn(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, es,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -66,17 +65,18 @@ inline bool make_map(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, in
 inline bool map_bf16(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer,
                      uint32_t box_outer) {
     return make_map(m, ptr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, inner, outer, inner * 2, 64,
-                    box_outer, true);
+                    box_outer, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 // ---------------------------------------------------------------------------
 // launch helpers
 // ---------------------------------------------------------------------------
-template <int BN, int A_MN, int B_MN, int DQ, int EPI, int STAGES>
+template <int BN, int A_MN, int B_MN, int DQ, int EPI, int STAGES, int MT = 1>
 inline cudaError_t launch_gemm(const GemmParams& p, dim3 grid, cudaStream_t s, int prof_kind = -1) {
-    using Sh = GemmShape<BN, A_MN, B_MN, DQ>;
-    constexpr int smem = gemm_smem_bytes<BN, A_MN, B_MN, DQ, STAGES>();
-    auto kern = k_gemm<BN, A_MN, B_MN, DQ, EPI, STAGES>;
+    using Sh = GemmShape<BN, A_MN, B_MN, DQ, MT>;
+    constexpr int smem = gemm_smem_bytes<BN, A_MN, B_MN, DQ, STAGES, MT>();
+    static_assert(smem <= 232448, "shared memory per CTA");
+    auto kern = k_gemm<BN, A_MN, B_MN, DQ, EPI, STAGES, MT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     ProfileScope ps(prof_kind, s);
@@ -202,10 +202,14 @@ inline size_t linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int r, int
     return carve_linear_ws(nullptr, M, N, K, r, bwd).bytes;
 }
 
+// Packed codes viewed [rows][K/2 bytes].  32-byte boxes use the 32-byte
+// swizzle and 128-byte boxes the 128-byte swizzle, so that the dequant
+// threads' 16-byte reads of a tile are free of bank conflicts.
 inline bool map_codes(CUtensorMap* m, const qlora_nf4_weight& w, uint32_t box_bytes,
                       uint32_t box_rows) {
     return make_map(m, w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)w.cols / 2,
-                    (uint64_t)w.rows, (uint64_t)w.cols / 2, box_bytes, box_rows, false);
+                    (uint64_t)w.rows, (uint64_t)w.cols / 2, box_bytes, box_rows,
+                    box_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 // sU = bf16(scale * X A^T) into L.sU
@@ -256,8 +260,8 @@ inline qlora_status linear_fwd_impl(const void* X, const LinearArgs& a, const vo
         p.rows = (int)a.M;
         p.cols = (int)a.N;
         p.out_ld = a.N;
-        dim3 grid(ceil_div(a.N, 256), ceil_div(a.M, 128), 1);
-        if (launch_gemm<256, 0, 0, DQ_B_K, EPI_BF16, 3>(p, grid, s, QLORA_KERNEL_FWD_GEMM) != cudaSuccess)
+        dim3 grid(ceil_div(a.N, 256), ceil_div(a.M, 256), 1);
+        if (launch_gemm<256, 0, 0, DQ_B_K, EPI_BF16, 3, 2>(p, grid, s, QLORA_KERNEL_FWD_GEMM) != cudaSuccess)
             return QLORA_ERR_CUDA;
         return QLORA_OK;
     }
@@ -359,8 +363,8 @@ inline qlora_status linear_bwd_impl(const void* dY, const void* X, const LinearA
         p.out_ld = a.K;
         p.timeout_ns = wait_timeout_ns();
         p.inject = inject_mode();
-        dim3 grid(ceil_div(a.K, 256), ceil_div(a.M, 128), 1);
-        if (launch_gemm<256, 0, 1, DQ_B_MN, EPI_BF16, 3>(p, grid, s, QLORA_KERNEL_DX_GEMM) != cudaSuccess)
+        dim3 grid(ceil_div(a.K, 256), ceil_div(a.M, 256), 1);
+        if (launch_gemm<256, 0, 1, DQ_B_MN, EPI_BF16, 3, 2>(p, grid, s, QLORA_KERNEL_DX_GEMM) != cudaSuccess)
             return QLORA_ERR_CUDA;
     }
     if (a.r > 0) {
