@@ -45,7 +45,7 @@ cudaError_t launch_encode(const float* x, int64_t n, uint8_t* codes, cudaStream_
 // Block constants a' of a weight, written transposed as scales[kb * ld + n]
 // (kb = block column, n = row) for the GEMM producers.
 cudaError_t launch_expand_scales(const qlora_nf4_weight& w, float* scales, int64_t ld,
-                                 cudaStream_t s);
+                                 cudaStream_t s, int* flags, int nflags);
 
 // ---- GEMMs (gemm.cu) ----
 struct LinearArgs {

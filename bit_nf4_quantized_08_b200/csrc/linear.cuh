@@ -13,9 +13,12 @@
 #pragma once
 
 #include <algorithm>
+#include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "gemm.cuh"
+#include "gemm_pair.cuh"
 #include "internal.h"
 #include "quantize.cuh"
 
@@ -136,7 +139,7 @@ inline qlora_status skinny(const CUtensorMap& tA, const CUtensorMap& tB, int row
     p.out_ld = r;
     p.out_split_stride = (int64_t)rows * r;
     p.timeout_ns = wait_timeout_ns();
-    p.inject = inject_mode();
+    p.inject = inject_mode() == 1 ? 1 : 0;
     dim3 grid(1, tiles, splits);
     const int bn = lora_bn(r);
     cudaError_t e;
@@ -166,6 +169,15 @@ inline size_t small_m_part_bytes(int64_t M, int64_t N, int64_t K) {
     return splits > 1 ? (size_t)splits * M * N * 4 : 0;
 }
 
+inline int sm_count() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+}
+
+// Largest stream-K grid; also sizes the partial-tile workspace.
+constexpr int kMaxStreamK = 256;
+
 // Workspace layout shared by the query and the launches.
 struct LinearWs {
     float* scales;
@@ -173,6 +185,8 @@ struct LinearWs {
     uint16_t* sU;
     uint16_t* sG;
     float* part;
+    float* sk_part;  // stream-K partial tiles [kMaxStreamK][256*256]
+    int* sk_flags;   // [kMaxStreamK]
     size_t bytes;
 };
 
@@ -194,6 +208,9 @@ inline LinearWs carve_linear_ws(void* ws, int64_t M, int64_t N, int64_t K, int r
     }
     if (!bwd && M <= kSmallM) part = std::max(part, small_m_part_bytes(M, N, K));
     L.part = part ? static_cast<float*>(c.take(part)) : nullptr;
+    const bool big = bwd || M > kSmallM;
+    L.sk_part = big ? static_cast<float*>(c.take((size_t)kMaxStreamK * 256 * 256 * 4)) : nullptr;
+    L.sk_flags = big ? static_cast<int*>(c.take((size_t)kMaxStreamK * 4)) : nullptr;
     L.bytes = c.used;
     return L;
 }
@@ -205,11 +222,60 @@ inline size_t linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int r, int
 // Packed codes viewed [rows][K/2 bytes].  32-byte boxes use the 32-byte
 // swizzle and 128-byte boxes the 128-byte swizzle, so that the dequant
 // threads' 16-byte reads of a tile are free of bank conflicts.
+// Tile schedule of the dequant GEMMs: stream-K over a persistent grid of
+// one CTA per SM when there are at least two k-steps per CTA, else one CTA
+// per tile.  Debug mode 2 forces stream-K on 7 CTAs (tests of the merge).
+template <int DQ, int STAGES>
+inline cudaError_t launch_gemm_pair(const GemmParams& p, dim3 grid, cudaStream_t s, int prof_kind) {
+    constexpr int smem = pair_smem_bytes<DQ, STAGES>();
+    static_assert(smem <= 232448, "shared memory per CTA");
+    auto kern = k_gemm_pair<DQ, STAGES>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    ProfileScope ps(prof_kind, s);
+    note_launch();
+    kern<<<grid, PairShape<DQ>::THREADS, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
+// Which large-M GEMM runs: CTA pairs (default), or the single-CTA kernel on
+// the grid or stream-K schedule.  QLORA_SCHEDULE=pair|grid|streamk selects
+// one; test mode 2 forces stream-K, test mode 3 the single-CTA grid.
+enum { SCHED_PAIR = 0, SCHED_GRID = 1, SCHED_STREAMK = 2 };
+inline int large_m_schedule() {
+    if (inject_mode() == 2) return SCHED_STREAMK;
+    if (inject_mode() == 3) return SCHED_GRID;
+    static int v = [] {
+        const char* e = getenv("QLORA_SCHEDULE");
+        if (!e) return (int)SCHED_PAIR;
+        if (!strcmp(e, "grid")) return (int)SCHED_GRID;
+        if (!strcmp(e, "streamk")) return (int)SCHED_STREAMK;
+        return (int)SCHED_PAIR;
+    }();
+    return v;
+}
+
+inline dim3 schedule_gemm(GemmParams& p, int tiles_n, int tiles_m, const LinearWs& L) {
+    const int KS = p.ks_main + p.ks_lora;
+    const int64_t tiles = (int64_t)tiles_n * tiles_m;
+    int G = std::min(sm_count(), kMaxStreamK);
+    if (inject_mode() == 2) G = 7;
+    p.tiles_n = tiles_n;
+    p.tiles_total = (int)tiles;
+    p.sk_part = L.sk_part;
+    p.sk_flags = L.sk_flags;
+    const bool sk = large_m_schedule() == SCHED_STREAMK;
+    p.streamk = sk ? 1 : 0;
+    if (!sk) return dim3(tiles_n, tiles_m, 1);
+    return dim3((unsigned)std::min<int64_t>(G, tiles * KS), 1, 1);
+}
+
 inline bool map_codes(CUtensorMap* m, const qlora_nf4_weight& w, uint32_t box_bytes,
                       uint32_t box_rows) {
     return make_map(m, w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)w.cols / 2,
                     (uint64_t)w.rows, (uint64_t)w.cols / 2, box_bytes, box_rows,
-                    box_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_128B);
+                    box_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                    : (box_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B));
 }
 
 // sU = bf16(scale * X A^T) into L.sU
@@ -228,7 +294,9 @@ inline qlora_status linear_fwd_impl(const void* X, const LinearArgs& a, const vo
     (void)ws_bytes;
     const qlora_nf4_weight& w = *a.w;
     LinearWs L = carve_linear_ws(ws, a.M, a.N, a.K, a.r, 0);
-    if (launch_expand_scales(w, L.scales, L.scales_ld, s) != cudaSuccess) return QLORA_ERR_CUDA;
+    if (launch_expand_scales(w, L.scales, L.scales_ld, s, L.sk_flags, L.sk_flags ? kMaxStreamK : 0) !=
+        cudaSuccess)
+        return QLORA_ERR_CUDA;
     if (a.r > 0) {
         qlora_status st = compute_sU(X, a, A, L, s);
         if (st != QLORA_OK) return st;
@@ -242,7 +310,7 @@ inline qlora_status linear_fwd_impl(const void* X, const LinearArgs& a, const vo
     p.ks_main = (int)(a.K / 64);
     p.ks_lora = a.r > 0 ? ceil_div(a.r, 64) : 0;
     p.timeout_ns = wait_timeout_ns();
-    p.inject = inject_mode();
+    p.inject = inject_mode() == 1 ? 1 : 0;
     p.out = Y;
     if (a.M > kSmallM) {
         // Y = [X | sU] [W' | B]^T : 128 x 256 tiles, W' dequantized into the B slot.
@@ -260,7 +328,16 @@ inline qlora_status linear_fwd_impl(const void* X, const LinearArgs& a, const vo
         p.rows = (int)a.M;
         p.cols = (int)a.N;
         p.out_ld = a.N;
-        dim3 grid(ceil_div(a.N, 256), ceil_div(a.M, 256), 1);
+        if (!map_bf16(&p.tmOut, Y, a.N, a.M, 128)) return QLORA_ERR_CUDA;
+        if (large_m_schedule() == SCHED_PAIR) {
+            if (!map_codes(&p.tmCodes, w, 32, 128)) return QLORA_ERR_CUDA;
+            if (a.r > 0 && !map_bf16(&p.tmB2, B, a.r, a.N, 128)) return QLORA_ERR_CUDA;
+            dim3 grid(2 * ceil_div(a.N, 256), ceil_div(a.M, 512), 1);
+            if (launch_gemm_pair<DQ_B_K, 4>(p, grid, s, QLORA_KERNEL_FWD_GEMM) != cudaSuccess)
+                return QLORA_ERR_CUDA;
+            return QLORA_OK;
+        }
+        dim3 grid = schedule_gemm(p, ceil_div(a.N, 256), ceil_div(a.M, 256), L);
         if (launch_gemm<256, 0, 0, DQ_B_K, EPI_BF16, 3, 2>(p, grid, s, QLORA_KERNEL_FWD_GEMM) != cudaSuccess)
             return QLORA_ERR_CUDA;
         return QLORA_OK;
@@ -324,7 +401,8 @@ inline qlora_status linear_bwd_impl(const void* dY, const void* X, const LinearA
         }
         return QLORA_OK;
     }
-    if (dX && launch_expand_scales(w, L.scales, L.scales_ld, s) != cudaSuccess) return QLORA_ERR_CUDA;
+    if (dX && launch_expand_scales(w, L.scales, L.scales_ld, s, L.sk_flags, kMaxStreamK) != cudaSuccess)
+        return QLORA_ERR_CUDA;
     CUtensorMap tdY;
     if (!map_bf16(&tdY, dY, a.N, a.M, 128)) return QLORA_ERR_CUDA;
     if (a.r > 0) {
@@ -361,11 +439,19 @@ inline qlora_status linear_bwd_impl(const void* dY, const void* X, const LinearA
         p.cols = (int)a.K;
         p.out = dX;
         p.out_ld = a.K;
+        if (!map_bf16(&p.tmOut, dX, a.K, a.M, 128)) return QLORA_ERR_CUDA;
         p.timeout_ns = wait_timeout_ns();
-        p.inject = inject_mode();
-        dim3 grid(ceil_div(a.K, 256), ceil_div(a.M, 256), 1);
-        if (launch_gemm<256, 0, 1, DQ_B_MN, EPI_BF16, 3, 2>(p, grid, s, QLORA_KERNEL_DX_GEMM) != cudaSuccess)
-            return QLORA_ERR_CUDA;
+        p.inject = inject_mode() == 1 ? 1 : 0;
+        if (large_m_schedule() == SCHED_PAIR) {
+            if (!map_codes(&p.tmCodes, w, 64, 64)) return QLORA_ERR_CUDA;
+            dim3 grid(2 * ceil_div(a.K, 256), ceil_div(a.M, 512), 1);
+            if (launch_gemm_pair<DQ_B_MN, 4>(p, grid, s, QLORA_KERNEL_DX_GEMM) != cudaSuccess)
+                return QLORA_ERR_CUDA;
+        } else {
+            dim3 grid = schedule_gemm(p, ceil_div(a.K, 256), ceil_div(a.M, 256), L);
+            if (launch_gemm<256, 0, 1, DQ_B_MN, EPI_BF16, 3, 2>(p, grid, s, QLORA_KERNEL_DX_GEMM) != cudaSuccess)
+                return QLORA_ERR_CUDA;
+        }
     }
     if (a.r > 0) {
         // dA^T [K][r] = X^T sG : Aop = X viewed [k][m] (MN-major), Bop = sG viewed [j][m] (MN-major)

@@ -307,11 +307,13 @@ __global__ void __launch_bounds__(256) k_dequantize(const uint8_t* __restrict__ 
 }
 
 // Block constants a' transposed for the GEMM producers: scales[kb*ld + n].
+// Also zeroes `nflags` ints (the flags of the stream-K GEMM that follows).
 __global__ void k_expand_scales(int64_t rows, int64_t kbs, int dq, const float* __restrict__ absmax,
                                 const uint8_t* __restrict__ q8, const float* __restrict__ c1,
                                 const float* __restrict__ offset_ptr, float* __restrict__ scales,
-                                int64_t ld) {
+                                int64_t ld, int* __restrict__ flags, int nflags) {
     const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx < nflags) flags[idx] = 0;
     if (idx >= rows * kbs) return;
     const int64_t kb = idx / rows, n = idx - kb * rows;
     const int64_t b = n * kbs + kb;
@@ -415,14 +417,14 @@ inline cudaError_t launch_dequantize(const qlora_nf4_weight& w, uint16_t* out, c
 }
 
 inline cudaError_t launch_expand_scales(const qlora_nf4_weight& w, float* scales, int64_t ld,
-                                        cudaStream_t s) {
+                                        cudaStream_t s, int* flags = nullptr, int nflags = 0) {
     const int64_t kbs = w.cols / 64;
-    const int64_t total = w.rows * kbs;
+    const int64_t total = w.rows * kbs > nflags ? w.rows * kbs : nflags;
     if (total == 0) return cudaSuccess;
     note_launch();
     k_expand_scales<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(
         w.rows, kbs, w.double_quant, w.absmax, w.absmax_q8, w.absmax_scale, w.absmax_offset,
-        scales, ld);
+        scales, ld, flags, nflags);
     return cudaGetLastError();
 }
 

@@ -181,10 +181,14 @@ qlora_status qlora_nf4_encode(const float *x, int64_t n, uint8_t *codes, qlora_s
 void qlora_set_wait_timeout_ns(uint64_t ns);
 
 /*
- * Fault injection for the failure-detection tests.  Mode 1 makes the next
- * launches of the tensor-core GEMM skip their producer's loads, so that the
- * consumers' bounded waits run out and QLORA_ERR_TIMEOUT is recorded; mode 0
- * turns it off.  No GPU fault is raised: the kernels return normally.
+ * Test modes.  Mode 1 (fault injection for the failure-detection tests) makes
+ * the next launches of the tensor-core GEMM skip their producer's loads, so
+ * that the consumers' bounded waits run out and QLORA_ERR_TIMEOUT is
+ * recorded; no GPU fault is raised, the kernels return normally.  Mode 2
+ * runs the forward and dX GEMMs (M > 64) on the single-CTA kernel with the
+ * stream-K schedule over 7 CTAs whatever the shape (coverage of the
+ * split-tile merge); mode 3 on the single-CTA kernel with one CTA per tile.
+ * Mode 0: normal (CTA-pair kernel).
  */
 void qlora_debug_inject(int32_t mode);
 

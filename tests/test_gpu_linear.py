@@ -136,3 +136,33 @@ def test_timeout_is_reported_and_recovers(Q, O, cuda):
     assert st == Q.QLORA_ERR_TIMEOUT
     got, ref = _fwd_both(Q, O, q, inp, Wd_ref, 2.0, r)
     assert_close_tol(got, ref, "Y after recovery")
+
+
+@pytest.mark.parametrize("mode", [2, 3], ids=["streamk7", "single_cta_grid"])
+@pytest.mark.parametrize("M,N,K,r", [(300, 640, 512, 16), (513, 264, 256, 8), (257, 512, 192, 64)])
+def test_alternate_schedule_parity(Q, O, cuda, mode, M, N, K, r):
+    """Forward and dX on the single-CTA kernel, on the stream-K schedule
+    (forced onto 7 CTAs, so that tiles are split across CTAs and merged) and
+    on the grid schedule, match the oracle and are bitwise reproducible."""
+    q, inp, Wd_ref = _setup(Q, O, M, N, K, r, seed=7, b_std=0.05)
+    X, dY, A, B = (inp[k].cuda() for k in ("X", "dY", "A", "B"))
+    s = 2.0
+    Q.qlora_debug_inject(mode)
+    try:
+        Y1 = Q.qlora_linear_fwd(X, q, A, B, s)
+        Y2 = Q.qlora_linear_fwd(X, q, A, B, s)
+        dX1, dA1, dB1 = Q.qlora_linear_bwd(dY, X, q, A, B, s)
+        dX2, _, _ = Q.qlora_linear_bwd(dY, X, q, A, B, s)
+        assert Q.qlora_get_last_error() == 0
+    finally:
+        Q.qlora_debug_inject(0)
+    assert torch.equal(Y1.view(torch.int16), Y2.view(torch.int16))
+    assert torch.equal(dX1.view(torch.int16), dX2.view(torch.int16))
+    ref = O.linear_fwd(wl.bits(inp["X"]), Wd_ref, wl.bits(inp["A"]), wl.bits(inp["B"]), s)
+    assert_close_tol(Y1.float().cpu().numpy(), ref, "Y alternate schedule")
+    rdX, rdA, rdB = O.linear_bwd(wl.bits(inp["dY"]), wl.bits(inp["X"]), Wd_ref, wl.bits(inp["A"]),
+                                 wl.bits(inp["B"]), s)
+    assert_close_tol(dX1.float().cpu().numpy(), rdX, "dX alternate schedule")
+    # the default (CTA-pair) kernel gives the same values up to fp32 summation order
+    Y3 = Q.qlora_linear_fwd(X, q, A, B, s)
+    assert_close_tol(Y3.float().cpu().numpy(), ref, "Y default")
