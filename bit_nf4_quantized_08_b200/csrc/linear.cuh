@@ -19,6 +19,7 @@
 
 #include "gemm.cuh"
 #include "gemm_pair.cuh"
+#include "skinny.cuh"
 #include "internal.h"
 #include "quantize.cuh"
 
@@ -114,47 +115,64 @@ struct WsCarve {
     }
 };
 
-// Skinny GEMM out[rows][r] = scale * sum_k Aop[row][k] Bop[j][k], through
-// split-K fp32 partials and a fixed-order reduction.
+// Skinny GEMM out[rows][r] = scale * sum_k Aop[row][k] Bop[j][k]: 128-row
+// tiles, the reduction split across a cluster of up to 8 CTAs and summed over
+// distributed shared memory (one launch, deterministic).
+template <int BN, int A_MN, int B_MN, int STAGES>
+inline cudaError_t launch_skinny(const SkinnyParams& p, int tiles, int cs, cudaStream_t s) {
+    constexpr int smem = skinny_smem_bytes<BN, STAGES>();
+    static_assert(smem <= 232448, "shared memory per CTA");
+    auto kern = k_skinny<BN, A_MN, B_MN, STAGES>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3((unsigned)(tiles * cs), 1, 1);
+    cfg.blockDim = dim3(SkinnyShape<BN>::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = (unsigned)cs;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    note_launch();
+    return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
 template <int A_MN, int B_MN>
 inline qlora_status skinny(const CUtensorMap& tA, const CUtensorMap& tB, int rows, int r,
                            int ksteps, float* part, float scale, int red_mode, void* out,
                            int64_t out_ld, cudaStream_t s) {
-    GemmParams p;
+    (void)part;
+    SkinnyParams p;
     memset(&p, 0, sizeof(p));
     p.tmA = tA;
     p.tmB = tB;
-    p.tmA2 = tA;
-    p.tmB2 = tB;
-    p.tmCodes = tA;
-    const int tiles = ceil_div(rows, 128);
-    int splits, per;
-    choose_splits(tiles, ksteps, &splits, &per);
-    p.ks_main = ksteps;
-    p.ks_lora = 0;
-    p.ks_per_split = per;
     p.rows = rows;
-    p.cols = r;
-    p.out = part;
-    p.out_ld = r;
-    p.out_split_stride = (int64_t)rows * r;
+    p.r = r;
+    p.ksteps = ksteps;
+    p.scale = scale;
+    p.out_mode = red_mode == RED_BF16 ? SK_OUT_BF16 : (red_mode == RED_F32 ? SK_OUT_F32 : SK_OUT_F32_T);
+    p.out = out;
+    p.out_ld = out_ld;
     p.timeout_ns = wait_timeout_ns();
     p.inject = inject_mode() == 1 ? 1 : 0;
-    dim3 grid(1, tiles, splits);
+    const int tiles = ceil_div(rows, 128);
+    int cs = 8;
+    while (cs > 1 && ((int64_t)tiles * cs > 2 * 148 || ksteps < 2 * cs)) cs >>= 1;
+    p.per = ceil_div(ksteps, cs);
     const int bn = lora_bn(r);
     cudaError_t e;
     if (bn == 64)
-        e = launch_gemm<64, A_MN, B_MN, DQ_NONE, EPI_F32, 6>(p, grid, s);
+        e = launch_skinny<64, A_MN, B_MN, 4>(p, tiles, cs, s);
     else if (bn == 128)
-        e = launch_gemm<128, A_MN, B_MN, DQ_NONE, EPI_F32, 5>(p, grid, s);
+        e = launch_skinny<128, A_MN, B_MN, 4>(p, tiles, cs, s);
     else
-        e = launch_gemm<256, A_MN, B_MN, DQ_NONE, EPI_F32, 4>(p, grid, s);
-    if (e != cudaSuccess) return QLORA_ERR_CUDA;
-    const int64_t total = (int64_t)rows * r;
-    note_launch();
-    k_splitk_reduce<<<ceil_div(total, 256), 256, 0, s>>>(part, splits, (int64_t)rows * r, rows, r, r,
-                                                         scale, red_mode, out, out_ld);
-    return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+        e = launch_skinny<256, A_MN, B_MN, 3>(p, tiles, cs, s);
+    return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
 inline size_t skinny_part_bytes(int rows, int r, int ksteps) {
