@@ -41,12 +41,33 @@ namespace qlora {
 // each holds at most one threshold T_key; base_key counts the thresholds at
 // or below the bucket's lower edge.  code(x) = base_key + (x >= T_key), where
 // threshold j is the smallest fp32 strictly above the exact midpoint of codes
-// j and j+1 (so an exact tie stays with the lower code).
-__device__ __forceinline__ int nf4_search(float x, const float2* tab) {
+// j and j+1 (so an exact tie stays with the lower code).  The tables have 64
+// entries and the key is masked to 6 bits, so any input (NaN included) reads
+// inside them.
+struct SearchSmem {
+    float thr[64];
+    int base[64];
+};
+
+__device__ __forceinline__ void load_search_tables(SearchSmem& st, const Nf4SearchTable& tab) {
+    for (int i = threadIdx.x; i < 64; i += blockDim.x) {
+        st.thr[i] = i < 33 ? tab.thr[i] : 3.0f;
+        st.base[i] = i < 33 ? tab.base[i] : 15;
+    }
+}
+
+__device__ __forceinline__ uint32_t nf4_search(float x, const SearchSmem& st) {
     const float t = fmaf(x, 16.0f, 12582928.0f);  // 1.5 * 2^23 + 16: RN to an integer
-    const uint32_t key = min(__float_as_uint(t) - 0x4B400000u, 32u);
-    const float2 e = tab[key];
-    return __float_as_int(e.y) + (x >= e.x ? 1 : 0);
+    const uint32_t key = __float_as_uint(t) & 63u;  // low bits of 0x4B400000 + key
+    return (uint32_t)st.base[key] + (x >= st.thr[key] ? 1u : 0u);
+}
+
+// Pack 8 codes (element order) into one word: byte i = (c[2i] << 4) | c[2i+1].
+__device__ __forceinline__ uint32_t pack8(const uint32_t (&c)[8]) {
+    uint32_t acc = c[0];
+#pragma unroll
+    for (int i = 1; i < 8; ++i) acc = acc * 16u + c[i];  // c0 ends in the top nibble
+    return __byte_perm(acc, 0u, 0x0123);                 // reverse bytes: (c0,c1) -> byte 0
 }
 
 // ---------------------------------------------------------------------------
@@ -56,15 +77,14 @@ __device__ __forceinline__ int nf4_search(float x, const float2* tab) {
 // pairwise-tree sum of block maxima for the double-quantization offset.
 // ---------------------------------------------------------------------------
 template <bool BF16>
-__global__ void __launch_bounds__(256) k_quantize_blocks(const void* __restrict__ W, int64_t n,
-                                                         uint8_t* __restrict__ codes,
-                                                         float* __restrict__ absmax,
-                                                         double* __restrict__ group_sums,
-                                                         Nf4SearchTable tab) {
-    __shared__ float2 s_tab[33];
+__global__ void __launch_bounds__(256, BF16 ? 4 : 2) k_quantize_blocks(const void* __restrict__ W, int64_t n,
+                                                            uint8_t* __restrict__ codes,
+                                                            float* __restrict__ absmax,
+                                                            double* __restrict__ group_sums,
+                                                            Nf4SearchTable tab) {
+    __shared__ SearchSmem st;
     __shared__ double s_wsum[8];
-    if (threadIdx.x < 33)
-        s_tab[threadIdx.x] = make_float2(tab.thr[threadIdx.x], __int_as_float(tab.base[threadIdx.x]));
+    load_search_tables(st, tab);
     __syncthreads();
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -83,7 +103,7 @@ __global__ void __launch_bounds__(256) k_quantize_blocks(const void* __restrict_
                                           static_cast<const float*>(W) + e0[it]);
 #pragma unroll
             for (int v = 0; v < WORDS / 4; ++v) {
-                uint4 q = __ldg(src + v);
+                uint4 q = __ldcs(src + v);
                 raw[it][4 * v + 0] = q.x;
                 raw[it][4 * v + 1] = q.y;
                 raw[it][4 * v + 2] = q.z;
@@ -93,12 +113,15 @@ __global__ void __launch_bounds__(256) k_quantize_blocks(const void* __restrict_
 #pragma unroll
             for (int v = 0; v < WORDS; ++v) raw[it][v] = 0u;
             if (e0[it] < n) {
-                for (int i = 0; i < 16 && e0[it] + i < n; ++i) {
-                    if (BF16) {
-                        uint32_t h = static_cast<const uint16_t*>(W)[e0[it] + i];
-                        raw[it][i >> 1] |= h << ((i & 1) * 16);
-                    } else {
-                        raw[it][i] = __float_as_uint(static_cast<const float*>(W)[e0[it] + i]);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    if (e0[it] + i < n) {
+                        if (BF16) {
+                            uint32_t h = static_cast<const uint16_t*>(W)[e0[it] + i];
+                            raw[it][i >> 1] |= h << ((i & 1) * 16);
+                        } else {
+                            raw[it][i] = __float_as_uint(static_cast<const float*>(W)[e0[it] + i]);
+                        }
                     }
                 }
             }
@@ -108,18 +131,19 @@ __global__ void __launch_bounds__(256) k_quantize_blocks(const void* __restrict_
     double rowsum[4];
 #pragma unroll
     for (int it = 0; it < 4; ++it) {
-        float v[16];
+        // block absmax (exact: a max of magnitudes)
+        float a;
+        if (BF16) {
+            uint32_t m = 0;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            if (BF16)
-                v[i] = __uint_as_float((i & 1) ? (raw[it][i >> 1] & 0xFFFF0000u)
-                                               : (raw[it][i >> 1] << 16));
-            else
-                v[i] = __uint_as_float(raw[it][i]);
+            for (int i = 0; i < 8; ++i) m = __vmaxu2(m, raw[it][i] & 0x7FFF7FFFu);
+            m = max(m & 0xFFFFu, m >> 16);
+            a = __uint_as_float(m << 16);
+        } else {
+            a = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(__uint_as_float(raw[it][i])));
         }
-        float a = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(v[i]));
         a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
         a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
 
@@ -127,23 +151,35 @@ __global__ void __launch_bounds__(256) k_quantize_blocks(const void* __restrict_
         const bool bvalid = b < nb;
         if (bvalid && (lane & 3) == 0 && absmax) absmax[b] = a;
 
-        float p = 1.0f;
-        if (a < 1.17549435e-38f) p = 18446744073709551616.0f;  // 2^64, exact prescale
-        const float rcp = (a == 0.0f) ? 0.0f : __frcp_rn(__fmul_rn(a, p));
         uint32_t c[16];
+        if (a >= 1.17549435e-38f) {
+            const float rcp = __frcp_rn(a);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            float x = __fmul_rn(__fmul_rn(v[i], p), rcp);
-            c[i] = (uint32_t)nf4_search(x, s_tab);
-        }
-        uint32_t w0 = 0, w1 = 0;
+            for (int i = 0; i < 16; ++i) {
+                const uint32_t bits = BF16 ? ((i & 1) ? (raw[it][i >> 1] & 0xFFFF0000u) : (raw[it][i >> 1] << 16))
+                                           : raw[it][i];
+                c[i] = nf4_search(__fmul_rn(__uint_as_float(bits), rcp), st);
+            }
+        } else {
+            // zero or subnormal block: exact power-of-two prescale 2^64
+            const float p = 18446744073709551616.0f;
+            const float rcp = (a == 0.0f) ? 0.0f : __frcp_rn(__fmul_rn(a, p));
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            w0 |= ((c[2 * j] << 4) | c[2 * j + 1]) << (8 * j);
-            w1 |= ((c[8 + 2 * j] << 4) | c[8 + 2 * j + 1]) << (8 * j);
+            for (int i = 0; i < 16; ++i) {
+                const uint32_t bits = BF16 ? ((i & 1) ? (raw[it][i >> 1] & 0xFFFF0000u) : (raw[it][i >> 1] << 16))
+                                           : raw[it][i];
+                c[i] = nf4_search(__fmul_rn(__fmul_rn(__uint_as_float(bits), p), rcp), st);
+            }
         }
+        uint32_t lo[8], hi[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            lo[i] = c[i];
+            hi[i] = c[8 + i];
+        }
+        const uint32_t w0 = pack8(lo), w1 = pack8(hi);
         if (e0[it] + 16 <= n) {
-            *reinterpret_cast<uint2*>(codes + (e0[it] >> 1)) = make_uint2(w0, w1);
+            __stcs(reinterpret_cast<uint2*>(codes + (e0[it] >> 1)), make_uint2(w0, w1));
         } else if (e0[it] < n) {
             const int valid = (int)(n - e0[it]);
             for (int j = 0; 2 * j < valid; ++j) {
@@ -272,7 +308,10 @@ __global__ void __launch_bounds__(256) k_dq_quantize(const float* __restrict__ a
 }
 
 // ---------------------------------------------------------------------------
-// K4: standalone dequantization, one thread per 64-element block.
+// K4: standalone dequantization, one thread per 64-element block.  A warp
+// covers 32 consecutive blocks; each thread expands its block into a
+// 128-byte-swizzled shared-memory slot, then the warp writes its 4 KB of
+// output with fully coalesced 16-byte stores.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k_dequantize(const uint8_t* __restrict__ codes, int64_t n,
                                                     int dq, const float* __restrict__ absmax,
@@ -280,8 +319,37 @@ __global__ void __launch_bounds__(256) k_dequantize(const uint8_t* __restrict__ 
                                                     const float* __restrict__ c1,
                                                     const float* __restrict__ offset_ptr,
                                                     uint16_t* __restrict__ out) {
+    __shared__ __align__(16) uint8_t stage[8][4096];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t b = (int64_t)blockIdx.x * 256 + threadIdx.x;
     const int64_t nb = (n + 63) >> 6;
+    const int64_t wb0 = (int64_t)blockIdx.x * 256 + warp * 32;  // first block of this warp
+    const bool warp_full = (wb0 + 32) * 64 <= n;
+    if (warp_full) {
+        const float a = dq ? block_scale_dq(q8[b], c1[b >> 8], *offset_ptr) : absmax[b];
+        const uint4* src = reinterpret_cast<const uint4*>(codes + b * 32);
+        const uint4 c0 = __ldcs(src), c1v = __ldcs(src + 1);
+        const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1v.x, c1v.y, c1v.z, c1v.w};
+        const Nf4BlockTable t = nf4_block_table(a);
+        const uint32_t slot = smem_u32(&stage[warp][0]) + lane * 128;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            uint32_t o[4];
+            nf4_expand_word(words[i], t, o);
+            st_shared_v4(slot + ((i ^ (lane & 7)) << 4), o[0], o[1], o[2], o[3]);
+        }
+        __syncwarp();
+        uint4* dst = reinterpret_cast<uint4*>(out + wb0 * 64);
+        const uint32_t sbase = smem_u32(&stage[warp][0]);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int lin = i * 512 + lane * 16;  // linear byte offset in the warp's 4 KB
+            const int blk = lin >> 7, q = (lin >> 4) & 7;
+            const uint4 v = ld_shared_v4(sbase + blk * 128 + ((q ^ (blk & 7)) << 4));
+            __stcs(dst + i * 32 + lane, v);
+        }
+        return;
+    }
     if (b >= nb) return;
     const float a = dq ? block_scale_dq(q8[b], c1[b >> 8], *offset_ptr) : absmax[b];
     if ((b + 1) * 64 <= n) {
@@ -322,14 +390,13 @@ __global__ void k_expand_scales(int64_t rows, int64_t kbs, int dq, const float* 
 
 __global__ void k_encode(const float* __restrict__ x, int64_t n, uint8_t* __restrict__ codes,
                          Nf4SearchTable tab) {
-    __shared__ float2 s_tab[33];
-    if (threadIdx.x < 33)
-        s_tab[threadIdx.x] = make_float2(tab.thr[threadIdx.x], __int_as_float(tab.base[threadIdx.x]));
+    __shared__ SearchSmem st;
+    load_search_tables(st, tab);
     __syncthreads();
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
          i += (int64_t)gridDim.x * blockDim.x) {
         float v = fminf(fmaxf(x[i], -1.0f), 1.0f);
-        codes[i] = (uint8_t)nf4_search(v, s_tab);
+        codes[i] = (uint8_t)nf4_search(v, st);
     }
 }
 
