@@ -126,10 +126,12 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
-def source_hash():
+def source_hash(files=None):
+    """sha256 (first 16 hex digits) over the named kernel sources, or over
+    every file of the CUDA source tree when no list is given."""
     h = hashlib.sha256()
     d = os.path.join(ROOT, "bit_nf4_quantized_08_b200", "csrc")
-    for fn in sorted(os.listdir(d)):
+    for fn in sorted(files if files else os.listdir(d)):
         with open(os.path.join(d, fn), "rb") as f:
             h.update(fn.encode())
             h.update(f.read())
@@ -138,14 +140,15 @@ def source_hash():
 
 def load_traffic(kind):
     """Per-launch DRAM bytes of a kernel from a committed ncu capture, or None
-    when absent or taken on different kernel sources."""
+    when absent or taken on different kernel sources (the entry names the
+    source files its hash covers)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
     e = d.get(kind)
-    if not e or e.get("source_hash") != source_hash():
+    if not e or e.get("source_hash") != source_hash(e.get("files")):
         return None
     return e.get("dram_bytes_per_launch")
 
