@@ -6,7 +6,7 @@ quantization of the block constants, as a C-ABI CUDA library
 (``include/qlora_nf4.h``) with a thin torch binding.
 """
 from ._lib import QloraError, QLORA_OK, QLORA_ERR_INVALID_ARG, QLORA_ERR_UNSUPPORTED, \
-    QLORA_ERR_CUDA, QLORA_ERR_TIMEOUT  # noqa: F401
+    QLORA_ERR_CUDA, QLORA_ERR_TIMEOUT, QLORA_ERR_WORKSPACE, QLORA_STATIC_QUANTIZE_MAX_ELEMS  # noqa: F401
 from .api import (  # noqa: F401
     NF4Weight,
     qlora_debug_inject,
@@ -17,6 +17,7 @@ from .api import (  # noqa: F401
     qlora_nf4_dequantize,
     qlora_nf4_encode,
     qlora_nf4_quantize,
+    qlora_nf4_quantize_static,
     qlora_nf4_quantize_workspace,
     qlora_nf4_table,
     qlora_set_wait_timeout_ns,

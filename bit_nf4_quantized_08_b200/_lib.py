@@ -23,11 +23,13 @@ QLORA_ERR_WORKSPACE = 5
 STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "TIMEOUT", 5: "WORKSPACE"}
 QLORA_F32 = 0
 QLORA_BF16 = 1
+QLORA_STATIC_QUANTIZE_MAX_ELEMS = 1 << 26
 
 # Every function the header declares (checked against the header by the tests).
 EXPORTS = (
     "qlora_nf4_quantize_workspace",
     "qlora_nf4_quantize",
+    "qlora_nf4_quantize_static",
     "qlora_nf4_dequantize",
     "qlora_linear_workspace",
     "qlora_linear_fwd",
@@ -85,6 +87,8 @@ def lib() -> ctypes.CDLL:
     L.qlora_nf4_quantize_workspace.restype = sz
     L.qlora_nf4_quantize.argtypes = [vp, i32, W, vp, sz, vp]
     L.qlora_nf4_quantize.restype = i32
+    L.qlora_nf4_quantize_static.argtypes = [vp, i32, W, vp]
+    L.qlora_nf4_quantize_static.restype = i32
     L.qlora_nf4_dequantize.argtypes = [W, vp, vp]
     L.qlora_nf4_dequantize.restype = i32
     L.qlora_linear_workspace.argtypes = [i64, W, i32, i32]

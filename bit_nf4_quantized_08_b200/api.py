@@ -107,6 +107,27 @@ def qlora_nf4_quantize(W: torch.Tensor, double_quant: bool = True, out: NF4Weigh
     return out
 
 
+def qlora_nf4_quantize_static(W: torch.Tensor, out: NF4Weight) -> NF4Weight:
+    """qlora_nf4_quantize into caller-allocated outputs, with the library's
+    fixed internal scratch instead of a workspace (at most
+    QLORA_STATIC_QUANTIZE_MAX_ELEMS elements; calls on one device must not
+    overlap)."""
+    if W.dim() != 2 or not W.is_cuda or not W.is_contiguous():
+        raise ValueError("W must be a contiguous 2-D CUDA tensor")
+    if W.dtype == torch.bfloat16:
+        dt = QLORA_BF16
+    elif W.dtype == torch.float32:
+        dt = QLORA_F32
+    else:
+        raise TypeError("W must be bf16 or fp32")
+    if (out.rows, out.cols) != tuple(W.shape):
+        raise ValueError("out does not match the shape of W")
+    cw = out.c_struct()
+    check(lib().qlora_nf4_quantize_static(_ptr(W), dt, ctypes.byref(cw), _stream()),
+          "qlora_nf4_quantize_static")
+    return out
+
+
 def qlora_nf4_dequantize(w: NF4Weight, out: torch.Tensor | None = None) -> torch.Tensor:
     """doubleDequant: the bf16 weight [rows, cols] the layer multiplies with."""
     if out is None:

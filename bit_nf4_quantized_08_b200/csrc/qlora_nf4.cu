@@ -91,6 +91,37 @@ static size_t quantize_ws(int64_t n, int dq) {
     return align256((size_t)nb * 4) + align256((size_t)ng * 8);
 }
 
+// Scratch of qlora_nf4_quantize_static: the fp32 maximum of every 64-element
+// block, then the fp64 sum of every 16384-element group, for tensors of up to
+// QLORA_STATIC_QUANTIZE_MAX_ELEMS elements.  A fixed device array so that the
+// call needs no allocation; each call writes every slot it reads.
+static constexpr int64_t kStaticAbsmaxBytes = (QLORA_STATIC_QUANTIZE_MAX_ELEMS / 64) * 4;
+static constexpr int64_t kStaticSumsBytes = (QLORA_STATIC_QUANTIZE_MAX_ELEMS / 16384) * 8;
+static __device__ __align__(256) unsigned char g_quant_scratch[kStaticAbsmaxBytes + kStaticSumsBytes];
+
+// Device address of g_quant_scratch on the current device, looked up once
+// per device ordinal and kept.
+static constexpr int kMaxDevices = 64;
+static std::atomic<void*> g_scratch_addr[kMaxDevices];
+static std::mutex g_scratch_mu;
+
+static qlora_status static_quant_scratch(void** out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return QLORA_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return QLORA_ERR_UNSUPPORTED;
+    void* p = g_scratch_addr[dev].load(std::memory_order_acquire);
+    if (!p) {
+        std::lock_guard<std::mutex> lk(g_scratch_mu);
+        p = g_scratch_addr[dev].load(std::memory_order_relaxed);
+        if (!p) {
+            if (cudaGetSymbolAddress(&p, g_quant_scratch) != cudaSuccess || !p) return QLORA_ERR_CUDA;
+            g_scratch_addr[dev].store(p, std::memory_order_release);
+        }
+    }
+    *out = p;
+    return QLORA_OK;
+}
+
 static qlora_status check_linear(int64_t M, const qlora_nf4_weight* w, int32_t r) {
     qlora_status st = check_weight(w, true);
     if (st != QLORA_OK) return st;
@@ -138,6 +169,38 @@ qlora_status qlora_nf4_quantize(const void* W, qlora_dtype wdtype, const qlora_n
     float* absmax = static_cast<float*>(ws);
     double* sums = reinterpret_cast<double*>(static_cast<char*>(ws) + align256((size_t)nb * 4));
     const int64_t ng = (n + 16383) / 16384;
+    if (launch_quantize_blocks(W, is_bf16, n, out->codes, absmax, sums, s) != cudaSuccess)
+        return QLORA_ERR_CUDA;
+    if (launch_dq_offset(sums, ng, nb, out->absmax_offset, s) != cudaSuccess) return QLORA_ERR_CUDA;
+    if (launch_dq_quantize(absmax, nb, out->absmax_offset, out->absmax_q8, out->absmax_scale, s) !=
+        cudaSuccess)
+        return QLORA_ERR_CUDA;
+    return QLORA_OK;
+}
+
+qlora_status qlora_nf4_quantize_static(const void* W, qlora_dtype wdtype, const qlora_nf4_weight* out,
+                                       qlora_stream_t stream) {
+    qlora_status st = check_weight(out, true);
+    if (st != QLORA_OK) return st;
+    if (wdtype != QLORA_F32 && wdtype != QLORA_BF16) return QLORA_ERR_INVALID_ARG;
+    const int64_t n = out->rows * out->cols;
+    if (n == 0) return QLORA_OK;
+    if (!W || !aligned(W, 16)) return QLORA_ERR_INVALID_ARG;
+    if (n > QLORA_STATIC_QUANTIZE_MAX_ELEMS) return QLORA_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int is_bf16 = wdtype == QLORA_BF16;
+    if (!out->double_quant) {
+        if (launch_quantize_blocks(W, is_bf16, n, out->codes, out->absmax, nullptr, s) != cudaSuccess)
+            return QLORA_ERR_CUDA;
+        return QLORA_OK;
+    }
+    void* scratch = nullptr;
+    st = static_quant_scratch(&scratch);
+    if (st != QLORA_OK) return st;
+    const int64_t nb = (n + 63) / 64;
+    const int64_t ng = (n + 16383) / 16384;
+    float* absmax = static_cast<float*>(scratch);
+    double* sums = reinterpret_cast<double*>(static_cast<char*>(scratch) + kStaticAbsmaxBytes);
     if (launch_quantize_blocks(W, is_bf16, n, out->codes, absmax, sums, s) != cudaSuccess)
         return QLORA_ERR_CUDA;
     if (launch_dq_offset(sums, ng, nb, out->absmax_offset, s) != cudaSuccess) return QLORA_ERR_CUDA;

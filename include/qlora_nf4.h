@@ -49,7 +49,8 @@ typedef enum {
     QLORA_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
     QLORA_ERR_TIMEOUT = 4,     /* a bounded in-kernel wait ran out (reported
                                   by qlora_get_last_error only) */
-    QLORA_ERR_WORKSPACE = 5    /* reserved */
+    QLORA_ERR_WORKSPACE = 5    /* the tensor is larger than the fixed internal
+                                  scratch of qlora_nf4_quantize_static */
 } qlora_status;
 
 typedef enum { QLORA_F32 = 0, QLORA_BF16 = 1 } qlora_dtype;
@@ -109,6 +110,38 @@ size_t qlora_nf4_quantize_workspace(int64_t rows, int64_t cols, int32_t blocksiz
  */
 qlora_status qlora_nf4_quantize(const void *W, qlora_dtype wdtype, const qlora_nf4_weight *out,
                                 void *ws, size_t ws_bytes, qlora_stream_t stream);
+
+/*
+ * Largest rows*cols that qlora_nf4_quantize_static accepts: 2^26 elements
+ * (every linear of a LLaMA-7B block; the largest is 11008 x 4096).
+ */
+#define QLORA_STATIC_QUANTIZE_MAX_ELEMS ((int64_t)1 << 26)
+
+/*
+ * The same quantization as qlora_nf4_quantize, with identical outputs, but
+ * without a workspace argument and without allocating any device memory.
+ * The pages have no counterpart of this call: it exists for callers that
+ * cannot hand the library a device buffer, for example a plain C host
+ * program or a plug-in of a framework that exposes no scratch allocator, or
+ * that must not allocate once they are running under a fixed memory budget.
+ *
+ * The scratch (fp32 block maxima and fp64 group sums for the double
+ * quantization) is a fixed device array inside the library, 4 MiB + 32 KiB,
+ * reserved when the library's module is loaded on a device.  Every byte of
+ * it that is read is first written by the same call, so nothing is cleared.
+ *   - rows*cols above QLORA_STATIC_QUANTIZE_MAX_ELEMS returns
+ *     QLORA_ERR_WORKSPACE and enqueues nothing.
+ *   - The first call on each device (with that device current) looks up the
+ *     scratch address with cudaGetSymbolAddress and keeps it; make that
+ *     first call before any stream capture.  After cudaDeviceReset the kept
+ *     address is stale: do not call this function again in that process.
+ *   - One scratch per device: calls that may overlap on the same device
+ *     (different streams without ordering, or several host threads) race on
+ *     it and give wrong results.  Order such calls on one stream.
+ * Other arguments, errors and determinism as for qlora_nf4_quantize.
+ */
+qlora_status qlora_nf4_quantize_static(const void *W, qlora_dtype wdtype,
+                                       const qlora_nf4_weight *out, qlora_stream_t stream);
 
 /*
  * doubleDequant (digest sec. 4): writes the bf16 weight w' [rows, cols] that
