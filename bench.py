@@ -51,8 +51,10 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extras", action="store_true", help="skip the small-M sweep and 2^30 quantize/dequant")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
-    ap.add_argument("--profile-case", choices=["fwd", "dx", "quantize", "dequantize", "smallm"],
-                    help="run one small case three times, untimed (for ncu captures)")
+    ap.add_argument("--profile-case", choices=["fwd", "dx", "quantize", "dequantize", "smallm",
+                                               "fwd_block", "dx_block"],
+                    help="run one small case three times, untimed (for ncu captures); "
+                         "*_block runs the seven block linears once each")
     return ap.parse_args()
 
 
@@ -490,7 +492,19 @@ def run_profile_case(case):
     import bit_nf4_quantized_08_b200 as Q
     from bit_nf4_quantized_08_b200 import workloads as wl
     dev = torch.device("cuda", 0)
-    if case in ("quantize", "dequantize"):
+    if case in ("fwd_block", "dx_block"):
+        cfg = wl.CONFIGS["llama7b"]
+        M, r, s = cfg["M"], cfg["r"], cfg["alpha"] / cfg["r"]
+        for i, (_, N, K) in enumerate(cfg["linears"]):
+            W = wl.weight(N, K, seed=0, dtype=torch.bfloat16, device=dev, index_base=16 * i)
+            w = Q.qlora_nf4_quantize(W)
+            del W
+            inp = wl.linear_inputs(M, N, K, r, seed=0, device=dev, index_base=16 * i)
+            if case == "dx_block":
+                Q.qlora_linear_bwd(inp["dY"], inp["X"], w, inp["A"], inp["B"], s)
+            else:
+                Q.qlora_linear_fwd(inp["X"], w, inp["A"], inp["B"], s)
+    elif case in ("quantize", "dequantize"):
         W = wl.weight(1 << 13, 1 << 13, seed=0, dtype=torch.bfloat16, device=dev)
         w = Q.qlora_nf4_quantize(W)
         for _ in range(3):
