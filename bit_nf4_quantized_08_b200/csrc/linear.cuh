@@ -115,14 +115,15 @@ struct WsCarve {
     }
 };
 
-// Skinny GEMM out[rows][r] = scale * sum_k Aop[row][k] Bop[j][k]: 128-row
+// Skinny GEMMs out[rows][r] = scale * sum_k Aop[row][k] Bop[j][k]: 128-row
 // tiles, the reduction split across a cluster of up to 8 CTAs and summed over
-// distributed shared memory (one launch, deterministic).
-template <int BN, int A_MN, int B_MN, int STAGES>
+// distributed shared memory (deterministic); one launch for one or two
+// independent problems of the same r.
+template <int BN, int STAGES>
 inline cudaError_t launch_skinny(const SkinnyParams& p, int tiles, int cs, cudaStream_t s) {
     constexpr int smem = skinny_smem_bytes<BN, STAGES>();
     static_assert(smem <= 232448, "shared memory per CTA");
-    auto kern = k_skinny<BN, A_MN, B_MN, STAGES>;
+    auto kern = k_skinny<BN, STAGES>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg;
@@ -142,43 +143,56 @@ inline cudaError_t launch_skinny(const SkinnyParams& p, int tiles, int cs, cudaS
     return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
-template <int A_MN, int B_MN>
-inline qlora_status skinny(const CUtensorMap& tA, const CUtensorMap& tB, int rows, int r,
-                           int ksteps, float* part, float scale, int red_mode, void* out,
-                           int64_t out_ld, cudaStream_t s) {
-    (void)part;
+// One skinny problem: operands (tensor maps and majorness), extent and output.
+struct SkinnyDesc {
+    CUtensorMap tA, tB;
+    int a_mn, b_mn;
+    int rows, ksteps;
+    float scale;
+    int out_mode;  // SK_OUT_*
+    void* out;
+    int64_t out_ld;
+};
+
+inline qlora_status skinny(const SkinnyDesc* d, int nprob, int r, cudaStream_t s) {
     SkinnyParams p;
     memset(&p, 0, sizeof(p));
-    p.tmA = tA;
-    p.tmB = tB;
-    p.rows = rows;
-    p.r = r;
-    p.ksteps = ksteps;
-    p.scale = scale;
-    p.out_mode = red_mode == RED_BF16 ? SK_OUT_BF16 : (red_mode == RED_F32 ? SK_OUT_F32 : SK_OUT_F32_T);
-    p.out = out;
-    p.out_ld = out_ld;
+    int tiles = 0, kmin = 1 << 30;
+    for (int i = 0; i < nprob; ++i) {
+        tiles += ceil_div(d[i].rows, 128);
+        kmin = std::min(kmin, d[i].ksteps);
+    }
+    // clusters of up to 8 CTAs, two resident CTAs per SM, >= 2 k-steps per CTA
+    int cs = 8;
+    while (cs > 1 && ((int64_t)tiles * cs > 2 * 148 || kmin < 2 * cs)) cs >>= 1;
+    for (int i = 0; i < nprob; ++i) {
+        SkinnyProblem& q = p.pr[i];
+        q.tmA = d[i].tA;
+        q.tmB = d[i].tB;
+        q.a_mn = d[i].a_mn;
+        q.b_mn = d[i].b_mn;
+        q.rows = d[i].rows;
+        q.r = r;
+        q.ksteps = d[i].ksteps;
+        q.per = ceil_div(d[i].ksteps, cs);
+        q.tiles = ceil_div(d[i].rows, 128);
+        q.scale = d[i].scale;
+        q.out_mode = d[i].out_mode;
+        q.out = d[i].out;
+        q.out_ld = d[i].out_ld;
+    }
+    p.nprob = nprob;
     p.timeout_ns = wait_timeout_ns();
     p.inject = inject_mode() == 1 ? 1 : 0;
-    const int tiles = ceil_div(rows, 128);
-    int cs = 8;
-    while (cs > 1 && ((int64_t)tiles * cs > 2 * 148 || ksteps < 2 * cs)) cs >>= 1;
-    p.per = ceil_div(ksteps, cs);
     const int bn = lora_bn(r);
     cudaError_t e;
     if (bn == 64)
-        e = launch_skinny<64, A_MN, B_MN, 4>(p, tiles, cs, s);
+        e = launch_skinny<64, 4>(p, tiles, cs, s);
     else if (bn == 128)
-        e = launch_skinny<128, A_MN, B_MN, 4>(p, tiles, cs, s);
+        e = launch_skinny<128, 4>(p, tiles, cs, s);
     else
-        e = launch_skinny<256, A_MN, B_MN, 3>(p, tiles, cs, s);
+        e = launch_skinny<256, 3>(p, tiles, cs, s);
     return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
-}
-
-inline size_t skinny_part_bytes(int rows, int r, int ksteps) {
-    int splits, per;
-    choose_splits(ceil_div(rows, 128), ksteps, &splits, &per);
-    return (size_t)splits * rows * r * 4;
 }
 
 inline size_t small_m_part_bytes(int64_t M, int64_t N, int64_t K) {
@@ -216,15 +230,7 @@ inline LinearWs carve_linear_ws(void* ws, int64_t M, int64_t N, int64_t K, int r
     L.sU = r > 0 ? static_cast<uint16_t*>(c.take((size_t)M * r * 2)) : nullptr;
     L.sG = (r > 0 && bwd) ? static_cast<uint16_t*>(c.take((size_t)M * r * 2)) : nullptr;
     size_t part = 0;
-    if (r > 0) {
-        part = std::max(part, skinny_part_bytes((int)M, r, (int)(K / 64)));
-        if (bwd) {
-            part = std::max(part, skinny_part_bytes((int)M, r, ceil_div(N, 64)));
-            part = std::max(part, skinny_part_bytes((int)K, r, ceil_div(M, 64)));
-            part = std::max(part, skinny_part_bytes((int)N, r, ceil_div(M, 64)));
-        }
-    }
-    if (!bwd && M <= kSmallM) part = std::max(part, small_m_part_bytes(M, N, K));
+    if (!bwd && M <= kSmallM) part = small_m_part_bytes(M, N, K);
     L.part = part ? static_cast<float*>(c.take(part)) : nullptr;
     const bool big = bwd || M > kSmallM;
     L.sk_part = big ? static_cast<float*>(c.take((size_t)kMaxStreamK * 256 * 256 * 4)) : nullptr;
@@ -296,14 +302,18 @@ inline bool map_codes(CUtensorMap* m, const qlora_nf4_weight& w, uint32_t box_by
                                     : (box_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B));
 }
 
-// sU = bf16(scale * X A^T) into L.sU
-inline qlora_status compute_sU(const void* X, const LinearArgs& a, const void* A,
-                               const LinearWs& L, cudaStream_t s) {
-    CUtensorMap tX, tA;
-    if (!map_bf16(&tX, X, a.K, a.M, 128)) return QLORA_ERR_CUDA;
-    if (!map_bf16(&tA, A, a.K, a.r, lora_bn(a.r))) return QLORA_ERR_CUDA;
-    return skinny<0, 0>(tX, tA, (int)a.M, a.r, (int)(a.K / 64), L.part, a.scale, RED_BF16, L.sU,
-                        a.r, s);
+// sU = bf16(scale * X A^T): Aop = X [m][k] (K-major), Bop = A [j][k] (K-major)
+inline bool desc_sU(SkinnyDesc* d, const void* X, const LinearArgs& a, const void* A, void* sU) {
+    memset(d, 0, sizeof(*d));
+    if (!map_bf16(&d->tA, X, a.K, a.M, 128)) return false;
+    if (!map_bf16(&d->tB, A, a.K, a.r, lora_bn(a.r))) return false;
+    d->rows = (int)a.M;
+    d->ksteps = (int)(a.K / 64);
+    d->scale = a.scale;
+    d->out_mode = SK_OUT_BF16;
+    d->out = sU;
+    d->out_ld = a.r;
+    return true;
 }
 
 inline qlora_status linear_fwd_impl(const void* X, const LinearArgs& a, const void* A,
@@ -316,7 +326,9 @@ inline qlora_status linear_fwd_impl(const void* X, const LinearArgs& a, const vo
         cudaSuccess)
         return QLORA_ERR_CUDA;
     if (a.r > 0) {
-        qlora_status st = compute_sU(X, a, A, L, s);
+        SkinnyDesc d;
+        if (!desc_sU(&d, X, a, A, L.sU)) return QLORA_ERR_CUDA;
+        qlora_status st = skinny(&d, 1, a.r, s);
         if (st != QLORA_OK) return st;
     }
     GemmParams p;
@@ -424,13 +436,21 @@ inline qlora_status linear_bwd_impl(const void* dY, const void* X, const LinearA
     CUtensorMap tdY;
     if (!map_bf16(&tdY, dY, a.N, a.M, 128)) return QLORA_ERR_CUDA;
     if (a.r > 0) {
-        qlora_status st = compute_sU(X, a, A, L, s);
-        if (st != QLORA_OK) return st;
-        // sG = bf16(scale * dY B): Aop = dY [m][n] (K-major), Bop = B viewed [j][n] (MN-major)
-        CUtensorMap tBmn;
-        if (!map_bf16(&tBmn, B, a.r, a.N, 64)) return QLORA_ERR_CUDA;
-        st = skinny<0, 1>(tdY, tBmn, (int)a.M, a.r, ceil_div(a.N, 64), L.part, a.scale, RED_BF16,
-                          L.sG, a.r, s);
+        // sU = bf16(scale X A^T) and sG = bf16(scale dY B) in one launch;
+        // sG: Aop = dY [m][n] (K-major), Bop = B viewed [j][n] (MN-major)
+        SkinnyDesc d[2];
+        if (!desc_sU(&d[0], X, a, A, L.sU)) return QLORA_ERR_CUDA;
+        memset(&d[1], 0, sizeof(d[1]));
+        d[1].tA = tdY;
+        if (!map_bf16(&d[1].tB, B, a.r, a.N, 64)) return QLORA_ERR_CUDA;
+        d[1].b_mn = 1;
+        d[1].rows = (int)a.M;
+        d[1].ksteps = ceil_div(a.N, 64);
+        d[1].scale = a.scale;
+        d[1].out_mode = SK_OUT_BF16;
+        d[1].out = L.sG;
+        d[1].out_ld = a.r;
+        qlora_status st = skinny(d, 2, a.r, s);
         if (st != QLORA_OK) return st;
     }
     if (dX) {
@@ -473,17 +493,29 @@ inline qlora_status linear_bwd_impl(const void* dY, const void* X, const LinearA
     }
     if (a.r > 0) {
         // dA^T [K][r] = X^T sG : Aop = X viewed [k][m] (MN-major), Bop = sG viewed [j][m] (MN-major)
-        CUtensorMap tXmn, tGmn, tdYmn, tUmn;
-        if (!map_bf16(&tXmn, X, a.K, a.M, 64)) return QLORA_ERR_CUDA;
-        if (!map_bf16(&tGmn, L.sG, a.r, a.M, 64)) return QLORA_ERR_CUDA;
-        qlora_status st = skinny<1, 1>(tXmn, tGmn, (int)a.K, a.r, ceil_div(a.M, 64), L.part, 1.0f,
-                                       RED_F32_T, dA, a.K, s);
-        if (st != QLORA_OK) return st;
         // dB [N][r] = dY^T sU : Aop = dY viewed [n][m] (MN-major), Bop = sU viewed [j][m]
-        if (!map_bf16(&tdYmn, dY, a.N, a.M, 64)) return QLORA_ERR_CUDA;
-        if (!map_bf16(&tUmn, L.sU, a.r, a.M, 64)) return QLORA_ERR_CUDA;
-        st = skinny<1, 1>(tdYmn, tUmn, (int)a.N, a.r, ceil_div(a.M, 64), L.part, 1.0f, RED_F32, dB,
-                          a.r, s);
+        // (both in one launch)
+        SkinnyDesc d[2];
+        memset(d, 0, sizeof(d));
+        if (!map_bf16(&d[0].tA, X, a.K, a.M, 64)) return QLORA_ERR_CUDA;
+        if (!map_bf16(&d[0].tB, L.sG, a.r, a.M, 64)) return QLORA_ERR_CUDA;
+        d[0].rows = (int)a.K;
+        d[0].out_mode = SK_OUT_F32_T;
+        d[0].out = dA;
+        d[0].out_ld = a.K;
+        if (!map_bf16(&d[1].tA, dY, a.N, a.M, 64)) return QLORA_ERR_CUDA;
+        if (!map_bf16(&d[1].tB, L.sU, a.r, a.M, 64)) return QLORA_ERR_CUDA;
+        d[1].rows = (int)a.N;
+        d[1].out_mode = SK_OUT_F32;
+        d[1].out = dB;
+        d[1].out_ld = a.r;
+        for (int i = 0; i < 2; ++i) {
+            d[i].a_mn = 1;
+            d[i].b_mn = 1;
+            d[i].ksteps = ceil_div(a.M, 64);
+            d[i].scale = 1.0f;
+        }
+        qlora_status st = skinny(d, 2, a.r, s);
         if (st != QLORA_OK) return st;
     }
     return QLORA_OK;

@@ -4,10 +4,14 @@
 // out[i][j] = scale * sum_k Aop[i][k] * Bop[j][k]   (i < rows, j < r)
 // They are HBM-bound (each streams X or dY once), so the reduction dimension
 // is split across the CS CTAs of a thread-block cluster: each CTA runs a TMA
-// -> tcgen05 pipeline over its k-range into TMEM, parks its fp32 partial tile
-// in its own shared memory, and after a cluster barrier CTA z sums rows
-// [z*128/CS, (z+1)*128/CS) of all CS partials over distributed shared memory
-// in a fixed order (deterministic) and writes the final output directly.
+// -> tcgen05 pipeline over its k-range into TMEM.  Once every CTA of the
+// cluster has drained its pipeline, each pushes every row of its fp32
+// partial tile into the (now idle) pipeline buffers of the CTA that owns the
+// row, with distributed-shared-memory stores; after a second cluster barrier
+// each owner sums its rows over the CS partials in rank order (deterministic)
+// and writes the final output.  One launch carries one or two independent
+// problems of the same r (U and G, or dA and dB); the cluster index selects
+// the problem and its 128-row tile.
 #pragma once
 
 #include "common.cuh"
@@ -17,15 +21,22 @@ namespace qlora {
 
 enum { SK_OUT_BF16 = 0, SK_OUT_F32 = 1, SK_OUT_F32_T = 2 };
 
-struct SkinnyParams {
+struct SkinnyProblem {
     CUtensorMap tmA, tmB;
-    int rows, r;          // output extent
-    int ksteps;           // 64-wide k-steps of the whole reduction
-    int per;              // k-steps per cluster rank
+    int rows, r;     // output extent
+    int ksteps;      // 64-wide k-steps of the whole reduction
+    int per;         // k-steps per cluster rank
+    int a_mn, b_mn;  // operand majorness (1: MN-major)
+    int tiles;       // 128-row tiles
     float scale;
     int out_mode;
     void* out;
-    int64_t out_ld;       // elements
+    int64_t out_ld;  // elements
+};
+
+struct SkinnyParams {
+    SkinnyProblem pr[2];
+    int nprob;
     uint64_t timeout_ns;
     int inject;
 };
@@ -35,45 +46,40 @@ struct SkinnyShape {
     static constexpr int A_BYTES = 128 * 128;
     static constexpr int B_BYTES = BN * 128;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int PART_LD = BN + 4;  // fp32 partial row pitch (floats), breaks bank aliasing
-    static constexpr int PART_BYTES = 128 * PART_LD * 4;
+    static constexpr int PART_LD = BN + 4;  // fp32 row pitch of the reduction buffer (floats)
+    static constexpr int MAX_CS = 8;
+    // reduction buffer [cs][rows_per][PART_LD], cs * rows_per <= 128 + cs - 1
+    static constexpr int RED_BYTES = (128 + MAX_CS) * PART_LD * 4;
     static constexpr int THREADS = 32 * 6;  // producer, MMA, 4 epilogue warps
 };
 
 template <int BN, int STAGES>
-constexpr int skinny_smem_bytes() {
+constexpr int skinny_region_bytes() {
     constexpr int pipe = SkinnyShape<BN>::STAGE_BYTES * STAGES;
-    constexpr int part = SkinnyShape<BN>::PART_BYTES;
-    return (pipe > part ? pipe : part) + 1024 + 256;
+    constexpr int red = SkinnyShape<BN>::RED_BYTES;
+    return pipe > red ? pipe : red;
 }
 
-__device__ __forceinline__ float ld_shared_cluster_f32(uint32_t addr) {
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-    return v;
+template <int BN, int STAGES>
+constexpr int skinny_smem_bytes() {
+    return skinny_region_bytes<BN, STAGES>() + 1024 + 256;
 }
 
-// Sum of the fp32 at local offset `off` over CTAs 0..cs-1 of the cluster, in
-// rank order (all loads issued before the ordered additions).
-__device__ __forceinline__ float cluster_sum(uint32_t off, uint32_t cs) {
-    float v[8];
-#pragma unroll
-    for (int zz = 0; zz < 8; ++zz) v[zz] = zz < (int)cs ? ld_shared_cluster_f32(mapa_shared(off, zz)) : 0.0f;
-    float acc = v[0];
-#pragma unroll
-    for (int zz = 1; zz < 8; ++zz)
-        if (zz < (int)cs) acc = __fadd_rn(acc, v[zz]);
-    return acc;
+__device__ __forceinline__ void st_shared_cluster_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                                     uint32_t d) {
+    asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+                 "r"(d)
+                 : "memory");
 }
 
-template <int BN, int A_MN, int B_MN, int STAGES>
+template <int BN, int STAGES>
 __global__ void __launch_bounds__(SkinnyShape<BN>::THREADS, 1) k_skinny(const __grid_constant__ SkinnyParams p) {
     using S = SkinnyShape<BN>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
     const uint32_t base = (raw_base + 1023u) & ~1023u;
     uint8_t* gbase = smem_raw + (base - raw_base);
-    constexpr int REGION = S::STAGE_BYTES * STAGES > S::PART_BYTES ? S::STAGE_BYTES * STAGES : S::PART_BYTES;
+    constexpr int REGION = skinny_region_bytes<BN, STAGES>();
     const uint32_t bar_base = base + REGION;
     auto full = [&](int s) { return bar_base + 8u * s; };
     auto empty = [&](int s) { return bar_base + 8u * (STAGES + s); };
@@ -83,13 +89,18 @@ __global__ void __launch_bounds__(SkinnyShape<BN>::THREADS, 1) k_skinny(const __
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const WaitCfg wc{p.timeout_ns};
-    const uint32_t cs = cluster_nctarank();
-    const uint32_t z = cluster_ctarank();
-    const int tile = blockIdx.x / (int)cs;
+    const int cs = (int)cluster_nctarank();
+    const int z = (int)cluster_ctarank();
+    int tile = blockIdx.x / cs;
+    const int pi = (p.nprob > 1 && tile >= p.pr[0].tiles) ? 1 : 0;
+    if (pi) tile -= p.pr[0].tiles;
+    const SkinnyProblem& P = p.pr[pi];
+    const int a_mn = P.a_mn, b_mn = P.b_mn;
     const int m0 = tile * 128;
-    const int k0 = (int)z * p.per;
-    const int k1 = min(p.ksteps, k0 + p.per);
+    const int k0 = z * P.per;
+    const int k1 = min(P.ksteps, k0 + P.per);
     const int nk = k1 > k0 ? k1 - k0 : 0;
+    const int rows_per = (128 + cs - 1) / cs;  // tile rows owned by each rank
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -101,8 +112,8 @@ __global__ void __launch_bounds__(SkinnyShape<BN>::THREADS, 1) k_skinny(const __
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
-        prefetch_tensormap(&p.tmA);
-        prefetch_tensormap(&p.tmB);
+        prefetch_tensormap(&P.tmA);
+        prefetch_tensormap(&P.tmB);
     }
     if (warp == 1) tmem_alloc(smem_u32(tmem_holder), BN < 32 ? 32 : BN);
     tc_fence_before();
@@ -110,6 +121,7 @@ __global__ void __launch_bounds__(SkinnyShape<BN>::THREADS, 1) k_skinny(const __
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
+    // ---------------------------------------------------------------- k-range pipeline
     if (warp == 0) {
         if (lane == 0 && !p.inject) {
             int last_use[STAGES];
@@ -121,25 +133,26 @@ __global__ void __launch_bounds__(SkinnyShape<BN>::THREADS, 1) k_skinny(const __
                 const uint32_t sA = base + s * S::STAGE_BYTES;
                 const uint32_t sB = sA + S::A_BYTES;
                 mbar_arrive_expect_tx(full(s), S::A_BYTES + S::B_BYTES);
-                if (A_MN) {
-                    tma_load_2d(sA, &p.tmA, full(s), m0, k * 64);
-                    tma_load_2d(sA + 8192, &p.tmA, full(s), m0 + 64, k * 64);
+                if (a_mn) {
+                    tma_load_2d(sA, &P.tmA, full(s), m0, k * 64);
+                    tma_load_2d(sA + 8192, &P.tmA, full(s), m0 + 64, k * 64);
                 } else {
-                    tma_load_2d(sA, &p.tmA, full(s), k * 64, m0);
+                    tma_load_2d(sA, &P.tmA, full(s), k * 64, m0);
                 }
-                if (B_MN) {
-                    for (int c = 0; c < BN / 64; ++c) tma_load_2d(sB + 8192 * c, &p.tmB, full(s), 64 * c, k * 64);
+                if (b_mn) {
+                    for (int c = 0; c < BN / 64; ++c) tma_load_2d(sB + 8192 * c, &P.tmB, full(s), 64 * c, k * 64);
                 } else {
-                    tma_load_2d(sB, &p.tmB, full(s), k * 64, 0);
+                    tma_load_2d(sB, &P.tmB, full(s), k * 64, 0);
                 }
                 last_use[s] = u;
             }
+            // every load has landed before the buffers are reused below
             for (int s = 0; s < STAGES; ++s)
                 if (last_use[s] >= 0) mbar_wait(full(s), last_use[s] & 1, wc);
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16_f32(128, BN, A_MN, B_MN);
+            const uint32_t idesc = idesc_bf16_f32(128, BN, a_mn, b_mn);
             bool ok = true;
             for (int i = 0; i < nk; ++i) {
                 const int s = i % STAGES, u = i / STAGES;
@@ -149,26 +162,42 @@ __global__ void __launch_bounds__(SkinnyShape<BN>::THREADS, 1) k_skinny(const __
                 const uint32_t sB = sA + S::A_BYTES;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t ad = A_MN ? smem_desc_sw128(sA + kk * 2048, 8192, 1024)
+                    const uint64_t ad = a_mn ? smem_desc_sw128(sA + kk * 2048, 8192, 1024)
                                              : smem_desc_sw128(sA + kk * 32, 16, 1024);
-                    const uint64_t bd = B_MN ? smem_desc_sw128(sB + kk * 2048, 8192, 1024)
+                    const uint64_t bd = b_mn ? smem_desc_sw128(sB + kk * 2048, 8192, 1024)
                                              : smem_desc_sw128(sB + kk * 32, 16, 1024);
                     umma_bf16(tmem, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
                 }
                 umma_commit(empty(s));
             }
             umma_commit(acc_full);
-            if (!ok) mbar_wait(acc_full, 0, wc);
+            // the MMAs (and their reads of shared memory) are complete before
+            // the buffers are reused below
+            mbar_wait(acc_full, 0, wc);
         }
-    } else {
-        // ---------------------------------------------------------------- partial tile -> own smem
-        const int quarter = warp & 3;
-        const int row = quarter * 32 + lane;
+    }
+    bool skip = false;
+    if (warp >= 2) {
         const bool ok = mbar_wait(acc_full, 0, wc);
         if (ok) tc_fence_after();
-        const bool skip = __any_sync(0xffffffffu, !ok || *abort_flag != 0 || nk == 0);
-        float* part = reinterpret_cast<float*>(gbase);
-        for (int c0 = 0; c0 < BN; c0 += 32) {
+        skip = __any_sync(0xffffffffu, !ok || *abort_flag != 0 || nk == 0);
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // every CTA of the cluster is done with its pipeline buffers
+
+    // ---------------------------------------------------------------- push partial rows to their owners
+    if (warp >= 2) {
+        tc_fence_after();
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;  // tile row = TMEM lane of this thread
+        const int owner = row / rows_per;
+        const int orow = row - owner * rows_per;
+        const uint32_t dst_local = base + (uint32_t)((z * rows_per + orow) * S::PART_LD) * 4u;
+        const uint32_t dst = mapa_shared(dst_local, (uint32_t)owner);
+        const int rc = (P.r + 3) & ~3;
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN && c0 < rc; c0 += 32) {
             uint32_t v[32];
             if (!skip) {
                 __syncwarp();
@@ -180,43 +209,57 @@ __global__ void __launch_bounds__(SkinnyShape<BN>::THREADS, 1) k_skinny(const __
             }
 #pragma unroll
             for (int q = 0; q < 32; q += 4)
-                *reinterpret_cast<uint4*>(part + row * S::PART_LD + c0 + q) =
-                    make_uint4(v[q], v[q + 1], v[q + 2], v[q + 3]);
+                if (c0 + q < rc) st_shared_cluster_v4(dst + (uint32_t)(c0 + q) * 4u, v[q], v[q + 1], v[q + 2], v[q + 3]);
         }
     }
-    tc_fence_before();
-    __syncthreads();
-    cluster_sync();  // every CTA's partial tile is in its shared memory
+    cluster_sync();  // every partial row has landed in its owner's buffer
 
-    // ---------------------------------------------------------------- fixed-order cluster reduction
+    // ---------------------------------------------------------------- fixed-order local reduction
     if (warp >= 2) {
         const int t = threadIdx.x - 64;  // 0..127
-        const int rows_per = 128 / (int)cs;
-        const int r0 = (int)z * rows_per;
-        const uint32_t part_base = base;
-        if (p.out_mode == SK_OUT_F32_T) {
-            // out[j][m0 + row]: consecutive threads take consecutive rows
-            for (int e = t; e < rows_per * p.r; e += 128) {
-                const int j = e / rows_per, rr = r0 + e % rows_per;
-                if (m0 + rr >= p.rows) continue;
-                const float acc = cluster_sum(part_base + (uint32_t)(rr * S::PART_LD + j) * 4u, cs);
-                static_cast<float*>(p.out)[(int64_t)j * p.out_ld + m0 + rr] = __fmul_rn(acc, p.scale);
+        const int r0 = z * rows_per;
+        const int nrows = max(0, min(rows_per, min(128, P.rows - m0) - r0));
+        const float* red = reinterpret_cast<const float*>(gbase);
+        constexpr int LD = S::PART_LD;
+        if (P.out_mode == SK_OUT_F32_T) {
+            // out[j][m0 + r0 + rr]: consecutive threads take consecutive rows
+            float* out = static_cast<float*>(P.out);
+            for (int e = t; e < nrows * P.r; e += 128) {
+                const int j = e / nrows, rr = e - j * nrows;
+                float acc = red[rr * LD + j];
+                for (int zz = 1; zz < cs; ++zz) acc = __fadd_rn(acc, red[(zz * rows_per + rr) * LD + j]);
+                out[(int64_t)j * P.out_ld + m0 + r0 + rr] = __fmul_rn(acc, P.scale);
             }
         } else {
-            for (int e = t; e < rows_per * p.r; e += 128) {
-                const int rr = r0 + e / p.r, j = e % p.r;
-                if (m0 + rr >= p.rows) continue;
-                const float acc = __fmul_rn(cluster_sum(part_base + (uint32_t)(rr * S::PART_LD + j) * 4u, cs), p.scale);
-                if (p.out_mode == SK_OUT_F32) {
-                    static_cast<float*>(p.out)[(int64_t)(m0 + rr) * p.out_ld + j] = acc;
+            // four consecutive columns per thread (r % 8 == 0)
+            const int r4 = P.r >> 2;
+            for (int e = t; e < nrows * r4; e += 128) {
+                const int rr = e / r4, j = (e - rr * r4) * 4;
+                float4 acc = *reinterpret_cast<const float4*>(&red[rr * LD + j]);
+                for (int zz = 1; zz < cs; ++zz) {
+                    const float4 b = *reinterpret_cast<const float4*>(&red[(zz * rows_per + rr) * LD + j]);
+                    acc.x = __fadd_rn(acc.x, b.x);
+                    acc.y = __fadd_rn(acc.y, b.y);
+                    acc.z = __fadd_rn(acc.z, b.z);
+                    acc.w = __fadd_rn(acc.w, b.w);
+                }
+                acc.x = __fmul_rn(acc.x, P.scale);
+                acc.y = __fmul_rn(acc.y, P.scale);
+                acc.z = __fmul_rn(acc.z, P.scale);
+                acc.w = __fmul_rn(acc.w, P.scale);
+                const int64_t o = (int64_t)(m0 + r0 + rr) * P.out_ld + j;
+                if (P.out_mode == SK_OUT_F32) {
+                    *reinterpret_cast<float4*>(static_cast<float*>(P.out) + o) = acc;
                 } else {
-                    const uint32_t h = pack_bf16x2(acc, 0.0f) & 0xFFFFu;
-                    static_cast<uint16_t*>(p.out)[(int64_t)(m0 + rr) * p.out_ld + j] = (uint16_t)h;
+                    uint2 h;
+                    h.x = pack_bf16x2(acc.x, acc.y);
+                    h.y = pack_bf16x2(acc.z, acc.w);
+                    *reinterpret_cast<uint2*>(static_cast<uint16_t*>(P.out) + o) = h;
                 }
             }
         }
     }
-    cluster_sync();  // no CTA leaves while a peer may still read its partial
+    __syncthreads();
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, BN < 32 ? 32 : BN);

@@ -44,6 +44,9 @@ FWD_CASES = [
     (3, 1000, 512, 64),
     (1, 256, 128, 8),
     (33, 136, 192, 32),
+    (300, 640, 512, 128),
+    (200, 264, 192, 256),
+    (17, 384, 256, 128),
 ]
 
 
@@ -56,7 +59,8 @@ def test_fwd_parity(Q, O, cuda, M, N, K, r):
 
 
 @pytest.mark.parametrize("M,N,K,r", [(300, 640, 512, 16), (129, 264, 256, 8), (65, 512, 128, 64),
-                                     (200, 256, 320, 0), (7, 264, 192, 8), (130, 520, 256, 24)])
+                                     (200, 256, 320, 0), (7, 264, 192, 8), (130, 520, 256, 24),
+                                     (200, 264, 192, 128), (96, 136, 128, 256), (1100, 264, 1088, 64)])
 def test_bwd_parity(Q, O, cuda, M, N, K, r):
     q, inp, Wd_ref = _setup(Q, O, M, N, K, r, seed=2, b_std=0.05)
     s = 2.0
