@@ -189,6 +189,13 @@ class Block:
         self.fwd_gemm_flops = sum(2 * self.M * L["N"] * L["K"] + 2 * self.M * self.r * L["N"] for L in self.layers)
         self.dx_gemm_flops = sum(2 * self.M * L["N"] * L["K"] + 2 * self.M * self.r * L["K"] for L in self.layers)
         self.quant_bytes = sum(L["N"] * L["K"] * (2 + WEIGHT_BYTES_PER_ELEM) for L in self.layers)
+        # LoRA skinny GEMMs per step: forward U; backward U and G; dA and dB
+        M, r = self.M, self.r
+        self.lora_bytes = sum(
+            (2 * M * L["K"] + 2 * r * L["K"] + 2 * M * r)
+            + (2 * M * L["K"] + 2 * r * L["K"] + 2 * M * L["N"] + 2 * L["N"] * r + 4 * M * r)
+            + (2 * M * L["K"] + 2 * M * L["N"] + 4 * M * r + 4 * r * L["K"] + 4 * L["N"] * r)
+            for L in self.layers)
 
     def step(self):
         Q, ws = self.Q, self.ws
@@ -370,17 +377,37 @@ def main():
     torch.cuda.synchronize()
     assert Q.qlora_get_last_error() == 0
 
+    # kernels of one step (the host launch counter of an eager step)
+    l0 = Q.qlora_kernel_launches()
+    blk.step()
+    launches_per_step = Q.qlora_kernel_launches() - l0
+    # eager steps: the host launches every kernel of the step
+    eager_times = time_steps(torch, blk.step, min(args.steps, 5), flush, barrier)
+    # the timed steps replay one CUDA graph of the step (no host launch cost)
+    side = torch.cuda.Stream(device=device)
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        blk.step()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        blk.step()
+    graph.replay()
+    torch.cuda.synchronize()
+
     clocks = ClockSampler(local_rank)
     clocks.start()
-    launches0 = Q.qlora_kernel_launches()
-    Q.qlora_profile_enable(True)
-    times = time_steps(torch, blk.step, args.steps, flush, barrier)
-    launches = Q.qlora_kernel_launches() - launches0
+    times = time_steps(torch, graph.replay, args.steps, flush, barrier)
     clk = clocks.stop()
-    prof = {k: Q.qlora_profile_read(k) for k in ("quantize", "fwd_gemm", "dx_gemm")}
-    Q.qlora_profile_enable(False)
+    launches = launches_per_step * args.steps
     status = Q.qlora_get_last_error()
     assert status == 0, f"device status {status}"
+    # per-kernel device times from a separate eager pass with launch events
+    Q.qlora_profile_enable(True)
+    time_steps(torch, blk.step, args.steps, flush, barrier)
+    prof = {k: Q.qlora_profile_read(k) for k in ("quantize", "fwd_gemm", "dx_gemm", "lora_gemm")}
+    Q.qlora_profile_enable(False)
 
     total_ms = sum(times)
     t = torch.tensor([total_ms], dtype=torch.float64, device=device)
@@ -407,6 +434,11 @@ def main():
     if qn:
         breakdown["quantize_GBps"] = round(blk.quant_bytes * args.steps / (qms * 1e-3) / 1e9, 1)
         breakdown["quantize_frac_hbm"] = round(breakdown["quantize_GBps"] / peaks["hbm_gbs"], 3)
+    lms, ln = prof["lora_gemm"]
+    if ln:
+        breakdown["lora_gemm_GBps"] = round(blk.lora_bytes * args.steps / (lms * 1e-3) / 1e9, 1)
+        breakdown["lora_gemm_frac_hbm"] = round(breakdown["lora_gemm_GBps"] / peaks["hbm_gbs"], 3)
+        breakdown["lora_gemm_share_of_step"] = round(lms / total_ms, 3)
     for k in ("fwd_gemm", "dx_gemm"):
         ms_k, n_k = prof[k]
         fl = (blk.fwd_gemm_flops if k == "fwd_gemm" else blk.dx_gemm_flops) * args.steps
@@ -468,7 +500,9 @@ def main():
             "data": "synthetic",
             "config": {"workload": WORKLOAD, "global_batch": 2048 * world, "seq_len": 512,
                        "flops_per_step": blk_flops_cache(wl), "l2": "flushed between steps (256 MiB write)",
-                       "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
+                       "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
+                       "launch": "one CUDA graph per step (captured from the library calls)",
+                       "eager_ms_per_step": round(sum(eager_times) / len(eager_times), 4)},
             "roofline": roofline, "breakdown": breakdown, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": int(launches), "clocks": clk, "extra": extra,
         }

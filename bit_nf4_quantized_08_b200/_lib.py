@@ -43,7 +43,7 @@ EXPORTS = (
     "qlora_profile_enable",
     "qlora_profile_read",
 )
-KERNEL_KINDS = {"quantize": 0, "dequantize": 1, "fwd_gemm": 2, "dx_gemm": 3, "smallm_gemm": 4}
+KERNEL_KINDS = {"quantize": 0, "dequantize": 1, "fwd_gemm": 2, "dx_gemm": 3, "smallm_gemm": 4, "lora_gemm": 5}
 
 
 class QloraError(RuntimeError):

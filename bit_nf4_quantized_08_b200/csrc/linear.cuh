@@ -13,6 +13,8 @@
 #pragma once
 
 #include <algorithm>
+#include <atomic>
+#include <chrono>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
@@ -20,6 +22,7 @@
 #include "gemm.cuh"
 #include "gemm_pair.cuh"
 #include "skinny.cuh"
+#include "smallm.cuh"
 #include "internal.h"
 #include "quantize.cuh"
 
@@ -119,11 +122,63 @@ struct WsCarve {
 // tiles, the reduction split across a cluster of up to 8 CTAs and summed over
 // distributed shared memory (deterministic); one launch for one or two
 // independent problems of the same r.
-template <int BN, int STAGES>
-inline cudaError_t launch_skinny(const SkinnyParams& p, int tiles, int cs, cudaStream_t s) {
-    constexpr int smem = skinny_smem_bytes<BN, STAGES>();
+// How many clusters of cs CTAs of k_skinny<BN> can be resident at
+// once on the current device (queried once per device, BN and cs).
+template <int BN>
+inline int skinny_active_clusters(int cs) {
+    static std::mutex mu;
+    static int cache[64][4];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 1;
+    const int lg = cs == 1 ? 0 : (cs == 2 ? 1 : (cs == 4 ? 2 : 3));
+    std::lock_guard<std::mutex> lk(mu);
+    if (cache[dev][lg] > 0) return cache[dev][lg];
+    constexpr int smem = SkinnyShape<BN>::SMEM;
+    auto kern = k_skinny<BN>;
+    int n = 0;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess) {
+        cudaLaunchConfig_t cfg;
+        memset(&cfg, 0, sizeof(cfg));
+        cfg.gridDim = dim3((unsigned)(cs * 64), 1, 1);
+        cfg.blockDim = dim3(SkinnyShape<BN>::THREADS, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeClusterDimension;
+        at[0].val.clusterDim.x = (unsigned)cs;
+        at[0].val.clusterDim.y = 1;
+        at[0].val.clusterDim.z = 1;
+        cfg.attrs = at;
+        cfg.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+            cudaGetLastError();
+            n = 0;
+        }
+    }
+    if (n < 1) n = 1;
+    cache[dev][lg] = n;
+    return n;
+}
+
+template <int BN>
+inline cudaError_t launch_skinny(SkinnyParams& p, int tiles, int kmin, int kmax, cudaStream_t s) {
+    constexpr int smem = SkinnyShape<BN>::SMEM;
     static_assert(smem <= 232448, "shared memory per CTA");
-    auto kern = k_skinny<BN, STAGES>;
+    // Cluster size: fewest rounds of resident clusters times k-steps per CTA
+    // (plus a fixed per-CTA cost of about three k-steps), at least one
+    // k-step per CTA of the shorter problem.
+    int cs = 1;
+    int64_t best = -1;
+    for (int c = 8; c >= 1; c >>= 1) {
+        if (c > 1 && kmin < c) continue;
+        const int64_t rounds = ceil_div(tiles, skinny_active_clusters<BN>(c));
+        const int64_t cost = rounds * (ceil_div(kmax, c) + 3);
+        if (best < 0 || cost < best) {
+            best = cost;
+            cs = c;
+        }
+    }
+    for (int i = 0; i < p.nprob; ++i) p.pr[i].per = ceil_div(p.pr[i].ksteps, cs);
+    auto kern = k_skinny<BN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg;
@@ -139,6 +194,7 @@ inline cudaError_t launch_skinny(const SkinnyParams& p, int tiles, int cs, cudaS
     at[0].val.clusterDim.z = 1;
     cfg.attrs = at;
     cfg.numAttrs = 1;
+    ProfileScope ps(QLORA_KERNEL_LORA_GEMM, s);
     note_launch();
     return cudaLaunchKernelEx(&cfg, kern, p);
 }
@@ -157,14 +213,12 @@ struct SkinnyDesc {
 inline qlora_status skinny(const SkinnyDesc* d, int nprob, int r, cudaStream_t s) {
     SkinnyParams p;
     memset(&p, 0, sizeof(p));
-    int tiles = 0, kmin = 1 << 30;
+    int tiles = 0, kmin = 1 << 30, kmax = 0;
     for (int i = 0; i < nprob; ++i) {
         tiles += ceil_div(d[i].rows, 128);
         kmin = std::min(kmin, d[i].ksteps);
+        kmax = std::max(kmax, d[i].ksteps);
     }
-    // clusters of up to 8 CTAs, two resident CTAs per SM, >= 2 k-steps per CTA
-    int cs = 8;
-    while (cs > 1 && ((int64_t)tiles * cs > 2 * 148 || kmin < 2 * cs)) cs >>= 1;
     for (int i = 0; i < nprob; ++i) {
         SkinnyProblem& q = p.pr[i];
         q.tmA = d[i].tA;
@@ -174,7 +228,6 @@ inline qlora_status skinny(const SkinnyDesc* d, int nprob, int r, cudaStream_t s
         q.rows = d[i].rows;
         q.r = r;
         q.ksteps = d[i].ksteps;
-        q.per = ceil_div(d[i].ksteps, cs);
         q.tiles = ceil_div(d[i].rows, 128);
         q.scale = d[i].scale;
         q.out_mode = d[i].out_mode;
@@ -187,19 +240,18 @@ inline qlora_status skinny(const SkinnyDesc* d, int nprob, int r, cudaStream_t s
     const int bn = lora_bn(r);
     cudaError_t e;
     if (bn == 64)
-        e = launch_skinny<64, 4>(p, tiles, cs, s);
+        e = launch_skinny<64>(p, tiles, kmin, kmax, s);
     else if (bn == 128)
-        e = launch_skinny<128, 4>(p, tiles, cs, s);
+        e = launch_skinny<128>(p, tiles, kmin, kmax, s);
     else
-        e = launch_skinny<256, 3>(p, tiles, cs, s);
+        e = launch_skinny<256>(p, tiles, kmin, kmax, s);
     return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
-inline size_t small_m_part_bytes(int64_t M, int64_t N, int64_t K) {
-    int splits, per;
-    choose_splits(ceil_div(N, 128), (int)(K / 64), &splits, &per);
-    return splits > 1 ? (size_t)splits * M * N * 4 : 0;
-}
+// Most CTAs of the small-M kernel's persistent grid (partial tiles and flags).
+constexpr int kMaxSmallMCtas = 256;
+
+inline int small_m_nt(int64_t M) { return M <= 16 ? 16 : (M <= 32 ? 32 : 64); }
 
 inline int sm_count() {
     int dev = 0, n = 148;
@@ -216,7 +268,8 @@ struct LinearWs {
     int64_t scales_ld;
     uint16_t* sU;
     uint16_t* sG;
-    float* part;
+    float* part;          // small-M partial tiles
+    uint32_t* sm_flags;   // small-M partial flags
     float* sk_part;  // stream-K partial tiles [kMaxStreamK][256*256]
     int* sk_flags;   // [kMaxStreamK]
     size_t bytes;
@@ -225,14 +278,14 @@ struct LinearWs {
 inline LinearWs carve_linear_ws(void* ws, int64_t M, int64_t N, int64_t K, int r, int bwd) {
     WsCarve c{static_cast<char*>(ws), 0};
     LinearWs L;
+    const bool big = bwd || M > kSmallM;
     L.scales_ld = ((N + 255) / 256) * 256;
-    L.scales = static_cast<float*>(c.take((size_t)(K / 64) * L.scales_ld * 4));
+    L.scales = big ? static_cast<float*>(c.take((size_t)(K / 64) * L.scales_ld * 4)) : nullptr;
     L.sU = r > 0 ? static_cast<uint16_t*>(c.take((size_t)M * r * 2)) : nullptr;
     L.sG = (r > 0 && bwd) ? static_cast<uint16_t*>(c.take((size_t)M * r * 2)) : nullptr;
-    size_t part = 0;
-    if (!bwd && M <= kSmallM) part = small_m_part_bytes(M, N, K);
-    L.part = part ? static_cast<float*>(c.take(part)) : nullptr;
-    const bool big = bwd || M > kSmallM;
+    // small-M forward: partial tiles [kMaxSmallMCtas][NT][128] and flags [kMaxSmallMCtas][4]
+    L.part = big ? nullptr : static_cast<float*>(c.take((size_t)kMaxSmallMCtas * small_m_nt(M) * 128 * 4));
+    L.sm_flags = big ? nullptr : static_cast<uint32_t*>(c.take((size_t)kMaxSmallMCtas * 4 * 4));
     L.sk_part = big ? static_cast<float*>(c.take((size_t)kMaxStreamK * 256 * 256 * 4)) : nullptr;
     L.sk_flags = big ? static_cast<int*>(c.take((size_t)kMaxStreamK * 4)) : nullptr;
     L.bytes = c.used;
@@ -253,7 +306,7 @@ template <int DQ, int STAGES>
 inline cudaError_t launch_gemm_pair(const GemmParams& p, dim3 grid, cudaStream_t s, int prof_kind) {
     constexpr int smem = pair_smem_bytes<DQ, STAGES>();
     static_assert(smem <= 232448, "shared memory per CTA");
-    auto kern = k_gemm_pair<DQ, STAGES>;
+    auto kern = p.streamk ? k_gemm_pair<DQ, STAGES, true> : k_gemm_pair<DQ, STAGES, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     ProfileScope ps(prof_kind, s);
@@ -262,21 +315,78 @@ inline cudaError_t launch_gemm_pair(const GemmParams& p, dim3 grid, cudaStream_t
     return cudaGetLastError();
 }
 
-// Which large-M GEMM runs: CTA pairs (default), or the single-CTA kernel on
-// the grid or stream-K schedule.  QLORA_SCHEDULE=pair|grid|streamk selects
-// one; test mode 2 forces stream-K, test mode 3 the single-CTA grid.
-enum { SCHED_PAIR = 0, SCHED_GRID = 1, SCHED_STREAMK = 2 };
+// Which large-M GEMM runs: CTA pairs with one pair per tile (default), CTA
+// pairs with the stream-K schedule, or the single-CTA kernel on the grid or
+// stream-K schedule.  QLORA_SCHEDULE=pair|pairsk|grid|streamk selects one;
+// test mode 2 forces single-CTA stream-K, mode 3 the single-CTA grid, mode 4
+// pair stream-K on 4 pairs.
+enum { SCHED_PAIR = 0, SCHED_GRID = 1, SCHED_STREAMK = 2, SCHED_PAIR_SK = 3 };
 inline int large_m_schedule() {
     if (inject_mode() == 2) return SCHED_STREAMK;
     if (inject_mode() == 3) return SCHED_GRID;
+    if (inject_mode() == 4) return SCHED_PAIR_SK;
     static int v = [] {
         const char* e = getenv("QLORA_SCHEDULE");
         if (!e) return (int)SCHED_PAIR;
         if (!strcmp(e, "grid")) return (int)SCHED_GRID;
         if (!strcmp(e, "streamk")) return (int)SCHED_STREAMK;
+        if (!strcmp(e, "pairsk")) return (int)SCHED_PAIR_SK;
         return (int)SCHED_PAIR;
     }();
     return v;
+}
+
+// CTA pairs of k_gemm_pair<DQ, STAGES> that can be resident at once on the
+// current device (queried once per device).
+template <int DQ, int STAGES>
+inline int pair_active_clusters() {
+    static std::mutex mu;
+    static int cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 1;
+    std::lock_guard<std::mutex> lk(mu);
+    if (cache[dev] > 0) return cache[dev];
+    constexpr int smem = pair_smem_bytes<DQ, STAGES>();
+    auto kern = k_gemm_pair<DQ, STAGES, true>;
+    int n = 0;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess) {
+        cudaLaunchConfig_t cfg;
+        memset(&cfg, 0, sizeof(cfg));
+        cfg.gridDim = dim3(2 * 64, 1, 1);
+        cfg.blockDim = dim3(PairShape<DQ>::THREADS, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+            cudaGetLastError();
+            n = 0;
+        }
+    }
+    if (n < 1) n = 1;
+    cache[dev] = n;
+    return n;
+}
+
+// Tile schedule of the pair GEMM over tiles_m x tiles_n tiles of 512 x 256:
+// one pair per tile, or (SCHED_PAIR_SK) stream-K over all resident pairs;
+// test mode 4 runs stream-K on 4 pairs, so that tiles are cut between pairs
+// and merged even at small sizes.
+template <int DQ, int STAGES>
+inline dim3 schedule_pair(GemmParams& p, int tiles_n, int tiles_m, const LinearWs& L) {
+    const int64_t tiles = (int64_t)tiles_n * tiles_m;
+    p.tiles_n = tiles_n;
+    p.tiles_total = (int)tiles;
+    p.sk_part = L.sk_part;
+    p.sk_flags = L.sk_flags;
+    p.streamk = 0;
+    int G = 0;
+    if (inject_mode() == 4)
+        G = 4;
+    else if (large_m_schedule() == SCHED_PAIR_SK)
+        G = std::min(pair_active_clusters<DQ, STAGES>(), kMaxStreamK / 2);
+    if (G > 0 && L.sk_part && L.sk_flags) {
+        p.streamk = 1;
+        return dim3((unsigned)(2 * G), 1, 1);
+    }
+    return dim3((unsigned)(2 * tiles_n), (unsigned)tiles_m, 1);
 }
 
 inline dim3 schedule_gemm(GemmParams& p, int tiles_n, int tiles_m, const LinearWs& L) {
@@ -316,14 +426,84 @@ inline bool desc_sU(SkinnyDesc* d, const void* X, const LinearArgs& a, const voi
     return true;
 }
 
+// Launch identifier of the small-M kernel's partial-tile flags: a flag holds
+// the epoch of the launch that published it, so stale flags of earlier
+// launches (or an uninitialized workspace) never match.  Starts at a
+// clock-derived value and never returns 0.
+inline uint32_t next_epoch() {
+    static std::atomic<uint32_t> e{(uint32_t)(std::chrono::steady_clock::now().time_since_epoch().count() * 2654435761ull) | 1u};
+    uint32_t v = e.fetch_add(1) + 1;
+    if (v == 0) v = e.fetch_add(1) + 1;
+    return v;
+}
+
+template <int NT, int NG>
+inline cudaError_t launch_small_m_kernel(const SmallMParams& p, int grid, cudaStream_t s) {
+    constexpr int smem = SmallMShape<NT, NG>::SMEM;
+    static_assert(smem <= 232448, "shared memory per CTA");
+    auto kern = k_smallm<NT, NG>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    ProfileScope ps(QLORA_KERNEL_SMALLM_GEMM, s);
+    note_launch();
+    kern<<<grid, SmallMShape<NT, NG>::THREADS, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
+// Y = X W'^T + sU B^T for M <= 64 on a persistent stream-K grid (one CTA per
+// SM, at least four (tile, k-step) units per CTA).
+inline qlora_status launch_small_m(const void* X, const LinearArgs& a, const void* B, void* Y,
+                                   const LinearWs& L, cudaStream_t s) {
+    const qlora_nf4_weight& w = *a.w;
+    const int NT = small_m_nt(a.M);
+    SmallMParams p;
+    memset(&p, 0, sizeof(p));
+    if (!map_codes(&p.tmCodes, w, 32, 128)) return QLORA_ERR_CUDA;
+    if (!map_bf16(&p.tmX, X, a.K, a.M, NT)) return QLORA_ERR_CUDA;
+    if (a.r > 0) {
+        if (!map_bf16(&p.tmB, B, a.r, a.N, 128)) return QLORA_ERR_CUDA;
+        if (!map_bf16(&p.tmU, L.sU, a.r, a.M, NT)) return QLORA_ERR_CUDA;
+    } else {
+        p.tmB = p.tmX;
+        p.tmU = p.tmX;
+    }
+    p.q8 = w.absmax_q8;
+    p.c1 = w.absmax_scale;
+    p.offset = w.absmax_offset;
+    p.absmax = w.absmax;
+    p.dq = w.double_quant;
+    p.N = (int)a.N;
+    p.M = (int)a.M;
+    p.kbs = (int)(a.K / 64);
+    p.ks_main = (int)(a.K / 64);
+    p.ks_lora = a.r > 0 ? ceil_div(a.r, 64) : 0;
+    p.tiles = ceil_div(a.N, 128);
+    p.Y = static_cast<uint16_t*>(Y);
+    p.part = L.part;
+    p.flags = L.sm_flags;
+    p.epoch = next_epoch();
+    p.timeout_ns = wait_timeout_ns();
+    p.inject = inject_mode() == 1 ? 1 : 0;
+    const int64_t units = (int64_t)p.tiles * (p.ks_main + p.ks_lora);
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(std::min(sm_count(), kMaxSmallMCtas), units / 4));
+    cudaError_t e;
+    if (NT == 16)
+        e = launch_small_m_kernel<16, 3>(p, grid, s);
+    else if (NT == 32)
+        e = launch_small_m_kernel<32, 3>(p, grid, s);
+    else
+        e = launch_small_m_kernel<64, 3>(p, grid, s);
+    return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
 inline qlora_status linear_fwd_impl(const void* X, const LinearArgs& a, const void* A,
                                     const void* B, void* Y, void* ws, size_t ws_bytes,
                                     cudaStream_t s) {
     (void)ws_bytes;
     const qlora_nf4_weight& w = *a.w;
     LinearWs L = carve_linear_ws(ws, a.M, a.N, a.K, a.r, 0);
-    if (launch_expand_scales(w, L.scales, L.scales_ld, s, L.sk_flags, L.sk_flags ? kMaxStreamK : 0) !=
-        cudaSuccess)
+    if (a.M > kSmallM &&
+        launch_expand_scales(w, L.scales, L.scales_ld, s, L.sk_flags, L.sk_flags ? kMaxStreamK : 0) != cudaSuccess)
         return QLORA_ERR_CUDA;
     if (a.r > 0) {
         SkinnyDesc d;
@@ -359,10 +539,10 @@ inline qlora_status linear_fwd_impl(const void* X, const LinearArgs& a, const vo
         p.cols = (int)a.N;
         p.out_ld = a.N;
         if (!map_bf16(&p.tmOut, Y, a.N, a.M, 128)) return QLORA_ERR_CUDA;
-        if (large_m_schedule() == SCHED_PAIR) {
+        if (large_m_schedule() == SCHED_PAIR || large_m_schedule() == SCHED_PAIR_SK) {
             if (!map_codes(&p.tmCodes, w, 32, 128)) return QLORA_ERR_CUDA;
             if (a.r > 0 && !map_bf16(&p.tmB2, B, a.r, a.N, 128)) return QLORA_ERR_CUDA;
-            dim3 grid(2 * ceil_div(a.N, 256), ceil_div(a.M, 512), 1);
+            dim3 grid = schedule_pair<DQ_B_K, 4>(p, ceil_div(a.N, 256), ceil_div(a.M, 512), L);
             if (launch_gemm_pair<DQ_B_K, 4>(p, grid, s, QLORA_KERNEL_FWD_GEMM) != cudaSuccess)
                 return QLORA_ERR_CUDA;
             return QLORA_OK;
@@ -372,47 +552,8 @@ inline qlora_status linear_fwd_impl(const void* X, const LinearArgs& a, const vo
             return QLORA_ERR_CUDA;
         return QLORA_OK;
     }
-    // small M: Y^T = [W' | B] [X | sU]^T, weight rows on the 128-lane side.
-    const int bn = a.M <= 32 ? 32 : 64;
-    if (!map_bf16(&p.tmB, X, a.K, a.M, bn)) return QLORA_ERR_CUDA;
-    p.tmA = p.tmB;
-    if (!map_codes(&p.tmCodes, w, 32, 128)) return QLORA_ERR_CUDA;
-    if (a.r > 0) {
-        if (!map_bf16(&p.tmA2, B, a.r, a.N, 128)) return QLORA_ERR_CUDA;
-        if (!map_bf16(&p.tmB2, L.sU, a.r, a.M, bn)) return QLORA_ERR_CUDA;
-    } else {
-        p.tmA2 = p.tmB;
-        p.tmB2 = p.tmB;
-    }
-    const int tiles = ceil_div(a.N, 128);
-    int splits, per;
-    choose_splits(tiles, p.ks_main, &splits, &per);
-    p.ks_per_split = per;
-    p.rows = (int)a.N;
-    p.cols = (int)a.M;
-    dim3 grid(1, tiles, splits);
-    cudaError_t e;
-    if (splits == 1) {
-        p.out_ld = a.N;
-        if (bn == 32)
-            e = launch_gemm<32, 0, 0, DQ_A_K, EPI_BF16_T, 6>(p, grid, s, QLORA_KERNEL_SMALLM_GEMM);
-        else
-            e = launch_gemm<64, 0, 0, DQ_A_K, EPI_BF16_T, 6>(p, grid, s, QLORA_KERNEL_SMALLM_GEMM);
-        return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
-    }
-    p.out = L.part;
-    p.out_ld = a.N;
-    p.out_split_stride = a.M * a.N;
-    if (bn == 32)
-        e = launch_gemm<32, 0, 0, DQ_A_K, EPI_F32_T, 6>(p, grid, s, QLORA_KERNEL_SMALLM_GEMM);
-    else
-        e = launch_gemm<64, 0, 0, DQ_A_K, EPI_F32_T, 6>(p, grid, s, QLORA_KERNEL_SMALLM_GEMM);
-    if (e != cudaSuccess) return QLORA_ERR_CUDA;
-    const int64_t total = a.M * a.N;
-    note_launch();
-    k_splitk_reduce<<<ceil_div(total, 256), 256, 0, s>>>(L.part, splits, a.M * a.N, (int)a.M,
-                                                         (int)a.N, a.N, 1.0f, RED_BF16, Y, a.N);
-    return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+    // small M: Y^T = [W' | B] [X | sU]^T, weight rows on the 128-lane side
+    return launch_small_m(X, a, B, Y, L, s);
 }
 
 inline qlora_status linear_bwd_impl(const void* dY, const void* X, const LinearArgs& a,
@@ -480,9 +621,9 @@ inline qlora_status linear_bwd_impl(const void* dY, const void* X, const LinearA
         if (!map_bf16(&p.tmOut, dX, a.K, a.M, 128)) return QLORA_ERR_CUDA;
         p.timeout_ns = wait_timeout_ns();
         p.inject = inject_mode() == 1 ? 1 : 0;
-        if (large_m_schedule() == SCHED_PAIR) {
+        if (large_m_schedule() == SCHED_PAIR || large_m_schedule() == SCHED_PAIR_SK) {
             if (!map_codes(&p.tmCodes, w, 64, 64)) return QLORA_ERR_CUDA;
-            dim3 grid(2 * ceil_div(a.K, 256), ceil_div(a.M, 512), 1);
+            dim3 grid = schedule_pair<DQ_B_MN, 4>(p, ceil_div(a.K, 256), ceil_div(a.M, 512), L);
             if (launch_gemm_pair<DQ_B_MN, 4>(p, grid, s, QLORA_KERNEL_DX_GEMM) != cudaSuccess)
                 return QLORA_ERR_CUDA;
         } else {

@@ -38,6 +38,8 @@ static size_t g_prof_used = 0;
 
 ProfileScope::ProfileScope(int k, cudaStream_t st) : kind(k), s(st), slot(-1) {
     if (k < 0 || !g_prof_on.load()) return;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone) return;
     std::lock_guard<std::mutex> lk(g_prof_mu);
     if (g_prof_used == g_prof_pool.size()) {
         cudaEvent_t a, b;
@@ -295,6 +297,17 @@ void qlora_profile_enable(int32_t on) {
     std::lock_guard<std::mutex> lk(g_prof_mu);
     g_prof.clear();
     g_prof_used = 0;
+    // create the event pairs up front, so that recording adds no event
+    // creation to the measured launches
+    while (on && g_prof_pool.size() < 2048) {
+        cudaEvent_t a, b;
+        if (cudaEventCreate(&a) != cudaSuccess) break;
+        if (cudaEventCreate(&b) != cudaSuccess) {
+            cudaEventDestroy(a);
+            break;
+        }
+        g_prof_pool.push_back({a, b});
+    }
     g_prof_on.store(on ? 1 : 0);
 }
 

@@ -4,14 +4,17 @@
 // out[i][j] = scale * sum_k Aop[i][k] * Bop[j][k]   (i < rows, j < r)
 // They are HBM-bound (each streams X or dY once), so the reduction dimension
 // is split across the CS CTAs of a thread-block cluster: each CTA runs a TMA
-// -> tcgen05 pipeline over its k-range into TMEM.  Once every CTA of the
-// cluster has drained its pipeline, each pushes every row of its fp32
-// partial tile into the (now idle) pipeline buffers of the CTA that owns the
-// row, with distributed-shared-memory stores; after a second cluster barrier
-// each owner sums its rows over the CS partials in rank order (deterministic)
-// and writes the final output.  One launch carries one or two independent
-// problems of the same r (U and G, or dA and dB); the cluster index selects
-// the problem and its 128-row tile.
+// -> tcgen05 pipeline over its k-range into TMEM, then sends every row of
+// its fp32 partial tile to the CTA that owns the row with asynchronous
+// distributed-shared-memory stores that complete on the owner's mbarrier.
+// Each owner waits for its CS partials, sums them in rank order
+// (deterministic) and writes the final output.  One launch carries one or
+// two independent problems of the same r (U and G, or dA and dB); the
+// cluster index selects the problem and its 128-row tile.
+//
+// The reduction buffer has its own shared memory, except for r > 128
+// (RED_OVERLAY), where it reuses the pipeline buffers once every CTA of the
+// cluster has drained its pipeline.
 #pragma once
 
 #include "common.cuh"
@@ -47,44 +50,52 @@ struct SkinnyShape {
     static constexpr int B_BYTES = BN * 128;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int PART_LD = BN + 4;  // fp32 row pitch of the reduction buffer (floats)
-    static constexpr int MAX_CS = 8;
-    // reduction buffer [cs][rows_per][PART_LD], cs * rows_per <= 128 + cs - 1
-    static constexpr int RED_BYTES = (128 + MAX_CS) * PART_LD * 4;
+    // reduction buffer [cs][128 / cs][PART_LD] (cs a power of two <= 8)
+    static constexpr int RED_BYTES = 128 * PART_LD * 4;
+    static constexpr bool RED_OVERLAY = BN > 128;
+    static constexpr int STAGES = BN <= 64 ? 7 : (BN <= 128 ? 4 : 3);
+    static constexpr int PIPE_BYTES = STAGE_BYTES * STAGES;
+    static constexpr int RED_OFF = RED_OVERLAY ? 0 : PIPE_BYTES;
+    static constexpr int REGION = RED_OVERLAY ? (PIPE_BYTES > RED_BYTES ? PIPE_BYTES : RED_BYTES)
+                                              : PIPE_BYTES + RED_BYTES;
+    static constexpr int SMEM = REGION + 1024 + 256;
     static constexpr int THREADS = 32 * 6;  // producer, MMA, 4 epilogue warps
 };
 
-template <int BN, int STAGES>
-constexpr int skinny_region_bytes() {
-    constexpr int pipe = SkinnyShape<BN>::STAGE_BYTES * STAGES;
-    constexpr int red = SkinnyShape<BN>::RED_BYTES;
-    return pipe > red ? pipe : red;
+__device__ __forceinline__ void cluster_arrive() {
+    __syncwarp();
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+    __syncwarp();
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-template <int BN, int STAGES>
-constexpr int skinny_smem_bytes() {
-    return skinny_region_bytes<BN, STAGES>() + 1024 + 256;
+// 16 bytes into another CTA's shared memory; completes 16 transaction bytes
+// on the destination CTA's mbarrier (both addresses in the cluster window).
+__device__ __forceinline__ void st_async_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d,
+                                            uint32_t bar) {
+    asm volatile(
+        "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(addr),
+        "r"(a), "r"(b), "r"(c), "r"(d), "r"(bar)
+        : "memory");
 }
 
-__device__ __forceinline__ void st_shared_cluster_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
-                                                     uint32_t d) {
-    asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
-                 "r"(d)
-                 : "memory");
-}
-
-template <int BN, int STAGES>
+template <int BN>
 __global__ void __launch_bounds__(SkinnyShape<BN>::THREADS, 1) k_skinny(const __grid_constant__ SkinnyParams p) {
     using S = SkinnyShape<BN>;
+    constexpr int STAGES = S::STAGES;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
     const uint32_t base = (raw_base + 1023u) & ~1023u;
     uint8_t* gbase = smem_raw + (base - raw_base);
-    constexpr int REGION = skinny_region_bytes<BN, STAGES>();
-    const uint32_t bar_base = base + REGION;
+    const uint32_t red_base = base + S::RED_OFF;
+    const uint32_t bar_base = base + S::REGION;
     auto full = [&](int s) { return bar_base + 8u * s; };
     auto empty = [&](int s) { return bar_base + 8u * (STAGES + s); };
     const uint32_t acc_full = bar_base + 8u * (2 * STAGES);
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + REGION + 8 * (2 * STAGES + 1));
+    const uint32_t red_full = bar_base + 8u * (2 * STAGES + 1);
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + S::REGION + 8 * (2 * STAGES + 2));
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -100,7 +111,8 @@ __global__ void __launch_bounds__(SkinnyShape<BN>::THREADS, 1) k_skinny(const __
     const int k0 = z * P.per;
     const int k1 = min(P.ksteps, k0 + P.per);
     const int nk = k1 > k0 ? k1 - k0 : 0;
-    const int rows_per = (128 + cs - 1) / cs;  // tile rows owned by each rank
+    const int rows_per = 128 / cs;  // tile rows owned by each rank
+    const int rc = (P.r + 3) & ~3;  // columns sent per row
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -108,6 +120,9 @@ __global__ void __launch_bounds__(SkinnyShape<BN>::THREADS, 1) k_skinny(const __
             mbar_init(empty(s), 1);
         }
         mbar_init(acc_full, 1);
+        mbar_init(red_full, 1);
+        // every rank (this one included) sends rows_per rows of rc floats here
+        mbar_arrive_expect_tx(red_full, (uint32_t)(cs * rows_per * rc * 4));
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -120,6 +135,10 @@ __global__ void __launch_bounds__(SkinnyShape<BN>::THREADS, 1) k_skinny(const __
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
+    // First cluster barrier: every CTA's red_full is initialized (waited on
+    // before the first remote store).  With RED_OVERLAY it also marks the
+    // end of every CTA's pipeline, so it is arrived at after the main loop.
+    if (!S::RED_OVERLAY) cluster_arrive();
 
     // ---------------------------------------------------------------- k-range pipeline
     if (warp == 0) {
@@ -146,17 +165,16 @@ __global__ void __launch_bounds__(SkinnyShape<BN>::THREADS, 1) k_skinny(const __
                 }
                 last_use[s] = u;
             }
-            // every load has landed before the buffers are reused below
+            // every load has landed before the buffers are reused or the CTA exits
             for (int s = 0; s < STAGES; ++s)
                 if (last_use[s] >= 0) mbar_wait(full(s), last_use[s] & 1, wc);
         }
     } else if (warp == 1) {
         if (lane == 0) {
             const uint32_t idesc = idesc_bf16_f32(128, BN, a_mn, b_mn);
-            bool ok = true;
             for (int i = 0; i < nk; ++i) {
                 const int s = i % STAGES, u = i / STAGES;
-                if (!mbar_wait(full(s), u & 1, wc)) { ok = false; *abort_flag = 1; break; }
+                if (!mbar_wait(full(s), u & 1, wc)) { *abort_flag = 1; break; }
                 tc_fence_after();
                 const uint32_t sA = base + s * S::STAGE_BYTES;
                 const uint32_t sB = sA + S::A_BYTES;
@@ -172,54 +190,61 @@ __global__ void __launch_bounds__(SkinnyShape<BN>::THREADS, 1) k_skinny(const __
             }
             umma_commit(acc_full);
             // the MMAs (and their reads of shared memory) are complete before
-            // the buffers are reused below
+            // the buffers are reused or the CTA exits
             mbar_wait(acc_full, 0, wc);
         }
     }
-    bool skip = false;
-    if (warp >= 2) {
-        const bool ok = mbar_wait(acc_full, 0, wc);
-        if (ok) tc_fence_after();
-        skip = __any_sync(0xffffffffu, !ok || *abort_flag != 0 || nk == 0);
-    }
-    tc_fence_before();
-    __syncthreads();
-    cluster_sync();  // every CTA of the cluster is done with its pipeline buffers
 
-    // ---------------------------------------------------------------- push partial rows to their owners
-    if (warp >= 2) {
-        tc_fence_after();
+    if (warp < 2) {
+        // producer and MMA warps: nothing left but the two cluster barriers
+        if (S::RED_OVERLAY) cluster_arrive();
+        cluster_wait();
+        cluster_arrive();
+        cluster_wait();
+    } else {
+        // ------------------------------------------------------------ send partial rows to their owners
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;  // tile row = TMEM lane of this thread
+        const bool ok = mbar_wait(acc_full, 0, wc);
+        if (ok) tc_fence_after();
+        const bool skip = __any_sync(0xffffffffu, !ok || *abort_flag != 0 || nk == 0);
+        if (S::RED_OVERLAY) cluster_arrive();
+        cluster_wait();
         const int owner = row / rows_per;
         const int orow = row - owner * rows_per;
-        const uint32_t dst_local = base + (uint32_t)((z * rows_per + orow) * S::PART_LD) * 4u;
-        const uint32_t dst = mapa_shared(dst_local, (uint32_t)owner);
-        const int rc = (P.r + 3) & ~3;
+        const uint32_t dst =
+            mapa_shared(red_base + (uint32_t)((z * rows_per + orow) * S::PART_LD) * 4u, (uint32_t)owner);
+        const uint32_t dst_bar = mapa_shared(red_full, (uint32_t)owner);
 #pragma unroll 1
-        for (int c0 = 0; c0 < BN && c0 < rc; c0 += 32) {
-            uint32_t v[32];
+        for (int c0 = 0; c0 < BN && c0 < rc; c0 += 64) {
+            uint32_t v0[32], v1[32];
             if (!skip) {
                 __syncwarp();
-                tmem_ld_32x32b_x32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)c0, v);
+                tmem_ld_32x32b_x32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)c0, v0);
+                tmem_ld_32x32b_x32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(c0 + 32), v1);
                 tmem_ld_wait();
             } else {
 #pragma unroll
-                for (int q = 0; q < 32; ++q) v[q] = 0u;
+                for (int q = 0; q < 32; ++q) v0[q] = v1[q] = 0u;
             }
 #pragma unroll
             for (int q = 0; q < 32; q += 4)
-                if (c0 + q < rc) st_shared_cluster_v4(dst + (uint32_t)(c0 + q) * 4u, v[q], v[q + 1], v[q + 2], v[q + 3]);
+                if (c0 + q < rc) st_async_v4(dst + (uint32_t)(c0 + q) * 4u, v0[q], v0[q + 1], v0[q + 2], v0[q + 3], dst_bar);
+#pragma unroll
+            for (int q = 0; q < 32; q += 4)
+                if (c0 + 32 + q < rc)
+                    st_async_v4(dst + (uint32_t)(c0 + 32 + q) * 4u, v1[q], v1[q + 1], v1[q + 2], v1[q + 3], dst_bar);
         }
-    }
-    cluster_sync();  // every partial row has landed in its owner's buffer
+        // second cluster barrier (waited on before exit): no CTA leaves
+        // while another may still send to it
+        cluster_arrive();
 
-    // ---------------------------------------------------------------- fixed-order local reduction
-    if (warp >= 2) {
+        // ------------------------------------------------------------ fixed-order reduction of the owned rows
+        const bool got = mbar_wait(red_full, 0, wc);
         const int t = threadIdx.x - 64;  // 0..127
         const int r0 = z * rows_per;
-        const int nrows = max(0, min(rows_per, min(128, P.rows - m0) - r0));
-        const float* red = reinterpret_cast<const float*>(gbase);
+        const int nrows = got ? max(0, min(rows_per, min(128, P.rows - m0) - r0)) : 0;
+        const float* red = reinterpret_cast<const float*>(gbase + S::RED_OFF);
         constexpr int LD = S::PART_LD;
         if (P.out_mode == SK_OUT_F32_T) {
             // out[j][m0 + r0 + rr]: consecutive threads take consecutive rows
@@ -258,7 +283,9 @@ __global__ void __launch_bounds__(SkinnyShape<BN>::THREADS, 1) k_skinny(const __
                 }
             }
         }
+        cluster_wait();
     }
+    tc_fence_before();
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();

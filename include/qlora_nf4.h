@@ -220,8 +220,10 @@ void qlora_set_wait_timeout_ns(uint64_t ns);
  * recorded; no GPU fault is raised, the kernels return normally.  Mode 2
  * runs the forward and dX GEMMs (M > 64) on the single-CTA kernel with the
  * stream-K schedule over 7 CTAs whatever the shape (coverage of the
- * split-tile merge); mode 3 on the single-CTA kernel with one CTA per tile.
- * Mode 0: normal (CTA-pair kernel).
+ * split-tile merge); mode 3 on the single-CTA kernel with one CTA per tile;
+ * mode 4 on the CTA-pair kernel with the stream-K schedule over 4 pairs.
+ * Mode 0: normal (CTA-pair kernel; one pair per tile, or stream-K over all
+ * resident pairs when the tiles would leave a partly idle last round).
  */
 void qlora_debug_inject(int32_t mode);
 
@@ -229,9 +231,11 @@ void qlora_debug_inject(int32_t mode);
  * Measurement hooks (used by the benchmark).
  * qlora_kernel_launches: number of kernels this library has launched in this
  *   process (all devices, all streams).
- * qlora_profile_enable(1) clears the records and starts recording a CUDA
- *   event pair around every launch of the tracked kernels below, on the
- *   stream the kernel is launched on; 0 stops recording.
+ * qlora_profile_enable(1) clears the records, creates the event pool (the
+ *   first time) and starts recording a CUDA event pair around every launch
+ *   of the tracked kernels below, on the stream the kernel is launched on
+ *   (not while that stream is being captured into a graph); 0 stops
+ *   recording.
  * qlora_profile_read: synchronizes the recorded events and returns, for one
  *   kind, the summed device time (ms) and the number of launches recorded.
  *   Returns QLORA_ERR_INVALID_ARG for an unknown kind.
@@ -242,7 +246,8 @@ typedef enum {
     QLORA_KERNEL_FWD_GEMM = 2,  /* forward dequant-GEMM, M > 64 */
     QLORA_KERNEL_DX_GEMM = 3,   /* backward dX dequant-GEMM */
     QLORA_KERNEL_SMALLM_GEMM = 4, /* forward dequant-GEMM, M <= 64 */
-    QLORA_KERNEL_KINDS = 5
+    QLORA_KERNEL_LORA_GEMM = 5, /* rank-r LoRA GEMMs (U, G, dA, dB) */
+    QLORA_KERNEL_KINDS = 6
 } qlora_kernel_kind;
 
 uint64_t qlora_kernel_launches(void);

@@ -47,6 +47,10 @@ FWD_CASES = [
     (300, 640, 512, 128),
     (200, 264, 192, 256),
     (17, 384, 256, 128),
+    # small M over many tiles: stream-K shares cut tiles between CTAs
+    (5, 2000, 2048, 64),
+    (48, 1096, 1024, 16),
+    (64, 296, 4096, 0),
 ]
 
 
@@ -142,12 +146,14 @@ def test_timeout_is_reported_and_recovers(Q, O, cuda):
     assert_close_tol(got, ref, "Y after recovery")
 
 
-@pytest.mark.parametrize("mode", [2, 3], ids=["streamk7", "single_cta_grid"])
-@pytest.mark.parametrize("M,N,K,r", [(300, 640, 512, 16), (513, 264, 256, 8), (257, 512, 192, 64)])
+@pytest.mark.parametrize("mode", [2, 3, 4], ids=["streamk7", "single_cta_grid", "pair_streamk4"])
+@pytest.mark.parametrize("M,N,K,r", [(300, 640, 512, 16), (513, 264, 256, 8), (257, 512, 192, 64),
+                                     (1100, 1280, 1024, 32), (200, 256, 1024, 8)])
 def test_alternate_schedule_parity(Q, O, cuda, mode, M, N, K, r):
     """Forward and dX on the single-CTA kernel, on the stream-K schedule
     (forced onto 7 CTAs, so that tiles are split across CTAs and merged) and
-    on the grid schedule, match the oracle and are bitwise reproducible."""
+    on the grid schedule, and on the CTA-pair kernel with stream-K forced onto
+    4 pairs, match the oracle and are bitwise reproducible."""
     q, inp, Wd_ref = _setup(Q, O, M, N, K, r, seed=7, b_std=0.05)
     X, dY, A, B = (inp[k].cuda() for k in ("X", "dY", "A", "B"))
     s = 2.0
@@ -170,3 +176,48 @@ def test_alternate_schedule_parity(Q, O, cuda, mode, M, N, K, r):
     # the default (CTA-pair) kernel gives the same values up to fp32 summation order
     Y3 = Q.qlora_linear_fwd(X, q, A, B, s)
     assert_close_tol(Y3.float().cpu().numpy(), ref, "Y default")
+
+
+def test_small_m_graph_replay(Q, O, cuda):
+    """The small-M forward captured in a CUDA graph and replayed on new
+    inputs: every replay matches the oracle (the partial-tile flags of one
+    replay are never taken for the next one's)."""
+    M, N, K, r = 7, 1536, 2048, 32
+    q, inp, Wd_ref = _setup(Q, O, M, N, K, r, seed=8)
+    X = inp["X"].cuda()
+    A, B = inp["A"].cuda(), inp["B"].cuda()
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(Q.qlora_linear_workspace(M, q, r, False), dtype=torch.uint8, device="cuda")
+    Q.qlora_linear_fwd(X, q, A, B, 2.0, Y=Y, ws=ws)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        Q.qlora_linear_fwd(X, q, A, B, 2.0, Y=Y, ws=ws)
+    for rep in range(3):
+        Xn = wl.linear_inputs(M, N, K, r, seed=20 + rep)["X"]
+        X.copy_(Xn.cuda())
+        g.replay()
+        torch.cuda.synchronize()
+        ref = O.linear_fwd(wl.bits(Xn), Wd_ref, wl.bits(inp["A"]), wl.bits(inp["B"]), 2.0)
+        assert_close_tol(Y.float().cpu().numpy(), ref, f"Y replay {rep}")
+    assert Q.qlora_get_last_error() == 0
+
+
+def test_small_m_timeout_is_reported_and_recovers(Q, O, cuda):
+    """Failure detection on the small-M kernel: skipped loads make the
+    bounded waits run out, TIMEOUT is reported, the next call is correct."""
+    M, N, K, r = 16, 1024, 1024, 16
+    q, inp, Wd_ref = _setup(Q, O, M, N, K, r, seed=9)
+    X, A, B = inp["X"].cuda(), inp["A"].cuda(), inp["B"].cuda()
+    Q.qlora_get_last_error()
+    Q.qlora_set_wait_timeout_ns(20_000_000)
+    Q.qlora_debug_inject(1)
+    try:
+        Q.qlora_linear_fwd(X, q, A, B, 2.0)
+        st = Q.qlora_get_last_error()
+    finally:
+        Q.qlora_debug_inject(0)
+        Q.qlora_set_wait_timeout_ns(0)
+    assert st == Q.QLORA_ERR_TIMEOUT
+    got, ref = _fwd_both(Q, O, q, inp, Wd_ref, 2.0, r)
+    assert_close_tol(got, ref, "Y after recovery")
