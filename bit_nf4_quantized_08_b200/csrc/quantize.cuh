@@ -248,20 +248,21 @@ __global__ void __launch_bounds__(1024) k_dq_offset(const double* __restrict__ s
 
 // Nearest 8-bit code of y in [-1, 1]: candidate from rint(127 y), then the
 // exact fp64 distances of it and its two neighbours; ties to the lower index.
-__device__ __forceinline__ int nearest_t8(float y) {
+// t8 = the 256 fp32 code values t8[k] = fl32((k - 127) / 127) (shared memory).
+__device__ __forceinline__ int nearest_t8(float y, const float* t8) {
     int k0 = __float2int_rn(__fmul_rn(y, 127.0f)) + 127;
     k0 = min(max(k0, 0), 254);
     int best = k0;
-    double bd = fabs((double)y - (double)t8_value(k0));
+    double bd = fabs((double)y - (double)t8[k0]);
     if (k0 > 0) {
-        double d = fabs((double)y - (double)t8_value(k0 - 1));
+        double d = fabs((double)y - (double)t8[k0 - 1]);
         if (d <= bd) {
             bd = d;
             best = k0 - 1;
         }
     }
     if (k0 < 254) {
-        double d = fabs((double)y - (double)t8_value(k0 + 1));
+        double d = fabs((double)y - (double)t8[k0 + 1]);
         if (d < bd) best = k0 + 1;
     }
     return best;
@@ -274,6 +275,9 @@ __global__ void __launch_bounds__(256) k_dq_quantize(const float* __restrict__ a
                                                      const float* __restrict__ offset_ptr,
                                                      uint8_t* __restrict__ q8,
                                                      float* __restrict__ c1) {
+    __shared__ float t8[256];
+    t8[threadIdx.x] = t8_value(threadIdx.x);  // blockDim.x == 256
+    __syncthreads();
     const int64_t g = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     const int64_t ng = (nb + 255) >> 8;
@@ -294,7 +298,7 @@ __global__ void __launch_bounds__(256) k_dq_quantize(const float* __restrict__ a
     const float rc = (c == 0.0f) ? 0.0f : __frcp_rn(__fmul_rn(c, p));
     uint32_t q[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) q[i] = (uint32_t)nearest_t8(__fmul_rn(__fmul_rn(d[i], p), rc));
+    for (int i = 0; i < 8; ++i) q[i] = (uint32_t)nearest_t8(__fmul_rn(__fmul_rn(d[i], p), rc), t8);
     if (b0 + 8 <= nb) {
         uint2 v;
         v.x = q[0] | (q[1] << 8) | (q[2] << 16) | (q[3] << 24);

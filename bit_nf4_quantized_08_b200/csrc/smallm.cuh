@@ -51,38 +51,46 @@ struct SmallMParams {
 
 template <int NT, int NG>
 struct SmallMShape {
-    static constexpr int A_BYTES = 128 * 128;   // 128 rows x 64 k bf16 (dequantized W' or B)
+    // Two rings: TMA stages (X or sU tile + NF4 codes of one k-step, deep, to
+    // keep enough weight bytes in flight per SM) and A slots (the 128 x 64
+    // bf16 operand the dequant warps write, or the LoRA B tile).
+    static constexpr int A_BYTES = 128 * 128;   // 128 rows x 64 k bf16
+    static constexpr int A_SLOTS = 4;
+    static constexpr int X_BYTES = NT * 128;    // NT rows x 64 k bf16 (multiple of 1024)
     static constexpr int CODE_BYTES = 128 * 32;
-    static constexpr int X_BYTES = NT * 128;    // NT rows x 64 k bf16
-    static constexpr int STAGE_RAW = A_BYTES + CODE_BYTES + X_BYTES;
-    static constexpr int STAGE_BYTES = (STAGE_RAW + 1023) / 1024 * 1024;
-    static constexpr int STAGES = 6;
+    static constexpr int T_BYTES = X_BYTES + CODE_BYTES;
+    static constexpr int T_STAGES = NT >= 64 ? 10 : 16;
+    static constexpr int T_OFF = A_BYTES * A_SLOTS;
+    static constexpr int T8_OFF = T_OFF + T_BYTES * T_STAGES;  // fp32 t8 table [256]
+    static constexpr int BAR_OFF = T8_OFF + 1024;
+    static constexpr int SMEM = BAR_OFF + 512 + 1024;
     static constexpr int ACC_COLS = NT < 32 ? 32 : NT;  // one TMEM accumulator
     static constexpr int TMEM_COLS = 2 * ACC_COLS;
     static constexpr int FIRST_DQ_WARP = 6;
     static constexpr int THREADS = 32 * (FIRST_DQ_WARP + 4 * NG);
-    static constexpr int T8_OFF = STAGE_BYTES * STAGES;  // fp32 t8 table [256]
-    static constexpr int BAR_OFF = T8_OFF + 1024;
-    static constexpr int SMEM = BAR_OFF + 256 + 1024;
 };
 
 template <int NT, int NG>
 __global__ void __launch_bounds__(SmallMShape<NT, NG>::THREADS, 1)
     k_smallm(const __grid_constant__ SmallMParams p) {
     using S = SmallMShape<NT, NG>;
-    constexpr int STAGES = S::STAGES;
+    constexpr int TS = S::T_STAGES, AS = S::A_SLOTS;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
     const uint32_t base = (raw_base + 1023u) & ~1023u;
     uint8_t* gbase = smem_raw + (base - raw_base);
     float* t8s = reinterpret_cast<float*>(gbase + S::T8_OFF);
+    auto slotA = [&](int a) { return base + (uint32_t)(a * S::A_BYTES); };
+    auto stX = [&](int s) { return base + (uint32_t)(S::T_OFF + s * S::T_BYTES); };
+    auto stC = [&](int s) { return base + (uint32_t)(S::T_OFF + s * S::T_BYTES + S::X_BYTES); };
     const uint32_t bar_base = base + S::BAR_OFF;
     auto full_tma = [&](int s) { return bar_base + 8u * s; };
-    auto full_dq = [&](int s) { return bar_base + 8u * (STAGES + s); };
-    auto empty = [&](int s) { return bar_base + 8u * (2 * STAGES + s); };
-    auto acc_full = [&](int b) { return bar_base + 8u * (3 * STAGES + b); };
-    auto acc_empty = [&](int b) { return bar_base + 8u * (3 * STAGES + 2 + b); };
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + S::BAR_OFF + 8 * (3 * STAGES + 4));
+    auto empty_tma = [&](int s) { return bar_base + 8u * (TS + s); };
+    auto a_full = [&](int a) { return bar_base + 8u * (2 * TS + a); };
+    auto a_empty = [&](int a) { return bar_base + 8u * (2 * TS + AS + a); };
+    auto acc_full = [&](int b) { return bar_base + 8u * (2 * TS + 2 * AS + b); };
+    auto acc_empty = [&](int b) { return bar_base + 8u * (2 * TS + 2 * AS + 2 + b); };
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + S::BAR_OFF + 8 * (2 * TS + 2 * AS + 4));
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -94,10 +102,13 @@ __global__ void __launch_bounds__(SmallMShape<NT, NG>::THREADS, 1)
     const int nunits = (int)(r_end - r_begin);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
+        for (int s = 0; s < TS; ++s) {
             mbar_init(full_tma(s), 1);
-            mbar_init(full_dq(s), 4);  // the four warps of the stage's dequant group
-            mbar_init(empty(s), 1);
+            mbar_init(empty_tma(s), 1);
+        }
+        for (int a = 0; a < AS; ++a) {
+            mbar_init(a_full(a), 4);  // the four warps of the unit's dequant group
+            mbar_init(a_empty(a), 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(acc_full(b), 1);
@@ -124,30 +135,28 @@ __global__ void __launch_bounds__(SmallMShape<NT, NG>::THREADS, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0 && !p.inject) {
-            int last_use[STAGES];
-            for (int s = 0; s < STAGES; ++s) last_use[s] = -1;
+            int last_use[TS];
+            for (int s = 0; s < TS; ++s) last_use[s] = -1;
             for (int it = 0; it < nunits; ++it) {
-                const int s = it % STAGES, u = it / STAGES;
-                if (!mbar_wait(empty(s), (u & 1) ^ 1, wc)) { *abort_flag = 1; break; }
+                const int s = it % TS, u = it / TS;
+                if (!mbar_wait(empty_tma(s), (u & 1) ^ 1, wc)) { *abort_flag = 1; break; }
                 const int64_t unit = r_begin + it;
                 const int tile = (int)(unit / KS), k = (int)(unit - (int64_t)tile * KS);
                 const int n0 = tile * 128;
-                const uint32_t sA = base + s * S::STAGE_BYTES;
-                const uint32_t sC = sA + S::A_BYTES;
-                const uint32_t sX = sC + S::CODE_BYTES;
                 if (k < p.ks_main) {
                     mbar_arrive_expect_tx(full_tma(s), S::CODE_BYTES + S::X_BYTES);
-                    tma_load_2d(sC, &p.tmCodes, full_tma(s), k * 32, n0);
-                    tma_load_2d(sX, &p.tmX, full_tma(s), k * 64, 0);
+                    tma_load_2d(stC(s), &p.tmCodes, full_tma(s), k * 32, n0);
+                    tma_load_2d(stX(s), &p.tmX, full_tma(s), k * 64, 0);
                 } else {
-                    const int kc = k - p.ks_main;
-                    mbar_arrive_expect_tx(full_tma(s), S::A_BYTES + S::X_BYTES);
-                    tma_load_2d(sA, &p.tmB, full_tma(s), kc * 64, n0);
-                    tma_load_2d(sX, &p.tmU, full_tma(s), kc * 64, 0);
+                    // LoRA step: the sU tile here; the B tile is loaded into the
+                    // unit's A slot by its dequant group (which is never more
+                    // than one use of the slot ahead of the MMA)
+                    mbar_arrive_expect_tx(full_tma(s), S::X_BYTES);
+                    tma_load_2d(stX(s), &p.tmU, full_tma(s), (k - p.ks_main) * 64, 0);
                 }
                 last_use[s] = u;
             }
-            for (int s = 0; s < STAGES; ++s)
+            for (int s = 0; s < TS; ++s)
                 if (last_use[s] >= 0) mbar_wait(full_tma(s), last_use[s] & 1, wc);
         }
     } else if (warp == 1) {
@@ -168,16 +177,16 @@ __global__ void __launch_bounds__(SmallMShape<NT, NG>::THREADS, 1)
                 }
                 tc_fence_after();
                 for (int j = 0; ok && j < len; ++j, ++it) {
-                    const int s = it % STAGES, u = it / STAGES;
-                    if (!mbar_wait(full_dq(s), u & 1, wc)) { ok = false; *abort_flag = 1; break; }
+                    const int s = it % TS, a = it % AS;
+                    if (!mbar_wait(a_full(a), (it / AS) & 1, wc)) { ok = false; *abort_flag = 1; break; }
                     tc_fence_after();
-                    const uint32_t sA = base + s * S::STAGE_BYTES;
-                    const uint32_t sX = sA + S::A_BYTES + S::CODE_BYTES;
+                    const uint32_t sA = slotA(a), sX = stX(s);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         umma_bf16(tmem + (uint32_t)(ab * S::ACC_COLS), smem_desc_sw128(sA + kk * 32, 16, 1024),
                                   smem_desc_sw128(sX + kk * 32, 16, 1024), idesc, (j > 0 || kk > 0) ? 1u : 0u);
-                    umma_commit(empty(s));
+                    umma_commit(a_empty(a));
+                    umma_commit(empty_tma(s));
                 }
                 umma_commit(acc_full(ab));  // one phase per segment, also when cut short
                 ++seg;
@@ -292,42 +301,74 @@ __global__ void __launch_bounds__(SmallMShape<NT, NG>::THREADS, 1)
         const uint32_t code_off = sw32(t * 32), code_off2 = sw32(t * 32 + 16);
         const uint32_t out_off = t * 128;
         const float off = p.dq ? *p.offset : 0.0f;
-        // block constant of unit `it` of this CTA (0 for rows past the weight
-        // and for LoRA steps); loaded two visits ahead of its use
-        auto fetch = [&](int it) -> float {
-            if (it >= nunits) return 0.0f;
+        // raw block constant of unit `it` of this CTA: the 8-bit code and c1
+        // (or the fp32 absmax), loaded two visits ahead of its use; a' itself
+        // is formed at the use, so that no instruction waits on the loads
+        // early.  Rows past the weight and LoRA steps get a' = 0.
+        struct Raw {
+            int q;     // q8 code, or -1 for "a' = 0"
+            float c;   // c1 (double quantization) or absmax
+        };
+        auto fetch = [&](int it) -> Raw {
+            Raw r{-1, 0.0f};
+            if (it >= nunits) return r;
             const int64_t unit = r_begin + it;
             const int tile = (int)(unit / KS), k = (int)(unit - (int64_t)tile * KS);
             const int n = tile * 128 + t;
-            if (k >= p.ks_main || n >= p.N) return 0.0f;
+            if (k >= p.ks_main || n >= p.N) return r;
             const int64_t b = (int64_t)n * p.kbs + k;
-            if (!p.dq) return __ldg(p.absmax + b);
-            const int q = __ldg(p.q8 + b);
-            const float c = __ldg(p.c1 + (b >> 8));
-            return __fadd_rn(__fmul_rn(t8s[q], c), off);
+            if (!p.dq) {
+                r.q = 0;
+                r.c = __ldg(p.absmax + b);
+            } else {
+                r.q = __ldg(p.q8 + b);
+                r.c = __ldg(p.c1 + (b >> 8));
+            }
+            return r;
         };
-        float a_next0 = fetch(g), a_next1 = fetch(g + NG);
+        auto block_const = [&](const Raw& r) -> float {
+            if (r.q < 0) return 0.0f;
+            return p.dq ? __fadd_rn(__fmul_rn(t8s[r.q], r.c), off) : r.c;
+        };
+        Raw r_next0 = fetch(g), r_next1 = fetch(g + NG);
         bool dead = false;
         for (int it = g; it < nunits; it += NG) {
-            const float a = a_next0;
-            a_next0 = a_next1;
-            a_next1 = fetch(it + 2 * NG);
+            const Raw rw = r_next0;
+            r_next0 = r_next1;
+            r_next1 = fetch(it + 2 * NG);
             if (dead) continue;
-            const int s = it % STAGES, u = it / STAGES;
-            if (!mbar_wait(full_tma(s), u & 1, wc)) {
+            const int s = it % TS, a = it % AS;
+            if (!mbar_wait(full_tma(s), (it / TS) & 1, wc)) {
                 *abort_flag = 1;
                 dead = true;
                 continue;
             }
             const int64_t unit = r_begin + it;
             const int tile = (int)(unit / KS), k = (int)(unit - (int64_t)tile * KS);
-            if (k < p.ks_main) {
-                const uint32_t sA = base + s * S::STAGE_BYTES;
-                const uint32_t sC = sA + S::A_BYTES;
+            // the A slot is free once the MMAs of its previous unit are done
+            if (!mbar_wait(a_empty(a), ((it / AS) & 1) ^ 1, wc)) {
+                *abort_flag = 1;
+                dead = true;
+                continue;
+            }
+            if (k >= p.ks_main) {
+                // LoRA step: one thread loads the B tile into the slot; its
+                // arrival carries the transaction bytes, the other three warps
+                // arrive below
+                if (dw % 4 == 0) {
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(a_full(a), S::A_BYTES);
+                        tma_load_2d(slotA(a), &p.tmB, a_full(a), (k - p.ks_main) * 64, tile * 128);
+                    }
+                    continue;
+                }
+            } else {
+                const uint32_t sA = slotA(a);
+                const uint32_t sC = stC(s);
                 const uint4 c0 = ld_shared_v4(sC + code_off);
                 const uint4 c1 = ld_shared_v4(sC + code_off2);
                 const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-                const Nf4BlockTable tb = nf4_block_table(a);
+                const Nf4BlockTable tb = nf4_block_table(block_const(rw));
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
                     uint32_t o[4];
@@ -338,7 +379,7 @@ __global__ void __launch_bounds__(SmallMShape<NT, NG>::THREADS, 1)
             }
             (void)tile;
             __syncwarp();
-            if (lane == 0) mbar_arrive(full_dq(s));
+            if (lane == 0) mbar_arrive(a_full(a));
         }
     }
 

@@ -51,6 +51,10 @@ FWD_CASES = [
     (5, 2000, 2048, 64),
     (48, 1096, 1024, 16),
     (64, 296, 4096, 0),
+    # long per-CTA unit ranges: the stage and operand rings wrap many times,
+    # LoRA steps fall in the middle of ranges
+    (16, 4096, 8192, 64),
+    (40, 2048, 4096, 128),
 ]
 
 
