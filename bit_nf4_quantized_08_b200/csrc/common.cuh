@@ -69,6 +69,32 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
     }
 }
 
+// mbar_wait for waiters that can afford to react late (epilogue warps that
+// wait for a whole tile, a producer ahead of its consumers): between polls
+// the warp sleeps, so that it does not take issue slots from the warps that
+// do the work.
+__device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity, const WaitCfg& cfg,
+                                                uint32_t sleep_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    uint64_t t0 = globaltimer_ns();
+    while (true) {
+        __nanosleep(sleep_ns);
+        if (mbar_try_wait(bar, parity)) return true;
+        if (globaltimer_ns() - t0 > cfg.timeout_ns) {
+            set_status(4);
+            return false;
+        }
+    }
+}
+
+// Programmatic dependent launch.  pdl_trigger lets the next kernel of the
+// stream (launched with programmatic serialization) start its prologue;
+// pdl_wait blocks until the previous kernel of the stream has completed and
+// its memory operations are visible.  Both are no-ops for kernels launched
+// without the attribute.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }

@@ -136,6 +136,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairShape<DQ>::THREA
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
+        pdl_trigger();
         prefetch_tensormap(&p.tmA);
         prefetch_tensormap(&p.tmCodes);
         prefetch_tensormap(&p.tmOut);
@@ -152,6 +153,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairShape<DQ>::THREA
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer (both CTAs)
+        // the block constants and the LoRA operand come from earlier kernels
+        if (lane == 0) pdl_wait();
         if (lane == 0 && !p.inject) {
             int last_use[STAGES];
             for (int s = 0; s < STAGES; ++s) last_use[s] = -1;

@@ -18,6 +18,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "gemm.cuh"
 #include "gemm_pair.cuh"
@@ -90,6 +91,35 @@ inline cudaError_t launch_gemm(const GemmParams& p, dim3 grid, cudaStream_t s, i
     note_launch();
     kern<<<grid, Sh::THREADS, smem, s>>>(p);
     return cudaGetLastError();
+}
+
+// Launch with programmatic stream serialization (the kernel may start while
+// the previous kernel of the stream finishes; it calls griddepcontrol.wait
+// before touching that kernel's results) and an optional cluster shape.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, int smem, cudaStream_t s,
+                              int cluster_x, Args&&... args) {
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[2];
+    int n = 0;
+    at[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+    if (cluster_x > 0) {
+        at[n].id = cudaLaunchAttributeClusterDimension;
+        at[n].val.clusterDim.x = (unsigned)cluster_x;
+        at[n].val.clusterDim.y = 1;
+        at[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    cfg.attrs = at;
+    cfg.numAttrs = n;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
 inline int ceil_div(int64_t a, int64_t b) { return (int)((a + b - 1) / b); }
@@ -181,22 +211,10 @@ inline cudaError_t launch_skinny(SkinnyParams& p, int tiles, int kmin, int kmax,
     auto kern = k_skinny<BN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg;
-    memset(&cfg, 0, sizeof(cfg));
-    cfg.gridDim = dim3((unsigned)(tiles * cs), 1, 1);
-    cfg.blockDim = dim3(SkinnyShape<BN>::THREADS, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute at[1];
-    at[0].id = cudaLaunchAttributeClusterDimension;
-    at[0].val.clusterDim.x = (unsigned)cs;
-    at[0].val.clusterDim.y = 1;
-    at[0].val.clusterDim.z = 1;
-    cfg.attrs = at;
-    cfg.numAttrs = 1;
     ProfileScope ps(QLORA_KERNEL_LORA_GEMM, s);
     note_launch();
-    return cudaLaunchKernelEx(&cfg, kern, p);
+    return launch_pdl(kern, dim3((unsigned)(tiles * cs), 1, 1), dim3(SkinnyShape<BN>::THREADS, 1, 1), smem, s, cs,
+                      p);
 }
 
 // One skinny problem: operands (tensor maps and majorness), extent and output.
@@ -210,9 +228,12 @@ struct SkinnyDesc {
     int64_t out_ld;
 };
 
-inline qlora_status skinny(const SkinnyDesc* d, int nprob, int r, cudaStream_t s) {
+// wait_first: the operands may have been written by the kernel just before on
+// the stream (or by an unknown earlier one), so the loads wait for it.
+inline qlora_status skinny(const SkinnyDesc* d, int nprob, int r, cudaStream_t s, int wait_first) {
     SkinnyParams p;
     memset(&p, 0, sizeof(p));
+    p.wait_first = wait_first;
     int tiles = 0, kmin = 1 << 30, kmax = 0;
     for (int i = 0; i < nprob; ++i) {
         tiles += ceil_div(d[i].rows, 128);
@@ -311,8 +332,8 @@ inline cudaError_t launch_gemm_pair(const GemmParams& p, dim3 grid, cudaStream_t
     if (e != cudaSuccess) return e;
     ProfileScope ps(prof_kind, s);
     note_launch();
-    kern<<<grid, PairShape<DQ>::THREADS, smem, s>>>(p);
-    return cudaGetLastError();
+    // cluster shape from the kernel's __cluster_dims__
+    return launch_pdl(kern, grid, dim3(PairShape<DQ>::THREADS, 1, 1), smem, s, 0, p);
 }
 
 // Which large-M GEMM runs: CTA pairs with one pair per tile (default), CTA
@@ -446,8 +467,7 @@ inline cudaError_t launch_small_m_kernel(const SmallMParams& p, int grid, cudaSt
     if (e != cudaSuccess) return e;
     ProfileScope ps(QLORA_KERNEL_SMALLM_GEMM, s);
     note_launch();
-    kern<<<grid, SmallMShape<NT, NG>::THREADS, smem, s>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3((unsigned)grid, 1, 1), dim3(SmallMShape<NT, NG>::THREADS, 1, 1), smem, s, 0, p);
 }
 
 // Y = X W'^T + sU B^T for M <= 64 on a persistent stream-K grid (one CTA per
@@ -508,7 +528,9 @@ inline qlora_status linear_fwd_impl(const void* X, const LinearArgs& a, const vo
     if (a.r > 0) {
         SkinnyDesc d;
         if (!desc_sU(&d, X, a, A, L.sU)) return QLORA_ERR_CUDA;
-        qlora_status st = skinny(&d, 1, a.r, s);
+        // after the block-constant expansion (M > 64) the operands are inputs
+        // that no running kernel writes; for small M it is the first kernel
+        qlora_status st = skinny(&d, 1, a.r, s, a.M > kSmallM ? 0 : 1);
         if (st != QLORA_OK) return st;
     }
     GemmParams p;
@@ -591,7 +613,8 @@ inline qlora_status linear_bwd_impl(const void* dY, const void* X, const LinearA
         d[1].out_mode = SK_OUT_BF16;
         d[1].out = L.sG;
         d[1].out_ld = a.r;
-        qlora_status st = skinny(d, 2, a.r, s);
+        // inputs only; without dX there is no block-constant expansion before
+        qlora_status st = skinny(d, 2, a.r, s, dX ? 0 : 1);
         if (st != QLORA_OK) return st;
     }
     if (dX) {
@@ -656,7 +679,8 @@ inline qlora_status linear_bwd_impl(const void* dY, const void* X, const LinearA
             d[i].ksteps = ceil_div(a.M, 64);
             d[i].scale = 1.0f;
         }
-        qlora_status st = skinny(d, 2, a.r, s);
+        // sG and sU come from the LoRA GEMMs above
+        qlora_status st = skinny(d, 2, a.r, s, 1);
         if (st != QLORA_OK) return st;
     }
     return QLORA_OK;

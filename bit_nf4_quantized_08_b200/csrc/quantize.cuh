@@ -384,6 +384,8 @@ __global__ void k_expand_scales(int64_t rows, int64_t kbs, int dq, const float* 
                                 const uint8_t* __restrict__ q8, const float* __restrict__ c1,
                                 const float* __restrict__ offset_ptr, float* __restrict__ scales,
                                 int64_t ld, int* __restrict__ flags, int nflags) {
+    // the LoRA GEMM that follows reads none of this kernel's outputs
+    pdl_trigger();
     const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (idx < nflags) flags[idx] = 0;
     if (idx >= rows * kbs) return;

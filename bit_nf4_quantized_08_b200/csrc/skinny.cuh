@@ -42,6 +42,7 @@ struct SkinnyParams {
     int nprob;
     uint64_t timeout_ns;
     int inject;
+    int wait_first;  // the operands may come from the previous kernel: wait before loading
 };
 
 template <int BN>
@@ -142,6 +143,13 @@ __global__ void __launch_bounds__(SkinnyShape<BN>::THREADS, 1) k_skinny(const __
 
     // ---------------------------------------------------------------- k-range pipeline
     if (warp == 0) {
+        // Operands from the previous kernel: wait for it first.  The next
+        // kernel may start once this one has passed that point (it may read
+        // inputs that this kernel's predecessors wrote).
+        if (lane == 0) {
+            if (p.wait_first) pdl_wait();
+            pdl_trigger();
+        }
         if (lane == 0 && !p.inject) {
             int last_use[STAGES];
             for (int s = 0; s < STAGES; ++s) last_use[s] = -1;
@@ -285,6 +293,9 @@ __global__ void __launch_bounds__(SkinnyShape<BN>::THREADS, 1) k_skinny(const __
         }
         cluster_wait();
     }
+    // the kernel does not complete before the previous one (its dependents
+    // may rely on both)
+    if (threadIdx.x == 0) pdl_wait();
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {

@@ -119,6 +119,7 @@ __global__ void __launch_bounds__(SmallMShape<NT, NG>::THREADS, 1)
     }
     for (int i = threadIdx.x; i < 256; i += blockDim.x) t8s[i] = t8_value(i);
     if (warp == 0 && lane == 0) {
+        pdl_trigger();
         prefetch_tensormap(&p.tmCodes);
         prefetch_tensormap(&p.tmX);
         if (p.ks_lora) {
@@ -135,6 +136,7 @@ __global__ void __launch_bounds__(SmallMShape<NT, NG>::THREADS, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0 && !p.inject) {
+            bool waited = false;
             int last_use[TS];
             for (int s = 0; s < TS; ++s) last_use[s] = -1;
             for (int it = 0; it < nunits; ++it) {
@@ -150,7 +152,12 @@ __global__ void __launch_bounds__(SmallMShape<NT, NG>::THREADS, 1)
                 } else {
                     // LoRA step: the sU tile here; the B tile is loaded into the
                     // unit's A slot by its dequant group (which is never more
-                    // than one use of the slot ahead of the MMA)
+                    // than one use of the slot ahead of the MMA).  sU comes
+                    // from the kernel before this one.
+                    if (!waited) {
+                        pdl_wait();
+                        waited = true;
+                    }
                     mbar_arrive_expect_tx(full_tma(s), S::X_BYTES);
                     tma_load_2d(stX(s), &p.tmU, full_tma(s), (k - p.ks_main) * 64, 0);
                 }
@@ -383,6 +390,8 @@ __global__ void __launch_bounds__(SmallMShape<NT, NG>::THREADS, 1)
         }
     }
 
+    // the kernel does not complete before the previous one
+    if (threadIdx.x == 0) pdl_wait();
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
