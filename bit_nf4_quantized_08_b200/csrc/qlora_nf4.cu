@@ -173,8 +173,7 @@ qlora_status qlora_nf4_quantize(const void* W, qlora_dtype wdtype, const qlora_n
     const int64_t ng = (n + 16383) / 16384;
     if (launch_quantize_blocks(W, is_bf16, n, out->codes, absmax, sums, s) != cudaSuccess)
         return QLORA_ERR_CUDA;
-    if (launch_dq_offset(sums, ng, nb, out->absmax_offset, s) != cudaSuccess) return QLORA_ERR_CUDA;
-    if (launch_dq_quantize(absmax, nb, out->absmax_offset, out->absmax_q8, out->absmax_scale, s) !=
+    if (launch_double_quant(sums, ng, absmax, nb, out->absmax_offset, out->absmax_q8, out->absmax_scale, s) !=
         cudaSuccess)
         return QLORA_ERR_CUDA;
     return QLORA_OK;
@@ -205,8 +204,7 @@ qlora_status qlora_nf4_quantize_static(const void* W, qlora_dtype wdtype, const 
     double* sums = reinterpret_cast<double*>(static_cast<char*>(scratch) + kStaticAbsmaxBytes);
     if (launch_quantize_blocks(W, is_bf16, n, out->codes, absmax, sums, s) != cudaSuccess)
         return QLORA_ERR_CUDA;
-    if (launch_dq_offset(sums, ng, nb, out->absmax_offset, s) != cudaSuccess) return QLORA_ERR_CUDA;
-    if (launch_dq_quantize(absmax, nb, out->absmax_offset, out->absmax_q8, out->absmax_scale, s) !=
+    if (launch_double_quant(sums, ng, absmax, nb, out->absmax_offset, out->absmax_q8, out->absmax_scale, s) !=
         cudaSuccess)
         return QLORA_ERR_CUDA;
     return QLORA_OK;

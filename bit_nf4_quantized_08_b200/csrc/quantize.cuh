@@ -271,18 +271,56 @@ __device__ __forceinline__ int nearest_t8(float y, const float* t8) {
 // ---------------------------------------------------------------------------
 // K3: second-level quantization; one warp per group of 256 block constants.
 // ---------------------------------------------------------------------------
+// With sums != nullptr every CTA first forms the offset itself from the
+// nsums group sums (the same pairwise tree as K2, over 256 threads) and CTA 0
+// also stores it; otherwise the offset is read from offset_ptr.
 __global__ void __launch_bounds__(256) k_dq_quantize(const float* __restrict__ absmax, int64_t nb,
-                                                     const float* __restrict__ offset_ptr,
+                                                     float* __restrict__ offset_ptr,
                                                      uint8_t* __restrict__ q8,
-                                                     float* __restrict__ c1) {
+                                                     float* __restrict__ c1,
+                                                     const double* __restrict__ sums, int64_t nsums) {
     __shared__ float t8[256];
+    __shared__ double s_w[8];
+    __shared__ float s_off;
     t8[threadIdx.x] = t8_value(threadIdx.x);  // blockDim.x == 256
+    if (sums) {
+        int64_t p2 = 1;
+        while (p2 < nsums) p2 <<= 1;
+        const int64_t chunk = p2 > 256 ? p2 / 256 : 1;
+        double stack[40];
+        int64_t cnt = 0;
+        const int64_t lo = (int64_t)threadIdx.x * chunk;
+        for (int64_t i = 0; i < chunk; ++i) {
+            const int64_t idx = lo + i;
+            double v = idx < nsums ? sums[idx] : 0.0;
+            int lvl = 0;
+            while ((cnt >> lvl) & 1) {
+                v = stack[lvl] + v;
+                ++lvl;
+            }
+            stack[lvl] = v;
+            ++cnt;
+        }
+        int top = 0;
+        while ((1ll << top) < chunk) ++top;
+        double t = stack[top];
+        for (int o = 1; o < 32; o <<= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+        if ((threadIdx.x & 31) == 0) s_w[threadIdx.x >> 5] = t;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            const double u = ((s_w[0] + s_w[1]) + (s_w[2] + s_w[3])) + ((s_w[4] + s_w[5]) + (s_w[6] + s_w[7]));
+            s_off = __double2float_rn(__ddiv_rn(u, (double)nb));
+            if (blockIdx.x == 0) *offset_ptr = s_off;
+        }
+    } else if (threadIdx.x == 0) {
+        s_off = *offset_ptr;
+    }
     __syncthreads();
     const int64_t g = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     const int64_t ng = (nb + 255) >> 8;
     if (g >= ng) return;
-    const float off = *offset_ptr;
+    const float off = s_off;
     const int64_t b0 = g * 256 + lane * 8;
     float d[8];
     float c = 0.0f;
@@ -469,13 +507,25 @@ inline cudaError_t launch_dq_offset(const double* group_sums, int64_t ngroups, i
     return cudaGetLastError();
 }
 
-inline cudaError_t launch_dq_quantize(const float* absmax, int64_t nb, const float* offset,
-                                      uint8_t* q8, float* c1, cudaStream_t s) {
+inline cudaError_t launch_dq_quantize(const float* absmax, int64_t nb, float* offset, uint8_t* q8, float* c1,
+                                      cudaStream_t s, const double* sums = nullptr, int64_t nsums = 0) {
     const int64_t ng = (nb + 255) / 256;
     if (ng == 0) return cudaSuccess;
     note_launch();
-    k_dq_quantize<<<(unsigned)((ng + 7) / 8), 256, 0, s>>>(absmax, nb, offset, q8, c1);
+    k_dq_quantize<<<(unsigned)((ng + 7) / 8), 256, 0, s>>>(absmax, nb, offset, q8, c1, sums, nsums);
     return cudaGetLastError();
+}
+
+// Double quantization of the block maxima: offset, then 8-bit codes.  Up to
+// kFusedSums group sums every CTA of the 8-bit kernel forms the offset
+// itself (one launch); above, a separate one-CTA kernel does it first.
+constexpr int64_t kFusedSums = 8192;
+inline cudaError_t launch_double_quant(const double* sums, int64_t nsums, const float* absmax, int64_t nb,
+                                       float* offset, uint8_t* q8, float* c1, cudaStream_t s) {
+    if (nsums <= kFusedSums && inject_mode() != 5) return launch_dq_quantize(absmax, nb, offset, q8, c1, s, sums, nsums);
+    cudaError_t e = launch_dq_offset(sums, nsums, nb, offset, s);
+    if (e != cudaSuccess) return e;
+    return launch_dq_quantize(absmax, nb, offset, q8, c1, s);
 }
 
 inline cudaError_t launch_dequantize(const qlora_nf4_weight& w, uint16_t* out, cudaStream_t s) {

@@ -221,7 +221,9 @@ void qlora_set_wait_timeout_ns(uint64_t ns);
  * runs the forward and dX GEMMs (M > 64) on the single-CTA kernel with the
  * stream-K schedule over 7 CTAs whatever the shape (coverage of the
  * split-tile merge); mode 3 on the single-CTA kernel with one CTA per tile;
- * mode 4 on the CTA-pair kernel with the stream-K schedule over 4 pairs.
+ * mode 4 on the CTA-pair kernel with the stream-K schedule over 4 pairs;
+ * mode 5 forms the double-quantization offset in its own kernel even for
+ * tensors whose 8-bit pass would form it itself.
  * Mode 0: normal (CTA-pair kernel; one pair per tile, or stream-K over all
  * resident pairs when the tiles would leave a partly idle last round).
  */

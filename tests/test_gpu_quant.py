@@ -145,3 +145,23 @@ def test_encode_exhaustive(Q, O, cuda):
             bad = int((got != exp).sum())
             assert bad == 0, f"{bad} mismatches in chunk starting at {first:#x}"
             start += n
+
+
+@pytest.mark.parametrize("shape", [(4096, 4096), (37, 200), (1, 16384 * 3 + 64)])
+def test_separate_offset_kernel_matches(Q, O, cuda, shape):
+    """The double-quantization offset formed by the 8-bit pass itself and by
+    its own kernel (test mode 5) are the same fp32 value, and both match the
+    oracle."""
+    W = wl.weight(shape[0], shape[1], seed=11, dtype=torch.bfloat16)
+    q_fused, ref = _run_both(Q, O, W, True)
+    Q.qlora_debug_inject(5)
+    try:
+        q_sep = Q.qlora_nf4_quantize(W.cuda(), double_quant=True)
+        torch.cuda.synchronize()
+        assert Q.qlora_get_last_error() == 0
+    finally:
+        Q.qlora_debug_inject(0)
+    for x, y in [(q_fused.codes, q_sep.codes), (q_fused.absmax_q8, q_sep.absmax_q8),
+                 (q_fused.absmax_scale.view(torch.int32), q_sep.absmax_scale.view(torch.int32)),
+                 (q_fused.absmax_offset.view(torch.int32), q_sep.absmax_offset.view(torch.int32))]:
+        assert torch.equal(x, y)
