@@ -52,6 +52,10 @@ struct GemmParams {
     int tiles_n, tiles_total;
     float* sk_part;   // [gridDim.x][BM*BN] fp32 partial tiles
     int* sk_flags;    // [gridDim.x], zero before the launch
+    // CTA-pair kernel: wait for the previous kernel of the stream only before
+    // the first LoRA k-step (that kernel has itself waited for the block
+    // constants before it let this one launch); 0: before any load
+    int late_wait;
 };
 
 // MT = number of 128-row MMA sub-tiles on the A side (1 or 2).  With MT = 2

@@ -153,8 +153,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairShape<DQ>::THREA
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer (both CTAs)
-        // the block constants and the LoRA operand come from earlier kernels
-        if (lane == 0) pdl_wait();
+        // the block constants and the LoRA operand come from earlier kernels;
+        // with late_wait only the LoRA operand is still being written
+        if (lane == 0 && !p.late_wait) pdl_wait();
+        bool waited = !p.late_wait;
         if (lane == 0 && !p.inject) {
             int last_use[STAGES];
             for (int s = 0; s < STAGES; ++s) last_use[s] = -1;
@@ -167,6 +169,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairShape<DQ>::THREA
                 const int nb0 = sg.tn * 256 + 128 * (int)rank;  // first Bop column of this CTA
                 for (int k = sg.k0; k < sg.k1; ++k, ++it) {
                     const int s = it % STAGES, u = it / STAGES;
+                    if (k >= p.ks_main && !waited) {
+                        pdl_wait();
+                        waited = true;
+                    }
                     if (!mbar_wait(empty(s), (u & 1) ^ 1, wc)) { *abort_flag = 1; ok = false; break; }
                     const uint32_t sA = base + s * S::STAGE_BYTES;
                     const uint32_t sB = sA + S::A_BYTES;
@@ -215,6 +221,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairShape<DQ>::THREA
             for (int s = 0; s < STAGES; ++s)
                 if (last_use[s] >= 0) mbar_wait(full_tma(s), last_use[s] & 1, wc);
         }
+        // the kernel does not complete before the previous one
+        if (lane == 0 && !waited) pdl_wait();
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer (leader)
         if (rank == 0 && lane == 0) {

@@ -23,6 +23,19 @@ struct ProfileScope {
 uint64_t wait_timeout_ns();
 int inject_mode();
 
+// Per-device side stream of the backward: work that does not feed the next
+// kernel of the caller's stream (dA, dB) runs there, beside the dX GEMM, on
+// the SMs that the GEMM's grid leaves idle.  side_stream_acquire returns
+// false (serial path) when the side stream cannot be used: test mode 6, a
+// first use while the caller's stream is capturing, or a failed creation.
+// On true the side-stream lock is held until side_stream_release().
+struct SideStream {
+    cudaStream_t st;
+    cudaEvent_t fork, join;
+};
+bool side_stream_acquire(cudaStream_t s, SideStream* out);
+void side_stream_release();
+
 // ---- quantizer (quantize.cu) ----
 // Host-built search table of the fast nearest-code search (33 buckets of
 // width 1/16 over [-1, 1], see quantize.cu).

@@ -93,35 +93,6 @@ inline cudaError_t launch_gemm(const GemmParams& p, dim3 grid, cudaStream_t s, i
     return cudaGetLastError();
 }
 
-// Launch with programmatic stream serialization (the kernel may start while
-// the previous kernel of the stream finishes; it calls griddepcontrol.wait
-// before touching that kernel's results) and an optional cluster shape.
-template <typename... KArgs, typename... Args>
-inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, int smem, cudaStream_t s,
-                              int cluster_x, Args&&... args) {
-    cudaLaunchConfig_t cfg;
-    memset(&cfg, 0, sizeof(cfg));
-    cfg.gridDim = grid;
-    cfg.blockDim = block;
-    cfg.dynamicSmemBytes = (size_t)smem;
-    cfg.stream = s;
-    cudaLaunchAttribute at[2];
-    int n = 0;
-    at[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    at[n].val.programmaticStreamSerializationAllowed = 1;
-    ++n;
-    if (cluster_x > 0) {
-        at[n].id = cudaLaunchAttributeClusterDimension;
-        at[n].val.clusterDim.x = (unsigned)cluster_x;
-        at[n].val.clusterDim.y = 1;
-        at[n].val.clusterDim.z = 1;
-        ++n;
-    }
-    cfg.attrs = at;
-    cfg.numAttrs = n;
-    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
-}
-
 inline int ceil_div(int64_t a, int64_t b) { return (int)((a + b - 1) / b); }
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
@@ -190,31 +161,58 @@ inline int skinny_active_clusters(int cs) {
 }
 
 template <int BN>
-inline cudaError_t launch_skinny(SkinnyParams& p, int tiles, int kmin, int kmax, cudaStream_t s) {
+inline cudaError_t launch_skinny(SkinnyParams& p, int tiles, int kmin, int kmax, cudaStream_t s, int force_cs) {
     constexpr int smem = SkinnyShape<BN>::SMEM;
     static_assert(smem <= 232448, "shared memory per CTA");
     // Cluster size: fewest rounds of resident clusters times k-steps per CTA
     // (plus a fixed per-CTA cost of about three k-steps), at least one
-    // k-step per CTA of the shorter problem.
+    // k-step per CTA of the shorter problem.  force_cs > 0 fixes it (work
+    // placed beside another kernel, on whatever SMs that one leaves free).
     int cs = 1;
-    int64_t best = -1;
-    for (int c = 8; c >= 1; c >>= 1) {
-        if (c > 1 && kmin < c) continue;
-        const int64_t rounds = ceil_div(tiles, skinny_active_clusters<BN>(c));
-        const int64_t cost = rounds * (ceil_div(kmax, c) + 3);
-        if (best < 0 || cost < best) {
-            best = cost;
-            cs = c;
+    if (force_cs > 0 || p.pack) {
+        cs = 1;
+    } else {
+        int64_t best = -1;
+        for (int c = 8; c >= 1; c >>= 1) {
+            if (c > 1 && kmin < c) continue;
+            const int64_t rounds = ceil_div(tiles, skinny_active_clusters<BN>(c));
+            const int64_t cost = rounds * (ceil_div(kmax, c) + 3);
+            if (best < 0 || cost < best) {
+                best = cost;
+                cs = c;
+            }
         }
     }
     for (int i = 0; i < p.nprob; ++i) p.pr[i].per = ceil_div(p.pr[i].ksteps, cs);
+    p.total_tiles = tiles;
     auto kern = k_skinny<BN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     ProfileScope ps(QLORA_KERNEL_LORA_GEMM, s);
     note_launch();
+    if (p.pack)  // two independent tiles per cluster of 2: one TPC each
+        return launch_pdl(kern, dim3((unsigned)((tiles + 1) & ~1), 1, 1), dim3(SkinnyShape<BN>::THREADS, 1, 1), smem,
+                          s, 2, p);
     return launch_pdl(kern, dim3((unsigned)(tiles * cs), 1, 1), dim3(SkinnyShape<BN>::THREADS, 1, 1), smem, s, cs,
                       p);
+}
+
+template <int BN>
+inline cudaError_t launch_lora_stream(SkinnyParams& p, int tiles, int nctas, cudaStream_t s) {
+    constexpr int smem = StreamShape<BN>::SMEM;
+    static_assert(smem <= 232448, "shared memory per CTA");
+    for (int i = 0; i < p.nprob; ++i) p.pr[i].per = p.pr[i].ksteps;
+    p.total_tiles = tiles;
+    p.pack = 0;
+    auto kern = k_lora_stream<BN>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    ProfileScope ps(QLORA_KERNEL_LORA_GEMM, s);
+    note_launch();
+    // clusters of 2 only for placement (the CTAs are independent): whole
+    // TPCs, never one SM of a TPC that a CTA-pair kernel beside it could use
+    const int grid = (std::max(1, std::min(tiles, nctas)) + 1) & ~1;
+    return launch_pdl(kern, dim3((unsigned)grid, 1, 1), dim3(StreamShape<BN>::THREADS, 1, 1), smem, s, 2, p);
 }
 
 // One skinny problem: operands (tensor maps and majorness), extent and output.
@@ -230,10 +228,28 @@ struct SkinnyDesc {
 
 // wait_first: the operands may have been written by the kernel just before on
 // the stream (or by an unknown earlier one), so the loads wait for it.
-inline qlora_status skinny(const SkinnyDesc* d, int nprob, int r, cudaStream_t s, int wait_first) {
+// place: SKP_SPLIT (cluster size from the cost model, the reduction split
+// across it), SKP_ONE (one CTA per 128-row tile), SKP_PACKED (one CTA per
+// tile, two tiles per TPC: work that leaves whole TPCs to a CTA-pair GEMM
+// beside it), SKP_STREAM (the persistent kernel on nctas CTAs, each taking
+// tiles round-robin: work beside a kernel that holds the other SMs).
+enum { SKP_SPLIT = 0, SKP_ONE = 1, SKP_PACKED = 2, SKP_STREAM = 3 };
+// SKP_STREAM with ctrs (two ints, zero before the launch): tiles taken in
+// problem order from ctrs[0]; problem dep_prob reads problem 0's output.
+// wait_mask (SKP_STREAM with wait_first == 0): problems that read the
+// previous kernel's output, waited for before their first tile.
+inline qlora_status skinny(const SkinnyDesc* d, int nprob, int r, cudaStream_t s, int wait_first,
+                           int place = SKP_SPLIT, int nctas = 0, int* ctrs = nullptr, int dep_prob = -1,
+                           int wait_mask = 0) {
     SkinnyParams p;
     memset(&p, 0, sizeof(p));
     p.wait_first = wait_first;
+    p.pack = place == SKP_PACKED ? 1 : 0;
+    p.tile_ctr = ctrs;
+    p.done_ctr = ctrs ? ctrs + 1 : nullptr;
+    p.dep_prob = ctrs ? dep_prob : -1;
+    p.wait_mask = wait_mask;
+    const int force_cs = place == SKP_ONE ? 1 : 0;
     int tiles = 0, kmin = 1 << 30, kmax = 0;
     for (int i = 0; i < nprob; ++i) {
         tiles += ceil_div(d[i].rows, 128);
@@ -260,12 +276,21 @@ inline qlora_status skinny(const SkinnyDesc* d, int nprob, int r, cudaStream_t s
     p.inject = inject_mode() == 1 ? 1 : 0;
     const int bn = lora_bn(r);
     cudaError_t e;
+    if (place == SKP_STREAM) {
+        if (bn == 64)
+            e = launch_lora_stream<64>(p, tiles, nctas, s);
+        else if (bn == 128)
+            e = launch_lora_stream<128>(p, tiles, nctas, s);
+        else
+            e = launch_lora_stream<256>(p, tiles, nctas, s);
+        return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+    }
     if (bn == 64)
-        e = launch_skinny<64>(p, tiles, kmin, kmax, s);
+        e = launch_skinny<64>(p, tiles, kmin, kmax, s, force_cs);
     else if (bn == 128)
-        e = launch_skinny<128>(p, tiles, kmin, kmax, s);
+        e = launch_skinny<128>(p, tiles, kmin, kmax, s, force_cs);
     else
-        e = launch_skinny<256>(p, tiles, kmin, kmax, s);
+        e = launch_skinny<256>(p, tiles, kmin, kmax, s, force_cs);
     return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
@@ -292,7 +317,7 @@ struct LinearWs {
     float* part;          // small-M partial tiles
     uint32_t* sm_flags;   // small-M partial flags
     float* sk_part;  // stream-K partial tiles [kMaxStreamK][256*256]
-    int* sk_flags;   // [kMaxStreamK]
+    int* sk_flags;   // [kMaxStreamK] stream-K flags, then the 2 tile counters of the backward's side launch
     size_t bytes;
 };
 
@@ -308,7 +333,7 @@ inline LinearWs carve_linear_ws(void* ws, int64_t M, int64_t N, int64_t K, int r
     L.part = big ? nullptr : static_cast<float*>(c.take((size_t)kMaxSmallMCtas * small_m_nt(M) * 128 * 4));
     L.sm_flags = big ? nullptr : static_cast<uint32_t*>(c.take((size_t)kMaxSmallMCtas * 4 * 4));
     L.sk_part = big ? static_cast<float*>(c.take((size_t)kMaxStreamK * 256 * 256 * 4)) : nullptr;
-    L.sk_flags = big ? static_cast<int*>(c.take((size_t)kMaxStreamK * 4)) : nullptr;
+    L.sk_flags = big ? static_cast<int*>(c.take((size_t)(kMaxStreamK + 2) * 4)) : nullptr;
     L.bytes = c.used;
     return L;
 }
@@ -523,14 +548,16 @@ inline qlora_status linear_fwd_impl(const void* X, const LinearArgs& a, const vo
     const qlora_nf4_weight& w = *a.w;
     LinearWs L = carve_linear_ws(ws, a.M, a.N, a.K, a.r, 0);
     if (a.M > kSmallM &&
-        launch_expand_scales(w, L.scales, L.scales_ld, s, L.sk_flags, L.sk_flags ? kMaxStreamK : 0) != cudaSuccess)
+        launch_expand_scales(w, L.scales, L.scales_ld, s, L.sk_flags, L.sk_flags ? kMaxStreamK + 2 : 0) != cudaSuccess)
         return QLORA_ERR_CUDA;
     if (a.r > 0) {
         SkinnyDesc d;
         if (!desc_sU(&d, X, a, A, L.sU)) return QLORA_ERR_CUDA;
-        // after the block-constant expansion (M > 64) the operands are inputs
-        // that no running kernel writes; for small M it is the first kernel
-        qlora_status st = skinny(&d, 1, a.r, s, a.M > kSmallM ? 0 : 1);
+        // M > 64: one CTA per 128-row tile (16 for 2048 tokens), launched
+        // after the block-constant expansion has completed; the pair GEMM
+        // starts beside it on the other SMs and waits for sU only before its
+        // LoRA k-step.  Small M: the cost-model cluster size.
+        qlora_status st = skinny(&d, 1, a.r, s, 1, a.M > kSmallM ? SKP_PACKED : SKP_SPLIT);
         if (st != QLORA_OK) return st;
     }
     GemmParams p;
@@ -564,6 +591,7 @@ inline qlora_status linear_fwd_impl(const void* X, const LinearArgs& a, const vo
         if (large_m_schedule() == SCHED_PAIR || large_m_schedule() == SCHED_PAIR_SK) {
             if (!map_codes(&p.tmCodes, w, 32, 128)) return QLORA_ERR_CUDA;
             if (a.r > 0 && !map_bf16(&p.tmB2, B, a.r, a.N, 128)) return QLORA_ERR_CUDA;
+            p.late_wait = a.r > 0 ? 1 : 0;
             dim3 grid = schedule_pair<DQ_B_K, 4>(p, ceil_div(a.N, 256), ceil_div(a.M, 512), L);
             if (launch_gemm_pair<DQ_B_K, 4>(p, grid, s, QLORA_KERNEL_FWD_GEMM) != cudaSuccess)
                 return QLORA_ERR_CUDA;
@@ -576,6 +604,127 @@ inline qlora_status linear_fwd_impl(const void* X, const LinearArgs& a, const vo
     }
     // small M: Y^T = [W' | B] [X | sU]^T, weight rows on the 128-lane side
     return launch_small_m(X, a, B, Y, L, s);
+}
+
+// sG = bf16(scale dY B): Aop = dY [m][n] (K-major), Bop = B viewed [j][n] (MN-major).
+inline bool desc_sG(SkinnyDesc* d, const CUtensorMap& tdY, const LinearArgs& a, const void* B, void* sG) {
+    memset(d, 0, sizeof(*d));
+    d->tA = tdY;
+    if (!map_bf16(&d->tB, B, a.r, a.N, 64)) return false;
+    d->b_mn = 1;
+    d->rows = (int)a.M;
+    d->ksteps = ceil_div(a.N, 64);
+    d->scale = a.scale;
+    d->out_mode = SK_OUT_BF16;
+    d->out = sG;
+    d->out_ld = a.r;
+    return true;
+}
+
+// dA^T [K][r] = X^T sG : Aop = X viewed [k][m] (MN-major), Bop = sG viewed [j][m] (MN-major)
+// dB [N][r] = dY^T sU : Aop = dY viewed [n][m] (MN-major), Bop = sU viewed [j][m]
+inline bool desc_dA_dB(SkinnyDesc* d, const void* dY, const void* X, const LinearArgs& a, const LinearWs& L,
+                       float* dA, float* dB) {
+    memset(d, 0, 2 * sizeof(*d));
+    if (!map_bf16(&d[0].tA, X, a.K, a.M, 64)) return false;
+    if (!map_bf16(&d[0].tB, L.sG, a.r, a.M, 64)) return false;
+    d[0].rows = (int)a.K;
+    d[0].out_mode = SK_OUT_F32_T;
+    d[0].out = dA;
+    d[0].out_ld = a.K;
+    if (!map_bf16(&d[1].tA, dY, a.N, a.M, 64)) return false;
+    if (!map_bf16(&d[1].tB, L.sU, a.r, a.M, 64)) return false;
+    d[1].rows = (int)a.N;
+    d[1].out_mode = SK_OUT_F32;
+    d[1].out = dB;
+    d[1].out_ld = a.r;
+    for (int i = 0; i < 2; ++i) {
+        d[i].a_mn = 1;
+        d[i].b_mn = 1;
+        d[i].ksteps = ceil_div(a.M, 64);
+        d[i].scale = 1.0f;
+    }
+    return true;
+}
+
+// dX = [dY | sG] [w' ; A] on stream s.  late_wait: the kernel before it on s
+// has waited for the block-constant expansion, only sG is still being written.
+inline qlora_status launch_dx_gemm(const void* A, void* dX, const LinearArgs& a, const LinearWs& L,
+                                   const CUtensorMap& tdY, int late_wait, cudaStream_t s) {
+    const qlora_nf4_weight& w = *a.w;
+    GemmParams p;
+    memset(&p, 0, sizeof(p));
+    p.tmA = tdY;
+    p.tmB = tdY;
+    if (!map_codes(&p.tmCodes, w, 128, 64)) return QLORA_ERR_CUDA;
+    if (a.r > 0) {
+        if (!map_bf16(&p.tmA2, L.sG, a.r, a.M, 128)) return QLORA_ERR_CUDA;
+        if (!map_bf16(&p.tmB2, A, a.K, a.r, 64)) return QLORA_ERR_CUDA;
+    } else {
+        p.tmA2 = tdY;
+        p.tmB2 = tdY;
+    }
+    p.scales = L.scales;
+    p.scales_ld = L.scales_ld;
+    p.dq_rows = (int)a.N;
+    p.dq_kbs = (int)(a.K / 64);
+    p.ks_main = ceil_div(a.N, 64);
+    p.ks_lora = a.r > 0 ? ceil_div(a.r, 64) : 0;
+    p.ks_per_split = p.ks_main;
+    p.rows = (int)a.M;
+    p.cols = (int)a.K;
+    p.out = dX;
+    p.out_ld = a.K;
+    if (!map_bf16(&p.tmOut, dX, a.K, a.M, 128)) return QLORA_ERR_CUDA;
+    p.timeout_ns = wait_timeout_ns();
+    p.inject = inject_mode() == 1 ? 1 : 0;
+    if (large_m_schedule() == SCHED_PAIR || large_m_schedule() == SCHED_PAIR_SK) {
+        if (!map_codes(&p.tmCodes, w, 64, 64)) return QLORA_ERR_CUDA;
+        p.late_wait = late_wait;
+        dim3 grid = schedule_pair<DQ_B_MN, 4>(p, ceil_div(a.K, 256), ceil_div(a.M, 512), L);
+        if (launch_gemm_pair<DQ_B_MN, 4>(p, grid, s, QLORA_KERNEL_DX_GEMM) != cudaSuccess) return QLORA_ERR_CUDA;
+    } else {
+        dim3 grid = schedule_gemm(p, ceil_div(a.K, 256), ceil_div(a.M, 256), L);
+        if (launch_gemm<256, 0, 1, DQ_B_MN, EPI_BF16, 3, 2>(p, grid, s, QLORA_KERNEL_DX_GEMM) != cudaSuccess)
+            return QLORA_ERR_CUDA;
+    }
+    return QLORA_OK;
+}
+
+// The backward forks its adapter GEMMs onto the side stream when the dX GEMM
+// runs on the CTA-pair kernel, one pair per tile.
+inline bool side_fork_ok() { return large_m_schedule() == SCHED_PAIR; }
+
+// Backward with dX and an adapter, on the caller's stream s and the side
+// stream:
+//   s:    expansion -> sG (one CTA per 128-token tile, after the expansion)
+//         -> dX GEMM (starts beside the sG kernel, waits for sG only before
+//         its LoRA k-step) -> wait for the side stream
+//   side: wait for sG -> sU -> dA, dB (one CTA per tile each), on the SMs the
+//         GEMM leaves free
+inline qlora_status linear_bwd_forked(const void* dY, const void* X, const LinearArgs& a, const void* A,
+                                      const void* B, void* dX, float* dA, float* dB, const LinearWs& L,
+                                      const CUtensorMap& tdY, const SideStream& side, cudaStream_t s) {
+    SkinnyDesc dg;
+    if (!desc_sG(&dg, tdY, a, B, L.sG)) return QLORA_ERR_CUDA;
+    qlora_status st = skinny(&dg, 1, a.r, s, 1, SKP_PACKED);
+    if (st != QLORA_OK) return st;
+    if (cudaEventRecord(side.fork, s) != cudaSuccess) return QLORA_ERR_CUDA;
+    if (cudaStreamWaitEvent(side.st, side.fork, 0) != cudaSuccess) return QLORA_ERR_CUDA;
+    // from here on the side stream is joined back whatever happens
+    st = launch_dx_gemm(A, dX, a, L, tdY, 1, s);
+    // sU, dA and dB in one persistent launch over every SM: the CTAs that
+    // find an SM beside the GEMM take tiles from the shared counter while it
+    // runs, the rest start as it ends.  sU tiles (inputs only) start at once,
+    // dA tiles wait for sG (the kernel before), dB tiles for the sU tiles.
+    SkinnyDesc d3[3];
+    if (st == QLORA_OK && !desc_sU(&d3[0], X, a, A, L.sU)) st = QLORA_ERR_CUDA;
+    if (st == QLORA_OK && !desc_dA_dB(d3 + 1, dY, X, a, L, dA, dB)) st = QLORA_ERR_CUDA;
+    if (st == QLORA_OK)
+        st = skinny(d3, 3, a.r, side.st, 0, SKP_STREAM, sm_count(), L.sk_flags + kMaxStreamK, 2, 1 << 1);
+    if (cudaEventRecord(side.join, side.st) != cudaSuccess || cudaStreamWaitEvent(s, side.join, 0) != cudaSuccess)
+        st = QLORA_ERR_CUDA;
+    return st;
 }
 
 inline qlora_status linear_bwd_impl(const void* dY, const void* X, const LinearArgs& a,
@@ -594,91 +743,34 @@ inline qlora_status linear_bwd_impl(const void* dY, const void* X, const LinearA
         }
         return QLORA_OK;
     }
-    if (dX && launch_expand_scales(w, L.scales, L.scales_ld, s, L.sk_flags, kMaxStreamK) != cudaSuccess)
+    if (dX && launch_expand_scales(w, L.scales, L.scales_ld, s, L.sk_flags, kMaxStreamK + 2) != cudaSuccess)
         return QLORA_ERR_CUDA;
     CUtensorMap tdY;
     if (!map_bf16(&tdY, dY, a.N, a.M, 128)) return QLORA_ERR_CUDA;
+    SideStream side{nullptr, nullptr, nullptr};
+    if (dX && a.r > 0 && side_fork_ok() && side_stream_acquire(s, &side)) {
+        const qlora_status st = linear_bwd_forked(dY, X, a, A, B, dX, dA, dB, L, tdY, side, s);
+        side_stream_release();
+        return st;
+    }
+    // serial path: sU and sG in one launch, dX GEMM, dA and dB
     if (a.r > 0) {
-        // sU = bf16(scale X A^T) and sG = bf16(scale dY B) in one launch;
-        // sG: Aop = dY [m][n] (K-major), Bop = B viewed [j][n] (MN-major)
         SkinnyDesc d[2];
         if (!desc_sU(&d[0], X, a, A, L.sU)) return QLORA_ERR_CUDA;
-        memset(&d[1], 0, sizeof(d[1]));
-        d[1].tA = tdY;
-        if (!map_bf16(&d[1].tB, B, a.r, a.N, 64)) return QLORA_ERR_CUDA;
-        d[1].b_mn = 1;
-        d[1].rows = (int)a.M;
-        d[1].ksteps = ceil_div(a.N, 64);
-        d[1].scale = a.scale;
-        d[1].out_mode = SK_OUT_BF16;
-        d[1].out = L.sG;
-        d[1].out_ld = a.r;
-        // inputs only; without dX there is no block-constant expansion before
-        qlora_status st = skinny(d, 2, a.r, s, dX ? 0 : 1);
+        if (!desc_sG(&d[1], tdY, a, B, L.sG)) return QLORA_ERR_CUDA;
+        // waits for the kernel before (the expansion, a dependent launch that
+        // lets this one start early) before it loads: the workspace it writes
+        // may still be read by the call before
+        qlora_status st = skinny(d, 2, a.r, s, 1);
         if (st != QLORA_OK) return st;
     }
     if (dX) {
-        GemmParams p;
-        memset(&p, 0, sizeof(p));
-        p.tmA = tdY;
-        p.tmB = tdY;
-        if (!map_codes(&p.tmCodes, w, 128, 64)) return QLORA_ERR_CUDA;
-        if (a.r > 0) {
-            if (!map_bf16(&p.tmA2, L.sG, a.r, a.M, 128)) return QLORA_ERR_CUDA;
-            if (!map_bf16(&p.tmB2, A, a.K, a.r, 64)) return QLORA_ERR_CUDA;
-        } else {
-            p.tmA2 = tdY;
-            p.tmB2 = tdY;
-        }
-        p.scales = L.scales;
-        p.scales_ld = L.scales_ld;
-        p.dq_rows = (int)a.N;
-        p.dq_kbs = (int)(a.K / 64);
-        p.ks_main = ceil_div(a.N, 64);
-        p.ks_lora = a.r > 0 ? ceil_div(a.r, 64) : 0;
-        p.ks_per_split = p.ks_main;
-        p.rows = (int)a.M;
-        p.cols = (int)a.K;
-        p.out = dX;
-        p.out_ld = a.K;
-        if (!map_bf16(&p.tmOut, dX, a.K, a.M, 128)) return QLORA_ERR_CUDA;
-        p.timeout_ns = wait_timeout_ns();
-        p.inject = inject_mode() == 1 ? 1 : 0;
-        if (large_m_schedule() == SCHED_PAIR || large_m_schedule() == SCHED_PAIR_SK) {
-            if (!map_codes(&p.tmCodes, w, 64, 64)) return QLORA_ERR_CUDA;
-            dim3 grid = schedule_pair<DQ_B_MN, 4>(p, ceil_div(a.K, 256), ceil_div(a.M, 512), L);
-            if (launch_gemm_pair<DQ_B_MN, 4>(p, grid, s, QLORA_KERNEL_DX_GEMM) != cudaSuccess)
-                return QLORA_ERR_CUDA;
-        } else {
-            dim3 grid = schedule_gemm(p, ceil_div(a.K, 256), ceil_div(a.M, 256), L);
-            if (launch_gemm<256, 0, 1, DQ_B_MN, EPI_BF16, 3, 2>(p, grid, s, QLORA_KERNEL_DX_GEMM) != cudaSuccess)
-                return QLORA_ERR_CUDA;
-        }
+        qlora_status st = launch_dx_gemm(A, dX, a, L, tdY, 0, s);
+        if (st != QLORA_OK) return st;
     }
     if (a.r > 0) {
-        // dA^T [K][r] = X^T sG : Aop = X viewed [k][m] (MN-major), Bop = sG viewed [j][m] (MN-major)
-        // dB [N][r] = dY^T sU : Aop = dY viewed [n][m] (MN-major), Bop = sU viewed [j][m]
-        // (both in one launch)
         SkinnyDesc d[2];
-        memset(d, 0, sizeof(d));
-        if (!map_bf16(&d[0].tA, X, a.K, a.M, 64)) return QLORA_ERR_CUDA;
-        if (!map_bf16(&d[0].tB, L.sG, a.r, a.M, 64)) return QLORA_ERR_CUDA;
-        d[0].rows = (int)a.K;
-        d[0].out_mode = SK_OUT_F32_T;
-        d[0].out = dA;
-        d[0].out_ld = a.K;
-        if (!map_bf16(&d[1].tA, dY, a.N, a.M, 64)) return QLORA_ERR_CUDA;
-        if (!map_bf16(&d[1].tB, L.sU, a.r, a.M, 64)) return QLORA_ERR_CUDA;
-        d[1].rows = (int)a.N;
-        d[1].out_mode = SK_OUT_F32;
-        d[1].out = dB;
-        d[1].out_ld = a.r;
-        for (int i = 0; i < 2; ++i) {
-            d[i].a_mn = 1;
-            d[i].b_mn = 1;
-            d[i].ksteps = ceil_div(a.M, 64);
-            d[i].scale = 1.0f;
-        }
+        if (!desc_dA_dB(d, dY, X, a, L, dA, dB)) return QLORA_ERR_CUDA;
         // sG and sU come from the LoRA GEMMs above
         qlora_status st = skinny(d, 2, a.r, s, 1);
         if (st != QLORA_OK) return st;

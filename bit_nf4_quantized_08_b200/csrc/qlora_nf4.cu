@@ -62,6 +62,51 @@ ProfileScope::~ProfileScope() {
 uint64_t wait_timeout_ns() { return g_timeout_ns.load(); }
 int inject_mode() { return g_inject.load(); }
 
+static std::mutex g_side_mu;
+struct SideSlot {
+    bool tried;
+    SideStream ss;
+};
+static SideSlot g_side[64];
+
+bool side_stream_acquire(cudaStream_t s, SideStream* out) {
+    if (inject_mode() == 6) return false;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        cudaGetLastError();
+        return false;
+    }
+    g_side_mu.lock();
+    SideSlot& slot = g_side[dev];
+    if (!slot.tried) {
+        // streams and events are not created inside a stream capture
+        cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+        if (cudaStreamIsCapturing(s, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone) {
+            cudaGetLastError();
+            g_side_mu.unlock();
+            return false;
+        }
+        slot.tried = true;
+        SideStream ss{nullptr, nullptr, nullptr};
+        if (cudaStreamCreateWithFlags(&ss.st, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) == cudaSuccess &&
+            cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) == cudaSuccess) {
+            slot.ss = ss;
+        } else {
+            cudaGetLastError();
+            slot.ss = SideStream{nullptr, nullptr, nullptr};
+        }
+    }
+    if (!slot.ss.st) {
+        g_side_mu.unlock();
+        return false;
+    }
+    *out = slot.ss;
+    return true;
+}
+
+void side_stream_release() { g_side_mu.unlock(); }
+
 static bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 static const int64_t kMaxElems = (int64_t)1 << 40;

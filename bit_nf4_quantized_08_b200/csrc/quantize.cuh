@@ -422,8 +422,11 @@ __global__ void k_expand_scales(int64_t rows, int64_t kbs, int dq, const float* 
                                 const uint8_t* __restrict__ q8, const float* __restrict__ c1,
                                 const float* __restrict__ offset_ptr, float* __restrict__ scales,
                                 int64_t ld, int* __restrict__ flags, int nflags) {
-    // the LoRA GEMM that follows reads none of this kernel's outputs
+    // the LoRA GEMM that follows reads none of this kernel's outputs; this
+    // kernel's inputs (8-bit constants) and outputs (scales, flags of the
+    // GEMM before) belong to the kernel before it
     pdl_trigger();
+    pdl_wait();
     const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (idx < nflags) flags[idx] = 0;
     if (idx >= rows * kbs) return;
@@ -545,10 +548,11 @@ inline cudaError_t launch_expand_scales(const qlora_nf4_weight& w, float* scales
     const int64_t total = w.rows * kbs > nflags ? w.rows * kbs : nflags;
     if (total == 0) return cudaSuccess;
     note_launch();
-    k_expand_scales<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(
-        w.rows, kbs, w.double_quant, w.absmax, w.absmax_q8, w.absmax_scale, w.absmax_offset,
-        scales, ld, flags, nflags);
-    return cudaGetLastError();
+    // dependent launch: the CTAs can be resident before the kernel ahead
+    // ends and wait for it (pdl_wait) before any access
+    return launch_pdl(k_expand_scales, dim3((unsigned)((total + 255) / 256)), dim3(256), 0, s, 0, w.rows, kbs,
+                      (int)w.double_quant, (const float*)w.absmax, (const uint8_t*)w.absmax_q8,
+                      (const float*)w.absmax_scale, (const float*)w.absmax_offset, scales, ld, flags, nflags);
 }
 
 inline cudaError_t launch_encode(const float* x, int64_t n, uint8_t* codes, cudaStream_t s) {

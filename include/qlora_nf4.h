@@ -182,6 +182,13 @@ qlora_status qlora_linear_fwd(const void *X, int64_t M, const qlora_nf4_weight *
  *   only dX is produced.  With M == 0, dA and dB are set to zero.
  * Same shape requirements as qlora_linear_fwd.  Deterministic (no floating
  * point atomics on any output).
+ * Streams: all work is ordered on `stream`.  With dX and r > 0 the dA/dB
+ * GEMMs run on a per-device side stream of the library that waits for
+ * `stream` first, beside the dX GEMM, and `stream` waits for them before the
+ * call returns, so to the caller the call is one ordered step on `stream`
+ * (also inside a stream capture, once the side stream exists: it is created
+ * by the first such call made outside a capture).  Calls from several host
+ * threads are serialized on that side stream.
  */
 qlora_status qlora_linear_bwd(const void *dY, const void *X, int64_t M, const qlora_nf4_weight *w,
                               const void *A, const void *B, int32_t r, float scale, void *dX,
@@ -223,9 +230,11 @@ void qlora_set_wait_timeout_ns(uint64_t ns);
  * split-tile merge); mode 3 on the single-CTA kernel with one CTA per tile;
  * mode 4 on the CTA-pair kernel with the stream-K schedule over 4 pairs;
  * mode 5 forms the double-quantization offset in its own kernel even for
- * tensors whose 8-bit pass would form it itself.
- * Mode 0: normal (CTA-pair kernel; one pair per tile, or stream-K over all
- * resident pairs when the tiles would leave a partly idle last round).
+ * tensors whose 8-bit pass would form it itself; mode 6 runs the backward's
+ * dA and dB GEMMs on the caller's stream after the dX GEMM instead of beside
+ * it on the library's side stream.
+ * Mode 0: normal (CTA-pair kernel, one pair per tile; in the backward the
+ * dA/dB GEMMs beside the dX GEMM on the side stream).
  */
 void qlora_debug_inject(int32_t mode);
 

@@ -85,6 +85,99 @@ def test_bwd_parity(Q, O, cuda, M, N, K, r):
         assert_close_tol(dB.cpu().numpy(), rdB, "dB")
 
 
+def test_bwd_serial_path_matches(Q, O, cuda):
+    """The serial backward (test mode 6: sU and sG in one split-K launch, dX
+    GEMM, then dA and dB) and the default one (sG alone, dX GEMM beside it,
+    sU, dA and dB on the side stream) both match the oracle.  The two sum sG
+    in different orders, so they are not bitwise equal."""
+    M, N, K, r = 1100, 1280, 1024, 32
+    q, inp, Wd_ref = _setup(Q, O, M, N, K, r, seed=12, b_std=0.05)
+    X, dY, A, B = (inp[k].cuda() for k in ("X", "dY", "A", "B"))
+    s = 2.0
+    Q.qlora_debug_inject(6)
+    try:
+        serial = Q.qlora_linear_bwd(dY, X, q, A, B, s)
+        assert Q.qlora_get_last_error() == 0
+    finally:
+        Q.qlora_debug_inject(0)
+    forked = Q.qlora_linear_bwd(dY, X, q, A, B, s)
+    assert Q.qlora_get_last_error() == 0
+    rdX, rdA, rdB = O.linear_bwd(wl.bits(inp["dY"]), wl.bits(inp["X"]), Wd_ref, wl.bits(inp["A"]),
+                                 wl.bits(inp["B"]), s)
+    for tag, g in (("serial", serial), ("side stream", forked)):
+        assert_close_tol(g[0].float().cpu().numpy(), rdX, f"dX {tag}")
+        assert_close_tol(g[1].cpu().numpy(), rdA, f"dA {tag}")
+        assert_close_tol(g[2].cpu().numpy(), rdB, f"dB {tag}")
+
+
+@pytest.mark.parametrize("mode", [0, 6], ids=["side_stream", "serial"])
+def test_back_to_back_calls_share_workspace(Q, O, cuda, mode):
+    """Forward and backward calls of two layers issued back to back on one
+    stream with one workspace (the kernels of a call may start while the
+    call before finishes) give bitwise the results of the same calls run
+    one at a time with their own workspaces."""
+    shapes = [(600, 1024, 512, 32), (600, 512, 1024, 32)]
+    layers = []
+    for i, (M, N, K, r) in enumerate(shapes):
+        q, inp, _ = _setup(Q, O, M, N, K, r, seed=40 + i, b_std=0.05)
+        layers.append((q, {k: v.cuda() for k, v in inp.items()}))
+    ws_bytes = max(max(Q.qlora_linear_workspace(M, q, r, True), Q.qlora_linear_workspace(M, q, r, False))
+                   for (M, N, K, r), (q, _) in zip(shapes, layers))
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    Q.qlora_debug_inject(mode)
+    try:
+        chained = []
+        for q, t in layers:
+            chained.append(Q.qlora_linear_fwd(t["X"], q, t["A"], t["B"], 2.0, ws=ws))
+        for q, t in reversed(layers):
+            chained.extend(Q.qlora_linear_bwd(t["dY"], t["X"], q, t["A"], t["B"], 2.0, ws=ws))
+        torch.cuda.synchronize()
+        single = []
+        for q, t in layers:
+            single.append(Q.qlora_linear_fwd(t["X"], q, t["A"], t["B"], 2.0))
+            torch.cuda.synchronize()
+        for q, t in reversed(layers):
+            single.extend(Q.qlora_linear_bwd(t["dY"], t["X"], q, t["A"], t["B"], 2.0))
+            torch.cuda.synchronize()
+        assert Q.qlora_get_last_error() == 0
+    finally:
+        Q.qlora_debug_inject(0)
+    for i, (a_, b_) in enumerate(zip(chained, single)):
+        assert torch.equal(a_.view(torch.int32 if a_.dtype == torch.float32 else torch.int16),
+                           b_.view(torch.int32 if b_.dtype == torch.float32 else torch.int16)), f"output {i}"
+
+
+def test_bwd_graph_replay(Q, O, cuda):
+    """The backward captured in a CUDA graph, with dA and dB forked onto the
+    side stream and joined back inside the capture, replayed on new inputs:
+    every replay is bitwise equal to the eager call on the same inputs."""
+    M, N, K, r = 600, 1024, 512, 64
+    q, inp, _ = _setup(Q, O, M, N, K, r, seed=13, b_std=0.05)
+    X, dY, A, B = (inp[k].cuda() for k in ("X", "dY", "A", "B"))
+    dX = torch.empty(M, K, dtype=torch.bfloat16, device="cuda")
+    dA = torch.empty(r, K, dtype=torch.float32, device="cuda")
+    dB = torch.empty(N, r, dtype=torch.float32, device="cuda")
+    ws = torch.empty(Q.qlora_linear_workspace(M, q, r, True), dtype=torch.uint8, device="cuda")
+    Q.qlora_linear_bwd(dY, X, q, A, B, 2.0, dX=dX, dA=dA, dB=dB, ws=ws)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        Q.qlora_linear_bwd(dY, X, q, A, B, 2.0, dX=dX, dA=dA, dB=dB, ws=ws)
+    for rep in range(3):
+        new = wl.linear_inputs(M, N, K, r, seed=30 + rep)
+        X.copy_(new["X"].cuda())
+        dY.copy_(new["dY"].cuda())
+        g.replay()
+        torch.cuda.synchronize()
+        got = [t.clone() for t in (dX, dA, dB)]
+        ref = Q.qlora_linear_bwd(dY, X, q, A, B, 2.0)
+        torch.cuda.synchronize()
+        for a_, b_ in zip(got, ref):
+            assert torch.equal(a_.view(torch.int32 if a_.dtype == torch.float32 else torch.int16),
+                               b_.view(torch.int32 if b_.dtype == torch.float32 else torch.int16)), f"replay {rep}"
+    assert Q.qlora_get_last_error() == 0
+
+
 @pytest.mark.parametrize("M", [5, 300])
 def test_zero_B_is_noop(Q, O, cuda, M):
     """Reproduction blog invariant: B = 0 at step 0 gives the frozen base
