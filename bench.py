@@ -197,15 +197,19 @@ class Block:
             + (2 * M * L["K"] + 2 * M * L["N"] + 4 * M * r + 4 * r * L["K"] + 4 * L["N"] * r)
             for L in self.layers)
 
-    def step(self):
+    def step(self, adapter=True):
         Q, ws = self.Q, self.ws
         for L in self.layers:
             Q.qlora_nf4_quantize(L["W"], True, out=L["w"], ws=ws)
         for L in self.layers:
-            Q.qlora_linear_fwd(L["X"], L["w"], L["A"], L["B"], self.s, Y=L["Y"], ws=ws)
+            A, B = (L["A"], L["B"]) if adapter else (None, None)
+            Q.qlora_linear_fwd(L["X"], L["w"], A, B, self.s, Y=L["Y"], ws=ws)
         for L in reversed(self.layers):
-            Q.qlora_linear_bwd(L["dY"], L["X"], L["w"], L["A"], L["B"], self.s, dX=L["dX"], dA=L["dA"],
-                               dB=L["dB"], ws=ws)
+            if adapter:
+                Q.qlora_linear_bwd(L["dY"], L["X"], L["w"], L["A"], L["B"], self.s, dX=L["dX"], dA=L["dA"],
+                                   dB=L["dB"], ws=ws)
+            else:
+                Q.qlora_linear_bwd(L["dY"], L["X"], L["w"], None, None, self.s, dX=L["dX"], ws=ws)
 
 
 def max_over_ranks(torch, value, world, device):
@@ -419,6 +423,16 @@ def main():
     launches = launches_per_step * args.steps
     status = Q.qlora_get_last_error()
     assert status == 0, f"device status {status}"
+    # the same step without the adapter (r = 0), also a graph replay: the
+    # difference is the step time the LoRA GEMMs still add
+    base_graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(base_graph):
+        blk.step(adapter=False)
+    base_graph.replay()
+    torch.cuda.synchronize()
+    base_ms = max_over_ranks(torch, sum(time_steps(torch, base_graph.replay, args.steps, flush, barrier)),
+                             world, device) / args.steps
+    del base_graph
     # per-kernel device times from a separate eager pass with launch events
     Q.qlora_profile_enable(True)
     time_steps(torch, blk.step, args.steps, flush, barrier)
@@ -448,9 +462,13 @@ def main():
         breakdown["quantize_frac_hbm"] = round(breakdown["quantize_GBps"] / peaks["hbm_gbs"], 3)
     lms, ln = prof["lora_gemm"]
     if ln:
+        # event times of kernels that run beside the dequant GEMMs (dependent
+        # launch, side stream): their sum overlaps the GEMMs' times
         breakdown["lora_gemm_GBps"] = round(blk.lora_bytes * args.steps / (lms * 1e-3) / 1e9, 1)
         breakdown["lora_gemm_frac_hbm"] = round(breakdown["lora_gemm_GBps"] / peaks["hbm_gbs"], 3)
-        breakdown["lora_gemm_share_of_step"] = round(lms / total_ms, 3)
+        breakdown["lora_gemm_overlapped_share"] = round(lms / total_ms, 3)
+    breakdown["step_ms_without_adapter"] = round(base_ms, 4)
+    breakdown["adapter_added_ms"] = round(ms_per_step - base_ms, 4)
     for k in ("fwd_gemm", "dx_gemm"):
         ms_k, n_k = prof[k]
         fl = (blk.fwd_gemm_flops if k == "fwd_gemm" else blk.dx_gemm_flops) * args.steps

@@ -36,9 +36,11 @@ struct SideStream {
 bool side_stream_acquire(cudaStream_t s, SideStream* out);
 void side_stream_release();
 
-// ---- quantizer (quantize.cu) ----
+// ---- quantizer (quantize.cuh) ----
 // Host-built search table of the fast nearest-code search (33 buckets of
-// width 1/16 over [-1, 1], see quantize.cu).
+// width 1/16 over [-1, 1], see quantize.cuh): per bucket the largest fp32
+// below its decision threshold (3.0 without one) and the count of
+// thresholds below the bucket.
 struct Nf4SearchTable {
     float thr[33];
     int base[33];

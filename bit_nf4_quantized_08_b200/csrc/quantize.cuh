@@ -41,11 +41,14 @@ namespace qlora {
 // each holds at most one threshold T_key; base_key counts the thresholds at
 // or below the bucket's lower edge.  code(x) = base_key + (x >= T_key), where
 // threshold j is the smallest fp32 strictly above the exact midpoint of codes
-// j and j+1 (so an exact tie stays with the lower code).  The tables have 64
-// entries and the key is masked to 6 bits, so any input (NaN included) reads
-// inside them.
+// j and j+1 (so an exact tie stays with the lower code).  The table holds
+// P_key, the largest fp32 below T_key: x >= T_key exactly when x > P_key,
+// i.e. when fl(P_key - x) is negative (a difference of two finite floats is
+// zero only when they are equal), so the compare is one FADD and the sign
+// bit.  The tables have 64 entries and the key is masked to 6 bits, so any
+// input (NaN included) reads inside them.
 struct SearchSmem {
-    float thr[64];
+    float thr[64];  // P_key
     int base[64];
 };
 
@@ -56,10 +59,48 @@ __device__ __forceinline__ void load_search_tables(SearchSmem& st, const Nf4Sear
     }
 }
 
+// t = fl(16 x + 1.5 * 2^23 + 16): x rounded to an integer bucket key in the
+// low mantissa bits (0x4B400000 + key).
+__device__ __forceinline__ uint32_t nf4_lookup(float x, float t, const SearchSmem& st) {
+    const uint32_t key = __float_as_uint(t) & 63u;
+    return (uint32_t)st.base[key] + (__float_as_uint(__fsub_rn(st.thr[key], x)) >> 31);
+}
+
 __device__ __forceinline__ uint32_t nf4_search(float x, const SearchSmem& st) {
-    const float t = fmaf(x, 16.0f, 12582928.0f);  // 1.5 * 2^23 + 16: RN to an integer
-    const uint32_t key = __float_as_uint(t) & 63u;  // low bits of 0x4B400000 + key
-    return (uint32_t)st.base[key] + (x >= st.thr[key] ? 1u : 0u);
+    return nf4_lookup(x, fmaf(x, 16.0f, 12582928.0f), st);
+}
+
+// Two lanes of fp32x2 arithmetic (sm_100a packed FP32): the same IEEE
+// round-to-nearest products and fused multiply-adds as the scalar forms.
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t r, float& a, float& b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+// Codes of two elements x = fl(w * rcp) in one fp32x2 multiply and FMA.
+__device__ __forceinline__ void nf4_search2(float w0, float w1, uint64_t rcp2, const SearchSmem& st, uint32_t& c0,
+                                            uint32_t& c1) {
+    const uint64_t x2 = f2_mul(f2_pack(w0, w1), rcp2);
+    const uint64_t t2 = f2_fma(x2, f2_pack(16.0f, 16.0f), f2_pack(12582928.0f, 12582928.0f));
+    float x0, x1, t0, t1;
+    f2_unpack(x2, x0, x1);
+    f2_unpack(t2, t0, t1);
+    c0 = nf4_lookup(x0, t0, st);
+    c1 = nf4_lookup(x1, t1, st);
 }
 
 // Pack 8 codes (element order) into one word: byte i = (c[2i] << 4) | c[2i+1].
@@ -134,9 +175,13 @@ __global__ void __launch_bounds__(256, BF16 ? 4 : 2) k_quantize_blocks(const voi
         // block absmax (exact: a max of magnitudes)
         float a;
         if (BF16) {
-            uint32_t m = 0;
+            // packed bf16 max of magnitudes (the sign of each half is the xor
+            // of the signs, dropped at the end)
+            uint32_t m = raw[it][0];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) m = __vmaxu2(m, raw[it][i] & 0x7FFF7FFFu);
+            for (int i = 1; i < 8; ++i)
+                asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(m) : "r"(raw[it][i]));
+            m &= 0x7FFF7FFFu;
             m = max(m & 0xFFFFu, m >> 16);
             a = __uint_as_float(m << 16);
         } else {
@@ -154,11 +199,12 @@ __global__ void __launch_bounds__(256, BF16 ? 4 : 2) k_quantize_blocks(const voi
         uint32_t c[16];
         if (a >= 1.17549435e-38f) {
             const float rcp = __frcp_rn(a);
+            const uint64_t rcp2 = f2_pack(rcp, rcp);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const uint32_t bits = BF16 ? ((i & 1) ? (raw[it][i >> 1] & 0xFFFF0000u) : (raw[it][i >> 1] << 16))
-                                           : raw[it][i];
-                c[i] = nf4_search(__fmul_rn(__uint_as_float(bits), rcp), st);
+            for (int i = 0; i < 16; i += 2) {
+                const uint32_t b0 = BF16 ? (raw[it][i >> 1] << 16) : raw[it][i];
+                const uint32_t b1 = BF16 ? (raw[it][i >> 1] & 0xFFFF0000u) : raw[it][i + 1];
+                nf4_search2(__uint_as_float(b0), __uint_as_float(b1), rcp2, st, c[i], c[i + 1]);
             }
         } else {
             // zero or subnormal block: exact power-of-two prescale 2^64
@@ -182,10 +228,13 @@ __global__ void __launch_bounds__(256, BF16 ? 4 : 2) k_quantize_blocks(const voi
             __stcs(reinterpret_cast<uint2*>(codes + (e0[it] >> 1)), make_uint2(w0, w1));
         } else if (e0[it] < n) {
             const int valid = (int)(n - e0[it]);
-            for (int j = 0; 2 * j < valid; ++j) {
-                uint32_t byte = c[2 * j] << 4;
-                if (2 * j + 1 < valid) byte |= c[2 * j + 1];
-                codes[(e0[it] >> 1) + j] = (uint8_t)byte;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {  // static indices: c stays in registers
+                if (2 * j < valid) {
+                    uint32_t byte = c[2 * j] << 4;
+                    if (2 * j + 1 < valid) byte |= c[2 * j + 1];
+                    codes[(e0[it] >> 1) + j] = (uint8_t)byte;
+                }
             }
         }
 
@@ -477,7 +526,7 @@ inline Nf4SearchTable build_search_table() {
             if ((double)thr[j] <= lo) ++base;
             else if ((double)thr[j] <= hi) tk = thr[j];
         }
-        t.thr[k] = tk;
+        t.thr[k] = std::nextafter(tk, -INFINITY);  // P_key: x >= T_key  <=>  x > P_key
         t.base[k] = base;
     }
     return t;
