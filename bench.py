@@ -450,7 +450,7 @@ def main():
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops"]
     traffic = load_traffic(dom)
-    roofline = {"bound": "tensor", "kernel": f"k_gemm ({dom.replace('_', ' ')}, NF4 dequant in producer)",
+    roofline = {"bound": "tensor", "kernel": f"k_gemm_pair ({dom.replace('_', ' ')}, NF4 dequant in producer)",
                 "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                 "frac": round(achieved / peak, 4), "traffic": traffic,
                 "peak_source": f"{peak_src} bf16 dense (burst)",
