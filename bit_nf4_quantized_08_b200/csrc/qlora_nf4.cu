@@ -131,11 +131,13 @@ static qlora_status check_weight(const qlora_nf4_weight* w, bool need_codes) {
     return QLORA_OK;
 }
 
+// Workspace of qlora_nf4_quantize with double quantization: block maxima
+// [nb] f32, group sums [ng] f64, first-level offset partials (many groups).
 static size_t quantize_ws(int64_t n, int dq) {
     if (!dq || n == 0) return 0;
     const int64_t nb = (n + 63) / 64;
     const int64_t ng = (n + 16383) / 16384;
-    return align256((size_t)nb * 4) + align256((size_t)ng * 8);
+    return align256((size_t)nb * 4) + align256((size_t)ng * 8) + align256((size_t)dq_partial_count(ng) * 8);
 }
 
 // Scratch of qlora_nf4_quantize_static: the fp32 maximum of every 64-element
@@ -216,10 +218,11 @@ qlora_status qlora_nf4_quantize(const void* W, qlora_dtype wdtype, const qlora_n
     float* absmax = static_cast<float*>(ws);
     double* sums = reinterpret_cast<double*>(static_cast<char*>(ws) + align256((size_t)nb * 4));
     const int64_t ng = (n + 16383) / 16384;
+    double* partials = reinterpret_cast<double*>(reinterpret_cast<char*>(sums) + align256((size_t)ng * 8));
     if (launch_quantize_blocks(W, is_bf16, n, out->codes, absmax, sums, s) != cudaSuccess)
         return QLORA_ERR_CUDA;
-    if (launch_double_quant(sums, ng, absmax, nb, out->absmax_offset, out->absmax_q8, out->absmax_scale, s) !=
-        cudaSuccess)
+    if (launch_double_quant(sums, ng, absmax, nb, out->absmax_offset, out->absmax_q8, out->absmax_scale, s,
+                            partials) != cudaSuccess)
         return QLORA_ERR_CUDA;
     return QLORA_OK;
 }

@@ -23,6 +23,7 @@
 
 #include <cuda_bf16.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 
@@ -118,13 +119,19 @@ __device__ __forceinline__ uint32_t pack8(const uint32_t (&c)[8]) {
 // pairwise-tree sum of block maxima for the double-quantization offset.
 // ---------------------------------------------------------------------------
 template <bool BF16>
-__global__ void __launch_bounds__(256, BF16 ? 4 : 2) k_quantize_blocks(const void* __restrict__ W, int64_t n,
-                                                            uint8_t* __restrict__ codes,
-                                                            float* __restrict__ absmax,
-                                                            double* __restrict__ group_sums,
+__global__ void __launch_bounds__(256, BF16 ? 4 : 2) k_quantize_blocks(const void* W, int64_t n,
+                                                            uint8_t* codes,
+                                                            float* absmax,
+                                                            double* group_sums,
                                                             Nf4SearchTable tab) {
     __shared__ SearchSmem st;
     __shared__ double s_wsum[8];
+    // dependent launch: resident before the kernel ahead ends, no access to
+    // memory before it has.  The kernels that wait this way take no
+    // __restrict__ pointers: with them the compiler may move loads of
+    // "unchanging" data above griddepcontrol.wait.
+    pdl_trigger();
+    pdl_wait();
     load_search_tables(st, tab);
     __syncthreads();
 
@@ -257,23 +264,29 @@ __global__ void __launch_bounds__(256, BF16 ? 4 : 2) k_quantize_blocks(const voi
     }
 }
 
-// ---------------------------------------------------------------------------
-// K2: offset = fl32(S / nb), S = pairwise tree over the group sums padded
-// with zeros to a power of two.  One CTA of 1024 threads; thread t sums a
-// contiguous power-of-two chunk with a binary-counter pairwise sum.
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(1024) k_dq_offset(const double* __restrict__ sums, int64_t ng,
-                                                    int64_t nb, float* __restrict__ offset) {
-    __shared__ double s_w[32];
-    int64_t p2 = 1;
-    while (p2 < ng) p2 <<= 1;
-    const int64_t chunk = p2 > 1024 ? p2 / 1024 : 1;
+// fp64 pairwise-tree sum of x[lo, lo + chunk) (chunk a power of two; entries
+// at or past n count as 0) with a binary-counter stack.  From chunk >= 8 on,
+// eight independent loads at a time are folded as a fixed subtree first: the
+// same tree, with an eighth of the dependent memory round trips.
+__device__ __forceinline__ double pairwise_chunk(const double* x, int64_t lo, int64_t chunk,
+                                                 int64_t n) {
     double stack[40];
     int64_t cnt = 0;
-    const int64_t lo = (int64_t)threadIdx.x * chunk;
-    for (int64_t i = 0; i < chunk; ++i) {
-        int64_t idx = lo + i;
-        double v = idx < ng ? sums[idx] : 0.0;
+    const int step = chunk >= 8 ? 8 : 1;
+    for (int64_t i = 0; i < chunk; i += step) {
+        double v;
+        if (step == 8) {
+            double e[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int64_t idx = lo + i + j;
+                e[j] = idx < n ? x[idx] : 0.0;
+            }
+            v = ((e[0] + e[1]) + (e[2] + e[3])) + ((e[4] + e[5]) + (e[6] + e[7]));
+        } else {
+            const int64_t idx = lo + i;
+            v = idx < n ? x[idx] : 0.0;
+        }
         int lvl = 0;
         while ((cnt >> lvl) & 1) {
             v = stack[lvl] + v;
@@ -283,8 +296,24 @@ __global__ void __launch_bounds__(1024) k_dq_offset(const double* __restrict__ s
         ++cnt;
     }
     int top = 0;
-    while ((1ll << top) < chunk) ++top;
-    double t = stack[top];
+    while ((1ll << top) < cnt) ++top;
+    return stack[top];
+}
+
+// ---------------------------------------------------------------------------
+// K2: offset = fl32(S / nb), S = pairwise tree over the group sums padded
+// with zeros to a power of two.  One CTA of 1024 threads; thread t sums a
+// contiguous power-of-two chunk with a binary-counter pairwise sum.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024) k_dq_offset(const double* sums, int64_t ng,
+                                                    int64_t nb, float* offset) {
+    __shared__ double s_w[32];
+    pdl_trigger();
+    pdl_wait();
+    int64_t p2 = 1;
+    while (p2 < ng) p2 <<= 1;
+    const int64_t chunk = p2 > 1024 ? p2 / 1024 : 1;
+    double t = pairwise_chunk(sums, (int64_t)threadIdx.x * chunk, chunk, ng);
     for (int o = 1; o < 32; o <<= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
     if ((threadIdx.x & 31) == 0) s_w[threadIdx.x >> 5] = t;
     __syncthreads();
@@ -293,6 +322,25 @@ __global__ void __launch_bounds__(1024) k_dq_offset(const double* __restrict__ s
         for (int o = 1; o < 32; o <<= 1) u += __shfl_xor_sync(0xffffffffu, u, o);
         if (threadIdx.x == 0) *offset = __double2float_rn(__ddiv_rn(u, (double)nb));
     }
+}
+
+// First level of the offset tree for many group sums: CTA c sums leaves
+// [4096 c, 4096 c + 4096) of the zero-padded power-of-two leaf array, an
+// aligned subtree of the same pairwise tree (16 leaves per thread, then the
+// warp and CTA levels in the same pairing), so that a tree over the partials
+// gives the same total as one over all sums.
+constexpr int64_t kPartialLeaves = 4096;
+__global__ void __launch_bounds__(256) k_dq_partials(const double* sums, int64_t ng,
+                                                     double* partials) {
+    __shared__ double s_w[8];
+    pdl_trigger();
+    pdl_wait();
+    double t = pairwise_chunk(sums, (int64_t)blockIdx.x * kPartialLeaves + (int64_t)threadIdx.x * 16, 16, ng);
+    for (int o = 1; o < 32; o <<= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    if ((threadIdx.x & 31) == 0) s_w[threadIdx.x >> 5] = t;
+    __syncthreads();
+    if (threadIdx.x == 0)
+        partials[blockIdx.x] = ((s_w[0] + s_w[1]) + (s_w[2] + s_w[3])) + ((s_w[4] + s_w[5]) + (s_w[6] + s_w[7]));
 }
 
 // Nearest 8-bit code of y in [-1, 1]: candidate from rint(127 y), then the
@@ -323,36 +371,31 @@ __device__ __forceinline__ int nearest_t8(float y, const float* t8) {
 // With sums != nullptr every CTA first forms the offset itself from the
 // nsums group sums (the same pairwise tree as K2, over 256 threads) and CTA 0
 // also stores it; otherwise the offset is read from offset_ptr.
-__global__ void __launch_bounds__(256) k_dq_quantize(const float* __restrict__ absmax, int64_t nb,
-                                                     float* __restrict__ offset_ptr,
-                                                     uint8_t* __restrict__ q8,
-                                                     float* __restrict__ c1,
-                                                     const double* __restrict__ sums, int64_t nsums) {
+__global__ void __launch_bounds__(256) k_dq_quantize(const float* absmax, int64_t nb,
+                                                     float* offset_ptr,
+                                                     uint8_t* q8,
+                                                     float* c1,
+                                                     const double* sums, int64_t nsums) {
     __shared__ float t8[256];
     __shared__ double s_w[8];
     __shared__ float s_off;
-    t8[threadIdx.x] = t8_value(threadIdx.x);  // blockDim.x == 256
+    pdl_trigger();
+    t8[threadIdx.x] = t8_value(threadIdx.x);  // blockDim.x == 256; shared memory only
+    pdl_wait();
+    // this warp's first group: 8 block maxima per lane, loaded before the
+    // offset tree so that the two memory round trips overlap
+    const int64_t g = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    const int64_t ng = (nb + 255) >> 8;
+    const int64_t bf = g * 256 + lane * 8;
+    float am[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) am[i] = (g < ng && bf + i < nb) ? absmax[bf + i] : 0.0f;
     if (sums) {
         int64_t p2 = 1;
         while (p2 < nsums) p2 <<= 1;
         const int64_t chunk = p2 > 256 ? p2 / 256 : 1;
-        double stack[40];
-        int64_t cnt = 0;
-        const int64_t lo = (int64_t)threadIdx.x * chunk;
-        for (int64_t i = 0; i < chunk; ++i) {
-            const int64_t idx = lo + i;
-            double v = idx < nsums ? sums[idx] : 0.0;
-            int lvl = 0;
-            while ((cnt >> lvl) & 1) {
-                v = stack[lvl] + v;
-                ++lvl;
-            }
-            stack[lvl] = v;
-            ++cnt;
-        }
-        int top = 0;
-        while ((1ll << top) < chunk) ++top;
-        double t = stack[top];
+        double t = pairwise_chunk(sums, (int64_t)threadIdx.x * chunk, chunk, nsums);
         for (int o = 1; o < 32; o <<= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
         if ((threadIdx.x & 31) == 0) s_w[threadIdx.x >> 5] = t;
         __syncthreads();
@@ -365,37 +408,41 @@ __global__ void __launch_bounds__(256) k_dq_quantize(const float* __restrict__ a
         s_off = *offset_ptr;
     }
     __syncthreads();
-    const int64_t g = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    const int64_t ng = (nb + 255) >> 8;
-    if (g >= ng) return;
     const float off = s_off;
-    const int64_t b0 = g * 256 + lane * 8;
-    float d[8];
-    float c = 0.0f;
+    // one warp per group of 256 blocks; the grid is capped, so a warp takes
+    // every (gridDim.x * 8)-th group
+    for (int64_t gg = g; gg < ng; gg += (int64_t)gridDim.x * 8) {
+        const int64_t b0 = gg * 256 + lane * 8;
+        if (gg != g) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        d[i] = (b0 + i < nb) ? __fsub_rn(absmax[b0 + i], off) : 0.0f;
-        c = fmaxf(c, fabsf(d[i]));
+            for (int i = 0; i < 8; ++i) am[i] = b0 + i < nb ? absmax[b0 + i] : 0.0f;
+        }
+        float d[8];
+        float c = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            d[i] = (b0 + i < nb) ? __fsub_rn(am[i], off) : 0.0f;
+            c = fmaxf(c, fabsf(d[i]));
+        }
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) c = fmaxf(c, __shfl_xor_sync(0xffffffffu, c, o));
+        float p = 1.0f;
+        if (c < 1.17549435e-38f) p = 18446744073709551616.0f;
+        const float rc = (c == 0.0f) ? 0.0f : __frcp_rn(__fmul_rn(c, p));
+        uint32_t q[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) q[i] = (uint32_t)nearest_t8(__fmul_rn(__fmul_rn(d[i], p), rc), t8);
+        if (b0 + 8 <= nb) {
+            uint2 v;
+            v.x = q[0] | (q[1] << 8) | (q[2] << 16) | (q[3] << 24);
+            v.y = q[4] | (q[5] << 8) | (q[6] << 16) | (q[7] << 24);
+            *reinterpret_cast<uint2*>(q8 + b0) = v;
+        } else {
+            for (int i = 0; i < 8; ++i)
+                if (b0 + i < nb) q8[b0 + i] = (uint8_t)q[i];
+        }
+        if (lane == 0) c1[gg] = c;
     }
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) c = fmaxf(c, __shfl_xor_sync(0xffffffffu, c, o));
-    float p = 1.0f;
-    if (c < 1.17549435e-38f) p = 18446744073709551616.0f;
-    const float rc = (c == 0.0f) ? 0.0f : __frcp_rn(__fmul_rn(c, p));
-    uint32_t q[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) q[i] = (uint32_t)nearest_t8(__fmul_rn(__fmul_rn(d[i], p), rc), t8);
-    if (b0 + 8 <= nb) {
-        uint2 v;
-        v.x = q[0] | (q[1] << 8) | (q[2] << 16) | (q[3] << 24);
-        v.y = q[4] | (q[5] << 8) | (q[6] << 16) | (q[7] << 24);
-        *reinterpret_cast<uint2*>(q8 + b0) = v;
-    } else {
-        for (int i = 0; i < 8; ++i)
-            if (b0 + i < nb) q8[b0 + i] = (uint8_t)q[i];
-    }
-    if (lane == 0) c1[g] = c;
 }
 
 // ---------------------------------------------------------------------------
@@ -467,10 +514,10 @@ __global__ void __launch_bounds__(256) k_dequantize(const uint8_t* __restrict__ 
 
 // Block constants a' transposed for the GEMM producers: scales[kb*ld + n].
 // Also zeroes `nflags` ints (the flags of the stream-K GEMM that follows).
-__global__ void k_expand_scales(int64_t rows, int64_t kbs, int dq, const float* __restrict__ absmax,
-                                const uint8_t* __restrict__ q8, const float* __restrict__ c1,
-                                const float* __restrict__ offset_ptr, float* __restrict__ scales,
-                                int64_t ld, int* __restrict__ flags, int nflags) {
+__global__ void k_expand_scales(int64_t rows, int64_t kbs, int dq, const float* absmax,
+                                const uint8_t* q8, const float* c1,
+                                const float* offset_ptr, float* scales,
+                                int64_t ld, int* flags, int nflags) {
     // the LoRA GEMM that follows reads none of this kernel's outputs; this
     // kernel's inputs (8-bit constants) and outputs (scales, flags of the
     // GEMM before) belong to the kernel before it
@@ -544,37 +591,56 @@ inline cudaError_t launch_quantize_blocks(const void* W, int is_bf16, int64_t n,
     ProfileScope ps(QLORA_KERNEL_QUANTIZE, s);
     note_launch();
     if (is_bf16)
-        k_quantize_blocks<true><<<(unsigned)ng, 256, 0, s>>>(W, n, codes, absmax, group_sums,
-                                                              nf4_search_table());
-    else
-        k_quantize_blocks<false><<<(unsigned)ng, 256, 0, s>>>(W, n, codes, absmax, group_sums,
-                                                               nf4_search_table());
-    return cudaGetLastError();
+        return launch_pdl(k_quantize_blocks<true>, dim3((unsigned)ng), dim3(256), 0, s, 0, W, n, codes, absmax,
+                          group_sums, nf4_search_table());
+    return launch_pdl(k_quantize_blocks<false>, dim3((unsigned)ng), dim3(256), 0, s, 0, W, n, codes, absmax,
+                      group_sums, nf4_search_table());
 }
 
 inline cudaError_t launch_dq_offset(const double* group_sums, int64_t ngroups, int64_t nb,
                                     float* offset, cudaStream_t s) {
     note_launch();
-    k_dq_offset<<<1, 1024, 0, s>>>(group_sums, ngroups, nb, offset);
-    return cudaGetLastError();
+    return launch_pdl(k_dq_offset, dim3(1), dim3(1024), 0, s, 0, group_sums, ngroups, nb, offset);
 }
 
 inline cudaError_t launch_dq_quantize(const float* absmax, int64_t nb, float* offset, uint8_t* q8, float* c1,
                                       cudaStream_t s, const double* sums = nullptr, int64_t nsums = 0) {
     const int64_t ng = (nb + 255) / 256;
     if (ng == 0) return cudaSuccess;
+    int dev = 0, nsm = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        nsm = 148;
+    // at most 8 resident CTAs per SM; each forms the offset once
+    const int64_t grid = std::min<int64_t>((ng + 7) / 8, (int64_t)8 * nsm);
     note_launch();
-    k_dq_quantize<<<(unsigned)((ng + 7) / 8), 256, 0, s>>>(absmax, nb, offset, q8, c1, sums, nsums);
-    return cudaGetLastError();
+    return launch_pdl(k_dq_quantize, dim3((unsigned)grid), dim3(256), 0, s, 0, absmax, nb, offset, q8, c1, sums,
+                      nsums);
 }
 
 // Double quantization of the block maxima: offset, then 8-bit codes.  Up to
 // kFusedSums group sums every CTA of the 8-bit kernel forms the offset
-// itself (one launch); above, a separate one-CTA kernel does it first.
+// itself (one launch); above, k_dq_partials first reduces aligned 4096-leaf
+// subtrees into `partials` (dq_partial_count doubles) and the 8-bit kernel
+// forms the offset from those.  Test mode 5, or no partials buffer: the
+// one-CTA k_dq_offset kernel over all sums first.
 constexpr int64_t kFusedSums = 8192;
+inline int64_t dq_partial_count(int64_t nsums) {
+    if (nsums <= kFusedSums) return 0;
+    int64_t p2 = 1;
+    while (p2 < nsums) p2 <<= 1;
+    return p2 / kPartialLeaves;
+}
 inline cudaError_t launch_double_quant(const double* sums, int64_t nsums, const float* absmax, int64_t nb,
-                                       float* offset, uint8_t* q8, float* c1, cudaStream_t s) {
+                                       float* offset, uint8_t* q8, float* c1, cudaStream_t s,
+                                       double* partials = nullptr) {
     if (nsums <= kFusedSums && inject_mode() != 5) return launch_dq_quantize(absmax, nb, offset, q8, c1, s, sums, nsums);
+    const int64_t G = dq_partial_count(nsums);
+    if (G > 0 && partials && inject_mode() != 5) {
+        note_launch();
+        cudaError_t e = launch_pdl(k_dq_partials, dim3((unsigned)G), dim3(256), 0, s, 0, sums, nsums, partials);
+        if (e != cudaSuccess) return e;
+        return launch_dq_quantize(absmax, nb, offset, q8, c1, s, partials, G);
+    }
     cudaError_t e = launch_dq_offset(sums, nsums, nb, offset, s);
     if (e != cudaSuccess) return e;
     return launch_dq_quantize(absmax, nb, offset, q8, c1, s);

@@ -147,7 +147,7 @@ def test_encode_exhaustive(Q, O, cuda):
             start += n
 
 
-@pytest.mark.parametrize("shape", [(4096, 4096), (37, 200), (1, 16384 * 3 + 64)])
+@pytest.mark.parametrize("shape", [(4096, 4096), (37, 200), (1, 16384 * 3 + 64), (4096, 8192)])
 def test_separate_offset_kernel_matches(Q, O, cuda, shape):
     """The double-quantization offset formed by the 8-bit pass itself and by
     its own kernel (test mode 5) are the same fp32 value, and both match the
@@ -164,4 +164,26 @@ def test_separate_offset_kernel_matches(Q, O, cuda, shape):
     for x, y in [(q_fused.codes, q_sep.codes), (q_fused.absmax_q8, q_sep.absmax_q8),
                  (q_fused.absmax_scale.view(torch.int32), q_sep.absmax_scale.view(torch.int32)),
                  (q_fused.absmax_offset.view(torch.int32), q_sep.absmax_offset.view(torch.int32))]:
+        assert torch.equal(x, y)
+
+
+@pytest.mark.parametrize("shape", [(16384, 16384), (9000, 16384)])
+def test_partial_offset_tree_matches_single_cta(Q, cuda, shape):
+    """More than 8192 group sums: the offset from aligned 4096-leaf partial
+    subtrees (many CTAs) and from the one-CTA tree over all sums (test mode 5)
+    are the same fp32 value (same pairwise tree), so every output is equal."""
+    W = wl.weight(shape[0], shape[1], seed=12, dtype=torch.bfloat16, device="cuda")
+    q_part = Q.qlora_nf4_quantize(W, double_quant=True)
+    torch.cuda.synchronize()
+    assert Q.qlora_get_last_error() == 0
+    Q.qlora_debug_inject(5)
+    try:
+        q_one = Q.qlora_nf4_quantize(W, double_quant=True)
+        torch.cuda.synchronize()
+        assert Q.qlora_get_last_error() == 0
+    finally:
+        Q.qlora_debug_inject(0)
+    for x, y in [(q_part.codes, q_one.codes), (q_part.absmax_q8, q_one.absmax_q8),
+                 (q_part.absmax_scale.view(torch.int32), q_one.absmax_scale.view(torch.int32)),
+                 (q_part.absmax_offset.view(torch.int32), q_one.absmax_offset.view(torch.int32))]:
         assert torch.equal(x, y)
