@@ -161,15 +161,15 @@ inline int skinny_active_clusters(int cs) {
 }
 
 template <int BN>
-inline cudaError_t launch_skinny(SkinnyParams& p, int tiles, int kmin, int kmax, cudaStream_t s, int force_cs) {
+inline cudaError_t launch_skinny(SkinnyParams& p, int tiles, int kmin, int kmax, cudaStream_t s) {
     constexpr int smem = SkinnyShape<BN>::SMEM;
     static_assert(smem <= 232448, "shared memory per CTA");
     // Cluster size: fewest rounds of resident clusters times k-steps per CTA
     // (plus a fixed per-CTA cost of about three k-steps), at least one
-    // k-step per CTA of the shorter problem.  force_cs > 0 fixes it (work
-    // placed beside another kernel, on whatever SMs that one leaves free).
+    // k-step per CTA of the shorter problem.  Packed launches reduce each
+    // tile on one CTA.
     int cs = 1;
-    if (force_cs > 0 || p.pack) {
+    if (p.pack) {
         cs = 1;
     } else {
         int64_t best = -1;
@@ -229,11 +229,11 @@ struct SkinnyDesc {
 // wait_first: the operands may have been written by the kernel just before on
 // the stream (or by an unknown earlier one), so the loads wait for it.
 // place: SKP_SPLIT (cluster size from the cost model, the reduction split
-// across it), SKP_ONE (one CTA per 128-row tile), SKP_PACKED (one CTA per
-// tile, two tiles per TPC: work that leaves whole TPCs to a CTA-pair GEMM
-// beside it), SKP_STREAM (the persistent kernel on nctas CTAs, each taking
-// tiles round-robin: work beside a kernel that holds the other SMs).
-enum { SKP_SPLIT = 0, SKP_ONE = 1, SKP_PACKED = 2, SKP_STREAM = 3 };
+// across it), SKP_PACKED (one CTA per 128-row tile, two tiles per TPC: work
+// that leaves whole TPCs to a CTA-pair GEMM beside it), SKP_STREAM (the
+// persistent kernel on up to nctas CTAs: work beside a kernel that holds
+// most SMs; with ctrs the CTAs take tiles from a shared counter).
+enum { SKP_SPLIT = 0, SKP_PACKED = 1, SKP_STREAM = 2 };
 // SKP_STREAM with ctrs (two ints, zero before the launch): tiles taken in
 // problem order from ctrs[0]; problem dep_prob reads problem 0's output.
 // wait_mask (SKP_STREAM with wait_first == 0): problems that read the
@@ -249,7 +249,6 @@ inline qlora_status skinny(const SkinnyDesc* d, int nprob, int r, cudaStream_t s
     p.done_ctr = ctrs ? ctrs + 1 : nullptr;
     p.dep_prob = ctrs ? dep_prob : -1;
     p.wait_mask = wait_mask;
-    const int force_cs = place == SKP_ONE ? 1 : 0;
     int tiles = 0, kmin = 1 << 30, kmax = 0;
     for (int i = 0; i < nprob; ++i) {
         tiles += ceil_div(d[i].rows, 128);
@@ -286,11 +285,11 @@ inline qlora_status skinny(const SkinnyDesc* d, int nprob, int r, cudaStream_t s
         return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
     }
     if (bn == 64)
-        e = launch_skinny<64>(p, tiles, kmin, kmax, s, force_cs);
+        e = launch_skinny<64>(p, tiles, kmin, kmax, s);
     else if (bn == 128)
-        e = launch_skinny<128>(p, tiles, kmin, kmax, s, force_cs);
+        e = launch_skinny<128>(p, tiles, kmin, kmax, s);
     else
-        e = launch_skinny<256>(p, tiles, kmin, kmax, s, force_cs);
+        e = launch_skinny<256>(p, tiles, kmin, kmax, s);
     return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 

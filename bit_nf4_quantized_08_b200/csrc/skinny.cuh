@@ -448,6 +448,7 @@ __global__ void __launch_bounds__(StreamShape<BN>::THREADS, 1) k_lora_stream(con
                     const int target = 4 * p.pr[0].tiles;
                     const uint64_t t_start = globaltimer_ns();
                     while (ld_acquire_gpu(p.done_ctr) < target) {
+                        __nanosleep(256);
                         if (globaltimer_ns() - t_start > p.timeout_ns) {
                             set_status(4);
                             *abort_flag = 1;
