@@ -50,6 +50,17 @@ def test_quantize_workspace_sizes(Q):
     assert L.qlora_nf4_quantize_workspace(4096, 4096, 32, 1) == 0
     assert L.qlora_nf4_quantize_workspace(-1, 4, 64, 1) == 0
 
+    def a256(x):
+        return (x + 255) // 256 * 256
+
+    # more than 8192 group sums: one fp64 partial per 4096 leaves of the
+    # zero-padded power-of-two leaf array of the offset tree
+    for rows, cols, partials in ((16384, 16384, 4), (9000, 16384, 4), (8192, 16384, 0)):
+        n = rows * cols
+        nb, ng = -(-n // 64), -(-n // 16384)
+        want = a256(nb * 4) + a256(ng * 8) + a256(partials * 8)
+        assert L.qlora_nf4_quantize_workspace(rows, cols, 64, 1) == want, (rows, cols)
+
 
 def test_quantize_rejects(Q):
     from bit_nf4_quantized_08_b200._lib import lib, QLORA_ERR_INVALID_ARG, QLORA_ERR_UNSUPPORTED, QLORA_BF16
