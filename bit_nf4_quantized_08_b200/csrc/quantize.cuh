@@ -265,28 +265,25 @@ __global__ void __launch_bounds__(256, BF16 ? 4 : 2) k_quantize_blocks(const voi
 }
 
 // fp64 pairwise-tree sum of x[lo, lo + chunk) (chunk a power of two; entries
-// at or past n count as 0) with a binary-counter stack.  From chunk >= 8 on,
-// eight independent loads at a time are folded as a fixed subtree first: the
-// same tree, with an eighth of the dependent memory round trips.
+// at or past n count as 0; the values are non-negative) with a
+// binary-counter stack over subtrees of 8 leaves: eight independent loads at
+// a time are folded as a fixed subtree first (a chunk below 8 is one such
+// subtree padded with zeros), the same tree with an eighth of the dependent
+// memory round trips.
 __device__ __forceinline__ double pairwise_chunk(const double* x, int64_t lo, int64_t chunk,
                                                  int64_t n) {
     double stack[40];
     int64_t cnt = 0;
-    const int step = chunk >= 8 ? 8 : 1;
-    for (int64_t i = 0; i < chunk; i += step) {
-        double v;
-        if (step == 8) {
-            double e[8];
+    // leaves past the chunk (chunk < 8) or past n are +0.0: adding them
+    // changes no sum of the non-negative values summed here
+    for (int64_t i = 0; i < chunk; i += 8) {
+        double e[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int64_t idx = lo + i + j;
-                e[j] = idx < n ? x[idx] : 0.0;
-            }
-            v = ((e[0] + e[1]) + (e[2] + e[3])) + ((e[4] + e[5]) + (e[6] + e[7]));
-        } else {
-            const int64_t idx = lo + i;
-            v = idx < n ? x[idx] : 0.0;
+        for (int j = 0; j < 8; ++j) {
+            const int64_t idx = lo + i + j;
+            e[j] = (i + j < chunk && idx < n) ? x[idx] : 0.0;
         }
+        double v = ((e[0] + e[1]) + (e[2] + e[3])) + ((e[4] + e[5]) + (e[6] + e[7]));
         int lvl = 0;
         while ((cnt >> lvl) & 1) {
             v = stack[lvl] + v;
