@@ -339,6 +339,10 @@ struct StreamShape {
     static constexpr int B_BYTES = BN * 128;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int STAGES = BN <= 64 ? 8 : (BN <= 128 ? 6 : 4);
+    // stages are released in groups of CG k-steps: one tcgen05.commit per
+    // group (a commit costs about as much as the small MMAs it follows)
+    static constexpr int CG = 2;
+    static_assert(STAGES % CG == 0, "the ring holds whole commit groups");
     static constexpr int PIPE_BYTES = STAGE_BYTES * STAGES;
     static constexpr int SMEM = PIPE_BYTES + 1024 + 512;
     static constexpr int THREADS = 32 * 6;  // producer, MMA, 4 epilogue warps
@@ -462,7 +466,13 @@ __global__ void __launch_bounds__(StreamShape<BN>::THREADS, 1) k_lora_stream(con
                 const int m0 = tile * 128;
                 for (int k = 0; k < P.ksteps; ++k, ++it) {
                     const int s = it % STAGES, us = it / STAGES;
-                    if (!mbar_wait(empty(s), (us & 1) ^ 1, wc)) { *abort_flag = 1; break; }
+                    // the stage's previous k-step (it - STAGES) is in commit group
+                    // it / CG - STAGES / CG, released on the same group barrier
+                    const int gi = it / S::CG;
+                    if (!mbar_wait(empty(gi % (STAGES / S::CG)), ((gi / (STAGES / S::CG)) & 1) ^ 1, wc)) {
+                        *abort_flag = 1;
+                        break;
+                    }
                     const uint32_t sA = base + s * S::STAGE_BYTES;
                     const uint32_t sB = sA + S::A_BYTES;
                     mbar_arrive_expect_tx(full(s), S::A_BYTES + S::B_BYTES);
@@ -515,7 +525,7 @@ __global__ void __launch_bounds__(StreamShape<BN>::THREADS, 1) k_lora_stream(con
                                                    : smem_desc_sw128(sB + kk * 32, 16, 1024);
                         umma_bf16(acc, ad, bd, idesc, (k > 0 || kk > 0) ? 1u : 0u);
                     }
-                    umma_commit(empty(s));
+                    if (it % S::CG == S::CG - 1) umma_commit(empty((it / S::CG) % (STAGES / S::CG)));
                 }
                 // committed also after an abort, so that the wait below covers
                 // every MMA issued
