@@ -182,13 +182,15 @@ qlora_status qlora_linear_fwd(const void *X, int64_t M, const qlora_nf4_weight *
  *   only dX is produced.  With M == 0, dA and dB are set to zero.
  * Same shape requirements as qlora_linear_fwd.  Deterministic (no floating
  * point atomics on any output).
- * Streams: all work is ordered on `stream`.  With dX and r > 0 the dA/dB
- * GEMMs run on a per-device side stream of the library that waits for
- * `stream` first, beside the dX GEMM, and `stream` waits for them before the
- * call returns, so to the caller the call is one ordered step on `stream`
- * (also inside a stream capture, once the side stream exists: it is created
- * by the first such call made outside a capture).  Calls from several host
- * threads are serialized on that side stream.
+ * Streams: all work is ordered on `stream`.  With dX and r > 0 (and the
+ * default CTA-pair schedule) the sU, dA and dB GEMMs run on a per-device
+ * side stream of the library, beside the dX GEMM; the side stream first waits
+ * for `stream` (after the sG GEMM) and `stream` waits for it before the call
+ * returns, so to the caller the call is one ordered step on `stream` (also
+ * inside a stream capture, once the side stream exists: it is created by the
+ * first such call made outside a capture).  The library keeps that stream and
+ * two events per device for its lifetime.  Calls from several host threads
+ * are serialized on the side stream.
  */
 qlora_status qlora_linear_bwd(const void *dY, const void *X, int64_t M, const qlora_nf4_weight *w,
                               const void *A, const void *B, int32_t r, float scale, void *dX,
