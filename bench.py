@@ -2,8 +2,8 @@
 """Benchmark of the QLoRA NF4 frozen-linear hot path on B200.
 
 One step = one pass of the whole hot path over one batch of the
-LLaMA-7B-shaped decoder block (q/k/v/o 4096x4096, gate/up 11008x4096, down
-4096x11008; M = 4 x 512 tokens; LoRA r = 64, alpha = 16 on all seven):
+LLaMA-65B-shaped decoder block (q/k/v/o 8192x8192, gate/up 22016x8192, down
+8192x22016; M = 1 x 2048 tokens; LoRA r = 64, alpha = 16 on all seven):
   1. blockwise NF4 quantization + double quantization of the 7 bf16 weights
   2. forward Y = X W'^T + s (X A^T) B^T of the 7 linears
   3. backward dX, dA, dB of the 7 linears (no dW)
@@ -15,10 +15,13 @@ synchronize around the timed region, max over ranks.  Under torchrun every
 rank runs an independent replica (the layer does not shard: weak scaling).
 
 Also reported: the roofline of the dominant kernel (live CUDA-event times of
-its launches), an end-to-end figure through pinned host buffers, the CPU
-oracle on a bounded sample, sampled SM clocks, and extra measurements outside
-the step (small-M forward sweep on a 22016x8192 weight, standalone quantize
-and dequantize of 2^30 elements).
+its launches), an end-to-end figure through the C ABI with pinned host
+buffers (every input copied in and every result copied out inside the timed
+region), the CPU oracle on a bounded sample (all cores and one core) with its
+outputs compared against the GPU's, sampled SM clocks, and extra measurements
+outside the step (the LLaMA-7B block, the stress forward, the small-M forward
+sweep on a 22016x8192 weight, standalone quantize and dequantize of 2^30
+elements).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 """
@@ -38,7 +41,14 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "fused NF4-dequant+LoRA linear fwd/bwd TFLOP/s and weight GB/s vs B200 roofline"
-WORKLOAD = "llama7b-decoder-block: 7 NF4+DQ linears (q,k,v,o 4096x4096; gate,up 11008x4096; down 4096x11008), M=2048, r=64, alpha=16; quantize+fwd+bwd"
+HEADLINE = "llama65b"
+WORKLOADS = {
+    "llama65b": "llama65b-decoder-block: 7 NF4+DQ linears (q,k,v,o 8192x8192; gate,up 22016x8192; "
+                "down 8192x22016), M=2048 (1 x 2048 tokens), r=64, alpha=16; quantize+fwd+bwd",
+    "llama7b": "llama7b-decoder-block: 7 NF4+DQ linears (q,k,v,o 4096x4096; gate,up 11008x4096; "
+               "down 4096x11008), M=2048 (4 x 512 tokens), r=64, alpha=16; quantize+fwd+bwd",
+}
+WORKLOAD = WORKLOADS[HEADLINE]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 WEIGHT_BYTES_PER_ELEM = 0.5 + 1 / 64 + 4 / (64 * 256)  # NF4 codes + q8 + c1 (DQ)
 
@@ -55,6 +65,8 @@ def parse():
                                                "fwd_block", "dx_block"],
                     help="run one small case three times, untimed (for ncu captures); "
                          "*_block runs the seven block linears once each")
+    ap.add_argument("--block", choices=sorted(WORKLOADS), default=HEADLINE,
+                    help="decoder block of the *_block profile cases")
     return ap.parse_args()
 
 
@@ -160,10 +172,12 @@ def load_traffic(kind):
 # ---------------------------------------------------------------------------
 
 class Block:
-    """The seven linears of one decoder block with every buffer preallocated."""
+    """The seven linears of one decoder block with every buffer preallocated.
+    Layer li draws its tensors from generator indices 10*li + (0..9)."""
 
-    def __init__(self, torch, Q, wl, device, seed=0):
-        c = wl.CONFIGS["llama7b"]
+    def __init__(self, torch, Q, wl, device, cfg=HEADLINE, seed=0):
+        c = wl.CONFIGS[cfg]
+        self.cfg = cfg
         self.M, self.r, self.s = c["M"], c["r"], c["alpha"] / c["r"]
         self.layers = []
         ws_need = 0
@@ -184,8 +198,7 @@ class Block:
                           Q.qlora_linear_workspace(self.M, L["w"], self.r, True))
         self.ws = torch.empty(ws_need, dtype=torch.uint8, device=device)
         self.Q = Q
-        self.flops = sum(fwd_flops(self.M, L["N"], L["K"], self.r) + bwd_flops(self.M, L["N"], L["K"], self.r)
-                         for L in self.layers)
+        self.flops = block_flops(wl, cfg)
         self.fwd_gemm_flops = sum(2 * self.M * L["N"] * L["K"] + 2 * self.M * self.r * L["N"] for L in self.layers)
         self.dx_gemm_flops = sum(2 * self.M * L["N"] * L["K"] + 2 * self.M * self.r * L["K"] for L in self.layers)
         self.quant_bytes = sum(L["N"] * L["K"] * (2 + WEIGHT_BYTES_PER_ELEM) for L in self.layers)
@@ -210,6 +223,11 @@ class Block:
                                    dB=L["dB"], ws=ws)
             else:
                 Q.qlora_linear_bwd(L["dY"], L["X"], L["w"], None, None, self.s, dX=L["dX"], ws=ws)
+
+
+def block_flops(wl, cfg):
+    c = wl.CONFIGS[cfg]
+    return sum(fwd_flops(c["M"], N, K, c["r"]) + bwd_flops(c["M"], N, K, c["r"]) for _, N, K in c["linears"])
 
 
 def max_over_ranks(torch, value, world, device):
@@ -243,50 +261,294 @@ def time_steps(torch, fn, steps, flush, dist_barrier):
     return [s.elapsed_time(e) for s, e in zip(starts, ends)]
 
 
+def graph_of(torch, fn):
+    """A CUDA graph of fn() captured after one untimed run on a side stream."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        fn()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    g.replay()
+    torch.cuda.synchronize()
+    return g
+
+
+def replay_ms(torch, g, reps, flush):
+    """Median device time (ms) of reps graph replays, L2 flushed before each."""
+    times = []
+    for _ in range(reps):
+        flush()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.replay()
+        e1.record()
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1))
+    return statistics.median(times)
+
+
 # ---------------------------------------------------------------------------
-# CPU oracle sample (reported baseline and the reference arm)
+# end to end through the C ABI
 # ---------------------------------------------------------------------------
 
-def oracle_sample(torch, wl, seed=0):
-    """Bounded oracle sample of one step: for each of the 7 linears of the
-    block (M=2048, r=64): full quantize + DQ + dequantize of W, forward and dX
-    on 16 of the 2048 token rows, dA and dB in full.
-    Returns (flops, seconds, description, threads)."""
-    import numpy as np
+def e2e_measure(torch, blk, steps, flush, barrier, world, device):
+    """The step through the library's C entry points (ctypes, raw pointers),
+    with every input copied in from pinned host buffers (W, X, dY of the seven
+    linears) and every result copied out to pinned host buffers (Y, dX, dA,
+    dB) inside the timed region.  Inputs stream in on one copy stream in the
+    order the step uses them, results stream out on another as each call
+    finishes; each call waits only for its own inputs."""
+    import ctypes
+    from bit_nf4_quantized_08_b200 import _lib
+    lib = _lib.lib()
+    layers = blk.layers
+    cws = [L["w"].c_struct() for L in layers]
+    hin = {}
+    for i, L in enumerate(layers):
+        for k in ("W", "X", "dY"):
+            h = torch.empty(L[k].shape, dtype=L[k].dtype, pin_memory=True)
+            h.copy_(L[k])
+            hin[(i, k)] = h
+    hout = {(i, k): torch.empty(L[k].shape, dtype=L[k].dtype, pin_memory=True)
+            for i, L in enumerate(layers) for k in ("Y", "dX", "dA", "dB")}
+    h2d = sum(h.numel() * h.element_size() for h in hin.values())
+    d2h = sum(h.numel() * h.element_size() for h in hout.values())
+    order = ([(i, "W") for i in range(len(layers))] + [(i, "X") for i in range(len(layers))] +
+             [(i, "dY") for i in reversed(range(len(layers)))])
+    ev_in = {k: torch.cuda.Event() for k in order}
+    ev_fwd = [torch.cuda.Event() for _ in layers]
+    ev_bwd = [torch.cuda.Event() for _ in layers]
+    up, down = torch.cuda.Stream(device=device), torch.cuda.Stream(device=device)
+    ws, ws_bytes = blk.ws.data_ptr(), blk.ws.numel()
+    M, r, s = blk.M, blk.r, blk.s
+
+    def call(st, what):
+        if st != 0:
+            raise RuntimeError(f"{what}: status {st}")
+
+    def step():
+        cur = torch.cuda.current_stream()
+        hs = ctypes.c_void_p(cur.cuda_stream)
+        up.wait_stream(cur)  # the previous step is done with the device buffers
+        with torch.cuda.stream(up):
+            for key in order:
+                i, k = key
+                layers[i][k].copy_(hin[key], non_blocking=True)
+                ev_in[key].record(up)
+        for i, L in enumerate(layers):
+            cur.wait_event(ev_in[(i, "W")])
+            call(lib.qlora_nf4_quantize(L["W"].data_ptr(), _lib.QLORA_BF16, ctypes.byref(cws[i]), ws, ws_bytes,
+                                        hs), "qlora_nf4_quantize")
+        for i, L in enumerate(layers):
+            cur.wait_event(ev_in[(i, "X")])
+            call(lib.qlora_linear_fwd(L["X"].data_ptr(), M, ctypes.byref(cws[i]), L["A"].data_ptr(),
+                                      L["B"].data_ptr(), r, ctypes.c_float(s), L["Y"].data_ptr(), ws, ws_bytes,
+                                      hs), "qlora_linear_fwd")
+            ev_fwd[i].record(cur)
+            down.wait_event(ev_fwd[i])
+            with torch.cuda.stream(down):
+                hout[(i, "Y")].copy_(L["Y"], non_blocking=True)
+        for i in reversed(range(len(layers))):
+            L = layers[i]
+            cur.wait_event(ev_in[(i, "dY")])
+            call(lib.qlora_linear_bwd(L["dY"].data_ptr(), L["X"].data_ptr(), M, ctypes.byref(cws[i]),
+                                      L["A"].data_ptr(), L["B"].data_ptr(), r, ctypes.c_float(s),
+                                      L["dX"].data_ptr(), L["dA"].data_ptr(), L["dB"].data_ptr(), ws, ws_bytes,
+                                      hs), "qlora_linear_bwd")
+            ev_bwd[i].record(cur)
+            down.wait_event(ev_bwd[i])
+            with torch.cuda.stream(down):
+                for k in ("dX", "dA", "dB"):
+                    hout[(i, k)].copy_(L[k], non_blocking=True)
+        cur.wait_stream(down)  # the results are on the host when the step ends
+
+    step()
+    torch.cuda.synchronize()
+    n = max(3, min(steps, 5))
+    times = time_steps(torch, step, n, flush, barrier)
+    ms = max_over_ranks(torch, statistics.mean(times), world, device)
+    # the copied-out results are the device results
+    for i, L in enumerate(layers):
+        for k in ("Y", "dX", "dA", "dB"):
+            assert torch.equal(hout[(i, k)].view(torch.int16 if L[k].dtype == torch.bfloat16 else torch.int32),
+                               L[k].cpu().view(torch.int16 if L[k].dtype == torch.bfloat16 else torch.int32))
+    return {"value": round(whole_job_tflops(blk.flops, world, ms), 2), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms, 3),
+            "method": "C ABI entry points called with raw device pointers (ctypes); W, X, dY of the 7 linears "
+                      "copied in from pinned host memory on one stream in the order of use, Y, dX, dA, dB "
+                      "copied out to pinned host memory on another as each call ends, all inside the timed "
+                      "region; the copied-out results equal the device results"}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle: bounded samples (reported baseline, the reference arm) and the
+# check of the GPU's outputs
+# ---------------------------------------------------------------------------
+
+def _cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
+def oracle_sample(torch, wl, cfg, layers=None, rows_n=16, seed=0):
+    """The oracle on a bounded sample of the block step: for each selected
+    linear (default: all seven), full NF4+DQ quantize and dequantize of W,
+    Y and dX on rows_n sampled token rows, dA and dB in full (all M rows).
+    Input generation is not timed.  Returns a dict with the sample's flops,
+    its seconds (quantize/dequantize and the products separately), the
+    sampled rows and, per layer, the oracle's outputs."""
     from oracle import oracle as O
     O.build()
-    c = wl.CONFIGS["llama7b"]
+    c = wl.CONFIGS[cfg]
     M, r, s = c["M"], c["r"], c["alpha"] / c["r"]
-    rows = np.linspace(0, M - 1, 16).astype(np.int64)
+    rows = wl.sample_rows(M, rows_n, seed=seed)
     R = rows.size
-    flops, dt = 0, 0.0
-    for li, (_, N, K) in enumerate(c["linears"]):
+    out = {"flops": 0, "quant_s": 0.0, "gemm_s": 0.0, "rows": rows, "layers": {}}
+    for li, (name, N, K) in enumerate(c["linears"]):
+        if layers is not None and li not in layers:
+            continue
         base = 10 * li
         W = wl.weight(N, K, seed=seed, dtype=torch.bfloat16, index_base=base)
         inp = wl.linear_inputs(M, N, K, r, seed=seed, index_base=base)
         Xb, dYb, Ab, Bb = (wl.bits(inp[k]) for k in ("X", "dY", "A", "B"))
         Wbits = wl.bits(W).reshape(-1)
+        del W, inp
         t0 = time.perf_counter()
         q = O.nf4_quantize(Wbits, double_quant=True)
         Wd = O.nf4_dequantize(N * K, q).reshape(N, K)
-        O.linear_fwd(Xb, Wd, Ab, Bb, s, rows=rows)
-        O.linear_bwd(dYb, Xb, Wd, Ab, Bb, s, rows=rows)
-        dt += time.perf_counter() - t0
-        flops += (R * (2 * N * K + 2 * r * (K + N))      # forward rows
-                  + R * (2 * N * K + 2 * r * K)          # dX rows
-                  + 2 * M * r * (K + N)                  # U and G over all rows
-                  + 2 * M * r * K + 2 * M * N * r)       # dA, dB
-    desc = ("all 7 linears of the block (M=2048, r=64): full NF4+DQ quantize and dequantize "
-            "of W, Y and dX on 16 of 2048 token rows, dA and dB in full")
-    return flops, dt, desc, O.num_threads()
+        t1 = time.perf_counter()
+        Y = O.linear_fwd(Xb, Wd, Ab, Bb, s, rows=rows)
+        dX, dA, dB = O.linear_bwd(dYb, Xb, Wd, Ab, Bb, s, rows=rows)
+        t2 = time.perf_counter()
+        out["quant_s"] += t1 - t0
+        out["gemm_s"] += t2 - t1
+        out["flops"] += (R * (2 * N * K + 2 * r * (K + N))      # forward rows
+                         + R * (2 * N * K + 2 * r * K)          # dX rows
+                         + 2 * M * r * (K + N)                  # U and G over all rows
+                         + 2 * M * r * K + 2 * M * N * r)       # dA, dB
+        out["layers"][li] = {"codes": q["codes"], "q8": q["q8"], "Y": Y, "dX": dX, "dA": dA, "dB": dB}
+    out["seconds"] = out["quant_s"] + out["gemm_s"]
+    return out
+
+
+def _ratios(got, ref):
+    import numpy as np
+    d = np.asarray(got, np.float64) - ref
+    return (float(np.max(np.abs(d)) / max(np.max(np.abs(ref)), 1e-300)),
+            float(np.linalg.norm(d) / max(np.linalg.norm(ref), 1e-300)))
+
+
+def oracle_check(blk, sample):
+    """GPU outputs of the step against the oracle sample: codes and 8-bit
+    constants bit for bit, Y and dX on the sampled rows, dA and dB in full,
+    at max|d| <= 1e-2 max|ref| and ||d||_F <= 5e-3 ||ref||_F."""
+    import numpy as np
+    rows = sample["rows"]
+    worst = {"max_ratio": 0.0, "frob_ratio": 0.0}
+    bitexact = True
+    for li, ref in sample["layers"].items():
+        L = blk.layers[li]
+        bitexact &= bool(np.array_equal(L["w"].codes.cpu().numpy(), ref["codes"]))
+        bitexact &= bool(np.array_equal(L["w"].absmax_q8.cpu().numpy(), ref["q8"]))
+        for k in ("Y", "dX", "dA", "dB"):
+            got = L[k].float().cpu().numpy()
+            if k in ("Y", "dX"):
+                got = got[rows]
+            mr, fr = _ratios(got, ref[k])
+            worst["max_ratio"] = max(worst["max_ratio"], mr)
+            worst["frob_ratio"] = max(worst["frob_ratio"], fr)
+    ok = bitexact and worst["max_ratio"] <= 1e-2 and worst["frob_ratio"] <= 5e-3
+    return {"ok": ok, "quantize_bit_exact": bitexact, "worst_max_abs_err_over_max_ref": round(worst["max_ratio"], 6),
+            "worst_frob_err_over_frob_ref": round(worst["frob_ratio"], 6),
+            "compared": f"codes and q8 of all {len(sample['layers'])} weights bit for bit; Y and dX on "
+                        f"{rows.size} sampled token rows, dA and dB in full"}
+
+
+def cpu_baseline(torch, wl, cfg, gpu_block=None):
+    """The oracle timed on the host's cores: the bounded sample on all cores
+    (its outputs also checked against the GPU's when a block is given), the
+    first linear's sample on one core, and the full step's time extrapolated
+    from the all-core rates (labelled as such)."""
+    from oracle import oracle as O
+    O.build()
+    threads = O.num_threads()
+    smp = oracle_sample(torch, wl, cfg)
+    check = oracle_check(gpu_block, smp) if gpu_block is not None else None
+    O.set_num_threads(1)
+    try:
+        one = oracle_sample(torch, wl, cfg, layers=[0])
+    finally:
+        O.set_num_threads(threads)
+    c = wl.CONFIGS[cfg]
+    full_flops = block_flops(wl, cfg)
+    sampled_gemm_rate = smp["flops"] / smp["gemm_s"]
+    extrap_s = smp["quant_s"] + full_flops / sampled_gemm_rate
+    base = {"value": smp["flops"] / smp["seconds"] / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"all 7 linears of the {cfg} block (M={c['M']}, r={c['r']}): full NF4+DQ quantize and "
+                      f"dequantize of W, Y and dX on {smp['rows'].size} of {c['M']} token rows, dA and dB in full",
+            "seconds": round(smp["seconds"], 2), "cpu_model": _cpu_model(), "nproc": os.cpu_count(),
+            "single_thread": {"value": one["flops"] / one["seconds"] / 1e12, "unit": "TFLOP/s", "cores": 1,
+                              "seconds": round(one["seconds"], 2),
+                              "sample": f"the same sample for the first linear ({c['linears'][0][0]}) only"},
+            "all_cores": {"value": smp["flops"] / smp["seconds"] / 1e12, "unit": "TFLOP/s", "cores": threads},
+            "full_step_seconds_extrapolated": round(extrap_s, 1),
+            "extrapolation": "extrapolated: measured quantize+dequantize time of the 7 weights plus the full "
+                             "step's fwd+bwd flops at the sample's all-core product rate"}
+    return base, check
 
 
 # ---------------------------------------------------------------------------
-# extras: small-M sweep, 2^30 quantize / dequantize
+# extras: 7B block, stress forward, small-M sweep, 2^30 quantize / dequantize
 # ---------------------------------------------------------------------------
 
 def extras(torch, Q, wl, device, flush, peaks):
     out = {}
+    # LLaMA-7B decoder block (the same step, smaller shapes)
+    blk = Block(torch, Q, wl, device, cfg="llama7b")
+    for _ in range(3):
+        blk.step()
+    g = graph_of(torch, blk.step)
+    ms = replay_ms(torch, g, 10, flush)
+    del g
+    tf = blk.flops / (ms * 1e-3) / 1e12
+    out["llama7b_block_step_cuda_graph"] = {
+        "workload": WORKLOADS["llama7b"], "ms": round(ms, 4), "TFLOPs": round(tf, 1),
+        "frac_bf16_peak": round(tf / peaks["bf16_tflops"], 3)}
+    del blk
+    torch.cuda.empty_cache()
+
+    # stress forward: 4096x4096 weight with outliers, 2048 tokens, r = 16
+    c = wl.CONFIGS["stress"]
+    (_, N, K), = c["linears"]
+    M, r, s = c["M"], c["r"], c["alpha"] / c["r"]
+    W = wl.weight(N, K, seed=0, dtype=torch.bfloat16, outlier_frac=c["outlier_frac"],
+                  outlier_std=c["outlier_std"], device=device)
+    w = Q.qlora_nf4_quantize(W)
+    inp = wl.linear_inputs(M, N, K, r, seed=0, device=device)
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device=device)
+    ws = torch.empty(Q.qlora_linear_workspace(M, w, r, False), dtype=torch.uint8, device=device)
+    fn = lambda: Q.qlora_linear_fwd(inp["X"], w, inp["A"], inp["B"], s, Y=Y, ws=ws)  # noqa: E731
+    for _ in range(3):
+        fn()
+    g = graph_of(torch, fn)
+    ms = replay_ms(torch, g, 20, flush)
+    del g
+    tf = fwd_flops(M, N, K, r) / (ms * 1e-3) / 1e12
+    out["stress_fwd_4096x4096_M2048_r16_cuda_graph"] = {
+        "us": round(ms * 1e3, 2), "TFLOPs": round(tf, 1), "frac_bf16_peak": round(tf / peaks["bf16_tflops"], 3)}
+    del W, w, inp, Y, ws
+
     c = wl.CONFIGS["sweep"]
     (_, N, K), = c["linears"]
     r, s = c["r"], c["alpha"] / c["r"]
@@ -294,35 +556,22 @@ def extras(torch, Q, wl, device, flush, peaks):
     w = Q.qlora_nf4_quantize(W)
     del W
     sweep = {}
-    reps = 20
     for M in c["Ms"]:
         inp = wl.linear_inputs(M, N, K, r, seed=0, device=device)
         X, A, B = inp["X"], inp["A"], inp["B"]
         Y = torch.empty(M, N, dtype=torch.bfloat16, device=device)
         ws = torch.empty(Q.qlora_linear_workspace(M, w, r, False), dtype=torch.uint8, device=device)
+        fn = lambda: Q.qlora_linear_fwd(X, w, A, B, s, Y=Y, ws=ws)  # noqa: E731
         for _ in range(3):
-            Q.qlora_linear_fwd(X, w, A, B, s, Y=Y, ws=ws)
-        torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            Q.qlora_linear_fwd(X, w, A, B, s, Y=Y, ws=ws)
-        times = []
-        for _ in range(reps):
-            flush()
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            e0.record()
-            g.replay()
-            e1.record()
-            e1.synchronize()
-            times.append(e0.elapsed_time(e1))
-        ms = statistics.median(times)
+            fn()
+        g = graph_of(torch, fn)
+        ms = replay_ms(torch, g, 20, flush)
+        del g
         wbytes = N * K * WEIGHT_BYTES_PER_ELEM
         total = wbytes + M * K * 2 + r * K * 2 + N * r * 2 + M * N * 2
         sweep[str(M)] = {"us": round(ms * 1e3, 2), "weight_GBps": round(wbytes / ms / 1e6, 1),
                          "total_GBps": round(total / ms / 1e6, 1),
                          "frac_hbm": round(total / ms / 1e6 / peaks["hbm_gbs"], 3)}
-        del g
     out["small_m_fwd_22016x8192_r64_cuda_graph"] = sweep
 
     n = c["big_numel"]
@@ -335,27 +584,14 @@ def extras(torch, Q, wl, device, flush, peaks):
                      ("dequantize_2^30_bf16", lambda: Q.qlora_nf4_dequantize(qb, out=deq))):
         for _ in range(3):
             fn()
-        torch.cuda.synchronize()
         # one call captured in a CUDA graph and replayed, as the step: device
         # time of the call's kernels, without the host's launch cost
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            fn()
-        times = []
-        for _ in range(5):
-            flush()
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            e0.record()
-            g.replay()
-            e1.record()
-            e1.synchronize()
-            times.append(e0.elapsed_time(e1))
+        g = graph_of(torch, fn)
+        ms = replay_ms(torch, g, 5, flush)
         del g
-        ms = statistics.median(times)
         out[name + "_cuda_graph"] = {"us": round(ms * 1e3, 1), "GBps": round(algo / ms / 1e6, 1),
-                     "frac_hbm": round(algo / ms / 1e6 / peaks["hbm_gbs"], 3),
-                     "algorithmic_bytes": int(algo)}
+                                     "frac_hbm": round(algo / ms / 1e6 / peaks["hbm_gbs"], 3),
+                                     "algorithmic_bytes": int(algo)}
     del Wbig, qb, deq, wsq
     return out
 
@@ -371,7 +607,7 @@ def main():
     if args.impl == "reference":
         return run_reference(args, world, rank)
     if args.profile_case:
-        return run_profile_case(args.profile_case)
+        return run_profile_case(args.profile_case, args.block)
 
     import torch
     import torch.distributed as dist
@@ -398,7 +634,7 @@ def main():
     def flush():
         flush_buf.fill_(1)
 
-    blk = Block(torch, Q, wl, device, seed=rank)
+    blk = Block(torch, Q, wl, device, cfg=HEADLINE, seed=rank)
     for _ in range(max(3, args.warmup)):
         blk.step()
     torch.cuda.synchronize()
@@ -411,17 +647,7 @@ def main():
     # eager steps: the host launches every kernel of the step
     eager_times = time_steps(torch, blk.step, min(args.steps, 5), flush, barrier)
     # the timed steps replay one CUDA graph of the step (no host launch cost)
-    side = torch.cuda.Stream(device=device)
-    side.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(side):
-        blk.step()
-    torch.cuda.current_stream().wait_stream(side)
-    torch.cuda.synchronize()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        blk.step()
-    graph.replay()
-    torch.cuda.synchronize()
+    graph = graph_of(torch, blk.step)
 
     clocks = ClockSampler(local_rank)
     clocks.start()
@@ -430,13 +656,10 @@ def main():
     launches = launches_per_step * args.steps
     status = Q.qlora_get_last_error()
     assert status == 0, f"device status {status}"
+    del graph
     # the same step without the adapter (r = 0), also a graph replay: the
     # difference is the step time the LoRA GEMMs still add
-    base_graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(base_graph):
-        blk.step(adapter=False)
-    base_graph.replay()
-    torch.cuda.synchronize()
+    base_graph = graph_of(torch, lambda: blk.step(adapter=False))
     base_ms = max_over_ranks(torch, sum(time_steps(torch, base_graph.replay, args.steps, flush, barrier)),
                              world, device) / args.steps
     del base_graph
@@ -461,6 +684,7 @@ def main():
                 "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                 "frac": round(achieved / peak, 4), "traffic": traffic,
                 "peak_source": f"{peak_src} bf16 dense (burst)",
+                "frac_of_sustained": round(achieved / peaks.get("bf16_tflops_sustained", peak), 4),
                 "launches": dom_n, "avg_launch_us": round(dom_ms / max(dom_n, 1) * 1e3, 2)}
     breakdown = {}
     qms, qn = prof["quantize"]
@@ -483,61 +707,15 @@ def main():
             breakdown[k + "_TFLOPs"] = round(fl / (ms_k * 1e-3) / 1e12, 1)
             breakdown[k + "_share_of_step"] = round(ms_k / total_ms, 3)
 
-    # end to end through the public API with pinned host buffers
-    host_in = []
-    for L in blk.layers:
-        for key in ("W", "X", "dY"):
-            h = torch.empty(L[key].shape, dtype=L[key].dtype, pin_memory=True)
-            h.copy_(L[key])
-            host_in.append((h, L[key]))
-    host_out = []
-    for L in blk.layers:
-        for key in ("dA", "dB"):
-            host_out.append((torch.empty(L[key].shape, dtype=L[key].dtype, pin_memory=True), L[key]))
-    h2d = sum(h.numel() * h.element_size() for h, _ in host_in)
-    d2h = sum(h.numel() * h.element_size() for h, _ in host_out)
+    e2e = e2e_measure(torch, blk, args.steps, flush, barrier, world, device)
 
-    # inputs stream in on a copy stream in the order the step uses them (the
-    # weights for the quantizer, then X for the forward, then dY for the
-    # backward, last layer first); each kernel waits only for its own inputs
-    copy_stream = torch.cuda.Stream(device=device)
-    hosts = {(i, key): h for i, L in enumerate(blk.layers) for key in ("W", "X", "dY")
-             for h, d in host_in if d is L[key]}
-    order = ([(i, "W") for i in range(len(blk.layers))] + [(i, "X") for i in range(len(blk.layers))] +
-             [(i, "dY") for i in reversed(range(len(blk.layers)))])
-    events = {k: torch.cuda.Event() for k in order}
-
-    def e2e_step():
-        Qm, ws, cur = blk.Q, blk.ws, torch.cuda.current_stream()
-        copy_stream.wait_stream(cur)  # the previous step is done with the device buffers
-        with torch.cuda.stream(copy_stream):
-            for (i, key) in order:
-                blk.layers[i][key].copy_(hosts[(i, key)], non_blocking=True)
-                events[(i, key)].record(copy_stream)
-        for i, L in enumerate(blk.layers):
-            cur.wait_event(events[(i, "W")])
-            Qm.qlora_nf4_quantize(L["W"], True, out=L["w"], ws=ws)
-        for i, L in enumerate(blk.layers):
-            cur.wait_event(events[(i, "X")])
-            Qm.qlora_linear_fwd(L["X"], L["w"], L["A"], L["B"], blk.s, Y=L["Y"], ws=ws)
-        for i in reversed(range(len(blk.layers))):
-            L = blk.layers[i]
-            cur.wait_event(events[(i, "dY")])
-            Qm.qlora_linear_bwd(L["dY"], L["X"], L["w"], L["A"], L["B"], blk.s, dX=L["dX"], dA=L["dA"],
-                                dB=L["dB"], ws=ws)
-            for key in ("dA", "dB"):
-                for h, d in host_out:
-                    if d is L[key]:
-                        h.copy_(d, non_blocking=True)
-
-    e2e_steps = max(3, min(args.steps, 5))
-    e2e_times = time_steps(torch, e2e_step, e2e_steps, flush, barrier)
-    e2e_ms = max_over_ranks(torch, statistics.mean(e2e_times), world, device)
-    e2e = {"value": round(whole_job_tflops(blk.flops, world, e2e_ms), 2), "unit": "TFLOP/s",
-           "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-           "ms_per_step": round(e2e_ms, 3),
-           "method": "public API calls; pinned-host inputs copied on a second stream in the order of use, "
-                     "overlapped with the kernels; dA, dB copied back"}
+    # the oracle on the host cores (rank 0 only), its outputs compared with
+    # the GPU's outputs of this step
+    cpu, check = None, None
+    if rank == 0 and not args.no_cpu:
+        blk.step()
+        torch.cuda.synchronize()
+        cpu, check = cpu_baseline(torch, wl, HEADLINE, gpu_block=blk)
 
     extra = None
     if not args.no_extras:
@@ -545,42 +723,33 @@ def main():
         torch.cuda.empty_cache()
         extra = extras(torch, Q, wl, device, flush, peaks)
 
-    cpu = None
-    if rank == 0 and not args.no_cpu:
-        flops, dt, desc, threads = oracle_sample(torch, wl)
-        cpu = {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-               "sample": desc, "seconds": round(dt, 2)}
-
     if world > 1:
         dist.barrier()
     if rank == 0:
+        c = wl.CONFIGS[HEADLINE]
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": round(ms_per_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": WORKLOAD, "global_batch": 2048 * world, "seq_len": 512,
-                       "flops_per_step": blk_flops_cache(wl), "l2": "flushed between steps (256 MiB write)",
+            "config": {"workload": WORKLOAD, "global_batch": c["M"] * world, "seq_len": c["M"],
+                       "flops_per_step": block_flops(wl, HEADLINE), "l2": "flushed between steps (256 MiB write)",
                        "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
                        "launch": "one CUDA graph per step (captured from the library calls)",
                        "eager_ms_per_step": round(sum(eager_times) / len(eager_times), 4)},
-            "roofline": roofline, "breakdown": breakdown, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": int(launches), "clocks": clk, "extra": extra,
+            "roofline": roofline, "breakdown": breakdown, "cpu_baseline": cpu, "oracle_check": check,
+            "e2e": e2e, "gpu_launches": int(launches), "clocks": clk, "extra": extra,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
 
 
-def blk_flops_cache(wl):
-    c = wl.CONFIGS["llama7b"]
-    return sum(fwd_flops(c["M"], N, K, c["r"]) + bwd_flops(c["M"], N, K, c["r"]) for _, N, K in c["linears"])
-
-
-def run_profile_case(case):
+def run_profile_case(case, block_cfg):
     """A small case of one kernel, launched three times: the gate-shaped
     linear (11008x4096, M=2048, r=64) for the GEMMs, 2^26 elements for the
-    quantizer, the 22016x8192 weight at M=16 for the small-M forward."""
+    quantizer, the 22016x8192 weight at M=16 for the small-M forward; the
+    *_block cases run each linear of one decoder block once."""
     import torch
     from bit_nf4_quantized_08_b200 import build as qbuild
     qbuild.build()
@@ -588,17 +757,18 @@ def run_profile_case(case):
     from bit_nf4_quantized_08_b200 import workloads as wl
     dev = torch.device("cuda", 0)
     if case in ("fwd_block", "dx_block"):
-        cfg = wl.CONFIGS["llama7b"]
+        cfg = wl.CONFIGS[block_cfg]
         M, r, s = cfg["M"], cfg["r"], cfg["alpha"] / cfg["r"]
         for i, (_, N, K) in enumerate(cfg["linears"]):
-            W = wl.weight(N, K, seed=0, dtype=torch.bfloat16, device=dev, index_base=16 * i)
+            W = wl.weight(N, K, seed=0, dtype=torch.bfloat16, device=dev, index_base=10 * i)
             w = Q.qlora_nf4_quantize(W)
             del W
-            inp = wl.linear_inputs(M, N, K, r, seed=0, device=dev, index_base=16 * i)
+            inp = wl.linear_inputs(M, N, K, r, seed=0, device=dev, index_base=10 * i)
             if case == "dx_block":
                 Q.qlora_linear_bwd(inp["dY"], inp["X"], w, inp["A"], inp["B"], s)
             else:
                 Q.qlora_linear_fwd(inp["X"], w, inp["A"], inp["B"], s)
+            del w, inp
     elif case in ("quantize", "dequantize"):
         W = wl.weight(1 << 13, 1 << 13, seed=0, dtype=torch.bfloat16, device=dev)
         w = Q.qlora_nf4_quantize(W)
@@ -625,26 +795,34 @@ def run_profile_case(case):
 
 
 def run_reference(args, world, rank):
-    """Reference arm: the CPU oracle, as it stands, timed on a bounded sample
-    of the same workload per step (rank 0 only)."""
+    """Reference arm: the CPU oracle, as it stands, on the host cores.  Each
+    step is the oracle's bounded sample of one linear of the block (the seven
+    in turn): full quantize + dequantize of its weight, Y and dX on 16 sampled
+    token rows, dA and dB in full.  Rank 0 only."""
     if rank != 0:
         return 0
     import torch
     from bit_nf4_quantized_08_b200 import workloads as wl
-    for _ in range(max(0, min(args.warmup, 1))):
-        oracle_sample(torch, wl)
+    from oracle import oracle as O
+    O.build()
+    nlin = len(wl.CONFIGS[HEADLINE]["linears"])
+    for i in range(max(0, min(args.warmup, 1))):
+        oracle_sample(torch, wl, HEADLINE, layers=[i % nlin])
     tot_flops, tot_s = 0, 0.0
-    desc, threads = "", 1
-    for _ in range(args.steps):
-        f, dt, desc, threads = oracle_sample(torch, wl)
-        tot_flops += f
-        tot_s += dt
+    for i in range(args.steps):
+        smp = oracle_sample(torch, wl, HEADLINE, layers=[i % nlin])
+        tot_flops += smp["flops"]
+        tot_s += smp["seconds"]
     value = tot_flops / tot_s / 1e12
+    threads = O.num_threads()
+    desc = ("per step, one linear of the block in turn (M=2048, r=64): full NF4+DQ quantize and dequantize of W, "
+            "Y and dX on 16 of 2048 token rows, dA and dB in full")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_s / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": {"workload": WORKLOAD + " (bounded CPU sample per step)"},
-            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc,
+                             "cpu_model": _cpu_model()},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0

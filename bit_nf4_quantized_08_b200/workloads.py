@@ -81,6 +81,20 @@ def linear_inputs(M: int, N: int, K: int, r: int, seed: int = 0, device="cpu", i
     return out
 
 
+def sample_rows(M: int, n: int = 64, seed: int = 0):
+    """Token rows on which outputs of a full-size layer are compared with the
+    oracle: the first and the last row plus n - 2 distinct rows drawn (seeded,
+    without replacement) from the ones in between; all rows when M <= n.
+    Returns a sorted int64 NumPy array."""
+    import numpy as np
+    if M <= n:
+        return np.arange(M, dtype=np.int64)
+    g = _gen(seed, 900, "cpu")
+    mid = torch.randperm(M - 2, generator=g)[: n - 2] + 1
+    rows = sorted({0, M - 1, *mid.tolist()})
+    return np.asarray(rows, dtype=np.int64)
+
+
 def bits(t: torch.Tensor):
     """Raw bit pattern of a bf16 tensor as a NumPy uint16 array (CPU copy)."""
     import numpy as np

@@ -49,6 +49,8 @@ def _declare(L: ctypes.CDLL) -> ctypes.CDLL:
     L.oracle_linear_fwd.argtypes = [i64, i64, i64, i32, f64, p, p, p, p, p, i64, p]
     L.oracle_linear_bwd.argtypes = [i64, i64, i64, i32, f64, p, p, p, p, p, p, i64, p, p, p]
     L.oracle_num_threads.restype = i32
+    L.oracle_set_num_threads.argtypes = [i32]
+    L.oracle_set_num_threads.restype = None
     L.oracle_t8_nearest.argtypes = [ctypes.c_float]
     L.oracle_t8_nearest.restype = i32
     return L
@@ -78,6 +80,11 @@ def _ptr(a: np.ndarray | None):
 
 def num_threads() -> int:
     return int(lib().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Threads the oracle's OpenMP loops use from now on."""
+    lib().oracle_set_num_threads(int(n))
 
 
 def normal_quantile(p: float) -> float:

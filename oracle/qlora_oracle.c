@@ -432,3 +432,14 @@ int oracle_num_threads(void)
     return 1;
 #endif
 }
+
+/* Number of OpenMP threads the oracle's loops use from now on (n >= 1);
+ * used to time the oracle on one core beside all of them. */
+void oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n >= 1) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
