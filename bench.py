@@ -182,9 +182,11 @@ class Block:
         self.layers = []
         ws_need = 0
         for li, (name, N, K) in enumerate(c["linears"]):
+            # drawn on the host (the arrays the oracle and the tests get), then moved
             base = 10 * li
-            W = wl.weight(N, K, seed=seed, dtype=torch.bfloat16, device=device, index_base=base)
-            inp = wl.linear_inputs(self.M, N, K, self.r, seed=seed, device=device, index_base=base)
+            W = wl.weight(N, K, seed=seed, dtype=torch.bfloat16, index_base=base).to(device)
+            inp = {k: v.to(device) for k, v in
+                   wl.linear_inputs(self.M, N, K, self.r, seed=seed, index_base=base).items()}
             w = Q.NF4Weight.empty(N, K, True, device)
             L = dict(name=name, N=N, K=K, W=W, w=w, X=inp["X"], dY=inp["dY"], A=inp["A"], B=inp["B"],
                      Y=torch.empty(self.M, N, dtype=torch.bfloat16, device=device),
@@ -533,9 +535,9 @@ def extras(torch, Q, wl, device, flush, peaks):
     (_, N, K), = c["linears"]
     M, r, s = c["M"], c["r"], c["alpha"] / c["r"]
     W = wl.weight(N, K, seed=0, dtype=torch.bfloat16, outlier_frac=c["outlier_frac"],
-                  outlier_std=c["outlier_std"], device=device)
+                  outlier_std=c["outlier_std"]).to(device)
     w = Q.qlora_nf4_quantize(W)
-    inp = wl.linear_inputs(M, N, K, r, seed=0, device=device)
+    inp = {k: v.to(device) for k, v in wl.linear_inputs(M, N, K, r, seed=0).items()}
     Y = torch.empty(M, N, dtype=torch.bfloat16, device=device)
     ws = torch.empty(Q.qlora_linear_workspace(M, w, r, False), dtype=torch.uint8, device=device)
     fn = lambda: Q.qlora_linear_fwd(inp["X"], w, inp["A"], inp["B"], s, Y=Y, ws=ws)  # noqa: E731
@@ -552,12 +554,12 @@ def extras(torch, Q, wl, device, flush, peaks):
     c = wl.CONFIGS["sweep"]
     (_, N, K), = c["linears"]
     r, s = c["r"], c["alpha"] / c["r"]
-    W = wl.weight(N, K, seed=0, dtype=torch.bfloat16, device=device)
+    W = wl.weight(N, K, seed=0, dtype=torch.bfloat16).to(device)
     w = Q.qlora_nf4_quantize(W)
     del W
     sweep = {}
     for M in c["Ms"]:
-        inp = wl.linear_inputs(M, N, K, r, seed=0, device=device)
+        inp = {k: v.to(device) for k, v in wl.linear_inputs(M, N, K, r, seed=0).items()}
         X, A, B = inp["X"], inp["A"], inp["B"]
         Y = torch.empty(M, N, dtype=torch.bfloat16, device=device)
         ws = torch.empty(Q.qlora_linear_workspace(M, w, r, False), dtype=torch.uint8, device=device)
@@ -574,8 +576,24 @@ def extras(torch, Q, wl, device, flush, peaks):
                          "frac_hbm": round(total / ms / 1e6 / peaks["hbm_gbs"], 3)}
     out["small_m_fwd_22016x8192_r64_cuda_graph"] = sweep
 
+    # LoRA merge of the same weight (dequantize + s B A, bf16 out)
+    A = wl.linear_inputs(1, N, K, r, seed=0)["A"].to(device)
+    B = wl.linear_inputs(1, N, K, r, seed=0)["B"].to(device)
+    Wm = torch.empty(N, K, dtype=torch.bfloat16, device=device)
+    fn = lambda: Q.qlora_lora_merge(w, A, B, s, out=Wm)  # noqa: E731
+    for _ in range(3):
+        fn()
+    g = graph_of(torch, fn)
+    ms = replay_ms(torch, g, 20, flush)
+    del g
+    mbytes = N * K * (WEIGHT_BYTES_PER_ELEM + 2) + (N + K) * r * 2
+    out["lora_merge_22016x8192_r64_cuda_graph"] = {
+        "us": round(ms * 1e3, 1), "GBps": round(mbytes / ms / 1e6, 1),
+        "frac_hbm": round(mbytes / ms / 1e6 / peaks["hbm_gbs"], 3), "algorithmic_bytes": int(mbytes)}
+    del Wm, A, B, w
+
     n = c["big_numel"]
-    Wbig = wl.weight(n // 8192, 8192, seed=0, dtype=torch.bfloat16, device=device)
+    Wbig = wl.weight(n // 8192, 8192, seed=0, dtype=torch.bfloat16).to(device)
     qb = Q.NF4Weight.empty(n // 8192, 8192, True, device)
     wsq = torch.empty(Q.qlora_nf4_quantize_workspace(n // 8192, 8192, True), dtype=torch.uint8, device=device)
     deq = torch.empty(n // 8192, 8192, dtype=torch.bfloat16, device=device)

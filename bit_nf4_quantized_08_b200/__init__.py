@@ -14,6 +14,8 @@ from .api import (  # noqa: F401
     qlora_linear_bwd,
     qlora_linear_fwd,
     qlora_linear_workspace,
+    qlora_lora_merge,
+    qlora_lora_unmerge,
     qlora_nf4_dequantize,
     qlora_nf4_encode,
     qlora_nf4_quantize,

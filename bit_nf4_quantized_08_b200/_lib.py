@@ -34,6 +34,8 @@ EXPORTS = (
     "qlora_linear_workspace",
     "qlora_linear_fwd",
     "qlora_linear_bwd",
+    "qlora_lora_merge",
+    "qlora_lora_unmerge",
     "qlora_get_last_error",
     "qlora_nf4_table",
     "qlora_nf4_encode",
@@ -43,7 +45,8 @@ EXPORTS = (
     "qlora_profile_enable",
     "qlora_profile_read",
 )
-KERNEL_KINDS = {"quantize": 0, "dequantize": 1, "fwd_gemm": 2, "dx_gemm": 3, "smallm_gemm": 4, "lora_gemm": 5}
+KERNEL_KINDS = {"quantize": 0, "dequantize": 1, "fwd_gemm": 2, "dx_gemm": 3, "smallm_gemm": 4, "lora_gemm": 5,
+                "merge": 6}
 
 
 class QloraError(RuntimeError):
@@ -97,6 +100,10 @@ def lib() -> ctypes.CDLL:
     L.qlora_linear_fwd.restype = i32
     L.qlora_linear_bwd.argtypes = [vp, vp, i64, W, vp, vp, i32, f32, vp, vp, vp, vp, sz, vp]
     L.qlora_linear_bwd.restype = i32
+    L.qlora_lora_merge.argtypes = [W, vp, vp, i32, f32, vp, vp]
+    L.qlora_lora_merge.restype = i32
+    L.qlora_lora_unmerge.argtypes = [vp, i64, i64, vp, vp, i32, f32, vp, vp]
+    L.qlora_lora_unmerge.restype = i32
     L.qlora_get_last_error.argtypes = [vp]
     L.qlora_get_last_error.restype = i32
     L.qlora_nf4_table.argtypes = [vp]

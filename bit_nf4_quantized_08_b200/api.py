@@ -181,6 +181,29 @@ def qlora_linear_bwd(dY: torch.Tensor, X: torch.Tensor, w: NF4Weight, A: torch.T
     return dX, dA, dB
 
 
+def qlora_lora_merge(w: NF4Weight, A: torch.Tensor, B: torch.Tensor, scale: float,
+                     out: torch.Tensor | None = None) -> torch.Tensor:
+    """W_merged = bf16(dequant(W) + scale B A), the dense bf16 weight with the
+    adapter folded in."""
+    if out is None:
+        out = torch.empty(w.rows, w.cols, dtype=torch.bfloat16, device=w.codes.device)
+    cw = w.c_struct()
+    check(lib().qlora_lora_merge(ctypes.byref(cw), _ptr(A), _ptr(B), A.shape[0], float(scale), _ptr(out),
+                                 _stream()), "qlora_lora_merge")
+    return out
+
+
+def qlora_lora_unmerge(W_merged: torch.Tensor, A: torch.Tensor, B: torch.Tensor, scale: float,
+                       out: torch.Tensor | None = None) -> torch.Tensor:
+    """bf16(W_merged - scale B A): the base weight back from a merged one."""
+    rows, cols = W_merged.shape
+    if out is None:
+        out = torch.empty(rows, cols, dtype=torch.bfloat16, device=W_merged.device)
+    check(lib().qlora_lora_unmerge(_ptr(W_merged), rows, cols, _ptr(A), _ptr(B), A.shape[0], float(scale),
+                                   _ptr(out), _stream()), "qlora_lora_unmerge")
+    return out
+
+
 def qlora_get_last_error(stream: torch.cuda.Stream | None = None) -> int:
     return int(lib().qlora_get_last_error(_stream(stream)))
 

@@ -13,6 +13,7 @@
 #include "gemm.cuh"
 #include "internal.h"
 #include "linear.cuh"
+#include "merge.cuh"
 #include "nf4.cuh"
 #include "quantize.cuh"
 
@@ -183,6 +184,53 @@ static qlora_status check_linear(int64_t M, const qlora_nf4_weight* w, int32_t r
     return QLORA_OK;
 }
 
+// LoRA merge (base = NF4 weight) or unmerge (base = dense bf16 weight):
+// out = bf16(base + scale * B A), one CTA per 128 x 128 tile.
+static qlora_status lora_merge_impl(const qlora_nf4_weight* w, const void* dense, int64_t N, int64_t K,
+                                    const void* A, const void* B, int32_t r, float scale, void* out,
+                                    cudaStream_t s) {
+    MergeParams p;
+    memset(&p, 0, sizeof(p));
+    if (!map_bf16(&p.tmB, B, (uint64_t)r, (uint64_t)N, 128)) return QLORA_ERR_CUDA;
+    if (!map_bf16(&p.tmA, A, (uint64_t)K, (uint64_t)r, 64)) return QLORA_ERR_CUDA;
+    if (w) {
+        p.codes = w->codes;
+        p.dq = w->double_quant;
+        p.absmax = w->absmax;
+        p.q8 = w->absmax_q8;
+        p.c1 = w->absmax_scale;
+        p.offset = w->absmax_offset;
+    } else {
+        p.dense = static_cast<const uint16_t*>(dense);
+    }
+    p.out = static_cast<uint16_t*>(out);
+    p.N = (int)N;
+    p.K = (int)K;
+    p.r_chunks = (r + 63) / 64;
+    p.scale = scale;
+    p.timeout_ns = wait_timeout_ns();
+    const int smem = MergeShape::smem(p.r_chunks);
+    if (cudaFuncSetAttribute(k_lora_merge, cudaFuncAttributeMaxDynamicSharedMemorySize, MergeShape::MAX_SMEM) !=
+        cudaSuccess)
+        return QLORA_ERR_CUDA;
+    dim3 grid((unsigned)((K + 127) / 128), (unsigned)((N + 127) / 128));
+    ProfileScope ps(QLORA_KERNEL_MERGE, s);
+    note_launch();
+    k_lora_merge<<<grid, MergeShape::THREADS, smem, s>>>(p);
+    return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+static qlora_status check_merge(int64_t N, int64_t K, const void* A, const void* B, int32_t r,
+                                const void* out) {
+    if (N < 0 || K < 0 || r < 1) return QLORA_ERR_INVALID_ARG;
+    if (N == 0 || K == 0) return QLORA_OK;
+    if (K % 64 != 0 || N % 8 != 0 || r % 8 != 0 || r > 256) return QLORA_ERR_UNSUPPORTED;
+    if (N >= ((int64_t)1 << 31) || K >= ((int64_t)1 << 31) || N > kMaxElems / K) return QLORA_ERR_UNSUPPORTED;
+    if (!A || !aligned(A, 16) || !B || !aligned(B, 16) || !out || !aligned(out, 16))
+        return QLORA_ERR_INVALID_ARG;
+    return QLORA_OK;
+}
+
 }  // namespace qlora
 
 using namespace qlora;
@@ -305,6 +353,26 @@ qlora_status qlora_linear_bwd(const void* dY, const void* X, int64_t M, const ql
     if (!ws || !aligned(ws, 16) || ws_bytes < need) return QLORA_ERR_INVALID_ARG;
     LinearArgs a{M, w->rows, w->cols, r, scale, w};
     return linear_bwd_impl(dY, X, a, A, B, dX, dA, dB, ws, ws_bytes,
+                           reinterpret_cast<cudaStream_t>(stream));
+}
+
+qlora_status qlora_lora_merge(const qlora_nf4_weight* w, const void* A, const void* B, int32_t r,
+                              float scale, void* W_merged, qlora_stream_t stream) {
+    qlora_status st = check_weight(w, true);
+    if (st != QLORA_OK) return st;
+    st = check_merge(w->rows, w->cols, A, B, r, W_merged);
+    if (st != QLORA_OK || w->rows * w->cols == 0) return st;
+    return lora_merge_impl(w, nullptr, w->rows, w->cols, A, B, r, scale, W_merged,
+                           reinterpret_cast<cudaStream_t>(stream));
+}
+
+qlora_status qlora_lora_unmerge(const void* W_merged, int64_t rows, int64_t cols, const void* A,
+                                const void* B, int32_t r, float scale, void* W_out,
+                                qlora_stream_t stream) {
+    qlora_status st = check_merge(rows, cols, A, B, r, W_out);
+    if (st != QLORA_OK || rows * cols == 0) return st;
+    if (!W_merged || !aligned(W_merged, 16)) return QLORA_ERR_INVALID_ARG;
+    return lora_merge_impl(nullptr, W_merged, rows, cols, A, B, r, -scale, W_out,
                            reinterpret_cast<cudaStream_t>(stream));
 }
 

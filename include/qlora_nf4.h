@@ -198,6 +198,37 @@ qlora_status qlora_linear_bwd(const void *dY, const void *X, int64_t M, const ql
                               qlora_stream_t stream);
 
 /*
+ * LoRA merge (QLoRA tutorial "11.3 QLoRA", pitfalls: merging the adapter
+ * into a 4-bit base adds error, so the base is dequantized first; LoRA
+ * reproduction blog, "LoRA formula and tensor shapes": the adapter adds
+ * (alpha/r) B A to W0):
+ *   W_merged[n,k] = bf16_round_nearest_even( w'[n,k] + scale * sum_j B[n,j] A[j,k] )
+ *   w  the quantized frozen weight [N, K] (w' its doubleDequant bf16 values),
+ *   A [r, K] bf16, B [N, r] bf16, W_merged [N, K] bf16 (written).
+ * The rank-r sum accumulates in fp32 on the tensor cores; the base is added
+ * with one fused multiply-add in fp32 and the result rounded once to bf16.
+ * Requires K % 64 == 0, N % 8 == 0, 1 <= r <= 256, r % 8 == 0 (UNSUPPORTED
+ * otherwise); r < 1 is INVALID_ARG.  Pointers 16-byte aligned.  Async on
+ * `stream`; writes only W_merged.  The merged dense weight serves inference
+ * without the adapter path (Y = X W_merged^T).
+ */
+qlora_status qlora_lora_merge(const qlora_nf4_weight *w, const void *A, const void *B, int32_t r,
+                              float scale, void *W_merged, qlora_stream_t stream);
+
+/*
+ * LoRA unmerge, the inverse of qlora_lora_merge on a dense bf16 weight:
+ *   W_out[n,k] = bf16_round_nearest_even( W_merged[n,k] - scale * sum_j B[n,j] A[j,k] )
+ * W_merged, W_out [rows, cols] bf16 (W_out written; it may not overlap
+ * W_merged), A [r, cols], B [rows, r] bf16.  It gives back the base weight
+ * (up to the bf16 rounding of the merge) so that the frozen base and the
+ * adapter path can be used apart again.  Same requirements as
+ * qlora_lora_merge.
+ */
+qlora_status qlora_lora_unmerge(const void *W_merged, int64_t rows, int64_t cols, const void *A,
+                                const void *B, int32_t r, float scale, void *W_out,
+                                qlora_stream_t stream);
+
+/*
  * Synchronizes `stream`, then returns (and clears) the device status word of
  * the current device: QLORA_ERR_TIMEOUT if a bounded in-kernel wait ran out
  * since the last call, QLORA_ERR_CUDA if the stream reports an error,
@@ -260,7 +291,8 @@ typedef enum {
     QLORA_KERNEL_DX_GEMM = 3,   /* backward dX dequant-GEMM */
     QLORA_KERNEL_SMALLM_GEMM = 4, /* forward dequant-GEMM, M <= 64 */
     QLORA_KERNEL_LORA_GEMM = 5, /* rank-r LoRA GEMMs (U, G, dA, dB) */
-    QLORA_KERNEL_KINDS = 6
+    QLORA_KERNEL_MERGE = 6,     /* LoRA merge / unmerge */
+    QLORA_KERNEL_KINDS = 7
 } qlora_kernel_kind;
 
 uint64_t qlora_kernel_launches(void);

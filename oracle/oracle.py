@@ -51,6 +51,8 @@ def _declare(L: ctypes.CDLL) -> ctypes.CDLL:
     L.oracle_num_threads.restype = i32
     L.oracle_set_num_threads.argtypes = [i32]
     L.oracle_set_num_threads.restype = None
+    L.oracle_lora_merge.argtypes = [i64, i64, i32, f64, i32, p, p, p, p, p]
+    L.oracle_lora_merge.restype = None
     L.oracle_t8_nearest.argtypes = [ctypes.c_float]
     L.oracle_t8_nearest.restype = i32
     return L
@@ -211,3 +213,18 @@ def linear_bwd(dY: np.ndarray, X: np.ndarray, W: np.ndarray, A: np.ndarray, B: n
     lib().oracle_linear_bwd(M, N, K, r, float(s), _ptr(dY), _ptr(X), _ptr(W), _ptr(A), _ptr(B),
                             _ptr(rows), nrows, _ptr(dX), _ptr(dA), _ptr(dB))
     return dX, dA, dB
+
+
+def lora_merge(W: np.ndarray, A: np.ndarray, B: np.ndarray, s: float, sign: int = 1,
+               want_exact: bool = False):
+    """bf16 bits of W + sign * s * B A, rounded once from fp64 (merge: W the
+    dequantized base, sign +1; unmerge: W the merged weight, sign -1).
+    With ``want_exact`` also returns the fp64 value before the rounding."""
+    W, A, B = map(_bits, (W, A, B))
+    N, K = W.shape
+    r = A.shape[0]
+    assert A.shape == (r, K) and B.shape == (N, r)
+    out = np.zeros((N, K), np.uint16)
+    exact = np.zeros((N, K), np.float64) if want_exact else None
+    lib().oracle_lora_merge(N, K, r, float(s), int(sign), _ptr(W), _ptr(A), _ptr(B), _ptr(out), _ptr(exact))
+    return (out, exact) if want_exact else out

@@ -424,6 +424,54 @@ void oracle_linear_bwd(int64_t M, int64_t N, int64_t K, int r, double s,
     free(U);
 }
 
+/* ------------------------------------------------------------------ */
+/* LoRA merge / unmerge                                                 */
+/* ------------------------------------------------------------------ */
+
+/* double -> bf16 with one round-to-nearest-even step: the value is scaled by
+ * a power of two so that its bf16 unit in the last place becomes 1 (8
+ * significant bits; below 2^-126 the subnormal spacing 2^-133), rounded with
+ * nearbyint (ties to even in the default rounding mode) and scaled back;
+ * both scalings are exact.  The result has at most 8 significant bits, so
+ * the conversion to fp32 is exact and its top 16 bits are the bf16 code. */
+static uint16_t f64_to_bf16_rne(double x)
+{
+    if (x == 0.0) return signbit(x) ? 0x8000u : 0u;
+    double ax = fabs(x);
+    int e;
+    frexp(ax, &e);          /* ax = m 2^e, m in [1/2, 1) */
+    int ulp_exp = e - 8;
+    if (ulp_exp < -133) ulp_exp = -133;
+    double v = ldexp(nearbyint(ldexp(ax, -ulp_exp)), ulp_exp);
+    uint16_t h = (uint16_t)(bits_from_f32((float)v) >> 16);
+    return signbit(x) ? (uint16_t)(h | 0x8000u) : h;
+}
+
+/*
+ * LoRA merge ([P2] pitfalls: dequantize the 4-bit base before merging; [P5]
+ * "LoRA formula and tensor shapes": the adapter adds (alpha/r) B A to W0):
+ *   out[n,k] = bf16_rne( W[n,k] + sign * s * sum_j B[n,j] A[j,k] )
+ * W [N,K] (the dequantized base for a merge, the merged weight for an
+ * unmerge with sign = -1), A [r,K], B [N,r]: bf16 bits.  The sum runs in
+ * fp64 in index order and the value is rounded once.  `exact` (optional)
+ * receives the fp64 value before the rounding.
+ */
+void oracle_lora_merge(int64_t N, int64_t K, int r, double s, int sign, const uint16_t *W,
+                       const uint16_t *A, const uint16_t *B, uint16_t *out, double *exact)
+{
+    #pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < K; ++k) {
+            double acc = 0.0;
+            for (int j = 0; j < r; ++j)
+                acc += (double)bf16_to_f32(B[n * r + j]) * (double)bf16_to_f32(A[(int64_t)j * K + k]);
+            double v = (double)bf16_to_f32(W[n * K + k]) + (double)sign * s * acc;
+            out[n * K + k] = f64_to_bf16_rne(v);
+            if (exact) exact[n * K + k] = v;
+        }
+    }
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP

@@ -105,6 +105,27 @@ def test_linear_rejects(Q):
     assert f(None, 0, ctypes.byref(w), FAKE, FAKE, 8, 2.0, None, FAKE, big, None) == 0
 
 
+def test_merge_rejects(Q):
+    from bit_nf4_quantized_08_b200._lib import lib, QLORA_ERR_INVALID_ARG, QLORA_ERR_UNSUPPORTED
+    L = lib()
+    m, u = L.qlora_lora_merge, L.qlora_lora_unmerge
+    w = _w(256, 256)
+    assert m(ctypes.byref(w), FAKE, FAKE, 12, 2.0, FAKE, None) == QLORA_ERR_UNSUPPORTED
+    assert m(ctypes.byref(w), FAKE, FAKE, 264, 2.0, FAKE, None) == QLORA_ERR_UNSUPPORTED
+    assert m(ctypes.byref(w), FAKE, FAKE, 0, 2.0, FAKE, None) == QLORA_ERR_INVALID_ARG
+    assert m(ctypes.byref(_w(256, 200)), FAKE, FAKE, 8, 2.0, FAKE, None) == QLORA_ERR_UNSUPPORTED
+    assert m(ctypes.byref(_w(260, 256)), FAKE, FAKE, 8, 2.0, FAKE, None) == QLORA_ERR_UNSUPPORTED
+    assert m(ctypes.byref(w), None, FAKE, 8, 2.0, FAKE, None) == QLORA_ERR_INVALID_ARG
+    assert m(ctypes.byref(w), FAKE, FAKE, 8, 2.0, FAKE + 8, None) == QLORA_ERR_INVALID_ARG
+    assert m(None, FAKE, FAKE, 8, 2.0, FAKE, None) == QLORA_ERR_INVALID_ARG
+    assert u(FAKE, 256, 256, FAKE, FAKE, 12, 2.0, FAKE, None) == QLORA_ERR_UNSUPPORTED
+    assert u(None, 256, 256, FAKE, FAKE, 8, 2.0, FAKE, None) == QLORA_ERR_INVALID_ARG
+    assert u(FAKE, -1, 256, FAKE, FAKE, 8, 2.0, FAKE, None) == QLORA_ERR_INVALID_ARG
+    assert u(FAKE, 256, 100, FAKE, FAKE, 8, 2.0, FAKE, None) == QLORA_ERR_UNSUPPORTED
+    # empty: valid, nothing to do
+    assert u(None, 0, 256, FAKE, FAKE, 8, 2.0, FAKE, None) == 0
+
+
 def test_linear_workspace_queries(Q):
     from bit_nf4_quantized_08_b200._lib import lib
     L = lib()

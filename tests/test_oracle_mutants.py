@@ -28,6 +28,10 @@ MUTANTS = [
     ("bf16_truncates", "uint32_t rounded = u + 0x7FFFu + lsb;", "uint32_t rounded = u + 0u * lsb;"),
     ("absmax_not_abs", "float av = fabsf(v);", "float av = v;"),
     ("t8_scale_128", "out[k] = (float)(k - 127) / 127.0f;", "out[k] = (float)(k - 127) / 128.0f;"),
+    ("merge_ignores_sign", "(double)sign * s * acc;", "s * acc;"),
+    ("merge_transposed_A", "* (double)bf16_to_f32(A[(int64_t)j * K + k]);\n            double v",
+     "* (double)bf16_to_f32(A[k * r + j]);\n            double v"),
+    ("merge_rounds_down", "ldexp(nearbyint(ldexp(ax, -ulp_exp)), ulp_exp)", "ldexp(floor(ldexp(ax, -ulp_exp)), ulp_exp)"),
 ]
 
 PINS = [
@@ -45,6 +49,7 @@ PINS = [
     pins.test_fwd_vs_torch_linear,
     pins.test_bwd_vs_autograd,
     pins.test_zero_B_noop_and_zero_dA,
+    pins.test_lora_merge_brute_force,
 ]
 
 

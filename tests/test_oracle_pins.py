@@ -416,3 +416,87 @@ def test_q8_ties_go_low(O):
             assert O.t8_nearest(float(np.nextafter(np.float32(m), np.float32(2)))) == k + 1
             checked += 1
     assert checked > 100
+
+
+# ---------------------------------------------------------------------------
+# LoRA merge / unmerge
+# ---------------------------------------------------------------------------
+
+def _bf16_value(h: int) -> Fraction:
+    """Exact value of a finite bf16 code."""
+    return Fraction(float(np.array([h << 16], np.uint32).view(np.float32)[0]))
+
+
+def _bf16_nearest_even(x: Fraction) -> int:
+    """Brute force: the finite bf16 code nearest to the exact rational x, ties
+    to the code with an even last bit (positive codes enumerated; the sign is
+    symmetric)."""
+    neg = x < 0
+    ax = -x if neg else x
+    best, bd = None, None
+    # candidates: every positive finite code (0x0000 .. 0x7F7F); the search
+    # narrows to the two around ax through the order of the codes
+    lo, hi = 0, 0x7F7F
+    while hi - lo > 1:
+        mid = (lo + hi) // 2
+        if _bf16_value(mid) <= ax:
+            lo = mid
+        else:
+            hi = mid
+    for h in (lo, hi):
+        d = abs(_bf16_value(h) - ax)
+        if bd is None or d < bd or (d == bd and h % 2 == 0):
+            best, bd = h, d
+    return best | (0x8000 if neg and best != 0 else 0)
+
+
+def _bits_of(vals):
+    return (np.asarray(vals, np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+
+def test_lora_merge_brute_force(O):
+    """Merge and unmerge against exact rational arithmetic: every output is
+    the bf16 code nearest to W + sign s sum_j B A (ties to even), on random
+    bf16 inputs plus constructed exact ties (normal and subnormal)."""
+    rng = np.random.default_rng(5)
+    N, K, r = 6, 64, 8
+    W = _bits_of(rng.normal(0, 0.02, (N, K)))
+    A = _bits_of(rng.normal(0, 1 / r, (r, K)))
+    B = _bits_of(rng.normal(0, 0.05, (N, r)))
+    # row 0: exact ties (s = 2).  W = 1.0 and 1.0078125 with s B A = 2^-8,
+    # half a unit in the last place of both; W = 0 with s B A = 1.5 * 2^-133,
+    # halfway between the two smallest subnormals
+    # (row 1 carries the subnormal case, so that its tiny B entry meets no
+    # other term that would land on a midpoint)
+    B[0:2, :] = 0
+    A[:, :4] = 0
+    W[0, 0] = 0x3F80
+    W[0, 1] = 0x3F81
+    W[1, 2] = 0x0000
+    B[0, 0] = _bits_of([2.0 ** -4])[0]
+    A[0, 0] = _bits_of([2.0 ** -5])[0]
+    A[0, 1] = _bits_of([2.0 ** -5])[0]
+    B[1, 1] = _bits_of([2.0 ** -67])[0]
+    A[1, 2] = _bits_of([1.5 * 2.0 ** -67])[0]
+    s = 2.0
+    for sign in (1, -1):
+        got = O.lora_merge(W, A, B, s, sign)
+        Wf, Af, Bf = (np.array(x, np.uint32) for x in (W, A, B))
+        for n in range(N):
+            for k in range(K):
+                acc = sum(_bf16_value(int(Bf[n, j])) * _bf16_value(int(Af[j, k])) for j in range(r))
+                x = _bf16_value(int(Wf[n, k])) + sign * Fraction(s) * acc
+                assert int(got[n, k]) == _bf16_nearest_even(x), (sign, n, k)
+    got = O.lora_merge(W, A, B, s, 1)
+    assert got[0, 0] == 0x3F80   # 1 + 2^-8: tie, to the even code (1.0)
+    assert got[0, 1] == 0x3F82   # 1.0078125 + 2^-8: tie, to the even code
+    assert got[1, 2] == 0x0002   # 1.5 * 2^-133: tie, to the even subnormal
+
+
+def test_lora_merge_zero_B_is_identity(O):
+    """B = 0 (the adapter's initial state): the merged weight is the base."""
+    rng = np.random.default_rng(6)
+    W = _bits_of(rng.normal(0, 0.02, (16, 128)))
+    A = _bits_of(rng.normal(0, 0.1, (8, 128)))
+    B = np.zeros((16, 8), np.uint16)
+    np.testing.assert_array_equal(O.lora_merge(W, A, B, 2.0), W)
