@@ -44,9 +44,11 @@ METRIC = "fused NF4-dequant+LoRA linear fwd/bwd TFLOP/s and weight GB/s vs B200 
 HEADLINE = "llama65b"
 WORKLOADS = {
     "llama65b": "llama65b-decoder-block: 7 NF4+DQ linears (q,k,v,o 8192x8192; gate,up 22016x8192; "
-                "down 8192x22016), M=2048 (1 x 2048 tokens), r=64, alpha=16; quantize+fwd+bwd",
+                "down 8192x22016) with a LoRA adapter each, M=2048 (1 x 2048 tokens), r=64, alpha=16; "
+                "quantize+fwd+bwd; q/k/v and gate/up as fused projections sharing their input",
     "llama7b": "llama7b-decoder-block: 7 NF4+DQ linears (q,k,v,o 4096x4096; gate,up 11008x4096; "
-               "down 4096x11008), M=2048 (4 x 512 tokens), r=64, alpha=16; quantize+fwd+bwd",
+               "down 4096x11008) with a LoRA adapter each, M=2048 (4 x 512 tokens), r=64, alpha=16; "
+               "quantize+fwd+bwd; q/k/v and gate/up as fused projections sharing their input",
 }
 WORKLOAD = WORKLOADS[HEADLINE]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -64,7 +66,7 @@ def parse():
     ap.add_argument("--profile-case", choices=["fwd", "dx", "quantize", "dequantize", "smallm",
                                                "fwd_block", "dx_block"],
                     help="run one small case three times, untimed (for ncu captures); "
-                         "*_block runs the seven block linears once each")
+                         "*_block runs each projection of one decoder block once")
     ap.add_argument("--block", choices=sorted(WORKLOADS), default=HEADLINE,
                     help="decoder block of the *_block profile cases")
     return ap.parse_args()
@@ -172,45 +174,51 @@ def load_traffic(kind):
 # ---------------------------------------------------------------------------
 
 class Block:
-    """The seven linears of one decoder block with every buffer preallocated.
-    Layer li draws its tensors from generator indices 10*li + (0..9)."""
+    """One decoder block with every buffer preallocated.  fused=True: the
+    block as its four projections, q/k/v and gate/up each one NF4 weight
+    whose row segments share the input (one adapter per segment, one
+    qlora_fused_linear call per projection); fused=False: the seven linears
+    as separate weights and calls.  Group g draws its tensors from generator
+    indices 10*g + (0..9) on the host (the oracle's arrays)."""
 
-    def __init__(self, torch, Q, wl, device, cfg=HEADLINE, seed=0):
+    def __init__(self, torch, Q, wl, device, cfg=HEADLINE, seed=0, fused=True):
         c = wl.CONFIGS[cfg]
-        self.cfg = cfg
+        self.cfg, self.fused = cfg, fused
         self.M, self.r, self.s = c["M"], c["r"], c["alpha"] / c["r"]
         self.layers = []
         ws_need = 0
-        for li, (name, N, K) in enumerate(c["linears"]):
-            # drawn on the host (the arrays the oracle and the tests get), then moved
-            base = 10 * li
+        for gi, (name, nseg, S, K) in enumerate(block_groups(wl, cfg, fused)):
+            base = 10 * gi
+            N = nseg * S
             W = wl.weight(N, K, seed=seed, dtype=torch.bfloat16, index_base=base).to(device)
             inp = {k: v.to(device) for k, v in
-                   wl.linear_inputs(self.M, N, K, self.r, seed=seed, index_base=base).items()}
+                   wl.fused_inputs(self.M, nseg, S, K, self.r, seed=seed, index_base=base).items()}
             w = Q.NF4Weight.empty(N, K, True, device)
-            L = dict(name=name, N=N, K=K, W=W, w=w, X=inp["X"], dY=inp["dY"], A=inp["A"], B=inp["B"],
+            L = dict(name=name, nseg=nseg, S=S, N=N, K=K, W=W, w=w, X=inp["X"], dY=inp["dY"], A=inp["A"],
+                     B=inp["B"],
                      Y=torch.empty(self.M, N, dtype=torch.bfloat16, device=device),
                      dX=torch.empty(self.M, K, dtype=torch.bfloat16, device=device),
-                     dA=torch.empty(self.r, K, dtype=torch.float32, device=device),
+                     dA=torch.empty(nseg * self.r, K, dtype=torch.float32, device=device),
                      dB=torch.empty(N, self.r, dtype=torch.float32, device=device))
             self.layers.append(L)
         for L in self.layers:
             ws_need = max(ws_need, Q.qlora_nf4_quantize_workspace(L["N"], L["K"], True),
-                          Q.qlora_linear_workspace(self.M, L["w"], self.r, False),
-                          Q.qlora_linear_workspace(self.M, L["w"], self.r, True))
+                          Q.qlora_fused_linear_workspace(self.M, L["w"], L["nseg"], self.r, False),
+                          Q.qlora_fused_linear_workspace(self.M, L["w"], L["nseg"], self.r, True))
         self.ws = torch.empty(ws_need, dtype=torch.uint8, device=device)
         self.Q = Q
         self.flops = block_flops(wl, cfg)
-        self.fwd_gemm_flops = sum(2 * self.M * L["N"] * L["K"] + 2 * self.M * self.r * L["N"] for L in self.layers)
-        self.dx_gemm_flops = sum(2 * self.M * L["N"] * L["K"] + 2 * self.M * self.r * L["K"] for L in self.layers)
+        M, r = self.M, self.r
+        self.fwd_gemm_flops = sum(2 * M * L["N"] * L["K"] + 2 * M * r * L["N"] for L in self.layers)
+        self.dx_gemm_flops = sum(2 * M * L["N"] * L["K"] + 2 * M * L["nseg"] * r * L["K"] for L in self.layers)
         self.quant_bytes = sum(L["N"] * L["K"] * (2 + WEIGHT_BYTES_PER_ELEM) for L in self.layers)
         # LoRA skinny GEMMs per step: forward U; backward U and G; dA and dB
-        M, r = self.M, self.r
-        self.lora_bytes = sum(
-            (2 * M * L["K"] + 2 * r * L["K"] + 2 * M * r)
-            + (2 * M * L["K"] + 2 * r * L["K"] + 2 * M * L["N"] + 2 * L["N"] * r + 4 * M * r)
-            + (2 * M * L["K"] + 2 * M * L["N"] + 4 * M * r + 4 * r * L["K"] + 4 * L["N"] * r)
-            for L in self.layers)
+        self.lora_bytes = 0
+        for L in self.layers:
+            rt, N, K = L["nseg"] * r, L["N"], L["K"]
+            self.lora_bytes += ((2 * M * K + 2 * rt * K + 2 * M * rt)
+                                + (2 * M * K + 2 * rt * K + 2 * M * N + 2 * N * r + 4 * M * rt)
+                                + (2 * M * K + 2 * M * N + 4 * M * rt + 4 * rt * K + 4 * N * r))
 
     def step(self, adapter=True):
         Q, ws = self.Q, self.ws
@@ -218,13 +226,21 @@ class Block:
             Q.qlora_nf4_quantize(L["W"], True, out=L["w"], ws=ws)
         for L in self.layers:
             A, B = (L["A"], L["B"]) if adapter else (None, None)
-            Q.qlora_linear_fwd(L["X"], L["w"], A, B, self.s, Y=L["Y"], ws=ws)
+            Q.qlora_fused_linear_fwd(L["X"], L["w"], L["nseg"], A, B, self.s, Y=L["Y"], ws=ws)
         for L in reversed(self.layers):
             if adapter:
-                Q.qlora_linear_bwd(L["dY"], L["X"], L["w"], L["A"], L["B"], self.s, dX=L["dX"], dA=L["dA"],
-                                   dB=L["dB"], ws=ws)
+                Q.qlora_fused_linear_bwd(L["dY"], L["X"], L["w"], L["nseg"], L["A"], L["B"], self.s, dX=L["dX"],
+                                         dA=L["dA"], dB=L["dB"], ws=ws)
             else:
-                Q.qlora_linear_bwd(L["dY"], L["X"], L["w"], None, None, self.s, dX=L["dX"], ws=ws)
+                Q.qlora_fused_linear_bwd(L["dY"], L["X"], L["w"], L["nseg"], None, None, self.s, dX=L["dX"],
+                                         ws=ws)
+
+
+def block_groups(wl, cfg, fused=True):
+    """(name, nseg, rows per segment, K) of the block's projections."""
+    if fused:
+        return wl.FUSED_GROUPS[cfg]
+    return [(name, 1, N, K) for name, N, K in wl.CONFIGS[cfg]["linears"]]
 
 
 def block_flops(wl, cfg):
@@ -348,9 +364,9 @@ def e2e_measure(torch, blk, steps, flush, barrier, world, device):
                                         hs), "qlora_nf4_quantize")
         for i, L in enumerate(layers):
             cur.wait_event(ev_in[(i, "X")])
-            call(lib.qlora_linear_fwd(L["X"].data_ptr(), M, ctypes.byref(cws[i]), L["A"].data_ptr(),
-                                      L["B"].data_ptr(), r, ctypes.c_float(s), L["Y"].data_ptr(), ws, ws_bytes,
-                                      hs), "qlora_linear_fwd")
+            call(lib.qlora_fused_linear_fwd(L["X"].data_ptr(), M, ctypes.byref(cws[i]), L["nseg"],
+                                            L["A"].data_ptr(), L["B"].data_ptr(), r, ctypes.c_float(s),
+                                            L["Y"].data_ptr(), ws, ws_bytes, hs), "qlora_fused_linear_fwd")
             ev_fwd[i].record(cur)
             down.wait_event(ev_fwd[i])
             with torch.cuda.stream(down):
@@ -358,10 +374,10 @@ def e2e_measure(torch, blk, steps, flush, barrier, world, device):
         for i in reversed(range(len(layers))):
             L = layers[i]
             cur.wait_event(ev_in[(i, "dY")])
-            call(lib.qlora_linear_bwd(L["dY"].data_ptr(), L["X"].data_ptr(), M, ctypes.byref(cws[i]),
-                                      L["A"].data_ptr(), L["B"].data_ptr(), r, ctypes.c_float(s),
-                                      L["dX"].data_ptr(), L["dA"].data_ptr(), L["dB"].data_ptr(), ws, ws_bytes,
-                                      hs), "qlora_linear_bwd")
+            call(lib.qlora_fused_linear_bwd(L["dY"].data_ptr(), L["X"].data_ptr(), M, ctypes.byref(cws[i]),
+                                            L["nseg"], L["A"].data_ptr(), L["B"].data_ptr(), r, ctypes.c_float(s),
+                                            L["dX"].data_ptr(), L["dA"].data_ptr(), L["dB"].data_ptr(), ws,
+                                            ws_bytes, hs), "qlora_fused_linear_bwd")
             ev_bwd[i].record(cur)
             down.wait_event(ev_bwd[i])
             with torch.cuda.stream(down):
@@ -381,8 +397,8 @@ def e2e_measure(torch, blk, steps, flush, barrier, world, device):
                                L[k].cpu().view(torch.int16 if L[k].dtype == torch.bfloat16 else torch.int32))
     return {"value": round(whole_job_tflops(blk.flops, world, ms), 2), "unit": "TFLOP/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms, 3),
-            "method": "C ABI entry points called with raw device pointers (ctypes); W, X, dY of the 7 linears "
-                      "copied in from pinned host memory on one stream in the order of use, Y, dX, dA, dB "
+            "method": "C ABI entry points called with raw device pointers (ctypes); W, X, dY of the block's "
+                      "projections copied in from pinned host memory on one stream in the order of use, Y, dX, dA, dB "
                       "copied out to pinned host memory on another as each call ends, all inside the timed "
                       "region; the copied-out results equal the device results"}
 
@@ -403,13 +419,13 @@ def _cpu_model():
     return None
 
 
-def oracle_sample(torch, wl, cfg, layers=None, rows_n=16, seed=0):
+def oracle_sample(torch, wl, cfg, layers=None, rows_n=16, seed=0, fused=True):
     """The oracle on a bounded sample of the block step: for each selected
-    linear (default: all seven), full NF4+DQ quantize and dequantize of W,
-    Y and dX on rows_n sampled token rows, dA and dB in full (all M rows).
-    Input generation is not timed.  Returns a dict with the sample's flops,
-    its seconds (quantize/dequantize and the products separately), the
-    sampled rows and, per layer, the oracle's outputs."""
+    projection (default: all of them), full NF4+DQ quantize and dequantize
+    of its weight, Y and dX on rows_n sampled token rows, dA and dB in full
+    (all M rows).  Input generation is not timed.  Returns a dict with the
+    sample's flops, its seconds (quantize/dequantize and the products
+    separately), the sampled rows and, per projection, the oracle's outputs."""
     from oracle import oracle as O
     O.build()
     c = wl.CONFIGS[cfg]
@@ -417,12 +433,13 @@ def oracle_sample(torch, wl, cfg, layers=None, rows_n=16, seed=0):
     rows = wl.sample_rows(M, rows_n, seed=seed)
     R = rows.size
     out = {"flops": 0, "quant_s": 0.0, "gemm_s": 0.0, "rows": rows, "layers": {}}
-    for li, (name, N, K) in enumerate(c["linears"]):
-        if layers is not None and li not in layers:
+    for gi, (name, nseg, S, K) in enumerate(block_groups(wl, cfg, fused)):
+        if layers is not None and gi not in layers:
             continue
-        base = 10 * li
+        base = 10 * gi
+        N = nseg * S
         W = wl.weight(N, K, seed=seed, dtype=torch.bfloat16, index_base=base)
-        inp = wl.linear_inputs(M, N, K, r, seed=seed, index_base=base)
+        inp = wl.fused_inputs(M, nseg, S, K, r, seed=seed, index_base=base)
         Xb, dYb, Ab, Bb = (wl.bits(inp[k]) for k in ("X", "dY", "A", "B"))
         Wbits = wl.bits(W).reshape(-1)
         del W, inp
@@ -430,16 +447,16 @@ def oracle_sample(torch, wl, cfg, layers=None, rows_n=16, seed=0):
         q = O.nf4_quantize(Wbits, double_quant=True)
         Wd = O.nf4_dequantize(N * K, q).reshape(N, K)
         t1 = time.perf_counter()
-        Y = O.linear_fwd(Xb, Wd, Ab, Bb, s, rows=rows)
-        dX, dA, dB = O.linear_bwd(dYb, Xb, Wd, Ab, Bb, s, rows=rows)
+        Y = O.fused_linear_fwd(Xb, Wd, Ab, Bb, s, nseg, rows=rows)
+        dX, dA, dB = O.fused_linear_bwd(dYb, Xb, Wd, Ab, Bb, s, nseg, rows=rows)
         t2 = time.perf_counter()
         out["quant_s"] += t1 - t0
         out["gemm_s"] += t2 - t1
-        out["flops"] += (R * (2 * N * K + 2 * r * (K + N))      # forward rows
-                         + R * (2 * N * K + 2 * r * K)          # dX rows
-                         + 2 * M * r * (K + N)                  # U and G over all rows
-                         + 2 * M * r * K + 2 * M * N * r)       # dA, dB
-        out["layers"][li] = {"codes": q["codes"], "q8": q["q8"], "Y": Y, "dX": dX, "dA": dA, "dB": dB}
+        out["flops"] += nseg * (R * (2 * S * K + 2 * r * (K + S))      # forward rows
+                                + R * (2 * S * K + 2 * r * K)          # dX rows
+                                + 2 * M * r * (K + S)                  # U and G over all rows
+                                + 2 * M * r * K + 2 * M * S * r)       # dA, dB
+        out["layers"][gi] = {"codes": q["codes"], "q8": q["q8"], "Y": Y, "dX": dX, "dA": dA, "dB": dB}
     out["seconds"] = out["quant_s"] + out["gemm_s"]
     return out
 
@@ -473,7 +490,7 @@ def oracle_check(blk, sample):
     ok = bitexact and worst["max_ratio"] <= 1e-2 and worst["frob_ratio"] <= 5e-3
     return {"ok": ok, "quantize_bit_exact": bitexact, "worst_max_abs_err_over_max_ref": round(worst["max_ratio"], 6),
             "worst_frob_err_over_frob_ref": round(worst["frob_ratio"], 6),
-            "compared": f"codes and q8 of all {len(sample['layers'])} weights bit for bit; Y and dX on "
+            "compared": f"codes and q8 of all {len(sample['layers'])} projection weights bit for bit; Y and dX on "
                         f"{rows.size} sampled token rows, dA and dB in full"}
 
 
@@ -489,7 +506,7 @@ def cpu_baseline(torch, wl, cfg, gpu_block=None):
     check = oracle_check(gpu_block, smp) if gpu_block is not None else None
     O.set_num_threads(1)
     try:
-        one = oracle_sample(torch, wl, cfg, layers=[0])
+        one = oracle_sample(torch, wl, cfg, layers=[1])
     finally:
         O.set_num_threads(threads)
     c = wl.CONFIGS[cfg]
@@ -497,15 +514,16 @@ def cpu_baseline(torch, wl, cfg, gpu_block=None):
     sampled_gemm_rate = smp["flops"] / smp["gemm_s"]
     extrap_s = smp["quant_s"] + full_flops / sampled_gemm_rate
     base = {"value": smp["flops"] / smp["seconds"] / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-            "sample": f"all 7 linears of the {cfg} block (M={c['M']}, r={c['r']}): full NF4+DQ quantize and "
-                      f"dequantize of W, Y and dX on {smp['rows'].size} of {c['M']} token rows, dA and dB in full",
+            "sample": f"every projection of the {cfg} block (7 linears as q/k/v, o, gate/up, down; M={c['M']}, "
+                      f"r={c['r']}): full NF4+DQ quantize and dequantize of W, Y and dX on {smp['rows'].size} "
+                      f"of {c['M']} token rows, dA and dB in full",
             "seconds": round(smp["seconds"], 2), "cpu_model": _cpu_model(), "nproc": os.cpu_count(),
             "single_thread": {"value": one["flops"] / one["seconds"] / 1e12, "unit": "TFLOP/s", "cores": 1,
                               "seconds": round(one["seconds"], 2),
-                              "sample": f"the same sample for the first linear ({c['linears'][0][0]}) only"},
+                              "sample": "the same sample for the o projection (8192x8192 for the 65B block) only"},
             "all_cores": {"value": smp["flops"] / smp["seconds"] / 1e12, "unit": "TFLOP/s", "cores": threads},
             "full_step_seconds_extrapolated": round(extrap_s, 1),
-            "extrapolation": "extrapolated: measured quantize+dequantize time of the 7 weights plus the full "
+            "extrapolation": "extrapolated: measured quantize+dequantize time of the block's weights plus the full "
                              "step's fwd+bwd flops at the sample's all-core product rate"}
     return base, check
 
@@ -516,19 +534,22 @@ def cpu_baseline(torch, wl, cfg, gpu_block=None):
 
 def extras(torch, Q, wl, device, flush, peaks):
     out = {}
-    # LLaMA-7B decoder block (the same step, smaller shapes)
-    blk = Block(torch, Q, wl, device, cfg="llama7b")
-    for _ in range(3):
-        blk.step()
-    g = graph_of(torch, blk.step)
-    ms = replay_ms(torch, g, 10, flush)
-    del g
-    tf = blk.flops / (ms * 1e-3) / 1e12
-    out["llama7b_block_step_cuda_graph"] = {
-        "workload": WORKLOADS["llama7b"], "ms": round(ms, 4), "TFLOPs": round(tf, 1),
-        "frac_bf16_peak": round(tf / peaks["bf16_tflops"], 3)}
-    del blk
-    torch.cuda.empty_cache()
+    # the LLaMA-7B decoder block (the same step, smaller shapes), and both
+    # blocks as seven separate linears (one weight and one call each)
+    for key, cfg, fused in (("llama7b_block_step_cuda_graph", "llama7b", True),
+                            ("llama7b_block_7_separate_linears_cuda_graph", "llama7b", False),
+                            ("llama65b_block_7_separate_linears_cuda_graph", "llama65b", False)):
+        blk = Block(torch, Q, wl, device, cfg=cfg, fused=fused)
+        for _ in range(3):
+            blk.step()
+        g = graph_of(torch, blk.step)
+        ms = replay_ms(torch, g, 10, flush)
+        del g
+        tf = blk.flops / (ms * 1e-3) / 1e12
+        out[key] = {"workload": WORKLOADS[cfg] if fused else WORKLOADS[cfg].split(";")[0] + "; separate calls",
+                    "ms": round(ms, 4), "TFLOPs": round(tf, 1), "frac_bf16_peak": round(tf / peaks["bf16_tflops"], 3)}
+        del blk
+        torch.cuda.empty_cache()
 
     # stress forward: 4096x4096 weight with outliers, 2048 tokens, r = 16
     c = wl.CONFIGS["stress"]
@@ -777,15 +798,15 @@ def run_profile_case(case, block_cfg):
     if case in ("fwd_block", "dx_block"):
         cfg = wl.CONFIGS[block_cfg]
         M, r, s = cfg["M"], cfg["r"], cfg["alpha"] / cfg["r"]
-        for i, (_, N, K) in enumerate(cfg["linears"]):
-            W = wl.weight(N, K, seed=0, dtype=torch.bfloat16, device=dev, index_base=10 * i)
+        for i, (_, nseg, S, K) in enumerate(block_groups(wl, block_cfg)):
+            W = wl.weight(nseg * S, K, seed=0, dtype=torch.bfloat16, device=dev, index_base=10 * i)
             w = Q.qlora_nf4_quantize(W)
             del W
-            inp = wl.linear_inputs(M, N, K, r, seed=0, device=dev, index_base=10 * i)
+            inp = wl.fused_inputs(M, nseg, S, K, r, seed=0, device=dev, index_base=10 * i)
             if case == "dx_block":
-                Q.qlora_linear_bwd(inp["dY"], inp["X"], w, inp["A"], inp["B"], s)
+                Q.qlora_fused_linear_bwd(inp["dY"], inp["X"], w, nseg, inp["A"], inp["B"], s)
             else:
-                Q.qlora_linear_fwd(inp["X"], w, inp["A"], inp["B"], s)
+                Q.qlora_fused_linear_fwd(inp["X"], w, nseg, inp["A"], inp["B"], s)
             del w, inp
     elif case in ("quantize", "dequantize"):
         W = wl.weight(1 << 13, 1 << 13, seed=0, dtype=torch.bfloat16, device=dev)
@@ -823,7 +844,7 @@ def run_reference(args, world, rank):
     from bit_nf4_quantized_08_b200 import workloads as wl
     from oracle import oracle as O
     O.build()
-    nlin = len(wl.CONFIGS[HEADLINE]["linears"])
+    nlin = len(block_groups(wl, HEADLINE))
     for i in range(max(0, min(args.warmup, 1))):
         oracle_sample(torch, wl, HEADLINE, layers=[i % nlin])
     tot_flops, tot_s = 0, 0.0
@@ -833,8 +854,8 @@ def run_reference(args, world, rank):
         tot_s += smp["seconds"]
     value = tot_flops / tot_s / 1e12
     threads = O.num_threads()
-    desc = ("per step, one linear of the block in turn (M=2048, r=64): full NF4+DQ quantize and dequantize of W, "
-            "Y and dX on 16 of 2048 token rows, dA and dB in full")
+    desc = ("per step, one projection of the block in turn (q/k/v, o, gate/up, down; M=2048, r=64): full NF4+DQ "
+            "quantize and dequantize of its weight, Y and dX on 16 of 2048 token rows, dA and dB in full")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_s / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",

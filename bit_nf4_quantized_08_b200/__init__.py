@@ -10,6 +10,9 @@ from ._lib import QloraError, QLORA_OK, QLORA_ERR_INVALID_ARG, QLORA_ERR_UNSUPPO
 from .api import (  # noqa: F401
     NF4Weight,
     qlora_debug_inject,
+    qlora_fused_linear_bwd,
+    qlora_fused_linear_fwd,
+    qlora_fused_linear_workspace,
     qlora_get_last_error,
     qlora_linear_bwd,
     qlora_linear_fwd,

@@ -34,6 +34,9 @@ EXPORTS = (
     "qlora_linear_workspace",
     "qlora_linear_fwd",
     "qlora_linear_bwd",
+    "qlora_fused_linear_workspace",
+    "qlora_fused_linear_fwd",
+    "qlora_fused_linear_bwd",
     "qlora_lora_merge",
     "qlora_lora_unmerge",
     "qlora_get_last_error",
@@ -100,6 +103,12 @@ def lib() -> ctypes.CDLL:
     L.qlora_linear_fwd.restype = i32
     L.qlora_linear_bwd.argtypes = [vp, vp, i64, W, vp, vp, i32, f32, vp, vp, vp, vp, sz, vp]
     L.qlora_linear_bwd.restype = i32
+    L.qlora_fused_linear_workspace.argtypes = [i64, W, i32, i32, i32]
+    L.qlora_fused_linear_workspace.restype = sz
+    L.qlora_fused_linear_fwd.argtypes = [vp, i64, W, i32, vp, vp, i32, f32, vp, vp, sz, vp]
+    L.qlora_fused_linear_fwd.restype = i32
+    L.qlora_fused_linear_bwd.argtypes = [vp, vp, i64, W, i32, vp, vp, i32, f32, vp, vp, vp, vp, sz, vp]
+    L.qlora_fused_linear_bwd.restype = i32
     L.qlora_lora_merge.argtypes = [W, vp, vp, i32, f32, vp, vp]
     L.qlora_lora_merge.restype = i32
     L.qlora_lora_unmerge.argtypes = [vp, i64, i64, vp, vp, i32, f32, vp, vp]

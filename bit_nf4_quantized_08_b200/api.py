@@ -181,6 +181,52 @@ def qlora_linear_bwd(dY: torch.Tensor, X: torch.Tensor, w: NF4Weight, A: torch.T
     return dX, dA, dB
 
 
+def qlora_fused_linear_workspace(M: int, w: NF4Weight, nseg: int, r: int, bwd: bool) -> int:
+    cw = w.c_struct()
+    return int(lib().qlora_fused_linear_workspace(M, ctypes.byref(cw), nseg, r, int(bwd)))
+
+
+def qlora_fused_linear_fwd(X: torch.Tensor, w: NF4Weight, nseg: int, A: torch.Tensor | None,
+                           B: torch.Tensor | None, scale: float, Y: torch.Tensor | None = None,
+                           ws: torch.Tensor | None = None) -> torch.Tensor:
+    """Forward of a fused projection: nseg linears stored as the row segments
+    of one NF4 weight, sharing X; A [nseg*r, K], B [N, r]."""
+    M = X.shape[0]
+    r = 0 if A is None else A.shape[0] // nseg
+    if Y is None:
+        Y = torch.empty(M, w.rows, dtype=torch.bfloat16, device=X.device)
+    need = qlora_fused_linear_workspace(M, w, nseg, r, False)
+    wsb = _workspace(need, X.device, ws)
+    cw = w.c_struct()
+    check(lib().qlora_fused_linear_fwd(_ptr(X), M, ctypes.byref(cw), nseg, _ptr(A), _ptr(B), r, float(scale),
+                                       _ptr(Y), _ptr(wsb), wsb.numel(), _stream()), "qlora_fused_linear_fwd")
+    return Y
+
+
+def qlora_fused_linear_bwd(dY: torch.Tensor, X: torch.Tensor, w: NF4Weight, nseg: int, A: torch.Tensor | None,
+                           B: torch.Tensor | None, scale: float, dX: torch.Tensor | None = None,
+                           dA: torch.Tensor | None = None, dB: torch.Tensor | None = None,
+                           ws: torch.Tensor | None = None, want_dx: bool = True):
+    """(dX, dA, dB) of a fused projection; dX sums every segment's input
+    gradient, dA [nseg*r, K] and dB [N, r] hold every adapter's."""
+    M = X.shape[0]
+    r = 0 if A is None else A.shape[0] // nseg
+    if want_dx and dX is None:
+        dX = torch.empty(M, w.cols, dtype=torch.bfloat16, device=X.device)
+    if r > 0:
+        if dA is None:
+            dA = torch.empty(nseg * r, w.cols, dtype=torch.float32, device=X.device)
+        if dB is None:
+            dB = torch.empty(w.rows, r, dtype=torch.float32, device=X.device)
+    need = qlora_fused_linear_workspace(M, w, nseg, r, True)
+    wsb = _workspace(need, X.device, ws)
+    cw = w.c_struct()
+    check(lib().qlora_fused_linear_bwd(_ptr(dY), _ptr(X), M, ctypes.byref(cw), nseg, _ptr(A), _ptr(B), r,
+                                       float(scale), _ptr(dX) if want_dx else None, _ptr(dA), _ptr(dB),
+                                       _ptr(wsb), wsb.numel(), _stream()), "qlora_fused_linear_bwd")
+    return dX, dA, dB
+
+
 def qlora_lora_merge(w: NF4Weight, A: torch.Tensor, B: torch.Tensor, scale: float,
                      out: torch.Tensor | None = None) -> torch.Tensor:
     """W_merged = bf16(dequant(W) + scale B A), the dense bf16 weight with the

@@ -56,7 +56,17 @@ struct GemmParams {
     // the first LoRA k-step (that kernel has itself waited for the block
     // constants before it let this one launch); 0: before any load
     int late_wait;
+    // adapters of a fused projection (one weight, nseg row segments of
+    // lora_seg_rows rows, each with its own rank-lora_seg_r adapter): the
+    // LoRA k-steps of an output tile read the sU columns of the tile's
+    // segment, starting at (n0 / lora_seg_rows) * lora_seg_r; 0 = one adapter
+    int lora_seg_rows, lora_seg_r;
 };
+
+// First sU column of the adapter of the output rows starting at n0.
+__device__ __forceinline__ int lora_col0(const GemmParams& p, int n0) {
+    return p.lora_seg_rows ? (n0 / p.lora_seg_rows) * p.lora_seg_r : 0;
+}
 
 // MT = number of 128-row MMA sub-tiles on the A side (1 or 2).  With MT = 2
 // one dequantized B tile feeds two accumulators (256 A rows per CTA), which
@@ -253,7 +263,8 @@ __global__ void __launch_bounds__(GemmShape<BN, A_MN, B_MN, DQ, MT>::THREADS, 1)
                                 tma_load_2d(sA + mt * 16384, mA, full_tma(s), m0 + 128 * mt, kc * 64);
                                 tma_load_2d(sA + mt * 16384 + 8192, mA, full_tma(s), m0 + 128 * mt + 64, kc * 64);
                             } else {
-                                tma_load_2d(sA + mt * 16384, mA, full_tma(s), kc * 64, m0 + 128 * mt);
+                                tma_load_2d(sA + mt * 16384, mA, full_tma(s), kc * 64 + (lora ? lora_col0(p, n0) : 0),
+                                            m0 + 128 * mt);
                             }
                         }
                     }

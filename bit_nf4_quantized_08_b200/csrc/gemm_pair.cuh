@@ -196,7 +196,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairShape<DQ>::THREA
                     const CUtensorMap* mA = lora ? &p.tmA2 : &p.tmA;
 #pragma unroll
                     for (int mt = 0; mt < 2; ++mt)
-                        tma_load_2d(sA + mt * 16384, mA, full_tma(s), kc * 64, m0 + 256 * mt + 128 * (int)rank);
+                        tma_load_2d(sA + mt * 16384, mA, full_tma(s), kc * 64 + (lora ? lora_col0(p, sg.tn * 256) : 0),
+                                    m0 + 256 * mt + 128 * (int)rank);
                     if (lora) {
                         if (B_MN) {
                             for (int c = 0; c < 2; ++c)

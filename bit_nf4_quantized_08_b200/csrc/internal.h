@@ -63,11 +63,18 @@ cudaError_t launch_expand_scales(const qlora_nf4_weight& w, float* scales, int64
                                  cudaStream_t s, int* flags, int nflags);
 
 // ---- GEMMs (gemm.cu) ----
+// r is the rank of each adapter.  A fused projection (nseg > 1) is one
+// weight whose N rows are nseg segments of seg_rows rows that share the
+// input X, segment i with its own adapter: rows i*r .. i*r + r - 1 of
+// A [nseg*r][K] and rows i*seg_rows .. of B [N][r].
 struct LinearArgs {
     int64_t M, N, K;
     int r;
     float scale;
     const qlora_nf4_weight* w;
+    int nseg;
+    int64_t seg_rows;
+    int rt() const { return r * nseg; }  // columns of sU and sG
 };
 qlora_status linear_fwd_impl(const void* X, const LinearArgs& a, const void* A, const void* B,
                              void* Y, void* ws, size_t ws_bytes, cudaStream_t s);

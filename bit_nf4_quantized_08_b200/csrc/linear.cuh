@@ -224,6 +224,8 @@ struct SkinnyDesc {
     int out_mode;  // SK_OUT_*
     void* out;
     int64_t out_ld;
+    int r;         // output columns (0: the launch's r)
+    int seg_mode, seg_rows, seg_r;  // SK_SEG_* (fused projections)
 };
 
 // wait_first: the operands may have been written by the kernel just before on
@@ -262,7 +264,10 @@ inline qlora_status skinny(const SkinnyDesc* d, int nprob, int r, cudaStream_t s
         q.a_mn = d[i].a_mn;
         q.b_mn = d[i].b_mn;
         q.rows = d[i].rows;
-        q.r = r;
+        q.r = d[i].r > 0 ? d[i].r : r;
+        q.seg_mode = d[i].seg_mode;
+        q.seg_rows = d[i].seg_rows;
+        q.seg_r = d[i].seg_r;
         q.ksteps = d[i].ksteps;
         q.tiles = ceil_div(d[i].rows, 128);
         q.scale = d[i].scale;
@@ -458,16 +463,18 @@ inline bool map_codes(CUtensorMap* m, const qlora_nf4_weight& w, uint32_t box_by
 }
 
 // sU = bf16(scale * X A^T): Aop = X [m][k] (K-major), Bop = A [j][k] (K-major)
+// (A = [A_0; A_1; ...] of a fused projection: every adapter's sU in one pass over X)
 inline bool desc_sU(SkinnyDesc* d, const void* X, const LinearArgs& a, const void* A, void* sU) {
     memset(d, 0, sizeof(*d));
     if (!map_bf16(&d->tA, X, a.K, a.M, 128)) return false;
-    if (!map_bf16(&d->tB, A, a.K, a.r, lora_bn(a.r))) return false;
+    if (!map_bf16(&d->tB, A, a.K, a.rt(), lora_bn(a.rt()))) return false;
     d->rows = (int)a.M;
     d->ksteps = (int)(a.K / 64);
     d->scale = a.scale;
     d->out_mode = SK_OUT_BF16;
     d->out = sU;
-    d->out_ld = a.r;
+    d->out_ld = a.rt();
+    d->r = a.rt();
     return true;
 }
 
@@ -506,7 +513,11 @@ inline qlora_status launch_small_m(const void* X, const LinearArgs& a, const voi
     if (!map_bf16(&p.tmX, X, a.K, a.M, NT)) return QLORA_ERR_CUDA;
     if (a.r > 0) {
         if (!map_bf16(&p.tmB, B, a.r, a.N, 128)) return QLORA_ERR_CUDA;
-        if (!map_bf16(&p.tmU, L.sU, a.r, a.M, NT)) return QLORA_ERR_CUDA;
+        if (!map_bf16(&p.tmU, L.sU, a.rt(), a.M, NT)) return QLORA_ERR_CUDA;
+        if (a.nseg > 1) {
+            p.seg_rows = (int)a.seg_rows;
+            p.seg_r = a.r;
+        }
     } else {
         p.tmB = p.tmX;
         p.tmU = p.tmX;
@@ -545,7 +556,7 @@ inline qlora_status linear_fwd_impl(const void* X, const LinearArgs& a, const vo
                                     cudaStream_t s) {
     (void)ws_bytes;
     const qlora_nf4_weight& w = *a.w;
-    LinearWs L = carve_linear_ws(ws, a.M, a.N, a.K, a.r, 0);
+    LinearWs L = carve_linear_ws(ws, a.M, a.N, a.K, a.rt(), 0);
     if (a.M > kSmallM &&
         launch_expand_scales(w, L.scales, L.scales_ld, s, L.sk_flags, L.sk_flags ? kMaxStreamK + 2 : 0) != cudaSuccess)
         return QLORA_ERR_CUDA;
@@ -556,7 +567,7 @@ inline qlora_status linear_fwd_impl(const void* X, const LinearArgs& a, const vo
         // after the block-constant expansion has completed; the pair GEMM
         // starts beside it on the other SMs and waits for sU only before its
         // LoRA k-step.  Small M: the cost-model cluster size.
-        qlora_status st = skinny(&d, 1, a.r, s, 1, a.M > kSmallM ? SKP_PACKED : SKP_SPLIT);
+        qlora_status st = skinny(&d, 1, a.rt(), s, 1, a.M > kSmallM ? SKP_PACKED : SKP_SPLIT);
         if (st != QLORA_OK) return st;
     }
     GemmParams p;
@@ -570,13 +581,17 @@ inline qlora_status linear_fwd_impl(const void* X, const LinearArgs& a, const vo
     p.timeout_ns = wait_timeout_ns();
     p.inject = inject_mode() == 1 ? 1 : 0;
     p.out = Y;
+    if (a.r > 0 && a.nseg > 1) {
+        p.lora_seg_rows = (int)a.seg_rows;
+        p.lora_seg_r = a.r;
+    }
     if (a.M > kSmallM) {
         // Y = [X | sU] [W' | B]^T : 128 x 256 tiles, W' dequantized into the B slot.
         if (!map_bf16(&p.tmA, X, a.K, a.M, 128)) return QLORA_ERR_CUDA;
         p.tmB = p.tmA;
         if (!map_codes(&p.tmCodes, w, 32, 256)) return QLORA_ERR_CUDA;
         if (a.r > 0) {
-            if (!map_bf16(&p.tmA2, L.sU, a.r, a.M, 128)) return QLORA_ERR_CUDA;
+            if (!map_bf16(&p.tmA2, L.sU, a.rt(), a.M, 128)) return QLORA_ERR_CUDA;
             if (!map_bf16(&p.tmB2, B, a.r, a.N, 256)) return QLORA_ERR_CUDA;
         } else {
             p.tmA2 = p.tmA;
@@ -606,6 +621,8 @@ inline qlora_status linear_fwd_impl(const void* X, const LinearArgs& a, const vo
 }
 
 // sG = bf16(scale dY B): Aop = dY [m][n] (K-major), Bop = B viewed [j][n] (MN-major).
+// (fused projection: sG = [dY_0 B_0 | dY_1 B_1 | ...], each k-step of dY rows
+// shifted onto its own segment's output columns)
 inline bool desc_sG(SkinnyDesc* d, const CUtensorMap& tdY, const LinearArgs& a, const void* B, void* sG) {
     memset(d, 0, sizeof(*d));
     d->tA = tdY;
@@ -616,7 +633,13 @@ inline bool desc_sG(SkinnyDesc* d, const CUtensorMap& tdY, const LinearArgs& a, 
     d->scale = a.scale;
     d->out_mode = SK_OUT_BF16;
     d->out = sG;
-    d->out_ld = a.r;
+    d->out_ld = a.rt();
+    d->r = a.rt();
+    if (a.nseg > 1) {
+        d->seg_mode = SK_SEG_REDUCE;
+        d->seg_rows = (int)a.seg_rows;
+        d->seg_r = a.r;
+    }
     return true;
 }
 
@@ -626,17 +649,24 @@ inline bool desc_dA_dB(SkinnyDesc* d, const void* dY, const void* X, const Linea
                        float* dA, float* dB) {
     memset(d, 0, 2 * sizeof(*d));
     if (!map_bf16(&d[0].tA, X, a.K, a.M, 64)) return false;
-    if (!map_bf16(&d[0].tB, L.sG, a.r, a.M, 64)) return false;
+    if (!map_bf16(&d[0].tB, L.sG, a.rt(), a.M, 64)) return false;
     d[0].rows = (int)a.K;
     d[0].out_mode = SK_OUT_F32_T;
     d[0].out = dA;
     d[0].out_ld = a.K;
+    d[0].r = a.rt();
     if (!map_bf16(&d[1].tA, dY, a.N, a.M, 64)) return false;
-    if (!map_bf16(&d[1].tB, L.sU, a.r, a.M, 64)) return false;
+    if (!map_bf16(&d[1].tB, L.sU, a.rt(), a.M, 64)) return false;
     d[1].rows = (int)a.N;
     d[1].out_mode = SK_OUT_F32;
     d[1].out = dB;
     d[1].out_ld = a.r;
+    d[1].r = a.r;
+    if (a.nseg > 1) {  // the dB rows of a segment read that segment's sU columns
+        d[1].seg_mode = SK_SEG_ROWS;
+        d[1].seg_rows = (int)a.seg_rows;
+        d[1].seg_r = a.r;
+    }
     for (int i = 0; i < 2; ++i) {
         d[i].a_mn = 1;
         d[i].b_mn = 1;
@@ -657,8 +687,8 @@ inline qlora_status launch_dx_gemm(const void* A, void* dX, const LinearArgs& a,
     p.tmB = tdY;
     if (!map_codes(&p.tmCodes, w, 128, 64)) return QLORA_ERR_CUDA;
     if (a.r > 0) {
-        if (!map_bf16(&p.tmA2, L.sG, a.r, a.M, 128)) return QLORA_ERR_CUDA;
-        if (!map_bf16(&p.tmB2, A, a.K, a.r, 64)) return QLORA_ERR_CUDA;
+        if (!map_bf16(&p.tmA2, L.sG, a.rt(), a.M, 128)) return QLORA_ERR_CUDA;
+        if (!map_bf16(&p.tmB2, A, a.K, a.rt(), 64)) return QLORA_ERR_CUDA;
     } else {
         p.tmA2 = tdY;
         p.tmB2 = tdY;
@@ -668,7 +698,7 @@ inline qlora_status launch_dx_gemm(const void* A, void* dX, const LinearArgs& a,
     p.dq_rows = (int)a.N;
     p.dq_kbs = (int)(a.K / 64);
     p.ks_main = ceil_div(a.N, 64);
-    p.ks_lora = a.r > 0 ? ceil_div(a.r, 64) : 0;
+    p.ks_lora = a.r > 0 ? ceil_div(a.rt(), 64) : 0;
     p.ks_per_split = p.ks_main;
     p.rows = (int)a.M;
     p.cols = (int)a.K;
@@ -706,7 +736,7 @@ inline qlora_status linear_bwd_forked(const void* dY, const void* X, const Linea
                                       const CUtensorMap& tdY, const SideStream& side, cudaStream_t s) {
     SkinnyDesc dg;
     if (!desc_sG(&dg, tdY, a, B, L.sG)) return QLORA_ERR_CUDA;
-    qlora_status st = skinny(&dg, 1, a.r, s, 1, SKP_PACKED);
+    qlora_status st = skinny(&dg, 1, a.rt(), s, 1, SKP_PACKED);
     if (st != QLORA_OK) return st;
     if (cudaEventRecord(side.fork, s) != cudaSuccess) return QLORA_ERR_CUDA;
     if (cudaStreamWaitEvent(side.st, side.fork, 0) != cudaSuccess) return QLORA_ERR_CUDA;
@@ -720,7 +750,7 @@ inline qlora_status linear_bwd_forked(const void* dY, const void* X, const Linea
     if (st == QLORA_OK && !desc_sU(&d3[0], X, a, A, L.sU)) st = QLORA_ERR_CUDA;
     if (st == QLORA_OK && !desc_dA_dB(d3 + 1, dY, X, a, L, dA, dB)) st = QLORA_ERR_CUDA;
     if (st == QLORA_OK)
-        st = skinny(d3, 3, a.r, side.st, 0, SKP_STREAM, sm_count(), L.sk_flags + kMaxStreamK, 2, 1 << 1);
+        st = skinny(d3, 3, a.rt(), side.st, 0, SKP_STREAM, sm_count(), L.sk_flags + kMaxStreamK, 2, 1 << 1);
     if (cudaEventRecord(side.join, side.st) != cudaSuccess || cudaStreamWaitEvent(s, side.join, 0) != cudaSuccess)
         st = QLORA_ERR_CUDA;
     return st;
@@ -731,11 +761,11 @@ inline qlora_status linear_bwd_impl(const void* dY, const void* X, const LinearA
                                     void* ws, size_t ws_bytes, cudaStream_t s) {
     (void)ws_bytes;
     const qlora_nf4_weight& w = *a.w;
-    LinearWs L = carve_linear_ws(ws, a.M, a.N, a.K, a.r, 1);
+    LinearWs L = carve_linear_ws(ws, a.M, a.N, a.K, a.rt(), 1);
     if (a.M == 0) {
         if (a.r > 0) {
             note_launch();
-            k_fill_zero_f32<<<64, 256, 0, s>>>(dA, (int64_t)a.r * a.K);
+            k_fill_zero_f32<<<64, 256, 0, s>>>(dA, (int64_t)a.rt() * a.K);
             note_launch();
             k_fill_zero_f32<<<64, 256, 0, s>>>(dB, a.N * a.r);
             if (cudaGetLastError() != cudaSuccess) return QLORA_ERR_CUDA;
@@ -760,7 +790,7 @@ inline qlora_status linear_bwd_impl(const void* dY, const void* X, const LinearA
         // waits for the kernel before (the expansion, a dependent launch that
         // lets this one start early) before it loads: the workspace it writes
         // may still be read by the call before
-        qlora_status st = skinny(d, 2, a.r, s, 1);
+        qlora_status st = skinny(d, 2, a.rt(), s, 1);
         if (st != QLORA_OK) return st;
     }
     if (dX) {
@@ -771,7 +801,7 @@ inline qlora_status linear_bwd_impl(const void* dY, const void* X, const LinearA
         SkinnyDesc d[2];
         if (!desc_dA_dB(d, dY, X, a, L, dA, dB)) return QLORA_ERR_CUDA;
         // sG and sU come from the LoRA GEMMs above
-        qlora_status st = skinny(d, 2, a.r, s, 1);
+        qlora_status st = skinny(d, 2, a.rt(), s, 1);
         if (st != QLORA_OK) return st;
     }
     return QLORA_OK;

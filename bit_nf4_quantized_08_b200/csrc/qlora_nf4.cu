@@ -231,6 +231,19 @@ static qlora_status check_merge(int64_t N, int64_t K, const void* A, const void*
     return QLORA_OK;
 }
 
+// A fused projection: nseg equal row segments, each segment a whole number
+// of 256-row output tiles (so that no tile of any kernel straddles two
+// adapters), nseg * r <= 256 adapter columns in all.
+static qlora_status check_fused(int64_t M, const qlora_nf4_weight* w, int32_t nseg, int32_t r) {
+    qlora_status st = check_linear(M, w, r);
+    if (st != QLORA_OK) return st;
+    if (nseg < 1) return QLORA_ERR_INVALID_ARG;
+    if (nseg == 1) return QLORA_OK;
+    if (nseg > 8 || w->rows % nseg != 0 || (w->rows / nseg) % 256 != 0 || (int64_t)nseg * r > 256)
+        return QLORA_ERR_UNSUPPORTED;
+    return QLORA_OK;
+}
+
 }  // namespace qlora
 
 using namespace qlora;
@@ -317,30 +330,41 @@ qlora_status qlora_nf4_dequantize(const qlora_nf4_weight* w, void* out, qlora_st
     return QLORA_OK;
 }
 
+size_t qlora_fused_linear_workspace(int64_t M, const qlora_nf4_weight* w, int32_t nseg, int32_t r,
+                                    int32_t bwd) {
+    if (check_fused(M, w, nseg, r) != QLORA_OK) return 0;
+    return linear_workspace_bytes(M, w->rows, w->cols, r * nseg, bwd ? 1 : 0);
+}
+
 size_t qlora_linear_workspace(int64_t M, const qlora_nf4_weight* w, int32_t r, int32_t bwd) {
-    if (check_linear(M, w, r) != QLORA_OK) return 0;
-    return linear_workspace_bytes(M, w->rows, w->cols, r, bwd ? 1 : 0);
+    return qlora_fused_linear_workspace(M, w, 1, r, bwd);
+}
+
+qlora_status qlora_fused_linear_fwd(const void* X, int64_t M, const qlora_nf4_weight* w, int32_t nseg,
+                                    const void* A, const void* B, int32_t r, float scale, void* Y,
+                                    void* ws, size_t ws_bytes, qlora_stream_t stream) {
+    qlora_status st = check_fused(M, w, nseg, r);
+    if (st != QLORA_OK) return st;
+    if (M == 0) return QLORA_OK;
+    if (!X || !aligned(X, 16) || !Y || !aligned(Y, 16)) return QLORA_ERR_INVALID_ARG;
+    if (r > 0 && (!A || !aligned(A, 16) || !B || !aligned(B, 16))) return QLORA_ERR_INVALID_ARG;
+    const size_t need = linear_workspace_bytes(M, w->rows, w->cols, r * nseg, 0);
+    if (!ws || !aligned(ws, 16) || ws_bytes < need) return QLORA_ERR_INVALID_ARG;
+    LinearArgs a{M, w->rows, w->cols, r, scale, w, nseg, w->rows / nseg};
+    return linear_fwd_impl(X, a, A, B, Y, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 qlora_status qlora_linear_fwd(const void* X, int64_t M, const qlora_nf4_weight* w, const void* A,
                               const void* B, int32_t r, float scale, void* Y, void* ws,
                               size_t ws_bytes, qlora_stream_t stream) {
-    qlora_status st = check_linear(M, w, r);
-    if (st != QLORA_OK) return st;
-    if (M == 0) return QLORA_OK;
-    if (!X || !aligned(X, 16) || !Y || !aligned(Y, 16)) return QLORA_ERR_INVALID_ARG;
-    if (r > 0 && (!A || !aligned(A, 16) || !B || !aligned(B, 16))) return QLORA_ERR_INVALID_ARG;
-    const size_t need = linear_workspace_bytes(M, w->rows, w->cols, r, 0);
-    if (!ws || !aligned(ws, 16) || ws_bytes < need) return QLORA_ERR_INVALID_ARG;
-    LinearArgs a{M, w->rows, w->cols, r, scale, w};
-    return linear_fwd_impl(X, a, A, B, Y, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+    return qlora_fused_linear_fwd(X, M, w, 1, A, B, r, scale, Y, ws, ws_bytes, stream);
 }
 
-qlora_status qlora_linear_bwd(const void* dY, const void* X, int64_t M, const qlora_nf4_weight* w,
-                              const void* A, const void* B, int32_t r, float scale, void* dX,
-                              float* dA, float* dB, void* ws, size_t ws_bytes,
-                              qlora_stream_t stream) {
-    qlora_status st = check_linear(M, w, r);
+qlora_status qlora_fused_linear_bwd(const void* dY, const void* X, int64_t M, const qlora_nf4_weight* w,
+                                    int32_t nseg, const void* A, const void* B, int32_t r, float scale,
+                                    void* dX, float* dA, float* dB, void* ws, size_t ws_bytes,
+                                    qlora_stream_t stream) {
+    qlora_status st = check_fused(M, w, nseg, r);
     if (st != QLORA_OK) return st;
     if (r > 0 && (!A || !aligned(A, 16) || !B || !aligned(B, 16) || !dA || !aligned(dA, 16) ||
                   !dB || !aligned(dB, 16)))
@@ -349,11 +373,18 @@ qlora_status qlora_linear_bwd(const void* dY, const void* X, int64_t M, const ql
         if (!dY || !aligned(dY, 16) || !X || !aligned(X, 16)) return QLORA_ERR_INVALID_ARG;
         if (dX && !aligned(dX, 16)) return QLORA_ERR_INVALID_ARG;
     }
-    const size_t need = linear_workspace_bytes(M, w->rows, w->cols, r, 1);
+    const size_t need = linear_workspace_bytes(M, w->rows, w->cols, r * nseg, 1);
     if (!ws || !aligned(ws, 16) || ws_bytes < need) return QLORA_ERR_INVALID_ARG;
-    LinearArgs a{M, w->rows, w->cols, r, scale, w};
+    LinearArgs a{M, w->rows, w->cols, r, scale, w, nseg, w->rows / nseg};
     return linear_bwd_impl(dY, X, a, A, B, dX, dA, dB, ws, ws_bytes,
                            reinterpret_cast<cudaStream_t>(stream));
+}
+
+qlora_status qlora_linear_bwd(const void* dY, const void* X, int64_t M, const qlora_nf4_weight* w,
+                              const void* A, const void* B, int32_t r, float scale, void* dX,
+                              float* dA, float* dB, void* ws, size_t ws_bytes,
+                              qlora_stream_t stream) {
+    return qlora_fused_linear_bwd(dY, X, M, w, 1, A, B, r, scale, dX, dA, dB, ws, ws_bytes, stream);
 }
 
 qlora_status qlora_lora_merge(const qlora_nf4_weight* w, const void* A, const void* B, int32_t r,

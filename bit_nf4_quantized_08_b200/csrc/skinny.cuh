@@ -35,7 +35,24 @@ struct SkinnyProblem {
     int out_mode;
     void* out;
     int64_t out_ld;  // elements
+    // adapters of a fused projection (row segments of seg_rows, rank seg_r
+    // each).  SK_SEG_REDUCE: the MN-major B operand's columns are shifted by
+    // -(segment of the k-step's reduction index) * seg_r, so each output
+    // column block only gathers its own segment (G = dY B per segment);
+    // SK_SEG_ROWS: shifted by +(segment of the tile's output rows) * seg_r
+    // (dB of a segment reads its own sU columns).  Shifted-out columns read
+    // the load's zero fill.
+    int seg_mode, seg_rows, seg_r;
 };
+
+enum { SK_SEG_NONE = 0, SK_SEG_REDUCE = 1, SK_SEG_ROWS = 2 };
+
+// Column offset of the B operand of problem P at k-step k of the tile at row m0.
+__device__ __forceinline__ int skinny_b_col0(const SkinnyProblem& P, int k, int m0) {
+    if (P.seg_mode == SK_SEG_REDUCE) return -((k * 64) / P.seg_rows) * P.seg_r;
+    if (P.seg_mode == SK_SEG_ROWS) return (m0 / P.seg_rows) * P.seg_r;
+    return 0;
+}
 
 struct SkinnyParams {
     SkinnyProblem pr[3];
@@ -185,7 +202,8 @@ __global__ void __launch_bounds__(SkinnyShape<BN>::THREADS, 1) k_skinny(const __
                     tma_load_2d(sA, &P.tmA, full(s), k * 64, m0);
                 }
                 if (b_mn) {
-                    for (int c = 0; c < BN / 64; ++c) tma_load_2d(sB + 8192 * c, &P.tmB, full(s), 64 * c, k * 64);
+                    for (int c = 0; c < BN / 64; ++c)
+                        tma_load_2d(sB + 8192 * c, &P.tmB, full(s), 64 * c + skinny_b_col0(P, k, m0), k * 64);
                 } else {
                     tma_load_2d(sB, &P.tmB, full(s), k * 64, 0);
                 }
@@ -483,7 +501,8 @@ __global__ void __launch_bounds__(StreamShape<BN>::THREADS, 1) k_lora_stream(con
                         tma_load_2d(sA, &P.tmA, full(s), k * 64, m0);
                     }
                     if (P.b_mn) {
-                        for (int c = 0; c < BN / 64; ++c) tma_load_2d(sB + 8192 * c, &P.tmB, full(s), 64 * c, k * 64);
+                        for (int c = 0; c < BN / 64; ++c)
+                            tma_load_2d(sB + 8192 * c, &P.tmB, full(s), 64 * c + skinny_b_col0(P, k, m0), k * 64);
                     } else {
                         tma_load_2d(sB, &P.tmB, full(s), k * 64, 0);
                     }

@@ -41,6 +41,7 @@ struct SmallMParams {
     int dq;
     int N, M, kbs;        // kbs = K / 64
     int ks_main, ks_lora, tiles;
+    int seg_rows, seg_r;  // fused projection: sU columns of tile t start at (128 t / seg_rows) seg_r
     uint16_t* Y;          // [M][N] bf16
     float* part;          // [gridDim.x][NT][128] fp32 partial tiles
     uint32_t* flags;      // [gridDim.x][4] epoch of the published partial, per TMEM quarter
@@ -159,7 +160,8 @@ __global__ void __launch_bounds__(SmallMShape<NT, NG>::THREADS, 1)
                         waited = true;
                     }
                     mbar_arrive_expect_tx(full_tma(s), S::X_BYTES);
-                    tma_load_2d(stX(s), &p.tmU, full_tma(s), (k - p.ks_main) * 64, 0);
+                    const int ucol0 = p.seg_rows ? (n0 / p.seg_rows) * p.seg_r : 0;
+                    tma_load_2d(stX(s), &p.tmU, full_tma(s), (k - p.ks_main) * 64 + ucol0, 0);
                 }
                 last_use[s] = u;
             }

@@ -36,6 +36,17 @@ CONFIGS = {
 }
 
 
+# The same blocks as fused projections: (name, nseg, rows per segment, K).
+# q/k/v share the attention input and gate/up the MLP input, so each group is
+# one weight of nseg row segments with one adapter per segment.
+FUSED_GROUPS = {
+    "llama7b": [("qkv", 3, 4096, 4096), ("o", 1, 4096, 4096), ("gate_up", 2, 11008, 4096),
+                ("down", 1, 4096, 11008)],
+    "llama65b": [("qkv", 3, 8192, 8192), ("o", 1, 8192, 8192), ("gate_up", 2, 22016, 8192),
+                 ("down", 1, 8192, 22016)],
+}
+
+
 def _gen(seed: int, index: int, device) -> torch.Generator:
     g = torch.Generator(device=device)
     g.manual_seed(int(seed) * 1000 + int(index))
@@ -79,6 +90,20 @@ def linear_inputs(M: int, N: int, K: int, r: int, seed: int = 0, device="cpu", i
         out["A"] = None
         out["B"] = None
     return out
+
+
+def fused_inputs(M: int, nseg: int, S: int, K: int, r: int, seed: int = 0, device="cpu", index_base: int = 0,
+                 b_std: float = 0.01) -> dict:
+    """Inputs of a fused projection of nseg linears of S rows each sharing X:
+    X ~ N(0,1) [M,K], dY ~ N(0,1) [M, nseg*S], A ~ N(0, 1/r) [nseg*r, K]
+    (one rank-r adapter per segment), B ~ N(0, b_std) [nseg*S, r] (bf16)."""
+    N = nseg * S
+    return {
+        "X": normal((M, K), 1.0, seed, index_base + TENSOR_INDEX["X"], device=device),
+        "dY": normal((M, N), 1.0, seed, index_base + TENSOR_INDEX["dY"], device=device),
+        "A": normal((nseg * r, K), 1.0 / r, seed, index_base + TENSOR_INDEX["A"], device=device),
+        "B": normal((N, r), b_std, seed, index_base + TENSOR_INDEX["B"], device=device),
+    }
 
 
 def sample_rows(M: int, n: int = 64, seed: int = 0):

@@ -198,6 +198,37 @@ qlora_status qlora_linear_bwd(const void *dY, const void *X, int64_t M, const ql
                               qlora_stream_t stream);
 
 /*
+ * Fused projection: nseg linears that share one input X (q, k and v of an
+ * attention block, or gate and up of its MLP), stored as ONE quantized weight
+ * w [N = nseg * S, K] whose row segment i (rows i*S .. i*S + S - 1) is linear
+ * i, each with its own rank-r adapter (LoRA on every linear layer: QLoRA
+ * paper digest sec. 6 results; paper notes, "results").  Per segment i the
+ * forward and backward are those of qlora_linear_fwd / qlora_linear_bwd:
+ *   Y[:, seg i]  = X w'_i^T + scale (X A_i^T) B_i^T
+ *   dX           = sum_i ( dY[:, seg i] w'_i + scale G_i A_i ),  G_i = dY[:, seg i] B_i
+ *   dA_i         = scale G_i^T X,   dB_i = scale dY[:, seg i]^T (X A_i^T)
+ *   A [nseg*r, K] bf16 (A_i = rows i*r ..), B [N, r] bf16 (B_i = rows of seg i),
+ *   dA [nseg*r, K] fp32, dB [N, r] fp32; X [M, K], Y/dY [M, N], dX [M, K] bf16.
+ * The adapters' U = X A^T (all segments in one pass over X) and G, the dX
+ * GEMM (one reduction over all N rows and all nseg*r adapter columns), dA and
+ * dB each run as one launch for the whole projection.
+ * Requires 1 <= nseg <= 8, N % nseg == 0, S = N / nseg a multiple of 256 when
+ * nseg > 1, nseg * r <= 256, and everything qlora_linear_fwd requires
+ * (UNSUPPORTED otherwise; nseg < 1 is INVALID_ARG).  nseg == 1 is exactly
+ * qlora_linear_fwd / qlora_linear_bwd.  The workspace query takes the same
+ * nseg and r.
+ */
+size_t qlora_fused_linear_workspace(int64_t M, const qlora_nf4_weight *w, int32_t nseg, int32_t r,
+                                    int32_t bwd);
+qlora_status qlora_fused_linear_fwd(const void *X, int64_t M, const qlora_nf4_weight *w, int32_t nseg,
+                                    const void *A, const void *B, int32_t r, float scale, void *Y,
+                                    void *ws, size_t ws_bytes, qlora_stream_t stream);
+qlora_status qlora_fused_linear_bwd(const void *dY, const void *X, int64_t M, const qlora_nf4_weight *w,
+                                    int32_t nseg, const void *A, const void *B, int32_t r, float scale,
+                                    void *dX, float *dA, float *dB, void *ws, size_t ws_bytes,
+                                    qlora_stream_t stream);
+
+/*
  * LoRA merge (QLoRA tutorial "11.3 QLoRA", pitfalls: merging the adapter
  * into a 4-bit base adds error, so the base is dequantized first; LoRA
  * reproduction blog, "LoRA formula and tensor shapes": the adapter adds

@@ -228,3 +228,34 @@ def lora_merge(W: np.ndarray, A: np.ndarray, B: np.ndarray, s: float, sign: int 
     exact = np.zeros((N, K), np.float64) if want_exact else None
     lib().oracle_lora_merge(N, K, r, float(s), int(sign), _ptr(W), _ptr(A), _ptr(B), _ptr(out), _ptr(exact))
     return (out, exact) if want_exact else out
+
+
+def fused_linear_fwd(X: np.ndarray, W: np.ndarray, A: np.ndarray, B: np.ndarray, s: float, nseg: int,
+                     rows: np.ndarray | None = None) -> np.ndarray:
+    """Fused projection of nseg linears sharing X: row segment i of W with
+    adapter (A rows i*r.., B rows of segment i); Y is the concatenation of
+    the segments' outputs (each one linear_fwd)."""
+    N = W.shape[0]
+    r = A.shape[0] // nseg
+    S = N // nseg
+    parts = [linear_fwd(X, W[i * S:(i + 1) * S], A[i * r:(i + 1) * r], B[i * S:(i + 1) * S], s, rows)
+             for i in range(nseg)]
+    return np.concatenate(parts, axis=1)
+
+
+def fused_linear_bwd(dY: np.ndarray, X: np.ndarray, W: np.ndarray, A: np.ndarray, B: np.ndarray, s: float,
+                     nseg: int, rows: np.ndarray | None = None):
+    """(dX, dA, dB) of the fused projection: dX is the sum (fp64) of the
+    segments' input gradients, dA and dB the segments' adapter gradients
+    stacked in segment order."""
+    N = W.shape[0]
+    r = A.shape[0] // nseg
+    S = N // nseg
+    dX, dA, dB = None, [], []
+    for i in range(nseg):
+        gx, ga, gb = linear_bwd(dY[:, i * S:(i + 1) * S], X, W[i * S:(i + 1) * S], A[i * r:(i + 1) * r],
+                                B[i * S:(i + 1) * S], s, rows)
+        dX = gx if dX is None else dX + gx
+        dA.append(ga)
+        dB.append(gb)
+    return dX, np.concatenate(dA, axis=0), np.concatenate(dB, axis=0)

@@ -4,9 +4,10 @@ with the merged weight gives the fused NF4 + adapter forward's outputs.
 
 The GPU sums the rank-r product in fp32 on the tensor cores, the oracle in
 fp64; both round once to bf16.  Every output code must equal the oracle's,
-except where the exact value lies so close to a bf16 rounding midpoint that
-the fp32 error bound of the GPU's sum reaches across it: there either
-neighbour is accepted."""
+except where the exact value lies so close to a bf16 rounding boundary that
+the fp32 error bound of the GPU's arithmetic reaches across it: there the
+GPU's code must be the rounding of a value within that bound, and such codes
+must be rare."""
 import numpy as np
 import pytest
 import torch
@@ -21,27 +22,33 @@ def _f(bits):
     return (np.asarray(bits, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
+def _half_ulp(x):
+    """Half the bf16 spacing at each |x| (2^-134 in the subnormal range)."""
+    ax = np.abs(x)
+    e = np.floor(np.log2(np.maximum(ax, 2.0 ** -126)))
+    return np.ldexp(1.0, (e - 8).astype(np.int64))
+
+
 def _assert_rounded_like_oracle(got, ref, exact, W, A, B, s, r, what):
     """got, ref: bf16 codes; exact: the oracle's fp64 value before rounding.
-    A mismatch must be one unit in the last place, with the exact value within
-    the bound of the GPU's fp32 arithmetic of the midpoint between the two."""
+    Where got differs from the oracle's code, got must still be the rounding
+    of some value within the error bound of the GPU's fp32 arithmetic around
+    the exact value (so only values that sit that close to a rounding
+    boundary may round the other way), and such codes must be rare."""
     bad = np.nonzero(got != ref)
     if bad[0].size == 0:
         return
-    g, e = _f(got[bad]), _f(ref[bad])
+    g = _f(got[bad])
     v = exact[bad]
     n, k = bad
-    # |sum_j B[n,j] A[j,k]| bound of the terms, for the rounding error of an
-    # fp32 sum in any order (2 r u sum|t|) and of the final fma (2 u |v|)
+    # bound of the GPU's error before its final rounding: the fp32 sum of the
+    # r products in any order (2 r u sum|t|) and the final fma (2 u |v|)
     absBA = np.einsum("ij,ji->i", np.abs(_f(B)[n, :]), np.abs(_f(A)[:, k]))
     u = 2.0 ** -24
     bound = 2 * r * u * abs(s) * absBA + 2 * u * np.abs(v)
-    mid = (g + e) / 2
-    adjacent = np.abs(np.asarray(got[bad], np.int32) - np.asarray(ref[bad], np.int32)) == 1
-    near = np.abs(v - mid) <= bound
-    ok = adjacent & near
+    ok = np.abs(g - v) <= bound + _half_ulp(g)
     assert ok.all(), f"{what}: {int((~ok).sum())} of {got.size} codes differ from the oracle beyond the bound"
-    assert bad[0].size <= max(10, got.size // 10000), f"{what}: {bad[0].size} near-tie differences"
+    assert bad[0].size <= max(10, got.size // 10000), f"{what}: {bad[0].size} near-boundary differences"
 
 
 def _inputs(N, K, r, seed, dq=True):

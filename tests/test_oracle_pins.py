@@ -500,3 +500,34 @@ def test_lora_merge_zero_B_is_identity(O):
     A = _bits_of(rng.normal(0, 0.1, (8, 128)))
     B = np.zeros((16, 8), np.uint16)
     np.testing.assert_array_equal(O.lora_merge(W, A, B, 2.0), W)
+
+
+# ---------------------------------------------------------------------------
+# fused projections (q/k/v or gate/up sharing X, one adapter per segment)
+# ---------------------------------------------------------------------------
+
+def test_fused_projection_vs_autograd(O):
+    """The oracle's fused projection against torch autograd in fp64 on the
+    explicit per-segment model: Y[:, seg i] = X W_i^T + s (X A_i^T) B_i^T,
+    loss = sum(Y * dY); dX, dA, dB from backward (dX summed over the
+    segments by autograd itself)."""
+    rng = np.random.default_rng(8)
+    M, S, K, r, nseg, s = 7, 12, 64, 4, 3, 1.5
+    N = nseg * S
+    X, W, A, B, dY = (_bits_of(rng.normal(0, sd, shp)) for sd, shp in
+                      ((1.0, (M, K)), (0.05, (N, K)), (0.2, (nseg * r, K)), (0.1, (N, r)), (1.0, (M, N))))
+
+    def t(b, grad=False):
+        v = torch.from_numpy((np.asarray(b, np.uint32) << 16).view(np.float32).astype(np.float64))
+        return v.requires_grad_(grad)
+
+    Xt, At, Bt = t(X, True), t(A, True), t(B, True)
+    Wt, dYt = t(W), t(dY)
+    Y = torch.cat([Xt @ Wt[i * S:(i + 1) * S].T + s * (Xt @ At[i * r:(i + 1) * r].T) @ Bt[i * S:(i + 1) * S].T
+                   for i in range(nseg)], dim=1)
+    (Y * dYt).sum().backward()
+    np.testing.assert_allclose(O.fused_linear_fwd(X, W, A, B, s, nseg), Y.detach().numpy(), rtol=1e-12, atol=1e-12)
+    gx, ga, gb = O.fused_linear_bwd(dY, X, W, A, B, s, nseg)
+    np.testing.assert_allclose(gx, Xt.grad.numpy(), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(ga, At.grad.numpy(), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(gb, Bt.grad.numpy(), rtol=1e-12, atol=1e-12)
