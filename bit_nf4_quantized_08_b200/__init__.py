@@ -9,6 +9,8 @@ from ._lib import QloraError, QLORA_OK, QLORA_ERR_INVALID_ARG, QLORA_ERR_UNSUPPO
     QLORA_ERR_CUDA, QLORA_ERR_TIMEOUT, QLORA_ERR_WORKSPACE, QLORA_STATIC_QUANTIZE_MAX_ELEMS  # noqa: F401
 from .api import (  # noqa: F401
     NF4Weight,
+    PagedBuffer,
+    qlora_adamw_step,
     qlora_debug_inject,
     qlora_fused_linear_bwd,
     qlora_fused_linear_fwd,

@@ -39,6 +39,10 @@ EXPORTS = (
     "qlora_fused_linear_bwd",
     "qlora_lora_merge",
     "qlora_lora_unmerge",
+    "qlora_adamw_step",
+    "qlora_paged_alloc",
+    "qlora_paged_free",
+    "qlora_paged_prefetch",
     "qlora_get_last_error",
     "qlora_nf4_table",
     "qlora_nf4_encode",
@@ -71,6 +75,20 @@ class CNF4Weight(ctypes.Structure):
         ("absmax_q8", ctypes.c_void_p),
         ("absmax_scale", ctypes.c_void_p),
         ("absmax_offset", ctypes.c_void_p),
+    ]
+
+
+class CAdamWConfig(ctypes.Structure):
+    """Mirror of ``qlora_adamw_config``."""
+
+    _fields_ = [
+        ("lr", ctypes.c_float),
+        ("beta1", ctypes.c_float),
+        ("beta2", ctypes.c_float),
+        ("eps", ctypes.c_float),
+        ("weight_decay", ctypes.c_float),
+        ("grad_scale", ctypes.c_float),
+        ("step", ctypes.c_int64),
     ]
 
 
@@ -113,6 +131,14 @@ def lib() -> ctypes.CDLL:
     L.qlora_lora_merge.restype = i32
     L.qlora_lora_unmerge.argtypes = [vp, i64, i64, vp, vp, i32, f32, vp, vp]
     L.qlora_lora_unmerge.restype = i32
+    L.qlora_adamw_step.argtypes = [vp, vp, vp, vp, vp, i64, ctypes.POINTER(CAdamWConfig), vp]
+    L.qlora_adamw_step.restype = i32
+    L.qlora_paged_alloc.argtypes = [sz, ctypes.POINTER(ctypes.c_void_p)]
+    L.qlora_paged_alloc.restype = i32
+    L.qlora_paged_free.argtypes = [vp]
+    L.qlora_paged_free.restype = i32
+    L.qlora_paged_prefetch.argtypes = [vp, sz, i32, vp]
+    L.qlora_paged_prefetch.restype = i32
     L.qlora_get_last_error.argtypes = [vp]
     L.qlora_get_last_error.restype = i32
     L.qlora_nf4_table.argtypes = [vp]

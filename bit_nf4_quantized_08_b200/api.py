@@ -14,7 +14,7 @@ from dataclasses import dataclass
 import torch
 
 from . import _lib
-from ._lib import CNF4Weight, QLORA_BF16, QLORA_F32, check, lib
+from ._lib import CAdamWConfig, CNF4Weight, QLORA_BF16, QLORA_F32, check, lib
 
 BLOCKSIZE = 64
 DQ_BLOCK = 256
@@ -248,6 +248,56 @@ def qlora_lora_unmerge(W_merged: torch.Tensor, A: torch.Tensor, B: torch.Tensor,
     check(lib().qlora_lora_unmerge(_ptr(W_merged), rows, cols, _ptr(A), _ptr(B), A.shape[0], float(scale),
                                    _ptr(out), _stream()), "qlora_lora_unmerge")
     return out
+
+
+class PagedBuffer:
+    """Paged (unified) memory from qlora_paged_alloc for optimizer state:
+    reachable from the host and the device through one pointer; its pages
+    migrate on demand or on prefetch().  Freed with free() or when the
+    object is collected."""
+
+    def __init__(self, nbytes: int):
+        p = ctypes.c_void_p()
+        check(lib().qlora_paged_alloc(int(nbytes), ctypes.byref(p)), "qlora_paged_alloc")
+        self.ptr = p.value or 0
+        self.nbytes = int(nbytes)
+
+    def prefetch(self, to_host: bool, stream: torch.cuda.Stream | None = None) -> None:
+        check(lib().qlora_paged_prefetch(self.ptr, self.nbytes, int(bool(to_host)), _stream(stream)),
+              "qlora_paged_prefetch")
+
+    def host_view(self, dtype=None):
+        """NumPy view of the buffer on the host (synchronize the device first)."""
+        import numpy as np
+        buf = (ctypes.c_uint8 * self.nbytes).from_address(self.ptr)
+        return np.frombuffer(buf, dtype=dtype or np.uint8)
+
+    def data_ptr(self) -> int:
+        return self.ptr
+
+    def free(self) -> None:
+        if self.ptr:
+            check(lib().qlora_paged_free(self.ptr), "qlora_paged_free")
+            self.ptr = 0
+
+    def __del__(self):
+        try:
+            self.free()
+        except Exception:
+            pass
+
+
+def qlora_adamw_step(param: torch.Tensor, exp_avg, exp_avg_sq, grad: torch.Tensor,
+                     param_bf16: torch.Tensor | None = None, *, lr: float, step: int, beta1: float = 0.9,
+                     beta2: float = 0.999, eps: float = 1e-8, weight_decay: float = 0.0,
+                     grad_scale: float = 1.0) -> None:
+    """One AdamW step on fp32 param (in place) with fp32 moments exp_avg,
+    exp_avg_sq (tensors or PagedBuffer) and fp32 grad; param_bf16 receives
+    the bf16 copy."""
+    n = param.numel()
+    cfg = CAdamWConfig(lr, beta1, beta2, eps, weight_decay, grad_scale, int(step))
+    check(lib().qlora_adamw_step(param.data_ptr(), exp_avg.data_ptr(), exp_avg_sq.data_ptr(), grad.data_ptr(),
+                                 _ptr(param_bf16), n, ctypes.byref(cfg), _stream()), "qlora_adamw_step")
 
 
 def qlora_get_last_error(stream: torch.cuda.Stream | None = None) -> int:

@@ -8,7 +8,10 @@
 #include <mutex>
 #include <vector>
 
+#include <math.h>
+
 #include "../../include/qlora_nf4.h"
+#include "adamw.cuh"
 #include "common.cuh"
 #include "gemm.cuh"
 #include "internal.h"
@@ -405,6 +408,73 @@ qlora_status qlora_lora_unmerge(const void* W_merged, int64_t rows, int64_t cols
     if (!W_merged || !aligned(W_merged, 16)) return QLORA_ERR_INVALID_ARG;
     return lora_merge_impl(nullptr, W_merged, rows, cols, A, B, r, -scale, W_out,
                            reinterpret_cast<cudaStream_t>(stream));
+}
+
+qlora_status qlora_adamw_step(float* param, float* exp_avg, float* exp_avg_sq, const float* grad,
+                              void* param_bf16, int64_t n, const qlora_adamw_config* cfg,
+                              qlora_stream_t stream) {
+    if (!cfg || n < 0) return QLORA_ERR_INVALID_ARG;
+    if (cfg->step < 1 || !(cfg->lr >= 0.0f) || !(cfg->beta1 >= 0.0f && cfg->beta1 < 1.0f) ||
+        !(cfg->beta2 >= 0.0f && cfg->beta2 < 1.0f) || !(cfg->eps > 0.0f) || !(cfg->weight_decay >= 0.0f))
+        return QLORA_ERR_INVALID_ARG;
+    if (n == 0) return QLORA_OK;
+    if (!param || !exp_avg || !exp_avg_sq || !grad || !aligned(param, 16) || !aligned(exp_avg, 16) ||
+        !aligned(exp_avg_sq, 16) || !aligned(grad, 16))
+        return QLORA_ERR_INVALID_ARG;
+    if (param_bf16 && !aligned(param_bf16, 8)) return QLORA_ERR_INVALID_ARG;
+    AdamWParams a;
+    a.p = param;
+    a.m = exp_avg;
+    a.v = exp_avg_sq;
+    a.g = grad;
+    a.p_bf16 = static_cast<uint16_t*>(param_bf16);
+    a.n = n;
+    a.lr = cfg->lr;
+    a.b1 = cfg->beta1;
+    a.b2 = cfg->beta2;
+    a.eps = cfg->eps;
+    a.decay = (float)(1.0 - (double)cfg->lr * (double)cfg->weight_decay);
+    const double bc1 = 1.0 - pow((double)cfg->beta1, (double)cfg->step);
+    const double bc2 = 1.0 - pow((double)cfg->beta2, (double)cfg->step);
+    a.step_size = (float)((double)cfg->lr / bc1);
+    a.rsqrt_bc2 = (float)(1.0 / sqrt(bc2));
+    a.grad_scale = cfg->grad_scale;
+    const int64_t nv = (n + 3) / 4;
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((nv + 255) / 256, (int64_t)sm_count() * 8));
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    note_launch();
+    k_adamw<<<grid, 256, 0, s>>>(a);
+    return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+qlora_status qlora_paged_alloc(size_t bytes, void** ptr) {
+    if (!ptr) return QLORA_ERR_INVALID_ARG;
+    *ptr = nullptr;
+    if (bytes == 0) return QLORA_OK;
+    if (cudaMallocManaged(ptr, bytes, cudaMemAttachGlobal) != cudaSuccess) {
+        cudaGetLastError();
+        *ptr = nullptr;
+        return QLORA_ERR_CUDA;
+    }
+    return QLORA_OK;
+}
+
+qlora_status qlora_paged_free(void* ptr) {
+    if (!ptr) return QLORA_OK;
+    return cudaFree(ptr) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+qlora_status qlora_paged_prefetch(const void* ptr, size_t bytes, int32_t to_host, qlora_stream_t stream) {
+    if (!ptr && bytes) return QLORA_ERR_INVALID_ARG;
+    if (bytes == 0) return QLORA_OK;
+    int dev = 0;
+    if (!to_host && cudaGetDevice(&dev) != cudaSuccess) return QLORA_ERR_CUDA;
+    if (cudaMemPrefetchAsync(ptr, bytes, to_host ? cudaCpuDeviceId : dev,
+                             reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) {
+        cudaGetLastError();
+        return QLORA_ERR_CUDA;
+    }
+    return QLORA_OK;
 }
 
 qlora_status qlora_get_last_error(qlora_stream_t stream) {

@@ -16,8 +16,9 @@
  * Conventions for every entry point
  *  - All tensor pointers are DEVICE pointers to caller-owned memory, dense and
  *    row-major.  The library keeps no pointer after a call returns and
- *    allocates no device memory: temporary storage comes from the caller's
- *    workspace, whose size the matching *_workspace() query gives.
+ *    allocates no device memory (except qlora_paged_alloc, whose job it is):
+ *    temporary storage comes from the caller's workspace, whose size the
+ *    matching *_workspace() query gives.
  *  - Work is enqueued asynchronously on `stream` (NULL = legacy default).
  *  - Arguments are validated on the host before anything is launched; a bad
  *    argument returns QLORA_ERR_INVALID_ARG or QLORA_ERR_UNSUPPORTED and
@@ -258,6 +259,51 @@ qlora_status qlora_lora_merge(const qlora_nf4_weight *w, const void *A, const vo
 qlora_status qlora_lora_unmerge(const void *W_merged, int64_t rows, int64_t cols, const void *A,
                                 const void *B, int32_t r, float scale, void *W_out,
                                 qlora_stream_t stream);
+
+/*
+ * Optimizer step of the adapters (QLoRA paper digest, sec. 4 steps: Adam
+ * updates the LoRA matrices only; the frozen 4-bit weight is never updated).
+ * AdamW with decoupled weight decay on n fp32 parameters, with bias
+ * correction for step t = cfg->step (t >= 1, counting this step):
+ *   g = grad * grad_scale
+ *   param <- param * (1 - lr * weight_decay)
+ *   m <- beta1 m + (1 - beta1) g;   v <- beta2 v + (1 - beta2) g^2
+ *   param <- param - (lr / (1 - beta1^t)) m / (sqrt(v) / sqrt(1 - beta2^t) + eps)
+ * computed in fp32, element by element.  param, exp_avg (m), exp_avg_sq (v)
+ * are updated in place; grad is read; param_bf16 (may be NULL) receives the
+ * bf16 round-to-nearest-even copy of the new parameters, for the linear calls.
+ * Every adapter of a block can be one flat buffer (the backward's dA and dB
+ * written into views of the flat gradient), so one call updates them all.
+ * Pointers 16-byte aligned (param_bf16 8-byte).  m and v may be paged memory
+ * from qlora_paged_alloc.  Invalid hyper-parameters (step < 1, lr < 0,
+ * betas outside [0, 1), eps <= 0, weight_decay < 0): INVALID_ARG.
+ */
+typedef struct {
+    float lr, beta1, beta2, eps, weight_decay, grad_scale;
+    int64_t step;
+} qlora_adamw_config;
+
+qlora_status qlora_adamw_step(float *param, float *exp_avg, float *exp_avg_sq, const float *grad,
+                              void *param_bf16, int64_t n, const qlora_adamw_config *cfg,
+                              qlora_stream_t stream);
+
+/*
+ * Paged optimizer state (QLoRA blog note sec. 4 and tutorial "11.3 QLoRA",
+ * "paged optimizers": optimizer states live in unified memory, so that under
+ * a memory spike their pages move to host RAM and come back when the
+ * optimizer step touches them).
+ * qlora_paged_alloc: the one allocating call of the library: `bytes` of
+ *   managed (unified) memory, reachable from the host and every device
+ *   through the same pointer; *ptr = NULL for bytes == 0.  The caller owns
+ *   it and frees it with qlora_paged_free.  CUDA failure: QLORA_ERR_CUDA.
+ * qlora_paged_prefetch: migrates [ptr, ptr + bytes) ahead of use, to host
+ *   memory (to_host != 0: page the state out before a memory-heavy phase) or
+ *   to the current device (before the optimizer step), ordered on `stream`.
+ *   Without a prefetch, pages still migrate on demand when touched.
+ */
+qlora_status qlora_paged_alloc(size_t bytes, void **ptr);
+qlora_status qlora_paged_free(void *ptr);
+qlora_status qlora_paged_prefetch(const void *ptr, size_t bytes, int32_t to_host, qlora_stream_t stream);
 
 /*
  * Synchronizes `stream`, then returns (and clears) the device status word of

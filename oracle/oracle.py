@@ -51,6 +51,8 @@ def _declare(L: ctypes.CDLL) -> ctypes.CDLL:
     L.oracle_num_threads.restype = i32
     L.oracle_set_num_threads.argtypes = [i32]
     L.oracle_set_num_threads.restype = None
+    L.oracle_adamw_step.argtypes = [i64, f64, f64, f64, f64, f64, f64, i64, p, p, p, p]
+    L.oracle_adamw_step.restype = None
     L.oracle_lora_merge.argtypes = [i64, i64, i32, f64, i32, p, p, p, p, p]
     L.oracle_lora_merge.restype = None
     L.oracle_t8_nearest.argtypes = [ctypes.c_float]
@@ -259,3 +261,14 @@ def fused_linear_bwd(dY: np.ndarray, X: np.ndarray, W: np.ndarray, A: np.ndarray
         dA.append(ga)
         dB.append(gb)
     return dX, np.concatenate(dA, axis=0), np.concatenate(dB, axis=0)
+
+
+def adamw_step(p: np.ndarray, m: np.ndarray, v: np.ndarray, grad: np.ndarray, *, lr: float, step: int,
+               beta1: float = 0.9, beta2: float = 0.999, eps: float = 1e-8, weight_decay: float = 0.0,
+               grad_scale: float = 1.0) -> None:
+    """One AdamW step in fp64, in place on the float64 arrays p, m, v."""
+    for a in (p, m, v):
+        assert a.dtype == np.float64 and a.flags["C_CONTIGUOUS"]
+    g = np.ascontiguousarray(grad, np.float64)
+    lib().oracle_adamw_step(p.size, float(lr), float(beta1), float(beta2), float(eps), float(weight_decay),
+                            float(grad_scale), int(step), _ptr(p), _ptr(m), _ptr(v), _ptr(g))

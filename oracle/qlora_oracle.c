@@ -472,6 +472,33 @@ void oracle_lora_merge(int64_t N, int64_t K, int r, double s, int sign, const ui
     }
 }
 
+/* ------------------------------------------------------------------ */
+/* optimizer step of the adapters                                       */
+/* ------------------------------------------------------------------ */
+
+/*
+ * AdamW ([P4] sec. 4 steps: Adam updates L1 and L2 only) with decoupled
+ * weight decay and bias correction at step t >= 1, in fp64:
+ *   g = grad * grad_scale
+ *   p <- p (1 - lr wd)
+ *   m <- b1 m + (1 - b1) g,  v <- b2 v + (1 - b2) g^2
+ *   p <- p - lr * (m / (1 - b1^t)) / (sqrt(v / (1 - b2^t)) + eps)
+ */
+void oracle_adamw_step(int64_t n, double lr, double b1, double b2, double eps, double wd,
+                       double grad_scale, int64_t t, double *p, double *m, double *v,
+                       const double *grad)
+{
+    const double bc1 = 1.0 - pow(b1, (double)t);
+    const double bc2 = 1.0 - pow(b2, (double)t);
+    for (int64_t i = 0; i < n; ++i) {
+        double g = grad[i] * grad_scale;
+        p[i] = p[i] * (1.0 - lr * wd);
+        m[i] = b1 * m[i] + (1.0 - b1) * g;
+        v[i] = b2 * v[i] + (1.0 - b2) * g * g;
+        p[i] = p[i] - lr * (m[i] / bc1) / (sqrt(v[i] / bc2) + eps);
+    }
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP

@@ -126,6 +126,24 @@ def test_merge_rejects(Q):
     assert u(None, 0, 256, FAKE, FAKE, 8, 2.0, FAKE, None) == 0
 
 
+def test_adamw_and_paged_reject(Q):
+    from bit_nf4_quantized_08_b200._lib import lib, CAdamWConfig, QLORA_ERR_INVALID_ARG
+    L = lib()
+    good = CAdamWConfig(1e-3, 0.9, 0.999, 1e-8, 0.0, 1.0, 1)
+    for bad in (CAdamWConfig(1e-3, 0.9, 0.999, 1e-8, 0.0, 1.0, 0), CAdamWConfig(-1.0, 0.9, 0.999, 1e-8, 0.0, 1.0, 1),
+                CAdamWConfig(1e-3, 1.0, 0.999, 1e-8, 0.0, 1.0, 1), CAdamWConfig(1e-3, 0.9, 0.999, 0.0, 0.0, 1.0, 1)):
+        assert L.qlora_adamw_step(FAKE, FAKE, FAKE, FAKE, None, 16, ctypes.byref(bad), None) == QLORA_ERR_INVALID_ARG
+    assert L.qlora_adamw_step(FAKE + 4, FAKE, FAKE, FAKE, None, 16, ctypes.byref(good), None) == QLORA_ERR_INVALID_ARG
+    assert L.qlora_adamw_step(FAKE, FAKE, FAKE, FAKE, FAKE + 2, 16, ctypes.byref(good), None) == QLORA_ERR_INVALID_ARG
+    assert L.qlora_adamw_step(None, None, None, None, None, 0, ctypes.byref(good), None) == 0
+    assert L.qlora_adamw_step(FAKE, FAKE, FAKE, FAKE, None, 16, None, None) == QLORA_ERR_INVALID_ARG
+    assert L.qlora_paged_alloc(16, None) == QLORA_ERR_INVALID_ARG
+    p = ctypes.c_void_p(1)
+    assert L.qlora_paged_alloc(0, ctypes.byref(p)) == 0 and not p.value
+    assert L.qlora_paged_free(None) == 0
+    assert L.qlora_paged_prefetch(None, 16, 1, None) == QLORA_ERR_INVALID_ARG
+
+
 def test_linear_workspace_queries(Q):
     from bit_nf4_quantized_08_b200._lib import lib
     L = lib()

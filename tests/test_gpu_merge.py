@@ -29,7 +29,7 @@ def _half_ulp(x):
     return np.ldexp(1.0, (e - 8).astype(np.int64))
 
 
-def _assert_rounded_like_oracle(got, ref, exact, W, A, B, s, r, what):
+def _assert_rounded_like_oracle(got, ref, exact, W, A, B, s, r, what, rare=1e-4):
     """got, ref: bf16 codes; exact: the oracle's fp64 value before rounding.
     Where got differs from the oracle's code, got must still be the rounding
     of some value within the error bound of the GPU's fp32 arithmetic around
@@ -48,7 +48,7 @@ def _assert_rounded_like_oracle(got, ref, exact, W, A, B, s, r, what):
     bound = 2 * r * u * abs(s) * absBA + 2 * u * np.abs(v)
     ok = np.abs(g - v) <= bound + _half_ulp(g)
     assert ok.all(), f"{what}: {int((~ok).sum())} of {got.size} codes differ from the oracle beyond the bound"
-    assert bad[0].size <= max(10, got.size // 10000), f"{what}: {bad[0].size} near-boundary differences"
+    assert bad[0].size <= max(10, rare * got.size), f"{what}: {bad[0].size} near-boundary differences"
 
 
 def _inputs(N, K, r, seed, dq=True):
@@ -74,9 +74,13 @@ def test_merge_unmerge_parity(Q, O, cuda, N, K, r, dq):
     ref_m, ex_m = O.lora_merge(Wd, Ab, Bb, s, 1, want_exact=True)
     got_m = wl.bits(Wm)
     _assert_rounded_like_oracle(got_m, ref_m, ex_m, Wd, Ab, Bb, s, r, "merge")
-    # unmerge of the GPU's merged weight against the oracle's unmerge of it
+    # unmerge of the GPU's merged weight against the oracle's unmerge of it.
+    # The exact unmerged value is the base plus the merge's rounding error,
+    # which puts far more values near a rounding midpoint than a generic sum
+    # (about 0.3 % within the fp32 error of the midpoint with fp32 products,
+    # also when emulated on the host), so such differences are less rare
     ref_b, ex_b = O.lora_merge(got_m, Ab, Bb, s, -1, want_exact=True)
-    _assert_rounded_like_oracle(wl.bits(Wb), ref_b, ex_b, got_m, Ab, Bb, s, r, "unmerge")
+    _assert_rounded_like_oracle(wl.bits(Wb), ref_b, ex_b, got_m, Ab, Bb, s, r, "unmerge", rare=1e-2)
 
 
 def test_merge_with_zero_B_is_the_dequantized_weight(Q, O, cuda):

@@ -31,6 +31,8 @@ MUTANTS = [
     ("merge_ignores_sign", "(double)sign * s * acc;", "s * acc;"),
     ("merge_transposed_A", "* (double)bf16_to_f32(A[(int64_t)j * K + k]);\n            double v",
      "* (double)bf16_to_f32(A[k * r + j]);\n            double v"),
+    ("adamw_no_bias_correction", "p[i] - lr * (m[i] / bc1)", "p[i] - lr * (m[i])"),
+    ("adamw_coupled_decay", "p[i] = p[i] * (1.0 - lr * wd);", "g += wd * p[i];"),
     ("merge_rounds_down", "ldexp(nearbyint(ldexp(ax, -ulp_exp)), ulp_exp)", "ldexp(floor(ldexp(ax, -ulp_exp)), ulp_exp)"),
 ]
 
@@ -50,6 +52,7 @@ PINS = [
     pins.test_bwd_vs_autograd,
     pins.test_zero_B_noop_and_zero_dA,
     pins.test_lora_merge_brute_force,
+    pins.test_adamw_vs_torch_optim,
 ]
 
 

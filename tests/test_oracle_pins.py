@@ -531,3 +531,28 @@ def test_fused_projection_vs_autograd(O):
     np.testing.assert_allclose(gx, Xt.grad.numpy(), rtol=1e-12, atol=1e-12)
     np.testing.assert_allclose(ga, At.grad.numpy(), rtol=1e-12, atol=1e-12)
     np.testing.assert_allclose(gb, Bt.grad.numpy(), rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# adapter optimizer step
+# ---------------------------------------------------------------------------
+
+def test_adamw_vs_torch_optim(O):
+    """The oracle's AdamW step against torch.optim.AdamW in fp64 over four
+    steps with weight decay and a gradient scale."""
+    rng = np.random.default_rng(9)
+    n = 257
+    p0 = rng.normal(0, 0.1, n)
+    grads = [rng.normal(0, 1e-3, n) for _ in range(4)]
+    lr, b1, b2, eps, wd, gs = 2e-4, 0.9, 0.999, 1e-8, 0.01, 0.5
+    pt = torch.tensor(p0.copy(), dtype=torch.float64, requires_grad=True)
+    opt = torch.optim.AdamW([pt], lr=lr, betas=(b1, b2), eps=eps, weight_decay=wd)
+    p, m, v = p0.copy(), np.zeros(n), np.zeros(n)
+    for t, g in enumerate(grads, start=1):
+        pt.grad = torch.tensor(g * gs, dtype=torch.float64)
+        opt.step()
+        O.adamw_step(p, m, v, g, lr=lr, step=t, beta1=b1, beta2=b2, eps=eps, weight_decay=wd, grad_scale=gs)
+        np.testing.assert_allclose(p, pt.detach().numpy(), rtol=1e-13, atol=1e-16)
+        st = opt.state[pt]
+        np.testing.assert_allclose(m, st["exp_avg"].numpy(), rtol=1e-13, atol=1e-20)
+        np.testing.assert_allclose(v, st["exp_avg_sq"].numpy(), rtol=1e-13, atol=1e-24)
