@@ -24,6 +24,7 @@
 #include "gemm_pair.cuh"
 #include "skinny.cuh"
 #include "smallm.cuh"
+#include "smallm_mma.cuh"
 #include "internal.h"
 #include "quantize.cuh"
 
@@ -303,6 +304,15 @@ constexpr int kMaxSmallMCtas = 256;
 
 inline int small_m_nt(int64_t M) { return M <= 16 ? 16 : (M <= 32 ? 32 : 64); }
 
+// M <= kSmallMma: the register-fed warp-MMA kernel (smallm_mma.cuh) on a
+// persistent grid of at most kSmallMmaMaxCtas CTAs of 16 warps; its
+// workspace holds two fp32 partial slots of 1024 floats per warp and one
+// counter per 32-row group.
+constexpr int kSmallMma = 32;
+constexpr int kSmallMmaMaxCtas = 160;
+constexpr int kSmallMmaWarps = 16;
+constexpr int kSmallMmaPartFloats = 2 * 1024;
+
 inline int sm_count() {
     int dev = 0, n = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
@@ -334,8 +344,12 @@ inline LinearWs carve_linear_ws(void* ws, int64_t M, int64_t N, int64_t K, int r
     L.sU = r > 0 ? static_cast<uint16_t*>(c.take((size_t)M * r * 2)) : nullptr;
     L.sG = (r > 0 && bwd) ? static_cast<uint16_t*>(c.take((size_t)M * r * 2)) : nullptr;
     // small-M forward: partial tiles [kMaxSmallMCtas][NT][128] and flags [kMaxSmallMCtas][4]
-    L.part = big ? nullptr : static_cast<float*>(c.take((size_t)kMaxSmallMCtas * small_m_nt(M) * 128 * 4));
-    L.sm_flags = big ? nullptr : static_cast<uint32_t*>(c.take((size_t)kMaxSmallMCtas * 4 * 4));
+    // (M <= 32: partial slots of the warp-MMA kernel and one counter per 32 rows)
+    const size_t part_floats = M <= kSmallMma ? (size_t)kSmallMmaMaxCtas * kSmallMmaWarps * kSmallMmaPartFloats
+                                              : (size_t)kMaxSmallMCtas * small_m_nt(M) * 128;
+    const size_t nflags = M <= kSmallMma ? (size_t)((N + 31) / 32) : (size_t)kMaxSmallMCtas * 4;
+    L.part = big ? nullptr : static_cast<float*>(c.take(part_floats * 4));
+    L.sm_flags = big ? nullptr : static_cast<uint32_t*>(c.take(nflags * 4));
     L.sk_part = big ? static_cast<float*>(c.take((size_t)kMaxStreamK * 256 * 256 * 4)) : nullptr;
     L.sk_flags = big ? static_cast<int*>(c.take((size_t)(kMaxStreamK + 2) * 4)) : nullptr;
     L.bytes = c.used;
@@ -501,10 +515,68 @@ inline cudaError_t launch_small_m_kernel(const SmallMParams& p, int grid, cudaSt
     return launch_pdl(kern, dim3((unsigned)grid, 1, 1), dim3(SmallMShape<NT, NG>::THREADS, 1, 1), smem, s, 0, p);
 }
 
-// Y = X W'^T + sU B^T for M <= 64 on a persistent stream-K grid (one CTA per
-// SM, at least four (tile, k-step) units per CTA).
+template <int NT8, int R>
+inline cudaError_t launch_small_m_mma_kernel(SmallMmaParams& p, cudaStream_t s) {
+    using S = SmallMmaShape<NT8, R>;
+    static_assert(S::SMEM <= 232448, "shared memory per CTA");
+    const int groups = (int)((p.N + S::GROWS - 1) / S::GROWS);
+    p.GL = p.KB + p.lora_ks;
+    p.items = (int64_t)groups * p.GL;
+    // at least 8 items per warp; at most one CTA per SM
+    const int64_t ctas = std::max<int64_t>(1, std::min<int64_t>(std::min(sm_count(), kSmallMmaMaxCtas),
+                                                                p.items / (8 * S::WARPS)));
+    auto kern = k_smallm_mma<NT8, R>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM);
+    if (e != cudaSuccess) return e;
+    ProfileScope ps(QLORA_KERNEL_SMALLM_GEMM, s);
+    note_launch();
+    return launch_pdl(kern, dim3((unsigned)ctas, 1, 1), dim3(S::THREADS, 1, 1), S::SMEM, s, 0, p);
+}
+
+// Y = X W'^T + sU B^T for M <= 32: table-lookup expansion into warp MMAs.
+inline qlora_status launch_small_m_mma(const void* X, const LinearArgs& a, const void* B, void* Y,
+                                       const LinearWs& L, cudaStream_t s) {
+    const qlora_nf4_weight& w = *a.w;
+    SmallMmaParams p;
+    memset(&p, 0, sizeof(p));
+    p.codes = w.codes;
+    p.q8 = w.absmax_q8;
+    p.c1 = w.absmax_scale;
+    p.offset = w.absmax_offset;
+    p.absmax = w.absmax;
+    p.dq = w.double_quant;
+    p.X = static_cast<const uint16_t*>(X);
+    p.B = static_cast<const uint16_t*>(B);
+    p.sU = L.sU;
+    p.M = (int)a.M;
+    p.N = (int)a.N;
+    p.K = (int)a.K;
+    p.KB = (int)(a.K / 64);
+    p.r = a.r;
+    p.rt = a.rt();
+    p.seg_rows = a.nseg > 1 ? (int)a.seg_rows : 0;
+    p.lora_ks = a.r > 0 ? ceil_div(a.r, 64) : 0;
+    p.inv_scale = 1.0f / kSmallMTableScale;
+    p.Y = static_cast<uint16_t*>(Y);
+    p.part = L.part;
+    p.counters = L.sm_flags;
+    p.epoch = next_epoch() & 0xFFFFFFu;
+    if (p.epoch == 0) p.epoch = 1;
+    cudaError_t e;
+    if (a.M <= 8)
+        e = launch_small_m_mma_kernel<1, 4>(p, s);
+    else if (a.M <= 16)
+        e = launch_small_m_mma_kernel<2, 4>(p, s);
+    else
+        e = launch_small_m_mma_kernel<4, 2>(p, s);
+    return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+// Y = X W'^T + sU B^T for 32 < M <= 64 on a persistent stream-K grid (one CTA
+// per SM, at least four (tile, k-step) units per CTA).
 inline qlora_status launch_small_m(const void* X, const LinearArgs& a, const void* B, void* Y,
                                    const LinearWs& L, cudaStream_t s) {
+    if (a.M <= kSmallMma && inject_mode() != 1) return launch_small_m_mma(X, a, B, Y, L, s);
     const qlora_nf4_weight& w = *a.w;
     const int NT = small_m_nt(a.M);
     SmallMParams p;

@@ -301,9 +301,10 @@ def test_small_m_graph_replay(Q, O, cuda):
 
 
 def test_small_m_timeout_is_reported_and_recovers(Q, O, cuda):
-    """Failure detection on the small-M kernel: skipped loads make the
-    bounded waits run out, TIMEOUT is reported, the next call is correct."""
-    M, N, K, r = 16, 1024, 1024, 16
+    """Failure detection on the tcgen05 small-M kernel (33..64 tokens):
+    skipped loads make the bounded waits run out, TIMEOUT is reported, the
+    next call is correct.  (The warp-MMA kernel for M <= 32 has no waits.)"""
+    M, N, K, r = 40, 1024, 1024, 16
     q, inp, Wd_ref = _setup(Q, O, M, N, K, r, seed=9)
     X, A, B = inp["X"].cuda(), inp["A"].cuda(), inp["B"].cuda()
     Q.qlora_get_last_error()
