@@ -23,6 +23,8 @@ QLORA_ERR_WORKSPACE = 5
 STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "TIMEOUT", 5: "WORKSPACE"}
 QLORA_F32 = 0
 QLORA_BF16 = 1
+CODE_TYPES = {"nf4": 0, "fp4": 1}
+DQ_TYPES = {"int8": 0, "e4m3": 1}
 QLORA_STATIC_QUANTIZE_MAX_ELEMS = 1 << 26
 
 # Every function the header declares (checked against the header by the tests).
@@ -75,6 +77,8 @@ class CNF4Weight(ctypes.Structure):
         ("absmax_q8", ctypes.c_void_p),
         ("absmax_scale", ctypes.c_void_p),
         ("absmax_offset", ctypes.c_void_p),
+        ("code_type", ctypes.c_int32),
+        ("dq_type", ctypes.c_int32),
     ]
 
 

@@ -14,7 +14,7 @@ from dataclasses import dataclass
 import torch
 
 from . import _lib
-from ._lib import CAdamWConfig, CNF4Weight, QLORA_BF16, QLORA_F32, check, lib
+from ._lib import CAdamWConfig, CNF4Weight, CODE_TYPES, DQ_TYPES, QLORA_BF16, QLORA_F32, check, lib
 
 BLOCKSIZE = 64
 DQ_BLOCK = 256
@@ -36,7 +36,8 @@ class NF4Weight:
     codes [ceil(N*K/2)] uint8 (element 2i in the high nibble of byte i);
     without double quantization ``absmax`` [nb] fp32; with it ``absmax_q8``
     [nb] uint8, ``absmax_scale`` [ceil(nb/256)] fp32 and ``absmax_offset``
-    [1] fp32.
+    [1] fp32; nb = ceil(N*K / blocksize).  ``code_type`` "nf4" or "fp4",
+    ``dq_type`` "int8" or "e4m3" (the 8-bit code book of the constants).
     """
 
     rows: int
@@ -47,31 +48,37 @@ class NF4Weight:
     absmax_q8: torch.Tensor | None = None
     absmax_scale: torch.Tensor | None = None
     absmax_offset: torch.Tensor | None = None
+    blocksize: int = BLOCKSIZE
+    code_type: str = "nf4"
+    dq_type: str = "int8"
 
     @property
     def nblocks(self) -> int:
-        return (self.rows * self.cols + BLOCKSIZE - 1) // BLOCKSIZE
+        return (self.rows * self.cols + self.blocksize - 1) // self.blocksize
 
     def c_struct(self) -> CNF4Weight:
-        return CNF4Weight(self.rows, self.cols, BLOCKSIZE, int(self.double_quant),
+        return CNF4Weight(self.rows, self.cols, self.blocksize, int(self.double_quant),
                           _ptr(self.codes), _ptr(self.absmax), _ptr(self.absmax_q8),
-                          _ptr(self.absmax_scale), _ptr(self.absmax_offset))
+                          _ptr(self.absmax_scale), _ptr(self.absmax_offset),
+                          CODE_TYPES[self.code_type], DQ_TYPES[self.dq_type])
 
     def storage_bytes(self) -> int:
         t = [self.codes, self.absmax, self.absmax_q8, self.absmax_scale, self.absmax_offset]
         return sum(x.numel() * x.element_size() for x in t if x is not None)
 
     @staticmethod
-    def empty(rows: int, cols: int, double_quant: bool = True, device="cuda") -> "NF4Weight":
+    def empty(rows: int, cols: int, double_quant: bool = True, device="cuda", blocksize: int = BLOCKSIZE,
+              code_type: str = "nf4", dq_type: str = "int8") -> "NF4Weight":
         n = rows * cols
-        nb = (n + BLOCKSIZE - 1) // BLOCKSIZE
+        nb = (n + blocksize - 1) // blocksize
         codes = torch.empty((n + 1) // 2, dtype=torch.uint8, device=device)
+        fmt = dict(blocksize=blocksize, code_type=code_type, dq_type=dq_type)
         if double_quant:
             return NF4Weight(rows, cols, True, codes,
                              absmax_q8=torch.empty(nb, dtype=torch.uint8, device=device),
                              absmax_scale=torch.empty((nb + DQ_BLOCK - 1) // DQ_BLOCK, dtype=torch.float32, device=device),
-                             absmax_offset=torch.empty(1, dtype=torch.float32, device=device))
-        return NF4Weight(rows, cols, False, codes, absmax=torch.empty(nb, dtype=torch.float32, device=device))
+                             absmax_offset=torch.empty(1, dtype=torch.float32, device=device), **fmt)
+        return NF4Weight(rows, cols, False, codes, absmax=torch.empty(nb, dtype=torch.float32, device=device), **fmt)
 
 
 def _workspace(nbytes: int, device, ws: torch.Tensor | None) -> torch.Tensor:
@@ -80,14 +87,17 @@ def _workspace(nbytes: int, device, ws: torch.Tensor | None) -> torch.Tensor:
     return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
 
 
-def qlora_nf4_quantize_workspace(rows: int, cols: int, double_quant: bool = True) -> int:
-    return int(lib().qlora_nf4_quantize_workspace(rows, cols, BLOCKSIZE, int(double_quant)))
+def qlora_nf4_quantize_workspace(rows: int, cols: int, double_quant: bool = True,
+                                 blocksize: int = BLOCKSIZE) -> int:
+    return int(lib().qlora_nf4_quantize_workspace(rows, cols, blocksize, int(double_quant)))
 
 
 def qlora_nf4_quantize(W: torch.Tensor, double_quant: bool = True, out: NF4Weight | None = None,
-                       ws: torch.Tensor | None = None) -> NF4Weight:
+                       ws: torch.Tensor | None = None, blocksize: int = BLOCKSIZE, code_type: str = "nf4",
+                       dq_type: str = "int8") -> NF4Weight:
     """Blockwise NF4 quantization (+ 8-bit double quantization) of a 2-D
-    bf16 or fp32 CUDA tensor."""
+    bf16 or fp32 CUDA tensor.  blocksize, code_type and dq_type choose the
+    variants (used only when ``out`` is not given; ``out`` carries its own)."""
     if W.dim() != 2 or not W.is_cuda or not W.is_contiguous():
         raise ValueError("W must be a contiguous 2-D CUDA tensor")
     if W.dtype == torch.bfloat16:
@@ -98,8 +108,8 @@ def qlora_nf4_quantize(W: torch.Tensor, double_quant: bool = True, out: NF4Weigh
         raise TypeError("W must be bf16 or fp32")
     rows, cols = W.shape
     if out is None:
-        out = NF4Weight.empty(rows, cols, double_quant, W.device)
-    need = qlora_nf4_quantize_workspace(rows, cols, out.double_quant)
+        out = NF4Weight.empty(rows, cols, double_quant, W.device, blocksize, code_type, dq_type)
+    need = qlora_nf4_quantize_workspace(rows, cols, out.double_quant, out.blocksize)
     wsb = _workspace(need, W.device, ws) if need else None
     cw = out.c_struct()
     check(lib().qlora_nf4_quantize(_ptr(W), dt, ctypes.byref(cw), _ptr(wsb), need, _stream()),

@@ -61,6 +61,7 @@ struct GemmParams {
     // LoRA k-steps of an output tile read the sU columns of the tile's
     // segment, starting at (n0 / lora_seg_rows) * lora_seg_r; 0 = one adapter
     int lora_seg_rows, lora_seg_r;
+    int code_type;  // 4-bit code book of the weight (0 NF4, 1 FP4)
 };
 
 // First sU column of the adapter of the output rows starting at n0.
@@ -400,7 +401,7 @@ __global__ void __launch_bounds__(GemmShape<BN, A_MN, B_MN, DQ, MT>::THREADS, 1)
                             const uint4 c0 = ld_shared_v4(sC + code_off);
                             const uint4 c1 = ld_shared_v4(sC + code_off2);
                             const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-                            const Nf4BlockTable tb = nf4_block_table(a);
+                            const Nf4BlockTable tb = nf4_block_table(a, p.code_type);
 #pragma unroll
                             for (int q = 0; q < 8; ++q) {
                                 uint32_t o[4];

@@ -319,7 +319,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairShape<DQ>::THREA
                         const uint4 c0 = ld_shared_v4(sC + code_off);
                         const uint4 c1 = ld_shared_v4(sC + code_off2);
                         const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-                        const Nf4BlockTable tb = nf4_block_table(a);
+                        const Nf4BlockTable tb = nf4_block_table(a, p.code_type);
 #pragma unroll
                         for (int q = 0; q < 8; ++q) {
                             uint32_t o[4];

@@ -41,19 +41,16 @@ void side_stream_release();
 // width 1/16 over [-1, 1], see quantize.cuh): per bucket the largest fp32
 // below its decision threshold (3.0 without one) and the count of
 // thresholds below the bucket.
+// inc: how many thresholds sit at the bucket's one threshold value (1; 2 for
+// the FP4 code book, whose +0 code is never chosen, so that its threshold
+// coincides with the next one).
 struct Nf4SearchTable {
     float thr[33];
     int base[33];
+    int inc[33];
 };
 const Nf4SearchTable& nf4_search_table();
 void nf4_table_host(float out[16]);
-
-cudaError_t launch_quantize_blocks(const void* W, int is_bf16, int64_t n, uint8_t* codes,
-                                   float* absmax, double* group_sums, cudaStream_t s);
-cudaError_t launch_dq_offset(const double* group_sums, int64_t ngroups, int64_t nb, float* offset,
-                             cudaStream_t s);
-cudaError_t launch_dq_quantize(const float* absmax, int64_t nb, const float* offset, uint8_t* q8,
-                               float* c1, cudaStream_t s);
 cudaError_t launch_dequantize(const qlora_nf4_weight& w, uint16_t* out, cudaStream_t s);
 cudaError_t launch_encode(const float* x, int64_t n, uint8_t* codes, cudaStream_t s);
 

@@ -307,7 +307,7 @@ inline int small_m_nt(int64_t M) { return M <= 16 ? 16 : (M <= 32 ? 32 : 64); }
 // M <= kSmallMma: the register-fed warp-MMA kernel (smallm_mma.cuh) on a
 // persistent grid of at most kSmallMmaMaxCtas CTAs of 16 warps; its
 // workspace holds two fp32 partial slots of 1024 floats per warp and one
-// counter per 32-row group.
+// counter per 16-row group.
 constexpr int kSmallMma = 32;
 constexpr int kSmallMmaMaxCtas = 160;
 constexpr int kSmallMmaWarps = 16;
@@ -347,7 +347,7 @@ inline LinearWs carve_linear_ws(void* ws, int64_t M, int64_t N, int64_t K, int r
     // (M <= 32: partial slots of the warp-MMA kernel and one counter per 32 rows)
     const size_t part_floats = M <= kSmallMma ? (size_t)kSmallMmaMaxCtas * kSmallMmaWarps * kSmallMmaPartFloats
                                               : (size_t)kMaxSmallMCtas * small_m_nt(M) * 128;
-    const size_t nflags = M <= kSmallMma ? (size_t)((N + 31) / 32) : (size_t)kMaxSmallMCtas * 4;
+    const size_t nflags = M <= kSmallMma ? (size_t)((N + 15) / 16) : (size_t)kMaxSmallMCtas * 4;
     L.part = big ? nullptr : static_cast<float*>(c.take(part_floats * 4));
     L.sm_flags = big ? nullptr : static_cast<uint32_t*>(c.take(nflags * 4));
     L.sk_part = big ? static_cast<float*>(c.take((size_t)kMaxStreamK * 256 * 256 * 4)) : nullptr;
@@ -520,11 +520,12 @@ inline cudaError_t launch_small_m_mma_kernel(SmallMmaParams& p, cudaStream_t s) 
     using S = SmallMmaShape<NT8, R>;
     static_assert(S::SMEM <= 232448, "shared memory per CTA");
     const int groups = (int)((p.N + S::GROWS - 1) / S::GROWS);
-    p.GL = p.KB + p.lora_ks;
+    p.QW = (p.KB + S::QB - 1) / S::QB;
+    p.GL = p.QW + p.lora_ks;
     p.items = (int64_t)groups * p.GL;
-    // at least 8 items per warp; at most one CTA per SM
+    // at least 4 items per warp; at most one CTA per SM
     const int64_t ctas = std::max<int64_t>(1, std::min<int64_t>(std::min(sm_count(), kSmallMmaMaxCtas),
-                                                                p.items / (8 * S::WARPS)));
+                                                                p.items / (4 * S::WARPS)));
     auto kern = k_smallm_mma<NT8, R>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM);
     if (e != cudaSuccess) return e;
@@ -556,7 +557,8 @@ inline qlora_status launch_small_m_mma(const void* X, const LinearArgs& a, const
     p.rt = a.rt();
     p.seg_rows = a.nseg > 1 ? (int)a.seg_rows : 0;
     p.lora_ks = a.r > 0 ? ceil_div(a.r, 64) : 0;
-    p.inv_scale = 1.0f / kSmallMTableScale;
+    p.fmt = weight_format(w);
+    p.inv_scale = w.code_type ? 1.0f / 1.5f : 1.0f / 1.18881f;
     p.Y = static_cast<uint16_t*>(Y);
     p.part = L.part;
     p.counters = L.sm_flags;
@@ -564,11 +566,11 @@ inline qlora_status launch_small_m_mma(const void* X, const LinearArgs& a, const
     if (p.epoch == 0) p.epoch = 1;
     cudaError_t e;
     if (a.M <= 8)
-        e = launch_small_m_mma_kernel<1, 4>(p, s);
+        e = launch_small_m_mma_kernel<1, 2>(p, s);
     else if (a.M <= 16)
-        e = launch_small_m_mma_kernel<2, 4>(p, s);
+        e = launch_small_m_mma_kernel<2, 2>(p, s);
     else
-        e = launch_small_m_mma_kernel<4, 2>(p, s);
+        e = launch_small_m_mma_kernel<4, 1>(p, s);
     return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
@@ -599,6 +601,7 @@ inline qlora_status launch_small_m(const void* X, const LinearArgs& a, const voi
     p.offset = w.absmax_offset;
     p.absmax = w.absmax;
     p.dq = w.double_quant;
+    p.fmt = weight_format(w);
     p.N = (int)a.N;
     p.M = (int)a.M;
     p.kbs = (int)(a.K / 64);
@@ -653,6 +656,7 @@ inline qlora_status linear_fwd_impl(const void* X, const LinearArgs& a, const vo
     p.timeout_ns = wait_timeout_ns();
     p.inject = inject_mode() == 1 ? 1 : 0;
     p.out = Y;
+    p.code_type = w.code_type;
     if (a.r > 0 && a.nseg > 1) {
         p.lora_seg_rows = (int)a.seg_rows;
         p.lora_seg_r = a.r;
@@ -767,6 +771,7 @@ inline qlora_status launch_dx_gemm(const void* A, void* dX, const LinearArgs& a,
     }
     p.scales = L.scales;
     p.scales_ld = L.scales_ld;
+    p.code_type = w.code_type;
     p.dq_rows = (int)a.N;
     p.dq_kbs = (int)(a.K / 64);
     p.ks_main = ceil_div(a.N, 64);

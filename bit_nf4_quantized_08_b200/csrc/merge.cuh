@@ -38,6 +38,7 @@ struct MergeParams {
     const uint16_t* dense;    // dense bf16 base [N][K] (unmerge); null for an NF4 base
     uint16_t* out;            // bf16 [N][K]
     int N, K, r_chunks;       // r_chunks = ceil(r / 64)
+    QFormat fmt;              // code book, 8-bit code book, block size of the NF4 base
     float scale;              // +s (merge) or -s (unmerge)
     uint64_t timeout_ns;
 };
@@ -125,8 +126,9 @@ __global__ void __launch_bounds__(MergeShape::THREADS) k_lora_merge(const __grid
             const int kb = k0 / 64 + h;
             float a = 0.0f;
             if (kb < kbs) {
-                const int64_t b = (int64_t)n * kbs + kb;
-                a = p.dq ? block_scale_dq(__ldg(p.q8 + b), __ldg(p.c1 + (b >> 8)), __ldg(p.offset)) : __ldg(p.absmax + b);
+                const int64_t b = ((int64_t)n * kbs + kb) >> p.fmt.bs_shift;
+                a = p.dq ? block_scale_dq(__ldg(p.q8 + b), __ldg(p.c1 + (b >> 8)), __ldg(p.offset), p.fmt.dq_type)
+                         : __ldg(p.absmax + b);
             }
             a_blk[h] = a;
         }
@@ -136,8 +138,8 @@ __global__ void __launch_bounds__(MergeShape::THREADS) k_lora_merge(const __grid
     if (got) {
         Nf4BlockTable tb[2];
         if (!p.dense) {
-            tb[0] = nf4_block_table(a_blk[0]);
-            tb[1] = nf4_block_table(a_blk[1]);
+            tb[0] = nf4_block_table(a_blk[0], p.fmt.code_type);
+            tb[1] = nf4_block_table(a_blk[1], p.fmt.code_type);
         }
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {

@@ -27,10 +27,23 @@ namespace qlora {
         0x00000000u, 0x3da2fb01u, 0x3e24cadfu, 0x3e7c04dau, 0x3ead0336u, 0x3ee1a4b5u,       \
         0x3f1007a9u, 0x3f3913b0u, 0x3f800000u
 
-static constexpr uint32_t kNF4Bits[16] = {QLORA_NF4_BITS};          // host copy
-__constant__ uint32_t c_nf4_bits[16] = {QLORA_NF4_BITS};           // device copy
+// FP4 code book (the "Float4 (FP4)" data type the QLoRA paper digest, sec. 6,
+// compares NF4 with): the 16 values of a 4-bit float with 1 sign, 2
+// exponent (bias 1) and 1 mantissa bit -- magnitudes 0, 0.5, 1, 1.5, 2, 3,
+// 4, 6 -- divided by 6 and sorted; -0 (index 7) and +0 (index 8) both
+// appear, and the nearest-code rule (ties to the lower index) never picks 8.
+#define QLORA_FP4_BITS                                                                       \
+    0xbf800000u, 0xbf2aaaabu, 0xbf000000u, 0xbeaaaaabu, 0xbe800000u, 0xbe2aaaabu, 0xbdaaaaabu, \
+        0x80000000u, 0x00000000u, 0x3daaaaabu, 0x3e2aaaabu, 0x3e800000u, 0x3eaaaaabu,       \
+        0x3f000000u, 0x3f2aaaabu, 0x3f800000u
 
-__device__ __forceinline__ float nf4_value(int j) { return __uint_as_float(c_nf4_bits[j]); }
+static constexpr uint32_t kNF4Bits[16] = {QLORA_NF4_BITS};          // host copy
+static constexpr uint32_t kCodeBits[2][16] = {{QLORA_NF4_BITS}, {QLORA_FP4_BITS}};
+__constant__ uint32_t c_code_bits[2][16] = {{QLORA_NF4_BITS}, {QLORA_FP4_BITS}};  // device copy
+
+// Value j of the 4-bit code book of code type ct (0: NF4, 1: FP4).
+__device__ __forceinline__ float code_value(int ct, int j) { return __uint_as_float(c_code_bits[ct][j]); }
+__device__ __forceinline__ float nf4_value(int j) { return code_value(0, j); }
 
 // Byte planes of the 16 bf16 outputs of one block: L[q] holds the low bytes
 // of codes 4q..4q+3, H[q] the high bytes.
@@ -38,11 +51,11 @@ struct Nf4BlockTable {
     uint32_t L[4], H[4];
 };
 
-__device__ __forceinline__ Nf4BlockTable nf4_block_table(float a) {
+__device__ __forceinline__ Nf4BlockTable nf4_block_table(float a, int ct = 0) {
     uint32_t P[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i)
-        P[i] = pack_bf16x2(__fmul_rn(nf4_value(2 * i), a), __fmul_rn(nf4_value(2 * i + 1), a));
+        P[i] = pack_bf16x2(__fmul_rn(code_value(ct, 2 * i), a), __fmul_rn(code_value(ct, 2 * i + 1), a));
     Nf4BlockTable t;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -88,10 +101,45 @@ __device__ __forceinline__ float t8_value(int k) {
     return __fdiv_rn((float)(k - 127), 127.0f);
 }
 
-// Block constant a' (digest sec. 4 doubleDequant, first dequant):
-// fl32(fl32(t8[q8] * c1) + offset) with double quantization, else absmax.
-__device__ __forceinline__ float block_scale_dq(uint8_t q8, float c1, float offset) {
-    return __fadd_rn(__fmul_rn(t8_value(q8), c1), offset);
+// fp32 value of the FP8 double-quantization code k (0..252): the k-th of the
+// 253 distinct finite E4M3 values (1 sign, 4 exponent bits with bias 7, 3
+// mantissa bits; exponent field 0 subnormal; the all-ones pattern is not a
+// number, so the largest value is 448) in ascending order, divided by 448:
+// fl32(v / 448) with the quotient taken in fp64 (the "c2^FP8" of the digest,
+// sec. 4 double quantization).
+__device__ __forceinline__ float e4m3_value(int k) {
+    const int j = k < 126 ? 125 - k : k - 127;  // rank among the positive values
+    if (k == 126) return 0.0f;
+    double v;
+    if (j < 7) {
+        v = (double)(j + 1) * 0.001953125;  // (m / 8) 2^-6, m = 1..7
+    } else {
+        const int e = 1 + (j - 7) / 8, m = (j - 7) % 8;
+        v = ldexp(1.0 + m / 8.0, e - 7);
+    }
+    const float f = __double2float_rn(__ddiv_rn(v, 448.0));
+    return k < 126 ? -f : f;
 }
+
+// Value of the 8-bit double-quantization code k of code book dt
+// (0: linear t8, 1: FP8 E4M3).
+__device__ __forceinline__ float dq_value(int dt, int k) { return dt ? e4m3_value(k) : t8_value(k); }
+
+// Block constant a' (digest sec. 4 doubleDequant, first dequant):
+// fl32(fl32(c8[q8] * c1) + offset) with double quantization, else absmax.
+__device__ __forceinline__ float block_scale_dq(uint8_t q8, float c1, float offset, int dt = 0) {
+    return __fadd_rn(__fmul_rn(dq_value(dt, q8), c1), offset);
+}
+
+// Storage format of a quantized weight beyond the NF4 / linear 8-bit /
+// 64-element defaults: code book, double-quantization code book, and block
+// size 64 << bs_shift.  Block b of size bs covers the flattened elements
+// [b bs, (b+1) bs), so the block of the 64-element column kb64 of row n is
+// (n * K/64 + kb64) >> bs_shift.
+struct QFormat {
+    int code_type;  // 0 NF4, 1 FP4
+    int dq_type;    // 0 linear 8-bit, 1 FP8 E4M3
+    int bs_shift;   // 0, 1, 2: block size 64, 128, 256
+};
 
 }  // namespace qlora

@@ -121,7 +121,9 @@ static qlora_status check_weight(const qlora_nf4_weight* w, bool need_codes) {
     if (w->rows < 0 || w->cols < 0) return QLORA_ERR_INVALID_ARG;
     if (w->rows > 0 && w->cols > kMaxElems / w->rows) return QLORA_ERR_INVALID_ARG;
     if (w->double_quant != 0 && w->double_quant != 1) return QLORA_ERR_INVALID_ARG;
-    if (w->blocksize != 64) return QLORA_ERR_UNSUPPORTED;
+    if (w->code_type != QLORA_CODE_NF4 && w->code_type != QLORA_CODE_FP4) return QLORA_ERR_INVALID_ARG;
+    if (w->dq_type != QLORA_DQ_INT8 && w->dq_type != QLORA_DQ_FP8) return QLORA_ERR_INVALID_ARG;
+    if (w->blocksize != 64 && w->blocksize != 128 && w->blocksize != 256) return QLORA_ERR_UNSUPPORTED;
     const int64_t n = w->rows * w->cols;
     if (n == 0) return QLORA_OK;
     if (need_codes && (!w->codes || !aligned(w->codes, 16))) return QLORA_ERR_INVALID_ARG;
@@ -137,9 +139,9 @@ static qlora_status check_weight(const qlora_nf4_weight* w, bool need_codes) {
 
 // Workspace of qlora_nf4_quantize with double quantization: block maxima
 // [nb] f32, group sums [ng] f64, first-level offset partials (many groups).
-static size_t quantize_ws(int64_t n, int dq) {
+static size_t quantize_ws(int64_t n, int dq, int64_t bs) {
     if (!dq || n == 0) return 0;
-    const int64_t nb = (n + 63) / 64;
+    const int64_t nb = (n + bs - 1) / bs;
     const int64_t ng = (n + 16383) / 16384;
     return align256((size_t)nb * 4) + align256((size_t)ng * 8) + align256((size_t)dq_partial_count(ng) * 8);
 }
@@ -197,6 +199,7 @@ static qlora_status lora_merge_impl(const qlora_nf4_weight* w, const void* dense
     if (!map_bf16(&p.tmB, B, (uint64_t)r, (uint64_t)N, 128)) return QLORA_ERR_CUDA;
     if (!map_bf16(&p.tmA, A, (uint64_t)K, (uint64_t)r, 64)) return QLORA_ERR_CUDA;
     if (w) {
+        p.fmt = weight_format(*w);
         p.codes = w->codes;
         p.dq = w->double_quant;
         p.absmax = w->absmax;
@@ -255,9 +258,9 @@ extern "C" {
 
 size_t qlora_nf4_quantize_workspace(int64_t rows, int64_t cols, int32_t blocksize,
                                     int32_t double_quant) {
-    if (rows < 0 || cols < 0 || blocksize != 64) return 0;
+    if (rows < 0 || cols < 0 || (blocksize != 64 && blocksize != 128 && blocksize != 256)) return 0;
     if (rows > 0 && cols > kMaxElems / rows) return 0;
-    return quantize_ws(rows * cols, double_quant);
+    return quantize_ws(rows * cols, double_quant, blocksize);
 }
 
 qlora_status qlora_nf4_quantize(const void* W, qlora_dtype wdtype, const qlora_nf4_weight* out,
@@ -269,13 +272,14 @@ qlora_status qlora_nf4_quantize(const void* W, qlora_dtype wdtype, const qlora_n
     if (n == 0) return QLORA_OK;
     if (!W || !aligned(W, 16)) return QLORA_ERR_INVALID_ARG;
     if (!out->double_quant && (!out->absmax || !aligned(out->absmax, 4))) return QLORA_ERR_INVALID_ARG;
-    const size_t need = quantize_ws(n, out->double_quant);
+    const size_t need = quantize_ws(n, out->double_quant, out->blocksize);
     if (need > 0 && (!ws || !aligned(ws, 16) || ws_bytes < need)) return QLORA_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const int is_bf16 = wdtype == QLORA_BF16;
-    const int64_t nb = (n + 63) / 64;
+    const int64_t nb = (n + out->blocksize - 1) / out->blocksize;
+    const QFormat fmt = weight_format(*out);
     if (!out->double_quant) {
-        if (launch_quantize_blocks(W, is_bf16, n, out->codes, out->absmax, nullptr, s) != cudaSuccess)
+        if (launch_quantize_blocks(W, is_bf16, n, out->codes, out->absmax, nullptr, s, fmt) != cudaSuccess)
             return QLORA_ERR_CUDA;
         return QLORA_OK;
     }
@@ -283,10 +287,10 @@ qlora_status qlora_nf4_quantize(const void* W, qlora_dtype wdtype, const qlora_n
     double* sums = reinterpret_cast<double*>(static_cast<char*>(ws) + align256((size_t)nb * 4));
     const int64_t ng = (n + 16383) / 16384;
     double* partials = reinterpret_cast<double*>(reinterpret_cast<char*>(sums) + align256((size_t)ng * 8));
-    if (launch_quantize_blocks(W, is_bf16, n, out->codes, absmax, sums, s) != cudaSuccess)
+    if (launch_quantize_blocks(W, is_bf16, n, out->codes, absmax, sums, s, fmt) != cudaSuccess)
         return QLORA_ERR_CUDA;
     if (launch_double_quant(sums, ng, absmax, nb, out->absmax_offset, out->absmax_q8, out->absmax_scale, s,
-                            partials) != cudaSuccess)
+                            partials, fmt.dq_type) != cudaSuccess)
         return QLORA_ERR_CUDA;
     return QLORA_OK;
 }
@@ -302,22 +306,23 @@ qlora_status qlora_nf4_quantize_static(const void* W, qlora_dtype wdtype, const 
     if (n > QLORA_STATIC_QUANTIZE_MAX_ELEMS) return QLORA_ERR_WORKSPACE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const int is_bf16 = wdtype == QLORA_BF16;
+    const QFormat fmt = weight_format(*out);
     if (!out->double_quant) {
-        if (launch_quantize_blocks(W, is_bf16, n, out->codes, out->absmax, nullptr, s) != cudaSuccess)
+        if (launch_quantize_blocks(W, is_bf16, n, out->codes, out->absmax, nullptr, s, fmt) != cudaSuccess)
             return QLORA_ERR_CUDA;
         return QLORA_OK;
     }
     void* scratch = nullptr;
     st = static_quant_scratch(&scratch);
     if (st != QLORA_OK) return st;
-    const int64_t nb = (n + 63) / 64;
+    const int64_t nb = (n + out->blocksize - 1) / out->blocksize;
     const int64_t ng = (n + 16383) / 16384;
     float* absmax = static_cast<float*>(scratch);
     double* sums = reinterpret_cast<double*>(static_cast<char*>(scratch) + kStaticAbsmaxBytes);
-    if (launch_quantize_blocks(W, is_bf16, n, out->codes, absmax, sums, s) != cudaSuccess)
+    if (launch_quantize_blocks(W, is_bf16, n, out->codes, absmax, sums, s, fmt) != cudaSuccess)
         return QLORA_ERR_CUDA;
-    if (launch_double_quant(sums, ng, absmax, nb, out->absmax_offset, out->absmax_q8, out->absmax_scale, s) !=
-        cudaSuccess)
+    if (launch_double_quant(sums, ng, absmax, nb, out->absmax_offset, out->absmax_q8, out->absmax_scale, s,
+                            nullptr, fmt.dq_type) != cudaSuccess)
         return QLORA_ERR_CUDA;
     return QLORA_OK;
 }

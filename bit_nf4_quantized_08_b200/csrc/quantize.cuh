@@ -51,24 +51,31 @@ namespace qlora {
 struct SearchSmem {
     float thr[64];  // P_key
     int base[64];
+    int inc[64];
 };
 
 __device__ __forceinline__ void load_search_tables(SearchSmem& st, const Nf4SearchTable& tab) {
     for (int i = threadIdx.x; i < 64; i += blockDim.x) {
         st.thr[i] = i < 33 ? tab.thr[i] : 3.0f;
         st.base[i] = i < 33 ? tab.base[i] : 15;
+        st.inc[i] = i < 33 ? tab.inc[i] : 0;
     }
 }
 
 // t = fl(16 x + 1.5 * 2^23 + 16): x rounded to an integer bucket key in the
 // low mantissa bits (0x4B400000 + key).
+// CT = 1 (FP4): a bucket's threshold may count twice (inc = 2).
+template <int CT = 0>
 __device__ __forceinline__ uint32_t nf4_lookup(float x, float t, const SearchSmem& st) {
     const uint32_t key = __float_as_uint(t) & 63u;
-    return (uint32_t)st.base[key] + (__float_as_uint(__fsub_rn(st.thr[key], x)) >> 31);
+    const uint32_t above = __float_as_uint(__fsub_rn(st.thr[key], x)) >> 31;
+    if (CT == 0) return (uint32_t)st.base[key] + above;
+    return (uint32_t)st.base[key] + above * (uint32_t)st.inc[key];
 }
 
+template <int CT = 0>
 __device__ __forceinline__ uint32_t nf4_search(float x, const SearchSmem& st) {
-    return nf4_lookup(x, fmaf(x, 16.0f, 12582928.0f), st);
+    return nf4_lookup<CT>(x, fmaf(x, 16.0f, 12582928.0f), st);
 }
 
 // Two lanes of fp32x2 arithmetic (sm_100a packed FP32): the same IEEE
@@ -93,6 +100,7 @@ __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
 }
 
 // Codes of two elements x = fl(w * rcp) in one fp32x2 multiply and FMA.
+template <int CT = 0>
 __device__ __forceinline__ void nf4_search2(float w0, float w1, uint64_t rcp2, const SearchSmem& st, uint32_t& c0,
                                             uint32_t& c1) {
     const uint64_t x2 = f2_mul(f2_pack(w0, w1), rcp2);
@@ -100,8 +108,8 @@ __device__ __forceinline__ void nf4_search2(float w0, float w1, uint64_t rcp2, c
     float x0, x1, t0, t1;
     f2_unpack(x2, x0, x1);
     f2_unpack(t2, t0, t1);
-    c0 = nf4_lookup(x0, t0, st);
-    c1 = nf4_lookup(x1, t1, st);
+    c0 = nf4_lookup<CT>(x0, t0, st);
+    c1 = nf4_lookup<CT>(x1, t1, st);
 }
 
 // Pack 8 codes (element order) into one word: byte i = (c[2i] << 4) | c[2i+1].
@@ -113,17 +121,18 @@ __device__ __forceinline__ uint32_t pack8(const uint32_t (&c)[8]) {
 }
 
 // ---------------------------------------------------------------------------
-// K1: quantize.  One CTA (8 warps) per group of 256 blocks (16384 elements);
-// warp w handles rows 4w..4w+3 of 512 elements; a lane holds 16 consecutive
-// elements, four lanes make one block.  Also writes the group's fp64
-// pairwise-tree sum of block maxima for the double-quantization offset.
+// K1: quantize.  One CTA (8 warps) per group of 16384 elements; warp w
+// handles rows 4w..4w+3 of 512 elements; a lane holds 16 consecutive
+// elements, 4 << bs_shift lanes make one block (64, 128 or 256 elements).
+// Also writes the group's fp64 pairwise-tree sum of block maxima for the
+// double-quantization offset.  CT: code book (0 NF4, 1 FP4).
 // ---------------------------------------------------------------------------
-template <bool BF16>
+template <bool BF16, int CT>
 __global__ void __launch_bounds__(256, BF16 ? 4 : 2) k_quantize_blocks(const void* W, int64_t n,
                                                             uint8_t* codes,
                                                             float* absmax,
                                                             double* group_sums,
-                                                            Nf4SearchTable tab) {
+                                                            Nf4SearchTable tab, int bs_shift) {
     __shared__ SearchSmem st;
     __shared__ double s_wsum[8];
     // dependent launch: resident before the kernel ahead ends, no access to
@@ -136,7 +145,9 @@ __global__ void __launch_bounds__(256, BF16 ? 4 : 2) k_quantize_blocks(const voi
     __syncthreads();
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t nb = (n + 63) >> 6;
+    const int bshift = 6 + bs_shift;                  // log2 of the block size
+    const int64_t nb = (n + (1 << bshift) - 1) >> bshift;
+    const int blanes = 4 << bs_shift;                 // lanes per block
     constexpr int WORDS = BF16 ? 8 : 16;  // 32-bit words per lane per row
     uint32_t raw[4][WORDS];
     int64_t e0[4];
@@ -196,12 +207,11 @@ __global__ void __launch_bounds__(256, BF16 ? 4 : 2) k_quantize_blocks(const voi
 #pragma unroll
             for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(__uint_as_float(raw[it][i])));
         }
-        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
-        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+        for (int o = 1; o < blanes; o <<= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
 
-        const int64_t b = e0[it] >> 6;
+        const int64_t b = e0[it] >> bshift;
         const bool bvalid = b < nb;
-        if (bvalid && (lane & 3) == 0 && absmax) absmax[b] = a;
+        if (bvalid && (lane & (blanes - 1)) == 0 && absmax) absmax[b] = a;
 
         uint32_t c[16];
         if (a >= 1.17549435e-38f) {
@@ -211,7 +221,7 @@ __global__ void __launch_bounds__(256, BF16 ? 4 : 2) k_quantize_blocks(const voi
             for (int i = 0; i < 16; i += 2) {
                 const uint32_t b0 = BF16 ? (raw[it][i >> 1] << 16) : raw[it][i];
                 const uint32_t b1 = BF16 ? (raw[it][i >> 1] & 0xFFFF0000u) : raw[it][i + 1];
-                nf4_search2(__uint_as_float(b0), __uint_as_float(b1), rcp2, st, c[i], c[i + 1]);
+                nf4_search2<CT>(__uint_as_float(b0), __uint_as_float(b1), rcp2, st, c[i], c[i + 1]);
             }
         } else {
             // zero or subnormal block: exact power-of-two prescale 2^64
@@ -221,7 +231,7 @@ __global__ void __launch_bounds__(256, BF16 ? 4 : 2) k_quantize_blocks(const voi
             for (int i = 0; i < 16; ++i) {
                 const uint32_t bits = BF16 ? ((i & 1) ? (raw[it][i >> 1] & 0xFFFF0000u) : (raw[it][i >> 1] << 16))
                                            : raw[it][i];
-                c[i] = nf4_search(__fmul_rn(__fmul_rn(__uint_as_float(bits), p), rcp), st);
+                c[i] = nf4_search<CT>(__fmul_rn(__fmul_rn(__uint_as_float(bits), p), rcp), st);
             }
         }
         uint32_t lo[8], hi[8];
@@ -245,12 +255,10 @@ __global__ void __launch_bounds__(256, BF16 ? 4 : 2) k_quantize_blocks(const voi
             }
         }
 
-        // fp64 pairwise tree over the row's 8 block maxima (blocks beyond
-        // the tensor contribute zeros).
+        // fp64 pairwise tree over the row's block maxima (8, 4 or 2 of them;
+        // blocks beyond the tensor contribute zeros).
         double d = bvalid ? (double)a : 0.0;
-        d += __shfl_xor_sync(0xffffffffu, d, 4);
-        d += __shfl_xor_sync(0xffffffffu, d, 8);
-        d += __shfl_xor_sync(0xffffffffu, d, 16);
+        for (int o = blanes; o < 32; o <<= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
         rowsum[it] = d;
     }
     if (group_sums) {
@@ -362,22 +370,39 @@ __device__ __forceinline__ int nearest_t8(float y, const float* t8) {
     return best;
 }
 
+// Nearest FP8 (E4M3) code of y: the first table entry >= y by binary search
+// over the 253 sorted values, then the exact fp64 distances of it and the
+// entry below; ties to the lower index.
+__device__ __forceinline__ int nearest_e4m3(float y, const float* t) {
+    int lo = 0, hi = 253;  // first index with t[index] >= y, in [lo, hi]
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (t[mid] < y) lo = mid + 1; else hi = mid;
+    }
+    if (lo == 253) return 252;
+    if (lo == 0) return 0;
+    const double dl = fabs((double)y - (double)t[lo - 1]), dh = fabs((double)t[lo] - (double)y);
+    return dl <= dh ? lo - 1 : lo;
+}
+
 // ---------------------------------------------------------------------------
 // K3: second-level quantization; one warp per group of 256 block constants.
 // ---------------------------------------------------------------------------
 // With sums != nullptr every CTA first forms the offset itself from the
 // nsums group sums (the same pairwise tree as K2, over 256 threads) and CTA 0
 // also stores it; otherwise the offset is read from offset_ptr.
+// dt: the 8-bit code book (0 linear, 1 FP8 E4M3).
 __global__ void __launch_bounds__(256) k_dq_quantize(const float* absmax, int64_t nb,
                                                      float* offset_ptr,
                                                      uint8_t* q8,
                                                      float* c1,
-                                                     const double* sums, int64_t nsums) {
+                                                     const double* sums, int64_t nsums, int dt) {
     __shared__ float t8[256];
     __shared__ double s_w[8];
     __shared__ float s_off;
     pdl_trigger();
-    t8[threadIdx.x] = t8_value(threadIdx.x);  // blockDim.x == 256; shared memory only
+    // blockDim.x == 256; shared memory only
+    t8[threadIdx.x] = dt ? (threadIdx.x < 253 ? e4m3_value(threadIdx.x) : 2.0f) : t8_value(threadIdx.x);
     pdl_wait();
     // this warp's first group: 8 block maxima per lane, loaded before the
     // offset tree so that the two memory round trips overlap
@@ -428,7 +453,10 @@ __global__ void __launch_bounds__(256) k_dq_quantize(const float* absmax, int64_
         const float rc = (c == 0.0f) ? 0.0f : __frcp_rn(__fmul_rn(c, p));
         uint32_t q[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) q[i] = (uint32_t)nearest_t8(__fmul_rn(__fmul_rn(d[i], p), rc), t8);
+        for (int i = 0; i < 8; ++i) {
+            const float y = __fmul_rn(__fmul_rn(d[i], p), rc);
+            q[i] = (uint32_t)(dt ? nearest_e4m3(y, t8) : nearest_t8(y, t8));
+        }
         if (b0 + 8 <= nb) {
             uint2 v;
             v.x = q[0] | (q[1] << 8) | (q[2] << 16) | (q[3] << 24);
@@ -453,19 +481,20 @@ __global__ void __launch_bounds__(256) k_dequantize(const uint8_t* __restrict__ 
                                                     const uint8_t* __restrict__ q8,
                                                     const float* __restrict__ c1,
                                                     const float* __restrict__ offset_ptr,
-                                                    uint16_t* __restrict__ out) {
+                                                    uint16_t* __restrict__ out, QFormat fmt) {
     __shared__ __align__(16) uint8_t stage[8][4096];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t b = (int64_t)blockIdx.x * 256 + threadIdx.x;
     const int64_t nb = (n + 63) >> 6;
     const int64_t wb0 = (int64_t)blockIdx.x * 256 + warp * 32;  // first block of this warp
     const bool warp_full = (wb0 + 32) * 64 <= n;
+    const int64_t bb = b >> fmt.bs_shift;  // the block (of the weight's size) holding this 64
     if (warp_full) {
-        const float a = dq ? block_scale_dq(q8[b], c1[b >> 8], *offset_ptr) : absmax[b];
+        const float a = dq ? block_scale_dq(q8[bb], c1[bb >> 8], *offset_ptr, fmt.dq_type) : absmax[bb];
         const uint4* src = reinterpret_cast<const uint4*>(codes + b * 32);
         const uint4 c0 = __ldcs(src), c1v = __ldcs(src + 1);
         const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1v.x, c1v.y, c1v.z, c1v.w};
-        const Nf4BlockTable t = nf4_block_table(a);
+        const Nf4BlockTable t = nf4_block_table(a, fmt.code_type);
         const uint32_t slot = smem_u32(&stage[warp][0]) + lane * 128;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -486,12 +515,12 @@ __global__ void __launch_bounds__(256) k_dequantize(const uint8_t* __restrict__ 
         return;
     }
     if (b >= nb) return;
-    const float a = dq ? block_scale_dq(q8[b], c1[b >> 8], *offset_ptr) : absmax[b];
+    const float a = dq ? block_scale_dq(q8[bb], c1[bb >> 8], *offset_ptr, fmt.dq_type) : absmax[bb];
     if ((b + 1) * 64 <= n) {
         const uint4* src = reinterpret_cast<const uint4*>(codes + b * 32);
         uint4 c0 = __ldg(src), c1v = __ldg(src + 1);
         const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1v.x, c1v.y, c1v.z, c1v.w};
-        const Nf4BlockTable t = nf4_block_table(a);
+        const Nf4BlockTable t = nf4_block_table(a, fmt.code_type);
         uint4* dst = reinterpret_cast<uint4*>(out + b * 64);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -503,7 +532,7 @@ __global__ void __launch_bounds__(256) k_dequantize(const uint8_t* __restrict__ 
         for (int64_t e = b * 64; e < n; ++e) {
             uint8_t byte = codes[e >> 1];
             int c = (e & 1) ? (byte & 15) : (byte >> 4);
-            __nv_bfloat16 h = __float2bfloat16_rn(__fmul_rn(nf4_value(c), a));
+            __nv_bfloat16 h = __float2bfloat16_rn(__fmul_rn(code_value(fmt.code_type, c), a));
             out[e] = *reinterpret_cast<uint16_t*>(&h);
         }
     }
@@ -514,7 +543,7 @@ __global__ void __launch_bounds__(256) k_dequantize(const uint8_t* __restrict__ 
 __global__ void k_expand_scales(int64_t rows, int64_t kbs, int dq, const float* absmax,
                                 const uint8_t* q8, const float* c1,
                                 const float* offset_ptr, float* scales,
-                                int64_t ld, int* flags, int nflags) {
+                                int64_t ld, int* flags, int nflags, QFormat fmt) {
     // the LoRA GEMM that follows reads none of this kernel's outputs; this
     // kernel's inputs (8-bit constants) and outputs (scales, flags of the
     // GEMM before) belong to the kernel before it
@@ -524,8 +553,8 @@ __global__ void k_expand_scales(int64_t rows, int64_t kbs, int dq, const float* 
     if (idx < nflags) flags[idx] = 0;
     if (idx >= rows * kbs) return;
     const int64_t kb = idx / rows, n = idx - kb * rows;
-    const int64_t b = n * kbs + kb;
-    scales[kb * ld + n] = dq ? block_scale_dq(q8[b], c1[b >> 8], *offset_ptr) : absmax[b];
+    const int64_t b = (n * kbs + kb) >> fmt.bs_shift;  // flattened block of the weight's block size
+    scales[kb * ld + n] = dq ? block_scale_dq(q8[b], c1[b >> 8], *offset_ptr, fmt.dq_type) : absmax[b];
 }
 
 __global__ void k_encode(const float* __restrict__ x, int64_t n, uint8_t* __restrict__ codes,
@@ -536,7 +565,7 @@ __global__ void k_encode(const float* __restrict__ x, int64_t n, uint8_t* __rest
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
          i += (int64_t)gridDim.x * blockDim.x) {
         float v = fminf(fmaxf(x[i], -1.0f), 1.0f);
-        codes[i] = (uint8_t)nf4_search(v, st);
+        codes[i] = (uint8_t)nf4_search<0>(v, st);
     }
 }
 
@@ -551,11 +580,23 @@ inline void nf4_table_host(float out[16]) {
     }
 }
 
-inline Nf4SearchTable build_search_table() {
+// Search table of a 16-value code book (ct 0 NF4, 1 FP4).  Threshold j is
+// the smallest fp32 above which the nearest value (ties to the lower index)
+// has an index above j: above the exact midpoint of values j and j+1, or,
+// when the two values are equal (the two zeros of FP4, where index 8 is
+// never the nearest), the next threshold.
+inline Nf4SearchTable build_search_table(int ct) {
     float v[16];
-    nf4_table_host(v);
+    for (int j = 0; j < 16; ++j) {
+        uint32_t u = kCodeBits[ct][j];
+        memcpy(&v[j], &u, 4);
+    }
     float thr[15];
-    for (int j = 0; j < 15; ++j) {
+    for (int j = 14; j >= 0; --j) {
+        if ((double)v[j] == (double)v[j + 1]) {
+            thr[j] = thr[j + 1];
+            continue;
+        }
         double mid = 0.5 * ((double)v[j] + (double)v[j + 1]);  // exact in fp64
         float f = (float)mid;
         if ((double)f <= mid) f = std::nextafter(f, INFINITY);
@@ -564,34 +605,41 @@ inline Nf4SearchTable build_search_table() {
     Nf4SearchTable t;
     for (int k = 0; k <= 32; ++k) {
         double lo = (k - 0.5) / 16.0 - 1.0, hi = (k + 0.5) / 16.0 - 1.0;
-        int base = 0;
+        int base = 0, inc = 0;
         float tk = 3.0f;  // no threshold inside the bucket
         for (int j = 0; j < 15; ++j) {
-            if ((double)thr[j] <= lo) ++base;
-            else if ((double)thr[j] <= hi) tk = thr[j];
+            if ((double)thr[j] <= lo) {
+                ++base;
+            } else if ((double)thr[j] <= hi) {
+                tk = thr[j];
+                ++inc;
+            }
         }
         t.thr[k] = std::nextafter(tk, -INFINITY);  // P_key: x >= T_key  <=>  x > P_key
         t.base[k] = base;
+        t.inc[k] = inc;
     }
     return t;
 }
 
-inline const Nf4SearchTable& nf4_search_table() {
-    static const Nf4SearchTable t = build_search_table();
-    return t;
+inline const Nf4SearchTable& search_table(int ct) {
+    static const Nf4SearchTable t[2] = {build_search_table(0), build_search_table(1)};
+    return t[ct];
 }
+inline const Nf4SearchTable& nf4_search_table() { return search_table(0); }
 
 inline cudaError_t launch_quantize_blocks(const void* W, int is_bf16, int64_t n, uint8_t* codes,
-                                          float* absmax, double* group_sums, cudaStream_t s) {
+                                          float* absmax, double* group_sums, cudaStream_t s,
+                                          QFormat fmt = QFormat{0, 0, 0}) {
     const int64_t ng = (n + 16383) / 16384;
     if (ng == 0) return cudaSuccess;
     ProfileScope ps(QLORA_KERNEL_QUANTIZE, s);
     note_launch();
-    if (is_bf16)
-        return launch_pdl(k_quantize_blocks<true>, dim3((unsigned)ng), dim3(256), 0, s, 0, W, n, codes, absmax,
-                          group_sums, nf4_search_table());
-    return launch_pdl(k_quantize_blocks<false>, dim3((unsigned)ng), dim3(256), 0, s, 0, W, n, codes, absmax,
-                      group_sums, nf4_search_table());
+    const Nf4SearchTable& tab = search_table(fmt.code_type);
+    auto kern = is_bf16 ? (fmt.code_type ? k_quantize_blocks<true, 1> : k_quantize_blocks<true, 0>)
+                        : (fmt.code_type ? k_quantize_blocks<false, 1> : k_quantize_blocks<false, 0>);
+    return launch_pdl(kern, dim3((unsigned)ng), dim3(256), 0, s, 0, W, n, codes, absmax, group_sums, tab,
+                      fmt.bs_shift);
 }
 
 inline cudaError_t launch_dq_offset(const double* group_sums, int64_t ngroups, int64_t nb,
@@ -601,7 +649,8 @@ inline cudaError_t launch_dq_offset(const double* group_sums, int64_t ngroups, i
 }
 
 inline cudaError_t launch_dq_quantize(const float* absmax, int64_t nb, float* offset, uint8_t* q8, float* c1,
-                                      cudaStream_t s, const double* sums = nullptr, int64_t nsums = 0) {
+                                      cudaStream_t s, const double* sums = nullptr, int64_t nsums = 0,
+                                      int dt = 0) {
     const int64_t ng = (nb + 255) / 256;
     if (ng == 0) return cudaSuccess;
     int dev = 0, nsm = 148;
@@ -611,7 +660,7 @@ inline cudaError_t launch_dq_quantize(const float* absmax, int64_t nb, float* of
     const int64_t grid = std::min<int64_t>((ng + 7) / 8, (int64_t)8 * nsm);
     note_launch();
     return launch_pdl(k_dq_quantize, dim3((unsigned)grid), dim3(256), 0, s, 0, absmax, nb, offset, q8, c1, sums,
-                      nsums);
+                      nsums, dt);
 }
 
 // Double quantization of the block maxima: offset, then 8-bit codes.  Up to
@@ -629,18 +678,23 @@ inline int64_t dq_partial_count(int64_t nsums) {
 }
 inline cudaError_t launch_double_quant(const double* sums, int64_t nsums, const float* absmax, int64_t nb,
                                        float* offset, uint8_t* q8, float* c1, cudaStream_t s,
-                                       double* partials = nullptr) {
-    if (nsums <= kFusedSums && inject_mode() != 5) return launch_dq_quantize(absmax, nb, offset, q8, c1, s, sums, nsums);
+                                       double* partials = nullptr, int dt = 0) {
+    if (nsums <= kFusedSums && inject_mode() != 5)
+        return launch_dq_quantize(absmax, nb, offset, q8, c1, s, sums, nsums, dt);
     const int64_t G = dq_partial_count(nsums);
     if (G > 0 && partials && inject_mode() != 5) {
         note_launch();
         cudaError_t e = launch_pdl(k_dq_partials, dim3((unsigned)G), dim3(256), 0, s, 0, sums, nsums, partials);
         if (e != cudaSuccess) return e;
-        return launch_dq_quantize(absmax, nb, offset, q8, c1, s, partials, G);
+        return launch_dq_quantize(absmax, nb, offset, q8, c1, s, partials, G, dt);
     }
     cudaError_t e = launch_dq_offset(sums, nsums, nb, offset, s);
     if (e != cudaSuccess) return e;
-    return launch_dq_quantize(absmax, nb, offset, q8, c1, s);
+    return launch_dq_quantize(absmax, nb, offset, q8, c1, s, nullptr, 0, dt);
+}
+
+inline QFormat weight_format(const qlora_nf4_weight& w) {
+    return QFormat{w.code_type, w.dq_type, w.blocksize == 256 ? 2 : (w.blocksize == 128 ? 1 : 0)};
 }
 
 inline cudaError_t launch_dequantize(const qlora_nf4_weight& w, uint16_t* out, cudaStream_t s) {
@@ -650,7 +704,7 @@ inline cudaError_t launch_dequantize(const qlora_nf4_weight& w, uint16_t* out, c
     ProfileScope ps(QLORA_KERNEL_DEQUANTIZE, s);
     note_launch();
     k_dequantize<<<(unsigned)((nb + 255) / 256), 256, 0, s>>>(
-        w.codes, n, w.double_quant, w.absmax, w.absmax_q8, w.absmax_scale, w.absmax_offset, out);
+        w.codes, n, w.double_quant, w.absmax, w.absmax_q8, w.absmax_scale, w.absmax_offset, out, weight_format(w));
     return cudaGetLastError();
 }
 
@@ -664,7 +718,8 @@ inline cudaError_t launch_expand_scales(const qlora_nf4_weight& w, float* scales
     // ends and wait for it (pdl_wait) before any access
     return launch_pdl(k_expand_scales, dim3((unsigned)((total + 255) / 256)), dim3(256), 0, s, 0, w.rows, kbs,
                       (int)w.double_quant, (const float*)w.absmax, (const uint8_t*)w.absmax_q8,
-                      (const float*)w.absmax_scale, (const float*)w.absmax_offset, scales, ld, flags, nflags);
+                      (const float*)w.absmax_scale, (const float*)w.absmax_offset, scales, ld, flags, nflags,
+                      weight_format(w));
 }
 
 inline cudaError_t launch_encode(const float* x, int64_t n, uint8_t* codes, cudaStream_t s) {

@@ -42,6 +42,7 @@ struct SmallMParams {
     int N, M, kbs;        // kbs = K / 64
     int ks_main, ks_lora, tiles;
     int seg_rows, seg_r;  // fused projection: sU columns of tile t start at (128 t / seg_rows) seg_r
+    QFormat fmt;          // code book, 8-bit code book, block size
     uint16_t* Y;          // [M][N] bf16
     float* part;          // [gridDim.x][NT][128] fp32 partial tiles
     uint32_t* flags;      // [gridDim.x][4] epoch of the published partial, per TMEM quarter
@@ -118,7 +119,7 @@ __global__ void __launch_bounds__(SmallMShape<NT, NG>::THREADS, 1)
         *abort_flag = 0;
         fence_mbar_init();
     }
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) t8s[i] = t8_value(i);
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) t8s[i] = dq_value(p.fmt.dq_type, i < 253 ? i : 0);
     if (warp == 0 && lane == 0) {
         pdl_trigger();
         prefetch_tensormap(&p.tmCodes);
@@ -325,7 +326,7 @@ __global__ void __launch_bounds__(SmallMShape<NT, NG>::THREADS, 1)
             const int tile = (int)(unit / KS), k = (int)(unit - (int64_t)tile * KS);
             const int n = tile * 128 + t;
             if (k >= p.ks_main || n >= p.N) return r;
-            const int64_t b = (int64_t)n * p.kbs + k;
+            const int64_t b = ((int64_t)n * p.kbs + k) >> p.fmt.bs_shift;
             if (!p.dq) {
                 r.q = 0;
                 r.c = __ldg(p.absmax + b);
@@ -377,7 +378,7 @@ __global__ void __launch_bounds__(SmallMShape<NT, NG>::THREADS, 1)
                 const uint4 c0 = ld_shared_v4(sC + code_off);
                 const uint4 c1 = ld_shared_v4(sC + code_off2);
                 const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-                const Nf4BlockTable tb = nf4_block_table(block_const(rw));
+                const Nf4BlockTable tb = nf4_block_table(block_const(rw), p.fmt.code_type);
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
                     uint32_t o[4];

@@ -28,10 +28,12 @@
 // it every thread reads 8 contiguous code bytes per weight row and 32
 // contiguous bytes of X per token for a block.
 //
-// Work split: items are (group of 16R weight rows, 64-wide k-step), the
-// LoRA up-projection as extra k-steps after the K/64 weight steps; every
-// warp of a persistent grid takes one contiguous share of the item list
-// (stream-K), so each streams the same number of weight bytes.  A group cut
+// Work split: items are (group of 16R weight rows, four 64-element blocks),
+// so that each row is read in whole 128-byte lines, with the LoRA
+// up-projection as extra 64-wide items after the weight items; every warp of
+// a persistent grid takes one contiguous share of the item list (stream-K),
+// so each streams the same number of weight bytes, and loads the codes of
+// its next item while it computes the current one.  A group cut
 // between warps is finished by whichever of its warps arrives last (an
 // integer counter): it adds every warp's fp32 partial in warp order
 // (deterministic) and writes Y.  Nothing waits on another warp.
@@ -42,7 +44,9 @@
 
 namespace qlora {
 
-constexpr float kSmallMTableScale = 1.18881f;
+// Prescale L of the table per code book: for NF4 it halves the bf16 error of
+// the 16 values; for FP4 (multiples of 1/12) 1.5 makes every value exact.
+__device__ __forceinline__ float small_m_table_scale(int ct) { return ct ? 1.5f : 1.18881f; }
 
 struct SmallMmaParams {
     const uint8_t* codes;   // [N][K/2]
@@ -56,8 +60,10 @@ struct SmallMmaParams {
     const uint16_t* sU;     // [M][rt] bf16
     int M, N, K, KB;        // KB = K / 64
     int r, rt, seg_rows, lora_ks;
-    float inv_scale;        // 1 / kSmallMTableScale
-    int GL;                 // items per group: KB + lora_ks
+    float inv_scale;        // 1 / L
+    QFormat fmt;            // code book, 8-bit code book, block size
+    int QW;                 // weight items per group: ceil(KB / QB)
+    int GL;                 // items per group: QW + lora_ks
     int64_t items;          // groups * GL
     uint16_t* Y;            // [M][N]
     float* part;            // [warps][2][16R][8 NT8] fp32 partials
@@ -71,6 +77,7 @@ struct SmallMmaShape {
     static constexpr int THREADS = 32 * WARPS;
     static constexpr int NPAD = 8 * NT8;
     static constexpr int GROWS = 16 * R;
+    static constexpr int QB = 4;  // 64-element blocks per weight item: a 128-byte line of every row
     // 64 KB table at the first 64 KB-aligned shared address, the fp32 t8
     // table of the double quantization below it
     static constexpr int SMEM = 2 * 65536;
@@ -128,11 +135,13 @@ __global__ void __launch_bounds__(SmallMmaShape<NT8, R>::THREADS, 1)
     // tables: entry e = {L nf4[e >> 4] (bits 0..15), L nf4[e & 15] (bits 16..31)}
     for (int idx = threadIdx.x; idx < 256 * 32; idx += blockDim.x) {
         const int e = idx >> 5, l = idx & 31;
-        const float vlo = __fmul_rn(nf4_value(e >> 4), kSmallMTableScale);
-        const float vhi = __fmul_rn(nf4_value(e & 15), kSmallMTableScale);
+        const float L = small_m_table_scale(p.fmt.code_type);
+        const float vlo = __fmul_rn(code_value(p.fmt.code_type, e >> 4), L);
+        const float vhi = __fmul_rn(code_value(p.fmt.code_type, e & 15), L);
         sts_u32(lut_base + (uint32_t)(e * 256 + l * 4), pack_bf16x2(vlo, vhi));
     }
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) sts_u32(t8s + 4u * i, __float_as_uint(t8_value(i)));
+    for (int i = threadIdx.x; i < 256; i += blockDim.x)
+        sts_u32(t8s + 4u * i, __float_as_uint(dq_value(p.fmt.dq_type, i < 253 ? i : 0)));
     __syncthreads();
     // the weight, X and the adapter operands may come from the kernels just
     // before (the quantizer, the sU GEMM, an earlier layer): wait for them
@@ -145,43 +154,59 @@ __global__ void __launch_bounds__(SmallMmaShape<NT8, R>::THREADS, 1)
     const int64_t I = p.items;
     const int64_t i0 = (I * w) / G, i1 = (I * (w + 1)) / G;
     const int64_t rowb = p.K / 2;  // code bytes per weight row
+    constexpr int QB = S::QB;
 
-    for (int64_t it = i0; it < i1;) {
-        const int g = (int)(it / p.GL);
-        const int kb0 = (int)(it - (int64_t)g * p.GL);
-        const int kb1 = (int)min((int64_t)p.GL, (int64_t)kb0 + (i1 - it));
+    // code bytes (8 per row and block: this thread's quarter of each 32-byte
+    // block chunk) and 8-bit block codes of one weight item, loaded one item
+    // ahead of its use
+    struct Pf {
+        uint2 cw[R][2][QB];
+        uint32_t q8[R][2];  // QB block codes, byte j = block j
+    };
+    auto prefetch = [&](int64_t item, Pf& f) {
+        const int g = (int)(item / p.GL), kq = (int)(item - (int64_t)g * p.GL);
+        if (kq >= p.QW) return;  // LoRA item: nothing to fetch ahead
         const int n0 = g * GROWS;
-        float acc[R][NT8][4];
 #pragma unroll
-        for (int a = 0; a < R; ++a)
+        for (int rt = 0; rt < R; ++rt)
 #pragma unroll
-            for (int b = 0; b < NT8; ++b)
+            for (int h = 0; h < 2; ++h) {
+                const int n = n0 + 16 * rt + gid + 8 * h;
+                uint32_t q = 0;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) acc[a][b][c] = 0.0f;
-
-        // rows of this thread: n0 + 16 rt + gid (+ 8)
-        for (int kb = kb0; kb < kb1; ++kb) {
-            if (kb < p.KB) {
-                // -------------------------------------------------- weight k-step
-                uint2 cw[R][2];
-                float sc[R][2];
-#pragma unroll
-                for (int rt = 0; rt < R; ++rt)
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int n = n0 + 16 * rt + gid + 8 * h;
-                        if (n < p.N) {
-                            cw[rt][h] = __ldcs(reinterpret_cast<const uint2*>(p.codes + (int64_t)n * rowb + kb * 32 + 8 * tig));
-                            const int64_t b = (int64_t)n * p.KB + kb;
-                            const float a = p.dq ? __fadd_rn(__fmul_rn(lds_f32(t8s + 4u * __ldg(p.q8 + b)),
-                                                                       __ldg(p.c1 + (b >> 8))), off)
-                                                 : __ldg(p.absmax + b);
-                            sc[rt][h] = __fmul_rn(a, p.inv_scale);
-                        } else {
-                            cw[rt][h] = make_uint2(0u, 0u);
-                            sc[rt][h] = 0.0f;
-                        }
+                for (int j = 0; j < QB; ++j) {
+                    const int kb = kq * QB + j;
+                    if (n < p.N && kb < p.KB) {
+                        f.cw[rt][h][j] = __ldcs(reinterpret_cast<const uint2*>(p.codes + (int64_t)n * rowb + kb * 32 + 8 * tig));
+                        if (p.dq) q |= (uint32_t)__ldg(p.q8 + (((int64_t)n * p.KB + kb) >> p.fmt.bs_shift)) << (8 * j);
+                    } else {
+                        f.cw[rt][h][j] = make_uint2(0u, 0u);
                     }
+                }
+                f.q8[rt][h] = q;
+            }
+    };
+
+    float acc[R][NT8][4];
+#pragma unroll
+    for (int a = 0; a < R; ++a)
+#pragma unroll
+        for (int b = 0; b < NT8; ++b)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[a][b][c] = 0.0f;
+    Pf cur, nxt;
+    if (i0 < i1) prefetch(i0, cur);
+    for (int64_t it = i0; it < i1; ++it) {
+        if (it + 1 < i1) prefetch(it + 1, nxt);
+        const int g = (int)(it / p.GL);
+        const int kq = (int)(it - (int64_t)g * p.GL);
+        const int n0 = g * GROWS;
+        if (kq < p.QW) {
+            // ------------------------------------------------------ weight item: QB blocks
+#pragma unroll
+            for (int j = 0; j < QB; ++j) {
+                const int kb = kq * QB + j;
+                if (kb >= p.KB) break;
                 uint32_t xf[NT8][8];
 #pragma unroll
                 for (int nt = 0; nt < NT8; ++nt) {
@@ -198,12 +223,26 @@ __global__ void __launch_bounds__(SmallMmaShape<NT8, R>::THREADS, 1)
                 }
 #pragma unroll
                 for (int rt = 0; rt < R; ++rt) {
+                    float sc[2];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int n = n0 + 16 * rt + gid + 8 * h;
+                        float a = 0.0f;
+                        if (n < p.N) {
+                            const int64_t b = ((int64_t)n * p.KB + kb) >> p.fmt.bs_shift;
+                            a = p.dq ? __fadd_rn(__fmul_rn(lds_f32(t8s + 4u * ((cur.q8[rt][h] >> (8 * j)) & 0xFFu)),
+                                                           __ldg(p.c1 + (b >> 8))), off)
+                                     : __ldg(p.absmax + b);
+                        }
+                        sc[h] = __fmul_rn(a, p.inv_scale);
+                    }
                     float d[NT8][4];
 #pragma unroll
                     for (int nt = 0; nt < NT8; ++nt)
 #pragma unroll
                         for (int q = 0; q < 4; ++q) d[nt][q] = 0.0f;
-                    const uint32_t g0x = cw[rt][0].x, g0y = cw[rt][0].y, g8x = cw[rt][1].x, g8y = cw[rt][1].y;
+                    const uint32_t g0x = cur.cw[rt][0][j].x, g0y = cur.cw[rt][0][j].y;
+                    const uint32_t g8x = cur.cw[rt][1][j].x, g8y = cur.cw[rt][1][j].y;
                     {   // chunk 0: bytes 0, 1
                         const uint32_t a0 = lut<0>(g0x, lane_base), a2 = lut<1>(g0x, lane_base);
                         const uint32_t a1 = lut<0>(g8x, lane_base), a3 = lut<1>(g8x, lane_base);
@@ -230,61 +269,64 @@ __global__ void __launch_bounds__(SmallMmaShape<NT8, R>::THREADS, 1)
                     }
 #pragma unroll
                     for (int nt = 0; nt < NT8; ++nt) {
-                        acc[rt][nt][0] = __fmaf_rn(sc[rt][0], d[nt][0], acc[rt][nt][0]);
-                        acc[rt][nt][1] = __fmaf_rn(sc[rt][0], d[nt][1], acc[rt][nt][1]);
-                        acc[rt][nt][2] = __fmaf_rn(sc[rt][1], d[nt][2], acc[rt][nt][2]);
-                        acc[rt][nt][3] = __fmaf_rn(sc[rt][1], d[nt][3], acc[rt][nt][3]);
+                        acc[rt][nt][0] = __fmaf_rn(sc[0], d[nt][0], acc[rt][nt][0]);
+                        acc[rt][nt][1] = __fmaf_rn(sc[0], d[nt][1], acc[rt][nt][1]);
+                        acc[rt][nt][2] = __fmaf_rn(sc[1], d[nt][2], acc[rt][nt][2]);
+                        acc[rt][nt][3] = __fmaf_rn(sc[1], d[nt][3], acc[rt][nt][3]);
                     }
                 }
-            } else {
-                // -------------------------------------------------- LoRA k-step: B rows x sU
-                const int j0 = (kb - p.KB) * 64 + 16 * tig;  // adapter column of this thread's 16
-                const bool v0 = j0 + 8 <= p.r, v1 = j0 + 16 <= p.r;
-                const int ucol = (p.seg_rows ? (n0 / p.seg_rows) * p.r : 0) + j0;
-                uint32_t xf[NT8][8];
+            }
+        } else {
+            // ------------------------------------------------------ LoRA item: 64 adapter columns, B rows x sU
+            const int j0 = (kq - p.QW) * 64 + 16 * tig;  // adapter column of this thread's 16
+            const bool v0 = j0 + 8 <= p.r, v1 = j0 + 16 <= p.r;
+            const int ucol = (p.seg_rows ? (n0 / p.seg_rows) * p.r : 0) + j0;
+            uint32_t xf[NT8][8];
 #pragma unroll
-                for (int nt = 0; nt < NT8; ++nt) {
-                    const int m = nt * 8 + gid;
+            for (int nt = 0; nt < NT8; ++nt) {
+                const int m = nt * 8 + gid;
+                uint4 u0 = make_uint4(0, 0, 0, 0), u1 = make_uint4(0, 0, 0, 0);
+                if (m < p.M) {
+                    const uint4* src = reinterpret_cast<const uint4*>(p.sU + (int64_t)m * p.rt + ucol);
+                    if (v0) u0 = __ldg(src);
+                    if (v1) u1 = __ldg(src + 1);
+                }
+                xf[nt][0] = u0.x; xf[nt][1] = u0.y; xf[nt][2] = u0.z; xf[nt][3] = u0.w;
+                xf[nt][4] = u1.x; xf[nt][5] = u1.y; xf[nt][6] = u1.z; xf[nt][7] = u1.w;
+            }
+#pragma unroll
+            for (int rt = 0; rt < R; ++rt) {
+                uint32_t bw[2][8];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int n = n0 + 16 * rt + gid + 8 * h;
                     uint4 u0 = make_uint4(0, 0, 0, 0), u1 = make_uint4(0, 0, 0, 0);
-                    if (m < p.M) {
-                        const uint4* src = reinterpret_cast<const uint4*>(p.sU + (int64_t)m * p.rt + ucol);
+                    if (n < p.N) {
+                        const uint4* src = reinterpret_cast<const uint4*>(p.B + (int64_t)n * p.r + j0);
                         if (v0) u0 = __ldg(src);
                         if (v1) u1 = __ldg(src + 1);
                     }
-                    xf[nt][0] = u0.x; xf[nt][1] = u0.y; xf[nt][2] = u0.z; xf[nt][3] = u0.w;
-                    xf[nt][4] = u1.x; xf[nt][5] = u1.y; xf[nt][6] = u1.z; xf[nt][7] = u1.w;
+                    bw[h][0] = u0.x; bw[h][1] = u0.y; bw[h][2] = u0.z; bw[h][3] = u0.w;
+                    bw[h][4] = u1.x; bw[h][5] = u1.y; bw[h][6] = u1.z; bw[h][7] = u1.w;
                 }
 #pragma unroll
-                for (int rt = 0; rt < R; ++rt) {
-                    uint32_t bw[2][8];
+                for (int c = 0; c < 4; ++c)
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int n = n0 + 16 * rt + gid + 8 * h;
-                        uint4 u0 = make_uint4(0, 0, 0, 0), u1 = make_uint4(0, 0, 0, 0);
-                        if (n < p.N) {
-                            const uint4* src = reinterpret_cast<const uint4*>(p.B + (int64_t)n * p.r + j0);
-                            if (v0) u0 = __ldg(src);
-                            if (v1) u1 = __ldg(src + 1);
-                        }
-                        bw[h][0] = u0.x; bw[h][1] = u0.y; bw[h][2] = u0.z; bw[h][3] = u0.w;
-                        bw[h][4] = u1.x; bw[h][5] = u1.y; bw[h][6] = u1.z; bw[h][7] = u1.w;
-                    }
-#pragma unroll
-                    for (int c = 0; c < 4; ++c)
-#pragma unroll
-                        for (int nt = 0; nt < NT8; ++nt)
-                            mma_16816(acc[rt][nt], bw[0][2 * c], bw[1][2 * c], bw[0][2 * c + 1], bw[1][2 * c + 1],
-                                      xf[nt][2 * c], xf[nt][2 * c + 1]);
-                }
+                    for (int nt = 0; nt < NT8; ++nt)
+                        mma_16816(acc[rt][nt], bw[0][2 * c], bw[1][2 * c], bw[0][2 * c + 1], bw[1][2 * c + 1],
+                                  xf[nt][2 * c], xf[nt][2 * c + 1]);
             }
         }
+        cur = nxt;
 
-        // -------------------------------------------------------------- output
-        const bool whole = kb0 == 0 && kb1 == p.GL;
+        // ---------------------------------------------------------- end of a segment: output
+        if (it + 1 < i1 && kq + 1 < p.GL) continue;
+        const int64_t gstart = (int64_t)g * p.GL;
+        const int64_t seg0 = i0 > gstart ? i0 : gstart;
+        const bool whole = seg0 == gstart && kq + 1 == p.GL;
         bool write_y = whole;
         if (!whole) {
-            const int64_t gstart = (int64_t)g * p.GL;
-            const int slot = it > gstart ? 0 : (i0 < gstart ? 1 : 0);
+            const int slot = seg0 > gstart ? 0 : (i0 < gstart ? 1 : 0);
             float* mine = p.part + ((int64_t)w * 2 + slot) * (GROWS * NPAD);
 #pragma unroll
             for (int rt = 0; rt < R; ++rt)
@@ -296,25 +338,25 @@ __global__ void __launch_bounds__(SmallMmaShape<NT8, R>::THREADS, 1)
                                make_float2(acc[rt][nt][2 * h], acc[rt][nt][2 * h + 1]));
             __threadfence();
             __syncwarp();
-            // arrivals of this launch at the group's counter (epoch in the high bits)
             // contributors: the warps from the one holding the group's first
             // item to the one holding its last, less any with an empty share
             const int wf = owner_warp(gstart, I, G), wl = owner_warp(gstart + p.GL - 1, I, G);
             uint32_t ncontrib = 0;
             for (int c = wf; c <= wl; ++c) ncontrib += ((I * c) / G < (I * (c + 1)) / G) ? 1u : 0u;
+            // arrivals of this launch at the group's counter (epoch in the high bits)
             uint32_t before = 0;
             if (lane == 0) {
                 uint32_t* ctr = p.counters + g;
-                uint32_t cur = *reinterpret_cast<volatile uint32_t*>(ctr);
+                uint32_t cv = *reinterpret_cast<volatile uint32_t*>(ctr);
                 while (true) {
-                    const bool same = (cur >> 8) == p.epoch;
-                    const uint32_t want = same ? cur + 1u : ((p.epoch << 8) | 1u);
-                    const uint32_t prev = atomicCAS(ctr, cur, want);
-                    if (prev == cur) {
-                        before = same ? (cur & 0xFFu) : 0u;
+                    const bool same = (cv >> 8) == p.epoch;
+                    const uint32_t want = same ? cv + 1u : ((p.epoch << 8) | 1u);
+                    const uint32_t prev = atomicCAS(ctr, cv, want);
+                    if (prev == cv) {
+                        before = same ? (cv & 0xFFu) : 0u;
                         break;
                     }
-                    cur = prev;
+                    cv = prev;
                 }
                 if (before + 1 == ncontrib) *ctr = 0u;  // last arrival: reset for the next launch
             }
@@ -364,7 +406,12 @@ __global__ void __launch_bounds__(SmallMmaShape<NT8, R>::THREADS, 1)
                         }
                 }
         }
-        it += kb1 - kb0;
+#pragma unroll
+        for (int a = 0; a < R; ++a)
+#pragma unroll
+            for (int b = 0; b < NT8; ++b)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) acc[a][b][c] = 0.0f;
     }
 }
 

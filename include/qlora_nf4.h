@@ -45,8 +45,9 @@ typedef struct CUstream_st *qlora_stream_t; /* same type as cudaStream_t */
 typedef enum {
     QLORA_OK = 0,
     QLORA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, negative size, small workspace */
-    QLORA_ERR_UNSUPPORTED = 2, /* valid but outside this build: blocksize != 64,
-                                  K % 64 != 0, N % 8 != 0, r % 8 != 0, r > 256 */
+    QLORA_ERR_UNSUPPORTED = 2, /* valid but outside this build: blocksize not 64,
+                                  128 or 256, K % 64 != 0, N % 8 != 0,
+                                  r % 8 != 0, r > 256 */
     QLORA_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
     QLORA_ERR_TIMEOUT = 4,     /* a bounded in-kernel wait ran out (reported
                                   by qlora_get_last_error only) */
@@ -58,9 +59,10 @@ typedef enum { QLORA_F32 = 0, QLORA_BF16 = 1 } qlora_dtype;
 
 /*
  * A quantized frozen weight W [rows = N, cols = K].
- * Blocks are 64 consecutive elements of the row-major flattened tensor
- * (QLoRA tutorial "11.3 QLoRA", section "double quantization": 64 parameters
- * share one constant); nb = ceil(rows*cols / 64), nb2 = ceil(nb / 256).
+ * Blocks are `blocksize` (64 in the pages) consecutive elements of the
+ * row-major flattened tensor (QLoRA tutorial "11.3 QLoRA", section "double
+ * quantization": 64 parameters share one constant);
+ * nb = ceil(rows*cols / blocksize), nb2 = ceil(nb / 256).
  *   codes          [ceil(rows*cols/2)] bytes.  Element 2i sits in the high
  *                  nibble of byte i, element 2i+1 in the low nibble; the
  *                  nibble is the index (0..15) of the nearest NF4 code.
@@ -78,18 +80,43 @@ typedef enum { QLORA_F32 = 0, QLORA_BF16 = 1 } qlora_dtype;
 typedef struct {
     int64_t rows;          /* N (d_out) */
     int64_t cols;          /* K (d_in)  */
-    int32_t blocksize;     /* must be 64 */
+    int32_t blocksize;     /* 64 (the pages' value), 128 or 256 */
     int32_t double_quant;  /* 0 or 1 */
     uint8_t *codes;
     float *absmax;
     uint8_t *absmax_q8;
     float *absmax_scale;
     float *absmax_offset;
+    int32_t code_type;     /* QLORA_CODE_NF4 (0) or QLORA_CODE_FP4 (1) */
+    int32_t dq_type;       /* QLORA_DQ_INT8 (0) or QLORA_DQ_FP8 (1) */
 } qlora_nf4_weight;
 
 /*
+ * Data-type variants (QLoRA paper digest, sec. 6: "Float4 (FP4)" against
+ * NFloat4; sec. 4: the double-quantized constants "c2^FP8"):
+ *  QLORA_CODE_NF4  the 16 NF4 values above.
+ *  QLORA_CODE_FP4  the 16 values of a 4-bit float with 1 sign, 2 exponent
+ *                  (bias 1) and 1 mantissa bit (magnitudes 0, 0.5, 1, 1.5, 2,
+ *                  3, 4, 6) divided by 6, sorted: index 7 is -0 and index 8
+ *                  +0; the nearest-code rule (ties to the lower index) never
+ *                  stores 8.
+ *  QLORA_DQ_INT8   t8[k] = (k - 127) / 127, k = 0..254 (as above).
+ *  QLORA_DQ_FP8    the 253 distinct finite values of the 8-bit float E4M3
+ *                  (1 sign, 4 exponent bits with bias 7, 3 mantissa bits;
+ *                  largest 448) divided by 448, sorted; q8 = 0..252.
+ * Every entry point accepts every combination, with block sizes 64, 128 and
+ * 256 (blocks of consecutive elements of the flattened tensor).  A struct
+ * that leaves the two fields 0 is the NF4 / linear 8-bit format.
+ */
+#define QLORA_CODE_NF4 0
+#define QLORA_CODE_FP4 1
+#define QLORA_DQ_INT8 0
+#define QLORA_DQ_FP8 1
+
+/*
  * Workspace bytes that qlora_nf4_quantize needs for a tensor of rows*cols
- * elements (0 when double_quant == 0).  Returns 0 for invalid sizes.
+ * elements in blocks of `blocksize` (0 when double_quant == 0).  Returns 0
+ * for invalid sizes.
  */
 size_t qlora_nf4_quantize_workspace(int64_t rows, int64_t cols, int32_t blocksize,
                                     int32_t double_quant);

@@ -46,6 +46,11 @@ def _declare(L: ctypes.CDLL) -> ctypes.CDLL:
     L.oracle_nf4_nearest_bits.argtypes = [u32, i64, p]
     L.oracle_nf4_quantize.argtypes = [p, i32, i64, i32, p, p, p, p, p]
     L.oracle_nf4_dequantize.argtypes = [i64, i32, p, p, p, p, ctypes.c_float, p]
+    L.oracle_quantize_ex.argtypes = [p, i32, i64, i32, i32, i32, i32, p, p, p, p, p]
+    L.oracle_dequantize_ex.argtypes = [i64, i32, i32, i32, i32, p, p, p, p, ctypes.c_float, p]
+    L.oracle_fp4_table.argtypes = [p]
+    L.oracle_e4m3_table.argtypes = [p]
+    L.oracle_e4m3_table.restype = i32
     L.oracle_linear_fwd.argtypes = [i64, i64, i64, i32, f64, p, p, p, p, p, i64, p]
     L.oracle_linear_bwd.argtypes = [i64, i64, i64, i32, f64, p, p, p, p, p, p, i64, p, p, p]
     L.oracle_num_threads.restype = i32
@@ -118,13 +123,32 @@ def nf4_nearest_bits(start: int, n: int) -> np.ndarray:
     return out
 
 
-def nf4_quantize(w: np.ndarray, double_quant: bool = True) -> dict:
-    """Blockwise NF4 quantization (+ double quantization) of a flat tensor.
+def fp4_table() -> np.ndarray:
+    out = np.zeros(16, np.float32)
+    lib().oracle_fp4_table(_ptr(out))
+    return out
+
+
+def e4m3_table() -> np.ndarray:
+    out = np.zeros(256, np.float32)
+    k = lib().oracle_e4m3_table(_ptr(out))
+    return out[:k].copy()
+
+
+CODE_TYPES = {"nf4": 0, "fp4": 1}
+DQ_TYPES = {"int8": 0, "e4m3": 1}
+
+
+def nf4_quantize(w: np.ndarray, double_quant: bool = True, blocksize: int = 64, code_type: str = "nf4",
+                 dq_type: str = "int8") -> dict:
+    """Blockwise 4-bit quantization (+ double quantization) of a flat tensor.
 
     ``w`` is either ``uint16`` (bf16 bit patterns) or ``float32``.
-    Returns ``codes`` (uint8, ceil(n/2)), ``absmax`` (float32, ceil(n/64)) and,
+    Returns ``codes`` (uint8, ceil(n/2)), ``absmax`` (float32, ceil(n/bs)) and,
     with double quantization, ``q8`` (uint8, nb), ``c1`` (float32, ceil(nb/256))
-    and ``offset`` (float).
+    and ``offset`` (float).  The defaults are the NF4 / linear 8-bit / block
+    64 format; ``code_type`` "fp4", ``dq_type`` "e4m3" and block sizes 128 and
+    256 are the variants.
     """
     w = np.ascontiguousarray(w).reshape(-1)
     if w.dtype == np.uint16:
@@ -134,34 +158,36 @@ def nf4_quantize(w: np.ndarray, double_quant: bool = True) -> dict:
     else:
         raise TypeError("w must be uint16 (bf16 bits) or float32")
     n = w.size
-    nb = (n + 63) // 64
+    nb = (n + blocksize - 1) // blocksize
     nb2 = (nb + 255) // 256
     codes = np.zeros((n + 1) // 2, np.uint8)
     absmax = np.zeros(nb, np.float32)
     q8 = np.zeros(nb, np.uint8)
     c1 = np.zeros(nb2, np.float32)
     off = np.zeros(1, np.float32)
-    lib().oracle_nf4_quantize(_ptr(w), is_bf16, n, int(bool(double_quant)), _ptr(codes),
-                              _ptr(absmax), _ptr(q8), _ptr(c1), _ptr(off))
+    lib().oracle_quantize_ex(_ptr(w), is_bf16, n, int(bool(double_quant)), int(blocksize), CODE_TYPES[code_type],
+                             DQ_TYPES[dq_type], _ptr(codes), _ptr(absmax), _ptr(q8), _ptr(c1), _ptr(off))
     out = {"codes": codes, "absmax": absmax}
     if double_quant:
         out.update(q8=q8, c1=c1, offset=float(off[0]))
     return out
 
 
-def nf4_dequantize(n: int, q: dict, double_quant: bool = True) -> np.ndarray:
+def nf4_dequantize(n: int, q: dict, double_quant: bool = True, blocksize: int = 64, code_type: str = "nf4",
+                   dq_type: str = "int8") -> np.ndarray:
     """doubleDequant: bf16 bit patterns (uint16, n) of the dequantized tensor."""
     out = np.zeros(n, np.uint16)
     codes = np.ascontiguousarray(q["codes"], np.uint8)
+    ct, dt = CODE_TYPES[code_type], DQ_TYPES[dq_type]
     if double_quant:
         q8 = np.ascontiguousarray(q["q8"], np.uint8)
         c1 = np.ascontiguousarray(q["c1"], np.float32)
-        lib().oracle_nf4_dequantize(n, 1, _ptr(codes), None, _ptr(q8), _ptr(c1),
-                                    ctypes.c_float(q["offset"]), _ptr(out))
+        lib().oracle_dequantize_ex(n, 1, int(blocksize), ct, dt, _ptr(codes), None, _ptr(q8), _ptr(c1),
+                                   ctypes.c_float(q["offset"]), _ptr(out))
     else:
         absmax = np.ascontiguousarray(q["absmax"], np.float32)
-        lib().oracle_nf4_dequantize(n, 0, _ptr(codes), _ptr(absmax), None, None,
-                                    ctypes.c_float(0.0), _ptr(out))
+        lib().oracle_dequantize_ex(n, 0, int(blocksize), ct, dt, _ptr(codes), _ptr(absmax), None, None,
+                                   ctypes.c_float(0.0), _ptr(out))
     return out
 
 

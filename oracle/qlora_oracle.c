@@ -137,6 +137,49 @@ void oracle_t8_table(float out[255])
     for (int k = 0; k < 255; ++k) out[k] = (float)(k - 127) / 127.0f;
 }
 
+/* FP4 code book (reading R11 of [P4] sec. 6 "Float4 (FP4)"): the values of a
+ * 4-bit float with 1 sign, 2 exponent and 1 mantissa bit (exponent bias 1,
+ * exponent field 0 = subnormal: 0 and 0.5), i.e. magnitudes
+ * {0, 0.5, 1, 1.5, 2, 3, 4, 6}, divided by the largest (6) so that they span
+ * [-1, 1], each rounded to fp32, all 16 codes sorted ascending: -0 and +0
+ * both appear (indices 7 and 8). */
+void oracle_fp4_table(float out[16])
+{
+    double mag[8];
+    for (int code = 0; code < 8; ++code) {
+        int e = code >> 1, m = code & 1;
+        mag[code] = (e == 0) ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    }
+    for (int i = 0; i < 8; ++i) {
+        out[7 - i] = -(float)(mag[i] / mag[7]);  /* index 7 = -0 */
+        out[8 + i] = (float)(mag[i] / mag[7]);
+    }
+}
+
+/* FP8 code book of the double quantization (reading R12 of [P4] sec. 4
+ * "c2^FP8"): the 253 distinct finite values of the 8-bit float E4M3 (1 sign,
+ * 4 exponent, 3 mantissa bits, bias 7, exponent field 0 = subnormal; the
+ * all-ones exponent with all-ones mantissa is not a number, so the largest
+ * value is 1.75 * 2^8 = 448), divided by 448, rounded to fp32, sorted
+ * ascending; -0 and +0 count once.  Returns the count (253). */
+int oracle_e4m3_table(float out[256])
+{
+    double pos[127];
+    int np = 0;
+    for (int e = 0; e < 16; ++e)
+        for (int m = 0; m < 8; ++m) {
+            if (e == 15 && m == 7) continue;        /* not a number */
+            if (e == 0 && m == 0) continue;         /* zero, added once below */
+            pos[np++] = (e == 0) ? ldexp(m / 8.0, -6) : ldexp(1.0 + m / 8.0, e - 7);
+        }
+    /* pos is ascending by construction */
+    int k = 0;
+    for (int i = np - 1; i >= 0; --i) out[k++] = (float)(-pos[i] / 448.0);
+    out[k++] = 0.0f;
+    for (int i = 0; i < np; ++i) out[k++] = (float)(pos[i] / 448.0);
+    return k;
+}
+
 /* Brute-force nearest entry of a sorted table, distances in fp64,
  * exact ties to the lower index (readings R4 and R6). */
 static int nearest_index(float x, const float *tab, int n)
@@ -204,19 +247,52 @@ static double pairwise_sum_padded(const float *v, int64_t n)
  * parameters share one constant, and the constants are quantized again to
  * 8 bits with one fp32 constant per 256 of them.
  */
+/* The 16-value code book of a 4-bit code type (0: NF4, 1: FP4) and the 8-bit
+ * code book of a double-quantization type (0: linear t8, 255 values; 1: FP8
+ * E4M3, 253 values); the latter returns its size. */
+static void code_table(int code_type, float out[16])
+{
+    if (code_type == 1) oracle_fp4_table(out); else oracle_nf4_table(out);
+}
+
+static int dq_table(int dq_type, float out[256])
+{
+    if (dq_type == 1) return oracle_e4m3_table(out);
+    oracle_t8_table(out);
+    return 255;
+}
+
+/*
+ * Blockwise 4-bit quantization with optional double quantization, for any
+ * block size (64, 128 or 256 consecutive elements share one constant), code
+ * type and double-quantization code book; oracle_nf4_quantize is the case
+ * (64, NF4, linear 8-bit).  Same steps and readings as below.
+ */
+void oracle_quantize_ex(const void *w, int is_bf16, int64_t n, int double_quant, int blocksize,
+                        int code_type, int dq_type, uint8_t *codes, float *absmax, uint8_t *q8,
+                        float *c1, float *offset);
+
 void oracle_nf4_quantize(const void *w, int is_bf16, int64_t n, int double_quant,
                          uint8_t *codes, float *absmax, uint8_t *q8, float *c1,
                          float *offset)
 {
+    oracle_quantize_ex(w, is_bf16, n, double_quant, 64, 0, 0, codes, absmax, q8, c1, offset);
+}
+
+void oracle_quantize_ex(const void *w, int is_bf16, int64_t n, int double_quant, int blocksize,
+                        int code_type, int dq_type, uint8_t *codes, float *absmax, uint8_t *q8,
+                        float *c1, float *offset)
+{
     float nf4[16];
-    oracle_nf4_table(nf4);
-    const int64_t nb = (n + 63) / 64;
+    code_table(code_type, nf4);
+    const int64_t bs = blocksize;
+    const int64_t nb = (n + bs - 1) / bs;
     memset(codes, 0, (size_t)((n + 1) / 2));
 
     #pragma omp parallel for schedule(static)
     for (int64_t b = 0; b < nb; ++b) {
-        int64_t lo = b * 64, hi = lo + 64 < n ? lo + 64 : n;
-        float vals[64];
+        int64_t lo = b * bs, hi = lo + bs < n ? lo + bs : n;
+        float vals[256];
         float a = 0.0f;
         for (int64_t i = lo; i < hi; ++i) {
             float v = is_bf16 ? bf16_to_f32(((const uint16_t *)w)[i]) : ((const float *)w)[i];
@@ -239,8 +315,8 @@ void oracle_nf4_quantize(const void *w, int is_bf16, int64_t n, int double_quant
     }
     if (!double_quant) return;
 
-    float t8[255];
-    oracle_t8_table(t8);
+    float t8[256];
+    const int nt8 = dq_table(dq_type, t8);
     double sum = pairwise_sum_padded(absmax, nb);
     float off = (nb > 0) ? (float)(sum / (double)nb) : 0.0f;
     *offset = off;
@@ -259,7 +335,7 @@ void oracle_nf4_quantize(const void *w, int is_bf16, int64_t n, int double_quant
         for (int64_t b = lo; b < hi; ++b) {
             float d = absmax[b] - off;
             float y = (d * p) * rc;
-            q8[b] = (uint8_t)nearest_index(y, t8, 255);
+            q8[b] = (uint8_t)nearest_index(y, t8, nt8);
         }
     }
 }
@@ -274,26 +350,35 @@ static float block_scale(int64_t b, int double_quant, const float *absmax,
     return t + offset;
 }
 
-/* doubleDequant of [P4] sec. 4: dequant(dequant(c1, c2), W) = W^BF16.
+/* doubleDequant of [P4] sec. 4: dequant(dequant(c1, c2), W) = W^BF16, for
+ * any block size, code type and double-quantization code book.
  * Writes n bf16 values (bits). */
-void oracle_nf4_dequantize(int64_t n, int double_quant, const uint8_t *codes,
-                           const float *absmax, const uint8_t *q8, const float *c1,
-                           float offset, uint16_t *out)
+void oracle_dequantize_ex(int64_t n, int double_quant, int blocksize, int code_type, int dq_type,
+                          const uint8_t *codes, const float *absmax, const uint8_t *q8,
+                          const float *c1, float offset, uint16_t *out)
 {
-    float nf4[16], t8[255];
-    oracle_nf4_table(nf4);
-    oracle_t8_table(t8);
-    const int64_t nb = (n + 63) / 64;
+    float nf4[16], t8[256];
+    code_table(code_type, nf4);
+    dq_table(dq_type, t8);
+    const int64_t bs = blocksize;
+    const int64_t nb = (n + bs - 1) / bs;
     #pragma omp parallel for schedule(static)
     for (int64_t b = 0; b < nb; ++b) {
         float a = block_scale(b, double_quant, absmax, q8, c1, offset, t8);
-        int64_t lo = b * 64, hi = lo + 64 < n ? lo + 64 : n;
+        int64_t lo = b * bs, hi = lo + bs < n ? lo + bs : n;
         for (int64_t i = lo; i < hi; ++i) {
             uint8_t byte = codes[i >> 1];
             int c = (i & 1) ? (byte & 15) : (byte >> 4);
             out[i] = f32_to_bf16_rne(nf4[c] * a);
         }
     }
+}
+
+void oracle_nf4_dequantize(int64_t n, int double_quant, const uint8_t *codes,
+                           const float *absmax, const uint8_t *q8, const float *c1,
+                           float offset, uint16_t *out)
+{
+    oracle_dequantize_ex(n, double_quant, 64, 0, 0, codes, absmax, q8, c1, offset, out);
 }
 
 /* ------------------------------------------------------------------ */

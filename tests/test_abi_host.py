@@ -35,9 +35,9 @@ def test_nf4_table_matches_oracle(Q, O):
                                   O.nf4_table().view(np.uint32))
 
 
-def _w(rows=256, cols=256, dq=1, blocksize=64, codes=FAKE):
+def _w(rows=256, cols=256, dq=1, blocksize=64, codes=FAKE, code_type=0, dq_type=0):
     from bit_nf4_quantized_08_b200._lib import CNF4Weight
-    return CNF4Weight(rows, cols, blocksize, dq, codes, FAKE, FAKE, FAKE, FAKE)
+    return CNF4Weight(rows, cols, blocksize, dq, codes, FAKE, FAKE, FAKE, FAKE, code_type, dq_type)
 
 
 def test_quantize_workspace_sizes(Q):
@@ -48,6 +48,8 @@ def test_quantize_workspace_sizes(Q):
     nb, ng = n // 64, n // 16384
     assert L.qlora_nf4_quantize_workspace(4096, 4096, 64, 1) == nb * 4 + ng * 8
     assert L.qlora_nf4_quantize_workspace(4096, 4096, 32, 1) == 0
+    assert L.qlora_nf4_quantize_workspace(4096, 4096, 128, 1) == (n // 128) * 4 + ng * 8
+    assert L.qlora_nf4_quantize_workspace(4096, 4096, 256, 1) == (n // 256) * 4 + ng * 8
     assert L.qlora_nf4_quantize_workspace(-1, 4, 64, 1) == 0
 
     def a256(x):
@@ -68,7 +70,10 @@ def test_quantize_rejects(Q):
     ws = FAKE
     big = 1 << 30
     assert L.qlora_nf4_quantize(FAKE, QLORA_BF16, None, ws, big, None) == QLORA_ERR_INVALID_ARG
-    assert L.qlora_nf4_quantize(FAKE, QLORA_BF16, ctypes.byref(_w(blocksize=128)), ws, big, None) == QLORA_ERR_UNSUPPORTED
+    assert L.qlora_nf4_quantize(FAKE, QLORA_BF16, ctypes.byref(_w(blocksize=32)), ws, big, None) == QLORA_ERR_UNSUPPORTED
+    assert L.qlora_nf4_quantize(FAKE, QLORA_BF16, ctypes.byref(_w(blocksize=512)), ws, big, None) == QLORA_ERR_UNSUPPORTED
+    assert L.qlora_nf4_quantize(FAKE, QLORA_BF16, ctypes.byref(_w(code_type=2)), ws, big, None) == QLORA_ERR_INVALID_ARG
+    assert L.qlora_nf4_quantize(FAKE, QLORA_BF16, ctypes.byref(_w(dq_type=-1)), ws, big, None) == QLORA_ERR_INVALID_ARG
     assert L.qlora_nf4_quantize(None, QLORA_BF16, ctypes.byref(_w()), ws, big, None) == QLORA_ERR_INVALID_ARG
     assert L.qlora_nf4_quantize(FAKE + 8, QLORA_BF16, ctypes.byref(_w()), ws, big, None) == QLORA_ERR_INVALID_ARG
     assert L.qlora_nf4_quantize(FAKE, 7, ctypes.byref(_w()), ws, big, None) == QLORA_ERR_INVALID_ARG

@@ -556,3 +556,101 @@ def test_adamw_vs_torch_optim(O):
         st = opt.state[pt]
         np.testing.assert_allclose(m, st["exp_avg"].numpy(), rtol=1e-13, atol=1e-20)
         np.testing.assert_allclose(v, st["exp_avg_sq"].numpy(), rtol=1e-13, atol=1e-24)
+
+
+# ---------------------------------------------------------------------------
+# data-type variants: FP4 codes, FP8 (E4M3) double quantization, block sizes
+# ---------------------------------------------------------------------------
+
+def test_fp4_table_closed_form(O):
+    """FP4 = 1 sign, 2 exponent (bias 1), 1 mantissa bit: magnitudes 0, 0.5,
+    1, 1.5, 2, 3, 4, 6 divided by 6, both signs, sorted; -0 and +0 at 7, 8."""
+    mags = []
+    for e in range(4):
+        for m in range(2):
+            mags.append(Fraction(m, 2) if e == 0 else (1 + Fraction(m, 2)) * Fraction(2) ** (e - 1))
+    mags = sorted(mags)
+    assert mags == [Fraction(x) for x in (0, 0.5, 1, 1.5, 2, 3, 4, 6)]
+    want = [-float(x / 6) for x in reversed(mags)] + [float(x / 6) for x in mags]
+    t = O.fp4_table()
+    np.testing.assert_array_equal(_f32bits(t), _f32bits(np.array(want, np.float32)))
+    assert np.signbit(t[7]) and not np.signbit(t[8]) and t[7] == 0 and t[8] == 0
+
+
+def test_e4m3_table_vs_torch(O):
+    """The E4M3 code book: every finite value of torch.float8_e4m3fn (a
+    library routine), zeros merged, sorted, divided by 448, in fp32."""
+    v = torch.arange(256, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn).to(torch.float64)
+    v = v[~torch.isnan(v)].unique().numpy()  # unique also merges -0 and +0
+    want = (np.sort(v) / 448.0).astype(np.float32)
+    want[want == 0] = 0.0  # the one merged zero is +0
+    t = O.e4m3_table()
+    assert t.size == 253 and want.size == 253
+    np.testing.assert_array_equal(_f32bits(t), _f32bits(want))
+
+
+@pytest.mark.parametrize("bs", [64, 128, 256])
+@pytest.mark.parametrize("code_type", ["nf4", "fp4"])
+def test_variant_roundtrip_lossless(O, bs, code_type):
+    """Blocks of bs elements that are exactly code-book values times their
+    absmax round-trip: the constant of block b is the max over elements
+    [b bs, (b+1) bs), every code comes back, and the dequantized bf16 value
+    is the bf16 of the input."""
+    rng = np.random.default_rng(bs)
+    t = O.fp4_table() if code_type == "fp4" else O.nf4_table()
+    usable = [j for j in range(16) if not (code_type == "fp4" and j == 8)]  # +0 is never chosen (ties low)
+    nb = 40
+    idx = rng.choice(usable, (nb, bs))
+    idx[:, 3] = 15
+    a = rng.uniform(1e-3, 3.0, nb).astype(np.float32)
+    w = (t[idx] * a[:, None]).astype(np.float32)
+    q = O.nf4_quantize(w.reshape(-1), double_quant=False, blocksize=bs, code_type=code_type)
+    np.testing.assert_array_equal(q["absmax"], a)
+    np.testing.assert_array_equal(q["absmax"], np.abs(w).max(axis=1))
+    codes = np.empty(nb * bs, np.uint8)
+    codes[0::2] = q["codes"] >> 4
+    codes[1::2] = q["codes"] & 15
+    np.testing.assert_array_equal(codes, idx.reshape(-1))
+    deq = O.nf4_dequantize(w.size, q, double_quant=False, blocksize=bs, code_type=code_type)
+    ref = torch.from_numpy(w.reshape(-1)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(deq, ref)
+
+
+def test_fp4_zero_ties_to_negative_zero(O):
+    """With two zeros in the FP4 code book, an exact tie goes to the lower
+    index: 0 and values nearer to 0 than to 1/12 get code 7 (-0)."""
+    w = np.array([1.0, 0.0, 1e-30, -1e-30, 0.04, 0.0417, -0.04] + [0.5] * 57, np.float32)
+    q = O.nf4_quantize(w, double_quant=False, code_type="fp4")
+    codes = np.empty(64, np.uint8)
+    codes[0::2] = q["codes"] >> 4
+    codes[1::2] = q["codes"] & 15
+    assert list(codes[:7]) == [15, 7, 7, 7, 7, 9, 7]
+
+
+@pytest.mark.parametrize("bs", [64, 256])
+def test_e4m3_double_quant(O, bs):
+    """FP8 (E4M3) double quantization: the 8-bit codes index the 253-value
+    code book; each code is the nearest entry (exact rationals, ties low);
+    equal block maxima stay lossless (c1 = 0, code of 0)."""
+    rng = np.random.default_rng(3)
+    w = rng.normal(0, 0.02, bs * 700).astype(np.float32)
+    q = O.nf4_quantize(w, double_quant=True, blocksize=bs, dq_type="e4m3")
+    t = O.e4m3_table()
+    assert q["q8"].max() < 253
+    absmax = np.abs(w.reshape(-1, bs)).max(axis=1)
+    off = np.float32(q["offset"])
+    for b in range(0, absmax.size, 37):
+        c = q["c1"][b // 256]
+        d = np.float32(absmax[b] - off)
+        y = np.float32(d * np.float32(np.float32(1.0) / c))
+        dist = [abs(Fraction(float(y)) - Fraction(float(x))) for x in t]
+        best = min(range(len(t)), key=lambda k: (dist[k], k))
+        assert q["q8"][b] == best
+    a = np.float32(0.0371)
+    w2 = (rng.uniform(-1, 1, (300, bs)) * a).astype(np.float32)
+    w2[:, 1] = a
+    q2 = O.nf4_quantize(w2.reshape(-1), double_quant=True, blocksize=bs, dq_type="e4m3")
+    assert float(q2["c1"].max()) == 0.0 and np.all(q2["q8"] == 126)
+    d2 = O.nf4_dequantize(w2.size, q2, double_quant=True, blocksize=bs, dq_type="e4m3")
+    q0 = O.nf4_quantize(w2.reshape(-1), double_quant=False, blocksize=bs)
+    np.testing.assert_array_equal(d2, O.nf4_dequantize(w2.size, q0, double_quant=False, blocksize=bs))
