@@ -12,6 +12,7 @@ from .api import (  # noqa: F401
     PagedBuffer,
     qlora_adamw_step,
     qlora_debug_inject,
+    qlora_dq_encode,
     qlora_fused_linear_bwd,
     qlora_fused_linear_fwd,
     qlora_fused_linear_workspace,

@@ -48,6 +48,7 @@ EXPORTS = (
     "qlora_get_last_error",
     "qlora_nf4_table",
     "qlora_nf4_encode",
+    "qlora_dq_encode",
     "qlora_set_wait_timeout_ns",
     "qlora_debug_inject",
     "qlora_kernel_launches",
@@ -149,6 +150,8 @@ def lib() -> ctypes.CDLL:
     L.qlora_nf4_table.restype = None
     L.qlora_nf4_encode.argtypes = [vp, i64, vp, vp]
     L.qlora_nf4_encode.restype = i32
+    L.qlora_dq_encode.argtypes = [vp, i64, vp, i32, vp]
+    L.qlora_dq_encode.restype = i32
     L.qlora_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
     L.qlora_set_wait_timeout_ns.restype = None
     L.qlora_debug_inject.argtypes = [i32]

@@ -328,6 +328,14 @@ def qlora_nf4_encode(x: torch.Tensor, codes: torch.Tensor | None = None) -> torc
     return codes
 
 
+def qlora_dq_encode(y: torch.Tensor, dq_type: str = "int8", codes: torch.Tensor | None = None) -> torch.Tensor:
+    """Nearest 8-bit code (double quantization) of every fp32 element of y."""
+    if codes is None:
+        codes = torch.empty(y.numel(), dtype=torch.uint8, device=y.device)
+    check(lib().qlora_dq_encode(_ptr(y), y.numel(), _ptr(codes), DQ_TYPES[dq_type], _stream()), "qlora_dq_encode")
+    return codes
+
+
 def qlora_set_wait_timeout_ns(ns: int) -> None:
     lib().qlora_set_wait_timeout_ns(int(ns))
 

@@ -10,6 +10,8 @@
 
 #include <math.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/qlora_nf4.h"
 #include "adamw.cuh"
 #include "common.cuh"
@@ -112,6 +114,16 @@ bool side_stream_acquire(cudaStream_t s, SideStream* out) {
 void side_stream_release() { g_side_mu.unlock(); }
 
 static bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// An NVTX range named after the entry point around the host side of every
+// call that launches work (header-only NVTX: a no-op unless a profiler or
+// tracer is attached), so that timelines group each call's kernels.
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 static const int64_t kMaxElems = (int64_t)1 << 40;
 
@@ -265,6 +277,7 @@ size_t qlora_nf4_quantize_workspace(int64_t rows, int64_t cols, int32_t blocksiz
 
 qlora_status qlora_nf4_quantize(const void* W, qlora_dtype wdtype, const qlora_nf4_weight* out,
                                 void* ws, size_t ws_bytes, qlora_stream_t stream) {
+    NvtxRange nvtx_range("qlora_nf4_quantize");
     qlora_status st = check_weight(out, true);
     if (st != QLORA_OK) return st;
     if (wdtype != QLORA_F32 && wdtype != QLORA_BF16) return QLORA_ERR_INVALID_ARG;
@@ -297,6 +310,7 @@ qlora_status qlora_nf4_quantize(const void* W, qlora_dtype wdtype, const qlora_n
 
 qlora_status qlora_nf4_quantize_static(const void* W, qlora_dtype wdtype, const qlora_nf4_weight* out,
                                        qlora_stream_t stream) {
+    NvtxRange nvtx_range("qlora_nf4_quantize_static");
     qlora_status st = check_weight(out, true);
     if (st != QLORA_OK) return st;
     if (wdtype != QLORA_F32 && wdtype != QLORA_BF16) return QLORA_ERR_INVALID_ARG;
@@ -328,6 +342,7 @@ qlora_status qlora_nf4_quantize_static(const void* W, qlora_dtype wdtype, const 
 }
 
 qlora_status qlora_nf4_dequantize(const qlora_nf4_weight* w, void* out, qlora_stream_t stream) {
+    NvtxRange nvtx_range("qlora_nf4_dequantize");
     qlora_status st = check_weight(w, true);
     if (st != QLORA_OK) return st;
     if (w->rows * w->cols == 0) return QLORA_OK;
@@ -351,6 +366,7 @@ size_t qlora_linear_workspace(int64_t M, const qlora_nf4_weight* w, int32_t r, i
 qlora_status qlora_fused_linear_fwd(const void* X, int64_t M, const qlora_nf4_weight* w, int32_t nseg,
                                     const void* A, const void* B, int32_t r, float scale, void* Y,
                                     void* ws, size_t ws_bytes, qlora_stream_t stream) {
+    NvtxRange nvtx_range("qlora_fused_linear_fwd");
     qlora_status st = check_fused(M, w, nseg, r);
     if (st != QLORA_OK) return st;
     if (M == 0) return QLORA_OK;
@@ -372,6 +388,7 @@ qlora_status qlora_fused_linear_bwd(const void* dY, const void* X, int64_t M, co
                                     int32_t nseg, const void* A, const void* B, int32_t r, float scale,
                                     void* dX, float* dA, float* dB, void* ws, size_t ws_bytes,
                                     qlora_stream_t stream) {
+    NvtxRange nvtx_range("qlora_fused_linear_bwd");
     qlora_status st = check_fused(M, w, nseg, r);
     if (st != QLORA_OK) return st;
     if (r > 0 && (!A || !aligned(A, 16) || !B || !aligned(B, 16) || !dA || !aligned(dA, 16) ||
@@ -397,6 +414,7 @@ qlora_status qlora_linear_bwd(const void* dY, const void* X, int64_t M, const ql
 
 qlora_status qlora_lora_merge(const qlora_nf4_weight* w, const void* A, const void* B, int32_t r,
                               float scale, void* W_merged, qlora_stream_t stream) {
+    NvtxRange nvtx_range("qlora_lora_merge");
     qlora_status st = check_weight(w, true);
     if (st != QLORA_OK) return st;
     st = check_merge(w->rows, w->cols, A, B, r, W_merged);
@@ -408,6 +426,7 @@ qlora_status qlora_lora_merge(const qlora_nf4_weight* w, const void* A, const vo
 qlora_status qlora_lora_unmerge(const void* W_merged, int64_t rows, int64_t cols, const void* A,
                                 const void* B, int32_t r, float scale, void* W_out,
                                 qlora_stream_t stream) {
+    NvtxRange nvtx_range("qlora_lora_unmerge");
     qlora_status st = check_merge(rows, cols, A, B, r, W_out);
     if (st != QLORA_OK || rows * cols == 0) return st;
     if (!W_merged || !aligned(W_merged, 16)) return QLORA_ERR_INVALID_ARG;
@@ -418,6 +437,7 @@ qlora_status qlora_lora_unmerge(const void* W_merged, int64_t rows, int64_t cols
 qlora_status qlora_adamw_step(float* param, float* exp_avg, float* exp_avg_sq, const float* grad,
                               void* param_bf16, int64_t n, const qlora_adamw_config* cfg,
                               qlora_stream_t stream) {
+    NvtxRange nvtx_range("qlora_adamw_step");
     if (!cfg || n < 0) return QLORA_ERR_INVALID_ARG;
     if (cfg->step < 1 || !(cfg->lr >= 0.0f) || !(cfg->beta1 >= 0.0f && cfg->beta1 < 1.0f) ||
         !(cfg->beta2 >= 0.0f && cfg->beta2 < 1.0f) || !(cfg->eps > 0.0f) || !(cfg->weight_decay >= 0.0f))
@@ -470,6 +490,7 @@ qlora_status qlora_paged_free(void* ptr) {
 }
 
 qlora_status qlora_paged_prefetch(const void* ptr, size_t bytes, int32_t to_host, qlora_stream_t stream) {
+    NvtxRange nvtx_range("qlora_paged_prefetch");
     if (!ptr && bytes) return QLORA_ERR_INVALID_ARG;
     if (bytes == 0) return QLORA_OK;
     int dev = 0;
@@ -497,10 +518,21 @@ qlora_status qlora_get_last_error(qlora_stream_t stream) {
 void qlora_nf4_table(float out[16]) { nf4_table_host(out); }
 
 qlora_status qlora_nf4_encode(const float* x, int64_t n, uint8_t* codes, qlora_stream_t stream) {
+    NvtxRange nvtx_range("qlora_nf4_encode");
     if (n < 0) return QLORA_ERR_INVALID_ARG;
     if (n == 0) return QLORA_OK;
     if (!x || !codes || !aligned(x, 4)) return QLORA_ERR_INVALID_ARG;
     if (launch_encode(x, n, codes, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return QLORA_ERR_CUDA;
+    return QLORA_OK;
+}
+
+qlora_status qlora_dq_encode(const float* y, int64_t n, uint8_t* codes, int32_t dq_type, qlora_stream_t stream) {
+    NvtxRange nvtx_range("qlora_dq_encode");
+    if (n < 0 || (dq_type != QLORA_DQ_INT8 && dq_type != QLORA_DQ_FP8)) return QLORA_ERR_INVALID_ARG;
+    if (n == 0) return QLORA_OK;
+    if (!y || !codes || !aligned(y, 4)) return QLORA_ERR_INVALID_ARG;
+    if (launch_dq_encode(y, n, codes, dq_type, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
         return QLORA_ERR_CUDA;
     return QLORA_OK;
 }

@@ -46,36 +46,44 @@ namespace qlora {
 // P_key, the largest fp32 below T_key: x >= T_key exactly when x > P_key,
 // i.e. when fl(P_key - x) is negative (a difference of two finite floats is
 // zero only when they are equal), so the compare is one FADD and the sign
-// bit.  The tables have 64 entries and the key is masked to 6 bits, so any
-// input (NaN included) reads inside them.
-struct SearchSmem {
-    float thr[64];  // P_key
-    int base[64];
+// bit.
+// The key is formed as t = fl(128 x + 1.5 * 2^26 + 128): at that magnitude
+// the fp32 spacing is 8, so t rounds 128 x + 128 to a multiple of 8, i.e.
+// t = C + 8 RN(16 x + 16) (the same round-to-nearest-even as rounding 16 x
+// + 16 to an integer), and its low mantissa bits hold 8 key: (P_key,
+// base_key) sit as one 8-byte entry at byte 8 key of a 512-byte aligned
+// table, whose address is one AND-OR of t's bits.  64 entries and a 6-bit
+// key mask: any input (NaN included) reads inside the table.
+struct __align__(512) SearchSmem {
+    uint2 e[64];   // {P_key bits, base_key}
     int inc[64];
 };
 
 __device__ __forceinline__ void load_search_tables(SearchSmem& st, const Nf4SearchTable& tab) {
     for (int i = threadIdx.x; i < 64; i += blockDim.x) {
-        st.thr[i] = i < 33 ? tab.thr[i] : 3.0f;
-        st.base[i] = i < 33 ? tab.base[i] : 15;
+        st.e[i] = make_uint2(__float_as_uint(i < 33 ? tab.thr[i] : 3.0f), (uint32_t)(i < 33 ? tab.base[i] : 15));
         st.inc[i] = i < 33 ? tab.inc[i] : 0;
     }
 }
 
-// t = fl(16 x + 1.5 * 2^23 + 16): x rounded to an integer bucket key in the
-// low mantissa bits (0x4B400000 + key).
+constexpr float kKeyMagic = 100663424.0f;  // 1.5 * 2^26 + 128
+
 // CT = 1 (FP4): a bucket's threshold may count twice (inc = 2).
 template <int CT = 0>
 __device__ __forceinline__ uint32_t nf4_lookup(float x, float t, const SearchSmem& st) {
-    const uint32_t key = __float_as_uint(t) & 63u;
-    const uint32_t above = __float_as_uint(__fsub_rn(st.thr[key], x)) >> 31;
-    if (CT == 0) return (uint32_t)st.base[key] + above;
-    return (uint32_t)st.base[key] + above * (uint32_t)st.inc[key];
+    const uint32_t tb = __float_as_uint(t);
+    uint32_t thr, base;
+    asm("ld.shared.v2.b32 {%0, %1}, [%2];"
+        : "=r"(thr), "=r"(base)
+        : "r"(smem_u32(st.e) | (tb & 0x1F8u)));
+    const uint32_t above = __float_as_uint(__fsub_rn(__uint_as_float(thr), x)) >> 31;
+    if (CT == 0) return base + above;
+    return base + above * (uint32_t)st.inc[(tb >> 3) & 63u];
 }
 
 template <int CT = 0>
 __device__ __forceinline__ uint32_t nf4_search(float x, const SearchSmem& st) {
-    return nf4_lookup<CT>(x, fmaf(x, 16.0f, 12582928.0f), st);
+    return nf4_lookup<CT>(x, fmaf(x, 128.0f, kKeyMagic), st);
 }
 
 // Two lanes of fp32x2 arithmetic (sm_100a packed FP32): the same IEEE
@@ -104,7 +112,7 @@ template <int CT = 0>
 __device__ __forceinline__ void nf4_search2(float w0, float w1, uint64_t rcp2, const SearchSmem& st, uint32_t& c0,
                                             uint32_t& c1) {
     const uint64_t x2 = f2_mul(f2_pack(w0, w1), rcp2);
-    const uint64_t t2 = f2_fma(x2, f2_pack(16.0f, 16.0f), f2_pack(12582928.0f, 12582928.0f));
+    const uint64_t t2 = f2_fma(x2, f2_pack(128.0f, 128.0f), f2_pack(kKeyMagic, kKeyMagic));
     float x0, x1, t0, t1;
     f2_unpack(x2, x0, x1);
     f2_unpack(t2, t0, t1);
@@ -348,26 +356,28 @@ __global__ void __launch_bounds__(256) k_dq_partials(const double* sums, int64_t
         partials[blockIdx.x] = ((s_w[0] + s_w[1]) + (s_w[2] + s_w[3])) + ((s_w[4] + s_w[5]) + (s_w[6] + s_w[7]));
 }
 
-// Nearest 8-bit code of y in [-1, 1]: candidate from rint(127 y), then the
-// exact fp64 distances of it and its two neighbours; ties to the lower index.
-// t8 = the 256 fp32 code values t8[k] = fl32((k - 127) / 127) (shared memory).
-__device__ __forceinline__ int nearest_t8(float y, const float* t8) {
+// Decision threshold k of the linear 8-bit code book, between t8[k] and
+// t8[k+1] (k = 0..253): the smallest fp32 strictly above their exact
+// midpoint (fp64 holds the midpoint of two fp32 values exactly), so that
+// y >= T_k exactly when the nearest code of y, ties to the lower index, is
+// above k.
+__device__ __forceinline__ float t8_threshold(int k) {
+    const double m = 0.5 * ((double)t8_value(k) + (double)t8_value(k + 1));
+    float f = __double2float_rn(m);
+    if ((double)f <= m) f = nextafterf(f, 3.0f);
+    return f;
+}
+
+// Nearest 8-bit code of y in [-1, 1]: the candidate rint(127 y) + 127 is the
+// nearest code or its neighbour (y is within half a step of t8[candidate]),
+// so two fp32 compares with the thresholds on either side decide; ties go
+// to the lower index.  thr = the 254 thresholds (shared memory).
+__device__ __forceinline__ int nearest_t8(float y, const float* thr) {
     int k0 = __float2int_rn(__fmul_rn(y, 127.0f)) + 127;
     k0 = min(max(k0, 0), 254);
-    int best = k0;
-    double bd = fabs((double)y - (double)t8[k0]);
-    if (k0 > 0) {
-        double d = fabs((double)y - (double)t8[k0 - 1]);
-        if (d <= bd) {
-            bd = d;
-            best = k0 - 1;
-        }
-    }
-    if (k0 < 254) {
-        double d = fabs((double)y - (double)t8[k0 + 1]);
-        if (d < bd) best = k0 + 1;
-    }
-    return best;
+    const int down = (k0 > 0 && y < thr[k0 - 1]) ? 1 : 0;
+    const int up = (k0 < 254 && y >= thr[k0]) ? 1 : 0;
+    return k0 - down + up;
 }
 
 // Nearest FP8 (E4M3) code of y: the first table entry >= y by binary search
@@ -397,12 +407,13 @@ __global__ void __launch_bounds__(256) k_dq_quantize(const float* absmax, int64_
                                                      uint8_t* q8,
                                                      float* c1,
                                                      const double* sums, int64_t nsums, int dt) {
-    __shared__ float t8[256];
+    __shared__ float t8[256];  // E4M3: the 253 code values; linear: the 254 decision thresholds
     __shared__ double s_w[8];
     __shared__ float s_off;
     pdl_trigger();
     // blockDim.x == 256; shared memory only
-    t8[threadIdx.x] = dt ? (threadIdx.x < 253 ? e4m3_value(threadIdx.x) : 2.0f) : t8_value(threadIdx.x);
+    t8[threadIdx.x] = dt ? (threadIdx.x < 253 ? e4m3_value(threadIdx.x) : 2.0f)
+                         : (threadIdx.x < 254 ? t8_threshold(threadIdx.x) : 3.0f);
     pdl_wait();
     // this warp's first group: 8 block maxima per lane, loaded before the
     // offset tree so that the two memory round trips overlap
@@ -569,6 +580,19 @@ __global__ void k_encode(const float* __restrict__ x, int64_t n, uint8_t* __rest
     }
 }
 
+// Nearest 8-bit code of every y (test entry point: the search of the double
+// quantization on arbitrary inputs).
+__global__ void k_dq_encode(const float* __restrict__ y, int64_t n, uint8_t* __restrict__ codes, int dt) {
+    __shared__ float t8[256];
+    t8[threadIdx.x] = dt ? (threadIdx.x < 253 ? e4m3_value(threadIdx.x) : 2.0f)
+                         : (threadIdx.x < 254 ? t8_threshold(threadIdx.x) : 3.0f);
+    __syncthreads();
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const float v = fminf(fmaxf(y[i], -1.0f), 1.0f);
+        codes[i] = (uint8_t)(dt ? nearest_e4m3(v, t8) : nearest_t8(v, t8));
+    }
+}
+
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
@@ -720,6 +744,15 @@ inline cudaError_t launch_expand_scales(const qlora_nf4_weight& w, float* scales
                       (int)w.double_quant, (const float*)w.absmax, (const uint8_t*)w.absmax_q8,
                       (const float*)w.absmax_scale, (const float*)w.absmax_offset, scales, ld, flags, nflags,
                       weight_format(w));
+}
+
+inline cudaError_t launch_dq_encode(const float* y, int64_t n, uint8_t* codes, int dt, cudaStream_t s) {
+    if (n == 0) return cudaSuccess;
+    int64_t blocks = (n + 255) / 256;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    note_launch();
+    k_dq_encode<<<(unsigned)blocks, 256, 0, s>>>(y, n, codes, dt);
+    return cudaGetLastError();
 }
 
 inline cudaError_t launch_encode(const float* x, int64_t n, uint8_t* codes, cudaStream_t s) {

@@ -218,7 +218,11 @@ qlora_status qlora_linear_fwd(const void *X, int64_t M, const qlora_nf4_weight *
  * inside a stream capture, once the side stream exists: it is created by the
  * first such call made outside a capture).  The library keeps that stream and
  * two events per device for its lifetime.  Calls from several host threads
- * are serialized on the side stream.
+ * are serialized on the side stream.  There is one side stream per device,
+ * shared by every caller stream: the sU/dA/dB work of backward calls issued
+ * on independent streams runs one call after another on it, and each caller
+ * stream's join may then also wait for side work of another stream's call
+ * (an ordering that costs time, never correctness).
  */
 qlora_status qlora_linear_bwd(const void *dY, const void *X, int64_t M, const qlora_nf4_weight *w,
                               const void *A, const void *B, int32_t r, float scale, void *dX,
@@ -352,6 +356,16 @@ void qlora_nf4_table(float out[16]);
 qlora_status qlora_nf4_encode(const float *x, int64_t n, uint8_t *codes, qlora_stream_t stream);
 
 /*
+ * Nearest-code search of the double quantization, exposed so that it can be
+ * checked on every fp32 input: codes[i] = index of the entry of the 8-bit
+ * code book dq_type (QLORA_DQ_INT8: 0..254, QLORA_DQ_FP8: 0..252) nearest to
+ * y[i] clamped to [-1, 1], exact ties to the lower index.  Device arrays of n
+ * elements.  Test entry point.
+ */
+qlora_status qlora_dq_encode(const float *y, int64_t n, uint8_t *codes, int32_t dq_type,
+                             qlora_stream_t stream);
+
+/*
  * Upper bound, in nanoseconds, of every in-kernel wait (default 10 s).
  * Test entry point; 0 restores the default.
  */
@@ -372,6 +386,11 @@ void qlora_set_wait_timeout_ns(uint64_t ns);
  * it on the library's side stream.
  * Mode 0: normal (CTA-pair kernel, one pair per tile; in the backward the
  * dA/dB GEMMs beside the dX GEMM on the side stream).
+ * The mode is process-wide: it changes the kernels of every later call from
+ * every thread and stream on every device, until it is set back to 0; it is
+ * meant for tests only.  Likewise the environment variable QLORA_SCHEDULE
+ * (pair | pairsk | grid | streamk: the schedule of the large-M GEMMs) is read
+ * once, at the first large-M call of the process, and applies to all calls.
  */
 void qlora_debug_inject(int32_t mode);
 

@@ -49,6 +49,8 @@ def _declare(L: ctypes.CDLL) -> ctypes.CDLL:
     L.oracle_quantize_ex.argtypes = [p, i32, i64, i32, i32, i32, i32, p, p, p, p, p]
     L.oracle_dequantize_ex.argtypes = [i64, i32, i32, i32, i32, p, p, p, p, ctypes.c_float, p]
     L.oracle_fp4_table.argtypes = [p]
+    L.oracle_dq_nearest_bits.argtypes = [u32, i64, i32, p]
+    L.oracle_dq_nearest_bits.restype = None
     L.oracle_e4m3_table.argtypes = [p]
     L.oracle_e4m3_table.restype = i32
     L.oracle_linear_fwd.argtypes = [i64, i64, i64, i32, f64, p, p, p, p, p, i64, p]
@@ -137,6 +139,13 @@ def e4m3_table() -> np.ndarray:
 
 CODE_TYPES = {"nf4": 0, "fp4": 1}
 DQ_TYPES = {"int8": 0, "e4m3": 1}
+
+
+def dq_nearest_bits(start: int, n: int, dq_type: str = "int8") -> np.ndarray:
+    """Nearest 8-bit code (brute force) of the n fp32 bit patterns from ``start``."""
+    out = np.zeros(n, np.uint8)
+    lib().oracle_dq_nearest_bits(ctypes.c_uint32(start), n, DQ_TYPES[dq_type], _ptr(out))
+    return out
 
 
 def nf4_quantize(w: np.ndarray, double_quant: bool = True, blocksize: int = 64, code_type: str = "nf4",

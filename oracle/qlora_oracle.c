@@ -218,6 +218,20 @@ void oracle_nf4_nearest_bits(uint32_t start, int64_t n, uint8_t *codes)
         codes[i] = (uint8_t)nearest_index(f32_from_bits(start + (uint32_t)i), nf4, 16);
 }
 
+/* Nearest entry of the 8-bit code book dq_type (0 linear, 1 E4M3) of n
+ * consecutive fp32 bit patterns from `start` (brute force over the table,
+ * distances in fp64, ties to the lower index).  Pins the GPU's search. */
+void oracle_dq_nearest_bits(uint32_t start, int64_t n, int dq_type, uint8_t *codes)
+{
+    float tab[256];
+    int nt;
+    if (dq_type == 1) nt = oracle_e4m3_table(tab);
+    else { oracle_t8_table(tab); nt = 255; }
+    #pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i)
+        codes[i] = (uint8_t)nearest_index(f32_from_bits(start + (uint32_t)i), tab, nt);
+}
+
 /* ------------------------------------------------------------------ */
 /* quantize                                                             */
 /* ------------------------------------------------------------------ */

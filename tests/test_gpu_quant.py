@@ -187,3 +187,45 @@ def test_partial_offset_tree_matches_single_cta(Q, cuda, shape):
                  (q_part.absmax_scale.view(torch.int32), q_one.absmax_scale.view(torch.int32)),
                  (q_part.absmax_offset.view(torch.int32), q_one.absmax_offset.view(torch.int32))]:
         assert torch.equal(x, y)
+
+
+def test_dq_encode_exhaustive_int8(Q, O, cuda):
+    """The 8-bit search of the double quantization (fp32 thresholds around the
+    rint candidate) equals the oracle's brute-force argmin over the 255-entry
+    code book on every fp32 value in [-1, 1] (both signs, zeros, subnormals)."""
+    hi = int(np.float32(1.0).view(np.uint32))
+    chunk = 1 << 26
+    for sign in (0, 0x80000000):
+        start = 0
+        while start <= hi:
+            n = min(chunk, hi + 1 - start)
+            first = sign | start
+            y = torch.arange(first, first + n, dtype=torch.int64, device="cuda").to(torch.int32).view(torch.float32)
+            got = Q.qlora_dq_encode(y, "int8")
+            exp = torch.from_numpy(O.dq_nearest_bits(first, n, "int8")).to("cuda")
+            bad = int((got != exp).sum())
+            assert bad == 0, f"{bad} mismatches in chunk starting at {first:#x}"
+            start += n
+
+
+def test_dq_encode_e4m3_near_every_midpoint(Q, O, cuda):
+    """The FP8 (E4M3) search equals the oracle's brute force on every fp32
+    within 2^16 units in the last place of each of the 252 midpoints of the
+    code book, and on 2^24 spread values of [-1, 1]."""
+    t = O.e4m3_table().astype(np.float64)
+    mids = np.float32((t[:-1] + t[1:]) / 2).view(np.uint32)
+    for m in mids.tolist():
+        first = max(0, (m & 0x7FFFFFFF) - (1 << 16)) | (m & 0x80000000)
+        n = 1 << 17
+        y = torch.arange(first, first + n, dtype=torch.int64, device="cuda").to(torch.int32).view(torch.float32)
+        got = Q.qlora_dq_encode(y, "e4m3").cpu().numpy()
+        exp = O.dq_nearest_bits(first, n, "e4m3")
+        assert np.array_equal(got, exp), f"mismatch near midpoint bits {m:#x}"
+    hi = int(np.float32(1.0).view(np.uint32))
+    stride = hi // (1 << 23)
+    for sign in (0, 0x80000000):
+        bits = (np.arange(1 << 23, dtype=np.uint64) * stride).astype(np.uint32) | np.uint32(sign)
+        y = torch.from_numpy(bits.view(np.float32)).cuda()
+        got = Q.qlora_dq_encode(y, "e4m3").cpu().numpy()
+        exp = np.concatenate([O.dq_nearest_bits(int(b), 1, "e4m3") for b in bits[:: 1 << 12]])
+        assert np.array_equal(got[:: 1 << 12], exp)
