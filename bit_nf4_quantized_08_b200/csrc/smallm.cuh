@@ -119,7 +119,7 @@ __global__ void __launch_bounds__(SmallMShape<NT, NG>::THREADS, 1)
         *abort_flag = 0;
         fence_mbar_init();
     }
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) t8s[i] = dq_value(p.fmt.dq_type, i < 253 ? i : 0);
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) t8s[i] = dq_value(p.fmt.dq_type, (p.fmt.dq_type == 0 || i < 253) ? i : 0);
     if (warp == 0 && lane == 0) {
         pdl_trigger();
         prefetch_tensormap(&p.tmCodes);

@@ -141,7 +141,7 @@ __global__ void __launch_bounds__(SmallMmaShape<NT8, R>::THREADS, 1)
         sts_u32(lut_base + (uint32_t)(e * 256 + l * 4), pack_bf16x2(vlo, vhi));
     }
     for (int i = threadIdx.x; i < 256; i += blockDim.x)
-        sts_u32(t8s + 4u * i, __float_as_uint(dq_value(p.fmt.dq_type, i < 253 ? i : 0)));
+        sts_u32(t8s + 4u * i, __float_as_uint(dq_value(p.fmt.dq_type, (p.fmt.dq_type == 0 || i < 253) ? i : 0)));
     __syncthreads();
     // the weight, X and the adapter operands may come from the kernels just
     // before (the quantizer, the sU GEMM, an earlier layer): wait for them

@@ -29,7 +29,7 @@ def _threshold_tensor(O, code_type):
         f = np.float32(m)
         vals += [f, np.nextafter(f, np.float32(2)), np.nextafter(f, np.float32(-2)), np.float32(t[j])]
     vals = np.array(vals, np.float32)
-    body = np.tile(vals, 64)[:255 * 256].reshape(255, 256)
+    body = np.tile(vals, -(-255 * 256 // vals.size))[:255 * 256].reshape(255, 256)
     return np.concatenate([np.ones((255, 1), np.float32), body[:, :255]], axis=1)
 
 
