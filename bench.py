@@ -613,6 +613,24 @@ def extras(torch, Q, wl, device, flush, peaks):
         "frac_hbm": round(mbytes / ms / 1e6 / peaks["hbm_gbs"], 3), "algorithmic_bytes": int(mbytes)}
     del Wm, A, B, w
 
+    # AdamW step over every adapter parameter of the LLaMA-65B block (A and B
+    # of the 7 linears as one flat buffer): 16 B read + 14 B written each
+    npar = sum(nseg * 64 * K + nseg * S * 64 for _, nseg, S, K in block_groups(wl, "llama65b"))
+    pf = torch.randn(npar, device=device) * 0.01
+    mf, vf, gf = torch.zeros_like(pf), torch.zeros_like(pf), torch.randn(npar, device=device) * 1e-3
+    pb = torch.empty(npar, dtype=torch.bfloat16, device=device)
+    fn = lambda: Q.qlora_adamw_step(pf, mf, vf, gf, pb, lr=1e-4, step=10, weight_decay=0.01)  # noqa: E731
+    for _ in range(3):
+        fn()
+    g = graph_of(torch, fn)
+    ms = replay_ms(torch, g, 20, flush)
+    del g
+    abytes = 30 * npar
+    out["adamw_llama65b_block_adapters_cuda_graph"] = {
+        "params": int(npar), "us": round(ms * 1e3, 1), "GBps": round(abytes / ms / 1e6, 1),
+        "frac_hbm": round(abytes / ms / 1e6 / peaks["hbm_gbs"], 3), "algorithmic_bytes": int(abytes)}
+    del pf, mf, vf, gf, pb
+
     n = c["big_numel"]
     Wbig = wl.weight(n // 8192, 8192, seed=0, dtype=torch.bfloat16).to(device)
     qb = Q.NF4Weight.empty(n // 8192, 8192, True, device)

@@ -304,10 +304,12 @@ constexpr int kMaxSmallMCtas = 256;
 
 inline int small_m_nt(int64_t M) { return M <= 16 ? 16 : (M <= 32 ? 32 : 64); }
 
-// M <= kSmallMma: the register-fed warp-MMA kernel (smallm_mma.cuh) on a
-// persistent grid of at most kSmallMmaMaxCtas CTAs of 16 warps; its
-// workspace holds two fp32 partial slots of 1024 floats per warp and one
-// counter per 16-row group.
+// M <= kSmallMma in test mode 7: the register-fed warp-MMA kernel
+// (smallm_mma.cuh) on a persistent grid of at most kSmallMmaMaxCtas CTAs of
+// 16 warps; its workspace holds two fp32 partial slots of 1024 floats per
+// warp and one counter per 16-row group.  (It is correct but slower than the
+// tcgen05 kernel on the 22016 x 8192 weight: latency-bound with 16 warps of
+// 128 registers and one 4 KB item of codes in flight per warp.)
 constexpr int kSmallMma = 32;
 constexpr int kSmallMmaMaxCtas = 160;
 constexpr int kSmallMmaWarps = 16;
@@ -574,11 +576,11 @@ inline qlora_status launch_small_m_mma(const void* X, const LinearArgs& a, const
     return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
-// Y = X W'^T + sU B^T for 32 < M <= 64 on a persistent stream-K grid (one CTA
-// per SM, at least four (tile, k-step) units per CTA).
+// Y = X W'^T + sU B^T for M <= 64 on a persistent stream-K grid (one CTA per
+// SM, at least four (tile, k-step) units per CTA).
 inline qlora_status launch_small_m(const void* X, const LinearArgs& a, const void* B, void* Y,
                                    const LinearWs& L, cudaStream_t s) {
-    if (a.M <= kSmallMma && inject_mode() != 1) return launch_small_m_mma(X, a, B, Y, L, s);
+    if (a.M <= kSmallMma && inject_mode() == 7) return launch_small_m_mma(X, a, B, Y, L, s);
     const qlora_nf4_weight& w = *a.w;
     const int NT = small_m_nt(a.M);
     SmallMParams p;

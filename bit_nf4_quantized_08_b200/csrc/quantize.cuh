@@ -47,14 +47,11 @@ namespace qlora {
 // i.e. when fl(P_key - x) is negative (a difference of two finite floats is
 // zero only when they are equal), so the compare is one FADD and the sign
 // bit.
-// The key is formed as t = fl(128 x + 1.5 * 2^26 + 128): at that magnitude
-// the fp32 spacing is 8, so t rounds 128 x + 128 to a multiple of 8, i.e.
-// t = C + 8 RN(16 x + 16) (the same round-to-nearest-even as rounding 16 x
-// + 16 to an integer), and its low mantissa bits hold 8 key: (P_key,
-// base_key) sit as one 8-byte entry at byte 8 key of a 512-byte aligned
-// table, whose address is one AND-OR of t's bits.  64 entries and a 6-bit
-// key mask: any input (NaN included) reads inside the table.
-struct __align__(512) SearchSmem {
+// t = fl(16 x + 1.5 * 2^23 + 16) holds the key in its low mantissa bits
+// (0x4B400000 + key); (P_key, base_key) sit as one 8-byte entry, so one
+// shared load per element fetches both.  64 entries and a 6-bit key mask:
+// any input (NaN included) reads inside the table.
+struct __align__(16) SearchSmem {
     uint2 e[64];   // {P_key bits, base_key}
     int inc[64];
 };
@@ -66,24 +63,21 @@ __device__ __forceinline__ void load_search_tables(SearchSmem& st, const Nf4Sear
     }
 }
 
-constexpr float kKeyMagic = 100663424.0f;  // 1.5 * 2^26 + 128
+constexpr float kKeyMagic = 12582928.0f;  // 1.5 * 2^23 + 16
 
 // CT = 1 (FP4): a bucket's threshold may count twice (inc = 2).
 template <int CT = 0>
 __device__ __forceinline__ uint32_t nf4_lookup(float x, float t, const SearchSmem& st) {
-    const uint32_t tb = __float_as_uint(t);
-    uint32_t thr, base;
-    asm("ld.shared.v2.b32 {%0, %1}, [%2];"
-        : "=r"(thr), "=r"(base)
-        : "r"(smem_u32(st.e) | (tb & 0x1F8u)));
-    const uint32_t above = __float_as_uint(__fsub_rn(__uint_as_float(thr), x)) >> 31;
-    if (CT == 0) return base + above;
-    return base + above * (uint32_t)st.inc[(tb >> 3) & 63u];
+    const uint32_t key = __float_as_uint(t) & 63u;
+    const uint2 e = st.e[key];
+    const uint32_t above = __float_as_uint(__fsub_rn(__uint_as_float(e.x), x)) >> 31;
+    if (CT == 0) return e.y + above;
+    return e.y + above * (uint32_t)st.inc[key];
 }
 
 template <int CT = 0>
 __device__ __forceinline__ uint32_t nf4_search(float x, const SearchSmem& st) {
-    return nf4_lookup<CT>(x, fmaf(x, 128.0f, kKeyMagic), st);
+    return nf4_lookup<CT>(x, fmaf(x, 16.0f, kKeyMagic), st);
 }
 
 // Two lanes of fp32x2 arithmetic (sm_100a packed FP32): the same IEEE
@@ -112,7 +106,7 @@ template <int CT = 0>
 __device__ __forceinline__ void nf4_search2(float w0, float w1, uint64_t rcp2, const SearchSmem& st, uint32_t& c0,
                                             uint32_t& c1) {
     const uint64_t x2 = f2_mul(f2_pack(w0, w1), rcp2);
-    const uint64_t t2 = f2_fma(x2, f2_pack(128.0f, 128.0f), f2_pack(kKeyMagic, kKeyMagic));
+    const uint64_t t2 = f2_fma(x2, f2_pack(16.0f, 16.0f), f2_pack(kKeyMagic, kKeyMagic));
     float x0, x1, t0, t1;
     f2_unpack(x2, x0, x1);
     f2_unpack(t2, t0, t1);

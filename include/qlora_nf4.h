@@ -383,7 +383,9 @@ void qlora_set_wait_timeout_ns(uint64_t ns);
  * mode 5 forms the double-quantization offset in its own kernel even for
  * tensors whose 8-bit pass would form it itself; mode 6 runs the backward's
  * dA and dB GEMMs on the caller's stream after the dX GEMM instead of beside
- * it on the library's side stream.
+ * it on the library's side stream; mode 7 runs the forward for M <= 32 on the
+ * register-fed warp-MMA kernel (code-byte table lookups, block constant on
+ * each block's fp32 partial) instead of the tcgen05 small-M kernel.
  * Mode 0: normal (CTA-pair kernel, one pair per tile; in the backward the
  * dA/dB GEMMs beside the dX GEMM on the side stream).
  * The mode is process-wide: it changes the kernels of every later call from

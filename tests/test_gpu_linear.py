@@ -301,10 +301,10 @@ def test_small_m_graph_replay(Q, O, cuda):
 
 
 def test_small_m_timeout_is_reported_and_recovers(Q, O, cuda):
-    """Failure detection on the tcgen05 small-M kernel (33..64 tokens):
-    skipped loads make the bounded waits run out, TIMEOUT is reported, the
-    next call is correct.  (The warp-MMA kernel for M <= 32 has no waits.)"""
-    M, N, K, r = 40, 1024, 1024, 16
+    """Failure detection on the tcgen05 small-M kernel: skipped loads make
+    the bounded waits run out, TIMEOUT is reported, the next call is
+    correct.  (The warp-MMA kernel of test mode 7 has no waits.)"""
+    M, N, K, r = 16, 1024, 1024, 16
     q, inp, Wd_ref = _setup(Q, O, M, N, K, r, seed=9)
     X, A, B = inp["X"].cuda(), inp["A"].cuda(), inp["B"].cuda()
     Q.qlora_get_last_error()
@@ -319,3 +319,30 @@ def test_small_m_timeout_is_reported_and_recovers(Q, O, cuda):
     assert st == Q.QLORA_ERR_TIMEOUT
     got, ref = _fwd_both(Q, O, q, inp, Wd_ref, 2.0, r)
     assert_close_tol(got, ref, "Y after recovery")
+
+
+@pytest.mark.parametrize("M,N,K,r,nseg", [(1, 256, 128, 8, 1), (3, 1000, 512, 64, 1), (8, 22016, 8192, 64, 1),
+                                          (16, 4096, 8192, 64, 1), (17, 384, 256, 128, 1), (32, 2048, 4096, 32, 1),
+                                          (16, 3 * 1024, 2048, 32, 3), (5, 2000, 2048, 64, 1)])
+def test_small_m_warp_mma_kernel(Q, O, cuda, M, N, K, r, nseg):
+    """The register-fed warp-MMA small-M kernel (test mode 7: block constant
+    applied to each 64-element block's fp32 partial, bf16 table values times
+    a fixed prescale) against the oracle; the fused projection case checks
+    its segment columns of sU."""
+    S = N // nseg
+    W = wl.weight(N, K, seed=90, dtype=torch.bfloat16)
+    inp = wl.fused_inputs(M, nseg, S, K, r, seed=90, b_std=0.05)
+    q = Q.qlora_nf4_quantize(W.cuda())
+    ref_q = O.nf4_quantize(wl.bits(W).reshape(-1))
+    Wd = O.nf4_dequantize(N * K, ref_q).reshape(N, K)
+    Q.qlora_debug_inject(7)
+    try:
+        Y = Q.qlora_fused_linear_fwd(inp["X"].cuda(), q, nseg, inp["A"].cuda(), inp["B"].cuda(), 2.0)
+        Y2 = Q.qlora_fused_linear_fwd(inp["X"].cuda(), q, nseg, inp["A"].cuda(), inp["B"].cuda(), 2.0)
+        torch.cuda.synchronize()
+        assert Q.qlora_get_last_error() == 0
+    finally:
+        Q.qlora_debug_inject(0)
+    assert torch.equal(Y.view(torch.int16), Y2.view(torch.int16))
+    ref = O.fused_linear_fwd(wl.bits(inp["X"]), Wd, wl.bits(inp["A"]), wl.bits(inp["B"]), 2.0, nseg)
+    assert_close_tol(Y.float().cpu().numpy(), ref, f"Y warp-MMA M={M}")
