@@ -38,16 +38,18 @@ void side_stream_release();
 
 // ---- quantizer (quantize.cuh) ----
 // Host-built search table of the fast nearest-code search (33 buckets of
-// width 1/16 over [-1, 1], see quantize.cuh): per bucket the largest fp32
-// below its decision threshold (3.0 without one) and the count of
-// thresholds below the bucket.
+// width 1/16 over [-1, 1]; bucket k holds the x with RN(64 x + 64) in
+// [4k, 4k + 3], see quantize.cuh): per bucket the largest fp32 below its
+// decision threshold (3.0 without one) and the count of thresholds below the
+// bucket.
 // inc: how many thresholds sit at the bucket's one threshold value (1; 2 for
 // the FP4 code book, whose +0 code is never chosen, so that its threshold
 // coincides with the next one).
+constexpr int kSearchBuckets = 33;
 struct Nf4SearchTable {
-    float thr[33];
-    int base[33];
-    int inc[33];
+    float thr[kSearchBuckets];
+    int base[kSearchBuckets];
+    int inc[kSearchBuckets];
 };
 const Nf4SearchTable& nf4_search_table();
 void nf4_table_host(float out[16]);

@@ -304,16 +304,15 @@ constexpr int kMaxSmallMCtas = 256;
 
 inline int small_m_nt(int64_t M) { return M <= 16 ? 16 : (M <= 32 ? 32 : 64); }
 
-// M <= kSmallMma in test mode 7: the register-fed warp-MMA kernel
+// M <= kSmallMmaDefault (or M <= kSmallMma in test mode 7): the register-fed warp-MMA kernel
 // (smallm_mma.cuh) on a persistent grid of at most kSmallMmaMaxCtas CTAs of
-// 16 warps; its workspace holds two fp32 partial slots of 1024 floats per
-// warp and one counter per 16-row group.  (It is correct but slower than the
-// tcgen05 kernel on the 22016 x 8192 weight: latency-bound with 16 warps of
-// 128 registers and one 4 KB item of codes in flight per warp.)
+// 16 warps; its workspace holds two fp32 partial slots per CTA and row slice
+// (32 rows x 16 tokens or 16 rows x 32 tokens) and one 64-bit counter per
+// row slice of a 128- or 64-row group.
 constexpr int kSmallMma = 32;
+constexpr int kSmallMmaDefault = 16;
 constexpr int kSmallMmaMaxCtas = 160;
-constexpr int kSmallMmaWarps = 16;
-constexpr int kSmallMmaPartFloats = 2 * 1024;
+constexpr int kSmallMmaPartFloatsPerCta = 32768;  // at least 2 slots x 4 slices x 32 rows x 32 tokens
 
 inline int sm_count() {
     int dev = 0, n = 148;
@@ -345,11 +344,16 @@ inline LinearWs carve_linear_ws(void* ws, int64_t M, int64_t N, int64_t K, int r
     L.scales = big ? static_cast<float*>(c.take((size_t)(K / 64) * L.scales_ld * 4)) : nullptr;
     L.sU = r > 0 ? static_cast<uint16_t*>(c.take((size_t)M * r * 2)) : nullptr;
     L.sG = (r > 0 && bwd) ? static_cast<uint16_t*>(c.take((size_t)M * r * 2)) : nullptr;
-    // small-M forward: partial tiles [kMaxSmallMCtas][NT][128] and flags [kMaxSmallMCtas][4]
-    // (M <= 32: partial slots of the warp-MMA kernel and one counter per 32 rows)
-    const size_t part_floats = M <= kSmallMma ? (size_t)kSmallMmaMaxCtas * kSmallMmaWarps * kSmallMmaPartFloats
-                                              : (size_t)kMaxSmallMCtas * small_m_nt(M) * 128;
-    const size_t nflags = M <= kSmallMma ? (size_t)((N + 15) / 16) : (size_t)kMaxSmallMCtas * 4;
+    // small-M forward: partial tiles [kMaxSmallMCtas][NT][128] and flags
+    // [kMaxSmallMCtas][4] of the tcgen05 kernel; for M <= 32 also room for
+    // the warp-MMA kernel's partial slots and its counter per 16 rows (test
+    // mode 7 picks that kernel at run time, so both layouts must fit)
+    size_t part_floats = (size_t)kMaxSmallMCtas * small_m_nt(M) * 128;
+    size_t nflags = (size_t)kMaxSmallMCtas * 4;
+    if (M <= kSmallMma) {
+        part_floats = std::max(part_floats, (size_t)kSmallMmaMaxCtas * kSmallMmaPartFloatsPerCta);
+        nflags = std::max(nflags, (size_t)((N + 15) / 16) * 2);  // 64-bit counters
+    }
     L.part = big ? nullptr : static_cast<float*>(c.take(part_floats * 4));
     L.sm_flags = big ? nullptr : static_cast<uint32_t*>(c.take(nflags * 4));
     L.sk_part = big ? static_cast<float*>(c.take((size_t)kMaxStreamK * 256 * 256 * 4)) : nullptr;
@@ -517,18 +521,18 @@ inline cudaError_t launch_small_m_kernel(const SmallMParams& p, int grid, cudaSt
     return launch_pdl(kern, dim3((unsigned)grid, 1, 1), dim3(SmallMShape<NT, NG>::THREADS, 1, 1), smem, s, 0, p);
 }
 
-template <int NT8, int R>
+template <int MT>
 inline cudaError_t launch_small_m_mma_kernel(SmallMmaParams& p, cudaStream_t s) {
-    using S = SmallMmaShape<NT8, R>;
-    static_assert(S::SMEM <= 232448, "shared memory per CTA");
-    const int groups = (int)((p.N + S::GROWS - 1) / S::GROWS);
-    p.QW = (p.KB + S::QB - 1) / S::QB;
-    p.GL = p.QW + p.lora_ks;
-    p.items = (int64_t)groups * p.GL;
-    // at least 4 items per warp; at most one CTA per SM
+    using S = SmallMmaShape<MT>;
+    static_assert(S::SMEM + 256 * 32 * 4 <= 232448, "shared memory per CTA");
+    static_assert(2 * 4 * S::PART_FLOATS <= kSmallMmaPartFloatsPerCta, "partial workspace");
+    const int64_t groups = (p.N + S::UROWS - 1) / S::UROWS;
+    p.KSU = (p.KB + 3) / 4 + (p.lora_ks + 3) / 4;
+    p.units = groups * p.KSU;
+    // at least 4 units per CTA; at most one CTA per SM
     const int64_t ctas = std::max<int64_t>(1, std::min<int64_t>(std::min(sm_count(), kSmallMmaMaxCtas),
-                                                                p.items / (4 * S::WARPS)));
-    auto kern = k_smallm_mma<NT8, R>;
+                                                                p.units / 4));
+    auto kern = k_smallm_mma<MT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM);
     if (e != cudaSuccess) return e;
     ProfileScope ps(QLORA_KERNEL_SMALLM_GEMM, s);
@@ -540,39 +544,39 @@ inline cudaError_t launch_small_m_mma_kernel(SmallMmaParams& p, cudaStream_t s) 
 inline qlora_status launch_small_m_mma(const void* X, const LinearArgs& a, const void* B, void* Y,
                                        const LinearWs& L, cudaStream_t s) {
     const qlora_nf4_weight& w = *a.w;
+    const int MT = a.M <= 16 ? 1 : 2;
     SmallMmaParams p;
     memset(&p, 0, sizeof(p));
-    p.codes = w.codes;
+    // codes [N][K/2] bytes: 128-byte boxes (four blocks of a row) of UROWS
+    // rows, 128-byte swizzle (a warp's 8-byte reads of 8 rows hit 8 banks)
+    if (!make_map(&p.tmCodes, w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)(a.K / 2), (uint64_t)a.N,
+                  (uint64_t)(a.K / 2), 128, MT == 1 ? SmallMmaShape<1>::UROWS : SmallMmaShape<2>::UROWS,
+                  CU_TENSOR_MAP_SWIZZLE_128B))
+        return QLORA_ERR_CUDA;
+    if (!map_bf16(&p.tmX, X, a.K, a.M, 16 * MT)) return QLORA_ERR_CUDA;
+    if (a.r > 0 && !map_bf16(&p.tmU, L.sU, a.rt(), a.M, 16 * MT)) return QLORA_ERR_CUDA;
     p.q8 = w.absmax_q8;
     p.c1 = w.absmax_scale;
     p.offset = w.absmax_offset;
     p.absmax = w.absmax;
     p.dq = w.double_quant;
-    p.X = static_cast<const uint16_t*>(X);
     p.B = static_cast<const uint16_t*>(B);
-    p.sU = L.sU;
     p.M = (int)a.M;
     p.N = (int)a.N;
-    p.K = (int)a.K;
     p.KB = (int)(a.K / 64);
     p.r = a.r;
-    p.rt = a.rt();
     p.seg_rows = a.nseg > 1 ? (int)a.seg_rows : 0;
     p.lora_ks = a.r > 0 ? ceil_div(a.r, 64) : 0;
     p.fmt = weight_format(w);
     p.inv_scale = w.code_type ? 1.0f / 1.5f : 1.0f / 1.18881f;
     p.Y = static_cast<uint16_t*>(Y);
     p.part = L.part;
-    p.counters = L.sm_flags;
-    p.epoch = next_epoch() & 0xFFFFFFu;
+    p.counters = reinterpret_cast<unsigned long long*>(L.sm_flags);
+    p.epoch = next_epoch();
     if (p.epoch == 0) p.epoch = 1;
-    cudaError_t e;
-    if (a.M <= 8)
-        e = launch_small_m_mma_kernel<1, 2>(p, s);
-    else if (a.M <= 16)
-        e = launch_small_m_mma_kernel<2, 2>(p, s);
-    else
-        e = launch_small_m_mma_kernel<4, 1>(p, s);
+    p.timeout_ns = wait_timeout_ns();
+    p.inject = inject_mode() == 1 ? 1 : 0;
+    const cudaError_t e = MT == 1 ? launch_small_m_mma_kernel<1>(p, s) : launch_small_m_mma_kernel<2>(p, s);
     return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
@@ -580,7 +584,11 @@ inline qlora_status launch_small_m_mma(const void* X, const LinearArgs& a, const
 // SM, at least four (tile, k-step) units per CTA).
 inline qlora_status launch_small_m(const void* X, const LinearArgs& a, const void* B, void* Y,
                                    const LinearWs& L, cudaStream_t s) {
-    if (a.M <= kSmallMma && inject_mode() == 7) return launch_small_m_mma(X, a, B, Y, L, s);
+    // M <= 16: the warp-MMA kernel (test mode 8: the tcgen05 kernel instead);
+    // 17 <= M <= 32: the tcgen05 kernel (test mode 7: the warp-MMA kernel)
+    const int mode = inject_mode();
+    if ((a.M <= kSmallMmaDefault && mode != 8) || (a.M <= kSmallMma && mode == 7))
+        return launch_small_m_mma(X, a, B, Y, L, s);
     const qlora_nf4_weight& w = *a.w;
     const int NT = small_m_nt(a.M);
     SmallMParams p;

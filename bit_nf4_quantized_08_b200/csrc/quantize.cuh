@@ -36,48 +36,52 @@ namespace qlora {
 // ---------------------------------------------------------------------------
 // fast nearest-code search
 // ---------------------------------------------------------------------------
-// x in [-1.03, 1.03] falls in bucket key = RN(16 x + 16) in 0..32, i.e. the
-// closed interval [(key - 1/2)/16 - 1, (key + 1/2)/16 - 1].  Buckets are
-// narrower than the smallest gap between two decision thresholds (0.080), so
-// each holds at most one threshold T_key; base_key counts the thresholds at
-// or below the bucket's lower edge.  code(x) = base_key + (x >= T_key), where
-// threshold j is the smallest fp32 strictly above the exact midpoint of codes
-// j and j+1 (so an exact tie stays with the lower code).  The table holds
-// P_key, the largest fp32 below T_key: x >= T_key exactly when x > P_key,
-// i.e. when fl(P_key - x) is negative (a difference of two finite floats is
-// zero only when they are equal), so the compare is one FADD and the sign
-// bit.
-// t = fl(16 x + 1.5 * 2^23 + 16) holds the key in its low mantissa bits
-// (0x4B400000 + key); (P_key, base_key) sit as one 8-byte entry, so one
-// shared load per element fetches both.  64 entries and a 6-bit key mask:
-// any input (NaN included) reads inside the table.
+// t = fl(128 x + 1.5 * 2^24 + 128) lies in [2^24, 2^25) for |x| <= 1.03,
+// where the spacing of fp32 values is 2, so t = 1.5 * 2^24 + 2 v with
+// v = RN(64 x + 64) and the low mantissa bits of t hold v; the bucket is
+// key = floor(v / 4), and (t's bits & 0xFC) = 4 key is already the byte
+// offset of the bucket's 4-byte table entries: one LOP forms the address
+// of both tables, and 4-byte entries at a 4-byte stride put every bucket on
+// its own shared-memory bank (keys 0 and 32 share one, and both are rare).
+// Bucket key covers x in [(4 key - 64.5) / 64, (4 key - 60.5) / 64], an
+// interval of width 1/16, narrower than the smallest gap between two
+// decision thresholds (0.080), so each bucket holds at most one threshold
+// T_key; base_key counts the thresholds at or below the bucket's lower edge.
+// code(x) = base_key + (x >= T_key), where threshold j is the smallest fp32
+// strictly above the exact midpoint of codes j and j+1 (so an exact tie
+// stays with the lower code).  The table holds P_key, the largest fp32 below
+// T_key (3.0 without a threshold): x >= T_key exactly when x > P_key.  The
+// 8-bit mask keeps any input (NaN included) inside the 64-entry tables.
 struct __align__(16) SearchSmem {
-    uint2 e[64];   // {P_key bits, base_key}
-    int inc[64];
+    float P[64];     // P_key
+    uint32_t B[64];  // base_key | extra_key << 16
 };
 
 __device__ __forceinline__ void load_search_tables(SearchSmem& st, const Nf4SearchTable& tab) {
     for (int i = threadIdx.x; i < 64; i += blockDim.x) {
-        st.e[i] = make_uint2(__float_as_uint(i < 33 ? tab.thr[i] : 3.0f), (uint32_t)(i < 33 ? tab.base[i] : 15));
-        st.inc[i] = i < 33 ? tab.inc[i] : 0;
+        st.P[i] = i < kSearchBuckets ? tab.thr[i] : 3.0f;
+        st.B[i] = i < kSearchBuckets ? (uint32_t)tab.base[i] | ((uint32_t)max(tab.inc[i] - 1, 0) << 16) : 15u;
     }
 }
 
-constexpr float kKeyMagic = 12582928.0f;  // 1.5 * 2^23 + 16
+constexpr float kKeyMagic = 25165952.0f;  // 1.5 * 2^24 + 128
+constexpr float kKeyScale = 128.0f;
 
-// CT = 1 (FP4): a bucket's threshold may count twice (inc = 2).
+// CT = 1 (FP4): a bucket's threshold may count twice (inc = 2, stored as
+// extra = inc - 1 in the entry's high half; NF4 entries have extra = 0).
 template <int CT = 0>
 __device__ __forceinline__ uint32_t nf4_lookup(float x, float t, const SearchSmem& st) {
-    const uint32_t key = __float_as_uint(t) & 63u;
-    const uint2 e = st.e[key];
-    const uint32_t above = __float_as_uint(__fsub_rn(__uint_as_float(e.x), x)) >> 31;
-    if (CT == 0) return e.y + above;
-    return e.y + above * (uint32_t)st.inc[key];
+    const uint32_t off = __float_as_uint(t) & 0xFCu;
+    const float P = *reinterpret_cast<const float*>(reinterpret_cast<const char*>(st.P) + off);
+    const uint32_t e = *reinterpret_cast<const uint32_t*>(reinterpret_cast<const char*>(st.B) + off);
+    const uint32_t above = P < x ? 1u : 0u;
+    if (CT == 0) return e + above;
+    return (e & 0xFFFFu) + above * ((e >> 16) + 1u);
 }
 
 template <int CT = 0>
 __device__ __forceinline__ uint32_t nf4_search(float x, const SearchSmem& st) {
-    return nf4_lookup<CT>(x, fmaf(x, 16.0f, kKeyMagic), st);
+    return nf4_lookup<CT>(x, fmaf(x, kKeyScale, kKeyMagic), st);
 }
 
 // Two lanes of fp32x2 arithmetic (sm_100a packed FP32): the same IEEE
@@ -101,12 +105,33 @@ __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
     return d;
 }
 
+// The two bf16 values of a packed word as an fp32 pair {low half, high
+// half} in one 64-bit register (built in place, so no register moves).
+__device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t r) {
+    uint64_t d;
+    asm("{\n\t.reg .b32 lo, hi;\n\tshl.b32 lo, %1, 16;\n\tand.b32 hi, %1, 0xFFFF0000;\n\tmov.b64 %0, {lo, hi};\n\t}"
+        : "=l"(d)
+        : "r"(r));
+    return d;
+}
+
 // Codes of two elements x = fl(w * rcp) in one fp32x2 multiply and FMA.
+template <int CT = 0>
+__device__ __forceinline__ void nf4_search2p(uint64_t w2, uint64_t rcp2, const SearchSmem& st, uint32_t& c0,
+                                             uint32_t& c1) {
+    const uint64_t x2 = f2_mul(w2, rcp2);
+    const uint64_t t2 = f2_fma(x2, f2_pack(kKeyScale, kKeyScale), f2_pack(kKeyMagic, kKeyMagic));
+    float x0, x1, t0, t1;
+    f2_unpack(x2, x0, x1);
+    f2_unpack(t2, t0, t1);
+    c0 = nf4_lookup<CT>(x0, t0, st);
+    c1 = nf4_lookup<CT>(x1, t1, st);
+}
 template <int CT = 0>
 __device__ __forceinline__ void nf4_search2(float w0, float w1, uint64_t rcp2, const SearchSmem& st, uint32_t& c0,
                                             uint32_t& c1) {
     const uint64_t x2 = f2_mul(f2_pack(w0, w1), rcp2);
-    const uint64_t t2 = f2_fma(x2, f2_pack(16.0f, 16.0f), f2_pack(kKeyMagic, kKeyMagic));
+    const uint64_t t2 = f2_fma(x2, f2_pack(kKeyScale, kKeyScale), f2_pack(kKeyMagic, kKeyMagic));
     float x0, x1, t0, t1;
     f2_unpack(x2, x0, x1);
     f2_unpack(t2, t0, t1);
@@ -114,29 +139,30 @@ __device__ __forceinline__ void nf4_search2(float w0, float w1, uint64_t rcp2, c
     c1 = nf4_lookup<CT>(x1, t1, st);
 }
 
-// Pack 8 codes (element order) into one word: byte i = (c[2i] << 4) | c[2i+1].
-__device__ __forceinline__ uint32_t pack8(const uint32_t (&c)[8]) {
-    uint32_t acc = c[0];
-#pragma unroll
-    for (int i = 1; i < 8; ++i) acc = acc * 16u + c[i];  // c0 ends in the top nibble
-    return __byte_perm(acc, 0u, 0x0123);                 // reverse bytes: (c0,c1) -> byte 0
-}
+// Resident CTAs per SM the bf16 quantizer is compiled for (registers per
+// thread = 65536 / (256 * this)).
+#ifndef QLORA_QUANT_MIN_CTAS
+#define QLORA_QUANT_MIN_CTAS 4
+#endif
 
 // ---------------------------------------------------------------------------
-// K1: quantize.  One CTA (8 warps) per group of 16384 elements; warp w
-// handles rows 4w..4w+3 of 512 elements; a lane holds 16 consecutive
-// elements, 4 << bs_shift lanes make one block (64, 128 or 256 elements).
-// Also writes the group's fp64 pairwise-tree sum of block maxima for the
-// double-quantization offset.  CT: code book (0 NF4, 1 FP4).
+// K1: quantize.  A persistent grid; CTA c (8 warps) takes the groups of
+// 16384 elements c, c + G, c + 2G, ...; in a group, warp w handles rows
+// 4w..4w+3 of 512 elements, a lane holds 16 consecutive elements, and
+// 4 << BS lanes make one block (64, 128 or 256 elements).  As soon as a row
+// is coded, the lane loads its row of the CTA's next group into the same
+// registers, so every lane keeps four 32-byte (bf16) loads in flight while
+// it computes.  Also writes each group's fp64 pairwise-tree sum of block
+// maxima for the double-quantization offset.  CT: code book (0 NF4, 1 FP4).
 // ---------------------------------------------------------------------------
-template <bool BF16, int CT>
-__global__ void __launch_bounds__(256, BF16 ? 4 : 2) k_quantize_blocks(const void* W, int64_t n,
+template <bool BF16, int CT, int BS>
+__global__ void __launch_bounds__(256, BF16 ? QLORA_QUANT_MIN_CTAS : 2) k_quantize_blocks(const void* W, int64_t n,
                                                             uint8_t* codes,
                                                             float* absmax,
                                                             double* group_sums,
-                                                            Nf4SearchTable tab, int bs_shift) {
+                                                            Nf4SearchTable tab) {
     __shared__ SearchSmem st;
-    __shared__ double s_wsum[8];
+    __shared__ float s_max[2][256 >> BS];  // block maxima of a group (0 past the tensor), by group parity
     // dependent launch: resident before the kernel ahead ends, no access to
     // memory before it has.  The kernels that wait this way take no
     // __restrict__ pointers: with them the compiler may move loads of
@@ -147,129 +173,154 @@ __global__ void __launch_bounds__(256, BF16 ? 4 : 2) k_quantize_blocks(const voi
     __syncthreads();
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int bshift = 6 + bs_shift;                  // log2 of the block size
+    constexpr int bshift = 6 + BS;                    // log2 of the block size
+    constexpr int blanes = 4 << BS;                   // lanes per block
     const int64_t nb = (n + (1 << bshift) - 1) >> bshift;
-    const int blanes = 4 << bs_shift;                 // lanes per block
+    const int64_t ng = (n + 16383) >> 14;
     constexpr int WORDS = BF16 ? 8 : 16;  // 32-bit words per lane per row
     uint32_t raw[4][WORDS];
-    int64_t e0[4];
+    // first element of this lane in row it of group g: 16384 g + lbase + 512 it
+    const int64_t lbase = (int64_t)warp * 2048 + lane * 16;
 
-#pragma unroll
-    for (int it = 0; it < 4; ++it) {
-        e0[it] = (int64_t)blockIdx.x * 16384 + (int64_t)(warp * 4 + it) * 512 + lane * 16;
-        if (e0[it] + 16 <= n) {
-            const uint4* src = BF16 ? reinterpret_cast<const uint4*>(
-                                          static_cast<const uint16_t*>(W) + e0[it])
-                                    : reinterpret_cast<const uint4*>(
-                                          static_cast<const float*>(W) + e0[it]);
+    auto load_row = [&](int64_t e, uint32_t (&r)[WORDS]) {
+        if (e + 16 <= n) {
+            const uint4* src = BF16 ? reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(W) + e)
+                                    : reinterpret_cast<const uint4*>(static_cast<const float*>(W) + e);
 #pragma unroll
             for (int v = 0; v < WORDS / 4; ++v) {
                 uint4 q = __ldcs(src + v);
-                raw[it][4 * v + 0] = q.x;
-                raw[it][4 * v + 1] = q.y;
-                raw[it][4 * v + 2] = q.z;
-                raw[it][4 * v + 3] = q.w;
+                r[4 * v + 0] = q.x;
+                r[4 * v + 1] = q.y;
+                r[4 * v + 2] = q.z;
+                r[4 * v + 3] = q.w;
             }
         } else {
 #pragma unroll
-            for (int v = 0; v < WORDS; ++v) raw[it][v] = 0u;
-            if (e0[it] < n) {
+            for (int v = 0; v < WORDS; ++v) r[v] = 0u;
+            if (e < n) {
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    if (e0[it] + i < n) {
+                    if (e + i < n) {
                         if (BF16) {
-                            uint32_t h = static_cast<const uint16_t*>(W)[e0[it] + i];
-                            raw[it][i >> 1] |= h << ((i & 1) * 16);
+                            uint32_t h = static_cast<const uint16_t*>(W)[e + i];
+                            r[i >> 1] |= h << ((i & 1) * 16);
                         } else {
-                            raw[it][i] = __float_as_uint(static_cast<const float*>(W)[e0[it] + i]);
+                            r[i] = __float_as_uint(static_cast<const float*>(W)[e + i]);
                         }
                     }
                 }
             }
         }
+    };
+
+    int64_t g = blockIdx.x;
+    if (g < ng) {
+#pragma unroll
+        for (int it = 0; it < 4; ++it) load_row(g * 16384 + lbase + 512 * it, raw[it]);
     }
-
-    double rowsum[4];
+    for (int par = 0; g < ng; g += gridDim.x, par ^= 1) {
+        const int64_t gn = g + gridDim.x;  // this CTA's next group
 #pragma unroll
-    for (int it = 0; it < 4; ++it) {
-        // block absmax (exact: a max of magnitudes)
-        float a;
-        if (BF16) {
-            // packed bf16 max of magnitudes (the sign of each half is the xor
-            // of the signs, dropped at the end)
-            uint32_t m = raw[it][0];
+        for (int it = 0; it < 4; ++it) {
+            const int64_t e = g * 16384 + lbase + 512 * it;
+            // block absmax (exact: a max of magnitudes)
+            float a;
+            if (BF16) {
+                // packed bf16 max of magnitudes (the sign of each half is the xor
+                // of the signs, dropped at the end)
+                uint32_t m = raw[it][0];
 #pragma unroll
-            for (int i = 1; i < 8; ++i)
-                asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(m) : "r"(raw[it][i]));
-            m &= 0x7FFF7FFFu;
-            m = max(m & 0xFFFFu, m >> 16);
-            a = __uint_as_float(m << 16);
-        } else {
-            a = 0.0f;
+                for (int i = 1; i < 8; ++i)
+                    asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(m) : "r"(raw[it][i]));
+                m &= 0x7FFF7FFFu;
+                m = max(m & 0xFFFFu, m >> 16);
+                a = __uint_as_float(m << 16);
+            } else {
+                a = 0.0f;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(__uint_as_float(raw[it][i])));
-        }
-        for (int o = 1; o < blanes; o <<= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-
-        const int64_t b = e0[it] >> bshift;
-        const bool bvalid = b < nb;
-        if (bvalid && (lane & (blanes - 1)) == 0 && absmax) absmax[b] = a;
-
-        uint32_t c[16];
-        if (a >= 1.17549435e-38f) {
-            const float rcp = __frcp_rn(a);
-            const uint64_t rcp2 = f2_pack(rcp, rcp);
-#pragma unroll
-            for (int i = 0; i < 16; i += 2) {
-                const uint32_t b0 = BF16 ? (raw[it][i >> 1] << 16) : raw[it][i];
-                const uint32_t b1 = BF16 ? (raw[it][i >> 1] & 0xFFFF0000u) : raw[it][i + 1];
-                nf4_search2<CT>(__uint_as_float(b0), __uint_as_float(b1), rcp2, st, c[i], c[i + 1]);
+                for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(__uint_as_float(raw[it][i])));
             }
-        } else {
-            // zero or subnormal block: exact power-of-two prescale 2^64
-            const float p = 18446744073709551616.0f;
-            const float rcp = (a == 0.0f) ? 0.0f : __frcp_rn(__fmul_rn(a, p));
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const uint32_t bits = BF16 ? ((i & 1) ? (raw[it][i >> 1] & 0xFFFF0000u) : (raw[it][i >> 1] << 16))
-                                           : raw[it][i];
-                c[i] = nf4_search<CT>(__fmul_rn(__fmul_rn(__uint_as_float(bits), p), rcp), st);
+            for (int o = 1; o < blanes; o <<= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+
+            const int64_t b = e >> bshift;
+            if ((lane & (blanes - 1)) == 0) {
+                const bool bvalid = b < nb;
+                if (bvalid && absmax) absmax[b] = a;
+                // leaf of the group's tree: block (warp * 4 + it) * (32 / blanes) + lane / blanes
+                s_max[par][((warp * 4 + it) << (3 - BS)) + (lane >> (2 + BS))] = bvalid ? a : 0.0f;
             }
-        }
-        uint32_t lo[8], hi[8];
+
+            // codes packed as they are found: byte j of w[h] = (code[8h + 2j] << 4) | code[8h + 2j + 1]
+            uint32_t w[2] = {0u, 0u};
+            if (a >= 1.17549435e-38f) {
+                const float rcp = __frcp_rn(a);
+                const uint64_t rcp2 = f2_pack(rcp, rcp);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            lo[i] = c[i];
-            hi[i] = c[8 + i];
-        }
-        const uint32_t w0 = pack8(lo), w1 = pack8(hi);
-        if (e0[it] + 16 <= n) {
-            __stcs(reinterpret_cast<uint2*>(codes + (e0[it] >> 1)), make_uint2(w0, w1));
-        } else if (e0[it] < n) {
-            const int valid = (int)(n - e0[it]);
+                for (int i = 0; i < 16; i += 2) {
+                    uint32_t c0, c1;
+                    if (BF16) {
+                        nf4_search2p<CT>(bf16x2_to_f2(raw[it][i >> 1]), rcp2, st, c0, c1);
+                    } else {
+                        nf4_search2<CT>(__uint_as_float(raw[it][i]), __uint_as_float(raw[it][i + 1]), rcp2, st, c0,
+                                        c1);
+                    }
+                    // byte (i & 7) / 2 of w[i / 8]; the pairs are added in order with
+                    // shift-and-add steps, a byte-reverse at the end
+                    w[i >> 3] = (w[i >> 3] << 8) + (c0 << 4) + c1;
+                }
+                w[0] = __byte_perm(w[0], 0u, 0x0123);
+                w[1] = __byte_perm(w[1], 0u, 0x0123);
+            } else {
+                // zero or subnormal block: exact power-of-two prescale 2^64
+                const float p = 18446744073709551616.0f;
+                const float rcp = (a == 0.0f) ? 0.0f : __frcp_rn(__fmul_rn(a, p));
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {  // static indices: c stays in registers
-                if (2 * j < valid) {
-                    uint32_t byte = c[2 * j] << 4;
-                    if (2 * j + 1 < valid) byte |= c[2 * j + 1];
-                    codes[(e0[it] >> 1) + j] = (uint8_t)byte;
+                for (int i = 0; i < 16; ++i) {
+                    const uint32_t bits = BF16 ? ((i & 1) ? (raw[it][i >> 1] & 0xFFFF0000u) : (raw[it][i >> 1] << 16))
+                                               : raw[it][i];
+                    const uint32_t c = nf4_search<CT>(__fmul_rn(__fmul_rn(__uint_as_float(bits), p), rcp), st);
+                    w[i >> 3] += c << (4 * ((i & 7) ^ 1));
+                }
+            }
+            // the row is coded: its registers take the next group's row
+            if (gn < ng) load_row(gn * 16384 + lbase + 512 * it, raw[it]);
+            if (e + 16 <= n) {
+                __stcs(reinterpret_cast<uint2*>(codes + (e >> 1)), make_uint2(w[0], w[1]));
+            } else if (e < n) {
+                const int valid = (int)(n - e);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    if (2 * j < valid) {
+                        uint32_t byte = (w[j >> 2] >> (8 * (j & 3))) & 0xFFu;
+                        if (2 * j + 1 >= valid) byte &= 0xF0u;  // no element after the last one
+                        codes[(e >> 1) + j] = (uint8_t)byte;
+                    }
                 }
             }
         }
-
-        // fp64 pairwise tree over the row's block maxima (8, 4 or 2 of them;
-        // blocks beyond the tensor contribute zeros).
-        double d = bvalid ? (double)a : 0.0;
-        for (int o = blanes; o < 32; o <<= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
-        rowsum[it] = d;
-    }
-    if (group_sums) {
-        if (lane == 0) s_wsum[warp] = (rowsum[0] + rowsum[1]) + (rowsum[2] + rowsum[3]);
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            double t0 = s_wsum[0] + s_wsum[1], t1 = s_wsum[2] + s_wsum[3];
-            double t2 = s_wsum[4] + s_wsum[5], t3 = s_wsum[6] + s_wsum[7];
-            group_sums[blockIdx.x] = (t0 + t1) + (t2 + t3);
+        if (group_sums) {
+            // fp64 pairwise tree over the group's 256 >> BS block maxima in
+            // block order: each lane of warp 0 folds its run of adjacent
+            // leaves, then the lanes pair up (x + y and y + x are the same
+            // IEEE sum, so both lanes of a pair agree).  The next group
+            // writes the other parity's leaves, and the one after waits at
+            // this barrier of the next group, after warp 0 has read these.
+            __syncthreads();
+            if (warp == 0) {
+                constexpr int PER = 8 >> BS;  // leaves per lane
+                double v[PER];
+#pragma unroll
+                for (int i = 0; i < PER; ++i) v[i] = (double)s_max[par][lane * PER + i];
+#pragma unroll
+                for (int w = 1; w < PER; w <<= 1)
+#pragma unroll
+                    for (int i = 0; i < PER; i += 2 * w) v[i] = v[i] + v[i + w];
+                double t = v[0];
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+                if (lane == 0) group_sums[g] = t;
+            }
         }
     }
 }
@@ -362,15 +413,22 @@ __device__ __forceinline__ float t8_threshold(int k) {
     return f;
 }
 
-// Nearest 8-bit code of y in [-1, 1]: the candidate rint(127 y) + 127 is the
-// nearest code or its neighbour (y is within half a step of t8[candidate]),
-// so two fp32 compares with the thresholds on either side decide; ties go
-// to the lower index.  thr = the 254 thresholds (shared memory).
+// Nearest 8-bit code of y in [-1, 1]: the candidate k0 = RN(127 y + 127),
+// formed by one FMA with 1.5 * 2^23 + 127 (the sum's low mantissa bits are
+// k0), is the nearest code or its neighbour (y is within half a step of
+// t8[k0]), so two fp32 compares with the thresholds on either side decide;
+// ties go to the lower index.  thr = the padded thresholds (shared memory):
+// thr[0] = -inf, thr[k + 1] = T_k (k = 0..253), thr[255..259] = +inf, so no
+// candidate needs a range check (any input, NaN included, reads inside).
+constexpr int kT8Pad = 260;
+__device__ __forceinline__ float t8_threshold_padded(int i) {
+    if (i == 0) return -INFINITY;
+    return i <= 254 ? t8_threshold(i - 1) : INFINITY;
+}
 __device__ __forceinline__ int nearest_t8(float y, const float* thr) {
-    int k0 = __float2int_rn(__fmul_rn(y, 127.0f)) + 127;
-    k0 = min(max(k0, 0), 254);
-    const int down = (k0 > 0 && y < thr[k0 - 1]) ? 1 : 0;
-    const int up = (k0 < 254 && y >= thr[k0]) ? 1 : 0;
+    const int k0 = (int)(__float_as_uint(__fmaf_rn(y, 127.0f, 12583039.0f)) & 0xFFu);
+    const int down = y < thr[k0] ? 1 : 0;
+    const int up = y >= thr[k0 + 1] ? 1 : 0;
     return k0 - down + up;
 }
 
@@ -401,23 +459,35 @@ __global__ void __launch_bounds__(256) k_dq_quantize(const float* absmax, int64_
                                                      uint8_t* q8,
                                                      float* c1,
                                                      const double* sums, int64_t nsums, int dt) {
-    __shared__ float t8[256];  // E4M3: the 253 code values; linear: the 254 decision thresholds
+    __shared__ float t8[kT8Pad];  // E4M3: the 253 code values; linear: the padded decision thresholds
     __shared__ double s_w[8];
     __shared__ float s_off;
     pdl_trigger();
-    // blockDim.x == 256; shared memory only
-    t8[threadIdx.x] = dt ? (threadIdx.x < 253 ? e4m3_value(threadIdx.x) : 2.0f)
-                         : (threadIdx.x < 254 ? t8_threshold(threadIdx.x) : 3.0f);
+    // shared memory only
+    for (int i = threadIdx.x; i < kT8Pad; i += blockDim.x)
+        t8[i] = dt ? (i < 253 ? e4m3_value(i) : 2.0f) : t8_threshold_padded(i);
     pdl_wait();
     // this warp's first group: 8 block maxima per lane, loaded before the
     // offset tree so that the two memory round trips overlap
     const int64_t g = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     const int64_t ng = (nb + 255) >> 8;
-    const int64_t bf = g * 256 + lane * 8;
-    float am[8];
+    // 8 consecutive maxima of lane's share of group gg (two 16-byte loads
+    // when all 8 exist)
+    auto load8 = [&](int64_t gg, float (&a)[8]) {
+        const int64_t b0 = gg * 256 + lane * 8;
+        if (gg < ng && b0 + 8 <= nb) {
+            const float4 v0 = *reinterpret_cast<const float4*>(absmax + b0);
+            const float4 v1 = *reinterpret_cast<const float4*>(absmax + b0 + 4);
+            a[0] = v0.x; a[1] = v0.y; a[2] = v0.z; a[3] = v0.w;
+            a[4] = v1.x; a[5] = v1.y; a[6] = v1.z; a[7] = v1.w;
+        } else {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) am[i] = (g < ng && bf + i < nb) ? absmax[bf + i] : 0.0f;
+            for (int i = 0; i < 8; ++i) a[i] = (gg < ng && b0 + i < nb) ? absmax[b0 + i] : 0.0f;
+        }
+    };
+    float am[8];
+    load8(g, am);
     if (sums) {
         int64_t p2 = 1;
         while (p2 < nsums) p2 <<= 1;
@@ -437,13 +507,13 @@ __global__ void __launch_bounds__(256) k_dq_quantize(const float* absmax, int64_
     __syncthreads();
     const float off = s_off;
     // one warp per group of 256 blocks; the grid is capped, so a warp takes
-    // every (gridDim.x * 8)-th group
-    for (int64_t gg = g; gg < ng; gg += (int64_t)gridDim.x * 8) {
+    // every (gridDim.x * 8)-th group, loading the next group's maxima while
+    // it quantizes the current one
+    const int64_t gstride = (int64_t)gridDim.x * 8;
+    for (int64_t gg = g; gg < ng; gg += gstride) {
         const int64_t b0 = gg * 256 + lane * 8;
-        if (gg != g) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) am[i] = b0 + i < nb ? absmax[b0 + i] : 0.0f;
-        }
+        float nx[8];
+        load8(gg + gstride, nx);
         float d[8];
         float c = 0.0f;
 #pragma unroll
@@ -472,6 +542,8 @@ __global__ void __launch_bounds__(256) k_dq_quantize(const float* absmax, int64_
                 if (b0 + i < nb) q8[b0 + i] = (uint8_t)q[i];
         }
         if (lane == 0) c1[gg] = c;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) am[i] = nx[i];
     }
 }
 
@@ -577,9 +649,9 @@ __global__ void k_encode(const float* __restrict__ x, int64_t n, uint8_t* __rest
 // Nearest 8-bit code of every y (test entry point: the search of the double
 // quantization on arbitrary inputs).
 __global__ void k_dq_encode(const float* __restrict__ y, int64_t n, uint8_t* __restrict__ codes, int dt) {
-    __shared__ float t8[256];
-    t8[threadIdx.x] = dt ? (threadIdx.x < 253 ? e4m3_value(threadIdx.x) : 2.0f)
-                         : (threadIdx.x < 254 ? t8_threshold(threadIdx.x) : 3.0f);
+    __shared__ float t8[kT8Pad];
+    for (int i = threadIdx.x; i < kT8Pad; i += blockDim.x)
+        t8[i] = dt ? (i < 253 ? e4m3_value(i) : 2.0f) : t8_threshold_padded(i);
     __syncthreads();
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
         const float v = fminf(fmaxf(y[i], -1.0f), 1.0f);
@@ -621,8 +693,9 @@ inline Nf4SearchTable build_search_table(int ct) {
         thr[j] = f;
     }
     Nf4SearchTable t;
-    for (int k = 0; k <= 32; ++k) {
-        double lo = (k - 0.5) / 16.0 - 1.0, hi = (k + 0.5) / 16.0 - 1.0;
+    for (int k = 0; k < kSearchBuckets; ++k) {
+        // key k: RN(64 x + 64) in [4k, 4k + 3]
+        const double lo = (4.0 * k - 64.5) / 64.0, hi = (4.0 * k - 60.5) / 64.0;
         int base = 0, inc = 0;
         float tk = 3.0f;  // no threshold inside the bucket
         for (int j = 0; j < 15; ++j) {
@@ -654,10 +727,19 @@ inline cudaError_t launch_quantize_blocks(const void* W, int is_bf16, int64_t n,
     ProfileScope ps(QLORA_KERNEL_QUANTIZE, s);
     note_launch();
     const Nf4SearchTable& tab = search_table(fmt.code_type);
-    auto kern = is_bf16 ? (fmt.code_type ? k_quantize_blocks<true, 1> : k_quantize_blocks<true, 0>)
-                        : (fmt.code_type ? k_quantize_blocks<false, 1> : k_quantize_blocks<false, 0>);
-    return launch_pdl(kern, dim3((unsigned)ng), dim3(256), 0, s, 0, W, n, codes, absmax, group_sums, tab,
-                      fmt.bs_shift);
+    using Kern = void (*)(const void*, int64_t, uint8_t*, float*, double*, Nf4SearchTable);
+    static constexpr Kern kTable[2][2][3] = {
+        {{k_quantize_blocks<false, 0, 0>, k_quantize_blocks<false, 0, 1>, k_quantize_blocks<false, 0, 2>},
+         {k_quantize_blocks<false, 1, 0>, k_quantize_blocks<false, 1, 1>, k_quantize_blocks<false, 1, 2>}},
+        {{k_quantize_blocks<true, 0, 0>, k_quantize_blocks<true, 0, 1>, k_quantize_blocks<true, 0, 2>},
+         {k_quantize_blocks<true, 1, 0>, k_quantize_blocks<true, 1, 1>, k_quantize_blocks<true, 1, 2>}}};
+    const Kern kern = kTable[is_bf16 ? 1 : 0][fmt.code_type ? 1 : 0][fmt.bs_shift];
+    // persistent: as many CTAs as are resident at once, at most one per group
+    int dev = 0, nsm = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        nsm = 148;
+    const int64_t grid = std::min<int64_t>(ng, (int64_t)nsm * (is_bf16 ? QLORA_QUANT_MIN_CTAS : 2));
+    return launch_pdl(kern, dim3((unsigned)grid), dim3(256), 0, s, 0, W, n, codes, absmax, group_sums, tab);
 }
 
 inline cudaError_t launch_dq_offset(const double* group_sums, int64_t ngroups, int64_t nb,

@@ -1,7 +1,7 @@
 // smallm_mma.cuh -- the forward for few tokens (M <= 32), where the layer is
 // bound by the bytes of the 4-bit weight.
 //
-//   Y^T [N x M] = W' [N x K] X^T + B [N x r] sU^T,   sU = bf16(s X A^T)
+//   Y [M x N] = X W'^T + sU B^T,   sU = bf16(s X A^T)
 //
 // The block constant is factored out of each 64-element block (QLoRA paper
 // digest, sec. 4 doubleDequant: w' = nf4[code] * a'):
@@ -10,33 +10,38 @@
 // from a table instead of being rebuilt per block; L = 1.18881 is a fixed
 // prescale that halves the bf16 rounding error of those 16 values (largest
 // relative error 1.6e-3 instead of 3.1e-3).  The inner sums are warp-level
-// tensor-core MMAs (m16n8k16, bf16 in, fp32 out) fed from registers: 16
-// weight rows by 8 tokens per instruction, so the expanded weight never
-// touches shared memory and no MMA completion has to be signalled.
+// tensor-core MMAs (m16n8k16, bf16 in, fp32 out) fed from registers, with
+// the tokens on the MMA's 16-row side (A) and 8 weight rows on its 8-column
+// side (B), so the expanded weight never touches shared memory.
 //
 // Lookup: a 256-entry table of bf16 pairs, one entry per code byte (the two
 // codes of two neighbouring elements), replicated for the 32 lanes at a
-// 256-byte stride in shared memory, so entry e of lane l sits at
-// base + e * 256 + l * 4: one PRMT forms the address from the code byte and
-// the lane's base, one conflict-free LDS returns the two bf16 values of an
-// MMA operand register.
+// 128-byte stride in shared memory (32 KB), so entry e of lane l sits at
+// e * 128 + l * 4 and every lane reads its own bank: a shift and a LOP3 form
+// the offset, one LDS returns the two bf16 values of a B operand register.
 //
 // K permutation: within each 64-element block, MMA k-index j of thread
-// group position t (the fragment's columns 2t, 2t+1, 2t+8, 2t+9 of chunk c)
+// group position t (the fragment's k rows 2t, 2t+1, 2t+8, 2t+9 of chunk c)
 // maps to the physical elements 16t + 4c + {0, 1, 2, 3}.  A sum over k does
 // not depend on the order, as long as both operands use the same map; with
 // it every thread reads 8 contiguous code bytes per weight row and 32
 // contiguous bytes of X per token for a block.
 //
-// Work split: items are (group of 16R weight rows, four 64-element blocks),
-// so that each row is read in whole 128-byte lines, with the LoRA
-// up-projection as extra 64-wide items after the weight items; every warp of
-// a persistent grid takes one contiguous share of the item list (stream-K),
-// so each streams the same number of weight bytes, and loads the codes of
-// its next item while it computes the current one.  A group cut
-// between warps is finished by whichever of its warps arrives last (an
-// integer counter): it adds every warp's fp32 partial in warp order
-// (deterministic) and writes Y.  Nothing waits on another warp.
+// Work split: a unit is (128 weight rows, four consecutive 64-element
+// blocks) for up to 16 tokens (64 rows for up to 32), so that every row of
+// the unit is one 128-byte line of codes; the LoRA up-projection adds units
+// of four 64-wide adapter blocks after a row group's weight units.  A
+// persistent grid of one CTA per SM takes contiguous shares of the unit list
+// (stream-K), so every SM streams the same number of weight bytes.  The 16
+// warps of a CTA split a unit into 4 row slices x 4 blocks; the codes (one
+// TMA box, 128-byte swizzle) and the four X blocks of each unit pass through
+// a 6-stage ring, and the last warp to finish with a stage loads the unit
+// that comes XS units later into it (no producer warp).  At the end of a row
+// group the four warps of a slice add their accumulators in block order
+// through shared memory; a group cut between CTAs is finished, per slice, by
+// whichever contributing CTA arrives last (an integer counter with a launch
+// epoch): it adds every contributor's fp32 partial in CTA order
+// (deterministic) and writes Y.  Nothing waits on another CTA.
 #pragma once
 
 #include "common.cuh"
@@ -49,370 +54,509 @@ namespace qlora {
 __device__ __forceinline__ float small_m_table_scale(int ct) { return ct ? 1.5f : 1.18881f; }
 
 struct SmallMmaParams {
-    const uint8_t* codes;   // [N][K/2]
-    const uint8_t* q8;      // [N * K/64] (double quantization)
+    CUtensorMap tmCodes;    // codes [N][K/2] bytes, box {128 B, UROWS rows}, 128-byte swizzle
+    CUtensorMap tmX;        // X [M][K] bf16, box {64, 16 MT}, 128-byte swizzle
+    CUtensorMap tmU;        // sU [M][rt] bf16, box {64, 16 MT}, 128-byte swizzle
+    const uint8_t* q8;      // [N * K/64 >> bs_shift] (double quantization)
     const float* c1;
     const float* offset;
-    const float* absmax;    // [N * K/64] without double quantization
+    const float* absmax;    // without double quantization
     int dq;
-    const uint16_t* X;      // [M][K] bf16
     const uint16_t* B;      // [N][r] bf16 (LoRA), unused when lora_ks == 0
-    const uint16_t* sU;     // [M][rt] bf16
-    int M, N, K, KB;        // KB = K / 64
-    int r, rt, seg_rows, lora_ks;
+    int M, N, KB;           // KB = K / 64
+    int r, seg_rows, lora_ks;
+    int KSU;                // units per row group: ceil(KB / 4) + ceil(lora_ks / 4)
+    int64_t units;          // groups * KSU
     float inv_scale;        // 1 / L
     QFormat fmt;            // code book, 8-bit code book, block size
-    int QW;                 // weight items per group: ceil(KB / QB)
-    int GL;                 // items per group: QW + lora_ks
-    int64_t items;          // groups * GL
     uint16_t* Y;            // [M][N]
-    float* part;            // [warps][2][16R][8 NT8] fp32 partials
-    uint32_t* counters;     // [groups]: (epoch << 8) | arrivals
-    uint32_t epoch;         // 24 bits, nonzero
+    float* part;            // [gridDim.x][2 slots][4 slices][SROWS rows][16 MT tokens] fp32 partials
+    unsigned long long* counters;  // [groups * 4 slices]: (epoch << 32) | arrivals
+    uint32_t epoch;         // nonzero
+    uint64_t timeout_ns;
+    int inject;             // test mode 1: issue no loads (the waits run out)
 };
 
-template <int NT8, int R>
+template <int MT>
 struct SmallMmaShape {
-    static constexpr int WARPS = 16;
+    static constexpr int WARPS = 16;              // 4 row slices x 4 blocks of a unit
+    static constexpr int RT = MT == 1 ? 4 : 2;    // 8-row tiles per warp
+    static constexpr int SROWS = 8 * RT;          // rows of a slice (32 or 16)
+    static constexpr int UROWS = 4 * SROWS;       // rows of a unit (128 or 64)
     static constexpr int THREADS = 32 * WARPS;
-    static constexpr int NPAD = 8 * NT8;
-    static constexpr int GROWS = 16 * R;
-    static constexpr int QB = 4;  // 64-element blocks per weight item: a 128-byte line of every row
-    // 64 KB table at the first 64 KB-aligned shared address, the fp32 t8
-    // table of the double quantization below it
-    static constexpr int SMEM = 2 * 65536;
-    static constexpr int PART_FLOATS = 2 * GROWS * NPAD;  // per warp
+    static constexpr int XS = 6;                  // ring stages
+    static constexpr int X_TILE = 16 * MT * 128;  // 16 MT tokens x 64 bf16
+    static constexpr int CODE_BYTES = UROWS * 128;  // codes of one unit (128-byte swizzle)
+    static constexpr int STAGE = CODE_BYTES + 4 * X_TILE;
+    // dynamic shared memory (1024-aligned): ring, t8 table, scale scratch,
+    // accumulator exchange, barriers and stage counters
+    static constexpr int OFF_T8 = XS * STAGE;
+    static constexpr int OFF_SC = OFF_T8 + 1024;                     // [WARPS][2][SROWS] fp32
+    static constexpr int OFF_XCH = OFF_SC + WARPS * 2 * SROWS * 4;  // [WARPS][RT * MT * 4][32] fp32
+    static constexpr int OFF_BAR = OFF_XCH + WARPS * RT * MT * 4 * 32 * 4;  // full[XS]
+    static constexpr int OFF_CNT = OFF_BAR + 8 * XS;                // done[XS], issued[XS], abort flag
+    static constexpr int SMEM = OFF_CNT + 8 * XS + 16 + 1024;       // + alignment slack
+    static constexpr int PART_FLOATS = SROWS * 16 * MT;  // one slice's partial tile
 };
 
+// (not volatile: pure functions of their registers, so the compiler may
+// interleave independent MMA chains)
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                           uint32_t b0, uint32_t b1) {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
         "{%0, %1, %2, %3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
+// d = A B (no accumulator input)
+__device__ __forceinline__ void mma_16816_z(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                            uint32_t b0, uint32_t b1) {
+    const float z = 0.0f;
+    asm(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%10, %10, %10, %10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(z));
+}
 
-__device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
-    uint32_t v;
-    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(a));
+
+// The lookup table (static shared memory): entry e of lane l at e * 128 + l * 4.
+__shared__ __align__(128) uint32_t g_small_m_lut[256 * 32];
+
+// Table entry of byte k (0..3) of word w for this lane (lane4 = lane * 4).
+// The table does not change after the kernel's first barrier, so the load is
+// not volatile (its address depends on code words read after the stage's
+// barrier wait).
+__device__ __forceinline__ uint32_t lut_byte(uint32_t w, int k, uint32_t lane4) {
+    const uint32_t off = (((w >> (8 * k)) << 7) & 0x7F80u) | lane4;
+    return *reinterpret_cast<const uint32_t*>(reinterpret_cast<const char*>(g_small_m_lut) + off);
+}
+__device__ __forceinline__ uint2 ld_shared_v2(uint32_t addr) {
+    uint2 v;
+    asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
     return v;
 }
-__device__ __forceinline__ float lds_f32(uint32_t a) { return __uint_as_float(lds_u32(a)); }
-__device__ __forceinline__ void sts_u32(uint32_t a, uint32_t v) {
-    asm volatile("st.shared.b32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+
+// Index of the CTA whose share [I c / G, I (c + 1) / G) holds unit x.
+__device__ __forceinline__ int owner_cta(int64_t x, int64_t I, int G) {
+    int c = (int)((x * G) / I);
+    while (c + 1 < G && (I * (c + 1)) / G <= x) ++c;
+    while (c > 0 && (I * c) / G > x) --c;
+    return c;
 }
 
-// Table entry of byte k (0..3) of word w for this lane: lane_base holds the
-// table base (64 KB aligned) plus lane * 4, so the address is
-// [lane_base.b3, lane_base.b2, w.byte_k, lane_base.b0].
-template <int KBYTE>
-__device__ __forceinline__ uint32_t lut(uint32_t w, uint32_t lane_base) {
-    return lds_u32(prmt(w, lane_base, 0x7604u | (KBYTE << 4)));
+__device__ __forceinline__ void named_sync(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
-// Index of the warp whose share [I w / G, I (w + 1) / G) holds item x.
-__device__ __forceinline__ int owner_warp(int64_t x, int64_t I, int G) {
-    int w = (int)((x * G) / I);
-    while (w + 1 < G && (I * (w + 1)) / G <= x) ++w;
-    while (w > 0 && (I * w) / G > x) --w;
-    return w;
-}
-
-template <int NT8, int R>
-__global__ void __launch_bounds__(SmallMmaShape<NT8, R>::THREADS, 1)
+template <int MT>
+__global__ void __launch_bounds__(SmallMmaShape<MT>::THREADS, 1)
     k_smallm_mma(const __grid_constant__ SmallMmaParams p) {
-    using S = SmallMmaShape<NT8, R>;
-    constexpr int NPAD = S::NPAD, GROWS = S::GROWS;
+    using S = SmallMmaShape<MT>;
+    constexpr int RT = S::RT, XS = S::XS, SROWS = S::SROWS, UROWS = S::UROWS, WARPS = S::WARPS;
+    constexpr int TOK = 16 * MT;
     extern __shared__ uint8_t smem_raw[];
-    const uint32_t sbase = smem_u32(smem_raw);
-    const uint32_t lut_base = (sbase + 0xFFFFu) & ~0xFFFFu;
-    // the fp32 t8 table (1 KB): below the lookup table when there is room, else after it
-    const uint32_t t8s = (lut_base - sbase >= 1024u) ? sbase : lut_base + 65536u;
+    const uint32_t raw_base = smem_u32(smem_raw);
+    const uint32_t base = (raw_base + 1023u) & ~1023u;
+    uint8_t* gb = smem_raw + (base - raw_base);
+    float* t8s = reinterpret_cast<float*>(gb + S::OFF_T8);
+    float* xch = reinterpret_cast<float*>(gb + S::OFF_XCH);
+    const uint32_t bar = base + S::OFF_BAR;
+    auto full = [&](int s) { return bar + 8u * s; };
+    int* done = reinterpret_cast<int*>(gb + S::OFF_CNT);  // warps finished with the stage's unit
+    int* issued = done + XS;                                // loads issued into the stage
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(gb + S::OFF_CNT + 8 * XS);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gid = lane >> 2, tig = lane & 3;
+    const int slice = warp >> 2, bq = warp & 3;  // row slice and block of a unit
+    const WaitCfg wc{p.timeout_ns};
 
-    // tables: entry e = {L nf4[e >> 4] (bits 0..15), L nf4[e & 15] (bits 16..31)}
-    for (int idx = threadIdx.x; idx < 256 * 32; idx += blockDim.x) {
-        const int e = idx >> 5, l = idx & 31;
+    // table: entry e = {L v[e >> 4] (bits 0..15), L v[e & 15] (bits 16..31)}
+    {
         const float L = small_m_table_scale(p.fmt.code_type);
-        const float vlo = __fmul_rn(code_value(p.fmt.code_type, e >> 4), L);
-        const float vhi = __fmul_rn(code_value(p.fmt.code_type, e & 15), L);
-        sts_u32(lut_base + (uint32_t)(e * 256 + l * 4), pack_bf16x2(vlo, vhi));
+        for (int idx = threadIdx.x; idx < 256 * 32; idx += blockDim.x) {
+            const int e = idx >> 5;
+            const float vlo = __fmul_rn(code_value(p.fmt.code_type, e >> 4), L);
+            const float vhi = __fmul_rn(code_value(p.fmt.code_type, e & 15), L);
+            g_small_m_lut[idx] = pack_bf16x2(vlo, vhi);
+        }
     }
     for (int i = threadIdx.x; i < 256; i += blockDim.x)
-        sts_u32(t8s + 4u * i, __float_as_uint(dq_value(p.fmt.dq_type, (p.fmt.dq_type == 0 || i < 253) ? i : 0)));
+        t8s[i] = dq_value(p.fmt.dq_type, (p.fmt.dq_type == 0 || i < 253) ? i : 0);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < XS; ++s) {
+            mbar_init(full(s), 1);
+            done[s] = 0;
+            issued[s] = 0;
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+        pdl_trigger();
+        prefetch_tensormap(&p.tmCodes);
+        prefetch_tensormap(&p.tmX);
+        if (p.lora_ks) prefetch_tensormap(&p.tmU);
+    }
     __syncthreads();
     // the weight, X and the adapter operands may come from the kernels just
     // before (the quantizer, the sU GEMM, an earlier layer): wait for them
     pdl_wait();
-    const uint32_t lane_base = lut_base + (uint32_t)lane * 4u;
+
+    const int QW = (p.KB + 3) >> 2;        // weight units per row group
+    const int64_t U = p.units;
+    const int G = gridDim.x;
+    const int64_t u0 = (U * blockIdx.x) / G, u1 = (U * (blockIdx.x + 1)) / G;
+    const int n_units = (int)(u1 - u0);
+    const int g_first = (int)(u0 / p.KSU), q_first = (int)(u0 - (int64_t)g_first * p.KSU);
+
+    // loads of the CTA's unit i (row group g, unit q of the group) into stage i % XS
+    auto issue = [&](int i, int g, int q) {
+        const int s = i % XS;
+        const uint32_t st = base + (uint32_t)(s * S::STAGE);
+        if (p.inject) return;
+        issued[s] += 1;
+        if (q < QW) {
+            const int nb = min(4, p.KB - 4 * q);
+            mbar_arrive_expect_tx(full(s), (uint32_t)(S::CODE_BYTES + nb * S::X_TILE));
+            tma_load_2d(st, &p.tmCodes, full(s), q * 128, g * UROWS);
+            for (int c = 0; c < nb; ++c)
+                tma_load_2d(st + (uint32_t)(S::CODE_BYTES + c * S::X_TILE), &p.tmX, full(s), (4 * q + c) * 64, 0);
+        } else {
+            const int ql = q - QW;
+            const int nb = min(4, p.lora_ks - 4 * ql);
+            const int ucol = p.seg_rows ? ((g * UROWS) / p.seg_rows) * p.r : 0;
+            mbar_arrive_expect_tx(full(s), (uint32_t)(nb * S::X_TILE));
+            for (int c = 0; c < nb; ++c)
+                tma_load_2d(st + (uint32_t)(S::CODE_BYTES + c * S::X_TILE), &p.tmU, full(s),
+                            (4 * ql + c) * 64 + ucol, 0);
+        }
+    };
+    if (threadIdx.x == 0) {
+        int g = g_first, q = q_first;
+        for (int i = 0; i < XS && i < n_units; ++i) {
+            issue(i, g, q);
+            if (++q == p.KSU) { q = 0; ++g; }
+        }
+    }
+
+    const uint32_t lane4 = (uint32_t)lane * 4u;
+    float* scr = reinterpret_cast<float*>(gb + S::OFF_SC) + warp * 2 * SROWS;  // [2][SROWS]
     const float off = p.dq ? __ldg(p.offset) : 0.0f;
 
-    const int G = gridDim.x * S::WARPS;
-    const int w = blockIdx.x * S::WARPS + warp;
-    const int64_t I = p.items;
-    const int64_t i0 = (I * w) / G, i1 = (I * (w + 1)) / G;
-    const int64_t rowb = p.K / 2;  // code bytes per weight row
-    constexpr int QB = S::QB;
-
-    // code bytes (8 per row and block: this thread's quarter of each 32-byte
-    // block chunk) and 8-bit block codes of one weight item, loaded one item
-    // ahead of its use
+    // raw block constant of row `lane` of the warp's slice (lanes < SROWS)
+    // for its block of unit (g, q), loaded one unit ahead of its use
     struct Pf {
-        uint2 cw[R][2][QB];
-        uint32_t q8[R][2];  // QB block codes, byte j = block j
+        int q;    // 8-bit code (double quantization) or 0; -1: a' = 0
+        float c;  // c1 or absmax
     };
-    auto prefetch = [&](int64_t item, Pf& f) {
-        const int g = (int)(item / p.GL), kq = (int)(item - (int64_t)g * p.GL);
-        if (kq >= p.QW) return;  // LoRA item: nothing to fetch ahead
-        const int n0 = g * GROWS;
-#pragma unroll
-        for (int rt = 0; rt < R; ++rt)
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int n = n0 + 16 * rt + gid + 8 * h;
-                uint32_t q = 0;
-#pragma unroll
-                for (int j = 0; j < QB; ++j) {
-                    const int kb = kq * QB + j;
-                    if (n < p.N && kb < p.KB) {
-                        f.cw[rt][h][j] = __ldcs(reinterpret_cast<const uint2*>(p.codes + (int64_t)n * rowb + kb * 32 + 8 * tig));
-                        if (p.dq) q |= (uint32_t)__ldg(p.q8 + (((int64_t)n * p.KB + kb) >> p.fmt.bs_shift)) << (8 * j);
-                    } else {
-                        f.cw[rt][h][j] = make_uint2(0u, 0u);
-                    }
-                }
-                f.q8[rt][h] = q;
+    auto fetch = [&](int g, int q, bool valid) {
+        Pf f{-1, 0.0f};
+        const int kb = 4 * q + bq;
+        if (!valid || q >= QW || kb >= p.KB || lane >= SROWS) return f;
+        const int n = g * UROWS + slice * SROWS + lane;
+        if (n < p.N) {
+            const int64_t b = ((int64_t)n * p.KB + kb) >> p.fmt.bs_shift;
+            if (p.dq) {
+                f.q = __ldg(p.q8 + b);
+                f.c = __ldg(p.c1 + (b >> 8));
+            } else {
+                f.q = 0;
+                f.c = __ldg(p.absmax + b);
             }
+        }
+        return f;
     };
 
-    float acc[R][NT8][4];
+    float acc[RT][MT][4];
 #pragma unroll
-    for (int a = 0; a < R; ++a)
+    for (int j = 0; j < RT; ++j)
 #pragma unroll
-        for (int b = 0; b < NT8; ++b)
+        for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-            for (int c = 0; c < 4; ++c) acc[a][b][c] = 0.0f;
-    Pf cur, nxt;
-    if (i0 < i1) prefetch(i0, cur);
-    for (int64_t it = i0; it < i1; ++it) {
-        if (it + 1 < i1) prefetch(it + 1, nxt);
-        const int g = (int)(it / p.GL);
-        const int kq = (int)(it - (int64_t)g * p.GL);
-        const int n0 = g * GROWS;
-        if (kq < p.QW) {
-            // ------------------------------------------------------ weight item: QB blocks
+            for (int e = 0; e < 4; ++e) acc[j][mt][e] = 0.0f;
+    bool dead = false;
+
+    // end of this CTA's segment of row group g (its last unit u).  Every warp
+    // comes here, also after a wait ran out, so that the slice's named
+    // barriers are always met.  The four block warps of the slice add their
+    // accumulators in block order; the slice's first warp then writes Y, or
+    // publishes the partial and lets the last contributor finish the rows.
+    auto finish_group = [&](int g, int64_t u) {
+        float* mx = xch + (int64_t)warp * (RT * MT * 4 * 32);
+        if (bq != 0) {
 #pragma unroll
-            for (int j = 0; j < QB; ++j) {
-                const int kb = kq * QB + j;
-                if (kb >= p.KB) break;
-                uint32_t xf[NT8][8];
+            for (int j = 0; j < RT; ++j)
 #pragma unroll
-                for (int nt = 0; nt < NT8; ++nt) {
-                    const int m = nt * 8 + gid;
-                    if (m < p.M) {
-                        const uint4* src = reinterpret_cast<const uint4*>(p.X + (int64_t)m * p.K + kb * 64 + 16 * tig);
-                        const uint4 u0 = __ldg(src), u1 = __ldg(src + 1);
-                        xf[nt][0] = u0.x; xf[nt][1] = u0.y; xf[nt][2] = u0.z; xf[nt][3] = u0.w;
-                        xf[nt][4] = u1.x; xf[nt][5] = u1.y; xf[nt][6] = u1.z; xf[nt][7] = u1.w;
-                    } else {
+                for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) xf[nt][q] = 0u;
-                    }
-                }
+                    for (int e = 0; e < 4; ++e) mx[((j * MT + mt) * 4 + e) * 32 + lane] = acc[j][mt][e];
+        }
+        named_sync(1 + slice, 128);
+        if (bq == 0) {
 #pragma unroll
-                for (int rt = 0; rt < R; ++rt) {
-                    float sc[2];
+            for (int w = 1; w < 4; ++w) {
+                const float* ox = xch + (int64_t)(warp + w) * (RT * MT * 4 * 32);
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int n = n0 + 16 * rt + gid + 8 * h;
-                        float a = 0.0f;
-                        if (n < p.N) {
-                            const int64_t b = ((int64_t)n * p.KB + kb) >> p.fmt.bs_shift;
-                            a = p.dq ? __fadd_rn(__fmul_rn(lds_f32(t8s + 4u * ((cur.q8[rt][h] >> (8 * j)) & 0xFFu)),
-                                                           __ldg(p.c1 + (b >> 8))), off)
-                                     : __ldg(p.absmax + b);
+                for (int j = 0; j < RT; ++j)
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            acc[j][mt][e] = __fadd_rn(acc[j][mt][e], ox[((j * MT + mt) * 4 + e) * 32 + lane]);
+            }
+        }
+        named_sync(1 + slice, 128);  // the exchange buffers are free again
+        if (bq == 0 && !*abort_flag) {
+            const int64_t gstart = (int64_t)g * p.KSU;
+            const bool whole = u0 <= gstart && u == gstart + p.KSU - 1;
+            const int nsl = g * UROWS + slice * SROWS;
+            bool write_y = whole;
+            if (!whole) {
+                const int slot = u0 >= gstart ? 0 : 1;  // the CTA's first segment uses slot 0
+                float* mine = p.part + (((int64_t)blockIdx.x * 2 + slot) * 4 + slice) * S::PART_FLOATS;
+#pragma unroll
+                for (int j = 0; j < RT; ++j)
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            __stcg(mine + (8 * j + 2 * tig + (e & 1)) * TOK + 16 * mt + gid + 8 * (e >> 1),
+                                   acc[j][mt][e]);
+                __threadfence();
+                __syncwarp();
+                // contributors: the CTAs from the one holding the group's first
+                // unit to the one holding its last, less any with an empty share
+                const int cf = owner_cta(gstart, U, G), cl = owner_cta(gstart + p.KSU - 1, U, G);
+                uint32_t ncontrib = 0;
+                for (int c = cf; c <= cl; ++c) ncontrib += ((U * c) / G < (U * (c + 1)) / G) ? 1u : 0u;
+                uint32_t before = 0;
+                if (lane == 0) {
+                    // arrivals of this launch (epoch in the high word; a value of
+                    // another epoch counts as none)
+                    unsigned long long* ctr = p.counters + (int64_t)g * 4 + slice;
+                    unsigned long long cv = *reinterpret_cast<volatile unsigned long long*>(ctr);
+                    const unsigned long long ep = (unsigned long long)p.epoch << 32;
+                    while (true) {
+                        const bool same = (cv & 0xFFFFFFFF00000000ull) == ep;
+                        const unsigned long long want = same ? cv + 1ull : (ep | 1ull);
+                        const unsigned long long prev = atomicCAS(ctr, cv, want);
+                        if (prev == cv) {
+                            before = same ? (uint32_t)(cv & 0xFFFFFFFFull) : 0u;
+                            break;
                         }
-                        sc[h] = __fmul_rn(a, p.inv_scale);
+                        cv = prev;
                     }
-                    float d[NT8][4];
+                    if (before + 1 == ncontrib) *ctr = 0ull;  // last arrival: reset for the next launch
+                }
+                before = __shfl_sync(0xffffffffu, before, 0);
+                if (before + 1 == ncontrib) {
+                    __threadfence();
 #pragma unroll
-                    for (int nt = 0; nt < NT8; ++nt)
+                    for (int j = 0; j < RT; ++j)
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) d[nt][q] = 0.0f;
-                    const uint32_t g0x = cur.cw[rt][0][j].x, g0y = cur.cw[rt][0][j].y;
-                    const uint32_t g8x = cur.cw[rt][1][j].x, g8y = cur.cw[rt][1][j].y;
-                    {   // chunk 0: bytes 0, 1
-                        const uint32_t a0 = lut<0>(g0x, lane_base), a2 = lut<1>(g0x, lane_base);
-                        const uint32_t a1 = lut<0>(g8x, lane_base), a3 = lut<1>(g8x, lane_base);
+                        for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-                        for (int nt = 0; nt < NT8; ++nt) mma_16816(d[nt], a0, a1, a2, a3, xf[nt][0], xf[nt][1]);
+                            for (int e = 0; e < 4; ++e) acc[j][mt][e] = 0.0f;
+                    for (int c = cf; c <= cl; ++c) {
+                        if ((U * c) / G == (U * (c + 1)) / G) continue;
+                        const int cslot = (U * c) / G >= gstart ? 0 : 1;
+                        const float* src = p.part + (((int64_t)c * 2 + cslot) * 4 + slice) * S::PART_FLOATS;
+#pragma unroll
+                        for (int j = 0; j < RT; ++j)
+#pragma unroll
+                            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                                for (int e = 0; e < 4; ++e)
+                                    acc[j][mt][e] = __fadd_rn(
+                                        acc[j][mt][e],
+                                        __ldcg(src + (8 * j + 2 * tig + (e & 1)) * TOK + 16 * mt + gid + 8 * (e >> 1)));
                     }
-                    {   // chunk 1: bytes 2, 3
-                        const uint32_t a0 = lut<2>(g0x, lane_base), a2 = lut<3>(g0x, lane_base);
-                        const uint32_t a1 = lut<2>(g8x, lane_base), a3 = lut<3>(g8x, lane_base);
-#pragma unroll
-                        for (int nt = 0; nt < NT8; ++nt) mma_16816(d[nt], a0, a1, a2, a3, xf[nt][2], xf[nt][3]);
-                    }
-                    {   // chunk 2: bytes 4, 5
-                        const uint32_t a0 = lut<0>(g0y, lane_base), a2 = lut<1>(g0y, lane_base);
-                        const uint32_t a1 = lut<0>(g8y, lane_base), a3 = lut<1>(g8y, lane_base);
-#pragma unroll
-                        for (int nt = 0; nt < NT8; ++nt) mma_16816(d[nt], a0, a1, a2, a3, xf[nt][4], xf[nt][5]);
-                    }
-                    {   // chunk 3: bytes 6, 7
-                        const uint32_t a0 = lut<2>(g0y, lane_base), a2 = lut<3>(g0y, lane_base);
-                        const uint32_t a1 = lut<2>(g8y, lane_base), a3 = lut<3>(g8y, lane_base);
-#pragma unroll
-                        for (int nt = 0; nt < NT8; ++nt) mma_16816(d[nt], a0, a1, a2, a3, xf[nt][6], xf[nt][7]);
-                    }
-#pragma unroll
-                    for (int nt = 0; nt < NT8; ++nt) {
-                        acc[rt][nt][0] = __fmaf_rn(sc[0], d[nt][0], acc[rt][nt][0]);
-                        acc[rt][nt][1] = __fmaf_rn(sc[0], d[nt][1], acc[rt][nt][1]);
-                        acc[rt][nt][2] = __fmaf_rn(sc[1], d[nt][2], acc[rt][nt][2]);
-                        acc[rt][nt][3] = __fmaf_rn(sc[1], d[nt][3], acc[rt][nt][3]);
-                    }
+                    write_y = true;
                 }
             }
-        } else {
-            // ------------------------------------------------------ LoRA item: 64 adapter columns, B rows x sU
-            const int j0 = (kq - p.QW) * 64 + 16 * tig;  // adapter column of this thread's 16
-            const bool v0 = j0 + 8 <= p.r, v1 = j0 + 16 <= p.r;
-            const int ucol = (p.seg_rows ? (n0 / p.seg_rows) * p.r : 0) + j0;
-            uint32_t xf[NT8][8];
+            if (write_y) {
 #pragma unroll
-            for (int nt = 0; nt < NT8; ++nt) {
-                const int m = nt * 8 + gid;
-                uint4 u0 = make_uint4(0, 0, 0, 0), u1 = make_uint4(0, 0, 0, 0);
-                if (m < p.M) {
-                    const uint4* src = reinterpret_cast<const uint4*>(p.sU + (int64_t)m * p.rt + ucol);
-                    if (v0) u0 = __ldg(src);
-                    if (v1) u1 = __ldg(src + 1);
+                for (int j = 0; j < RT; ++j) {
+                    const int n = nsl + 8 * j + 2 * tig;
+                    if (n >= p.N) continue;
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const int m = 16 * mt + gid + 8 * h;
+                            if (m >= p.M) continue;
+                            const uint32_t v = pack_bf16x2(acc[j][mt][2 * h], acc[j][mt][2 * h + 1]);
+                            uint16_t* dst = p.Y + (int64_t)m * p.N + n;
+                            if (n + 1 < p.N && ((reinterpret_cast<uintptr_t>(dst) & 3u) == 0)) {
+                                *reinterpret_cast<uint32_t*>(dst) = v;
+                            } else {
+                                dst[0] = (uint16_t)(v & 0xFFFFu);
+                                if (n + 1 < p.N) dst[1] = (uint16_t)(v >> 16);
+                            }
+                        }
                 }
-                xf[nt][0] = u0.x; xf[nt][1] = u0.y; xf[nt][2] = u0.z; xf[nt][3] = u0.w;
-                xf[nt][4] = u1.x; xf[nt][5] = u1.y; xf[nt][6] = u1.z; xf[nt][7] = u1.w;
             }
+        }
 #pragma unroll
-            for (int rt = 0; rt < R; ++rt) {
-                uint32_t bw[2][8];
+        for (int j = 0; j < RT; ++j)
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int n = n0 + 16 * rt + gid + 8 * h;
-                    uint4 u0 = make_uint4(0, 0, 0, 0), u1 = make_uint4(0, 0, 0, 0);
+            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[j][mt][e] = 0.0f;
+    };
+
+    int g = g_first, q = q_first;
+    Pf cur = fetch(g, q, n_units > 0);
+    for (int i = 0; i < n_units; ++i) {
+        const int s = i % XS;
+        const int64_t u = u0 + i;
+        const int nsl = g * UROWS + slice * SROWS;  // first row of this warp's slice
+        // the next unit's block constants
+        int gn = g, qn = q + 1;
+        if (qn == p.KSU) { qn = 0; ++gn; }
+        const Pf nxt = fetch(gn, qn, i + 1 < n_units);
+        if (!dead && !mbar_wait(full(s), (i / XS) & 1, wc)) {
+            *abort_flag = 1;
+            dead = true;
+        }
+        const bool wunit = q < QW;
+        const int kb = 4 * q + bq, jb = 4 * (q - QW) + bq;  // this warp's weight or adapter block
+        // a warp whose rows all lie past the weight, or whose block lies past
+        // K or r, only releases the stage
+        if (!dead && nsl < p.N && (wunit ? kb < p.KB : jb < p.lora_ks)) {
+            const uint32_t st = base + (uint32_t)(s * S::STAGE);
+            const uint32_t xs = st + (uint32_t)(S::CODE_BYTES + bq * S::X_TILE);
+            // X (or sU) fragments: tokens gid + 8 q, physical elements
+            // 16 tig .. 16 tig + 15 of the block (128-byte swizzled rows)
+            uint32_t xf[2 * MT][8];
+#pragma unroll
+            for (int qq = 0; qq < 2 * MT; ++qq) {
+                const int row = gid + 8 * qq;
+                const uint32_t rb = xs + (uint32_t)row * 128u;
+                const uint4 v0 = ld_shared_v4(rb + ((uint32_t)((2 * tig) ^ (row & 7)) << 4));
+                const uint4 v1 = ld_shared_v4(rb + ((uint32_t)((2 * tig + 1) ^ (row & 7)) << 4));
+                xf[qq][0] = v0.x; xf[qq][1] = v0.y; xf[qq][2] = v0.z; xf[qq][3] = v0.w;
+                xf[qq][4] = v1.x; xf[qq][5] = v1.y; xf[qq][6] = v1.z; xf[qq][7] = v1.w;
+            }
+            if (wunit) {
+                // -------------------------------------------------- weight block
+                float* sc = scr + (i & 1) * SROWS;
+                if (lane < SROWS) {
+                    float a = 0.0f;
+                    if (cur.q >= 0) a = p.dq ? __fadd_rn(__fmul_rn(t8s[cur.q], cur.c), off) : cur.c;
+                    sc[lane] = __fmul_rn(a, p.inv_scale);
+                }
+                __syncwarp();
+                // codes of unit row r = slice * SROWS + 8 j + gid: bytes
+                // 32 bq + 8 tig .. + 7 of its 128-byte line (128-byte swizzle)
+                uint32_t cw[RT][2];
+#pragma unroll
+                for (int j = 0; j < RT; ++j) {
+                    const int r = slice * SROWS + 8 * j + gid;
+                    const uint32_t chunk = (uint32_t)((2 * bq + (tig >> 1)) ^ (r & 7));
+                    const uint2 v = ld_shared_v2(st + (uint32_t)r * 128u + (chunk << 4) + (uint32_t)(tig & 1) * 8u);
+                    cw[j][0] = v.x;
+                    cw[j][1] = v.y;
+                }
+                // chunk by chunk over all row tiles: RT independent MMA chains
+                float d[RT][MT][4];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t b0[RT], b1[RT];
+#pragma unroll
+                    for (int j = 0; j < RT; ++j) {
+                        b0[j] = lut_byte(cw[j][c >> 1], 2 * (c & 1), lane4);
+                        b1[j] = lut_byte(cw[j][c >> 1], 2 * (c & 1) + 1, lane4);
+                    }
+#pragma unroll
+                    for (int j = 0; j < RT; ++j)
+#pragma unroll
+                        for (int mt = 0; mt < MT; ++mt) {
+                            if (c == 0)
+                                mma_16816_z(d[j][mt], xf[2 * mt][0], xf[2 * mt + 1][0], xf[2 * mt][1],
+                                            xf[2 * mt + 1][1], b0[j], b1[j]);
+                            else
+                                mma_16816(d[j][mt], xf[2 * mt][2 * c], xf[2 * mt + 1][2 * c], xf[2 * mt][2 * c + 1],
+                                          xf[2 * mt + 1][2 * c + 1], b0[j], b1[j]);
+                        }
+                }
+#pragma unroll
+                for (int j = 0; j < RT; ++j) {
+                    const float2 sj = *reinterpret_cast<const float2*>(sc + 8 * j + 2 * tig);
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) {
+                        acc[j][mt][0] = __fmaf_rn(sj.x, d[j][mt][0], acc[j][mt][0]);
+                        acc[j][mt][1] = __fmaf_rn(sj.y, d[j][mt][1], acc[j][mt][1]);
+                        acc[j][mt][2] = __fmaf_rn(sj.x, d[j][mt][2], acc[j][mt][2]);
+                        acc[j][mt][3] = __fmaf_rn(sj.y, d[j][mt][3], acc[j][mt][3]);
+                    }
+                }
+                // the adapter rows of the group into L2 a few units before their use
+                if (p.lora_ks && q == max(QW - 2, 0) && bq == 0 && lane < SROWS) {
+                    const int n = nsl + lane;
+                    if (n < p.N)
+                        for (int c = 0; c < p.r * 2; c += 128)
+                            asm volatile("prefetch.global.L2 [%0];" ::"l"(
+                                reinterpret_cast<const uint8_t*>(p.B + (int64_t)n * p.r) + c));
+                }
+            } else {
+                // -------------------------------------------------- adapter block: B rows x sU
+                const int j0 = jb * 64 + 16 * tig;  // adapter column of this lane's 16
+                const bool v0 = j0 + 8 <= p.r, v1 = j0 + 16 <= p.r;
+                uint4 bw[RT][2];
+#pragma unroll
+                for (int j = 0; j < RT; ++j) {
+                    const int n = nsl + 8 * j + gid;
+                    bw[j][0] = make_uint4(0, 0, 0, 0);
+                    bw[j][1] = make_uint4(0, 0, 0, 0);
                     if (n < p.N) {
                         const uint4* src = reinterpret_cast<const uint4*>(p.B + (int64_t)n * p.r + j0);
-                        if (v0) u0 = __ldg(src);
-                        if (v1) u1 = __ldg(src + 1);
+                        if (v0) bw[j][0] = __ldg(src);
+                        if (v1) bw[j][1] = __ldg(src + 1);
                     }
-                    bw[h][0] = u0.x; bw[h][1] = u0.y; bw[h][2] = u0.z; bw[h][3] = u0.w;
-                    bw[h][4] = u1.x; bw[h][5] = u1.y; bw[h][6] = u1.z; bw[h][7] = u1.w;
                 }
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
 #pragma unroll
-                    for (int nt = 0; nt < NT8; ++nt)
-                        mma_16816(acc[rt][nt], bw[0][2 * c], bw[1][2 * c], bw[0][2 * c + 1], bw[1][2 * c + 1],
-                                  xf[nt][2 * c], xf[nt][2 * c + 1]);
-            }
-        }
-        cur = nxt;
-
-        // ---------------------------------------------------------- end of a segment: output
-        if (it + 1 < i1 && kq + 1 < p.GL) continue;
-        const int64_t gstart = (int64_t)g * p.GL;
-        const int64_t seg0 = i0 > gstart ? i0 : gstart;
-        const bool whole = seg0 == gstart && kq + 1 == p.GL;
-        bool write_y = whole;
-        if (!whole) {
-            const int slot = seg0 > gstart ? 0 : (i0 < gstart ? 1 : 0);
-            float* mine = p.part + ((int64_t)w * 2 + slot) * (GROWS * NPAD);
+                    for (int j = 0; j < RT; ++j) {
+                        const uint4 h = bw[j][c >> 1];
+                        const uint32_t w0 = (c & 1) ? h.z : h.x, w1 = (c & 1) ? h.w : h.y;
 #pragma unroll
-            for (int rt = 0; rt < R; ++rt)
-#pragma unroll
-                for (int nt = 0; nt < NT8; ++nt)
-#pragma unroll
-                    for (int h = 0; h < 2; ++h)
-                        __stcg(reinterpret_cast<float2*>(mine + (16 * rt + gid + 8 * h) * NPAD + nt * 8 + 2 * tig),
-                               make_float2(acc[rt][nt][2 * h], acc[rt][nt][2 * h + 1]));
-            __threadfence();
-            __syncwarp();
-            // contributors: the warps from the one holding the group's first
-            // item to the one holding its last, less any with an empty share
-            const int wf = owner_warp(gstart, I, G), wl = owner_warp(gstart + p.GL - 1, I, G);
-            uint32_t ncontrib = 0;
-            for (int c = wf; c <= wl; ++c) ncontrib += ((I * c) / G < (I * (c + 1)) / G) ? 1u : 0u;
-            // arrivals of this launch at the group's counter (epoch in the high bits)
-            uint32_t before = 0;
-            if (lane == 0) {
-                uint32_t* ctr = p.counters + g;
-                uint32_t cv = *reinterpret_cast<volatile uint32_t*>(ctr);
-                while (true) {
-                    const bool same = (cv >> 8) == p.epoch;
-                    const uint32_t want = same ? cv + 1u : ((p.epoch << 8) | 1u);
-                    const uint32_t prev = atomicCAS(ctr, cv, want);
-                    if (prev == cv) {
-                        before = same ? (cv & 0xFFu) : 0u;
-                        break;
+                        for (int mt = 0; mt < MT; ++mt)
+                            mma_16816(acc[j][mt], xf[2 * mt][2 * c], xf[2 * mt + 1][2 * c], xf[2 * mt][2 * c + 1],
+                                      xf[2 * mt + 1][2 * c + 1], w0, w1);
                     }
-                    cv = prev;
-                }
-                if (before + 1 == ncontrib) *ctr = 0u;  // last arrival: reset for the next launch
-            }
-            before = __shfl_sync(0xffffffffu, before, 0);
-            if (before + 1 == ncontrib) {
-                __threadfence();
-                // add every contributor's partial in warp order
-#pragma unroll
-                for (int rt = 0; rt < R; ++rt)
-#pragma unroll
-                    for (int nt = 0; nt < NT8; ++nt)
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) acc[rt][nt][q] = 0.0f;
-                for (int c = wf; c <= wl; ++c) {
-                    if ((I * c) / G == (I * (c + 1)) / G) continue;
-                    const int cslot = ((I * c) / G < gstart) ? 1 : 0;
-                    const float* src = p.part + ((int64_t)c * 2 + cslot) * (GROWS * NPAD);
-#pragma unroll
-                    for (int rt = 0; rt < R; ++rt)
-#pragma unroll
-                        for (int nt = 0; nt < NT8; ++nt)
-#pragma unroll
-                            for (int h = 0; h < 2; ++h) {
-                                const float2 v = __ldcg(reinterpret_cast<const float2*>(
-                                    src + (16 * rt + gid + 8 * h) * NPAD + nt * 8 + 2 * tig));
-                                acc[rt][nt][2 * h] = __fadd_rn(acc[rt][nt][2 * h], v.x);
-                                acc[rt][nt][2 * h + 1] = __fadd_rn(acc[rt][nt][2 * h + 1], v.y);
-                            }
-                }
-                write_y = true;
             }
         }
-        if (write_y) {
-#pragma unroll
-            for (int rt = 0; rt < R; ++rt)
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int n = n0 + 16 * rt + gid + 8 * h;
-                    if (n >= p.N) continue;
-#pragma unroll
-                    for (int nt = 0; nt < NT8; ++nt)
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int m = nt * 8 + 2 * tig + e;
-                            if (m < p.M)
-                                p.Y[(int64_t)m * p.N + n] = (uint16_t)(pack_bf16x2(acc[rt][nt][2 * h + e], 0.0f) & 0xFFFFu);
-                        }
+        if (!dead) {
+            // release the stage; the last warp to do so loads unit i + XS into it
+            __syncwarp();
+            if (lane == 0) {
+                __threadfence_block();
+                if (atomicAdd(&done[s], 1) == WARPS - 1) {
+                    done[s] = 0;
+                    if (i + XS < n_units && !*abort_flag) {
+                        // the other warps' reads of the stage are ordered
+                        // before this thread's async-proxy writes
+                        __threadfence_block();
+                        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                        int gi = g, qi = q + XS;
+                        while (qi >= p.KSU) { qi -= p.KSU; ++gi; }
+                        issue(i + XS, gi, qi);
+                    }
                 }
+            }
         }
-#pragma unroll
-        for (int a = 0; a < R; ++a)
-#pragma unroll
-            for (int b = 0; b < NT8; ++b)
-#pragma unroll
-                for (int c = 0; c < 4; ++c) acc[a][b][c] = 0.0f;
+        if (q == p.KSU - 1 || i == n_units - 1) finish_group(g, u);
+        cur = nxt;
+        g = gn;
+        q = qn;
     }
+    // every load issued into the ring has landed before the CTA exits
+    __syncthreads();
+    if (threadIdx.x == 0)
+        for (int s = 0; s < XS; ++s)
+            if (issued[s] > 0) mbar_wait(full(s), (issued[s] - 1) & 1, wc);
 }
 
 }  // namespace qlora

@@ -385,9 +385,11 @@ void qlora_set_wait_timeout_ns(uint64_t ns);
  * dA and dB GEMMs on the caller's stream after the dX GEMM instead of beside
  * it on the library's side stream; mode 7 runs the forward for M <= 32 on the
  * register-fed warp-MMA kernel (code-byte table lookups, block constant on
- * each block's fp32 partial) instead of the tcgen05 small-M kernel.
+ * each block's fp32 partial), mode 8 the forward for M <= 16 on the tcgen05
+ * small-M kernel.
  * Mode 0: normal (CTA-pair kernel, one pair per tile; in the backward the
- * dA/dB GEMMs beside the dX GEMM on the side stream).
+ * dA/dB GEMMs beside the dX GEMM on the side stream; M <= 16 on the warp-MMA
+ * kernel, 17 <= M <= 64 on the tcgen05 small-M kernel).
  * The mode is process-wide: it changes the kernels of every later call from
  * every thread and stream on every device, until it is set back to 0; it is
  * meant for tests only.  Likewise the environment variable QLORA_SCHEDULE

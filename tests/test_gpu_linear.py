@@ -300,11 +300,12 @@ def test_small_m_graph_replay(Q, O, cuda):
     assert Q.qlora_get_last_error() == 0
 
 
-def test_small_m_timeout_is_reported_and_recovers(Q, O, cuda):
-    """Failure detection on the tcgen05 small-M kernel: skipped loads make
-    the bounded waits run out, TIMEOUT is reported, the next call is
-    correct.  (The warp-MMA kernel of test mode 7 has no waits.)"""
-    M, N, K, r = 16, 1024, 1024, 16
+@pytest.mark.parametrize("M", [16, 24])
+def test_small_m_timeout_is_reported_and_recovers(Q, O, cuda, M):
+    """Failure detection on the small-M kernels (M = 16: the warp-MMA kernel,
+    M = 24: the tcgen05 kernel): skipped loads make the bounded waits run
+    out, TIMEOUT is reported, the next call is correct."""
+    N, K, r = 1024, 1024, 16
     q, inp, Wd_ref = _setup(Q, O, M, N, K, r, seed=9)
     X, A, B = inp["X"].cuda(), inp["A"].cuda(), inp["B"].cuda()
     Q.qlora_get_last_error()
@@ -321,20 +322,40 @@ def test_small_m_timeout_is_reported_and_recovers(Q, O, cuda):
     assert_close_tol(got, ref, "Y after recovery")
 
 
-@pytest.mark.parametrize("M,N,K,r,nseg", [(1, 256, 128, 8, 1), (3, 1000, 512, 64, 1), (8, 22016, 8192, 64, 1),
-                                          (16, 4096, 8192, 64, 1), (17, 384, 256, 128, 1), (32, 2048, 4096, 32, 1),
-                                          (16, 3 * 1024, 2048, 32, 3), (5, 2000, 2048, 64, 1)])
-def test_small_m_warp_mma_kernel(Q, O, cuda, M, N, K, r, nseg):
+@pytest.mark.parametrize("M,N,K,r", [(1, 768, 1024, 16), (5, 2000, 2048, 64), (16, 4096, 8192, 64)])
+def test_small_m_tcgen05_kernel_for_few_tokens(Q, O, cuda, M, N, K, r):
+    """Test mode 8: the tcgen05 small-M kernel (bit-exact bf16 weight tiles)
+    for M <= 16, where the default is the warp-MMA kernel."""
+    q, inp, Wd_ref = _setup(Q, O, M, N, K, r, seed=91)
+    Q.qlora_debug_inject(8)
+    try:
+        got, ref = _fwd_both(Q, O, q, inp, Wd_ref, 2.0, r)
+        torch.cuda.synchronize()
+        assert Q.qlora_get_last_error() == 0
+    finally:
+        Q.qlora_debug_inject(0)
+    assert_close_tol(got, ref, f"Y tcgen05 M={M}")
+
+
+@pytest.mark.parametrize("M,N,K,r,nseg,dq", [(1, 256, 128, 8, 1, True), (3, 1000, 512, 64, 1, True),
+                                             (8, 22016, 8192, 64, 1, True), (16, 4096, 8192, 64, 1, True),
+                                             (17, 384, 256, 128, 1, True), (32, 2048, 4096, 32, 1, True),
+                                             (16, 3 * 1024, 2048, 32, 3, True), (5, 2000, 2048, 64, 1, True),
+                                             (16, 2 * 768, 1024, 16, 2, True), (24, 3 * 768, 1024, 16, 3, True),
+                                             (12, 1000, 1024, 24, 1, False), (30, 520, 640, 40, 1, False)])
+def test_small_m_warp_mma_kernel(Q, O, cuda, M, N, K, r, nseg, dq):
     """The register-fed warp-MMA small-M kernel (test mode 7: block constant
     applied to each 64-element block's fp32 partial, bf16 table values times
-    a fixed prescale) against the oracle; the fused projection case checks
-    its segment columns of sU."""
+    a fixed prescale) against the oracle; the fused projection cases check
+    its segment columns of sU, also where one 512-row group spans two
+    adapters (segments of 768 rows); two cases without double quantization
+    and with a partial last adapter tile (r = 24, 40)."""
     S = N // nseg
     W = wl.weight(N, K, seed=90, dtype=torch.bfloat16)
     inp = wl.fused_inputs(M, nseg, S, K, r, seed=90, b_std=0.05)
-    q = Q.qlora_nf4_quantize(W.cuda())
-    ref_q = O.nf4_quantize(wl.bits(W).reshape(-1))
-    Wd = O.nf4_dequantize(N * K, ref_q).reshape(N, K)
+    q = Q.qlora_nf4_quantize(W.cuda(), double_quant=dq)
+    ref_q = O.nf4_quantize(wl.bits(W).reshape(-1), double_quant=dq)
+    Wd = O.nf4_dequantize(N * K, ref_q, double_quant=dq).reshape(N, K)
     Q.qlora_debug_inject(7)
     try:
         Y = Q.qlora_fused_linear_fwd(inp["X"].cuda(), q, nseg, inp["A"].cuda(), inp["B"].cuda(), 2.0)
