@@ -134,6 +134,12 @@ __global__ void __launch_bounds__(SmallMShape<NT, NG>::THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
+    // Dependent launch: with an adapter the kernel before is the sU GEMM,
+    // which waited for its own predecessors before it let this one start, so
+    // only sU needs the wait (the producer takes it before the first adapter
+    // step).  Without one the kernel before may still be writing any input
+    // (the quantizer, say): every thread waits here.
+    if (p.ks_lora == 0) pdl_wait();
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer

@@ -198,9 +198,13 @@ __global__ void __launch_bounds__(SmallMmaShape<MT>::THREADS, 1)
         if (p.lora_ks) prefetch_tensormap(&p.tmU);
     }
     __syncthreads();
-    // the weight, X and the adapter operands may come from the kernels just
-    // before (the quantizer, the sU GEMM, an earlier layer): wait for them
-    pdl_wait();
+    // Dependent launch.  With an adapter the kernel before this one is the
+    // sU GEMM, which waited for its own predecessors before it let this
+    // kernel start: the codes, block constants and X are final, and only sU
+    // (read by the adapter units' loads) needs the wait, taken by the thread
+    // that issues those loads.  Without one the kernel before may still be
+    // writing any input (the quantizer, say): every thread waits here.
+    if (p.lora_ks == 0) pdl_wait();
 
     const int QW = (p.KB + 3) >> 2;        // weight units per row group
     const int64_t U = p.units;
@@ -222,6 +226,7 @@ __global__ void __launch_bounds__(SmallMmaShape<MT>::THREADS, 1)
             for (int c = 0; c < nb; ++c)
                 tma_load_2d(st + (uint32_t)(S::CODE_BYTES + c * S::X_TILE), &p.tmX, full(s), (4 * q + c) * 64, 0);
         } else {
+            pdl_wait();  // sU comes from the kernel before this one
             const int ql = q - QW;
             const int nb = min(4, p.lora_ks - 4 * ql);
             const int ucol = p.seg_rows ? ((g * UROWS) / p.seg_rows) * p.r : 0;
@@ -552,11 +557,14 @@ __global__ void __launch_bounds__(SmallMmaShape<MT>::THREADS, 1)
         g = gn;
         q = qn;
     }
-    // every load issued into the ring has landed before the CTA exits
+    // every load issued into the ring has landed before the CTA exits, and
+    // the kernel does not complete before the one it depends on
     __syncthreads();
-    if (threadIdx.x == 0)
+    if (threadIdx.x == 0) {
         for (int s = 0; s < XS; ++s)
             if (issued[s] > 0) mbar_wait(full(s), (issued[s] - 1) & 1, wc);
+        pdl_wait();
+    }
 }
 
 }  // namespace qlora
