@@ -79,11 +79,12 @@ struct SmallMmaParams {
 
 template <int MT>
 struct SmallMmaShape {
-    static constexpr int WARPS = 16;              // 4 row slices x 4 blocks of a unit
+    static constexpr int BPW = 2;                 // blocks of a unit per MMA warp
+    static constexpr int WARPS = 16 / BPW;        // MMA warps: 4 row slices x 4 / BPW block groups
     static constexpr int RT = MT == 1 ? 4 : 2;    // 8-row tiles per warp
     static constexpr int SROWS = 8 * RT;          // rows of a slice (32 or 16)
     static constexpr int UROWS = 4 * SROWS;       // rows of a unit (128 or 64)
-    static constexpr int THREADS = 32 * WARPS;
+    static constexpr int THREADS = 32 * (WARPS + 1);  // + the warp that loads the ring
     static constexpr int XS = 6;                  // ring stages
     static constexpr int X_TILE = 16 * MT * 128;  // 16 MT tokens x 64 bf16
     static constexpr int CODE_BYTES = UROWS * 128;  // codes of one unit (128-byte swizzle)
@@ -91,11 +92,11 @@ struct SmallMmaShape {
     // dynamic shared memory (1024-aligned): ring, t8 table, scale scratch,
     // accumulator exchange, barriers and stage counters
     static constexpr int OFF_T8 = XS * STAGE;
-    static constexpr int OFF_SC = OFF_T8 + 1024;                     // [WARPS][2][SROWS] fp32
-    static constexpr int OFF_XCH = OFF_SC + WARPS * 2 * SROWS * 4;  // [WARPS][RT * MT * 4][32] fp32
-    static constexpr int OFF_BAR = OFF_XCH + WARPS * RT * MT * 4 * 32 * 4;  // full[XS]
-    static constexpr int OFF_CNT = OFF_BAR + 8 * XS;                // done[XS], issued[XS], abort flag
-    static constexpr int SMEM = OFF_CNT + 8 * XS + 16 + 1024;       // + alignment slack
+    static constexpr int OFF_SC = OFF_T8 + 1024;                     // [WARPS][2][BPW][SROWS] fp32
+    static constexpr int OFF_XCH = OFF_SC + WARPS * 2 * BPW * SROWS * 4;  // [WARPS][RT * MT * 4][32] fp32
+    static constexpr int OFF_BAR = OFF_XCH + WARPS * RT * MT * 4 * 32 * 4;  // full[XS], empty[XS]
+    static constexpr int OFF_CNT = OFF_BAR + 16 * XS;               // issued[XS], abort flag
+    static constexpr int SMEM = OFF_CNT + 4 * XS + 16 + 1024;       // + alignment slack
     static constexpr int PART_FLOATS = SROWS * 16 * MT;  // one slice's partial tile
 };
 
@@ -146,6 +147,33 @@ __device__ __forceinline__ int owner_cta(int64_t x, int64_t I, int G) {
     return c;
 }
 
+// mbar_wait whose polls suspend the thread for up to hint_ns while the
+// phase is still open (no busy polling that takes issue slots from the MMA
+// warps on the same scheduler).  Gives up after cfg.timeout_ns.
+__device__ __forceinline__ bool mbar_wait_hint(uint32_t bar, uint32_t parity, const WaitCfg& cfg,
+                                               uint32_t hint_ns) {
+    auto poll = [&]() {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity), "r"(hint_ns)
+            : "memory");
+        return ok != 0;
+    };
+    if (poll()) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (!poll()) {
+        if (globaltimer_ns() - t0 > cfg.timeout_ns) {
+            set_status(4);
+            return false;
+        }
+    }
+    return true;
+}
+
 __device__ __forceinline__ void named_sync(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
@@ -164,12 +192,13 @@ __global__ void __launch_bounds__(SmallMmaShape<MT>::THREADS, 1)
     float* xch = reinterpret_cast<float*>(gb + S::OFF_XCH);
     const uint32_t bar = base + S::OFF_BAR;
     auto full = [&](int s) { return bar + 8u * s; };
-    int* done = reinterpret_cast<int*>(gb + S::OFF_CNT);  // warps finished with the stage's unit
-    int* issued = done + XS;                                // loads issued into the stage
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(gb + S::OFF_CNT + 8 * XS);
+    auto empty = [&](int s) { return bar + 8u * (XS + s); };
+    int* issued = reinterpret_cast<int*>(gb + S::OFF_CNT);  // loads issued into the stage
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(gb + S::OFF_CNT + 4 * XS);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gid = lane >> 2, tig = lane & 3;
-    const int slice = warp >> 2, bq = warp & 3;  // row slice and block of a unit
+    constexpr int BPW = S::BPW, WPS = 4 / BPW;   // blocks per warp, warps per slice
+    const int slice = warp / WPS, bpair = warp % WPS;  // row slice; blocks BPW bpair .. + BPW - 1 of a unit
     const WaitCfg wc{p.timeout_ns};
 
     // table: entry e = {L v[e >> 4] (bits 0..15), L v[e & 15] (bits 16..31)}
@@ -187,7 +216,7 @@ __global__ void __launch_bounds__(SmallMmaShape<MT>::THREADS, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < XS; ++s) {
             mbar_init(full(s), 1);
-            done[s] = 0;
+            mbar_init(empty(s), WARPS);
             issued[s] = 0;
         }
         *abort_flag = 0;
@@ -236,37 +265,50 @@ __global__ void __launch_bounds__(SmallMmaShape<MT>::THREADS, 1)
                             (4 * ql + c) * 64 + ucol, 0);
         }
     };
-    if (threadIdx.x == 0) {
-        int g = g_first, q = q_first;
-        for (int i = 0; i < XS && i < n_units; ++i) {
-            issue(i, g, q);
-            if (++q == p.KSU) { q = 0; ++g; }
+    if (warp == WARPS) {
+        // ------------------------------------------------------------ ring loader
+        if (lane == 0) {
+            int g = g_first, q = q_first;
+            for (int i = 0; i < n_units; ++i) {
+                // the MMA warps have released the stage's previous unit
+                if (i >= XS && (*abort_flag || !mbar_wait_hint(empty(i % XS), ((i / XS) - 1) & 1, wc, 2000))) {
+                    *abort_flag = 1;
+                    break;
+                }
+                issue(i, g, q);
+                if (++q == p.KSU) { q = 0; ++g; }
+            }
         }
-    }
+    } else {
 
     const uint32_t lane4 = (uint32_t)lane * 4u;
-    float* scr = reinterpret_cast<float*>(gb + S::OFF_SC) + warp * 2 * SROWS;  // [2][SROWS]
+    float* scr = reinterpret_cast<float*>(gb + S::OFF_SC) + warp * 2 * BPW * SROWS;  // [2][BPW][SROWS]
     const float off = p.dq ? __ldg(p.offset) : 0.0f;
 
-    // raw block constant of row `lane` of the warp's slice (lanes < SROWS)
-    // for its block of unit (g, q), loaded one unit ahead of its use
+    // raw block constants of row `lane` of the warp's slice (lanes < SROWS)
+    // for its blocks of unit (g, q), loaded two units ahead of their use
     struct Pf {
-        int q;    // 8-bit code (double quantization) or 0; -1: a' = 0
-        float c;  // c1 or absmax
+        int q[BPW];    // 8-bit code (double quantization) or 0; -1: a' = 0
+        float c[BPW];  // c1 or absmax
     };
     auto fetch = [&](int g, int q, bool valid) {
-        Pf f{-1, 0.0f};
-        const int kb = 4 * q + bq;
-        if (!valid || q >= QW || kb >= p.KB || lane >= SROWS) return f;
-        const int n = g * UROWS + slice * SROWS + lane;
-        if (n < p.N) {
-            const int64_t b = ((int64_t)n * p.KB + kb) >> p.fmt.bs_shift;
-            if (p.dq) {
-                f.q = __ldg(p.q8 + b);
-                f.c = __ldg(p.c1 + (b >> 8));
-            } else {
-                f.q = 0;
-                f.c = __ldg(p.absmax + b);
+        Pf f;
+#pragma unroll
+        for (int bb = 0; bb < BPW; ++bb) {
+            f.q[bb] = -1;
+            f.c[bb] = 0.0f;
+            const int kb = 4 * q + BPW * bpair + bb;
+            if (!valid || q >= QW || kb >= p.KB || lane >= SROWS) continue;
+            const int n = g * UROWS + slice * SROWS + lane;
+            if (n < p.N) {
+                const int64_t b = ((int64_t)n * p.KB + kb) >> p.fmt.bs_shift;
+                if (p.dq) {
+                    f.q[bb] = __ldg(p.q8 + b);
+                    f.c[bb] = __ldg(p.c1 + (b >> 8));
+                } else {
+                    f.q[bb] = 0;
+                    f.c[bb] = __ldg(p.absmax + b);
+                }
             }
         }
         return f;
@@ -283,12 +325,12 @@ __global__ void __launch_bounds__(SmallMmaShape<MT>::THREADS, 1)
 
     // end of this CTA's segment of row group g (its last unit u).  Every warp
     // comes here, also after a wait ran out, so that the slice's named
-    // barriers are always met.  The four block warps of the slice add their
+    // barriers are always met.  The block warps of the slice add their
     // accumulators in block order; the slice's first warp then writes Y, or
     // publishes the partial and lets the last contributor finish the rows.
     auto finish_group = [&](int g, int64_t u) {
         float* mx = xch + (int64_t)warp * (RT * MT * 4 * 32);
-        if (bq != 0) {
+        if (bpair != 0) {
 #pragma unroll
             for (int j = 0; j < RT; ++j)
 #pragma unroll
@@ -296,10 +338,10 @@ __global__ void __launch_bounds__(SmallMmaShape<MT>::THREADS, 1)
 #pragma unroll
                     for (int e = 0; e < 4; ++e) mx[((j * MT + mt) * 4 + e) * 32 + lane] = acc[j][mt][e];
         }
-        named_sync(1 + slice, 128);
-        if (bq == 0) {
+        named_sync(1 + slice, 32 * WPS);
+        if (bpair == 0) {
 #pragma unroll
-            for (int w = 1; w < 4; ++w) {
+            for (int w = 1; w < WPS; ++w) {
                 const float* ox = xch + (int64_t)(warp + w) * (RT * MT * 4 * 32);
 #pragma unroll
                 for (int j = 0; j < RT; ++j)
@@ -310,8 +352,8 @@ __global__ void __launch_bounds__(SmallMmaShape<MT>::THREADS, 1)
                             acc[j][mt][e] = __fadd_rn(acc[j][mt][e], ox[((j * MT + mt) * 4 + e) * 32 + lane]);
             }
         }
-        named_sync(1 + slice, 128);  // the exchange buffers are free again
-        if (bq == 0 && !*abort_flag) {
+        named_sync(1 + slice, 32 * WPS);  // the exchange buffers are free again
+        if (bpair == 0 && !*abort_flag) {
             const int64_t gstart = (int64_t)g * p.KSU;
             const bool whole = u0 <= gstart && u == gstart + p.KSU - 1;
             const int nsl = g * UROWS + slice * SROWS;
@@ -410,24 +452,26 @@ __global__ void __launch_bounds__(SmallMmaShape<MT>::THREADS, 1)
                 for (int e = 0; e < 4; ++e) acc[j][mt][e] = 0.0f;
     };
 
+    // block constants two units ahead: (g, q) is unit i, (g1, q1) unit i + 1
     int g = g_first, q = q_first;
-    Pf cur = fetch(g, q, n_units > 0);
+    int g1 = g, q1 = q + 1;
+    if (q1 == p.KSU) { q1 = 0; ++g1; }
+    Pf cur = fetch(g, q, n_units > 0), nxt = fetch(g1, q1, n_units > 1);
     for (int i = 0; i < n_units; ++i) {
         const int s = i % XS;
         const int64_t u = u0 + i;
         const int nsl = g * UROWS + slice * SROWS;  // first row of this warp's slice
-        // the next unit's block constants
-        int gn = g, qn = q + 1;
-        if (qn == p.KSU) { qn = 0; ++gn; }
-        const Pf nxt = fetch(gn, qn, i + 1 < n_units);
-        if (!dead && !mbar_wait(full(s), (i / XS) & 1, wc)) {
+        if (!dead && !mbar_wait_hint(full(s), (i / XS) & 1, wc, 1000)) {
             *abort_flag = 1;
             dead = true;
         }
         const bool wunit = q < QW;
+#pragma unroll
+        for (int bb = 0; bb < BPW; ++bb) {
+        const int bq = BPW * bpair + bb;
         const int kb = 4 * q + bq, jb = 4 * (q - QW) + bq;  // this warp's weight or adapter block
         // a warp whose rows all lie past the weight, or whose block lies past
-        // K or r, only releases the stage
+        // K or r, skips the block
         if (!dead && nsl < p.N && (wunit ? kb < p.KB : jb < p.lora_ks)) {
             const uint32_t st = base + (uint32_t)(s * S::STAGE);
             const uint32_t xs = st + (uint32_t)(S::CODE_BYTES + bq * S::X_TILE);
@@ -445,10 +489,10 @@ __global__ void __launch_bounds__(SmallMmaShape<MT>::THREADS, 1)
             }
             if (wunit) {
                 // -------------------------------------------------- weight block
-                float* sc = scr + (i & 1) * SROWS;
+                float* sc = scr + ((i & 1) * BPW + bb) * SROWS;
                 if (lane < SROWS) {
                     float a = 0.0f;
-                    if (cur.q >= 0) a = p.dq ? __fadd_rn(__fmul_rn(t8s[cur.q], cur.c), off) : cur.c;
+                    if (cur.q[bb] >= 0) a = p.dq ? __fadd_rn(__fmul_rn(t8s[cur.q[bb]], cur.c[bb]), off) : cur.c[bb];
                     sc[lane] = __fmul_rn(a, p.inv_scale);
                 }
                 __syncwarp();
@@ -533,29 +577,26 @@ __global__ void __launch_bounds__(SmallMmaShape<MT>::THREADS, 1)
                     }
             }
         }
-        if (!dead) {
-            // release the stage; the last warp to do so loads unit i + XS into it
-            __syncwarp();
-            if (lane == 0) {
-                __threadfence_block();
-                if (atomicAdd(&done[s], 1) == WARPS - 1) {
-                    done[s] = 0;
-                    if (i + XS < n_units && !*abort_flag) {
-                        // the other warps' reads of the stage are ordered
-                        // before this thread's async-proxy writes
-                        __threadfence_block();
-                        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                        int gi = g, qi = q + XS;
-                        while (qi >= p.KSU) { qi -= p.KSU; ++gi; }
-                        issue(i + XS, gi, qi);
-                    }
-                }
-            }
         }
+        if (!dead) {
+            // release the stage to the loader (an arrival with release semantics,
+            // after every lane's reads of it)
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty(s));
+        }
+        // unit i + 2's block constants, issued after the release so that the
+        // arrival does not wait for them
+        int g2 = g1, q2 = q1 + 1;
+        if (q2 == p.KSU) { q2 = 0; ++g2; }
+        const Pf nxt2 = fetch(g2, q2, i + 2 < n_units);
         if (q == p.KSU - 1 || i == n_units - 1) finish_group(g, u);
         cur = nxt;
-        g = gn;
-        q = qn;
+        nxt = nxt2;
+        g = g1;
+        q = q1;
+        g1 = g2;
+        q1 = q2;
+    }
     }
     // every load issued into the ring has landed before the CTA exits, and
     // the kernel does not complete before the one it depends on
