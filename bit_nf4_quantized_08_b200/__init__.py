@@ -6,7 +6,7 @@ quantization of the block constants, as a C-ABI CUDA library
 (``include/qlora_nf4.h``) with a thin torch binding.
 """
 from ._lib import QloraError, QLORA_OK, QLORA_ERR_INVALID_ARG, QLORA_ERR_UNSUPPORTED, \
-    QLORA_ERR_CUDA, QLORA_ERR_TIMEOUT, QLORA_ERR_WORKSPACE, QLORA_STATIC_QUANTIZE_MAX_ELEMS  # noqa: F401
+    QLORA_ERR_CUDA, QLORA_ERR_TIMEOUT, QLORA_ERR_WORKSPACE, QLORA_ERR_BOUNDS, QLORA_STATIC_QUANTIZE_MAX_ELEMS  # noqa: F401
 from .api import (  # noqa: F401
     NF4Weight,
     PagedBuffer,

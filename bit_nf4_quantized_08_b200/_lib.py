@@ -12,7 +12,9 @@ import ctypes
 import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libqlora_nf4.so")
+# QLORA_LIBRARY=debug selects the bounds-checked build (libqlora_nf4_debug.so)
+LIB_PATH = os.path.join(HERE, "libqlora_nf4_debug.so" if os.environ.get("QLORA_LIBRARY") == "debug"
+                        else "libqlora_nf4.so")
 
 QLORA_OK = 0
 QLORA_ERR_INVALID_ARG = 1
@@ -20,7 +22,8 @@ QLORA_ERR_UNSUPPORTED = 2
 QLORA_ERR_CUDA = 3
 QLORA_ERR_TIMEOUT = 4
 QLORA_ERR_WORKSPACE = 5
-STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "TIMEOUT", 5: "WORKSPACE"}
+QLORA_ERR_BOUNDS = 6
+STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "TIMEOUT", 5: "WORKSPACE", 6: "BOUNDS"}
 QLORA_F32 = 0
 QLORA_BF16 = 1
 CODE_TYPES = {"nf4": 0, "fp4": 1}
@@ -108,7 +111,8 @@ def lib() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise RuntimeError(
             f"CUDA library {LIB_PATH} is missing; build it with "
-            "`python -m bit_nf4_quantized_08_b200.build` (there is no CPU fallback)")
+            "`python -m bit_nf4_quantized_08_b200.build` (add --debug for the bounds-checked build; "
+            "there is no CPU fallback)")
     L = ctypes.CDLL(LIB_PATH)
     vp, i64, i32, f32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
     W = ctypes.POINTER(CNF4Weight)

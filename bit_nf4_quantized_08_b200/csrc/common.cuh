@@ -63,6 +63,20 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 
 __device__ __forceinline__ void set_status(int code) { atomicCAS(&g_status, 0, code); }
 
+// Bounds checks of the debug build (compiled with -DQLORA_DEBUG): a failed
+// check records QLORA_ERR_BOUNDS (6) in the status word and the guarded
+// store is skipped; nothing traps.  In the normal build the checks compile
+// to nothing.  Use: if (QLORA_CHECK(index < size)) ptr[index] = value;
+#ifdef QLORA_DEBUG
+__device__ __forceinline__ bool debug_check(bool ok) {
+    if (!ok) set_status(6);
+    return ok;
+}
+#define QLORA_CHECK(cond) (::qlora::debug_check(cond))
+#else
+#define QLORA_CHECK(cond) true
+#endif
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -50,6 +50,8 @@ struct GemmParams {
     // stream-K schedule (persistent grid of gridDim.x CTAs)
     int streamk;
     int tiles_n, tiles_total;
+    int n_in_x;              // pair grid schedule: weight column tiles in blockIdx.x / 2 (only when
+                             // there are more than 65535 of them; else token tiles in x, columns in y)
     float* sk_part;   // [gridDim.x][BM*BN] fp32 partial tiles
     int* sk_flags;    // [gridDim.x], zero before the launch
     // CTA-pair kernel: wait for the previous kernel of the stream only before

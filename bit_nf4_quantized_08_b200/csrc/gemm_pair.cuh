@@ -46,12 +46,17 @@ constexpr int pair_smem_bytes() {
 __device__ __forceinline__ uint32_t sw64(uint32_t off) { return off ^ (((off >> 7) & 3u) << 4); }
 
 // Work of one CTA pair: a list of segments (tile, k-step range).  Grid
-// schedule: one segment, the whole k-range of tile (blockIdx.y, blockIdx.x/2).
-// Stream-K schedule (p.streamk): the pair c of G = gridDim.x/2 owns the
-// contiguous share [c*I/G, (c+1)*I/G) of all I = tiles * KS (tile, k-step)
-// iterations, tiles ordered with tn fastest; a tile cut between pairs is
+// schedule: one segment, the whole k-range of tile (tm = blockIdx.x/2,
+// tn = blockIdx.y).  Stream-K schedule (p.streamk): the pair c of
+// G = gridDim.x/2 owns the contiguous share [c*I/G, (c+1)*I/G) of all
+// I = tiles * KS (tile, k-step) iterations; a tile cut between pairs is
 // finished by the pair that holds its first k-steps (the owner), which adds
-// the fp32 partial sums the other pairs publish, in pair order.
+// the fp32 partial sums the other pairs publish, in pair order.  Both orders
+// run the token tiles fastest: the pairs resident at once share a few weight
+// column tiles, so each tile of codes is read from DRAM once and then hits
+// in L2 for the other token tiles (with the token tiles slowest, a weight
+// larger than L2 -- the 65B gate/up codes are 180 MB -- was read once per
+// token tile).
 struct PairSeg {
     int tm, tn, k0, k1;
 };
@@ -76,16 +81,17 @@ struct PairSchedule {
         if (!SK) {
             if (grid_done) return false;
             grid_done = true;
-            sg.tn = blockIdx.x >> 1;
-            sg.tm = blockIdx.y;
+            sg.tm = p.n_in_x ? blockIdx.y : blockIdx.x >> 1;
+            sg.tn = p.n_in_x ? blockIdx.x >> 1 : blockIdx.y;
             sg.k0 = 0;
             sg.k1 = KS;
             return true;
         }
         if (pos >= end) return false;
         const int t = (int)(pos / KS);
-        sg.tm = t / p.tiles_n;
-        sg.tn = t % p.tiles_n;
+        const int tiles_m = p.tiles_total / p.tiles_n;
+        sg.tn = t / tiles_m;
+        sg.tm = t % tiles_m;
         sg.k0 = (int)(pos - (int64_t)t * KS);
         sg.k1 = (int)min((int64_t)KS, (int64_t)sg.k0 + (end - pos));
         pos += sg.k1 - sg.k0;
@@ -354,7 +360,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairShape<DQ>::THREA
             const int cid = blockIdx.x >> 1, G = gridDim.x >> 1;
             const int64_t I = (int64_t)p.tiles_total * KS;
             if (sk_owner && !*abort_flag) {
-                const int64_t t0 = (int64_t)(sg.tm * p.tiles_n + sg.tn) * KS;
+                const int64_t t0 = (int64_t)(sg.tn * (p.tiles_total / p.tiles_n) + sg.tm) * KS;
                 first_c = cid + 1;
                 last_c = cid;
                 for (int c = first_c; c < G; ++c) {

@@ -331,6 +331,8 @@ struct LinearWs {
     uint16_t* sG;
     float* part;          // small-M partial tiles
     uint32_t* sm_flags;   // small-M partial flags
+    size_t part_floats;   // capacity of part (floats)
+    size_t nflags;        // capacity of sm_flags (32-bit words)
     float* sk_part;  // stream-K partial tiles [kMaxStreamK][256*256]
     int* sk_flags;   // [kMaxStreamK] stream-K flags, then the 2 tile counters of the backward's side launch
     size_t bytes;
@@ -356,6 +358,8 @@ inline LinearWs carve_linear_ws(void* ws, int64_t M, int64_t N, int64_t K, int r
     }
     L.part = big ? nullptr : static_cast<float*>(c.take(part_floats * 4));
     L.sm_flags = big ? nullptr : static_cast<uint32_t*>(c.take(nflags * 4));
+    L.part_floats = big ? 0 : part_floats;
+    L.nflags = big ? 0 : nflags;
     L.sk_part = big ? static_cast<float*>(c.take((size_t)kMaxStreamK * 256 * 256 * 4)) : nullptr;
     L.sk_flags = big ? static_cast<int*>(c.take((size_t)(kMaxStreamK + 2) * 4)) : nullptr;
     L.bytes = c.used;
@@ -456,7 +460,11 @@ inline dim3 schedule_pair(GemmParams& p, int tiles_n, int tiles_m, const LinearW
         p.streamk = 1;
         return dim3((unsigned)(2 * G), 1, 1);
     }
-    return dim3((unsigned)(2 * tiles_n), (unsigned)tiles_m, 1);
+    // token tiles fastest (blockIdx.x / 2), weight column tiles in y (the
+    // grid's y extent is at most 65535: beyond it, columns in x)
+    p.n_in_x = tiles_n > 65535 ? 1 : 0;
+    if (p.n_in_x) return dim3((unsigned)(2 * tiles_n), (unsigned)tiles_m, 1);
+    return dim3((unsigned)(2 * tiles_m), (unsigned)tiles_n, 1);
 }
 
 inline dim3 schedule_gemm(GemmParams& p, int tiles_n, int tiles_m, const LinearWs& L) {
@@ -572,6 +580,8 @@ inline qlora_status launch_small_m_mma(const void* X, const LinearArgs& a, const
     p.Y = static_cast<uint16_t*>(Y);
     p.part = L.part;
     p.counters = reinterpret_cast<unsigned long long*>(L.sm_flags);
+    p.part_cap = (int64_t)L.part_floats;
+    p.counter_cap = (int64_t)(L.nflags / 2);
     p.epoch = next_epoch();
     if (p.epoch == 0) p.epoch = 1;
     p.timeout_ns = wait_timeout_ns();
@@ -621,6 +631,8 @@ inline qlora_status launch_small_m(const void* X, const LinearArgs& a, const voi
     p.Y = static_cast<uint16_t*>(Y);
     p.part = L.part;
     p.flags = L.sm_flags;
+    p.part_cap = (int64_t)L.part_floats;
+    p.flag_cap = (int64_t)L.nflags;
     p.epoch = next_epoch();
     p.timeout_ns = wait_timeout_ns();
     p.inject = inject_mode() == 1 ? 1 : 0;

@@ -181,9 +181,10 @@ __global__ void __launch_bounds__(MergeShape::THREADS) k_lora_merge(const __grid
                                      __fmaf_rn(p.scale, __uint_as_float(v[2 * j + 1]), hi));
             }
             uint4* dst = reinterpret_cast<uint4*>(p.out + (int64_t)n * p.K + kc);
+            if (QLORA_CHECK(n < p.N && kc + 32 <= p.K))
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-                __stcs(dst + i, make_uint4(res[4 * i], res[4 * i + 1], res[4 * i + 2], res[4 * i + 3]));
+                for (int i = 0; i < 4; ++i)
+                    __stcs(dst + i, make_uint4(res[4 * i], res[4 * i + 1], res[4 * i + 2], res[4 * i + 3]));
         }
     }
     tc_fence_before();

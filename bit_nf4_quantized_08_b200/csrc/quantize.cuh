@@ -246,7 +246,7 @@ __global__ void __launch_bounds__(256, BF16 ? QLORA_QUANT_MIN_CTAS : 2) k_quanti
             const int64_t b = e >> bshift;
             if ((lane & (blanes - 1)) == 0) {
                 const bool bvalid = b < nb;
-                if (bvalid && absmax) absmax[b] = a;
+                if (bvalid && absmax && QLORA_CHECK(b >= 0 && b < nb)) absmax[b] = a;
                 // leaf of the group's tree: block (warp * 4 + it) * (32 / blanes) + lane / blanes
                 s_max[par][((warp * 4 + it) << (3 - BS)) + (lane >> (2 + BS))] = bvalid ? a : 0.0f;
             }
@@ -286,7 +286,8 @@ __global__ void __launch_bounds__(256, BF16 ? QLORA_QUANT_MIN_CTAS : 2) k_quanti
             // the row is coded: its registers take the next group's row
             if (gn < ng) load_row(gn * 16384 + lbase + 512 * it, raw[it]);
             if (e + 16 <= n) {
-                __stcs(reinterpret_cast<uint2*>(codes + (e >> 1)), make_uint2(w[0], w[1]));
+                if (QLORA_CHECK(e >= 0 && (e >> 1) + 8 <= (n + 1) / 2))
+                    __stcs(reinterpret_cast<uint2*>(codes + (e >> 1)), make_uint2(w[0], w[1]));
             } else if (e < n) {
                 const int valid = (int)(n - e);
 #pragma unroll
@@ -294,7 +295,7 @@ __global__ void __launch_bounds__(256, BF16 ? QLORA_QUANT_MIN_CTAS : 2) k_quanti
                     if (2 * j < valid) {
                         uint32_t byte = (w[j >> 2] >> (8 * (j & 3))) & 0xFFu;
                         if (2 * j + 1 >= valid) byte &= 0xF0u;  // no element after the last one
-                        codes[(e >> 1) + j] = (uint8_t)byte;
+                        if (QLORA_CHECK((e >> 1) + j < (n + 1) / 2)) codes[(e >> 1) + j] = (uint8_t)byte;
                     }
                 }
             }
@@ -319,7 +320,7 @@ __global__ void __launch_bounds__(256, BF16 ? QLORA_QUANT_MIN_CTAS : 2) k_quanti
                 double t = v[0];
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-                if (lane == 0) group_sums[g] = t;
+                if (lane == 0 && QLORA_CHECK(g < ng)) group_sums[g] = t;
             }
         }
     }
@@ -536,12 +537,12 @@ __global__ void __launch_bounds__(256) k_dq_quantize(const float* absmax, int64_
             uint2 v;
             v.x = q[0] | (q[1] << 8) | (q[2] << 16) | (q[3] << 24);
             v.y = q[4] | (q[5] << 8) | (q[6] << 16) | (q[7] << 24);
-            *reinterpret_cast<uint2*>(q8 + b0) = v;
+            if (QLORA_CHECK(b0 >= 0 && b0 + 8 <= nb)) *reinterpret_cast<uint2*>(q8 + b0) = v;
         } else {
             for (int i = 0; i < 8; ++i)
                 if (b0 + i < nb) q8[b0 + i] = (uint8_t)q[i];
         }
-        if (lane == 0) c1[gg] = c;
+        if (lane == 0 && QLORA_CHECK(gg < ng)) c1[gg] = c;
 #pragma unroll
         for (int i = 0; i < 8; ++i) am[i] = nx[i];
     }
@@ -587,7 +588,7 @@ __global__ void __launch_bounds__(256) k_dequantize(const uint8_t* __restrict__ 
             const int lin = i * 512 + lane * 16;  // linear byte offset in the warp's 4 KB
             const int blk = lin >> 7, q = (lin >> 4) & 7;
             const uint4 v = ld_shared_v4(sbase + blk * 128 + ((q ^ (blk & 7)) << 4));
-            __stcs(dst + i * 32 + lane, v);
+            if (QLORA_CHECK((wb0 * 64 + (int64_t)(i * 32 + lane) * 8 + 8) <= n)) __stcs(dst + i * 32 + lane, v);
         }
         return;
     }
@@ -610,7 +611,7 @@ __global__ void __launch_bounds__(256) k_dequantize(const uint8_t* __restrict__ 
             uint8_t byte = codes[e >> 1];
             int c = (e & 1) ? (byte & 15) : (byte >> 4);
             __nv_bfloat16 h = __float2bfloat16_rn(__fmul_rn(code_value(fmt.code_type, c), a));
-            out[e] = *reinterpret_cast<uint16_t*>(&h);
+            if (QLORA_CHECK(e < n)) out[e] = *reinterpret_cast<uint16_t*>(&h);
         }
     }
 }

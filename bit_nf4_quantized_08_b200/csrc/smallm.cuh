@@ -46,6 +46,7 @@ struct SmallMParams {
     uint16_t* Y;          // [M][N] bf16
     float* part;          // [gridDim.x][NT][128] fp32 partial tiles
     uint32_t* flags;      // [gridDim.x][4] epoch of the published partial, per TMEM quarter
+    int64_t part_cap, flag_cap;  // capacities (floats, words): bounds checks of the debug build
     uint32_t epoch;
     uint64_t timeout_ns;
     int inject;
@@ -251,10 +252,11 @@ __global__ void __launch_bounds__(SmallMShape<NT, NG>::THREADS, 1)
                 // warp of the same TMEM quarter)
                 float* o = p.part + (int64_t)blockIdx.x * NT * 128;
 #pragma unroll
-                for (int j = 0; j < NT; ++j) o[j * 128 + row] = v[j];
+                for (int j = 0; j < NT; ++j)
+                    if (QLORA_CHECK((int64_t)blockIdx.x * NT * 128 + j * 128 + row < p.part_cap)) o[j * 128 + row] = v[j];
                 __threadfence();
                 __syncwarp();
-                if (lane == 0) {
+                if (lane == 0 && QLORA_CHECK((int64_t)blockIdx.x * 4 + quarter < p.flag_cap)) {
                     asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p.flags + blockIdx.x * 4 + quarter),
                                  "r"(p.epoch)
                                  : "memory");
@@ -304,7 +306,7 @@ __global__ void __launch_bounds__(SmallMShape<NT, NG>::THREADS, 1)
                 for (int j = 0; j < NT; ++j) {
                     if (j < p.M) {
                         const uint32_t h = pack_bf16x2(v[j], 0.0f) & 0xFFFFu;
-                        p.Y[(int64_t)j * p.N + n] = (uint16_t)h;
+                        if (QLORA_CHECK(n < p.N)) p.Y[(int64_t)j * p.N + n] = (uint16_t)h;
                     }
                 }
             }

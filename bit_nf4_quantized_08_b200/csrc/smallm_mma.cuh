@@ -72,6 +72,7 @@ struct SmallMmaParams {
     uint16_t* Y;            // [M][N]
     float* part;            // [gridDim.x][2 slots][4 slices][SROWS rows][16 MT tokens] fp32 partials
     unsigned long long* counters;  // [groups * 4 slices]: (epoch << 32) | arrivals
+    int64_t part_cap, counter_cap;  // capacities: bounds checks of the debug build
     uint32_t epoch;         // nonzero
     uint64_t timeout_ns;
     int inject;             // test mode 1: issue no loads (the waits run out)
@@ -367,8 +368,10 @@ __global__ void __launch_bounds__(SmallMmaShape<MT>::THREADS, 1)
                     for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
                         for (int e = 0; e < 4; ++e)
-                            __stcg(mine + (8 * j + 2 * tig + (e & 1)) * TOK + 16 * mt + gid + 8 * (e >> 1),
-                                   acc[j][mt][e]);
+                            if (QLORA_CHECK((mine - p.part) + (8 * j + 2 * tig + (e & 1)) * TOK + 16 * mt + gid +
+                                                8 * (e >> 1) < p.part_cap))
+                                __stcg(mine + (8 * j + 2 * tig + (e & 1)) * TOK + 16 * mt + gid + 8 * (e >> 1),
+                                       acc[j][mt][e]);
                 __threadfence();
                 __syncwarp();
                 // contributors: the CTAs from the one holding the group's first
@@ -377,7 +380,7 @@ __global__ void __launch_bounds__(SmallMmaShape<MT>::THREADS, 1)
                 uint32_t ncontrib = 0;
                 for (int c = cf; c <= cl; ++c) ncontrib += ((U * c) / G < (U * (c + 1)) / G) ? 1u : 0u;
                 uint32_t before = 0;
-                if (lane == 0) {
+                if (lane == 0 && QLORA_CHECK((int64_t)g * 4 + slice < p.counter_cap)) {
                     // arrivals of this launch (epoch in the high word; a value of
                     // another epoch counts as none)
                     unsigned long long* ctr = p.counters + (int64_t)g * 4 + slice;
@@ -434,6 +437,7 @@ __global__ void __launch_bounds__(SmallMmaShape<MT>::THREADS, 1)
                             if (m >= p.M) continue;
                             const uint32_t v = pack_bf16x2(acc[j][mt][2 * h], acc[j][mt][2 * h + 1]);
                             uint16_t* dst = p.Y + (int64_t)m * p.N + n;
+                            if (!QLORA_CHECK(m < p.M && n < p.N)) continue;
                             if (n + 1 < p.N && ((reinterpret_cast<uintptr_t>(dst) & 3u) == 0)) {
                                 *reinterpret_cast<uint32_t*>(dst) = v;
                             } else {

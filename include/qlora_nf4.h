@@ -51,8 +51,13 @@ typedef enum {
     QLORA_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
     QLORA_ERR_TIMEOUT = 4,     /* a bounded in-kernel wait ran out (reported
                                   by qlora_get_last_error only) */
-    QLORA_ERR_WORKSPACE = 5    /* the tensor is larger than the fixed internal
+    QLORA_ERR_WORKSPACE = 5,   /* the tensor is larger than the fixed internal
                                   scratch of qlora_nf4_quantize_static */
+    QLORA_ERR_BOUNDS = 6       /* debug build (libqlora_nf4_debug.so, compiled
+                                  with QLORA_DEBUG) only: a device-side bounds
+                                  check of a computed store index failed; the
+                                  store was skipped (reported by
+                                  qlora_get_last_error only; nothing traps) */
 } qlora_status;
 
 typedef enum { QLORA_F32 = 0, QLORA_BF16 = 1 } qlora_dtype;

@@ -30,6 +30,18 @@ def test_header_and_exports(Q):
         assert hasattr(lib, name), f"{name} not exported"
 
 
+def test_debug_build_loads_and_exports():
+    """The bounds-checked build (QLORA_DEBUG) loads without a GPU and exports
+    the same C ABI."""
+    from bit_nf4_quantized_08_b200 import build
+    path = build.build(debug=True)
+    dbg = ctypes.CDLL(path)
+    for name in _declared_functions():
+        assert hasattr(dbg, name), f"{name} not exported by the debug build"
+    dbg.qlora_get_last_error.argtypes = [ctypes.c_void_p]
+    dbg.qlora_get_last_error.restype = ctypes.c_int32
+
+
 def test_nf4_table_matches_oracle(Q, O):
     np.testing.assert_array_equal(np.array(Q.qlora_nf4_table(), np.float32).view(np.uint32),
                                   O.nf4_table().view(np.uint32))
