@@ -85,7 +85,7 @@ struct SmallMmaShape {
     static constexpr int RT = MT == 1 ? 4 : 2;    // 8-row tiles per warp
     static constexpr int SROWS = 8 * RT;          // rows of a slice (32 or 16)
     static constexpr int UROWS = 4 * SROWS;       // rows of a unit (128 or 64)
-    static constexpr int THREADS = 32 * (WARPS + 1);  // + the warp that loads the ring
+    static constexpr int THREADS = 32 * (WARPS + 2);  // + the warp that loads the ring, + the X reorderer
     static constexpr int XS = 6;                  // ring stages
     static constexpr int X_TILE = 16 * MT * 128;  // 16 MT tokens x 64 bf16
     static constexpr int CODE_BYTES = UROWS * 128;  // codes of one unit (128-byte swizzle)
@@ -95,8 +95,8 @@ struct SmallMmaShape {
     static constexpr int OFF_T8 = XS * STAGE;
     static constexpr int OFF_SC = OFF_T8 + 1024;                     // [WARPS][2][BPW][SROWS] fp32
     static constexpr int OFF_XCH = OFF_SC + WARPS * 2 * BPW * SROWS * 4;  // [WARPS][RT * MT * 4][32] fp32
-    static constexpr int OFF_BAR = OFF_XCH + WARPS * RT * MT * 4 * 32 * 4;  // full[XS], empty[XS]
-    static constexpr int OFF_CNT = OFF_BAR + 16 * XS;               // issued[XS], abort flag
+    static constexpr int OFF_BAR = OFF_XCH + WARPS * RT * MT * 4 * 32 * 4;  // full[XS], empty[XS], xready[XS]
+    static constexpr int OFF_CNT = OFF_BAR + 24 * XS;               // issued[XS], abort flag
     static constexpr int SMEM = OFF_CNT + 4 * XS + 16 + 1024;       // + alignment slack
     static constexpr int PART_FLOATS = SROWS * 16 * MT;  // one slice's partial tile
 };
@@ -194,6 +194,7 @@ __global__ void __launch_bounds__(SmallMmaShape<MT>::THREADS, 1)
     const uint32_t bar = base + S::OFF_BAR;
     auto full = [&](int s) { return bar + 8u * s; };
     auto empty = [&](int s) { return bar + 8u * (XS + s); };
+    auto xready = [&](int s) { return bar + 8u * (2 * XS + s); };
     int* issued = reinterpret_cast<int*>(gb + S::OFF_CNT);  // loads issued into the stage
     volatile int* abort_flag = reinterpret_cast<volatile int*>(gb + S::OFF_CNT + 4 * XS);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -218,6 +219,7 @@ __global__ void __launch_bounds__(SmallMmaShape<MT>::THREADS, 1)
         for (int s = 0; s < XS; ++s) {
             mbar_init(full(s), 1);
             mbar_init(empty(s), WARPS);
+            mbar_init(xready(s), 1);
             issued[s] = 0;
         }
         *abort_flag = 0;
@@ -276,9 +278,52 @@ __global__ void __launch_bounds__(SmallMmaShape<MT>::THREADS, 1)
                     *abort_flag = 1;
                     break;
                 }
+                // the reorderer's generic writes to the stage precede the TMA's
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 issue(i, g, q);
                 if (++q == p.KSU) { q = 0; ++g; }
             }
+        }
+    } else if (warp == WARPS + 1) {
+        // ------------------------------------------------------------ X reorderer
+        // Rewrites each X (or sU) block of a landed unit in place, from the
+        // TMA's 128-byte-swizzled rows into the MMA warps' operand order: the
+        // 16-byte quad of lane (g, t) for chunk c and token tile mt holds
+        // rows g and g + 8 (of tile mt) at the words 8 t + 2 c and 8 t + 2 c + 1,
+        // i.e. the four A registers of that lane's m16n8k16 fragment, at
+        // (((c * MT + mt) * 8 + g) * 4 + t) * 16.
+        int g = g_first, q = q_first;
+        for (int i = 0; i < n_units; ++i) {
+            const int s = i % XS;
+            if (*abort_flag || !mbar_wait_hint(full(s), (i / XS) & 1, wc, 1000)) {
+                *abort_flag = 1;
+                break;
+            }
+            const int nb = q < QW ? min(4, p.KB - 4 * q) : min(4, p.lora_ks - 4 * (q - QW));
+            for (int b = 0; b < nb; ++b) {
+                const uint32_t xs = base + (uint32_t)(s * S::STAGE + S::CODE_BYTES + b * S::X_TILE);
+                uint2 w[MT][4][2];  // [mt][c][row g, row g + 8] = words 8 t + 2 c, + 1
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const int r = 16 * mt + gid + 8 * h;
+                            const uint32_t chunk = (uint32_t)((2 * tig + (c >> 1)) ^ (r & 7));
+                            w[mt][c][h] = ld_shared_v2(xs + (uint32_t)r * 128u + (chunk << 4) + (uint32_t)(c & 1) * 8u);
+                        }
+                __syncwarp();
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        st_shared_v4(xs + (uint32_t)((((c * MT + mt) * 8 + gid) * 4 + tig) * 16), w[mt][c][0].x,
+                                     w[mt][c][1].x, w[mt][c][0].y, w[mt][c][1].y);
+                __syncwarp();
+            }
+            if (lane == 0) mbar_arrive(xready(s));
+            if (++q == p.KSU) { q = 0; ++g; }
         }
     } else {
 
@@ -465,7 +510,7 @@ __global__ void __launch_bounds__(SmallMmaShape<MT>::THREADS, 1)
         const int s = i % XS;
         const int64_t u = u0 + i;
         const int nsl = g * UROWS + slice * SROWS;  // first row of this warp's slice
-        if (!dead && !mbar_wait_hint(full(s), (i / XS) & 1, wc, 1000)) {
+        if (!dead && !mbar_wait_hint(xready(s), (i / XS) & 1, wc, 1000)) {
             *abort_flag = 1;
             dead = true;
         }
@@ -479,18 +524,14 @@ __global__ void __launch_bounds__(SmallMmaShape<MT>::THREADS, 1)
         if (!dead && nsl < p.N && (wunit ? kb < p.KB : jb < p.lora_ks)) {
             const uint32_t st = base + (uint32_t)(s * S::STAGE);
             const uint32_t xs = st + (uint32_t)(S::CODE_BYTES + bq * S::X_TILE);
-            // X (or sU) fragments: tokens gid + 8 q, physical elements
-            // 16 tig .. 16 tig + 15 of the block (128-byte swizzled rows)
-            uint32_t xf[2 * MT][8];
+            // X (or sU) fragments, reordered by the X warp: the quad of chunk
+            // c and token tile mt is the A operand (a0, a1, a2, a3) as it is
+            uint4 xq[MT][4];
 #pragma unroll
-            for (int qq = 0; qq < 2 * MT; ++qq) {
-                const int row = gid + 8 * qq;
-                const uint32_t rb = xs + (uint32_t)row * 128u;
-                const uint4 v0 = ld_shared_v4(rb + ((uint32_t)((2 * tig) ^ (row & 7)) << 4));
-                const uint4 v1 = ld_shared_v4(rb + ((uint32_t)((2 * tig + 1) ^ (row & 7)) << 4));
-                xf[qq][0] = v0.x; xf[qq][1] = v0.y; xf[qq][2] = v0.z; xf[qq][3] = v0.w;
-                xf[qq][4] = v1.x; xf[qq][5] = v1.y; xf[qq][6] = v1.z; xf[qq][7] = v1.w;
-            }
+            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    xq[mt][c] = ld_shared_v4(xs + (uint32_t)((((c * MT + mt) * 8 + gid) * 4 + tig) * 16));
             if (wunit) {
                 // -------------------------------------------------- weight block
                 float* sc = scr + ((i & 1) * BPW + bb) * SROWS;
@@ -526,11 +567,11 @@ __global__ void __launch_bounds__(SmallMmaShape<MT>::THREADS, 1)
 #pragma unroll
                         for (int mt = 0; mt < MT; ++mt) {
                             if (c == 0)
-                                mma_16816_z(d[j][mt], xf[2 * mt][0], xf[2 * mt + 1][0], xf[2 * mt][1],
-                                            xf[2 * mt + 1][1], b0[j], b1[j]);
+                                mma_16816_z(d[j][mt], xq[mt][0].x, xq[mt][0].y, xq[mt][0].z, xq[mt][0].w, b0[j],
+                                            b1[j]);
                             else
-                                mma_16816(d[j][mt], xf[2 * mt][2 * c], xf[2 * mt + 1][2 * c], xf[2 * mt][2 * c + 1],
-                                          xf[2 * mt + 1][2 * c + 1], b0[j], b1[j]);
+                                mma_16816(d[j][mt], xq[mt][c].x, xq[mt][c].y, xq[mt][c].z, xq[mt][c].w, b0[j],
+                                          b1[j]);
                         }
                 }
 #pragma unroll
@@ -576,8 +617,7 @@ __global__ void __launch_bounds__(SmallMmaShape<MT>::THREADS, 1)
                         const uint32_t w0 = (c & 1) ? h.z : h.x, w1 = (c & 1) ? h.w : h.y;
 #pragma unroll
                         for (int mt = 0; mt < MT; ++mt)
-                            mma_16816(acc[j][mt], xf[2 * mt][2 * c], xf[2 * mt + 1][2 * c], xf[2 * mt][2 * c + 1],
-                                      xf[2 * mt + 1][2 * c + 1], w0, w1);
+                            mma_16816(acc[j][mt], xq[mt][c].x, xq[mt][c].y, xq[mt][c].z, xq[mt][c].w, w0, w1);
                     }
             }
         }
