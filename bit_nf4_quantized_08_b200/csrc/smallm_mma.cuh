@@ -32,11 +32,13 @@
 // the unit is one 128-byte line of codes; the LoRA up-projection adds units
 // of four 64-wide adapter blocks after a row group's weight units.  A
 // persistent grid of one CTA per SM takes contiguous shares of the unit list
-// (stream-K), so every SM streams the same number of weight bytes.  The 16
-// warps of a CTA split a unit into 4 row slices x 4 blocks; the codes (one
-// TMA box, 128-byte swizzle) and the four X blocks of each unit pass through
-// a 6-stage ring, and the last warp to finish with a stage loads the unit
-// that comes XS units later into it (no producer warp).  At the end of a row
+// (stream-K), so every SM streams the same number of weight bytes.  The 8
+// MMA warps of a CTA split a unit into 4 row slices x 2 block pairs, and a
+// warp runs the MMA chains of its two blocks interleaved; the codes (one TMA
+// box, 128-byte swizzle) and the four X blocks of each unit pass through a
+// 6-stage ring filled by a loader warp (refilled as the MMA warps release a
+// stage), and a second helper warp rewrites each landed X block into the
+// MMA's operand order.  At the end of a row
 // group the four warps of a slice add their accumulators in block order
 // through shared memory; a group cut between CTAs is finished, per slice, by
 // whichever contributing CTA arrives last (an integer counter with a launch
@@ -515,85 +517,114 @@ __global__ void __launch_bounds__(SmallMmaShape<MT>::THREADS, 1)
             dead = true;
         }
         const bool wunit = q < QW;
+        const uint32_t st = base + (uint32_t)(s * S::STAGE);
+        // a warp whose rows all lie past the weight skips the unit
+        if (!dead && nsl < p.N && wunit) {
+            // ------------------------------------------------------ weight blocks
+            // Both blocks of the warp in one pass, so that their MMA chains
+            // (RT x BPW independent ones) interleave.  X (reordered by the X
+            // warp: the quad of chunk c and token tile mt is the A operand
+            // as it is) of a block past K reads as zeros; its codes are the
+            // TMA's zero fill and its block constant is 0.
+            uint4 xq[BPW][MT][4];
+#pragma unroll
+            for (int bb = 0; bb < BPW; ++bb) {
+                const int bq = BPW * bpair + bb;
+                const uint32_t xs = st + (uint32_t)(S::CODE_BYTES + bq * S::X_TILE);
+                const bool bv = 4 * q + bq < p.KB;
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        xq[bb][mt][c] = bv ? ld_shared_v4(xs + (uint32_t)((((c * MT + mt) * 8 + gid) * 4 + tig) * 16))
+                                           : make_uint4(0u, 0u, 0u, 0u);
+            }
+            float* sc = scr + (i & 1) * BPW * SROWS;  // [BPW][SROWS]
+            if (lane < SROWS) {
+#pragma unroll
+                for (int bb = 0; bb < BPW; ++bb) {
+                    float a = 0.0f;
+                    if (cur.q[bb] >= 0) a = p.dq ? __fadd_rn(__fmul_rn(t8s[cur.q[bb]], cur.c[bb]), off) : cur.c[bb];
+                    sc[bb * SROWS + lane] = __fmul_rn(a, p.inv_scale);
+                }
+            }
+            __syncwarp();
+            // codes of unit row r = slice * SROWS + 8 j + gid: bytes
+            // 32 bq + 8 tig .. + 7 of its 128-byte line (128-byte swizzle)
+            uint32_t cw[BPW][RT][2];
+#pragma unroll
+            for (int bb = 0; bb < BPW; ++bb)
+#pragma unroll
+                for (int j = 0; j < RT; ++j) {
+                    const int bq = BPW * bpair + bb;
+                    const int r = slice * SROWS + 8 * j + gid;
+                    const uint32_t chunk = (uint32_t)((2 * bq + (tig >> 1)) ^ (r & 7));
+                    const uint2 v = ld_shared_v2(st + (uint32_t)r * 128u + (chunk << 4) + (uint32_t)(tig & 1) * 8u);
+                    cw[bb][j][0] = v.x;
+                    cw[bb][j][1] = v.y;
+                }
+            // chunk by chunk over both blocks and all row tiles
+            float d[BPW][RT][MT][4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+#pragma unroll
+                for (int bb = 0; bb < BPW; ++bb) {
+                    uint32_t b0[RT], b1[RT];
+#pragma unroll
+                    for (int j = 0; j < RT; ++j) {
+                        b0[j] = lut_byte(cw[bb][j][c >> 1], 2 * (c & 1), lane4);
+                        b1[j] = lut_byte(cw[bb][j][c >> 1], 2 * (c & 1) + 1, lane4);
+                    }
+#pragma unroll
+                    for (int j = 0; j < RT; ++j)
+#pragma unroll
+                        for (int mt = 0; mt < MT; ++mt) {
+                            const uint4 x = xq[bb][mt][c];
+                            if (c == 0)
+                                mma_16816_z(d[bb][j][mt], x.x, x.y, x.z, x.w, b0[j], b1[j]);
+                            else
+                                mma_16816(d[bb][j][mt], x.x, x.y, x.z, x.w, b0[j], b1[j]);
+                        }
+                }
+            }
+#pragma unroll
+            for (int bb = 0; bb < BPW; ++bb)
+#pragma unroll
+                for (int j = 0; j < RT; ++j) {
+                    const float2 sj = *reinterpret_cast<const float2*>(sc + bb * SROWS + 8 * j + 2 * tig);
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) {
+                        acc[j][mt][0] = __fmaf_rn(sj.x, d[bb][j][mt][0], acc[j][mt][0]);
+                        acc[j][mt][1] = __fmaf_rn(sj.y, d[bb][j][mt][1], acc[j][mt][1]);
+                        acc[j][mt][2] = __fmaf_rn(sj.x, d[bb][j][mt][2], acc[j][mt][2]);
+                        acc[j][mt][3] = __fmaf_rn(sj.y, d[bb][j][mt][3], acc[j][mt][3]);
+                    }
+                }
+            // the adapter rows of the group into L2 a few units before their use
+            if (p.lora_ks && q == max(QW - 2, 0) && bpair == 0 && lane < SROWS) {
+                const int n = nsl + lane;
+                if (n < p.N)
+                    for (int c = 0; c < p.r * 2; c += 128)
+                        asm volatile("prefetch.global.L2 [%0];" ::"l"(
+                            reinterpret_cast<const uint8_t*>(p.B + (int64_t)n * p.r) + c));
+            }
+        }
 #pragma unroll
         for (int bb = 0; bb < BPW; ++bb) {
         const int bq = BPW * bpair + bb;
-        const int kb = 4 * q + bq, jb = 4 * (q - QW) + bq;  // this warp's weight or adapter block
+        const int jb = 4 * (q - QW) + bq;  // this warp's adapter block
         // a warp whose rows all lie past the weight, or whose block lies past
-        // K or r, skips the block
-        if (!dead && nsl < p.N && (wunit ? kb < p.KB : jb < p.lora_ks)) {
-            const uint32_t st = base + (uint32_t)(s * S::STAGE);
+        // r, skips the block
+        if (!dead && nsl < p.N && !wunit && jb < p.lora_ks) {
             const uint32_t xs = st + (uint32_t)(S::CODE_BYTES + bq * S::X_TILE);
-            // X (or sU) fragments, reordered by the X warp: the quad of chunk
-            // c and token tile mt is the A operand (a0, a1, a2, a3) as it is
+            // sU fragments, reordered by the X warp
             uint4 xq[MT][4];
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
                     xq[mt][c] = ld_shared_v4(xs + (uint32_t)((((c * MT + mt) * 8 + gid) * 4 + tig) * 16));
-            if (wunit) {
-                // -------------------------------------------------- weight block
-                float* sc = scr + ((i & 1) * BPW + bb) * SROWS;
-                if (lane < SROWS) {
-                    float a = 0.0f;
-                    if (cur.q[bb] >= 0) a = p.dq ? __fadd_rn(__fmul_rn(t8s[cur.q[bb]], cur.c[bb]), off) : cur.c[bb];
-                    sc[lane] = __fmul_rn(a, p.inv_scale);
-                }
-                __syncwarp();
-                // codes of unit row r = slice * SROWS + 8 j + gid: bytes
-                // 32 bq + 8 tig .. + 7 of its 128-byte line (128-byte swizzle)
-                uint32_t cw[RT][2];
-#pragma unroll
-                for (int j = 0; j < RT; ++j) {
-                    const int r = slice * SROWS + 8 * j + gid;
-                    const uint32_t chunk = (uint32_t)((2 * bq + (tig >> 1)) ^ (r & 7));
-                    const uint2 v = ld_shared_v2(st + (uint32_t)r * 128u + (chunk << 4) + (uint32_t)(tig & 1) * 8u);
-                    cw[j][0] = v.x;
-                    cw[j][1] = v.y;
-                }
-                // chunk by chunk over all row tiles: RT independent MMA chains
-                float d[RT][MT][4];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t b0[RT], b1[RT];
-#pragma unroll
-                    for (int j = 0; j < RT; ++j) {
-                        b0[j] = lut_byte(cw[j][c >> 1], 2 * (c & 1), lane4);
-                        b1[j] = lut_byte(cw[j][c >> 1], 2 * (c & 1) + 1, lane4);
-                    }
-#pragma unroll
-                    for (int j = 0; j < RT; ++j)
-#pragma unroll
-                        for (int mt = 0; mt < MT; ++mt) {
-                            if (c == 0)
-                                mma_16816_z(d[j][mt], xq[mt][0].x, xq[mt][0].y, xq[mt][0].z, xq[mt][0].w, b0[j],
-                                            b1[j]);
-                            else
-                                mma_16816(d[j][mt], xq[mt][c].x, xq[mt][c].y, xq[mt][c].z, xq[mt][c].w, b0[j],
-                                          b1[j]);
-                        }
-                }
-#pragma unroll
-                for (int j = 0; j < RT; ++j) {
-                    const float2 sj = *reinterpret_cast<const float2*>(sc + 8 * j + 2 * tig);
-#pragma unroll
-                    for (int mt = 0; mt < MT; ++mt) {
-                        acc[j][mt][0] = __fmaf_rn(sj.x, d[j][mt][0], acc[j][mt][0]);
-                        acc[j][mt][1] = __fmaf_rn(sj.y, d[j][mt][1], acc[j][mt][1]);
-                        acc[j][mt][2] = __fmaf_rn(sj.x, d[j][mt][2], acc[j][mt][2]);
-                        acc[j][mt][3] = __fmaf_rn(sj.y, d[j][mt][3], acc[j][mt][3]);
-                    }
-                }
-                // the adapter rows of the group into L2 a few units before their use
-                if (p.lora_ks && q == max(QW - 2, 0) && bq == 0 && lane < SROWS) {
-                    const int n = nsl + lane;
-                    if (n < p.N)
-                        for (int c = 0; c < p.r * 2; c += 128)
-                            asm volatile("prefetch.global.L2 [%0];" ::"l"(
-                                reinterpret_cast<const uint8_t*>(p.B + (int64_t)n * p.r) + c));
-                }
-            } else {
+            {
                 // -------------------------------------------------- adapter block: B rows x sU
                 const int j0 = jb * 64 + 16 * tig;  // adapter column of this lane's 16
                 const bool v0 = j0 + 8 <= p.r, v1 = j0 + 16 <= p.r;

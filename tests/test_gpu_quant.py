@@ -102,6 +102,16 @@ def test_edge_cases(Q, O, cuda, kind, dq):
     _run_both(Q, O, W.to(torch.bfloat16), dq)
 
 
+@pytest.mark.parametrize("dq", [True, False])
+def test_persistent_ragged_tail_bf16(Q, O, cuda, dq):
+    """More 16384-element groups than resident CTAs (592 on 148 SMs) and a
+    ragged last group: a CTA that codes a whole group loads the partial last
+    group as its next one (n = 11469717 = 700 whole groups + 917 elements,
+    an odd tail inside a block)."""
+    W = wl.weight(7, 1638531, seed=5, dtype=torch.bfloat16)
+    _run_both(Q, O, W, dq)
+
+
 def test_equal_absmax_is_lossless(Q, O, cuda):
     W = torch.from_numpy(_edge_tensor("equal_absmax"))
     q_dq, _ = _run_both(Q, O, W, True)
