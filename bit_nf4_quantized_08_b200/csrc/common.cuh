@@ -9,9 +9,50 @@
 #include <stdint.h>
 
 #include <cstring>
+#include <mutex>
 #include <utility>
 
 namespace qlora {
+
+// ---------------------------------------------------------------------------
+// tensor maps
+// ---------------------------------------------------------------------------
+typedef CUresult (*PFN_encodeTiled_t)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                      const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                      const cuuint32_t*, CUtensorMapInterleave,
+                                      CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                      CUtensorMapFloatOOBfill);
+
+inline PFN_encodeTiled_t encode_fn() {
+    static PFN_encodeTiled_t fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_encodeTiled_t>(p);
+    });
+    return fn;
+}
+
+// 2-D tiled map over a row-major [outer][inner] tensor.
+inline bool make_map(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int esize,
+                     uint64_t inner, uint64_t outer, uint64_t row_bytes, uint32_t box_inner,
+                     uint32_t box_outer, CUtensorMapSwizzle swz) {
+    PFN_encodeTiled_t fn = encode_fn();
+    if (!fn) return false;
+    (void)esize;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = fn(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
 
 // Launch with programmatic stream serialization (the kernel may start while
 // the previous kernel of the stream finishes; it calls griddepcontrol.wait
@@ -132,6 +173,33 @@ __device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity, c
             return false;
         }
     }
+}
+
+// mbar_wait whose polls suspend the thread for up to hint_ns while the
+// phase is still open (no busy polling that takes issue slots from the MMA
+// warps on the same scheduler).  Gives up after cfg.timeout_ns.
+__device__ __forceinline__ bool mbar_wait_hint(uint32_t bar, uint32_t parity, const WaitCfg& cfg,
+                                               uint32_t hint_ns) {
+    auto poll = [&]() {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity), "r"(hint_ns)
+            : "memory");
+        return ok != 0;
+    };
+    if (poll()) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (!poll()) {
+        if (globaltimer_ns() - t0 > cfg.timeout_ns) {
+            set_status(4);
+            return false;
+        }
+    }
+    return true;
 }
 
 // Programmatic dependent launch.  pdl_trigger lets the next kernel of the

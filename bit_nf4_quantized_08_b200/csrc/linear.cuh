@@ -30,46 +30,6 @@
 
 namespace qlora {
 
-// ---------------------------------------------------------------------------
-// tensor maps
-// ---------------------------------------------------------------------------
-typedef CUresult (*PFN_encodeTiled_t)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                      const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                      const cuuint32_t*, CUtensorMapInterleave,
-                                      CUtensorMapSwizzle, CUtensorMapL2promotion,
-                                      CUtensorMapFloatOOBfill);
-
-inline PFN_encodeTiled_t encode_fn() {
-    static PFN_encodeTiled_t fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_encodeTiled_t>(p);
-    });
-    return fn;
-}
-
-// 2-D tiled map over a row-major [outer][inner] tensor.
-inline bool make_map(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int esize,
-                     uint64_t inner, uint64_t outer, uint64_t row_bytes, uint32_t box_inner,
-                     uint32_t box_outer, CUtensorMapSwizzle swz) {
-    PFN_encodeTiled_t fn = encode_fn();
-    if (!fn) return false;
-    (void)esize;
-    cuuint64_t dims[2] = {inner, outer};
-    cuuint64_t strides[1] = {row_bytes};
-    cuuint32_t box[2] = {box_inner, box_outer};
-    cuuint32_t es[2] = {1, 1};
-    CUresult r = fn(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, es,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
 // bf16 row-major [outer][inner], 64 x box_outer boxes, 128-byte swizzle.
 inline bool map_bf16(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer,
                      uint32_t box_outer) {

@@ -55,12 +55,19 @@ namespace qlora {
 struct __align__(16) SearchSmem {
     float P[64];     // P_key
     uint32_t B[64];  // base_key | extra_key << 16
+    float Q[64];     // -P_key * 2^100 (NF4 compare on the FMA pipe)
+    float H[64];     // 16 base_key (the code in a byte's high nibble; NF4)
+    float L[64];     // 2^23 + base_key (the low nibble, on the 2^23 integer grid)
 };
 
 __device__ __forceinline__ void load_search_tables(SearchSmem& st, const Nf4SearchTable& tab) {
     for (int i = threadIdx.x; i < 64; i += blockDim.x) {
         st.P[i] = i < kSearchBuckets ? tab.thr[i] : 3.0f;
         st.B[i] = i < kSearchBuckets ? (uint32_t)tab.base[i] | ((uint32_t)max(tab.inc[i] - 1, 0) << 16) : 15u;
+        const float bk = i < kSearchBuckets ? (float)tab.base[i] : 15.0f;
+        st.Q[i] = -st.P[i] * 1.26765060e30f;  // exact: a power-of-two scale
+        st.H[i] = 16.0f * bk;
+        st.L[i] = 8388608.0f + bk;
     }
 }
 
@@ -115,214 +122,325 @@ __device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t r) {
     return d;
 }
 
-// Codes of two elements x = fl(w * rcp) in one fp32x2 multiply and FMA.
-template <int CT = 0>
-__device__ __forceinline__ void nf4_search2p(uint64_t w2, uint64_t rcp2, const SearchSmem& st, uint32_t& c0,
-                                             uint32_t& c1) {
-    const uint64_t x2 = f2_mul(w2, rcp2);
-    const uint64_t t2 = f2_fma(x2, f2_pack(kKeyScale, kKeyScale), f2_pack(kKeyMagic, kKeyMagic));
-    float x0, x1, t0, t1;
-    f2_unpack(x2, x0, x1);
-    f2_unpack(t2, t0, t1);
-    c0 = nf4_lookup<CT>(x0, t0, st);
-    c1 = nf4_lookup<CT>(x1, t1, st);
-}
-template <int CT = 0>
-__device__ __forceinline__ void nf4_search2(float w0, float w1, uint64_t rcp2, const SearchSmem& st, uint32_t& c0,
-                                            uint32_t& c1) {
-    const uint64_t x2 = f2_mul(f2_pack(w0, w1), rcp2);
-    const uint64_t t2 = f2_fma(x2, f2_pack(kKeyScale, kKeyScale), f2_pack(kKeyMagic, kKeyMagic));
-    float x0, x1, t0, t1;
-    f2_unpack(x2, x0, x1);
-    f2_unpack(t2, t0, t1);
-    c0 = nf4_lookup<CT>(x0, t0, st);
-    c1 = nf4_lookup<CT>(x1, t1, st);
+// sat(x * 2^100 + q) with q = -P * 2^100: 1 exactly when x > P, else 0.
+// The FMA rounds once, so the result has the sign of x - P.  With |P| at
+// least 0.0398 (the NF4 thresholds; 3.0 where a bucket has none), two
+// distinct fp32 values x and P differ by at least 2^-30, so a positive
+// difference scales to at least 2^70 and saturates to 1; x == P gives 0,
+// and a NaN x saturates to 0.
+__device__ __forceinline__ float above_sat(float x, float q) {
+    float a;
+    asm("fma.rn.sat.f32 %0, %1, 0f71800000, %2;" : "=f"(a) : "f"(x), "f"(q));
+    return a;
 }
 
-// Resident CTAs per SM the bf16 quantizer is compiled for (registers per
-// thread = 65536 / (256 * this)).
-#ifndef QLORA_QUANT_MIN_CTAS
-#define QLORA_QUANT_MIN_CTAS 4
-#endif
+// The packed byte (code(x0) << 4) | code(x1) of two elements x = fl(w * rcp)
+// (w2 = {w0, w1}), as the fp32 value 2^23 + byte (the byte in its low 8
+// bits): one fp32x2 multiply and bucket-key FMA for both.  NF4: the byte is
+// 16 (base0 + above0) + base1 + above1, from the high-nibble table of x0's
+// bucket and the low-nibble table of x1's, all exact small integers in fp32.
+// FP4 takes the general lookup.
+template <int CT>
+__device__ __forceinline__ uint32_t nf4_byte2(uint64_t w2, uint64_t rcp2, uint64_t k2, uint64_t m2,
+                                              const SearchSmem& st) {
+    const uint64_t x2 = f2_mul(w2, rcp2);
+    const uint64_t t2 = f2_fma(x2, k2, m2);
+    float x0, x1, t0, t1;
+    f2_unpack(x2, x0, x1);
+    f2_unpack(t2, t0, t1);
+    if (CT != 0) return 0x4B000000u + (nf4_lookup<CT>(x0, t0, st) << 4) + nf4_lookup<CT>(x1, t1, st);
+    const uint32_t o0 = __float_as_uint(t0) & 0xFCu, o1 = __float_as_uint(t1) & 0xFCu;
+    auto at = [](const float* tab, uint32_t off) {
+        return *reinterpret_cast<const float*>(reinterpret_cast<const char*>(tab) + off);
+    };
+    const float a0 = above_sat(x0, at(st.Q, o0)), a1 = above_sat(x1, at(st.Q, o1));
+    const float y0 = __fmaf_rn(a0, 16.0f, at(st.H, o0));
+    const float y1 = __fadd_rn(a1, at(st.L, o1));
+    return __float_as_uint(__fadd_rn(y0, y1));
+}
+
+// Four bytes b_k (the low byte of each word) as one word, b0 lowest.
+__device__ __forceinline__ uint32_t pack4_low_bytes(uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
+    return __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
+}
+
+// Shape of the quantizer: one CTA per SM, 16 coding warps and a loader warp;
+// a stage of the shared-memory ring holds one group of 16384 elements as
+// 128-byte rows (64 bf16 or 32 fp32) in the TMA's 128-byte swizzle, and a
+// lane codes 32 consecutive elements of a group.
+template <bool BF16>
+struct QuantRing {
+    static constexpr int CW = 16;                          // coding warps
+    static constexpr int THREADS = 32 * (CW + 1);          // + the loader warp
+    static constexpr int STAGE = 16384 * (BF16 ? 2 : 4);   // bytes of one group
+    static constexpr int NST = BF16 ? 6 : 3;               // stages
+    static constexpr int ROWS = STAGE / 128;               // 128-byte rows of a stage
+    static constexpr int BOX_ROWS = 256;                   // rows of one TMA box
+    static constexpr int OFF_BAR = NST * STAGE;            // full[NST], empty[NST]
+    static constexpr int OFF_PART = OFF_BAR + 16 * NST;    // double [NST + 1][CW]: warp subtree sums
+    static constexpr int OFF_FLAG = OFF_PART + 8 * (NST + 1) * CW;  // abort flag
+    static constexpr int SMEM = OFF_FLAG + 16 + 1024;      // + alignment slack
+};
+
+// One lane's share of a group: the block maxima of its 32 elements (raw, in
+// order), their codes, and the warp's fp64 pairwise subtree sum of its
+// blocks' maxima (the same value in every lane; 0 when not wanted).  e: the
+// lane's first element.  WHOLE: all 32 lie inside the tensor.
+template <bool BF16, int CT, int BS, bool WHOLE>
+__device__ __forceinline__ double quant_lane(const uint32_t (&raw)[BF16 ? 16 : 32], int64_t e, int64_t n,
+                                             int64_t nb, uint8_t* codes, float* absmax, bool sums,
+                                             const SearchSmem& st, int lane) {
+    constexpr int bshift = 6 + BS;   // log2 of the block size
+    constexpr int blanes = 2 << BS;  // lanes per block
+    // block absmax (exact: a max of magnitudes)
+    float a;
+    if (BF16) {
+        // packed bf16 max of magnitudes (the sign of each half is the xor of
+        // the signs, dropped at the end)
+        uint32_t m = raw[0];
+#pragma unroll
+        for (int k = 1; k < 16; ++k) asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(m) : "r"(raw[k]));
+        m &= 0x7FFF7FFFu;
+        m = max(m & 0xFFFFu, m >> 16);
+        a = __uint_as_float(m << 16);
+    } else {
+        a = 0.0f;
+#pragma unroll
+        for (int k = 0; k < 32; ++k) a = fmaxf(a, fabsf(__uint_as_float(raw[k])));
+    }
+#pragma unroll
+    for (int o = 1; o < blanes; o <<= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    const int64_t b = e >> bshift;
+    const bool bvalid = WHOLE || b < nb;
+    if ((lane & (blanes - 1)) == 0 && bvalid && absmax && QLORA_CHECK(b >= 0 && b < nb)) absmax[b] = a;
+
+    // codes: byte j of w[h] = (code[8h + 2j] << 4) | code[8h + 2j + 1]
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+    if (a >= 1.17549435e-38f) {
+        const float rcp = __frcp_rn(a);
+        const uint64_t rcp2 = f2_pack(rcp, rcp);
+        const uint64_t k2 = f2_pack(kKeyScale, kKeyScale), m2 = f2_pack(kKeyMagic, kKeyMagic);
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            uint32_t by[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int k = 4 * h + j;
+                const uint64_t w2 = BF16 ? bf16x2_to_f2(raw[k])
+                                         : f2_pack(__uint_as_float(raw[2 * k]), __uint_as_float(raw[2 * k + 1]));
+                by[j] = nf4_byte2<CT>(w2, rcp2, k2, m2, st);
+            }
+            w[h] = pack4_low_bytes(by[0], by[1], by[2], by[3]);
+        }
+    } else {
+        // zero or subnormal block: exact power-of-two prescale 2^64
+        const float p = 18446744073709551616.0f;
+        const float rcp = (a == 0.0f) ? 0.0f : __frcp_rn(__fmul_rn(a, p));
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+            const uint32_t bits = BF16 ? ((k & 1) ? (raw[k >> 1] & 0xFFFF0000u) : (raw[k >> 1] << 16)) : raw[k];
+            const uint32_t c = nf4_search<CT>(__fmul_rn(__fmul_rn(__uint_as_float(bits), p), rcp), st);
+            w[k >> 3] += c << (4 * ((k & 7) ^ 1));
+        }
+    }
+    if (WHOLE || e + 32 <= n) {
+        if (QLORA_CHECK(e >= 0 && (e >> 1) + 16 <= (n + 1) / 2))
+            __stcs(reinterpret_cast<uint4*>(codes + (e >> 1)), make_uint4(w[0], w[1], w[2], w[3]));
+    } else if (e < n) {
+        const int valid = (int)(n - e);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            if (2 * j < valid) {
+                uint32_t byte = (w[j >> 2] >> (8 * (j & 3))) & 0xFFu;
+                if (2 * j + 1 >= valid) byte &= 0xF0u;  // no element after the last one
+                if (QLORA_CHECK((e >> 1) + j < (n + 1) / 2)) codes[(e >> 1) + j] = (uint8_t)byte;
+            }
+        }
+    }
+    double t = 0.0;
+    if (sums) {
+        // the warp's leaves in pairwise order: partners blanes, 2 blanes, ..
+        // lanes apart (x + y and y + x are the same IEEE sum, so every lane
+        // ends with the same value)
+        t = bvalid ? (double)a : 0.0;
+#pragma unroll
+        for (int o = blanes; o < 32; o <<= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    }
+    return t;
+}
+
+// fp64 pairwise sum of the 16 warp subtree sums of a group, in warp order.
+__device__ __forceinline__ double quant_group_sum(const double* p) {
+    double v[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) v[k] = p[k];
+#pragma unroll
+    for (int d = 1; d < 16; d <<= 1)
+#pragma unroll
+        for (int k = 0; k < 16; k += 2 * d) v[k] = v[k] + v[k + d];
+    return v[0];
+}
 
 // ---------------------------------------------------------------------------
-// K1: quantize.  A persistent grid; CTA c (8 warps) takes the groups of
-// 16384 elements c, c + G, c + 2G, ...; in a group, warp w handles rows
-// 4w..4w+3 of 512 elements, a lane holds 16 consecutive elements, and
-// 4 << BS lanes make one block (64, 128 or 256 elements).  As soon as a row
-// is coded, the lane loads its row of the CTA's next group into the same
-// registers, so every lane keeps four 32-byte (bf16) loads in flight while
-// it computes.  Also writes each group's fp64 pairwise-tree sum of block
-// maxima for the double-quantization offset.  CT: code book (0 NF4, 1 FP4).
+// K1: quantize.  A persistent grid of one CTA per SM; CTA c takes the
+// groups of 16384 elements c, c + G, c + 2G, ...  The loader warp streams
+// every whole group into the ring with one TMA box per 256 rows (refilled as
+// the coding warps release a stage); a tensor's partial last group is read
+// with plain, bounds-checked loads instead.  In a group, lane l of coding
+// warp w takes elements [1024 w + 32 l, + 32) (bf16: half of row
+// 16 w + l / 2; fp32: row 32 w + l), so 2 << BS lanes make one block (64,
+// 128 or 256 elements); the swizzle puts the 16-byte chunks of the eight
+// lanes of a quarter warp in distinct banks.  Also writes each group's fp64
+// pairwise-tree sum of block maxima for the double-quantization offset: each
+// warp adds its own leaves (a subtree) with shuffles and leaves the sum in
+// shared memory before it releases the stage; the loader, which waits for
+// that release anyway, adds the 16 subtree sums.  CT: code book (0 NF4, 1
+// FP4).
 // ---------------------------------------------------------------------------
 template <bool BF16, int CT, int BS>
-__global__ void __launch_bounds__(256, BF16 ? QLORA_QUANT_MIN_CTAS : 2) k_quantize_blocks(const void* W, int64_t n,
-                                                            uint8_t* codes,
-                                                            float* absmax,
-                                                            double* group_sums,
-                                                            Nf4SearchTable tab) {
+__global__ void __launch_bounds__(QuantRing<BF16>::THREADS, 1)
+    k_quantize_blocks(const __grid_constant__ CUtensorMap tmW, const void* W, int64_t n, uint8_t* codes,
+                      float* absmax, double* group_sums, Nf4SearchTable tab, uint64_t timeout_ns) {
+    using R = QuantRing<BF16>;
+    constexpr int CW = R::CW, NST = R::NST;
+    constexpr int bshift = 6 + BS;  // log2 of the block size
     __shared__ SearchSmem st;
-    __shared__ float s_max[2][256 >> BS];  // block maxima of a group (0 past the tensor), by group parity
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_base = smem_u32(smem_raw);
+    const uint32_t base = (raw_base + 1023u) & ~1023u;
+    uint8_t* gb = smem_raw + (base - raw_base);
+    const uint32_t bar = base + R::OFF_BAR;
+    auto full = [&](int s) { return bar + 8u * s; };
+    auto empty = [&](int s) { return bar + 8u * (NST + s); };
+    double* part = reinterpret_cast<double*>(gb + R::OFF_PART);  // [NST + 1][CW]
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(gb + R::OFF_FLAG);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const WaitCfg wc{timeout_ns};
+    const int64_t ng = (n + 16383) >> 14, nfull = n >> 14;
+    const int64_t nb = (n + (1 << bshift) - 1) >> bshift;
+    const int G = gridDim.x;
+    // this CTA's groups, and how many of them are whole (the partial one, if
+    // any, is the tensor's last group, so it comes last here too)
+    const int64_t mine = blockIdx.x < ng ? (ng - blockIdx.x + G - 1) / G : 0;
+    const int64_t mine_full = blockIdx.x < nfull ? (nfull - blockIdx.x + G - 1) / G : 0;
+    const bool sums = group_sums != nullptr;
+
     // dependent launch: resident before the kernel ahead ends, no access to
-    // memory before it has.  The kernels that wait this way take no
+    // global memory before it has.  The kernels that wait this way take no
     // __restrict__ pointers: with them the compiler may move loads of
     // "unchanging" data above griddepcontrol.wait.
     pdl_trigger();
-    pdl_wait();
     load_search_tables(st, tab);
-    __syncthreads();
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    constexpr int bshift = 6 + BS;                    // log2 of the block size
-    constexpr int blanes = 4 << BS;                   // lanes per block
-    const int64_t nb = (n + (1 << bshift) - 1) >> bshift;
-    const int64_t ng = (n + 16383) >> 14;
-    constexpr int WORDS = BF16 ? 8 : 16;  // 32-bit words per lane per row
-    uint32_t raw[4][WORDS];
-    // first element of this lane in row it of group g: 16384 g + lbase + 512 it
-    const int64_t lbase = (int64_t)warp * 2048 + lane * 16;
-
-    auto load_row = [&](int64_t e, uint32_t (&r)[WORDS]) {
-        if (e + 16 <= n) {
-            const uint4* src = BF16 ? reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(W) + e)
-                                    : reinterpret_cast<const uint4*>(static_cast<const float*>(W) + e);
-#pragma unroll
-            for (int v = 0; v < WORDS / 4; ++v) {
-                uint4 q = __ldcs(src + v);
-                r[4 * v + 0] = q.x;
-                r[4 * v + 1] = q.y;
-                r[4 * v + 2] = q.z;
-                r[4 * v + 3] = q.w;
-            }
-        } else {
-#pragma unroll
-            for (int v = 0; v < WORDS; ++v) r[v] = 0u;
-            if (e < n) {
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    if (e + i < n) {
-                        if (BF16) {
-                            uint32_t h = static_cast<const uint16_t*>(W)[e + i];
-                            r[i >> 1] |= h << ((i & 1) * 16);
-                        } else {
-                            r[i] = __float_as_uint(static_cast<const float*>(W)[e + i]);
-                        }
-                    }
-                }
-            }
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NST; ++s) {
+            mbar_init(full(s), 1);
+            mbar_init(empty(s), CW);
         }
-    };
-
-    int64_t g = blockIdx.x;
-    if (g < ng) {
-#pragma unroll
-        for (int it = 0; it < 4; ++it) load_row(g * 16384 + lbase + 512 * it, raw[it]);
+        *abort_flag = 0;
+        fence_mbar_init();
+        if (mine_full > 0) prefetch_tensormap(&tmW);
     }
-    for (int par = 0; g < ng; g += gridDim.x, par ^= 1) {
-        const int64_t gn = g + gridDim.x;  // this CTA's next group
-#pragma unroll
-        for (int it = 0; it < 4; ++it) {
-            const int64_t e = g * 16384 + lbase + 512 * it;
-            // block absmax (exact: a max of magnitudes)
-            float a;
-            if (BF16) {
-                // packed bf16 max of magnitudes (the sign of each half is the xor
-                // of the signs, dropped at the end)
-                uint32_t m = raw[it][0];
-#pragma unroll
-                for (int i = 1; i < 8; ++i)
-                    asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(m) : "r"(raw[it][i]));
-                m &= 0x7FFF7FFFu;
-                m = max(m & 0xFFFFu, m >> 16);
-                a = __uint_as_float(m << 16);
-            } else {
-                a = 0.0f;
-#pragma unroll
-                for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(__uint_as_float(raw[it][i])));
-            }
-#pragma unroll
-            for (int o = 1; o < blanes; o <<= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    __syncthreads();
+    pdl_wait();
 
-            const int64_t b = e >> bshift;
-            if ((lane & (blanes - 1)) == 0) {
-                const bool bvalid = b < nb;
-                if (bvalid && absmax && QLORA_CHECK(b >= 0 && b < nb)) absmax[b] = a;
-                // leaf of the group's tree: block (warp * 4 + it) * (32 / blanes) + lane / blanes
-                s_max[par][((warp * 4 + it) << (3 - BS)) + (lane >> (2 + BS))] = bvalid ? a : 0.0f;
-            }
-
-            // codes packed as they are found: byte j of w[h] = (code[8h + 2j] << 4) | code[8h + 2j + 1]
-            uint32_t w[2] = {0u, 0u};
-            if (a >= 1.17549435e-38f) {
-                const float rcp = __frcp_rn(a);
-                const uint64_t rcp2 = f2_pack(rcp, rcp);
+    int issued[NST];  // loads issued into each stage (the loader lane)
 #pragma unroll
-                for (int i = 0; i < 16; i += 2) {
-                    uint32_t c0, c1;
+    for (int s = 0; s < NST; ++s) issued[s] = 0;
+    if (warp == CW) {
+        // ------------------------------------------------------------ loader
+        if (lane == 0) {
+            // group j of this CTA is released: its sum (stage j % NST)
+            auto group_done = [&](int64_t j) {
+                const int s = (int)(j % NST);
+                if (*abort_flag || !mbar_wait_sleep(empty(s), (uint32_t)((j / NST) & 1), wc, 64)) {
+                    *abort_flag = 1;
+                    return false;
+                }
+                const int64_t g = blockIdx.x + j * G;
+                if (sums && QLORA_CHECK(g < ng)) group_sums[g] = quant_group_sum(part + s * CW);
+                return true;
+            };
+            bool ok = true;
+            for (int64_t i = 0; i < mine_full && ok; ++i) {
+                const int s = (int)(i % NST);
+                // the coding warps have released the stage's previous group
+                if (i >= NST && !(ok = group_done(i - NST))) break;
+                const int64_t g = blockIdx.x + i * G;
+                mbar_arrive_expect_tx(full(s), (uint32_t)R::STAGE);
+#pragma unroll
+                for (int b = 0; b < R::ROWS / R::BOX_ROWS; ++b)
+                    tma_load_2d(base + (uint32_t)(s * R::STAGE + b * R::BOX_ROWS * 128), &tmW, full(s), 0,
+                                (int)(g * R::ROWS + b * R::BOX_ROWS));
+#pragma unroll
+                for (int t = 0; t < NST; ++t) issued[t] += (t == s);
+            }
+            for (int64_t j = mine_full > NST ? mine_full - NST : 0; j < mine_full && ok; ++j) ok = group_done(j);
+        }
+    } else {
+        // ------------------------------------------------------------ coding warps
+        // 128-byte row of the stage and first 16-byte chunk of this lane
+        const int row = BF16 ? 16 * warp + (lane >> 1) : 32 * warp + lane;
+        const int chunk0 = BF16 ? 4 * (lane & 1) : 0;
+        const uint32_t lane_off = (uint32_t)row * 128u;
+        const uint32_t sw = (uint32_t)(row & 7);
+        bool ok = true;
+        for (int64_t i = 0; i < mine_full; ++i) {
+            const int s = (int)(i % NST);
+            const int64_t e = (blockIdx.x + i * G) * 16384 + (int64_t)warp * 1024 + lane * 32;  // first element
+            // every lane waits (and so sees the TMA's writes); the warp leaves
+            // together if any lane gave up
+            ok = !*abort_flag && mbar_wait_hint(full(s), (uint32_t)((i / NST) & 1), wc, 1000);
+            if (!__all_sync(0xffffffffu, ok)) {
+                ok = false;
+                if (lane == 0) *abort_flag = 1;
+                break;
+            }
+            uint32_t raw[BF16 ? 16 : 32];
+            const uint32_t sb = base + (uint32_t)(s * R::STAGE) + lane_off;
+#pragma unroll
+            for (int v = 0; v < (BF16 ? 4 : 8); ++v) {
+                const uint4 q = ld_shared_v4(sb + ((((uint32_t)(chunk0 + v)) ^ sw) << 4));
+                raw[4 * v + 0] = q.x;
+                raw[4 * v + 1] = q.y;
+                raw[4 * v + 2] = q.z;
+                raw[4 * v + 3] = q.w;
+            }
+            const double t = quant_lane<BF16, CT, BS, true>(raw, e, n, nb, codes, absmax, sums, st, lane);
+            // the subtree sum, then the stage back to the loader (after every
+            // lane's reads of it)
+            if (lane == 0) part[s * CW + warp] = t;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty(s));
+        }
+        if (ok && mine > mine_full) {
+            // the tensor's partial last group: plain loads, bounds-checked
+            const int64_t e = (ng - 1) * 16384 + (int64_t)warp * 1024 + lane * 32;
+            uint32_t raw[BF16 ? 16 : 32];
+#pragma unroll
+            for (int v = 0; v < (BF16 ? 16 : 32); ++v) raw[v] = 0u;
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+                if (e + k < n) {
                     if (BF16) {
-                        nf4_search2p<CT>(bf16x2_to_f2(raw[it][i >> 1]), rcp2, st, c0, c1);
+                        const uint32_t h = static_cast<const uint16_t*>(W)[e + k];
+                        raw[k >> 1] |= h << ((k & 1) * 16);
                     } else {
-                        nf4_search2<CT>(__uint_as_float(raw[it][i]), __uint_as_float(raw[it][i + 1]), rcp2, st, c0,
-                                        c1);
-                    }
-                    // byte (i & 7) / 2 of w[i / 8]; the pairs are added in order with
-                    // shift-and-add steps, a byte-reverse at the end
-                    w[i >> 3] = (w[i >> 3] << 8) + (c0 << 4) + c1;
-                }
-                w[0] = __byte_perm(w[0], 0u, 0x0123);
-                w[1] = __byte_perm(w[1], 0u, 0x0123);
-            } else {
-                // zero or subnormal block: exact power-of-two prescale 2^64
-                const float p = 18446744073709551616.0f;
-                const float rcp = (a == 0.0f) ? 0.0f : __frcp_rn(__fmul_rn(a, p));
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const uint32_t bits = BF16 ? ((i & 1) ? (raw[it][i >> 1] & 0xFFFF0000u) : (raw[it][i >> 1] << 16))
-                                               : raw[it][i];
-                    const uint32_t c = nf4_search<CT>(__fmul_rn(__fmul_rn(__uint_as_float(bits), p), rcp), st);
-                    w[i >> 3] += c << (4 * ((i & 7) ^ 1));
-                }
-            }
-            // the row is coded: its registers take the next group's row
-            if (gn < ng) load_row(gn * 16384 + lbase + 512 * it, raw[it]);
-            if (e + 16 <= n) {
-                if (QLORA_CHECK(e >= 0 && (e >> 1) + 8 <= (n + 1) / 2))
-                    __stcs(reinterpret_cast<uint2*>(codes + (e >> 1)), make_uint2(w[0], w[1]));
-            } else if (e < n) {
-                const int valid = (int)(n - e);
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    if (2 * j < valid) {
-                        uint32_t byte = (w[j >> 2] >> (8 * (j & 3))) & 0xFFu;
-                        if (2 * j + 1 >= valid) byte &= 0xF0u;  // no element after the last one
-                        if (QLORA_CHECK((e >> 1) + j < (n + 1) / 2)) codes[(e >> 1) + j] = (uint8_t)byte;
+                        raw[k] = __float_as_uint(static_cast<const float*>(W)[e + k]);
                     }
                 }
             }
+            const double t = quant_lane<BF16, CT, BS, false>(raw, e, n, nb, codes, absmax, sums, st, lane);
+            if (lane == 0) part[NST * CW + warp] = t;
         }
-        if (group_sums) {
-            // fp64 pairwise tree over the group's 256 >> BS block maxima in
-            // block order: each lane of warp 0 folds its run of adjacent
-            // leaves, then the lanes pair up (x + y and y + x are the same
-            // IEEE sum, so both lanes of a pair agree).  The next group
-            // writes the other parity's leaves, and the one after waits at
-            // this barrier of the next group, after warp 0 has read these.
-            __syncthreads();
-            if (warp == 0) {
-                constexpr int PER = 8 >> BS;  // leaves per lane
-                double v[PER];
-#pragma unroll
-                for (int i = 0; i < PER; ++i) v[i] = (double)s_max[par][lane * PER + i];
-#pragma unroll
-                for (int w = 1; w < PER; w <<= 1)
-#pragma unroll
-                    for (int i = 0; i < PER; i += 2 * w) v[i] = v[i] + v[i + w];
-                double t = v[0];
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-                if (lane == 0 && QLORA_CHECK(g < ng)) group_sums[g] = t;
-            }
-        }
+    }
+    // every load issued into the ring has landed before the CTA exits, and
+    // the kernel does not complete before the one it depends on
+    __syncthreads();
+    if (warp == CW && lane == 0) {
+        if (sums && mine > mine_full && !*abort_flag && QLORA_CHECK(ng >= 1))
+            group_sums[ng - 1] = quant_group_sum(part + NST * CW);
+        for (int s = 0; s < NST; ++s)
+            if (issued[s] > 0) mbar_wait(full(s), (uint32_t)((issued[s] - 1) & 1), wc);
     }
 }
 
@@ -728,19 +846,41 @@ inline cudaError_t launch_quantize_blocks(const void* W, int is_bf16, int64_t n,
     ProfileScope ps(QLORA_KERNEL_QUANTIZE, s);
     note_launch();
     const Nf4SearchTable& tab = search_table(fmt.code_type);
-    using Kern = void (*)(const void*, int64_t, uint8_t*, float*, double*, Nf4SearchTable);
+    using Kern = void (*)(const CUtensorMap, const void*, int64_t, uint8_t*, float*, double*, Nf4SearchTable,
+                          uint64_t);
     static constexpr Kern kTable[2][2][3] = {
         {{k_quantize_blocks<false, 0, 0>, k_quantize_blocks<false, 0, 1>, k_quantize_blocks<false, 0, 2>},
          {k_quantize_blocks<false, 1, 0>, k_quantize_blocks<false, 1, 1>, k_quantize_blocks<false, 1, 2>}},
         {{k_quantize_blocks<true, 0, 0>, k_quantize_blocks<true, 0, 1>, k_quantize_blocks<true, 0, 2>},
          {k_quantize_blocks<true, 1, 0>, k_quantize_blocks<true, 1, 1>, k_quantize_blocks<true, 1, 2>}}};
-    const Kern kern = kTable[is_bf16 ? 1 : 0][fmt.code_type ? 1 : 0][fmt.bs_shift];
-    // persistent: as many CTAs as are resident at once, at most one per group
+    const int ib = is_bf16 ? 1 : 0, ic = fmt.code_type ? 1 : 0, is = fmt.bs_shift;
+    const Kern kern = kTable[ib][ic][is];
+    const int smem = is_bf16 ? QuantRing<true>::SMEM : QuantRing<false>::SMEM;
+    const int threads = is_bf16 ? QuantRing<true>::THREADS : QuantRing<false>::THREADS;
+    static std::once_flag attr_once[2][2][3];
+    static cudaError_t attr_err[2][2][3];
+    std::call_once(attr_once[ib][ic][is], [&] {
+        attr_err[ib][ic][is] = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    });
+    if (attr_err[ib][ic][is] != cudaSuccess) return attr_err[ib][ic][is];
+    // the whole groups as 128-byte rows (64 bf16 or 32 fp32), 256-row boxes
+    CUtensorMap tm;
+    memset(&tm, 0, sizeof(tm));
+    const int64_t nfull = n >> 14;
+    if (nfull > 0) {
+        const bool ok = is_bf16 ? make_map(&tm, W, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 64, (uint64_t)nfull * 256,
+                                           128, 64, QuantRing<true>::BOX_ROWS, CU_TENSOR_MAP_SWIZZLE_128B)
+                                : make_map(&tm, W, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 32, (uint64_t)nfull * 512,
+                                           128, 32, QuantRing<false>::BOX_ROWS, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (!ok) return cudaErrorInvalidValue;
+    }
+    // persistent: one CTA per SM, at most one per group
     int dev = 0, nsm = 148;
     if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         nsm = 148;
-    const int64_t grid = std::min<int64_t>(ng, (int64_t)nsm * (is_bf16 ? QLORA_QUANT_MIN_CTAS : 2));
-    return launch_pdl(kern, dim3((unsigned)grid), dim3(256), 0, s, 0, W, n, codes, absmax, group_sums, tab);
+    const int64_t grid = std::min<int64_t>(ng, (int64_t)nsm);
+    return launch_pdl(kern, dim3((unsigned)grid), dim3(threads), smem, s, 0, tm, W, n, codes, absmax, group_sums,
+                      tab, wait_timeout_ns());
 }
 
 inline cudaError_t launch_dq_offset(const double* group_sums, int64_t ngroups, int64_t nb,

@@ -80,15 +80,24 @@ struct SmallMmaParams {
     int inject;             // test mode 1: issue no loads (the waits run out)
 };
 
+// Ring stages of the warp-MMA small-M kernel (24 KB each), and blocks of a
+// unit per MMA warp (2: 8 MMA warps, 1: 16).
+#ifndef QLORA_SMALLM_XS
+#define QLORA_SMALLM_XS 6
+#endif
+#ifndef QLORA_SMALLM_BPW
+#define QLORA_SMALLM_BPW 2
+#endif
+
 template <int MT>
 struct SmallMmaShape {
-    static constexpr int BPW = 2;                 // blocks of a unit per MMA warp
+    static constexpr int BPW = QLORA_SMALLM_BPW;  // blocks of a unit per MMA warp
     static constexpr int WARPS = 16 / BPW;        // MMA warps: 4 row slices x 4 / BPW block groups
     static constexpr int RT = MT == 1 ? 4 : 2;    // 8-row tiles per warp
     static constexpr int SROWS = 8 * RT;          // rows of a slice (32 or 16)
     static constexpr int UROWS = 4 * SROWS;       // rows of a unit (128 or 64)
     static constexpr int THREADS = 32 * (WARPS + 2);  // + the warp that loads the ring, + the X reorderer
-    static constexpr int XS = 6;                  // ring stages
+    static constexpr int XS = QLORA_SMALLM_XS;    // ring stages
     static constexpr int X_TILE = 16 * MT * 128;  // 16 MT tokens x 64 bf16
     static constexpr int CODE_BYTES = UROWS * 128;  // codes of one unit (128-byte swizzle)
     static constexpr int STAGE = CODE_BYTES + 4 * X_TILE;
@@ -148,33 +157,6 @@ __device__ __forceinline__ int owner_cta(int64_t x, int64_t I, int G) {
     while (c + 1 < G && (I * (c + 1)) / G <= x) ++c;
     while (c > 0 && (I * c) / G > x) --c;
     return c;
-}
-
-// mbar_wait whose polls suspend the thread for up to hint_ns while the
-// phase is still open (no busy polling that takes issue slots from the MMA
-// warps on the same scheduler).  Gives up after cfg.timeout_ns.
-__device__ __forceinline__ bool mbar_wait_hint(uint32_t bar, uint32_t parity, const WaitCfg& cfg,
-                                               uint32_t hint_ns) {
-    auto poll = [&]() {
-        uint32_t ok;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(ok)
-            : "r"(bar), "r"(parity), "r"(hint_ns)
-            : "memory");
-        return ok != 0;
-    };
-    if (poll()) return true;
-    const uint64_t t0 = globaltimer_ns();
-    while (!poll()) {
-        if (globaltimer_ns() - t0 > cfg.timeout_ns) {
-            set_status(4);
-            return false;
-        }
-    }
-    return true;
 }
 
 __device__ __forceinline__ void named_sync(int id, int threads) {
