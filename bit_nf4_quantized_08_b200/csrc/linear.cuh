@@ -492,7 +492,7 @@ inline cudaError_t launch_small_m_kernel(const SmallMParams& p, int grid, cudaSt
 template <int MT>
 inline cudaError_t launch_small_m_mma_kernel(SmallMmaParams& p, cudaStream_t s) {
     using S = SmallMmaShape<MT>;
-    static_assert(S::SMEM + 256 * 32 * 4 <= 232448, "shared memory per CTA");
+    static_assert(S::SMEM + S::STATIC_SMEM <= 232448, "shared memory per CTA");
     static_assert(2 * 4 * S::PART_FLOATS <= kSmallMmaPartFloatsPerCta, "partial workspace");
     const int64_t groups = (p.N + S::UROWS - 1) / S::UROWS;
     p.KSU = (p.KB + 3) / 4 + (p.lora_ks + 3) / 4;

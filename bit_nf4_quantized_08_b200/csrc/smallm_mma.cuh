@@ -110,6 +110,7 @@ struct SmallMmaShape {
     static constexpr int OFF_CNT = OFF_BAR + 24 * XS;               // issued[XS], abort flag
     static constexpr int SMEM = OFF_CNT + 4 * XS + 16 + 1024;       // + alignment slack
     static constexpr int PART_FLOATS = SROWS * 16 * MT;  // one slice's partial tile
+    static constexpr int STATIC_SMEM = 256 * 32 * 4;     // the table (static shared memory)
 };
 
 // (not volatile: pure functions of their registers, so the compiler may
