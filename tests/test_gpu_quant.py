@@ -112,6 +112,15 @@ def test_persistent_ragged_tail_bf16(Q, O, cuda, dq):
     _run_both(Q, O, W, dq)
 
 
+@pytest.mark.parametrize("dq", [True, False])
+def test_persistent_ring_fp32(Q, O, cuda, dq):
+    """fp32 input (three 64 KB ring stages of two TMA boxes each) with more
+    than three whole groups per CTA, so every stage is refilled, and a
+    ragged last group (n = 9831419 = 600 whole groups + 1019 elements)."""
+    W = wl.weight(13, 756263, seed=6, dtype=torch.float32)
+    _run_both(Q, O, W, dq)
+
+
 def test_equal_absmax_is_lossless(Q, O, cuda):
     W = torch.from_numpy(_edge_tensor("equal_absmax"))
     q_dq, _ = _run_both(Q, O, W, True)

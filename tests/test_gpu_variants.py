@@ -62,6 +62,15 @@ def test_variant_quantize_bit_exact(Q, O, cuda, bs, ct, dt):
         _quant_both(Q, O, W, False, bs, ct, dt)
 
 
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_variant_ring_refill_and_tail(Q, O, cuda, dtype):
+    """FP4 with blocks of 256 and FP8 double quantization on a tensor with
+    more whole 16384-element groups than the quantizer's ring holds per CTA
+    (bf16: 6 stages, fp32: 3) and a ragged last group."""
+    W = wl.weight(11, 1411587, seed=72, dtype=dtype)  # 947 whole groups + 11809 elements
+    _quant_both(Q, O, W, True, 256, "fp4", "e4m3")
+
+
 @pytest.mark.parametrize("ct", ["nf4", "fp4"])
 @pytest.mark.parametrize("bs", [64, 256])
 def test_variant_thresholds_and_ragged(Q, O, cuda, ct, bs):
