@@ -308,13 +308,14 @@ inline LinearWs carve_linear_ws(void* ws, int64_t M, int64_t N, int64_t K, int r
     L.sG = (r > 0 && bwd) ? static_cast<uint16_t*>(c.take((size_t)M * r * 2)) : nullptr;
     // small-M forward: partial tiles [kMaxSmallMCtas][NT][128] and flags
     // [kMaxSmallMCtas][4] of the tcgen05 kernel; for M <= 32 also room for
-    // the warp-MMA kernel's partial slots and its counter per 16 rows (test
-    // mode 7 picks that kernel at run time, so both layouts must fit)
+    // the warp-MMA kernel's partial slots and its counters, one per row slice
+    // of each unit of 64 to 192 rows, at most N / 16 + 8 (test mode 7 picks
+    // that kernel at run time, so both layouts must fit)
     size_t part_floats = (size_t)kMaxSmallMCtas * small_m_nt(M) * 128;
     size_t nflags = (size_t)kMaxSmallMCtas * 4;
     if (M <= kSmallMma) {
         part_floats = std::max(part_floats, (size_t)kSmallMmaMaxCtas * kSmallMmaPartFloatsPerCta);
-        nflags = std::max(nflags, (size_t)((N + 15) / 16) * 2);  // 64-bit counters
+        nflags = std::max(nflags, (size_t)((N + 15) / 16 + 8) * 2);  // 64-bit counters: groups x slices
     }
     L.part = big ? nullptr : static_cast<float*>(c.take(part_floats * 4));
     L.sm_flags = big ? nullptr : static_cast<uint32_t*>(c.take(nflags * 4));
@@ -489,18 +490,18 @@ inline cudaError_t launch_small_m_kernel(const SmallMParams& p, int grid, cudaSt
     return launch_pdl(kern, dim3((unsigned)grid, 1, 1), dim3(SmallMShape<NT, NG>::THREADS, 1, 1), smem, s, 0, p);
 }
 
-template <int MT>
+template <int MT, int SL>
 inline cudaError_t launch_small_m_mma_kernel(SmallMmaParams& p, cudaStream_t s) {
-    using S = SmallMmaShape<MT>;
+    using S = SmallMmaShape<MT, SL>;
     static_assert(S::SMEM + S::STATIC_SMEM <= 232448, "shared memory per CTA");
-    static_assert(2 * 4 * S::PART_FLOATS <= kSmallMmaPartFloatsPerCta, "partial workspace");
+    static_assert(2 * S::SLICES * S::PART_FLOATS <= kSmallMmaPartFloatsPerCta, "partial workspace");
     const int64_t groups = (p.N + S::UROWS - 1) / S::UROWS;
     p.KSU = (p.KB + 3) / 4 + (p.lora_ks + 3) / 4;
     p.units = groups * p.KSU;
     // at least 4 units per CTA; at most one CTA per SM
     const int64_t ctas = std::max<int64_t>(1, std::min<int64_t>(std::min(sm_count(), kSmallMmaMaxCtas),
                                                                 p.units / 4));
-    auto kern = k_smallm_mma<MT>;
+    auto kern = k_smallm_mma<MT, SL>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM);
     if (e != cudaSuccess) return e;
     ProfileScope ps(QLORA_KERNEL_SMALLM_GEMM, s);
@@ -513,13 +514,16 @@ inline qlora_status launch_small_m_mma(const void* X, const LinearArgs& a, const
                                        const LinearWs& L, cudaStream_t s) {
     const qlora_nf4_weight& w = *a.w;
     const int MT = a.M <= 16 ? 1 : 2;
+    // six row slices (192-row units) unless a fused projection's segment
+    // boundary would fall inside a unit (each unit takes one adapter)
+    const bool six = MT == 1 && (a.nseg <= 1 || a.seg_rows % SmallMmaShape<1, 6>::UROWS == 0);
+    const int urows = six ? SmallMmaShape<1, 6>::UROWS : MT == 1 ? SmallMmaShape<1>::UROWS : SmallMmaShape<2>::UROWS;
     SmallMmaParams p;
     memset(&p, 0, sizeof(p));
     // codes [N][K/2] bytes: 128-byte boxes (four blocks of a row) of UROWS
     // rows, 128-byte swizzle (a warp's 8-byte reads of 8 rows hit 8 banks)
     if (!make_map(&p.tmCodes, w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)(a.K / 2), (uint64_t)a.N,
-                  (uint64_t)(a.K / 2), 128, MT == 1 ? SmallMmaShape<1>::UROWS : SmallMmaShape<2>::UROWS,
-                  CU_TENSOR_MAP_SWIZZLE_128B))
+                  (uint64_t)(a.K / 2), 128, (uint32_t)urows, CU_TENSOR_MAP_SWIZZLE_128B))
         return QLORA_ERR_CUDA;
     if (!map_bf16(&p.tmX, X, a.K, a.M, 16 * MT)) return QLORA_ERR_CUDA;
     if (a.r > 0 && !map_bf16(&p.tmU, L.sU, a.rt(), a.M, 16 * MT)) return QLORA_ERR_CUDA;
@@ -546,7 +550,9 @@ inline qlora_status launch_small_m_mma(const void* X, const LinearArgs& a, const
     if (p.epoch == 0) p.epoch = 1;
     p.timeout_ns = wait_timeout_ns();
     p.inject = inject_mode() == 1 ? 1 : 0;
-    const cudaError_t e = MT == 1 ? launch_small_m_mma_kernel<1>(p, s) : launch_small_m_mma_kernel<2>(p, s);
+    const cudaError_t e = six       ? launch_small_m_mma_kernel<1, 6>(p, s)
+                          : MT == 1 ? launch_small_m_mma_kernel<1, 4>(p, s)
+                                    : launch_small_m_mma_kernel<2, 4>(p, s);
     return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 

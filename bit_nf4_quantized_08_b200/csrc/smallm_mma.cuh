@@ -27,23 +27,24 @@
 // it every thread reads 8 contiguous code bytes per weight row and 32
 // contiguous bytes of X per token for a block.
 //
-// Work split: a unit is (128 weight rows, four consecutive 64-element
-// blocks) for up to 16 tokens (64 rows for up to 32), so that every row of
-// the unit is one 128-byte line of codes; the LoRA up-projection adds units
-// of four 64-wide adapter blocks after a row group's weight units.  A
+// Work split: a unit is (192 weight rows, four consecutive 64-element
+// blocks) for up to 16 tokens (128 rows where a fused projection's segment
+// boundary would fall inside 192; 64 rows for up to 32 tokens), so that every
+// row of the unit is one 128-byte line of codes; the LoRA up-projection adds
+// units of four 64-wide adapter blocks after a row group's weight units.  A
 // persistent grid of one CTA per SM takes contiguous shares of the unit list
-// (stream-K), so every SM streams the same number of weight bytes.  The 8
-// MMA warps of a CTA split a unit into 4 row slices x 2 block pairs, and a
-// warp runs the MMA chains of its two blocks interleaved; the codes (one TMA
-// box, 128-byte swizzle) and the four X blocks of each unit pass through a
-// 6-stage ring filled by a loader warp (refilled as the MMA warps release a
-// stage), and a second helper warp rewrites each landed X block into the
-// MMA's operand order.  At the end of a row
-// group the four warps of a slice add their accumulators in block order
-// through shared memory; a group cut between CTAs is finished, per slice, by
-// whichever contributing CTA arrives last (an integer counter with a launch
-// epoch): it adds every contributor's fp32 partial in CTA order
-// (deterministic) and writes Y.  Nothing waits on another CTA.
+// (stream-K), so every SM streams the same number of weight bytes.  The 12
+// (or 8) MMA warps of a CTA split a unit into 6 (or 4) row slices x 2 block
+// pairs, and a warp runs the MMA chains of its two blocks interleaved; the
+// codes (one TMA box, 128-byte swizzle) and the four X blocks of each unit
+// pass through a 5- (or 6-) stage ring filled by a loader warp (refilled as
+// the MMA warps release a stage), and a second helper warp rewrites each
+// landed X block into the MMA's operand order.  At the end of a row group the
+// two warps of a slice add their accumulators in block order through shared
+// memory; a group cut between CTAs is finished, per slice, by whichever
+// contributing CTA arrives last (an integer counter with a launch epoch): it
+// adds every contributor's fp32 partial in CTA order (deterministic) and
+// writes Y.  Nothing waits on another CTA.
 #pragma once
 
 #include "common.cuh"
@@ -72,32 +73,32 @@ struct SmallMmaParams {
     float inv_scale;        // 1 / L
     QFormat fmt;            // code book, 8-bit code book, block size
     uint16_t* Y;            // [M][N]
-    float* part;            // [gridDim.x][2 slots][4 slices][SROWS rows][16 MT tokens] fp32 partials
-    unsigned long long* counters;  // [groups * 4 slices]: (epoch << 32) | arrivals
+    float* part;            // [gridDim.x][2 slots][SLICES][SROWS rows][16 MT tokens] fp32 partials
+    unsigned long long* counters;  // [groups * SLICES]: (epoch << 32) | arrivals
     int64_t part_cap, counter_cap;  // capacities: bounds checks of the debug build
     uint32_t epoch;         // nonzero
     uint64_t timeout_ns;
     int inject;             // test mode 1: issue no loads (the waits run out)
 };
 
-// Ring stages of the warp-MMA small-M kernel (24 KB each), and blocks of a
-// unit per MMA warp (2: 8 MMA warps, 1: 16).
-#ifndef QLORA_SMALLM_XS
-#define QLORA_SMALLM_XS 6
-#endif
+// Blocks of a unit per MMA warp (2; 1 doubles the MMA warps).
 #ifndef QLORA_SMALLM_BPW
 #define QLORA_SMALLM_BPW 2
 #endif
 
-template <int MT>
+// MT: token tiles of 16; SL: row slices of a unit (4 or 6, i.e. 8 or 12 MMA
+// warps; 6 makes a unit of 192 rows for MT = 1, used where no fused
+// projection's segment boundary falls inside a unit).
+template <int MT, int SL = 4>
 struct SmallMmaShape {
     static constexpr int BPW = QLORA_SMALLM_BPW;  // blocks of a unit per MMA warp
-    static constexpr int WARPS = 16 / BPW;        // MMA warps: 4 row slices x 4 / BPW block groups
+    static constexpr int SLICES = SL;             // row slices of a unit
+    static constexpr int WARPS = SLICES * (4 / BPW);  // MMA warps: SLICES row slices x 4 / BPW block groups
     static constexpr int RT = MT == 1 ? 4 : 2;    // 8-row tiles per warp
     static constexpr int SROWS = 8 * RT;          // rows of a slice (32 or 16)
-    static constexpr int UROWS = 4 * SROWS;       // rows of a unit (128 or 64)
+    static constexpr int UROWS = SLICES * SROWS;  // rows of a unit (128, 192; 64 for MT = 2)
     static constexpr int THREADS = 32 * (WARPS + 2);  // + the warp that loads the ring, + the X reorderer
-    static constexpr int XS = QLORA_SMALLM_XS;    // ring stages
+    static constexpr int XS = SL == 4 ? 6 : 5;    // ring stages
     static constexpr int X_TILE = 16 * MT * 128;  // 16 MT tokens x 64 bf16
     static constexpr int CODE_BYTES = UROWS * 128;  // codes of one unit (128-byte swizzle)
     static constexpr int STAGE = CODE_BYTES + 4 * X_TILE;
@@ -164,10 +165,10 @@ __device__ __forceinline__ void named_sync(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
-template <int MT>
-__global__ void __launch_bounds__(SmallMmaShape<MT>::THREADS, 1)
+template <int MT, int SL>
+__global__ void __launch_bounds__(SmallMmaShape<MT, SL>::THREADS, 1)
     k_smallm_mma(const __grid_constant__ SmallMmaParams p) {
-    using S = SmallMmaShape<MT>;
+    using S = SmallMmaShape<MT, SL>;
     constexpr int RT = S::RT, XS = S::XS, SROWS = S::SROWS, UROWS = S::UROWS, WARPS = S::WARPS;
     constexpr int TOK = 16 * MT;
     extern __shared__ uint8_t smem_raw[];
@@ -391,7 +392,7 @@ __global__ void __launch_bounds__(SmallMmaShape<MT>::THREADS, 1)
             bool write_y = whole;
             if (!whole) {
                 const int slot = u0 >= gstart ? 0 : 1;  // the CTA's first segment uses slot 0
-                float* mine = p.part + (((int64_t)blockIdx.x * 2 + slot) * 4 + slice) * S::PART_FLOATS;
+                float* mine = p.part + (((int64_t)blockIdx.x * 2 + slot) * S::SLICES + slice) * S::PART_FLOATS;
 #pragma unroll
                 for (int j = 0; j < RT; ++j)
 #pragma unroll
@@ -410,10 +411,10 @@ __global__ void __launch_bounds__(SmallMmaShape<MT>::THREADS, 1)
                 uint32_t ncontrib = 0;
                 for (int c = cf; c <= cl; ++c) ncontrib += ((U * c) / G < (U * (c + 1)) / G) ? 1u : 0u;
                 uint32_t before = 0;
-                if (lane == 0 && QLORA_CHECK((int64_t)g * 4 + slice < p.counter_cap)) {
+                if (lane == 0 && QLORA_CHECK((int64_t)g * S::SLICES + slice < p.counter_cap)) {
                     // arrivals of this launch (epoch in the high word; a value of
                     // another epoch counts as none)
-                    unsigned long long* ctr = p.counters + (int64_t)g * 4 + slice;
+                    unsigned long long* ctr = p.counters + (int64_t)g * S::SLICES + slice;
                     unsigned long long cv = *reinterpret_cast<volatile unsigned long long*>(ctr);
                     const unsigned long long ep = (unsigned long long)p.epoch << 32;
                     while (true) {
@@ -440,7 +441,7 @@ __global__ void __launch_bounds__(SmallMmaShape<MT>::THREADS, 1)
                     for (int c = cf; c <= cl; ++c) {
                         if ((U * c) / G == (U * (c + 1)) / G) continue;
                         const int cslot = (U * c) / G >= gstart ? 0 : 1;
-                        const float* src = p.part + (((int64_t)c * 2 + cslot) * 4 + slice) * S::PART_FLOATS;
+                        const float* src = p.part + (((int64_t)c * 2 + cslot) * S::SLICES + slice) * S::PART_FLOATS;
 #pragma unroll
                         for (int j = 0; j < RT; ++j)
 #pragma unroll
