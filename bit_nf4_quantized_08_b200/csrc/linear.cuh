@@ -309,7 +309,7 @@ inline LinearWs carve_linear_ws(void* ws, int64_t M, int64_t N, int64_t K, int r
     // small-M forward: partial tiles [kMaxSmallMCtas][NT][128] and flags
     // [kMaxSmallMCtas][4] of the tcgen05 kernel; for M <= 32 also room for
     // the warp-MMA kernel's partial slots and its counters, one per row slice
-    // of each unit of 64 to 192 rows, at most N / 16 + 8 (test mode 7 picks
+    // of each unit of 64 to 224 rows, at most N / 16 + 8 (test mode 7 picks
     // that kernel at run time, so both layouts must fit)
     size_t part_floats = (size_t)kMaxSmallMCtas * small_m_nt(M) * 128;
     size_t nflags = (size_t)kMaxSmallMCtas * 4;
@@ -514,10 +514,11 @@ inline qlora_status launch_small_m_mma(const void* X, const LinearArgs& a, const
                                        const LinearWs& L, cudaStream_t s) {
     const qlora_nf4_weight& w = *a.w;
     const int MT = a.M <= 16 ? 1 : 2;
-    // six row slices (192-row units) unless a fused projection's segment
-    // boundary would fall inside a unit (each unit takes one adapter)
-    const bool six = MT == 1 && (a.nseg <= 1 || a.seg_rows % SmallMmaShape<1, 6>::UROWS == 0);
-    const int urows = six ? SmallMmaShape<1, 6>::UROWS : MT == 1 ? SmallMmaShape<1>::UROWS : SmallMmaShape<2>::UROWS;
+    // the wide unit (seven row slices, 224 rows) unless a fused projection's
+    // segment boundary would fall inside one (each unit takes one adapter)
+    using Wide = SmallMmaShape<1, QLORA_SMALLM_WIDE>;
+    const bool six = MT == 1 && (a.nseg <= 1 || a.seg_rows % Wide::UROWS == 0);
+    const int urows = six ? Wide::UROWS : MT == 1 ? SmallMmaShape<1>::UROWS : SmallMmaShape<2>::UROWS;
     SmallMmaParams p;
     memset(&p, 0, sizeof(p));
     // codes [N][K/2] bytes: 128-byte boxes (four blocks of a row) of UROWS
@@ -550,7 +551,7 @@ inline qlora_status launch_small_m_mma(const void* X, const LinearArgs& a, const
     if (p.epoch == 0) p.epoch = 1;
     p.timeout_ns = wait_timeout_ns();
     p.inject = inject_mode() == 1 ? 1 : 0;
-    const cudaError_t e = six       ? launch_small_m_mma_kernel<1, 6>(p, s)
+    const cudaError_t e = six       ? launch_small_m_mma_kernel<1, QLORA_SMALLM_WIDE>(p, s)
                           : MT == 1 ? launch_small_m_mma_kernel<1, 4>(p, s)
                                     : launch_small_m_mma_kernel<2, 4>(p, s);
     return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;

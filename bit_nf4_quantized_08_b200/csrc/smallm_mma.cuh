@@ -27,17 +27,17 @@
 // it every thread reads 8 contiguous code bytes per weight row and 32
 // contiguous bytes of X per token for a block.
 //
-// Work split: a unit is (192 weight rows, four consecutive 64-element
+// Work split: a unit is (224 weight rows, four consecutive 64-element
 // blocks) for up to 16 tokens (128 rows where a fused projection's segment
-// boundary would fall inside 192; 64 rows for up to 32 tokens), so that every
+// boundary would fall inside 224; 64 rows for up to 32 tokens), so that every
 // row of the unit is one 128-byte line of codes; the LoRA up-projection adds
 // units of four 64-wide adapter blocks after a row group's weight units.  A
 // persistent grid of one CTA per SM takes contiguous shares of the unit list
-// (stream-K), so every SM streams the same number of weight bytes.  The 12
-// (or 8) MMA warps of a CTA split a unit into 6 (or 4) row slices x 2 block
+// (stream-K), so every SM streams the same number of weight bytes.  The 14
+// (or 8) MMA warps of a CTA split a unit into 7 (or 4) row slices x 2 block
 // pairs, and a warp runs the MMA chains of its two blocks interleaved; the
 // codes (one TMA box, 128-byte swizzle) and the four X blocks of each unit
-// pass through a 5- (or 6-) stage ring filled by a loader warp (refilled as
+// pass through a 4- (or 6-) stage ring filled by a loader warp (refilled as
 // the MMA warps release a stage), and a second helper warp rewrites each
 // landed X block into the MMA's operand order.  At the end of a row group the
 // two warps of a slice add their accumulators in block order through shared
@@ -86,9 +86,12 @@ struct SmallMmaParams {
 #define QLORA_SMALLM_BPW 2
 #endif
 
-// MT: token tiles of 16; SL: row slices of a unit (4 or 6, i.e. 8 or 12 MMA
-// warps; 6 makes a unit of 192 rows for MT = 1, used where no fused
-// projection's segment boundary falls inside a unit).
+// MT: token tiles of 16; SL: row slices of a unit (4, or QLORA_SMALLM_WIDE
+// = 7 for MT = 1 where no fused projection's segment boundary falls inside a
+// unit: 8 or 14 MMA warps, units of 128 or 224 rows).
+#ifndef QLORA_SMALLM_WIDE
+#define QLORA_SMALLM_WIDE 7
+#endif
 template <int MT, int SL = 4>
 struct SmallMmaShape {
     static constexpr int BPW = QLORA_SMALLM_BPW;  // blocks of a unit per MMA warp
@@ -96,9 +99,9 @@ struct SmallMmaShape {
     static constexpr int WARPS = SLICES * (4 / BPW);  // MMA warps: SLICES row slices x 4 / BPW block groups
     static constexpr int RT = MT == 1 ? 4 : 2;    // 8-row tiles per warp
     static constexpr int SROWS = 8 * RT;          // rows of a slice (32 or 16)
-    static constexpr int UROWS = SLICES * SROWS;  // rows of a unit (128, 192; 64 for MT = 2)
+    static constexpr int UROWS = SLICES * SROWS;  // rows of a unit (128 or 224; 64 for MT = 2)
     static constexpr int THREADS = 32 * (WARPS + 2);  // + the warp that loads the ring, + the X reorderer
-    static constexpr int XS = SL == 4 ? 6 : 5;    // ring stages
+    static constexpr int XS = SL <= 4 ? 6 : SL <= 6 ? 5 : 4;  // ring stages
     static constexpr int X_TILE = 16 * MT * 128;  // 16 MT tokens x 64 bf16
     static constexpr int CODE_BYTES = UROWS * 128;  // codes of one unit (128-byte swizzle)
     static constexpr int STAGE = CODE_BYTES + 4 * X_TILE;
@@ -106,8 +109,11 @@ struct SmallMmaShape {
     // accumulator exchange, barriers and stage counters
     static constexpr int OFF_T8 = XS * STAGE;
     static constexpr int OFF_SC = OFF_T8 + 1024;                     // [WARPS][2][BPW][SROWS] fp32
-    static constexpr int OFF_XCH = OFF_SC + WARPS * 2 * BPW * SROWS * 4;  // [WARPS][RT * MT * 4][32] fp32
-    static constexpr int OFF_BAR = OFF_XCH + WARPS * RT * MT * 4 * 32 * 4;  // full[XS], empty[XS], xready[XS]
+    static constexpr int XCH_FLOATS = RT * MT * 4 * 32;  // one warp's accumulators
+    // [SLICES][warps per slice - 1][XCH_FLOATS] fp32: the slice's other warps
+    // hand their accumulators to its first
+    static constexpr int OFF_XCH = OFF_SC + WARPS * 2 * BPW * SROWS * 4;
+    static constexpr int OFF_BAR = OFF_XCH + (WARPS - SLICES) * XCH_FLOATS * 4;  // full[XS], empty[XS], xready[XS]
     static constexpr int OFF_CNT = OFF_BAR + 24 * XS;               // issued[XS], abort flag
     static constexpr int SMEM = OFF_CNT + 4 * XS + 16 + 1024;       // + alignment slack
     static constexpr int PART_FLOATS = SROWS * 16 * MT;  // one slice's partial tile
@@ -361,7 +367,7 @@ __global__ void __launch_bounds__(SmallMmaShape<MT, SL>::THREADS, 1)
     // accumulators in block order; the slice's first warp then writes Y, or
     // publishes the partial and lets the last contributor finish the rows.
     auto finish_group = [&](int g, int64_t u) {
-        float* mx = xch + (int64_t)warp * (RT * MT * 4 * 32);
+        float* mx = xch + (int64_t)(slice * (WPS - 1) + bpair - 1) * S::XCH_FLOATS;
         if (bpair != 0) {
 #pragma unroll
             for (int j = 0; j < RT; ++j)
@@ -374,7 +380,7 @@ __global__ void __launch_bounds__(SmallMmaShape<MT, SL>::THREADS, 1)
         if (bpair == 0) {
 #pragma unroll
             for (int w = 1; w < WPS; ++w) {
-                const float* ox = xch + (int64_t)(warp + w) * (RT * MT * 4 * 32);
+                const float* ox = xch + (int64_t)(slice * (WPS - 1) + w - 1) * S::XCH_FLOATS;
 #pragma unroll
                 for (int j = 0; j < RT; ++j)
 #pragma unroll
