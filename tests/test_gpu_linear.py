@@ -342,14 +342,17 @@ def test_small_m_tcgen05_kernel_for_few_tokens(Q, O, cuda, M, N, K, r):
                                              (17, 384, 256, 128, 1, True), (32, 2048, 4096, 32, 1, True),
                                              (16, 3 * 1024, 2048, 32, 3, True), (5, 2000, 2048, 64, 1, True),
                                              (16, 2 * 768, 1024, 16, 2, True), (24, 3 * 768, 1024, 16, 3, True),
-                                             (12, 1000, 1024, 24, 1, False), (30, 520, 640, 40, 1, False)])
+                                             (12, 1000, 1024, 24, 1, False), (30, 520, 640, 40, 1, False),
+                                             (16, 2 * 1792, 1024, 32, 2, True), (5, 3 * 1792, 512, 64, 3, True)])
 def test_small_m_warp_mma_kernel(Q, O, cuda, M, N, K, r, nseg, dq):
     """The register-fed warp-MMA small-M kernel (test mode 7: block constant
     applied to each 64-element block's fp32 partial, bf16 table values times
     a fixed prescale) against the oracle; the fused projection cases check
     its segment columns of sU, also where one 512-row group spans two
     adapters (segments of 768 rows); two cases without double quantization
-    and with a partial last adapter tile (r = 24, 40)."""
+    and with a partial last adapter tile (r = 24, 40); segments of 1792 rows
+    (a whole number of 224-row units: the wide unit with an adapter per
+    segment; 768 and 1024 take the 128-row unit)."""
     S = N // nseg
     W = wl.weight(N, K, seed=90, dtype=torch.bfloat16)
     inp = wl.fused_inputs(M, nseg, S, K, r, seed=90, b_std=0.05)
